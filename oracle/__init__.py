@@ -1,0 +1,169 @@
+"""CPU oracle for the MX block-quantized linear layer (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library does not use it, and it
+shares no code with the CUDA library.
+
+The arithmetic lives in ``mx_oracle.c`` (plain C, fp64), which restates the MX
+format of the blog "Quark Mixed-Precision Quantization for Wan2.2 Video Generation
+on AMD Instinct GPUs" (section "Quantization formats": OCP MXFP4 weights, dynamic
+MXFP4 or FP8 E4M3 activations, 32-element blocks with an E8M0 shared scale, RTN).
+This module only builds that library and marshals numpy arrays into it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+E2M1 = 0
+E4M3 = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mx_oracle.c")
+_LIB = os.path.join(_HERE, "libmx_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``mx_oracle.c`` with gcc into ``libmx_oracle.so`` next to it."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-Wall", "-Wextra",
+             "-D_GNU_SOURCE", _SRC, "-o", tmp, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        # MXO_LIB_OVERRIDE lets the mutation tests load a deliberately broken copy.
+        override = os.environ.get("MXO_LIB_OVERRIDE")
+        _lib = ctypes.CDLL(override if override else build())
+        L = _lib
+        i64, i32, vp, dbl = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_double
+        L.mxo_bf16_to_double.argtypes = [ctypes.c_uint16]
+        L.mxo_bf16_to_double.restype = dbl
+        L.mxo_encode_elem.argtypes = [dbl, i32]
+        L.mxo_encode_elem.restype = i32
+        L.mxo_decode_elem.argtypes = [i32, i32]
+        L.mxo_decode_elem.restype = dbl
+        L.mxo_scale_code.argtypes = [dbl, i32, i32]
+        L.mxo_scale_code.restype = i32
+        L.mxo_scale_value.argtypes = [i32]
+        L.mxo_scale_value.restype = dbl
+        L.mxo_quantize.argtypes = [vp, i64, i64, i32, vp, vp, i32]
+        L.mxo_quantize.restype = i32
+        L.mxo_dequantize.argtypes = [vp, vp, i64, i64, i32, vp]
+        L.mxo_dequantize.restype = i32
+        L.mxo_sf_tiled_bytes.argtypes = [i64, i64]
+        L.mxo_sf_tiled_bytes.restype = i64
+        L.mxo_sf_tiled_offset.argtypes = [i64, i64, i64]
+        L.mxo_sf_tiled_offset.restype = i64
+        L.mxo_sf_to_tiled.argtypes = [vp, i64, i64, vp]
+        L.mxo_sf_to_tiled.restype = i32
+        L.mxo_linear_rows.argtypes = [vp, vp, i32, vp, i64, i64, vp, vp, i64, vp, vp, i32]
+        L.mxo_linear_rows.restype = i32
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def encode_elem(y: float, fmt: int) -> int:
+    """Element code of y rounded to the E2M1 / E4M3 grid (RNE, saturating)."""
+    return lib().mxo_encode_elem(float(y), fmt)
+
+
+def decode_elem(code: int, fmt: int) -> float:
+    return lib().mxo_decode_elem(int(code), fmt)
+
+
+def scale_code(amax: float, fmt: int, nonfinite: bool = False) -> int:
+    return lib().mxo_scale_code(float(amax), int(nonfinite), fmt)
+
+
+def bf16_to_float(bits: int) -> float:
+    return lib().mxo_bf16_to_double(int(bits))
+
+
+def codes_row_bytes(K: int, fmt: int) -> int:
+    return K if fmt == E4M3 else K // 2
+
+
+def quantize(x_bits: np.ndarray, fmt: int, nthreads: int | None = None):
+    """x_bits: uint16 bf16 bit patterns [rows, K].  Returns (codes, sf_logical)."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    rows, K = x_bits.shape
+    codes = np.zeros((rows, codes_row_bytes(K, fmt)), dtype=np.uint8)
+    sf = np.zeros((rows, K // 32), dtype=np.uint8)
+    rc = lib().mxo_quantize(_ptr(x_bits), rows, K, fmt, _ptr(codes), _ptr(sf),
+                            nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle quantize rejected shape %r" % (x_bits.shape,))
+    return codes, sf
+
+
+def dequantize(codes: np.ndarray, sf: np.ndarray, K: int, fmt: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    rows = codes.shape[0]
+    out = np.zeros((rows, K), dtype=np.float64)
+    if lib().mxo_dequantize(_ptr(codes), _ptr(sf), rows, K, fmt, _ptr(out)) != 0:
+        raise ValueError("oracle dequantize rejected K=%d" % K)
+    return out
+
+
+def sf_tiled_bytes(rows: int, K: int) -> int:
+    return lib().mxo_sf_tiled_bytes(rows, K)
+
+
+def sf_tiled_offset(r: int, kb: int, K: int) -> int:
+    return lib().mxo_sf_tiled_offset(r, kb, K)
+
+
+def sf_to_tiled(sf: np.ndarray, K: int) -> np.ndarray:
+    """Logical scales [rows, K/32] -> bytes of the tiled 128x4 atom layout."""
+    sf = np.ascontiguousarray(sf, dtype=np.uint8)
+    rows = sf.shape[0]
+    out = np.zeros(sf_tiled_bytes(rows, K), dtype=np.uint8)
+    lib().mxo_sf_to_tiled(_ptr(sf), rows, K, _ptr(out))
+    return out
+
+
+def linear_rows(a_codes, a_sf, a_fmt, rows, K, w_codes, w_sf, bias_bits=None,
+                nthreads: int | None = None) -> np.ndarray:
+    """fp64 Y[rows, :] = deq(A)[rows] . deq(W)^T (+ bias) for the listed rows."""
+    a_codes = np.ascontiguousarray(a_codes, dtype=np.uint8)
+    a_sf = np.ascontiguousarray(a_sf, dtype=np.uint8)
+    w_codes = np.ascontiguousarray(w_codes, dtype=np.uint8)
+    w_sf = np.ascontiguousarray(w_sf, dtype=np.uint8)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    N = w_codes.shape[0]
+    y = np.zeros((rows.shape[0], N), dtype=np.float64)
+    bias_p = None
+    if bias_bits is not None:
+        bias_bits = np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        bias_p = _ptr(bias_bits)
+    rc = lib().mxo_linear_rows(_ptr(a_codes), _ptr(a_sf), a_fmt, _ptr(rows), rows.shape[0], K,
+                               _ptr(w_codes), _ptr(w_sf), N, bias_p, _ptr(y),
+                               nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle linear failed (rc=%d)" % rc)
+    return y
+
+
+def linear(a_codes, a_sf, a_fmt, K, w_codes, w_sf, bias_bits=None, nthreads=None):
+    M = a_codes.shape[0]
+    return linear_rows(a_codes, a_sf, a_fmt, np.arange(M, dtype=np.int64), K, w_codes, w_sf,
+                       bias_bits, nthreads)

@@ -1,0 +1,369 @@
+/*
+ * mx_oracle.c -- plain CPU reference for the MX block-quantized linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU-baseline
+ * leg of the benchmark may load this library.  The CUDA library never links it and
+ * shares no code, header, table or constant with it.
+ *
+ * What it computes (blog "Quark Mixed-Precision Quantization for Wan2.2 Video
+ * Generation on AMD Instinct GPUs", section "Quantization formats": W4A4 = OCP MXFP4
+ * weights with dynamic MXFP4 activations, W4A8 = MXFP4 weights with FP8 E4M3
+ * activations; the MX format itself is the OCP Microscaling spec v1.0, the blog's
+ * reference [7]):
+ *
+ *   * a tensor is cut into blocks of 32 consecutive elements along K;
+ *   * every block shares one E8M0 scale X = 2^(floor(log2(amax)) - emax)
+ *     (emax = 2 for E2M1, 8 for E4M3), clamped at E8M0's smallest value 2^-127;
+ *   * every element x is stored as RTN(x / X) on the element grid, with ties to
+ *     even and saturation at the largest finite element;
+ *   * the linear layer is Y = deq(Xq) . deq(Wq)^T (+ bias), here in fp64.
+ *
+ * Readings taken where the pages are silent (each one also listed in the design doc):
+ *   R1 scale = floor rule above (OCP v1.0);  R2 zero / subnormal amax -> scale code 0;
+ *   R3 a block holding Inf or NaN -> scale code 0xFF and all element codes 0;
+ *   R4 "RTN" = IEEE round-to-nearest-even, saturating to +-max;
+ *   R5 a negative value that rounds to zero keeps its sign bit;
+ *   R6 E2M1 element 2j sits in the low nibble of byte j, 2j+1 in the high nibble;
+ *   R7 tiled scale layout: 512-byte atoms of 128 rows x 4 k-blocks,
+ *      offset = (r%32)*16 + ((r/32)%4)*4 + kb%4, atoms ordered row-tile major;
+ *   R8 tolerance row norm = infinity norm of the oracle's output row.
+ *
+ * Everything is computed in double precision.  Every step is written out on its
+ * own; nothing is blocked, fused or reordered beyond splitting independent rows
+ * across host threads.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define MXO_E2M1 0
+#define MXO_E4M3 1
+
+/* Element format parameters.  E2M1: 2 exponent bits (bias 1), 1 mantissa bit,
+ * no Inf/NaN, largest magnitude 6.  E4M3 (the "FN" variant of OCP FP8): 4
+ * exponent bits (bias 7), 3 mantissa bits, only NaN is S.1111.111, largest
+ * magnitude 448 = S.1111.110.  emax is the exponent of the largest normal. */
+typedef struct {
+    int ebits, mbits, bias, emax;
+    double maxval;
+} mxo_fmt;
+
+static const mxo_fmt FMTS[2] = {
+    {2, 1, 1, 2, 6.0},
+    {4, 3, 7, 8, 448.0},
+};
+
+static const mxo_fmt *fmt_of(int f) { return (f == MXO_E4M3) ? &FMTS[1] : &FMTS[0]; }
+
+/* ---- bf16 ------------------------------------------------------------------ */
+
+/* bf16 is the upper half of an IEEE binary32; widen and convert exactly. */
+double mxo_bf16_to_double(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* ---- element grid ------------------------------------------------------------ */
+
+/* Magnitude bits (exponent field | mantissa field) of a value v that is already
+ * exactly on the format's grid and not above its largest finite value. */
+static int grid_bits(double v, const mxo_fmt *f)
+{
+    if (v == 0.0) return 0;
+    int e2;
+    frexp(v, &e2);              /* v = m * 2^e2, m in [0.5, 1) */
+    int e = e2 - 1;             /* v = (1.f) * 2^e             */
+    int emin = 1 - f->bias;
+    if (e < emin) {             /* subnormal: value = mant * 2^(emin - mbits) */
+        return (int)(v / ldexp(1.0, emin - f->mbits));
+    }
+    int mant = (int)(v / ldexp(1.0, e - f->mbits)) - (1 << f->mbits);
+    return ((e + f->bias) << f->mbits) | mant;
+}
+
+/* Round y to the element grid: round-to-nearest, ties-to-even (R4), saturating
+ * at +-max, sign kept on a zero result (R5).  Returns the element code. */
+int mxo_encode_elem(double y, int fmt)
+{
+    const mxo_fmt *f = fmt_of(fmt);
+    int nbits = f->ebits + f->mbits;
+    int sign = signbit(y) ? 1 : 0;
+    double a = fabs(y);
+    double v;
+    if (a >= f->maxval) {
+        v = f->maxval;
+    } else if (a == 0.0) {
+        v = 0.0;
+    } else {
+        int e2;
+        frexp(a, &e2);
+        int e = e2 - 1;
+        int emin = 1 - f->bias;
+        if (e < emin) e = emin;                 /* subnormal spacing below the min normal */
+        double q = ldexp(1.0, e - f->mbits);    /* grid spacing around a                  */
+        double n = nearbyint(a / q);            /* default rounding mode: ties to even    */
+        v = n * q;
+        if (v > f->maxval) v = f->maxval;       /* rounding up past max saturates         */
+    }
+    return (sign << nbits) | grid_bits(v, f);
+}
+
+/* Value of an element code; E4M3's S.1111.111 is NaN. */
+double mxo_decode_elem(int code, int fmt)
+{
+    const mxo_fmt *f = fmt_of(fmt);
+    int nbits = f->ebits + f->mbits;
+    int sign = (code >> nbits) & 1;
+    int ef = (code >> f->mbits) & ((1 << f->ebits) - 1);
+    int mf = code & ((1 << f->mbits) - 1);
+    if (fmt == MXO_E4M3 && ef == 15 && mf == 7) return NAN;
+    double mag;
+    if (ef == 0)
+        mag = ldexp((double)mf, 1 - f->bias - f->mbits);
+    else
+        mag = ldexp((double)((1 << f->mbits) + mf), ef - f->bias - f->mbits);
+    return sign ? -mag : mag;
+}
+
+/* ---- shared scale ------------------------------------------------------------ */
+
+/* E8M0 scale code of a block with absolute maximum amax (R1, R2, R3). */
+int mxo_scale_code(double amax, int nonfinite, int fmt)
+{
+    const mxo_fmt *f = fmt_of(fmt);
+    if (nonfinite) return 255;
+    if (amax == 0.0) return 0;
+    int e2;
+    frexp(amax, &e2);                    /* floor(log2(amax)) = e2 - 1 */
+    int sc = (e2 - 1) + 127 - f->emax;
+    return sc < 0 ? 0 : sc;
+}
+
+/* Value of an E8M0 scale code. */
+double mxo_scale_value(int sc)
+{
+    if (sc == 255) return NAN;
+    return ldexp(1.0, sc - 127);
+}
+
+/* ---- block and tensor quantization ------------------------------------------- */
+
+/* Quantize one block of 32 bf16 values into 32 element codes and a scale code. */
+static int quantize_block(const uint16_t *x, int fmt, int codes[32])
+{
+    double v[32];
+    double amax = 0.0;
+    int nonfinite = 0;
+    for (int i = 0; i < 32; ++i) {
+        v[i] = mxo_bf16_to_double(x[i]);
+        if (isnan(v[i]) || isinf(v[i])) nonfinite = 1;
+        else if (fabs(v[i]) > amax) amax = fabs(v[i]);
+    }
+    int sc = mxo_scale_code(amax, nonfinite, fmt);
+    for (int i = 0; i < 32; ++i) {
+        if (sc == 255) codes[i] = 0;
+        else codes[i] = mxo_encode_elem(v[i] / mxo_scale_value(sc), fmt);
+    }
+    return sc;
+}
+
+/* Bytes of element codes per row: K/2 (E2M1, two per byte, R6) or K (E4M3). */
+int64_t mxo_codes_row_bytes(int64_t K, int fmt) { return fmt == MXO_E4M3 ? K : K / 2; }
+
+typedef struct {
+    const uint16_t *x;
+    int64_t r0, r1, K;
+    int fmt;
+    uint8_t *codes;
+    uint8_t *sf;
+} quant_job;
+
+static void *quant_rows(void *arg)
+{
+    quant_job *j = (quant_job *)arg;
+    int64_t KB = j->K / 32;
+    int64_t rb = mxo_codes_row_bytes(j->K, j->fmt);
+    int codes[32];
+    for (int64_t r = j->r0; r < j->r1; ++r) {
+        for (int64_t kb = 0; kb < KB; ++kb) {
+            int sc = quantize_block(j->x + r * j->K + kb * 32, j->fmt, codes);
+            j->sf[r * KB + kb] = (uint8_t)sc;
+            uint8_t *out = j->codes + r * rb;
+            for (int i = 0; i < 32; ++i) {
+                int64_t k = kb * 32 + i;
+                if (j->fmt == MXO_E4M3) {
+                    out[k] = (uint8_t)codes[i];
+                } else if ((k & 1) == 0) {
+                    out[k / 2] = (uint8_t)(codes[i] & 0xF);
+                } else {
+                    out[k / 2] |= (uint8_t)((codes[i] & 0xF) << 4);
+                }
+            }
+        }
+    }
+    return NULL;
+}
+
+/* Split rows [0, rows) into nthreads contiguous ranges and run fn on each. */
+static void run_rows(void *(*fn)(void *), void *jobs, size_t job_size, int64_t rows, int nthreads,
+                     void (*set_range)(void *, int64_t, int64_t))
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > rows) nthreads = (int)(rows > 0 ? rows : 1);
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    int64_t per = (rows + nthreads - 1) / nthreads;
+    for (int t = 0; t < nthreads; ++t) {
+        void *job = (char *)jobs + (size_t)t * job_size;
+        int64_t r0 = t * per, r1 = r0 + per;
+        if (r1 > rows) r1 = rows;
+        if (r0 > rows) r0 = rows;
+        set_range(job, r0, r1);
+        if (nthreads == 1) fn(job);
+        else pthread_create(&th[t], NULL, fn, job);
+    }
+    if (nthreads > 1)
+        for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+    free(th);
+}
+
+static void set_quant_range(void *j, int64_t r0, int64_t r1)
+{
+    ((quant_job *)j)->r0 = r0;
+    ((quant_job *)j)->r1 = r1;
+}
+
+/* x: bf16 bits [rows, K] row-major.  codes: [rows, K/2] (E2M1) or [rows, K] (E4M3).
+ * sf: logical scale codes [rows, K/32] row-major.  K must be a multiple of 32. */
+int mxo_quantize(const uint16_t *x, int64_t rows, int64_t K, int fmt,
+                 uint8_t *codes, uint8_t *sf, int nthreads)
+{
+    if (K % 32 != 0 || rows < 0) return -1;
+    if (nthreads < 1) nthreads = 1;
+    quant_job *jobs = (quant_job *)calloc((size_t)nthreads, sizeof(quant_job));
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t].x = x; jobs[t].K = K; jobs[t].fmt = fmt; jobs[t].codes = codes; jobs[t].sf = sf;
+    }
+    run_rows(quant_rows, jobs, sizeof(quant_job), rows, nthreads, set_quant_range);
+    free(jobs);
+    return 0;
+}
+
+/* Element code k of a row of packed codes. */
+static int code_at(const uint8_t *row, int64_t k, int fmt)
+{
+    if (fmt == MXO_E4M3) return row[k];
+    uint8_t b = row[k / 2];
+    return (k & 1) ? (b >> 4) : (b & 0xF);
+}
+
+/* Dequantize: out[r, k] = decode(code[r, k]) * 2^(sf[r, k/32] - 127). */
+int mxo_dequantize(const uint8_t *codes, const uint8_t *sf, int64_t rows, int64_t K, int fmt,
+                   double *out)
+{
+    if (K % 32 != 0) return -1;
+    int64_t KB = K / 32, rb = mxo_codes_row_bytes(K, fmt);
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k)
+            out[r * K + k] = mxo_decode_elem(code_at(codes + r * rb, k, fmt), fmt) *
+                             mxo_scale_value(sf[r * KB + k / 32]);
+    return 0;
+}
+
+/* ---- tiled scale layout (R7) ------------------------------------------------- */
+
+/* Bytes of the tiled scale buffer: rows padded to 128, k-blocks padded to 4. */
+int64_t mxo_sf_tiled_bytes(int64_t rows, int64_t K)
+{
+    int64_t KB = K / 32;
+    return ((rows + 127) / 128) * 128 * ((KB + 3) / 4) * 4;
+}
+
+/* Byte offset of logical scale (r, kb) in the tiled layout. */
+int64_t mxo_sf_tiled_offset(int64_t r, int64_t kb, int64_t K)
+{
+    int64_t KB = K / 32;
+    int64_t atoms_k = (KB + 3) / 4;
+    int64_t atom = (r / 128) * atoms_k + kb / 4;
+    return atom * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + (kb % 4);
+}
+
+/* Scatter a logical [rows, K/32] scale array into the tiled layout; padding is 0. */
+int mxo_sf_to_tiled(const uint8_t *sf, int64_t rows, int64_t K, uint8_t *tiled)
+{
+    int64_t KB = K / 32;
+    memset(tiled, 0, (size_t)mxo_sf_tiled_bytes(rows, K));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t kb = 0; kb < KB; ++kb)
+            tiled[mxo_sf_tiled_offset(r, kb, K)] = sf[r * KB + kb];
+    return 0;
+}
+
+/* ---- the linear layer ---------------------------------------------------------- */
+
+typedef struct {
+    const uint8_t *a_codes, *a_sf;
+    int a_fmt;
+    const int64_t *rows;
+    int64_t i0, i1, K, N;
+    const double *wdeq;   /* [N, K] dequantized weights */
+    const uint16_t *bias; /* [N] bf16 or NULL */
+    double *y;            /* [nrows, N] */
+} lin_job;
+
+static void *lin_rows(void *arg)
+{
+    lin_job *j = (lin_job *)arg;
+    int64_t K = j->K, KB = K / 32, rb = mxo_codes_row_bytes(K, j->a_fmt);
+    double *a = (double *)malloc(sizeof(double) * (size_t)K);
+    for (int64_t i = j->i0; i < j->i1; ++i) {
+        int64_t m = j->rows[i];
+        for (int64_t k = 0; k < K; ++k)
+            a[k] = mxo_decode_elem(code_at(j->a_codes + m * rb, k, j->a_fmt), j->a_fmt) *
+                   mxo_scale_value(j->a_sf[m * KB + k / 32]);
+        for (int64_t n = 0; n < j->N; ++n) {
+            const double *w = j->wdeq + n * K;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += a[k] * w[k];
+            if (j->bias) acc += mxo_bf16_to_double(j->bias[n]);
+            j->y[i * j->N + n] = acc;
+        }
+    }
+    free(a);
+    return NULL;
+}
+
+static void set_lin_range(void *j, int64_t r0, int64_t r1)
+{
+    ((lin_job *)j)->i0 = r0;
+    ((lin_job *)j)->i1 = r1;
+}
+
+/* y[i, n] = sum_k deqA[rows[i], k] * deqW[n, k] + bias[n], in fp64.
+ * A: activation codes in fmt a_fmt with logical scales [M, K/32]; W: E2M1 codes
+ * [N, K/2] with logical scales [N, K/32]; rows: the nrows output rows wanted. */
+int mxo_linear_rows(const uint8_t *a_codes, const uint8_t *a_sf, int a_fmt,
+                    const int64_t *rows, int64_t nrows, int64_t K,
+                    const uint8_t *w_codes, const uint8_t *w_sf, int64_t N,
+                    const uint16_t *bias, double *y, int nthreads)
+{
+    if (K % 32 != 0) return -1;
+    double *wdeq = (double *)malloc(sizeof(double) * (size_t)(N * K));
+    if (!wdeq) return -2;
+    mxo_dequantize(w_codes, w_sf, N, K, MXO_E2M1, wdeq);
+    if (nthreads < 1) nthreads = 1;
+    lin_job *jobs = (lin_job *)calloc((size_t)nthreads, sizeof(lin_job));
+    for (int t = 0; t < nthreads; ++t) {
+        lin_job *j = &jobs[t];
+        j->a_codes = a_codes; j->a_sf = a_sf; j->a_fmt = a_fmt; j->rows = rows;
+        j->K = K; j->N = N; j->wdeq = wdeq; j->bias = bias; j->y = y;
+    }
+    run_rows(lin_rows, jobs, sizeof(lin_job), nrows, nthreads, set_lin_range);
+    free(jobs);
+    free(wdeq);
+    return 0;
+}

@@ -1,0 +1,59 @@
+"""The oracle pins must catch plausible mistakes.
+
+Each case compiles a copy of the oracle's C source with one deliberate slip (a wrong
+rounding mode, an off-by-one exponent, a swapped nibble, a transposed operand, ...)
+and runs the pin tests against it in a subprocess; the pins must fail.  The mistake
+is planted only in a temporary CPU-side copy of the oracle.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "mx_oracle.c")
+
+MUTANTS = [
+    ("ties_away_from_zero", "double n = nearbyint(a / q);", "double n = round(a / q);"),
+    ("scale_exponent_off_by_one", "int sc = (e2 - 1) + 127 - f->emax;", "int sc = e2 + 127 - f->emax;"),
+    ("e4m3_emax_7", "{4, 3, 7, 8, 448.0}", "{4, 3, 7, 7, 448.0}"),
+    ("no_saturation", [("if (v > f->maxval) v = f->maxval;       /* rounding",
+                        "if (0) v = f->maxval;       /* rounding"),
+                       ("if (a >= f->maxval) {", "if (a >= 4 * f->maxval) {")]),
+    ("negative_zero_dropped", "int sign = signbit(y) ? 1 : 0;", "int sign = (y < 0) ? 1 : 0;"),
+    ("nibbles_swapped", "} else if ((k & 1) == 0) {", "} else if ((k & 1) == 1) {"),
+    ("no_subnormal_floor", "if (e < emin) e = emin;                 /* subnormal",
+     "if (0) e = emin;                 /* subnormal"),
+    ("scale_multiplied", "else codes[i] = mxo_encode_elem(v[i] / mxo_scale_value(sc), fmt);",
+     "else codes[i] = mxo_encode_elem(v[i] * mxo_scale_value(sc), fmt);"),
+    ("weights_transposed", "const double *w = j->wdeq + n * K;", "const double *w = j->wdeq + n;"),
+    ("bias_dropped", "if (j->bias) acc += mxo_bf16_to_double(j->bias[n]);", "(void)0;"),
+    ("sf_atom_rows_swapped", "return atom * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + (kb % 4);",
+     "return atom * 512 + (r % 32) * 4 + ((r / 32) % 4) * 16 + (kb % 4);"),
+    ("dequant_wrong_block_index", "mxo_scale_value(sf[r * KB + k / 32]);",
+     "mxo_scale_value(sf[r * KB + (k / 32 + 1) % KB]);"),
+]
+
+
+def _edits(m):
+    return m[1] if isinstance(m[1], list) else [(m[1], m[2])]
+
+
+@pytest.mark.parametrize("mutant", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(mutant, tmp_path):
+    name = mutant[0]
+    src = open(SRC).read()
+    for old, new in _edits(mutant):
+        assert src.count(old) == 1, "mutation anchor not found: " + name
+        src = src.replace(old, new)
+    mut = tmp_path / ("mx_oracle_%s.c" % name)
+    mut.write_text(src)
+    so = tmp_path / ("libmx_oracle_%s.so" % name)
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-D_GNU_SOURCE",
+                           str(mut), "-o", str(so), "-lm", "-lpthread"])
+    env = dict(os.environ, MXO_LIB_OVERRIDE=str(so))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, "pins did not catch mutant %s:\n%s" % (name, r.stdout[-2000:])

@@ -1,0 +1,355 @@
+"""Pins of the CPU oracle against things other than itself.
+
+The MX format is the one the blog "Quark Mixed-Precision Quantization for Wan2.2
+Video Generation on AMD Instinct GPUs" uses (section "Quantization formats"): OCP
+MXFP4 (E2M1 elements) and FP8 E4M3 elements, 32-element blocks, one E8M0 scale per
+block, RTN.  The pins below use independent routes to the same answers:
+
+* element rounding: exhaustive over all bf16 bit patterns against a brute-force
+  nearest-value search over the enumerated grids (ties to the even code);
+* element grids: literal values from the format tables;
+* scale: closed form max(0, j + 127 - emax) for amax in [2^j, 2^(j+1));
+* hand-worked blocks: tests/golden/hand_blocks.json;
+* invariants: idempotence, power-of-two equivariance, sign symmetry, permutation;
+* the linear layer: exact rational brute force on tiny matrices, and the
+  lossless case where numpy's fp64 matmul is the answer.
+"""
+import json
+import math
+import os
+import struct
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+FMT = {"e2m1": oracle.E2M1, "e4m3": oracle.E4M3}
+
+
+# --- independent descriptions of the element grids ---------------------------------
+
+# E2M1 magnitudes by code 0..7, as listed in the OCP MX element-format table.
+E2M1_MAG = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def e4m3_mag(code):
+    """E4M3 magnitude from its bit fields: exponent bias 7, 3 mantissa bits,
+    subnormals m/8 * 2^-6; code 0x7F is NaN and not part of the grid."""
+    e, m = code >> 3, code & 7
+    if e == 0:
+        return m / 8.0 * 2.0 ** -6
+    return (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+E4M3_MAG = [e4m3_mag(c) for c in range(0x7F)]  # codes 0..126 (finite, non-negative)
+GRID = {oracle.E2M1: (E2M1_MAG, 3), oracle.E4M3: (E4M3_MAG, 7)}  # (magnitudes, sign bit)
+
+
+def brute_round(y, fmt):
+    """Nearest grid value by exhaustive search; ties to the even code; values past the
+    largest magnitude saturate; the sign bit follows the sign of y (even for 0)."""
+    mags, sbit = GRID[fmt]
+    a = abs(y)
+    best = None
+    for code, g in enumerate(mags):
+        d = abs(a - g)
+        if best is None or d < best[0] or (d == best[0] and code % 2 == 0):
+            best = (d, code)
+    code = best[1]
+    if a > mags[-1]:
+        code = len(mags) - 1
+    neg = math.copysign(1.0, y) < 0
+    return code | (int(neg) << sbit)
+
+
+def all_finite_bf16():
+    bits = np.arange(65536, dtype=np.uint32)
+    f = (bits << 16).view(np.float32)
+    keep = np.isfinite(f)
+    return bits[keep].astype(np.uint16), f[keep].astype(np.float64)
+
+
+# --- element grids -----------------------------------------------------------------------
+
+def test_e2m1_decode_table():
+    for c in range(16):
+        want = E2M1_MAG[c & 7] * (-1.0 if c & 8 else 1.0)
+        got = oracle.decode_elem(c, oracle.E2M1)
+        assert got == want and math.copysign(1, got) == math.copysign(1, want), c
+
+
+def test_e4m3_decode_table():
+    for c in range(256):
+        got = oracle.decode_elem(c, oracle.E4M3)
+        if c & 0x7F == 0x7F:
+            assert math.isnan(got)
+            continue
+        want = e4m3_mag(c & 0x7F) * (-1.0 if c & 0x80 else 1.0)
+        assert got == want, hex(c)
+    # a few literal anchors of the format
+    assert oracle.decode_elem(0x7E, oracle.E4M3) == 448.0
+    assert oracle.decode_elem(0x01, oracle.E4M3) == 2.0 ** -9
+    assert oracle.decode_elem(0x08, oracle.E4M3) == 2.0 ** -6
+    assert oracle.decode_elem(0x38, oracle.E4M3) == 1.0
+
+
+@pytest.mark.parametrize("fmt", [oracle.E2M1, oracle.E4M3])
+def test_element_rounding_exhaustive_bf16(fmt):
+    """Every finite bf16 value, and every finite bf16 value times 2^-k for small k
+    (to sweep the ties and subnormals of the target grid densely), rounds exactly as
+    a brute-force nearest search over the grid."""
+    _, vals = all_finite_bf16()
+    mags = np.array(GRID[fmt][0])
+    sbit = GRID[fmt][1]
+    for shift in (0, 3, 7):
+        ys = vals * 2.0 ** -shift
+        a = np.abs(ys)
+        d = np.abs(a[:, None] - mags[None, :])
+        dmin = d.min(axis=1, keepdims=True)
+        ties = d == dmin
+        # prefer the even code among the nearest ones
+        even = ties & (np.arange(len(mags))[None, :] % 2 == 0)
+        code = np.where(even.any(axis=1), even.argmax(axis=1), ties.argmax(axis=1))
+        code = np.where(a > mags[-1], len(mags) - 1, code)
+        code = code | (np.signbit(ys).astype(np.int64) << sbit)
+        got = np.array([oracle.encode_elem(y, fmt) for y in ys])
+        bad = np.nonzero(got != code)[0]
+        assert bad.size == 0, [(ys[i], got[i], code[i]) for i in bad[:5]]
+
+
+def test_brute_round_agrees_with_vectorised_search():
+    # the two test-side searches must agree with each other on a handful of values
+    for fmt in (oracle.E2M1, oracle.E4M3):
+        for y in (0.25, 0.75, -1.25, 5.0, 7.0, 1e-30, -0.0, 2.0 ** -10, 464.0, 500.0):
+            assert brute_round(y, fmt) == oracle.encode_elem(y, fmt)
+
+
+# --- the shared scale ---------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt,emax", [(oracle.E2M1, 2), (oracle.E4M3, 8)])
+def test_scale_code_closed_form(fmt, emax):
+    for j in range(-133, 128):
+        for mant in (1.0, 1.5, 2.0 - 2.0 ** -7):
+            amax = mant * 2.0 ** j
+            assert oracle.scale_code(amax, fmt) == max(0, j + 127 - emax), (j, mant)
+    assert oracle.scale_code(0.0, fmt) == 0
+    assert oracle.scale_code(1.0, fmt, nonfinite=True) == 255
+
+
+# --- hand-worked blocks -------------------------------------------------------------------
+
+def _expand(runs):
+    out = []
+    for v, n in runs:
+        out += [float.fromhex(v) if isinstance(v, str) else v] * n
+    return out
+
+
+def _bf16_bits(vals):
+    return np.array([struct.unpack("<I", struct.pack("<f", v))[0] >> 16 for v in vals],
+                    dtype=np.uint16)
+
+
+def load_hand_blocks():
+    with open(os.path.join(GOLDEN, "hand_blocks.json")) as f:
+        return json.load(f)["blocks"]
+
+
+@pytest.mark.parametrize("blk", load_hand_blocks(), ids=lambda b: b["name"])
+def test_hand_worked_block(blk):
+    fmt = FMT[blk["fmt"]]
+    x = _expand(blk["x"])
+    assert len(x) == 32
+    bits = _bf16_bits(x)
+    assert all(oracle.bf16_to_float(int(b)) == v for b, v in zip(bits, x))
+    codes, sf = oracle.quantize(bits[None, :], fmt)
+    assert int(sf[0, 0]) == blk["sf"]
+    want = _expand(blk["codes"])
+    if fmt == oracle.E4M3:
+        got = list(codes[0])
+    else:
+        got = []
+        for b in codes[0]:
+            got += [int(b) & 0xF, int(b) >> 4]
+    assert got == want
+    if "packed_first_bytes" in blk:
+        n = len(blk["packed_first_bytes"])
+        assert list(codes[0, :n]) == blk["packed_first_bytes"]
+
+
+# --- invariants ---------------------------------------------------------------------------
+
+def _random_blocks(rng, nblk, scale_spread=6):
+    x = rng.standard_normal((nblk, 32)) * 2.0 ** rng.integers(-scale_spread, scale_spread, (nblk, 1))
+    x[rng.random((nblk, 32)) < 0.05] *= 40.0
+    return _bf16_bits(x.astype(np.float32).ravel()).reshape(nblk, 32)
+
+
+@pytest.mark.parametrize("fmt", [oracle.E2M1, oracle.E4M3])
+def test_idempotence(fmt):
+    rng = np.random.default_rng(1)
+    bits = _random_blocks(rng, 2000)
+    codes, sf = oracle.quantize(bits, fmt)
+    deq = oracle.dequantize(codes, sf, 32, fmt)
+    deq_bits = _bf16_bits(deq.astype(np.float32).ravel()).reshape(deq.shape)
+    assert np.array_equal(deq, deq_bits_to_f64(deq_bits))  # exact in bf16
+    codes2, sf2 = oracle.quantize(deq_bits, fmt)
+    keep = sf[:, 0] > 0
+    assert keep.all()
+    assert np.array_equal(sf2, sf)
+    # a zero element may flip between +0 and -0 only if its input was +-0; none here
+    assert np.array_equal(codes2, codes)
+
+
+def deq_bits_to_f64(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("fmt", [oracle.E2M1, oracle.E4M3])
+def test_power_of_two_equivariance(fmt):
+    rng = np.random.default_rng(2)
+    bits = _random_blocks(rng, 500, scale_spread=3)
+    x = deq_bits_to_f64(bits)
+    codes, sf = oracle.quantize(bits, fmt)
+    for j in (-5, -1, 1, 7):
+        codes_j, sf_j = oracle.quantize(_bf16_bits((x * 2.0 ** j).astype(np.float32).ravel())
+                                        .reshape(bits.shape), fmt)
+        assert np.array_equal(codes_j, codes)
+        assert np.array_equal(sf_j.astype(int), sf.astype(int) + j)
+
+
+@pytest.mark.parametrize("fmt", [oracle.E2M1, oracle.E4M3])
+def test_sign_symmetry(fmt):
+    rng = np.random.default_rng(3)
+    bits = _random_blocks(rng, 500)
+    codes, sf = oracle.quantize(bits, fmt)
+    codes_n, sf_n = oracle.quantize(bits ^ np.uint16(0x8000), fmt)
+    assert np.array_equal(sf_n, sf)
+    flip = 0x88 if fmt == oracle.E2M1 else 0x80
+    assert np.array_equal(codes_n, codes ^ np.uint8(flip))
+
+
+@pytest.mark.parametrize("fmt", [oracle.E2M1, oracle.E4M3])
+def test_permutation_within_block(fmt):
+    rng = np.random.default_rng(4)
+    bits = _random_blocks(rng, 200)
+    codes, sf = oracle.quantize(bits, fmt)
+    perm = rng.permutation(32)
+    codes_p, sf_p = oracle.quantize(bits[:, perm], fmt)
+    assert np.array_equal(sf_p, sf)
+    unpack = lambda c: (np.stack([c & 0xF, c >> 4], -1).reshape(c.shape[0], -1)
+                        if fmt == oracle.E2M1 else c)
+    assert np.array_equal(unpack(codes_p), unpack(codes)[:, perm])
+
+
+def test_nonfinite_block_convention():
+    x = [1.0] * 32
+    x[5] = float("inf")
+    codes, sf = oracle.quantize(_bf16_bits(x)[None, :], oracle.E2M1)
+    assert sf[0, 0] == 255 and not codes.any()
+    assert math.isnan(oracle.dequantize(codes, sf, 32, oracle.E2M1)[0, 0])
+
+
+# --- tiled scale layout -----------------------------------------------------------------------
+
+def test_sf_tiled_layout_hand_offsets():
+    # K = 256 -> 8 k-blocks -> 2 atoms along k per 128-row tile
+    K = 256
+    assert oracle.sf_tiled_offset(0, 0, K) == 0
+    assert oracle.sf_tiled_offset(0, 3, K) == 3
+    assert oracle.sf_tiled_offset(1, 0, K) == 16
+    assert oracle.sf_tiled_offset(32, 0, K) == 4
+    assert oracle.sf_tiled_offset(97, 2, K) == 16 + 12 + 2
+    assert oracle.sf_tiled_offset(0, 4, K) == 512
+    assert oracle.sf_tiled_offset(128, 0, K) == 1024
+    assert oracle.sf_tiled_offset(130, 5, K) == 1024 + 512 + 2 * 16 + 1
+
+
+@pytest.mark.parametrize("rows,K", [(1, 32), (127, 96), (129, 160), (300, 1024)])
+def test_sf_tiled_layout_is_injective_and_padded(rows, K):
+    KB = K // 32
+    rng = np.random.default_rng(rows)
+    sf = rng.integers(1, 255, (rows, KB), dtype=np.uint8)
+    t = oracle.sf_to_tiled(sf, K)
+    assert t.size == ((rows + 127) // 128) * 128 * ((KB + 3) // 4) * 4
+    offs = {oracle.sf_tiled_offset(r, kb, K) for r in range(rows) for kb in range(KB)}
+    assert len(offs) == rows * KB
+    assert np.count_nonzero(t) == rows * KB  # padding bytes are zero
+    for r in (0, rows - 1):
+        for kb in (0, KB - 1):
+            assert t[oracle.sf_tiled_offset(r, kb, K)] == sf[r, kb]
+
+
+# --- the linear layer -------------------------------------------------------------------------
+
+def _exact_value(code, sfc, fmt):
+    mags, sbit = GRID[fmt]
+    mag = Fraction(mags[code & ((1 << sbit) - 1)])
+    v = mag * Fraction(2) ** (sfc - 127)
+    return -v if code >> sbit & 1 else v
+
+
+def _codes_list(codes, K, fmt):
+    if fmt == oracle.E4M3:
+        return [int(c) for c in codes[:K]]
+    out = []
+    for b in codes:
+        out += [int(b) & 0xF, int(b) >> 4]
+    return out
+
+
+@pytest.mark.parametrize("M,N,K,fmt", [(3, 4, 32, oracle.E2M1), (4, 2, 64, oracle.E2M1),
+                                       (2, 3, 64, oracle.E4M3), (1, 1, 32, oracle.E4M3)])
+def test_linear_brute_force_exact(M, N, K, fmt):
+    rng = np.random.default_rng(M * 100 + N * 10 + K)
+    x = _bf16_bits((rng.standard_normal((M, K)) * 3).astype(np.float32).ravel()).reshape(M, K)
+    w = _bf16_bits((rng.standard_normal((N, K)) * 0.05).astype(np.float32).ravel()).reshape(N, K)
+    b = _bf16_bits(rng.standard_normal(N).astype(np.float32))
+    xc, xs = oracle.quantize(x, fmt)
+    wc, ws = oracle.quantize(w, oracle.E2M1)
+    y = oracle.linear(xc, xs, fmt, K, wc, ws, b)
+    for m in range(M):
+        xa = _codes_list(xc[m], K, fmt)
+        for n in range(N):
+            wa = _codes_list(wc[n], K, oracle.E2M1)
+            acc = Fraction(0)
+            for k in range(K):
+                acc += (_exact_value(xa[k], int(xs[m, k // 32]), fmt) *
+                        _exact_value(wa[k], int(ws[n, k // 32]), oracle.E2M1))
+            acc += Fraction(oracle.bf16_to_float(int(b[n])))
+            assert abs(float(acc) - y[m, n]) <= 1e-12 * max(1.0, abs(float(acc))), (m, n)
+
+
+def _mx_representable(rng, rows, K, fmt):
+    """Random bf16 matrices that are exactly MX-representable: random element codes
+    with one block element forced to the largest magnitude, and random scales."""
+    mags, sbit = GRID[fmt]
+    KB = K // 32
+    codes = rng.integers(0, len(mags), (rows, K))
+    codes[:, ::32] = len(mags) - 1
+    signs = rng.integers(0, 2, (rows, K))
+    sfc = rng.integers(110, 135, (rows, KB))
+    vals = np.array(mags)[codes] * np.where(signs, -1.0, 1.0) * 2.0 ** (np.repeat(sfc, 32, 1) - 127)
+    return _bf16_bits(vals.astype(np.float32).ravel()).reshape(rows, K), vals, sfc
+
+
+@pytest.mark.parametrize("fmt", [oracle.E2M1, oracle.E4M3])
+def test_linear_lossless_case_matches_numpy(fmt):
+    rng = np.random.default_rng(11)
+    M, N, K = 37, 29, 256
+    xb, xv, xsf = _mx_representable(rng, M, K, fmt)
+    wb, wv, wsf = _mx_representable(rng, N, K, oracle.E2M1)
+    xc, xs = oracle.quantize(xb, fmt)
+    wc, ws = oracle.quantize(wb, oracle.E2M1)
+    assert np.array_equal(xs.astype(int), xsf) and np.array_equal(ws.astype(int), wsf)
+    assert np.array_equal(oracle.dequantize(xc, xs, K, fmt), xv)
+    y = oracle.linear(xc, xs, fmt, K, wc, ws)
+    ref = xv @ wv.T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-300)
+    # rows subset and multi-threaded split give the same numbers
+    rows = np.array([36, 0, 17])
+    y2 = oracle.linear_rows(xc, xs, fmt, rows, K, wc, ws, nthreads=3)
+    assert np.array_equal(y2, y[rows])
