@@ -1,0 +1,311 @@
+// api.cu -- the C ABI of libmxq.so (declared in include/mxq.h): argument checks,
+// workspace layout, and dispatch to the quantizer, dequantizer and GEMM kernels.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "mxq_internal.h"
+
+using namespace mxq;
+
+namespace {
+
+thread_local char g_err[512] = "";
+thread_local char g_path[256] = "";
+
+int fail(int code, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int ok()
+{
+    g_err[0] = 0;
+    return MXQ_OK;
+}
+
+constexpr int64_t kMaxElems = int64_t(1) << 34;  // rows*K; keeps 32-bit group / scale indices exact
+constexpr int64_t kWsAlign = 256;
+constexpr int64_t kLtWorkspace = int64_t(32) << 20;
+
+int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_ptr(const void* p, const char* name, uintptr_t align = 16)
+{
+    if (!p) return fail(MXQ_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!aligned(p, align)) return fail(MXQ_ERR_ALIGN, "%s is not %zu-byte aligned", name, (size_t)align);
+    return MXQ_OK;
+}
+
+int check_fmt(int fmt)
+{
+    if (fmt != MXQ_FMT_E2M1 && fmt != MXQ_FMT_E4M3) return fail(MXQ_ERR_INVALID_ARG, "unknown format %d", fmt);
+    return MXQ_OK;
+}
+
+int check_rows_k(int64_t rows, int64_t K, const char* what)
+{
+    if (rows <= 0 || K <= 0) return fail(MXQ_ERR_INVALID_ARG, "%s: sizes must be positive (rows=%lld K=%lld)", what,
+                                         (long long)rows, (long long)K);
+    if (K % 32 != 0) return fail(MXQ_ERR_SHAPE, "%s: K=%lld is not a multiple of 32", what, (long long)K);
+    if (rows > (int64_t(1) << 31) - 1 || rows * K > kMaxElems)
+        return fail(MXQ_ERR_SHAPE, "%s: tensor too large (rows=%lld K=%lld)", what, (long long)rows, (long long)K);
+    return MXQ_OK;
+}
+
+// The kernels are built for sm_100a only.
+int check_device()
+{
+    static thread_local int checked_dev = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(MXQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev == checked_dev) return MXQ_OK;
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0)
+        return fail(MXQ_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library runs on sm_100 only", dev, major, minor);
+    checked_dev = dev;
+    return MXQ_OK;
+}
+
+int cuda_rc(cudaError_t e, const char* what)
+{
+    if (e != cudaSuccess) return fail(MXQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return ok();
+}
+
+#define RETURN_IF(x)                 \
+    do {                             \
+        int rc_ = (x);               \
+        if (rc_ != MXQ_OK) return rc_; \
+    } while (0)
+
+int check_gemm(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K, const void* w_codes,
+               const void* w_sf, int64_t N, const void* bias, const void* y)
+{
+    RETURN_IF(check_fmt(a_fmt));
+    RETURN_IF(check_rows_k(M, K, "activation"));
+    RETURN_IF(check_rows_k(N, K, "weight"));
+    if (N % 8 != 0) return fail(MXQ_ERR_SHAPE, "N=%lld is not a multiple of 8", (long long)N);
+    if (a_fmt == MXQ_FMT_E4M3 && K % 128 != 0)
+        return fail(MXQ_ERR_SHAPE, "W4A8 native GEMM needs K %% 128 == 0 (K=%lld)", (long long)K);
+    RETURN_IF(check_ptr(a_codes, "a_codes"));
+    RETURN_IF(check_ptr(a_sf, "a_sf"));
+    RETURN_IF(check_ptr(w_codes, "w_codes", a_fmt == MXQ_FMT_E4M3 ? 32 : 16));
+    RETURN_IF(check_ptr(w_sf, "w_sf"));
+    RETURN_IF(check_ptr(y, "y"));
+    if (bias) RETURN_IF(check_ptr(bias, "bias"));
+    return MXQ_OK;
+}
+
+int64_t linear_ws(int64_t M, int64_t N, int64_t K, int fmt, int mode)
+{
+    int64_t ws = round_up(codes_bytes(M, K, fmt), kWsAlign) + round_up(sf_bytes(M, K), kWsAlign);
+    if (mode == MXQ_MODE_QDQ)
+        ws += round_up(M * K * 2, kWsAlign) + round_up(N * K * 2, kWsAlign) + kLtWorkspace;
+    return ws;
+}
+
+int run_gemm(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K, const void* w_codes,
+             const void* w_sf, int64_t N, const void* bias, void* y, cudaStream_t stream)
+{
+    GemmArgs g{a_codes, a_sf, a_fmt, M, N, K, w_codes, w_sf, bias, y};
+    const char* msg = nullptr;
+    int rc = launch_gemm(g, stream, &msg, g_path, sizeof g_path);
+    if (rc != MXQ_OK) return fail(rc, "gemm: %s", msg ? msg : "launch failed");
+    return ok();
+}
+
+// Quantize x into the workspace, then GEMM (native) or dequantize + bf16 GEMM (QDQ).
+int run_linear(const void* x, int64_t M, int64_t K, const void* w_codes, const void* w_sf, int64_t N,
+               const void* bias, int fmt, int mode, void* workspace, int64_t ws_bytes, void* y,
+               cudaStream_t stream)
+{
+    const int64_t need = linear_ws(M, N, K, fmt, mode);
+    if (ws_bytes < need)
+        return fail(MXQ_ERR_WORKSPACE, "workspace has %lld bytes, needs %lld", (long long)ws_bytes, (long long)need);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint8_t* xc = ws;
+    uint8_t* xs = xc + round_up(codes_bytes(M, K, fmt), kWsAlign);
+    RETURN_IF(cuda_rc(launch_quantize(x, M, K, fmt, xc, xs, stream), "quantize launch"));
+    if (mode == MXQ_MODE_NATIVE) return run_gemm(xc, xs, fmt, M, K, w_codes, w_sf, N, bias, y, stream);
+
+    uint8_t* xd = xs + round_up(sf_bytes(M, K), kWsAlign);
+    uint8_t* wd = xd + round_up(M * K * 2, kWsAlign);
+    uint8_t* lt = wd + round_up(N * K * 2, kWsAlign);
+    RETURN_IF(cuda_rc(launch_dequantize(xc, xs, M, K, fmt, xd, stream), "dequantize launch"));
+    RETURN_IF(cuda_rc(launch_dequantize(w_codes, w_sf, N, K, MXQ_FMT_E2M1, wd, stream), "dequantize launch"));
+    const char* msg = nullptr;
+    int rc = qdq_bf16_gemm(xd, wd, bias, y, M, N, K, lt, static_cast<size_t>(kLtWorkspace), stream, &msg);
+    if (rc != MXQ_OK) return fail(rc, "qdq gemm: %s", msg ? msg : "failed");
+    snprintf(g_path, sizeof g_path, "qdq %s dequant + cublasLt bf16", fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1");
+    return ok();
+}
+
+int check_mode(int mode)
+{
+    if (mode != MXQ_MODE_NATIVE && mode != MXQ_MODE_QDQ) return fail(MXQ_ERR_INVALID_ARG, "unknown mode %d", mode);
+    return MXQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mxq_version(void) { return 100; }
+
+int64_t mxq_codes_bytes(int64_t rows, int64_t K, int fmt)
+{
+    if (rows <= 0 || K <= 0 || (fmt != MXQ_FMT_E2M1 && fmt != MXQ_FMT_E4M3)) return -1;
+    return codes_bytes(rows, K, fmt);
+}
+
+int64_t mxq_sf_bytes(int64_t rows, int64_t K)
+{
+    if (rows <= 0 || K <= 0 || K % 32 != 0) return -1;
+    return sf_bytes(rows, K);
+}
+
+int64_t mxq_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int mode)
+{
+    if (M <= 0 || N <= 0 || K <= 0 || K % 32 != 0) return -1;
+    if ((fmt != MXQ_FMT_E2M1 && fmt != MXQ_FMT_E4M3) || (mode != MXQ_MODE_NATIVE && mode != MXQ_MODE_QDQ)) return -1;
+    return linear_ws(M, N, K, fmt, mode);
+}
+
+int mxq_quantize_weight(const void* w_bf16, int64_t N, int64_t K, void* codes, void* sf, void* stream)
+{
+    return mxq_quantize_act(w_bf16, N, K, MXQ_FMT_E2M1, codes, sf, stream);
+}
+
+int mxq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int fmt, void* codes, void* sf, void* stream)
+{
+    RETURN_IF(check_fmt(fmt));
+    RETURN_IF(check_rows_k(M, K, "quantize"));
+    RETURN_IF(check_ptr(x_bf16, "x"));
+    RETURN_IF(check_ptr(codes, "codes"));
+    RETURN_IF(check_ptr(sf, "sf"));
+    RETURN_IF(check_device());
+    snprintf(g_path, sizeof g_path, "quantize %s", fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1");
+    return cuda_rc(launch_quantize(x_bf16, M, K, fmt, codes, sf, static_cast<cudaStream_t>(stream)),
+                   "quantize launch");
+}
+
+int mxq_dequantize(const void* codes, const void* sf, int64_t rows, int64_t K, int fmt, void* out_bf16,
+                   void* stream)
+{
+    RETURN_IF(check_fmt(fmt));
+    RETURN_IF(check_rows_k(rows, K, "dequantize"));
+    RETURN_IF(check_ptr(codes, "codes"));
+    RETURN_IF(check_ptr(sf, "sf"));
+    RETURN_IF(check_ptr(out_bf16, "out"));
+    RETURN_IF(check_device());
+    snprintf(g_path, sizeof g_path, "dequantize %s", fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1");
+    return cuda_rc(launch_dequantize(codes, sf, rows, K, fmt, out_bf16, static_cast<cudaStream_t>(stream)),
+                   "dequantize launch");
+}
+
+int mxq_gemm(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K, const void* w_codes,
+             const void* w_sf, int64_t N, const void* bias_bf16, void* y_bf16, void* stream)
+{
+    RETURN_IF(check_gemm(a_codes, a_sf, a_fmt, M, K, w_codes, w_sf, N, bias_bf16, y_bf16));
+    RETURN_IF(check_device());
+    return run_gemm(a_codes, a_sf, a_fmt, M, K, w_codes, w_sf, N, bias_bf16, y_bf16,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int mxq_linear(const void* x_bf16, int64_t M, int64_t K, const void* w_codes, const void* w_sf, int64_t N,
+               const void* bias_bf16, int act_fmt, int mode, void* workspace, int64_t ws_bytes, void* y_bf16,
+               void* stream)
+{
+    RETURN_IF(check_mode(mode));
+    RETURN_IF(check_ptr(x_bf16, "x"));
+    RETURN_IF(check_ptr(workspace, "workspace", kWsAlign));
+    // the workspace stands in for the quantized activation in the GEMM checks
+    RETURN_IF(check_gemm(workspace, workspace, act_fmt, M, K, w_codes, w_sf, N, bias_bf16, y_bf16));
+    RETURN_IF(check_device());
+    return run_linear(x_bf16, M, K, w_codes, w_sf, N, bias_bf16, act_fmt, mode, workspace, ws_bytes, y_bf16,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int64_t mxq_block_workspace_bytes(const mxq_wdesc* w, const int64_t* M_in, uint32_t w4a8_bits, int mode)
+{
+    if (!w || !M_in) return -1;
+    int64_t need = 0;
+    for (int i = 0; i < 8; ++i) {
+        const int fmt = (w4a8_bits >> i) & 1u ? MXQ_FMT_E4M3 : MXQ_FMT_E2M1;
+        const int64_t b = mxq_workspace_bytes(M_in[i], w[i].N, w[i].K, fmt, mode);
+        if (b < 0) return -1;
+        need = std::max(need, b);
+    }
+    return need;
+}
+
+int mxq_dit_block_linears(const mxq_wdesc* w, const void* const* x_in, const int64_t* M_in, void* const* y_out,
+                          uint32_t w4a8_bits, int mode, void* workspace, int64_t ws_bytes, void* stream)
+{
+    if (!w || !x_in || !M_in || !y_out) return fail(MXQ_ERR_INVALID_ARG, "block: NULL array argument");
+    if (w4a8_bits > 0xFFu) return fail(MXQ_ERR_INVALID_ARG, "block: w4a8_bits has bits above 7 (0x%x)", w4a8_bits);
+    RETURN_IF(check_mode(mode));
+    RETURN_IF(check_ptr(workspace, "workspace", kWsAlign));
+    for (int i = 0; i < 8; ++i) {
+        const int fmt = (w4a8_bits >> i) & 1u ? MXQ_FMT_E4M3 : MXQ_FMT_E2M1;
+        RETURN_IF(check_ptr(x_in[i], "block x_in[i]"));
+        int rc = check_gemm(workspace, workspace, fmt, M_in[i], w[i].K, w[i].codes, w[i].sf, w[i].N, w[i].bias,
+                            y_out[i]);
+        if (rc != MXQ_OK) return fail(rc, "block linear %d: %s", i, g_err);
+    }
+    const int64_t need = mxq_block_workspace_bytes(w, M_in, w4a8_bits, mode);
+    if (ws_bytes < need)
+        return fail(MXQ_ERR_WORKSPACE, "block workspace has %lld bytes, needs %lld", (long long)ws_bytes,
+                    (long long)need);
+    RETURN_IF(check_device());
+    for (int i = 0; i < 8; ++i) {
+        const int fmt = (w4a8_bits >> i) & 1u ? MXQ_FMT_E4M3 : MXQ_FMT_E2M1;
+        int rc = run_linear(x_in[i], M_in[i], w[i].K, w[i].codes, w[i].sf, w[i].N, w[i].bias, fmt, mode, workspace,
+                            ws_bytes, y_out[i], static_cast<cudaStream_t>(stream));
+        if (rc != MXQ_OK) return fail(rc, "block linear %d: %s", i, g_err);
+    }
+    snprintf(g_path, sizeof g_path, "block %s w4a8_bits 0x%02x", mode == MXQ_MODE_QDQ ? "qdq" : "native",
+             w4a8_bits);
+    return ok();
+}
+
+int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_rowmajor, void* stream)
+{
+    RETURN_IF(check_rows_k(rows, K, "sf_to_logical"));
+    RETURN_IF(check_ptr(sf_tiled, "sf_tiled"));
+    if (!sf_rowmajor) return fail(MXQ_ERR_INVALID_ARG, "sf_rowmajor is NULL");
+    RETURN_IF(check_device());
+    return cuda_rc(launch_sf_to_logical(sf_tiled, rows, K, sf_rowmajor, static_cast<cudaStream_t>(stream)),
+                   "sf_to_logical launch");
+}
+
+int mxq_poll_status(void* stream)
+{
+    uint32_t v = 0;
+    int rc = read_and_clear_device_status(static_cast<cudaStream_t>(stream), &v);
+    if (rc != MXQ_OK) return fail(rc, "reading the device status word failed");
+    if (v != 0) return fail(static_cast<int>(v), "a GEMM kernel's bounded wait ran out");
+    return ok();
+}
+
+int mxq_set_debug(uint32_t flags)
+{
+    set_debug_flags(flags);
+    return MXQ_OK;
+}
+
+const char* mxq_last_error(void) { return g_err; }
+const char* mxq_last_path(void) { return g_path; }
+
+}  // extern "C"

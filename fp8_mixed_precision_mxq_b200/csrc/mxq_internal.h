@@ -1,0 +1,53 @@
+// mxq_internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mxq.h"
+
+namespace mxq {
+
+// Element formats of the activation operand.
+constexpr int kFmtE2M1 = MXQ_FMT_E2M1;
+constexpr int kFmtE4M3 = MXQ_FMT_E4M3;
+
+// Tiled scale-factor layout: 512-byte atoms of 128 rows x 4 k-blocks.
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t sf_atoms_k(int64_t K) { return ceil_div(K / 32, 4); }
+inline int64_t sf_bytes(int64_t rows, int64_t K) { return ceil_div(rows, 128) * 128 * sf_atoms_k(K) * 4; }
+inline int64_t codes_bytes(int64_t rows, int64_t K, int fmt) { return fmt == kFmtE4M3 ? rows * K : rows * K / 2; }
+
+// ---- launchers (return cudaError_t of the launch) ----
+cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, int fmt, void* codes, void* sf,
+                            cudaStream_t stream);
+cudaError_t launch_dequantize(const void* codes, const void* sf, int64_t rows, int64_t K, int fmt, void* out,
+                              cudaStream_t stream);
+cudaError_t launch_sf_to_logical(const void* sf, int64_t rows, int64_t K, void* out, cudaStream_t stream);
+
+struct GemmArgs {
+    const void* a_codes;
+    const void* a_sf;
+    int a_fmt;  // kFmtE2M1 -> kind::mxf4, kFmtE4M3 -> kind::mxf8f6f4
+    int64_t M, N, K;
+    const void* w_codes;
+    const void* w_sf;
+    const void* bias;  // bf16 [N] or null
+    void* y;           // bf16 [M, N]
+};
+
+// Builds the tensor maps and launches the tcgen05 GEMM.  Returns an mxq_status;
+// on failure *msg points to a static description.
+int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* path, size_t path_len);
+
+// Device status word written by kernels whose bounded waits ran out.
+int read_and_clear_device_status(cudaStream_t stream, uint32_t* out);
+void set_debug_flags(uint32_t flags);
+uint32_t debug_flags();
+
+// bf16 GEMM of the quantize-dequantize emulation path (cuBLASLt).
+int qdq_bf16_gemm(const void* xd, const void* wd, const void* bias, void* y, int64_t M, int64_t N, int64_t K,
+                  void* workspace, size_t ws_bytes, cudaStream_t stream, const char** msg);
+
+}  // namespace mxq

@@ -1,0 +1,278 @@
+// quant.cu -- MX block quantizer / dequantizer kernels (HBM-bound).
+//
+// The quantizer implements the MX format as the blog "Quark Mixed-Precision
+// Quantization for Wan2.2 Video Generation on AMD Instinct GPUs" uses it (section
+// "Quantization formats"): per block of 32 consecutive elements along K, the
+// absolute maximum gives an E8M0 scale 2^(floor(log2 amax) - emax) (emax 2 for
+// E2M1, 8 for E4M3; clamped at 2^-127), and each element x / scale is rounded to
+// nearest-even onto the element grid with saturation (RTN).
+//
+// Work split: the tensor is read as a flat run of 16-byte groups of 8 bf16; four
+// consecutive lanes hold one 32-element block, so the block absmax takes two
+// xor-shuffles.  Each warp covers 256 consecutive elements per step; a warp step
+// keeps several 16-byte loads in flight per lane.
+#include <cuda_bf16.h>
+
+#include "mxq_internal.h"
+
+namespace mxq {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// |x| bit patterns of the two bf16 halves of w, packed max.
+__device__ __forceinline__ uint32_t abs_max2(uint32_t a, uint32_t b)
+{
+    return __vmaxu2(a & 0x7FFF7FFFu, b & 0x7FFF7FFFu);
+}
+
+__device__ __forceinline__ float lo_f(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Two fp32 -> one byte of two E2M1 codes (first argument in the low nibble).
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(lo), "f"(hi));
+    return r;
+}
+
+// Two fp32 -> two E4M3 codes in a 16-bit word (first argument in the low byte).
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+// Byte offset of scale (r, kb) in the tiled 128x4 atom layout.
+__device__ __forceinline__ uint32_t sf_offset(uint32_t r, uint32_t kb, uint32_t atoms_k)
+{
+    return ((r >> 7) * atoms_k + (kb >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + (kb & 3u);
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restrict__ x, uint32_t n_groups,
+                                                            uint32_t KB, uint32_t atoms_k, uint32_t rows,
+                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ sf)
+{
+    constexpr uint32_t kEmax = FMT == kFmtE4M3 ? 8u : 2u;
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t nwarps = gridDim.x * (kThreads / 32);
+    const uint32_t warp = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+
+    for (uint32_t w0 = warp; w0 * 32u < n_groups; w0 += nwarps * kUnroll) {
+        uint4 v[kUnroll];
+        uint32_t g[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            g[u] = (w0 + u * nwarps) * 32u + lane;
+            v[u] = g[u] < n_groups ? ld_stream(x + g[u]) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            // block absmax over the quad of lanes holding the 32 elements
+            uint32_t m2 = __vmaxu2(abs_max2(v[u].x, v[u].y), abs_max2(v[u].z, v[u].w));
+            uint32_t amax = max(m2 & 0xFFFFu, m2 >> 16);
+            amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+            amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+            if (g[u] >= n_groups) continue;
+            const uint32_t eb = amax >> 7;  // biased exponent of amax (bf16 and E8M0 share bias 127)
+            const uint32_t sc = eb == 255u ? 255u : (eb > kEmax ? eb - kEmax : 0u);
+            const float inv = __uint_as_float((254u - min(sc, 253u)) << 23);  // 2^(127 - sc)
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            if (FMT == kFmtE2M1) {
+                uint32_t out = 0, sgn = 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    out |= cvt_e2m1x2(lo_f(w[i]) * inv, hi_f(w[i]) * inv) << (8 * i);
+                    sgn |= (((w[i] >> 12) & 0x8u) | ((w[i] >> 24) & 0x80u)) << (8 * i);
+                }
+                out |= sgn;  // a negative value that rounds to zero keeps its sign
+                if (sc == 255u) out = 0;
+                reinterpret_cast<uint32_t*>(codes)[g[u]] = out;
+            } else {
+                uint32_t out[2], sgn[2];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const uint32_t a = w[2 * i], b = w[2 * i + 1];
+                    out[i] = cvt_e4m3x2(lo_f(a) * inv, hi_f(a) * inv) |
+                             (cvt_e4m3x2(lo_f(b) * inv, hi_f(b) * inv) << 16);
+                    sgn[i] = ((a >> 8) & 0x80u) | ((a >> 16) & 0x8000u) | ((b << 8) & 0x800000u) |
+                             (b & 0x80000000u);
+                    out[i] |= sgn[i];
+                    if (sc == 255u) out[i] = 0;
+                }
+                reinterpret_cast<uint2*>(codes)[g[u]] = make_uint2(out[0], out[1]);
+            }
+            if ((lane & 3u) == 0) {
+                const uint32_t blk = g[u] >> 2;
+                const uint32_t r = blk / KB, kb = blk - r * KB;
+                sf[sf_offset(r, kb, atoms_k)] = static_cast<uint8_t>(sc);
+            }
+        }
+    }
+
+    // zero the padding of the tiled scale buffer: k-blocks KB..4*atoms_k-1 of real
+    // rows, and every k-block of rows rows..ceil128(rows)-1
+    const uint32_t kbp = atoms_k * 4u;
+    const uint32_t pad_k = kbp - KB;
+    const uint32_t rows_p = (rows + 127u) & ~127u;
+    const uint32_t n_pad_a = rows * pad_k;
+    const uint32_t n_pad = n_pad_a + (rows_p - rows) * kbp;
+    for (uint32_t p = blockIdx.x * kThreads + threadIdx.x; p < n_pad; p += gridDim.x * kThreads) {
+        uint32_t r, kb;
+        if (p < n_pad_a) {
+            r = p / pad_k;
+            kb = KB + (p - r * pad_k);
+        } else {
+            const uint32_t q = p - n_pad_a;
+            r = rows + q / kbp;
+            kb = q - (q / kbp) * kbp;
+        }
+        sf[sf_offset(r, kb, atoms_k)] = 0;
+    }
+}
+
+// Value of an E2M1 magnitude code (0..7) as fp32.
+__device__ __forceinline__ float e2m1_mag(uint32_t m)
+{
+    const uint32_t bits = m >= 2u ? ((((m >> 1) + 126u) << 23) | ((m & 1u) << 22)) : (m == 1u ? 0x3F000000u : 0u);
+    return __uint_as_float(bits);
+}
+
+// Value of an E4M3 code (sign included) as fp32; 0x7F / 0xFF are NaN.
+__device__ __forceinline__ float e4m3_val(uint32_t c)
+{
+    const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+    float v = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : static_cast<float>(m) * 0.001953125f;
+    if ((c & 0x7Fu) == 0x7Fu) v = __uint_as_float(0x7FC00000u);
+    return (c & 0x80u) ? -v : v;
+}
+
+// 2^(sc - 127) as fp32 (2^-127 is an fp32 subnormal); NaN for sc = 255.
+__device__ __forceinline__ float scale_val(uint32_t sc)
+{
+    if (sc == 255u) return __uint_as_float(0x7FC00000u);
+    return sc ? __uint_as_float(sc << 23) : __uint_as_float(0x00400000u);
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads) dequantize_kernel(const uint8_t* __restrict__ codes,
+                                                              const uint8_t* __restrict__ sf, uint32_t n_groups,
+                                                              uint32_t KB, uint32_t atoms_k,
+                                                              uint4* __restrict__ out)
+{
+    for (uint32_t g = blockIdx.x * kThreads + threadIdx.x; g < n_groups; g += gridDim.x * kThreads) {
+        const uint32_t blk = g >> 2;
+        const uint32_t r = blk / KB, kb = blk - r * KB;
+        const float s = scale_val(sf[sf_offset(r, kb, atoms_k)]);
+        float f[8];
+        if (FMT == kFmtE2M1) {
+            const uint32_t c = reinterpret_cast<const uint32_t*>(codes)[g];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t n = (c >> (4 * i)) & 0xFu;
+                const float v = e2m1_mag(n & 7u) * s;
+                f[i] = (n & 8u) ? -v : v;
+            }
+        } else {
+            const uint2 c = reinterpret_cast<const uint2*>(codes)[g];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = e4m3_val(((i < 4 ? c.x : c.y) >> (8 * (i & 3))) & 0xFFu) * s;
+        }
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+            o[i] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        out[g] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+__global__ void sf_to_logical_kernel(const uint8_t* __restrict__ sf, uint32_t rows, uint32_t KB, uint32_t atoms_k,
+                                     uint8_t* __restrict__ out)
+{
+    const uint32_t n = rows * KB;
+    for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const uint32_t r = i / KB, kb = i - r * KB;
+        out[i] = sf[sf_offset(r, kb, atoms_k)];
+    }
+}
+
+int num_sms()
+{
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, int fmt, void* codes, void* sf,
+                            cudaStream_t stream)
+{
+    const uint32_t n_groups = static_cast<uint32_t>(rows * K / 8);
+    const uint32_t KB = static_cast<uint32_t>(K / 32);
+    const uint32_t atoms_k = static_cast<uint32_t>(sf_atoms_k(K));
+    const int64_t want = ceil_div(n_groups, kThreads * kUnroll);
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * 8)));
+    if (fmt == kFmtE4M3)
+        quantize_kernel<kFmtE4M3><<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(x), n_groups, KB,
+                                                                 atoms_k, static_cast<uint32_t>(rows),
+                                                                 static_cast<uint8_t*>(codes),
+                                                                 static_cast<uint8_t*>(sf));
+    else
+        quantize_kernel<kFmtE2M1><<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(x), n_groups, KB,
+                                                                 atoms_k, static_cast<uint32_t>(rows),
+                                                                 static_cast<uint8_t*>(codes),
+                                                                 static_cast<uint8_t*>(sf));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const void* codes, const void* sf, int64_t rows, int64_t K, int fmt, void* out,
+                              cudaStream_t stream)
+{
+    const uint32_t n_groups = static_cast<uint32_t>(rows * K / 8);
+    const uint32_t KB = static_cast<uint32_t>(K / 32);
+    const uint32_t atoms_k = static_cast<uint32_t>(sf_atoms_k(K));
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(n_groups, kThreads),
+                                                                             num_sms() * 8)));
+    if (fmt == kFmtE4M3)
+        dequantize_kernel<kFmtE4M3><<<grid, kThreads, 0, stream>>>(static_cast<const uint8_t*>(codes),
+                                                                   static_cast<const uint8_t*>(sf), n_groups, KB,
+                                                                   atoms_k, static_cast<uint4*>(out));
+    else
+        dequantize_kernel<kFmtE2M1><<<grid, kThreads, 0, stream>>>(static_cast<const uint8_t*>(codes),
+                                                                   static_cast<const uint8_t*>(sf), n_groups, KB,
+                                                                   atoms_k, static_cast<uint4*>(out));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sf_to_logical(const void* sf, int64_t rows, int64_t K, void* out, cudaStream_t stream)
+{
+    const uint32_t n = static_cast<uint32_t>(rows * (K / 32));
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(n, 256), 4096)));
+    sf_to_logical_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint8_t*>(sf), static_cast<uint32_t>(rows),
+                                                   static_cast<uint32_t>(K / 32),
+                                                   static_cast<uint32_t>(sf_atoms_k(K)),
+                                                   static_cast<uint8_t*>(out));
+    return cudaGetLastError();
+}
+
+}  // namespace mxq

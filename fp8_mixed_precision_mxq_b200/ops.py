@@ -1,0 +1,168 @@
+"""Tensor-level entry points: the same calls as the C ABI (include/mxq.h), taking torch
+tensors for device memory and the current torch stream.  Nothing here computes:
+each function checks dtypes and devices, allocates outputs with torch, and calls the
+library."""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+from ._lib import FMT_E2M1, FMT_E4M3, MODE_NATIVE, MODE_QDQ, WDesc, check
+
+_FMTS = {"e2m1": FMT_E2M1, "e4m3": FMT_E4M3, FMT_E2M1: FMT_E2M1, FMT_E4M3: FMT_E4M3}
+_MODES = {"native": MODE_NATIVE, "qdq": MODE_QDQ, MODE_NATIVE: MODE_NATIVE, MODE_QDQ: MODE_QDQ}
+
+
+def _fmt(f) -> int:
+    return _FMTS[f]
+
+
+def _mode(m) -> int:
+    return _MODES[m]
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _p(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _cuda_bf16(t: torch.Tensor, name: str) -> None:
+    if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+        raise ValueError("%s must be a contiguous bf16 CUDA tensor" % name)
+
+
+def codes_bytes(rows: int, K: int, fmt="e2m1") -> int:
+    return int(_lib.lib().mxq_codes_bytes(rows, K, _fmt(fmt)))
+
+
+def sf_bytes(rows: int, K: int) -> int:
+    return int(_lib.lib().mxq_sf_bytes(rows, K))
+
+
+def workspace_bytes(M: int, N: int, K: int, fmt="e2m1", mode="native") -> int:
+    return int(_lib.lib().mxq_workspace_bytes(M, N, K, _fmt(fmt), _mode(mode)))
+
+
+@dataclass
+class QWeight:
+    """MXFP4 weight of one linear layer: codes [N, K/2], tiled scales, optional bias."""
+    codes: torch.Tensor
+    sf: torch.Tensor
+    N: int
+    K: int
+    bias: torch.Tensor | None = None
+
+    def desc(self) -> WDesc:
+        return WDesc(self.codes.data_ptr(), self.sf.data_ptr(),
+                     0 if self.bias is None else self.bias.data_ptr(), self.N, self.K)
+
+
+def quantize_act(x: torch.Tensor, fmt="e2m1", codes=None, sf=None, stream=None):
+    """x [M, K] bf16 -> (codes, tiled scales) in format fmt."""
+    _cuda_bf16(x, "x")
+    M, K = x.shape
+    f = _fmt(fmt)
+    if codes is None:
+        codes = torch.empty(max(1, codes_bytes(M, K, f)), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(max(1, sf_bytes(M, K)), dtype=torch.uint8, device=x.device)
+    check(_lib.lib().mxq_quantize_act(_p(x), M, K, f, _p(codes), _p(sf), _stream(stream)), "mxq_quantize_act")
+    return codes, sf
+
+
+def quantize_weight(w: torch.Tensor, bias: torch.Tensor | None = None, stream=None) -> QWeight:
+    """w [N, K] bf16 -> QWeight (MXFP4 codes [N, K/2] + tiled scales)."""
+    _cuda_bf16(w, "w")
+    N, K = w.shape
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    sf = torch.empty(max(1, sf_bytes(N, K)), dtype=torch.uint8, device=w.device)
+    check(_lib.lib().mxq_quantize_weight(_p(w), N, K, _p(codes), _p(sf), _stream(stream)), "mxq_quantize_weight")
+    if bias is not None:
+        _cuda_bf16(bias, "bias")
+    return QWeight(codes, sf, N, K, bias)
+
+
+def dequantize(codes: torch.Tensor, sf: torch.Tensor, rows: int, K: int, fmt="e2m1", out=None, stream=None):
+    if out is None:
+        out = torch.empty((rows, K), dtype=torch.bfloat16, device=codes.device)
+    check(_lib.lib().mxq_dequantize(_p(codes), _p(sf), rows, K, _fmt(fmt), _p(out), _stream(stream)),
+          "mxq_dequantize")
+    return out
+
+
+def gemm(a_codes, a_sf, fmt, M: int, K: int, w: QWeight, out=None, stream=None):
+    """GEMM on an already-quantized activation: y [M, N] bf16."""
+    if out is None:
+        out = torch.empty((M, w.N), dtype=torch.bfloat16, device=a_codes.device)
+    check(_lib.lib().mxq_gemm(_p(a_codes), _p(a_sf), _fmt(fmt), M, K, _p(w.codes), _p(w.sf), w.N, _p(w.bias),
+                              _p(out), _stream(stream)), "mxq_gemm")
+    return out
+
+
+def linear(x: torch.Tensor, w: QWeight, fmt="e2m1", mode="native", workspace=None, out=None, stream=None):
+    """y = x . deq(w)^T + bias with x quantized on the fly to fmt (E2M1 = W4A4, E4M3 = W4A8)."""
+    _cuda_bf16(x, "x")
+    M, K = x.shape
+    f, m = _fmt(fmt), _mode(mode)
+    need = workspace_bytes(M, w.N, K, f, m)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
+    check(_lib.lib().mxq_linear(_p(x), M, K, _p(w.codes), _p(w.sf), w.N, _p(w.bias), f, m, _p(workspace),
+                                workspace.numel() * workspace.element_size(), _p(out), _stream(stream)),
+          "mxq_linear")
+    return out
+
+
+def block_workspace_bytes(weights, rows, w4a8_bits: int, mode="native") -> int:
+    descs = (WDesc * 8)(*[w.desc() for w in weights])
+    ms = (ctypes.c_int64 * 8)(*rows)
+    return int(_lib.lib().mxq_block_workspace_bytes(descs, ms, w4a8_bits, _mode(mode)))
+
+
+def dit_block_linears(weights, xs, w4a8_bits: int, mode="native", workspace=None, outs=None, stream=None):
+    """The eight linears of one DiT block (QKV, attn-out, cross-Q/K/V/out, FFN-up,
+    FFN-down); bit i of w4a8_bits selects W4A8 for linear i."""
+    assert len(weights) == 8 and len(xs) == 8
+    rows = [int(x.shape[0]) for x in xs]
+    for x in xs:
+        _cuda_bf16(x, "block input")
+    if outs is None:
+        outs = [torch.empty((r, w.N), dtype=torch.bfloat16, device=xs[0].device) for r, w in zip(rows, weights)]
+    need = block_workspace_bytes(weights, rows, w4a8_bits, mode)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=xs[0].device)
+    descs = (WDesc * 8)(*[w.desc() for w in weights])
+    xin = (ctypes.c_void_p * 8)(*[x.data_ptr() for x in xs])
+    ms = (ctypes.c_int64 * 8)(*rows)
+    yout = (ctypes.c_void_p * 8)(*[y.data_ptr() for y in outs])
+    check(_lib.lib().mxq_dit_block_linears(descs, xin, ms, yout, w4a8_bits, _mode(mode), _p(workspace),
+                                           workspace.numel(), _stream(stream)), "mxq_dit_block_linears")
+    return outs
+
+
+def sf_to_logical(sf: torch.Tensor, rows: int, K: int, stream=None) -> torch.Tensor:
+    out = torch.empty((rows, K // 32), dtype=torch.uint8, device=sf.device)
+    check(_lib.lib().mxq_sf_to_logical(_p(sf), rows, K, _p(out), _stream(stream)), "mxq_sf_to_logical")
+    return out
+
+
+def poll_status(stream=None) -> int:
+    """Synchronizes the stream and returns the device status word (0 = fine)."""
+    return int(_lib.lib().mxq_poll_status(_stream(stream)))
+
+
+def set_debug(flags: int) -> None:
+    _lib.lib().mxq_set_debug(flags)
+
+
+def last_path() -> str:
+    return _lib.last_path()

@@ -1,0 +1,166 @@
+/*
+ * mxq.h -- C ABI of libmxq.so: the MX block-quantized linear layer on B200 (sm_100a).
+ *
+ * The operation is the one the blog "Quark Mixed-Precision Quantization for Wan2.2
+ * Video Generation on AMD Instinct GPUs" studies:
+ *   - W4A4 = OCP MXFP4 weights with dynamic MXFP4 activations, W4A8 = MXFP4 weights
+ *     with FP8 E4M3 activations (section "Quantization formats", its table);
+ *   - the MX format is the OCP Microscaling spec v1.0 (the blog's reference [7]):
+ *     blocks of 32 consecutive elements along K share one E8M0 scale
+ *     X = 2^(floor(log2(amax)) - emax) (emax 2 for E2M1, 8 for E4M3; clamped at
+ *     2^-127), and each element is stored as round-to-nearest-even(x / X) on the
+ *     element grid, saturating at the largest finite element ("RTN" in the
+ *     section "Results" tables);
+ *   - a block whose input holds Inf or NaN gets scale code 0xFF and zero codes;
+ *     a negative value that rounds to zero keeps its sign bit;
+ *   - the linear layer is Y = deq(Xq) . deq(Wq)^T (+ bias) with fp32 accumulation
+ *     and a bf16 output (section "Quantization formats", "Kernel note": native
+ *     MXFP4 GEMM for W4A4; quantize-dequantize emulation for W4A8);
+ *   - a per-expert, per-block policy picks W4A4 or W4A8 for each DiT block
+ *     (sections "Mixed-Precision selection" and "Practical workflow", step 6).
+ *
+ * Conventions for every entry point:
+ *   - Shapes follow torch.nn.Linear: X is [M, K] (tokens x in-features), W is
+ *     [N, K] (out x in-features), Y is [M, N]; all row-major, K contiguous.
+ *   - All data pointers are DEVICE pointers the caller allocated and owns (for
+ *     example torch tensors); the library never allocates or frees device memory
+ *     and never synchronizes.  `stream` is a cudaStream_t (NULL = legacy default
+ *     stream); all work is enqueued on it and runs asynchronously.
+ *   - Element codes: E2M1 packs two per byte, element 2j in the low nibble of
+ *     byte j and element 2j+1 in the high nibble ([rows, K/2] bytes); E4M3 uses one
+ *     byte per element ([rows, K] bytes).
+ *   - Scale factors (E8M0 bytes) are stored in the tiled layout the tcgen05
+ *     block-scaled MMA reads: 512-byte atoms of 128 rows x 4 k-blocks, the byte of
+ *     (row r, k-block kb) at offset (r%32)*16 + ((r/32)%4)*4 + kb%4 inside atom
+ *     (r/128)*ceil(K/128) + kb/4.  Rows are padded to 128 and k-blocks to a
+ *     multiple of 4; the quantizers write the padding as 0.
+ *   - Every call returns an mxq_status.  Arguments are validated before anything
+ *     is enqueued, so on an error nothing was launched; mxq_last_error() then
+ *     describes it.  Kernel launch failures return MXQ_ERR_CUDA.  The GEMM's
+ *     internal waits are bounded; if one ever runs out, the kernel records
+ *     MXQ_ERR_TIMEOUT in a device status word that mxq_poll_status() returns.
+ */
+#ifndef MXQ_H
+#define MXQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MXQ_OK = 0,
+    MXQ_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, unknown enum value   */
+    MXQ_ERR_SHAPE = 2,       /* K % 32 != 0, N % 8 != 0, W4A8 native with K % 128 != 0 */
+    MXQ_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned (32 for W4A8 weights) */
+    MXQ_ERR_UNSUPPORTED = 4, /* the current device is not sm_100                        */
+    MXQ_ERR_CUDA = 5,        /* a CUDA runtime / driver / cuBLASLt call failed          */
+    MXQ_ERR_TIMEOUT = 6,     /* a bounded device-side wait ran out                      */
+    MXQ_ERR_WORKSPACE = 7    /* the workspace passed is smaller than required           */
+} mxq_status;
+
+typedef enum { MXQ_FMT_E2M1 = 0, MXQ_FMT_E4M3 = 1 } mxq_fmt;      /* activation element format */
+typedef enum { MXQ_MODE_NATIVE = 0, MXQ_MODE_QDQ = 1 } mxq_mode;  /* GEMM execution mode       */
+
+/* Library version (major*10000 + minor*100 + patch). */
+int mxq_version(void);
+
+/* Bytes of the element codes of a [rows, K] tensor: rows*K/2 (E2M1) or rows*K (E4M3). */
+int64_t mxq_codes_bytes(int64_t rows, int64_t K, int fmt);
+
+/* Bytes of the tiled scale-factor buffer of a [rows, K] tensor:
+ * ceil(rows/128)*128 * ceil(K/128)*4. */
+int64_t mxq_sf_bytes(int64_t rows, int64_t K);
+
+/* Workspace bytes mxq_linear needs for these sizes, format and mode (native: the
+ * quantized activation; QDQ: also both dequantized operands in bf16 and a cuBLASLt
+ * workspace).  Returns -1 on invalid sizes. */
+int64_t mxq_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int mode);
+
+/* Weight quantization (load time), always to MXFP4 (E2M1).
+ * Blog section "Quantization formats": "OCP MXFP4 weights", RTN.
+ *   w_bf16 [N, K] bf16 (16-byte aligned) -> codes [N, K/2] bytes, sf tiled
+ *   (mxq_sf_bytes(N, K) bytes).  Requires K % 32 == 0. */
+int mxq_quantize_weight(const void* w_bf16, int64_t N, int64_t K, void* codes, void* sf, void* stream);
+
+/* Dynamic activation quantization to MXFP4 (fmt E2M1) or to E4M3 with 32-element
+ * E8M0 block scales (fmt E4M3).
+ * Blog section "Quantization formats": "dynamic MXFP4 activations" (W4A4) and
+ * "FP8 E4M3 ... activations" (W4A8).
+ *   x_bf16 [M, K] -> codes (mxq_codes_bytes(M, K, fmt) bytes), sf tiled.
+ *   Requires K % 32 == 0; x, codes and sf 16-byte aligned. */
+int mxq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int fmt, void* codes, void* sf, void* stream);
+
+/* Dequantization to bf16 (the "QDQ" of the blog's intro and "Kernel note"):
+ *   out[r, k] = bf16(decode(code[r, k]) * 2^(sf[r, k/32] - 127)).
+ * The product is exact in bf16 except for E4M3 subnormals with scale codes below
+ * about 6, which round.  Scale code 0xFF gives NaN. */
+int mxq_dequantize(const void* codes, const void* sf, int64_t rows, int64_t K, int fmt, void* out_bf16,
+                   void* stream);
+
+/* GEMM on already-quantized operands (native tcgen05 block-scaled MMA):
+ *   y[M, N] = bf16( sum_k deqA[m, k] * deqW[n, k] + bias[n] ), fp32 accumulation.
+ * a_fmt E2M1 -> kind::mxf4 (W4A4); E4M3 -> kind::mxf8f6f4 (W4A8, needs K % 128 == 0
+ * and a 32-byte aligned w_codes).  bias_bf16 may be NULL.  Requires N % 8 == 0.
+ * Blog section "Quantization formats", "Kernel note". */
+int mxq_gemm(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K, const void* w_codes,
+             const void* w_sf, int64_t N, const void* bias_bf16, void* y_bf16, void* stream);
+
+/* The quantized linear layer: quantize x (fmt act_fmt) into the workspace, then
+ *   mode NATIVE: mxq_gemm on the quantized operands;
+ *   mode QDQ:    dequantize both operands to bf16 and run a bf16 GEMM (cuBLASLt),
+ *                the quantize-dequantize emulation the blog's W4A8 numbers use.
+ * workspace: device buffer of at least mxq_workspace_bytes(M, N, K, act_fmt, mode)
+ * bytes, 256-byte aligned; its contents are scratch.  Blog sections "Quantization
+ * formats" and "Kernel note". */
+int mxq_linear(const void* x_bf16, int64_t M, int64_t K, const void* w_codes, const void* w_sf, int64_t N,
+               const void* bias_bf16, int act_fmt, int mode, void* workspace, int64_t ws_bytes, void* y_bf16,
+               void* stream);
+
+/* One linear layer's quantized weights. */
+typedef struct {
+    const void* codes; /* E2M1 [N, K/2]            */
+    const void* sf;    /* tiled scale factors      */
+    const void* bias;  /* bf16 [N] or NULL         */
+    int64_t N, K;
+} mxq_wdesc;
+
+/* The eight linears of one DiT block, issued in order on one stream:
+ *   0 QKV, 1 attn-out, 2 cross-Q, 3 cross-K, 4 cross-V, 5 cross-out, 6 FFN-up,
+ *   7 FFN-down.
+ * Linear i reads x_in[i] [M_in[i], w[i].K] and writes y_out[i] [M_in[i], w[i].N];
+ * bit i of w4a8_bits set -> that linear runs W4A8 (E4M3 activations), else W4A4.
+ * The per-expert, per-block policy of the blog (sections "Mixed-Precision
+ * selection", "Practical workflow" step 6) is applied by passing 0xFF or 0x00 (or a
+ * per-linear refinement) for each (expert, block).  workspace must hold
+ * mxq_block_workspace_bytes(...) bytes. */
+int mxq_dit_block_linears(const mxq_wdesc* w, const void* const* x_in, const int64_t* M_in,
+                          void* const* y_out, uint32_t w4a8_bits, int mode, void* workspace, int64_t ws_bytes,
+                          void* stream);
+
+/* Workspace bytes mxq_dit_block_linears needs for these weights and row counts. */
+int64_t mxq_block_workspace_bytes(const mxq_wdesc* w, const int64_t* M_in, uint32_t w4a8_bits, int mode);
+
+/* Tiled scale factors -> logical row-major [rows, K/32] bytes (for tests). */
+int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_rowmajor, void* stream);
+
+/* Synchronizes `stream`, then returns (and clears) the device status word: MXQ_OK,
+ * or MXQ_ERR_TIMEOUT if a bounded wait of a GEMM kernel ran out since the last poll. */
+int mxq_poll_status(void* stream);
+
+/* Debug flags (0 = none).  Bit 0: the GEMM's producer skips the first stage's load,
+ * so the consumer's bounded wait runs out and the kernel reports MXQ_ERR_TIMEOUT. */
+int mxq_set_debug(uint32_t flags);
+
+/* Thread-local description of the last error, and of the last path taken
+ * (for example "native mxf4 1cta 128x256 grid 148"). */
+const char* mxq_last_error(void);
+const char* mxq_last_path(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXQ_H */

@@ -1,0 +1,100 @@
+"""The C-ABI library loads, exports every symbol include/mxq.h declares, and rejects bad
+arguments before touching the GPU (these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp8_mixed_precision_mxq_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxq.h")
+
+V = ctypes.c_void_p
+A16 = V(4096)          # a 16-byte aligned non-null dummy pointer (never dereferenced)
+A8 = V(4096 + 8)       # misaligned
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(mxq_[a-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("mxq_quantize_weight", "mxq_quantize_act", "mxq_linear", "mxq_dit_block_linears",
+                 "mxq_gemm", "mxq_dequantize", "mxq_last_error"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = _lib.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert name in _lib.SIGNATURES, "binding lacks " + name
+
+
+def test_sizes():
+    L = _lib.lib()
+    assert L.mxq_codes_bytes(3, 64, 0) == 96
+    assert L.mxq_codes_bytes(3, 64, 1) == 192
+    assert L.mxq_sf_bytes(1, 32) == 128 * 4
+    assert L.mxq_sf_bytes(129, 160) == 256 * 8
+    assert L.mxq_sf_bytes(32760, 5120) == 32768 * 160
+    assert L.mxq_sf_bytes(5, 48) == -1
+    assert L.mxq_workspace_bytes(0, 8, 32, 0, 0) == -1
+    assert L.mxq_workspace_bytes(128, 256, 1024, 0, 0) == 128 * 512 + 128 * 32
+    assert L.mxq_workspace_bytes(128, 256, 1024, 1, 1) > L.mxq_workspace_bytes(128, 256, 1024, 1, 0)
+
+
+@pytest.mark.parametrize("args,status", [
+    ((None, 4, 64, 0, A16, A16, None), _lib.ERR_INVALID_ARG),      # null input
+    ((A16, 0, 64, 0, A16, A16, None), _lib.ERR_INVALID_ARG),       # M = 0
+    ((A16, 4, 48, 0, A16, A16, None), _lib.ERR_SHAPE),             # K % 32 != 0
+    ((A16, 4, 64, 2, A16, A16, None), _lib.ERR_INVALID_ARG),       # unknown format
+    ((A8, 4, 64, 0, A16, A16, None), _lib.ERR_ALIGN),              # misaligned input
+    ((A16, 4, 64, 1, A8, A16, None), _lib.ERR_ALIGN),              # misaligned codes
+])
+def test_quantize_rejects_bad_arguments(args, status):
+    L = _lib.lib()
+    assert L.mxq_quantize_act(*args) == status
+    assert _lib.last_error()
+
+
+def test_gemm_rejects_bad_arguments():
+    L = _lib.lib()
+    ok = (A16, A16, 0, 128, 256, A16, A16, 256, None, A16, None)
+    bad = [
+        ((A16, A16, 0, 128, 256, A16, A16, 250, None, A16, None), _lib.ERR_SHAPE),   # N % 8
+        ((A16, A16, 1, 128, 96, A16, A16, 256, None, A16, None), _lib.ERR_SHAPE),    # W4A8 K % 128
+        ((A16, A16, 1, 128, 256, A8, A16, 256, None, A16, None), _lib.ERR_ALIGN),    # W4A8 weight 32B
+        ((A16, A16, 0, 128, 256, A16, A16, 256, A8, A16, None), _lib.ERR_ALIGN),     # bias
+        ((A16, None, 0, 128, 256, A16, A16, 256, None, A16, None), _lib.ERR_INVALID_ARG),
+        ((A16, A16, 0, -3, 256, A16, A16, 256, None, A16, None), _lib.ERR_INVALID_ARG),
+    ]
+    for args, status in bad:
+        assert L.mxq_gemm(*args) == status, (args, _lib.last_error())
+    # valid arguments get past validation and only then need a device
+    rc = L.mxq_gemm(*ok)
+    assert rc in (_lib.ERR_CUDA, _lib.ERR_UNSUPPORTED, _lib.OK)
+
+
+def test_linear_rejects_small_workspace_and_bad_mode():
+    L = _lib.lib()
+    ws = V(1 << 20)
+    assert L.mxq_linear(A16, 128, 256, A16, A16, 256, None, 0, 7, ws, 1 << 30, A16, None) == _lib.ERR_INVALID_ARG
+    assert L.mxq_linear(A16, 128, 256, A16, A16, 256, None, 0, 0, V(4096 + 16), 1 << 30, A16,
+                        None) == _lib.ERR_ALIGN   # workspace must be 256-byte aligned
+
+
+def test_block_rejects_bad_mask():
+    L = _lib.lib()
+    descs = (_lib.WDesc * 8)()
+    xs = (ctypes.c_void_p * 8)()
+    ms = (ctypes.c_int64 * 8)()
+    ys = (ctypes.c_void_p * 8)()
+    assert L.mxq_dit_block_linears(descs, xs, ms, ys, 0x100, 0, A16, 0, None) == _lib.ERR_INVALID_ARG
+    assert L.mxq_dit_block_linears(None, xs, ms, ys, 0, 0, A16, 0, None) == _lib.ERR_INVALID_ARG
