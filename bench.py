@@ -1,0 +1,423 @@
+"""Benchmark of the MX block-quantized linear layer on B200.
+
+A step is one pass of the hot path over one batch: the dynamic activation quantizer
+followed by the block-scaled tcgen05 GEMM (mxq_linear), on the W4A4 FFN-up linear of a
+Wan2.2-A14B-shaped DiT block at 480p / 81 frames (M = 32760 tokens, K = 5120,
+N = 13824; Student-t activations with 1% outlier channels, N(0, 0.02^2) weights,
+random-init, synthetic).  The MXFP4 weight is quantized once, before timing (it is a
+load-time step).  Beside the headline number the JSON line carries:
+  roofline      the dominant kernel (the GEMM) against the tensor-core peak, timed
+                alone with CUDA events on its launch stream;
+  parts         the quantizer (GB/s against HBM) and the GEMM separately;
+  w4a8          the W4A8 FFN-down linear at 720p (quantize to E4M3 + mxf8f6f4 GEMM)
+                and its quantize-dequantize emulation (QDQ) path;
+  e2e           the same step through host buffers (pinned H2D of x, D2H of y);
+  cpu_baseline  the CPU oracle on a bounded sample of the same workload.
+
+Multi-GPU: the layer has no exchange step (token rows are independent), so N GPUs
+run N replicas, each on its own 32760-row batch (weak scaling, no collective on the
+data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0   # nominal dense ratio: 9 PFLOP/s FP4 vs 2.25 PFLOP/s bf16
+FP8_OVER_BF16 = 2.0   # 4.5 PFLOP/s FP8
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 5.0 and self.proc.poll() is None:
+                time.sleep(0.02)  # the timed region starts once sampling is live
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- timing
+def time_loop(fn, iters: int, stream) -> float:
+    """Average milliseconds of fn() over iters runs, CUDA events on `stream`."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(iters):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / iters
+
+
+def quant_bytes(M, K, fmt):
+    return 2 * M * K + (M * K if fmt == "e4m3" else M * K // 2) + M * K // 32
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def cpu_baseline(M, N, K, fmt, seed, budget_s=12.0):
+    """The CPU oracle as it stands: quantize a slice of activation rows and run the
+    fp64 linear for them against the pre-quantized weight, for about budget_s seconds."""
+    import numpy as np
+
+    import oracle
+    import synth
+    f = oracle.E2M1 if fmt == "e2m1" else oracle.E4M3
+    w = synth.weight(N, K, seed=seed)
+    wb = w.view(torch.int16).numpy().view(np.uint16)
+    wc, ws = oracle.quantize(wb, oracle.E2M1)
+    chunk = 32
+    rows_done, flops = 0, 0.0
+    t0 = time.perf_counter()
+    while True:
+        x = synth.activation(chunk, K, "student_t" if fmt == "e2m1" else "gelu", seed=seed + rows_done,
+                             outlier_frac=0.01, outlier_scale=50.0)
+        xb = x.view(torch.int16).numpy().view(np.uint16)
+        xc, xs = oracle.quantize(xb, f)
+        oracle.linear(xc, xs, f, K, wc, ws)
+        flops += 2.0 * chunk * N * K
+        rows_done += chunk
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.default_threads(), "kind": "oracle",
+            "sample": "%d of %d activation rows of the %dx%dx%d %s linear (quantize + fp64 GEMM on the "
+                      "dequantized operands; weight quantized beforehand), %.1f s" % (rows_done, M, M, N, K, fmt,
+                                                                                    dt)}
+
+
+# ---------------------------------------------------------------------------- main arms
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def run_mxq(args):
+    import synth
+    from fp8_mixed_precision_mxq_b200 import ops
+
+    world, rank, local = dist_setup()
+    peaks, peak_src = load_peaks()
+    wl_name = args.workload
+    c = synth.WORKLOADS[wl_name]
+    M, K, N, fmt = (args.M or c["M"]), c["K"], c["N"], c["fmt"]
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    # inputs (per-rank seed offset: every replica gets its own batch)
+    x = synth.activation(M, K, c["act"], seed=c["seed"] + 1000 * rank, device=dev,
+                         outlier_frac=c.get("outlier_frac", 0.0), outlier_scale=c["outlier_scale"])
+    w = synth.weight(N, K, seed=c["seed"], device=dev)
+    b = synth.bias(N, seed=c["seed"], device=dev)
+    qw = ops.quantize_weight(w, bias=b)
+    ws = torch.empty(ops.workspace_bytes(M, N, K, fmt), dtype=torch.uint8, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    assert ops.poll_status() == 0
+
+    def step():
+        ops.linear(x, qw, fmt=fmt, workspace=ws, out=y)
+
+    if args.only:
+        # profiling mode: only the named kernel, `steps` launches after the warm-up
+        return profile_one(args, ops, x, qw, ws, y, M, N, K, fmt, stream)
+
+    for _ in range(args.warmup):
+        step()
+    barrier(world)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        ms = time_loop(step, args.steps, stream)
+        barrier(world)
+    ms = max_over_ranks(ms, world)
+    status = ops.poll_status()
+    if status != 0:
+        raise RuntimeError("device status %d after the timed steps" % status)
+    flops = 2.0 * M * N * K
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # the two kernels of the step, each timed alone on the launch stream
+    xc = ws[: ops.codes_bytes(M, K, fmt)]
+    xs_off = (ops.codes_bytes(M, K, fmt) + 255) // 256 * 256
+    xs = ws[xs_off: xs_off + ops.sf_bytes(M, K)]
+    for _ in range(3):
+        ops.quantize_act(x, fmt, codes=xc, sf=xs)
+    q_ms = time_loop(lambda: ops.quantize_act(x, fmt, codes=xc, sf=xs), args.steps, stream)
+    for _ in range(3):
+        ops.gemm(xc, xs, fmt, M, K, qw, out=y)
+    g_ms = time_loop(lambda: ops.gemm(xc, xs, fmt, M, K, qw, out=y), args.steps, stream)
+    gemm_path = ops.last_path()
+    q_ms, g_ms = max_over_ranks(q_ms, world), max_over_ranks(g_ms, world)
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    g_tflops = flops / (g_ms * 1e-3) / 1e12
+    q_gbs = quant_bytes(M, K, fmt) / (q_ms * 1e-3) / 1e9
+
+    result = {
+        "metric": "W4A4 MX linear TFLOP/s (fused dynamic MXFP4 activation quantize + tcgen05 mxf4 GEMM)",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e2m1 x e2m1 -> fp32 accumulate -> bf16", "data": "synthetic",
+        "config": {"workload": "%s: Wan2.2-A14B FFN-up linear, M=%d K=%d N=%d, W4A4 (MXFP4 act + MXFP4 weight), "
+                               "bias, bf16 out" % (wl_name, M, K, N),
+                   "M": M, "K": K, "N": N, "act_fmt": fmt, "parallelism": "replicas%d" % world,
+                   "l2": "inputs larger than L2 (x %.0f MB, y %.0f MB; L2 126 MB)" % (M * K * 2 / 1e6,
+                                                                                       M * N * 2 / 1e6)},
+        "roofline": {"bound": "tensor", "kernel": "mx_gemm_kernel<mxf4>", "achieved": round(g_tflops, 1),
+                     "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(g_tflops / fp4_peak, 4),
+                     "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal FP4/bf16 dense ratio)" % (
+                         peak_src, peaks["bf16_tflops"], FP4_OVER_BF16),
+                     "ms": round(g_ms, 4), "traffic": None, "path": gemm_path},
+        "parts": {
+            "quantize": {"ms": round(q_ms, 4), "GB/s": round(q_gbs, 1), "peak_GB/s": peaks["hbm_gbs"],
+                         "frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4),
+                         "bytes": quant_bytes(M, K, fmt)},
+            "gemm": {"ms": round(g_ms, 4), "TFLOP/s": round(g_tflops, 1),
+                     "frac_fp4": round(g_tflops / fp4_peak, 4)},
+        },
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+    }
+
+    if args.w4a8:
+        result["w4a8"] = bench_w4a8(args, ops, synth, dev, stream, world, rank, peaks)
+
+    # end to end: host buffers, H2D of x and D2H of y inside the timed region
+    if args.e2e:
+        xh = x.cpu().pin_memory()
+        yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        xd = torch.empty_like(x)
+
+        def e2e_step():
+            xd.copy_(xh, non_blocking=True)
+            ops.linear(xd, qw, fmt=fmt, workspace=ws, out=y)
+            yh.copy_(y, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier(world)
+        e_steps = max(3, args.steps // 4)
+        e_ms = max_over_ranks(time_loop(e2e_step, e_steps, stream), world)
+        result["e2e"] = {"value": round(world * flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                         "ms_per_step": round(e_ms, 3), "steps": e_steps,
+                         "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2}
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(M, N, K, fmt, c["seed"], budget_s=args.cpu_seconds)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result))
+
+
+def profile_one(args, ops, x, qw, ws, y, M, N, K, fmt, stream):
+    xc = ws[: ops.codes_bytes(M, K, fmt)]
+    off = (ops.codes_bytes(M, K, fmt) + 255) // 256 * 256
+    xs = ws[off: off + ops.sf_bytes(M, K)]
+    ops.quantize_act(x, fmt, codes=xc, sf=xs)
+    if args.only == "gemm":
+        fn = lambda: ops.gemm(xc, xs, fmt, M, K, qw, out=y)  # noqa: E731
+    else:
+        fn = lambda: ops.quantize_act(x, fmt, codes=xc, sf=xs)  # noqa: E731
+    for _ in range(args.warmup):
+        fn()
+    ms = time_loop(fn, args.steps, stream)
+    status = ops.poll_status()
+    print(json.dumps({"only": args.only, "workload": args.workload, "M": M, "N": N, "K": K, "fmt": fmt,
+                      "ms": round(ms, 4), "status": status, "path": ops.last_path()}))
+    if status != 0:
+        raise RuntimeError("device status %d" % status)
+
+
+def bench_w4a8(args, ops, synth, dev, stream, world, rank, peaks):
+    c = synth.WORKLOADS["ffn_down_720p_w4a8"]
+    M, K, N = c["M"], c["K"], c["N"]
+    x = synth.activation(M, K, c["act"], seed=c["seed"] + 1000 * rank, device=dev,
+                         outlier_frac=c["outlier_frac"], outlier_scale=c["outlier_scale"])
+    w = synth.weight(N, K, seed=c["seed"], device=dev)
+    qw = ops.quantize_weight(w, bias=synth.bias(N, seed=c["seed"], device=dev))
+    ws = torch.empty(ops.workspace_bytes(M, N, K, "e4m3", "qdq"), dtype=torch.uint8, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    flops = 2.0 * M * N * K
+    out = {"workload": "ffn_down_720p_w4a8: Wan2.2-A14B FFN-down, M=%d K=%d N=%d, E4M3 act (32-elem E8M0) x "
+                       "MXFP4 weight" % (M, K, N)}
+    iters = max(3, args.steps // 2)
+    for mode in ("native", "qdq"):
+        for _ in range(2):
+            ops.linear(x, qw, "e4m3", mode=mode, workspace=ws, out=y)
+        ms = max_over_ranks(time_loop(lambda: ops.linear(x, qw, "e4m3", mode=mode, workspace=ws, out=y), iters,
+                                      stream), world)
+        out[mode] = {"ms": round(ms, 4), "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 1),
+                     "path": ops.last_path()}
+    xc = ws[: ops.codes_bytes(M, K, "e4m3")]
+    off = (ops.codes_bytes(M, K, "e4m3") + 255) // 256 * 256
+    xs = ws[off: off + ops.sf_bytes(M, K)]
+    ops.quantize_act(x, "e4m3", codes=xc, sf=xs)
+    q_ms = max_over_ranks(time_loop(lambda: ops.quantize_act(x, "e4m3", codes=xc, sf=xs), iters, stream), world)
+    g_ms = max_over_ranks(time_loop(lambda: ops.gemm(xc, xs, "e4m3", M, K, qw, out=y), iters, stream), world)
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    out["quantize_e4m3"] = {"ms": round(q_ms, 4), "GB/s": round(quant_bytes(M, K, "e4m3") / (q_ms * 1e-3) / 1e9, 1),
+                            "frac_hbm": round(quant_bytes(M, K, "e4m3") / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    out["gemm_mxf8f6f4"] = {"ms": round(g_ms, 4), "TFLOP/s": round(flops / (g_ms * 1e-3) / 1e12, 1),
+                            "frac_fp8": round(flops / (g_ms * 1e-3) / 1e12 / fp8_peak, 4),
+                            "peak_fp8": round(fp8_peak, 1)}
+    if ops.poll_status() != 0:
+        raise RuntimeError("device status set during the W4A8 measurement")
+    return out
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, on the machine's host cores, on a bounded sample
+    of the same workload per step.  Under torchrun only rank 0 runs it."""
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    c = synth.WORKLOADS[args.workload]
+    M, K, N, fmt = c["M"], c["K"], c["N"], c["fmt"]
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(M, N, K, fmt, c["seed"], budget_s=per_step / 2)
+    vals, samples = [], None
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r = cpu_baseline(M, N, K, fmt, c["seed"], budget_s=per_step)
+        vals.append(r["value"])
+        samples = r
+    dt = time.perf_counter() - t0
+    v = statistics.mean(vals)
+    out = {"impl": "reference", "metric": "W4A4 MX linear TFLOP/s (fused dynamic MXFP4 activation quantize + "
+                                          "tcgen05 mxf4 GEMM)",
+           "value": v, "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(dt / max(1, args.steps) * 1e3, 1),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": "%s (CPU oracle on a bounded row sample per step)" % args.workload,
+                      "M": M, "K": K, "N": N, "act_fmt": fmt},
+           "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": samples["cores"], "kind": "oracle",
+                            "sample": samples["sample"]},
+           "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+           "gpu_launches": 0}
+    print(json.dumps(out))
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mxq", "reference"], default="mxq")
+    ap.add_argument("--workload", default="ffn_up_480p_w4a4")
+    ap.add_argument("--no-w4a8", dest="w4a8", action="store_false")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--M", type=int, default=0, help="override the workload's row count (profiling)")
+    ap.add_argument("--only", choices=["gemm", "quantize"], default=None,
+                    help="profiling mode: launch only this kernel, --steps times")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_mxq(args)
+
+
+if __name__ == "__main__":
+    main()

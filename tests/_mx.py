@@ -8,9 +8,16 @@ import oracle
 FMT = {"e2m1": oracle.E2M1, "e4m3": oracle.E4M3}
 
 # GEMM acceptance: relative Frobenius error <= 2e-3, and per output row
-# max |y - y_ref| <= 1e-2 * max |y_ref| (the row's infinity norm).
+# max |y - y_ref| <= 1e-2 * max |y_ref| (the row's infinity norm).  The Frobenius
+# bound is a statistical one: bf16 round-to-nearest-even alone has a relative error
+# of up to 2^-8 per element, so an output of a handful of elements can exceed 2e-3
+# even when every element is correctly rounded.  Outputs with fewer than
+# SMALL_OUTPUT elements are held instead to a per-element bound: the bf16 unit
+# roundoff of the reference value plus a small fp32-accumulation allowance.
 REL_FRO = 2e-3
 ROW_INF = 1e-2
+SMALL_OUTPUT = 4096
+BF16_U = 2.0 ** -8
 
 
 def bits(t: torch.Tensor) -> np.ndarray:
@@ -33,7 +40,13 @@ def assert_gemm_close(y_gpu: np.ndarray, y_ref: np.ndarray, what: str = ""):
     assert np.isfinite(y_gpu).all(), what + ": non-finite output"
     diff = y_gpu - y_ref
     fro = np.linalg.norm(diff) / max(np.linalg.norm(y_ref), 1e-300)
-    assert fro <= REL_FRO, "%s: relative Frobenius error %.3e > %.1e" % (what, fro, REL_FRO)
+    if y_ref.size >= SMALL_OUTPUT:
+        assert fro <= REL_FRO, "%s: relative Frobenius error %.3e > %.1e" % (what, fro, REL_FRO)
+    else:
+        lim = BF16_U * np.abs(y_ref) + 1e-6 * np.abs(y_ref).max()
+        bad = np.nonzero(np.abs(diff) > lim)
+        assert bad[0].size == 0, "%s: element %s off by %.3e (bound %.3e)" % (
+            what, tuple(int(b[0]) for b in bad), np.abs(diff)[bad][0], lim[bad][0])
     row_err = np.abs(diff).max(axis=1)
     row_inf = np.abs(y_ref).max(axis=1)
     bad = np.nonzero(row_err > ROW_INF * row_inf)[0]

@@ -1,0 +1,91 @@
+"""The DiT-block entry point: eight linears of one Wan-A14B-shaped block with a W4A4 /
+W4A8 precision mask, and a two-expert stack driven by a per-expert, per-block mask
+(the policy of the blog's sections "Mixed-Precision selection" and "Practical
+workflow", step 6).  Every linear's output is checked against the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests import _mx
+from tests.test_gemm_gpu import oracle_linear
+
+pytestmark = pytest.mark.gpu
+
+
+def _ops():
+    from fp8_mixed_precision_mxq_b200 import ops
+    return ops
+
+
+def block(seed, device="cuda"):
+    ops = _ops()
+    ws, bs = synth.block_weights(seed, device=device)
+    return [ops.quantize_weight(w, bias=b) for w, b in zip(ws, bs)], ws, bs
+
+
+@pytest.mark.parametrize("bits", [0x00, 0xFF, 0x80, 0x5A])
+def test_block_linears_against_oracle(bits):
+    ops = _ops()
+    M, ctx = 192, 64
+    qws, ws, bs = block(seed=3)
+    xs = synth.block_inputs(M, seed=3, device="cuda", ctx=ctx)
+    ys = ops.dit_block_linears(qws, xs, bits)
+    assert ops.poll_status() == 0
+    assert ("0x%02x" % bits) in ops.last_path()
+    rows = {M: synth.sample_rows(M, tile=32).numpy(), ctx: np.arange(ctx)}
+    for i, (name, N, K, src) in enumerate(synth.BLOCK_LINEARS):
+        fmt = "e4m3" if (bits >> i) & 1 else "e2m1"
+        r = rows[xs[i].shape[0]]
+        ref = oracle_linear(xs[i], ws[i], bs[i], fmt, rows=r)
+        got = _mx.bf16_to_f64(ys[i][torch.from_numpy(r).cuda()])
+        _mx.assert_gemm_close(got, ref, "block linear %s (%s)" % (name, fmt))
+
+
+def test_block_qdq_mode_matches_native_within_tolerance():
+    ops = _ops()
+    M, ctx = 128, 32
+    qws, ws, bs = block(seed=4)
+    xs = synth.block_inputs(M, seed=4, device="cuda", ctx=ctx)
+    bits = 0x80
+    y_nat = ops.dit_block_linears(qws, xs, bits, mode="native")
+    y_qdq = ops.dit_block_linears(qws, xs, bits, mode="qdq")
+    assert ops.poll_status() == 0
+    for i in (0, 6, 7):
+        fmt = "e4m3" if (bits >> i) & 1 else "e2m1"
+        r = np.arange(xs[i].shape[0])
+        ref = oracle_linear(xs[i], ws[i], bs[i], fmt, rows=r)
+        _mx.assert_gemm_close(_mx.bf16_to_f64(y_nat[i]), ref, "native %d" % i)
+        _mx.assert_gemm_close(_mx.bf16_to_f64(y_qdq[i]), ref, "qdq %d" % i)
+
+
+def test_two_expert_stack_follows_the_mask():
+    """Two experts x three blocks with a per-(expert, block) mask: each block runs its
+    linears with the precision its mask bit names; the W4A8 blocks differ from what the
+    same weights give under W4A4, and each output matches the oracle in its own format."""
+    ops = _ops()
+    M, ctx = 96, 32
+    mask = synth.expert_masks(n_experts=2, n_blocks=3, n_w4a8=1, seed=7)
+    xs = synth.block_inputs(M, seed=9, device="cuda", ctx=ctx)
+    for e in range(2):
+        for blk in range(3):
+            qws, ws, bs = block(seed=100 + 10 * e + blk)
+            bits = 0xFF if mask[e, blk] else 0x00
+            ys = ops.dit_block_linears(qws, xs, bits)
+            fmt = "e4m3" if bits else "e2m1"
+            for i in (1, 7):
+                r = np.arange(xs[i].shape[0])
+                ref = oracle_linear(xs[i], ws[i], bs[i], fmt, rows=r)
+                _mx.assert_gemm_close(_mx.bf16_to_f64(ys[i]), ref, "expert %d block %d linear %d" % (e, blk, i))
+    assert ops.poll_status() == 0
+
+
+def test_block_rejects_wrong_workspace():
+    ops = _ops()
+    qws, _, _ = block(seed=5)
+    xs = synth.block_inputs(64, seed=5, device="cuda", ctx=16)
+    need = ops.block_workspace_bytes(qws, [x.shape[0] for x in xs], 0xFF)
+    small = torch.empty(need // 2, dtype=torch.uint8, device="cuda")
+    with pytest.raises(Exception) as ei:
+        ops.dit_block_linears(qws, xs, 0xFF, workspace=small)
+    assert "WORKSPACE" in str(ei.value)

@@ -74,11 +74,12 @@ def test_gemm_no_bias_and_guard_band(fmt):
     x, w, _ = make_case(M, N, K, fmt, seed=5, bias=False)
     qw = ops.quantize_weight(w)
     xc, xs = ops.quantize_act(x, fmt)
-    buf = torch.full(((M + 2) * N,), 1234.0, dtype=torch.bfloat16, device="cuda")
+    canary = 1232.0  # exact in bf16
+    buf = torch.full(((M + 2) * N,), canary, dtype=torch.bfloat16, device="cuda")
     y = buf[: M * N].view(M, N)
     ops.gemm(xc, xs, fmt, M, K, qw, out=y)
     torch.cuda.synchronize()
-    assert (buf[M * N:].float() == 1234.0).all(), "GEMM wrote past the end of y"
+    assert (buf[M * N:].float() == canary).all(), "GEMM wrote past the end of y"
     _mx.assert_gemm_close(_mx.bf16_to_f64(y), oracle_linear(x, w, None, fmt), "no-bias " + fmt)
 
 
