@@ -30,6 +30,7 @@ int ok()
 }
 
 constexpr int64_t kMaxElems = int64_t(1) << 34;  // rows*K; keeps 32-bit group / scale indices exact
+constexpr int64_t kMaxK = int64_t(1) << 16;       // K/32 < 2^11 keeps the row division of the quantizer exact
 constexpr int64_t kWsAlign = 256;
 constexpr int64_t kLtWorkspace = int64_t(32) << 20;
 
@@ -55,6 +56,8 @@ int check_rows_k(int64_t rows, int64_t K, const char* what)
     if (rows <= 0 || K <= 0) return fail(MXQ_ERR_INVALID_ARG, "%s: sizes must be positive (rows=%lld K=%lld)", what,
                                          (long long)rows, (long long)K);
     if (K % 32 != 0) return fail(MXQ_ERR_SHAPE, "%s: K=%lld is not a multiple of 32", what, (long long)K);
+    if (K > kMaxK) return fail(MXQ_ERR_SHAPE, "%s: K=%lld is above the supported maximum %lld", what, (long long)K,
+                               (long long)kMaxK);
     if (rows > (int64_t(1) << 31) - 1 || rows * K > kMaxElems)
         return fail(MXQ_ERR_SHAPE, "%s: tensor too large (rows=%lld K=%lld)", what, (long long)rows, (long long)K);
     return MXQ_OK;

@@ -30,10 +30,13 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p)
     return v;
 }
 
-// |x| bit patterns of the two bf16 halves of w, packed max.
-__device__ __forceinline__ uint32_t abs_max2(uint32_t a, uint32_t b)
+// Packed max of |a| and |b| over two bf16 lanes (sign of the result is the xor of the
+// signs, which the caller masks off); a NaN in either input yields NaN.
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b)
 {
-    return __vmaxu2(a & 0x7FFF7FFFu, b & 0x7FFF7FFFu);
+    uint32_t d;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
 __device__ __forceinline__ float lo_f(uint32_t w) { return __uint_as_float(w << 16); }
@@ -67,8 +70,9 @@ __device__ __forceinline__ uint32_t sf_offset(uint32_t r, uint32_t kb, uint32_t 
 
 template <int FMT>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restrict__ x, uint32_t n_groups,
-                                                            uint32_t KB, uint32_t atoms_k, uint32_t rows,
-                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ sf)
+                                                            uint32_t KB, uint64_t kb_magic, uint32_t atoms_k,
+                                                            uint32_t rows, uint8_t* __restrict__ codes,
+                                                            uint8_t* __restrict__ sf)
 {
     constexpr uint32_t kEmax = FMT == kFmtE4M3 ? 8u : 2u;
     const uint32_t lane = threadIdx.x & 31u;
@@ -86,8 +90,9 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             // block absmax over the quad of lanes holding the 32 elements
-            uint32_t m2 = __vmaxu2(abs_max2(v[u].x, v[u].y), abs_max2(v[u].z, v[u].w));
-            uint32_t amax = max(m2 & 0xFFFFu, m2 >> 16);
+            uint32_t m2 = absmax_bf16x2(absmax_bf16x2(v[u].x, v[u].y), absmax_bf16x2(v[u].z, v[u].w));
+            m2 = absmax_bf16x2(m2, __byte_perm(m2, 0, 0x1032));
+            uint32_t amax = m2 & 0x7FFFu;
             amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
             amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
             if (g[u] >= n_groups) continue;
@@ -121,7 +126,8 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
             }
             if ((lane & 3u) == 0) {
                 const uint32_t blk = g[u] >> 2;
-                const uint32_t r = blk / KB, kb = blk - r * KB;
+                const uint32_t r = static_cast<uint32_t>((static_cast<uint64_t>(blk) * kb_magic) >> 40);
+                const uint32_t kb = blk - r * KB;
                 sf[sf_offset(r, kb, atoms_k)] = static_cast<uint8_t>(sc);
             }
         }
@@ -232,14 +238,16 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, int fmt, voi
     const uint32_t atoms_k = static_cast<uint32_t>(sf_atoms_k(K));
     const int64_t want = ceil_div(n_groups, kThreads * kUnroll);
     const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * 8)));
+    // row = floor(block / KB) as a multiply-shift: exact for block < 2^29 and KB < 2^11
+    const uint64_t kb_magic = ((uint64_t(1) << 40) + KB - 1) / KB;
     if (fmt == kFmtE4M3)
         quantize_kernel<kFmtE4M3><<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(x), n_groups, KB,
-                                                                 atoms_k, static_cast<uint32_t>(rows),
+                                                                 kb_magic, atoms_k, static_cast<uint32_t>(rows),
                                                                  static_cast<uint8_t*>(codes),
                                                                  static_cast<uint8_t*>(sf));
     else
         quantize_kernel<kFmtE2M1><<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(x), n_groups, KB,
-                                                                 atoms_k, static_cast<uint32_t>(rows),
+                                                                 kb_magic, atoms_k, static_cast<uint32_t>(rows),
                                                                  static_cast<uint8_t*>(codes),
                                                                  static_cast<uint8_t*>(sf));
     return cudaGetLastError();
