@@ -10,15 +10,21 @@
 // kind::mxf8f6f4 with A in E4M3 and the E2M1 weight expanded by TMA into the
 // byte-padded shared-memory form (K = 32 per instruction).
 //
-// Structure (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0      TMA producer: A / W tiles (128-byte swizzle) and the scale-factor
-//               atoms (contiguous 512-byte chunks, plain bulk copies) into a
-//               4-stage shared-memory ring;
-//   warp 1      MMA issuer: copies each stage's scale atoms into TMEM
+// Structure (one CTA per SM, persistent over output tiles).  Two variants: a lone
+// CTA owning 128 x 256 tiles, and a CTA pair (a 2-CTA cluster on one TPC, MMAs with
+// cta_group::2) owning 256 x 256 tiles, where each CTA loads its own 128 activation
+// rows and half of the 256 weight rows, so each SM moves 2/3 of the bytes per FLOP.
+//   warp 0      TMA producer (each CTA): A / W tiles (128-byte swizzle) and the
+//               scale-factor atoms (512-byte chunks, as 2-D TMA boxes) into the
+//               shared-memory ring; a pair's loads all complete on the leader's barrier;
+//   warp 1      MMA issuer (leader CTA): copies each stage's scale atoms into TMEM
 //               (tcgen05.cp 32x128b.warpx4) and issues the block-scaled MMAs into
-//               a TMEM accumulator; allocates / frees TMEM;
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, + bias, -> bf16, staged
-//               in swizzled shared memory and written with TMA stores.
+//               the TMEM accumulators; commits release the stage in both CTAs;
+//               in every CTA this warp allocates and frees TMEM;
+//   warps 2..5  epilogue (each CTA): tcgen05.ld 32 columns at a time, + bias, -> bf16,
+//               staged in swizzled shared memory and written with TMA stores.
+// L2 policies: the weight is loaded evict-last (it is reused by every m-block and fits
+// in L2), the output is stored evict-first.
 // TMEM (512 columns): accumulator slot 0 = columns [0, 256), slot 1 = [224, 480),
 // scale factors = [480, 504).  The two slots overlap in [224, 256); the epilogue
 // drains that 32-column chunk first and signals it, so the next tile's MMAs can
@@ -42,48 +48,51 @@ __device__ uint32_t g_device_status;
 
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int kStages = 4;
+constexpr int BN = 256;                   // output columns per tile (both variants)
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr uint32_t kStageA = BM * 128;               // 128 rows x 128 bytes
-constexpr uint32_t kStageB = BN * 128;               // 256 rows x 128 bytes
-constexpr uint32_t kStageSFA = 2 * 512;              // up to two k-atoms
-constexpr uint32_t kStageSFB = 2 * 2 * 512;          // two 128-row halves x two k-atoms
-constexpr uint32_t kEpiBuf = 32 * 64;                // 32 rows x 32 bf16
-constexpr uint32_t kOffA = 0;
-constexpr uint32_t kOffB = kOffA + kStages * kStageA;
-constexpr uint32_t kOffSFA = kOffB + kStages * kStageB;
-constexpr uint32_t kOffSFB = kOffSFA + kStages * kStageSFA;
-constexpr uint32_t kOffEpi = kOffSFB + kStages * kStageSFB;
-constexpr uint32_t kOffBar = kOffEpi + kEpiWarps * 2 * kEpiBuf;
-constexpr uint32_t kNumBars = 2 * kStages + 2 + 2 + 1 + 1;
-constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;  // + alignment slack
+constexpr uint32_t kEpiBuf = 32 * 64;     // 32 rows x 32 bf16
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol1 = 224;
 constexpr uint32_t kSfaCol = 480;
 constexpr uint32_t kSfbCol = 488;
-constexpr int kGroupM = 16;  // m-blocks per rasterization group
 constexpr uint64_t kWaitNs = 1000000000ull;
 
-static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kOffEpi % 1024 == 0 && kOffB % 1024 == 0, "swizzled buffers need 1024-byte alignment");
+// Shared-memory plan of one CTA.  kPair = 1: the CTA owns a 128 x 256 tile and loads
+// all 256 weight rows; kPair = 2: a CTA pair owns a 256 x 256 tile, each CTA loads its
+// own 128 activation rows and 128 of the 256 weight rows (the pair MMA reads both).
+template <int kPair>
+struct Cfg {
+    static constexpr int kStages = kPair == 2 ? 6 : 4;
+    static constexpr int BM = 128 * kPair;
+    static constexpr int kRowsB = BN / kPair;
+    static constexpr uint32_t kStageA = 128 * 128;
+    static constexpr uint32_t kStageB = kRowsB * 128;
+    static constexpr uint32_t kStageSFA = 2 * 512;       // up to two k-atoms
+    static constexpr uint32_t kStageSFB = 2 * 2 * 512;   // both 128-row halves of the tile
+    static constexpr uint32_t kOffA = 0;
+    static constexpr uint32_t kOffB = kOffA + kStages * kStageA;
+    static constexpr uint32_t kOffSFA = kOffB + kStages * kStageB;
+    static constexpr uint32_t kOffSFB = kOffSFA + kStages * kStageSFA;
+    static constexpr uint32_t kOffEpi = kOffSFB + kStages * kStageSFB;
+    static constexpr uint32_t kOffBar = kOffEpi + kEpiWarps * 2 * kEpiBuf;
+    static constexpr uint32_t kNumBars = 2 * kStages + 6;
+    static constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16;
+    static constexpr int kGroupM = kPair == 2 ? 8 : 16;  // tile rows per rasterization group
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kOffB % 1024 == 0 && kOffSFA % 1024 == 0 && kOffEpi % 1024 == 0, "alignment");
+};
 
 struct Params {
-    const uint8_t* a_sf;
-    const uint8_t* w_sf;
     const __nv_bfloat16* bias;
     int M, N, K;
-    int m_blocks, n_blocks, num_tiles, k_stages, atoms_k, sf_rows_w;
+    int m_blocks, n_blocks, num_tiles, k_stages;
     uint32_t debug;
 };
 
-__device__ __forceinline__ void record_timeout()
-{
-    atomicCAS(&g_device_status, 0u, static_cast<uint32_t>(MXQ_ERR_TIMEOUT));
-}
+__device__ __forceinline__ void record_status(uint32_t code) { atomicCAS(&g_device_status, 0u, code); }
 
+template <int kGroupM>
 __device__ __forceinline__ void tile_coords(int t, int m_blocks, int n_blocks, int& mb, int& nb)
 {
     const int per_group = kGroupM * n_blocks;
@@ -95,180 +104,195 @@ __device__ __forceinline__ void tile_coords(int t, int m_blocks, int n_blocks, i
     mb = first_m + (local - nb * gsize);
 }
 
-template <bool kW4A8>
+template <bool kW4A8, int kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                   const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                    const __grid_constant__ CUtensorMap map_y, const Params p)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    using C = Cfg<kPair>;
+    constexpr int S = C::kStages;
+    constexpr int AK = kW4A8 ? 1 : 2;  // scale atoms (128 K-elements each) per stage
+
+    extern __shared__ __align__(1024) uint8_t smem[];
+    // the swizzled tiles need a 1024-byte aligned base; both CTAs of a pair see the same
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) record_status(MXQ_ERR_UNSUPPORTED);
+        return;
+    }
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* full = bars;
-    uint64_t* empty = bars + kStages;
-    uint64_t* tmem_full = bars + 2 * kStages;
-    uint64_t* tmem_empty = bars + 2 * kStages + 2;
-    uint64_t* overlap_free = bars + 2 * kStages + 4;
-    uint64_t* mma_done = bars + 2 * kStages + 5;
-    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + kNumBars);
+    uint64_t* empty = bars + S;
+    uint64_t* tmem_full = bars + 2 * S;
+    uint64_t* tmem_empty = bars + 2 * S + 2;
+    uint64_t* overlap_free = bars + 2 * S + 4;
+    uint64_t* mma_done = bars + 2 * S + 5;
+    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = kPair == 2 ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int pair_id = blockIdx.x / kPair;
+    const int n_pairs = gridDim.x / kPair;
 
-    // k-atoms (128 K-elements of scale factors) per pipeline stage
-    constexpr int AK = kW4A8 ? 1 : 2;
-
+    if (kPair == 2) cluster_sync();
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&map_a);
         prefetch_tmap(&map_b);
+        prefetch_tmap(&map_sfa);
+        prefetch_tmap(&map_sfb);
         prefetch_tmap(&map_y);
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&tmem_full[s], 1);
-            mbar_init(&tmem_empty[s], kEpiWarps);
+            mbar_init(&tmem_empty[s], kEpiWarps * kPair);
         }
-        mbar_init(overlap_free, kEpiWarps);
+        mbar_init(overlap_free, kEpiWarps * kPair);
         mbar_init(mma_done, 1);
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(tmem_base_smem, kTmemCols);
-        tmem_relinquish();
+        tmem_alloc<kPair>(tmem_base_smem, kTmemCols);
+        tmem_relinquish<kPair>();
     }
     tc_fence_before();
-    __syncthreads();
+    if (kPair == 2) cluster_sync(); else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_smem;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------------ producer (each CTA)
         if (lane == 0) {
-            uint32_t it = 0;          // stages issued (including a skipped one)
-            int64_t skipped = -1;     // debug: index of the stage whose load was skipped
+            const uint64_t pol_w = policy_evict_last();    // weights: reused by every m-block
+            const uint64_t pol_a = policy_evict_normal();  // activations: reused within a group
+            constexpr uint32_t kTx = kPair * (C::kStageA + (kW4A8 ? C::kStageB / 2 : C::kStageB) +
+                                              AK * 512u * 3u);
+            uint32_t it = 0;
+            int64_t skipped = -1;
             bool ok = true;
-            const int n_row_tiles_w = p.sf_rows_w;
-            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+            for (int t = pair_id; t < p.num_tiles && ok; t += n_pairs) {
                 int mb, nb;
-                tile_coords(t, p.m_blocks, p.n_blocks, mb, nb);
+                tile_coords<C::kGroupM>(t, p.m_blocks, p.n_blocks, mb, nb);
                 for (int ks = 0; ks < p.k_stages; ++ks, ++it) {
-                    const uint32_t s = it % kStages;
-                    if (!mbar_wait(&empty[s], ((it / kStages) & 1) ^ 1, kWaitNs)) {
-                        record_timeout();
+                    const uint32_t s = it % S;
+                    if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, kWaitNs)) {
+                        record_status(MXQ_ERR_TIMEOUT);
                         ok = false;
                         break;
                     }
-                    if ((p.debug & 1u) && it == 0 && blockIdx.x == 0) {
-                        skipped = 0;  // deliberately leave stage 0 unfilled
+                    if ((p.debug & 1u) && it == 0 && pair_id == 0 && leader) {
+                        skipped = 0;  // deliberately leave stage 0 unfilled: the MMA wait runs out
                         continue;
                     }
-                    const int ka0 = ks * AK;
-                    const int na = min(AK, p.atoms_k - ka0);
-                    const int rt0 = nb * 2;
-                    const int nh = min(2, n_row_tiles_w - rt0);
-                    const uint32_t tx = kStageA + (kW4A8 ? kStageB / 2 : kStageB) + na * 512u * (1 + nh);
-                    mbar_arrive_expect_tx(&full[s], tx);
-                    tma_load_2d(smem + kOffA + s * kStageA, &map_a, ks * 128, mb * BM, &full[s]);
-                    tma_load_2d(smem + kOffB + s * kStageB, &map_b, ks * 128, nb * BN, &full[s]);
-                    bulk_load(smem + kOffSFA + s * kStageSFA,
-                              p.a_sf + (static_cast<int64_t>(mb) * p.atoms_k + ka0) * 512, na * 512u, &full[s]);
-                    for (int h = 0; h < nh; ++h)
-                        bulk_load(smem + kOffSFB + s * kStageSFB + h * AK * 512,
-                                  p.w_sf + (static_cast<int64_t>(rt0 + h) * p.atoms_k + ka0) * 512, na * 512u,
-                                  &full[s]);
+                    if (leader) mbar_arrive_expect_tx(&full[s], kTx);
+                    const uint32_t bar = kPair == 2 ? mapa_shared(smem_u32(&full[s]), 0) : smem_u32(&full[s]);
+                    tma_load_2d<kPair>(smem + C::kOffA + s * C::kStageA, &map_a, ks * 128,
+                                       mb * C::BM + static_cast<int>(rank) * 128, bar, pol_a);
+                    tma_load_2d<kPair>(smem + C::kOffB + s * C::kStageB, &map_b, ks * 128,
+                                       nb * BN + static_cast<int>(rank) * C::kRowsB, bar, pol_w);
+                    tma_load_2d<kPair>(smem + C::kOffSFA + s * C::kStageSFA, &map_sfa, ks * AK * 128,
+                                       mb * kPair + static_cast<int>(rank), bar, pol_a);
+                    tma_load_2d<kPair>(smem + C::kOffSFB + s * C::kStageSFB, &map_sfb, ks * AK * 128, nb * 2,
+                                       bar, pol_w);
                 }
             }
-            // drain: every load still in flight lands before the CTA may exit
-            const uint32_t first = it > kStages ? it - kStages : 0;
-            for (uint32_t i = first; i < it; ++i) {
+            // drain: the last stages' loads have landed once their consumer released them
+            const uint32_t first = it > S ? it - S : 0;
+            for (uint32_t i = first; i < it && ok; ++i) {
                 if (static_cast<int64_t>(i) == skipped) continue;
-                if (!mbar_wait(&full[i % kStages], (i / kStages) & 1, kWaitNs)) record_timeout();
+                if (!mbar_wait(&empty[i % S], (i / S) & 1, kWaitNs)) {
+                    record_status(MXQ_ERR_TIMEOUT);
+                    break;
+                }
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t fa = kW4A8 ? 0u : 1u;   // A element type: E4M3 (mxf8f6f4) / E2M1 (mxf4)
-            const uint32_t fb = kW4A8 ? 5u : 1u;   // B element type: E2M1 in both kinds
+        // ------------------------------------------------------------ MMA issuer (leader CTA)
+        if (leader && lane == 0) {
+            const uint32_t fa = kW4A8 ? 0u : 1u;  // A element type: E4M3 (mxf8f6f4) / E2M1 (mxf4)
+            const uint32_t fb = kW4A8 ? 5u : 1u;  // B element type: E2M1 in both kinds
             uint32_t it = 0;
             int tcount = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++tcount) {
+            for (int t = pair_id; t < p.num_tiles && ok; t += n_pairs, ++tcount) {
                 const int slot = tcount & 1;
                 const uint32_t acc = tmem_base + (slot ? kAccCol1 : 0u);
                 if (!mbar_wait(&tmem_empty[slot], ((tcount >> 1) & 1) ^ 1, kWaitNs) ||
                     (tcount > 0 && !mbar_wait(overlap_free, (tcount - 1) & 1, kWaitNs))) {
-                    record_timeout();
+                    record_status(MXQ_ERR_TIMEOUT);
                     break;
                 }
                 tc_fence_after();
-                int mb, nb;
-                tile_coords(t, p.m_blocks, p.n_blocks, mb, nb);
-                const int nh = min(2, p.sf_rows_w - nb * 2);
                 for (int ks = 0; ks < p.k_stages; ++ks, ++it) {
-                    const uint32_t s = it % kStages;
-                    if (!mbar_wait(&full[s], (it / kStages) & 1, kWaitNs)) {
-                        record_timeout();
+                    const uint32_t s = it % S;
+                    if (!mbar_wait(&full[s], (it / S) & 1, kWaitNs)) {
+                        record_status(MXQ_ERR_TIMEOUT);
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int na = min(AK, p.atoms_k - ks * AK);
-                    const uint32_t sfa_s = smem_u32(smem + kOffSFA + s * kStageSFA);
-                    const uint32_t sfb_s = smem_u32(smem + kOffSFB + s * kStageSFB);
-                    for (int a = 0; a < na; ++a) {
-                        tc_copy_sf_atom(tmem_base + kSfaCol + 4 * a, sdesc_sf_atom(sfa_s + a * 512));
-                        for (int h = 0; h < nh; ++h)
-                            tc_copy_sf_atom(tmem_base + kSfbCol + 8 * a + 4 * h,
-                                            sdesc_sf_atom(sfb_s + (h * AK + a) * 512));
+                    const uint32_t sfa_s = smem_u32(smem + C::kOffSFA + s * C::kStageSFA);
+                    const uint32_t sfb_s = smem_u32(smem + C::kOffSFB + s * C::kStageSFB);
+#pragma unroll
+                    for (int a = 0; a < AK; ++a) {
+                        tc_copy_sf_atom<kPair>(tmem_base + kSfaCol + 4 * a, sdesc_sf_atom(sfa_s + a * 512));
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tc_copy_sf_atom<kPair>(tmem_base + kSfbCol + 8 * a + 4 * h,
+                                                   sdesc_sf_atom(sfb_s + (h * AK + a) * 512));
                     }
-                    const uint32_t a_s = smem_u32(smem + kOffA + s * kStageA);
-                    const uint32_t b_s = smem_u32(smem + kOffB + s * kStageB);
+                    const uint32_t a_s = smem_u32(smem + C::kOffA + s * C::kStageA);
+                    const uint32_t b_s = smem_u32(smem + C::kOffB + s * C::kStageB);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int k_elem = kW4A8 ? ks * 128 + j * 32 : ks * 256 + j * 64;
                         if (k_elem >= p.K) break;
                         const int atom = kW4A8 ? 0 : (j >> 1);
                         const uint32_t sf_id = kW4A8 ? static_cast<uint32_t>(j) : static_cast<uint32_t>((j & 1) * 2);
-                        const uint32_t idesc = idesc_block_scaled(fa, fb, BM, BN, sf_id, sf_id);
+                        const uint32_t idesc = idesc_block_scaled(fa, fb, C::BM, BN, sf_id, sf_id);
                         const uint64_t ad = sdesc_k_sw128(a_s + j * 32);
                         const uint64_t bd = sdesc_k_sw128(b_s + j * 32);
                         const uint32_t accumulate = (ks > 0 || j > 0) ? 1u : 0u;
                         if (kW4A8)
-                            mma_mxf8f6f4(acc, ad, bd, idesc, tmem_base + kSfaCol + 4 * atom,
-                                         tmem_base + kSfbCol + 8 * atom, accumulate);
+                            mma_mxf8f6f4<kPair>(acc, ad, bd, idesc, tmem_base + kSfaCol + 4 * atom,
+                                                tmem_base + kSfbCol + 8 * atom, accumulate);
                         else
-                            mma_mxf4(acc, ad, bd, idesc, tmem_base + kSfaCol + 4 * atom,
-                                     tmem_base + kSfbCol + 8 * atom, accumulate);
+                            mma_mxf4<kPair>(acc, ad, bd, idesc, tmem_base + kSfaCol + 4 * atom,
+                                            tmem_base + kSfbCol + 8 * atom, accumulate);
                     }
-                    tc_commit(&empty[s]);  // stage s is free once these MMAs completed
+                    tc_commit<kPair>(&empty[s]);  // stage s free (in both CTAs) once these MMAs completed
                 }
                 if (!ok) break;
-                tc_commit(&tmem_full[slot]);  // accumulator ready for the epilogue
+                tc_commit<kPair>(&tmem_full[slot]);  // accumulators ready for both CTAs' epilogues
             }
             // every MMA issued by this thread completes before TMEM is released
-            tc_commit(mma_done);
-            if (!mbar_wait(mma_done, 0, kWaitNs)) record_timeout();
+            tc_commit_local<kPair>(mma_done);
+            if (!mbar_wait(mma_done, 0, kWaitNs)) record_status(MXQ_ERR_TIMEOUT);
         }
     } else {
-        // ------------------------------------------------------------ epilogue
+        // ------------------------------------------------------------ epilogue (each CTA)
+        const uint64_t pol_y = policy_evict_first();
         const int ew = warp - 2;
         const int q = warp & 3;  // TMEM lane quarter this warp may access
-        uint8_t* ebuf0 = smem + kOffEpi + ew * 2 * kEpiBuf;
+        uint8_t* ebuf0 = smem + C::kOffEpi + ew * 2 * kEpiBuf;
+        const uint32_t bar_overlap = kPair == 2 ? mapa_shared(smem_u32(overlap_free), 0) : smem_u32(overlap_free);
         int eb = 0;
         int tcount = 0;
-        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++tcount) {
+        for (int t = pair_id; t < p.num_tiles; t += n_pairs, ++tcount) {
             const int slot = tcount & 1;
             if (!mbar_wait(&tmem_full[slot], (tcount >> 1) & 1, kWaitNs)) {
-                record_timeout();
+                record_status(MXQ_ERR_TIMEOUT);
                 break;
             }
             tc_fence_after();
             int mb, nb;
-            tile_coords(t, p.m_blocks, p.n_blocks, mb, nb);
+            tile_coords<C::kGroupM>(t, p.m_blocks, p.n_blocks, mb, nb);
             const uint32_t col0 = slot ? kAccCol1 : 0u;
-            const int row0 = mb * BM + q * 32;
+            const int row0 = mb * C::BM + static_cast<int>(rank) * 128 + q * 32;
             for (int ci = 0; ci < BN / 32; ++ci) {
                 // the 32 columns shared by both slots go first
                 const int c = slot ? ci : (ci == 0 ? BN / 32 - 1 : ci - 1);
@@ -278,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ci == 0) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(overlap_free);
+                    if (lane == 0) mbar_arrive_cluster(bar_overlap);
                 }
                 const int n = nb * BN + c * 32;
                 if (n >= p.N) continue;
@@ -318,23 +342,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(&map_y, buf, n, row0);
+                    tma_store_2d(&map_y, buf, n, row0, pol_y);
                     bulk_commit();
                 }
                 eb ^= 1;
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tmem_empty[slot]);
+            if (lane == 0)
+                mbar_arrive_cluster(kPair == 2 ? mapa_shared(smem_u32(&tmem_empty[slot]), 0)
+                                               : smem_u32(&tmem_empty[slot]));
         }
         if (lane == 0) bulk_wait<0>();
         __syncwarp();
     }
 
     tc_fence_before();
-    __syncthreads();
+    if (kPair == 2) cluster_sync(); else __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+    if (warp == 1) tmem_dealloc<kPair>(tmem_base, kTmemCols);
 }
 
 // ---------------------------------------------------------------------------- host
@@ -383,19 +409,57 @@ int read_and_clear_device_status(cudaStream_t stream, uint32_t* out)
     return MXQ_OK;
 }
 
+namespace {
+
+template <bool kW4A8, int kPair>
+cudaError_t launch_variant(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa,
+                           const CUtensorMap& msb, const CUtensorMap& my, const Params& p, int grid,
+                           cudaStream_t stream)
+{
+    using C = Cfg<kPair>;
+    auto kern = mx_gemm_kernel<kW4A8, kPair>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kPair;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = kPair == 2 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, my, p);
+}
+
+}  // namespace
+
 int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* path, size_t path_len)
 {
     const bool w4a8 = g.a_fmt == kFmtE4M3;
-    CUtensorMap ma, mb, my;
+    // CTA pairs for anything taller than one 128-row tile; a lone CTA otherwise.
+    const int pair = g.M > 128 ? 2 : 1;
+    const int rows_b = BN / pair;
+    const int64_t atoms_k = sf_atoms_k(g.K);
+    const int ak = w4a8 ? 1 : 2;
+    CUtensorMap ma, mb, msa, msb, my;
     const uint64_t a_row = w4a8 ? g.K : g.K / 2;
-    bool ok = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a_codes, a_row, g.M, a_row, 128, BM,
+    bool ok = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a_codes, a_row, g.M, a_row, 128, 128,
                           CU_TENSOR_MAP_SWIZZLE_128B);
     if (w4a8)
-        ok = ok && make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, g.w_codes, g.K, g.N, g.K / 2, 128, BN,
-                               CU_TENSOR_MAP_SWIZZLE_128B);
+        ok = ok && make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, g.w_codes, g.K, g.N, g.K / 2, 128,
+                               rows_b, CU_TENSOR_MAP_SWIZZLE_128B);
     else
-        ok = ok && make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.w_codes, g.K / 2, g.N, g.K / 2, 128, BN,
+        ok = ok && make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.w_codes, g.K / 2, g.N, g.K / 2, 128, rows_b,
                                CU_TENSOR_MAP_SWIZZLE_128B);
+    // scale atoms as 32-bit words: one 2-D row of atoms_k*128 words per 128-row tile
+    ok = ok && make_map_2d(&msa, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.a_sf, atoms_k * 128, ceil_div(g.M, 128),
+                           atoms_k * 512, ak * 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+    ok = ok && make_map_2d(&msb, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.w_sf, atoms_k * 128, ceil_div(g.N, 128),
+                           atoms_k * 512, ak * 128, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
     ok = ok && make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, g.N, g.M, g.N * 2, 32, 32,
                            CU_TENSOR_MAP_SWIZZLE_64B);
     if (!ok) {
@@ -403,40 +467,35 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
         return MXQ_ERR_CUDA;
     }
     Params p;
-    p.a_sf = static_cast<const uint8_t*>(g.a_sf);
-    p.w_sf = static_cast<const uint8_t*>(g.w_sf);
     p.bias = static_cast<const __nv_bfloat16*>(g.bias);
     p.M = static_cast<int>(g.M);
     p.N = static_cast<int>(g.N);
     p.K = static_cast<int>(g.K);
-    p.m_blocks = static_cast<int>(ceil_div(g.M, BM));
+    p.m_blocks = static_cast<int>(ceil_div(g.M, 128 * pair));
     p.n_blocks = static_cast<int>(ceil_div(g.N, BN));
     p.num_tiles = p.m_blocks * p.n_blocks;
     p.k_stages = static_cast<int>(ceil_div(g.K, w4a8 ? 128 : 256));
-    p.atoms_k = static_cast<int>(sf_atoms_k(g.K));
-    p.sf_rows_w = static_cast<int>(ceil_div(g.N, 128));
     p.debug = g_debug_flags;
 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int grid = std::min(p.num_tiles, sms);
+    const int grid = std::min(p.num_tiles, sms / pair) * pair;
     cudaError_t e;
-    if (w4a8) {
-        e = cudaFuncSetAttribute(mx_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e == cudaSuccess) mx_gemm_kernel<true><<<grid, kThreads, kSmemBytes, stream>>>(ma, mb, my, p);
-    } else {
-        e = cudaFuncSetAttribute(mx_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e == cudaSuccess) mx_gemm_kernel<false><<<grid, kThreads, kSmemBytes, stream>>>(ma, mb, my, p);
-    }
+    if (w4a8)
+        e = pair == 2 ? launch_variant<true, 2>(ma, mb, msa, msb, my, p, grid, stream)
+                      : launch_variant<true, 1>(ma, mb, msa, msb, my, p, grid, stream);
+    else
+        e = pair == 2 ? launch_variant<false, 2>(ma, mb, msa, msb, my, p, grid, stream)
+                      : launch_variant<false, 1>(ma, mb, msa, msb, my, p, grid, stream);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) {
         *msg = cudaGetErrorString(e);
         return MXQ_ERR_CUDA;
     }
     if (path)
-        snprintf(path, path_len, "native %s 1cta %dx%d grid %d tiles %d", w4a8 ? "mxf8f6f4" : "mxf4", BM, BN, grid,
-                 p.num_tiles);
+        snprintf(path, path_len, "native %s %s %dx%d grid %d tiles %d", w4a8 ? "mxf8f6f4" : "mxf4",
+                 pair == 2 ? "2cta" : "1cta", 128 * pair, BN, grid, p.num_tiles);
     return MXQ_OK;
 }
 

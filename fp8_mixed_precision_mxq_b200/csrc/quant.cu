@@ -100,26 +100,21 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
             const uint32_t sc = eb == 255u ? 255u : (eb > kEmax ? eb - kEmax : 0u);
             const float inv = __uint_as_float((254u - min(sc, 253u)) << 23);  // 2^(127 - sc)
             const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            // cvt rounds to nearest even, saturates, and keeps the sign of a value that
+            // rounds to zero (-0 = 0x8 / 0x80), as the format reading requires
             if (FMT == kFmtE2M1) {
-                uint32_t out = 0, sgn = 0;
+                uint32_t out = 0;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    out |= cvt_e2m1x2(lo_f(w[i]) * inv, hi_f(w[i]) * inv) << (8 * i);
-                    sgn |= (((w[i] >> 12) & 0x8u) | ((w[i] >> 24) & 0x80u)) << (8 * i);
-                }
-                out |= sgn;  // a negative value that rounds to zero keeps its sign
+                for (int i = 0; i < 4; ++i) out |= cvt_e2m1x2(lo_f(w[i]) * inv, hi_f(w[i]) * inv) << (8 * i);
                 if (sc == 255u) out = 0;
                 reinterpret_cast<uint32_t*>(codes)[g[u]] = out;
             } else {
-                uint32_t out[2], sgn[2];
+                uint32_t out[2];
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     const uint32_t a = w[2 * i], b = w[2 * i + 1];
                     out[i] = cvt_e4m3x2(lo_f(a) * inv, hi_f(a) * inv) |
                              (cvt_e4m3x2(lo_f(b) * inv, hi_f(b) * inv) << 16);
-                    sgn[i] = ((a >> 8) & 0x80u) | ((a >> 16) & 0x8000u) | ((b << 8) & 0x800000u) |
-                             (b & 0x80000000u);
-                    out[i] |= sgn[i];
                     if (sc == 255u) out[i] = 0;
                 }
                 reinterpret_cast<uint2*>(codes)[g[u]] = make_uint2(out[0], out[1]);
