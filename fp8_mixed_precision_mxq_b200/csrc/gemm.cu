@@ -17,18 +17,20 @@
 //   warp 0      TMA producer (each CTA): A / W tiles (128-byte swizzle) and the
 //               scale-factor atoms (512-byte chunks, as 2-D TMA boxes) into the
 //               shared-memory ring; a pair's loads all complete on the leader's barrier;
-//   warp 1      MMA issuer (leader CTA): copies each stage's scale atoms into TMEM
-//               (tcgen05.cp 32x128b.warpx4) and issues the block-scaled MMAs into
-//               the TMEM accumulators; commits release the stage in both CTAs;
-//               in every CTA this warp allocates and frees TMEM;
+//   warp 1      MMA issuer (leader CTA): for a batch of up to four landed stages,
+//               copies their scale atoms into TMEM (tcgen05.cp 32x128b.warpx4, one
+//               buffer per stage) and then issues their block-scaled MMAs; commits
+//               release each stage in both CTAs; in every CTA this warp allocates and
+//               frees TMEM.  A copy issued behind MMAs waits for them to drain, so the
+//               copies are batched to pay that once per batch rather than per stage;
 //   warps 2..5  epilogue (each CTA): tcgen05.ld 32 columns at a time, + bias, -> bf16,
 //               staged in swizzled shared memory and written with TMA stores.
 // L2 policies: the weight is loaded evict-last (it is reused by every m-block and fits
 // in L2), the output is stored evict-first.
-// TMEM (512 columns): accumulator slot 0 = columns [0, 256), slot 1 = [224, 480),
-// scale factors = [480, 504).  The two slots overlap in [224, 256); the epilogue
-// drains that 32-column chunk first and signals it, so the next tile's MMAs can
-// start while the rest of the previous accumulator is still being written out.
+// TMEM (512 columns): accumulator slot 0 = columns [0, 256), slot 1 = [208, 464),
+// two scale buffers = [464, 512).  The two slots overlap in [208, 256); the epilogue
+// drains those columns first and signals it, so the next tile's MMAs can start while
+// the rest of the previous accumulator is still being written out.
 // Every wait is bounded; a wait that runs out records MXQ_ERR_TIMEOUT in a device
 // status word and the kernel winds down (in-flight copies and MMAs drained, TMEM
 // freed) instead of hanging.
@@ -53,9 +55,14 @@ constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kEpiBuf = 32 * 64;     // 32 rows x 32 bf16
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCol1 = 224;
-constexpr uint32_t kSfaCol = 480;
-constexpr uint32_t kSfbCol = 488;
+// TMEM columns: accumulator slot 0 [0, 256), slot 1 [kAccCol1, kSfCol) (the slots
+// share 256 - kAccCol1 columns), then kSfBufs scale-factor buffers of 24 columns:
+// SFA at +0 (4 columns per k-atom), SFB at +8 (8 columns per k-atom: both halves).
+constexpr uint32_t kSfBufs = 3;            // scale buffers in TMEM = stages per copy batch
+constexpr uint32_t kSfBufCols = 24;
+constexpr uint32_t kSfCol = kTmemCols - kSfBufs * kSfBufCols;
+constexpr uint32_t kAccCol1 = kSfCol - 256;
+constexpr int kOverlapChunks = (256 - kAccCol1 + 31) / 32;  // 32-column chunks the slots share
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 // Shared-memory plan of one CTA.  kPair = 1: the CTA owns a 128 x 256 tile and loads
@@ -121,9 +128,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         return;
     }
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-    uint64_t* full = bars;
-    uint64_t* empty = bars + S;
-    uint64_t* tmem_full = bars + 2 * S;
+    uint64_t* full = bars;                  // a stage landed (the leader's barrier counts the pair)
+    uint64_t* empty = bars + S;             // a stage's MMAs completed (smem reusable)
+    uint64_t* tmem_full = bars + 2 * S;     // accumulator slot complete
     uint64_t* tmem_empty = bars + 2 * S + 2;
     uint64_t* overlap_free = bars + 2 * S + 4;
     uint64_t* mma_done = bars + 2 * S + 5;
@@ -213,9 +220,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader CTA)
         if (leader && lane == 0) {
-            const uint32_t fa = kW4A8 ? 0u : 1u;  // A element type: E4M3 (mxf8f6f4) / E2M1 (mxf4)
-            const uint32_t fb = kW4A8 ? 5u : 1u;  // B element type: E2M1 in both kinds
-            uint32_t it = 0;
+            // One thread issues everything; its instruction stream must stay well inside the
+            // 128 tensor-pipe cycles an MMA takes, so all addresses are precomputed words.
+            constexpr uint32_t fa = kW4A8 ? 0u : 1u;  // A element type: E4M3 (mxf8f6f4) / E2M1 (mxf4)
+            constexpr uint32_t fb = kW4A8 ? 5u : 1u;  // B element type: E2M1 in both kinds
+            constexpr int KPS = kW4A8 ? 128 : 256;    // K elements per stage
+            constexpr int KPM = kW4A8 ? 32 : 64;      // K elements per MMA
+            constexpr int B = static_cast<int>(kSfBufs);
+            const uint32_t a_lo0 = sdesc_sw128_lo(smem_u32(smem + C::kOffA));
+            const uint32_t b_lo0 = sdesc_sw128_lo(smem_u32(smem + C::kOffB));
+            const uint32_t sfa_s0 = smem_u32(smem + C::kOffSFA);
+            const uint32_t sfb_s0 = smem_u32(smem + C::kOffSFB);
+            uint32_t s = 0, ph = 0;  // ring slot and phase parity of the next stage to consume
             int tcount = 0;
             bool ok = true;
             for (int t = pair_id; t < p.num_tiles && ok; t += n_pairs, ++tcount) {
@@ -227,44 +243,62 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                for (int ks = 0; ks < p.k_stages; ++ks, ++it) {
-                    const uint32_t s = it % S;
-                    if (!mbar_wait(&full[s], (it / S) & 1, kWaitNs)) {
+                for (int ks = 0; ks < p.k_stages;) {
+                    // A batch of up to B landed stages: their scale copies go back to back into
+                    // the B scale buffers, then their MMAs.  A copy issued behind MMAs waits for
+                    // them to drain, so batching pays that once per batch rather than per stage.
+                    const int nbat = min(B, p.k_stages - ks);
+                    uint32_t ws = s, wp = ph;
+#pragma unroll
+                    for (int u = 0; u < B; ++u) {
+                        if (u < nbat && !mbar_wait(&full[ws], wp, kWaitNs)) ok = false;
+                        if (++ws == S) { ws = 0; wp ^= 1; }
+                    }
+                    if (!ok) {
                         record_status(MXQ_ERR_TIMEOUT);
-                        ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sfa_s = smem_u32(smem + C::kOffSFA + s * C::kStageSFA);
-                    const uint32_t sfb_s = smem_u32(smem + C::kOffSFB + s * C::kStageSFB);
+                    ws = s;
 #pragma unroll
-                    for (int a = 0; a < AK; ++a) {
-                        tc_copy_sf_atom<kPair>(tmem_base + kSfaCol + 4 * a, sdesc_sf_atom(sfa_s + a * 512));
+                    for (int u = 0; u < B; ++u) {
+                        if (u < nbat) {
+                            const uint32_t sft = tmem_base + kSfCol + u * kSfBufCols;
+                            const uint32_t sfa_s = sfa_s0 + ws * C::kStageSFA;
+                            const uint32_t sfb_s = sfb_s0 + ws * C::kStageSFB;
 #pragma unroll
-                        for (int h = 0; h < 2; ++h)
-                            tc_copy_sf_atom<kPair>(tmem_base + kSfbCol + 8 * a + 4 * h,
-                                                   sdesc_sf_atom(sfb_s + (h * AK + a) * 512));
+                            for (int a = 0; a < AK; ++a) {
+                                tc_copy_sf_atom<kPair>(sft + 4 * a, sdesc_sf_atom(sfa_s + a * 512));
+#pragma unroll
+                                for (int h = 0; h < 2; ++h)
+                                    tc_copy_sf_atom<kPair>(sft + 8 + 8 * a + 4 * h,
+                                                           sdesc_sf_atom(sfb_s + (h * AK + a) * 512));
+                            }
+                        }
+                        if (++ws == S) ws = 0;
                     }
-                    const uint32_t a_s = smem_u32(smem + C::kOffA + s * C::kStageA);
-                    const uint32_t b_s = smem_u32(smem + C::kOffB + s * C::kStageB);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int k_elem = kW4A8 ? ks * 128 + j * 32 : ks * 256 + j * 64;
-                        if (k_elem >= p.K) break;
-                        const int atom = kW4A8 ? 0 : (j >> 1);
-                        const uint32_t sf_id = kW4A8 ? static_cast<uint32_t>(j) : static_cast<uint32_t>((j & 1) * 2);
-                        const uint32_t idesc = idesc_block_scaled(fa, fb, C::BM, BN, sf_id, sf_id);
-                        const uint64_t ad = sdesc_k_sw128(a_s + j * 32);
-                        const uint64_t bd = sdesc_k_sw128(b_s + j * 32);
-                        const uint32_t accumulate = (ks > 0 || j > 0) ? 1u : 0u;
-                        if (kW4A8)
-                            mma_mxf8f6f4<kPair>(acc, ad, bd, idesc, tmem_base + kSfaCol + 4 * atom,
-                                                tmem_base + kSfbCol + 8 * atom, accumulate);
-                        else
-                            mma_mxf4<kPair>(acc, ad, bd, idesc, tmem_base + kSfaCol + 4 * atom,
-                                            tmem_base + kSfbCol + 8 * atom, accumulate);
+                    for (int u = 0; u < B; ++u) {
+                        if (u < nbat) {
+                            const uint32_t sft = tmem_base + kSfCol + u * kSfBufCols;
+                            const uint32_t a_lo = a_lo0 + s * (C::kStageA >> 4);
+                            const uint32_t b_lo = b_lo0 + s * (C::kStageB >> 4);
+                            const int kvalid = p.K - ks * KPS;
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const uint32_t sf_id = kW4A8 ? static_cast<uint32_t>(j) : static_cast<uint32_t>((j & 1) * 2);
+                                const uint32_t atom = kW4A8 ? 0u : static_cast<uint32_t>(j >> 1);
+                                if (j * KPM < kvalid)
+                                    mma_block_scaled<kPair, kW4A8>(acc, a_lo + 2 * j, b_lo + 2 * j, kSdescSw128Hi,
+                                                                   idesc_block_scaled(fa, fb, C::BM, BN, sf_id, sf_id),
+                                                                   sft + 4 * atom, sft + 8 + 8 * atom,
+                                                                   (ks > 0 || j > 0) ? 1u : 0u);
+                            }
+                            tc_commit<kPair>(&empty[s]);  // stage s free (in both CTAs) once these MMAs completed
+                            ++ks;
+                            if (++s == S) { s = 0; ph ^= 1; }
+                        }
                     }
-                    tc_commit<kPair>(&empty[s]);  // stage s free (in both CTAs) once these MMAs completed
                 }
                 if (!ok) break;
                 tc_commit<kPair>(&tmem_full[slot]);  // accumulators ready for both CTAs' epilogues
@@ -284,8 +318,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int tcount = 0;
         for (int t = pair_id; t < p.num_tiles; t += n_pairs, ++tcount) {
             const int slot = tcount & 1;
-            if (!mbar_wait(&tmem_full[slot], (tcount >> 1) & 1, kWaitNs)) {
-                record_status(MXQ_ERR_TIMEOUT);
+            const bool waited = mbar_wait(&tmem_full[slot], (tcount >> 1) & 1, kWaitNs);
+            if (!__all_sync(0xFFFFFFFFu, waited)) {  // the warp leaves together (tcgen05.ld is .aligned)
+                if (lane == 0) record_status(MXQ_ERR_TIMEOUT);
                 break;
             }
             tc_fence_after();
@@ -294,12 +329,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t col0 = slot ? kAccCol1 : 0u;
             const int row0 = mb * C::BM + static_cast<int>(rank) * 128 + q * 32;
             for (int ci = 0; ci < BN / 32; ++ci) {
-                // the 32 columns shared by both slots go first
-                const int c = slot ? ci : (ci == 0 ? BN / 32 - 1 : ci - 1);
+                // the columns shared by both slots (kOverlapChunks chunks) go first
+                const int c = slot ? ci : (ci < kOverlapChunks ? BN / 32 - kOverlapChunks + ci : ci - kOverlapChunks);
                 uint32_t r[32];
                 tmem_ld_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + col0 + c * 32, r);
                 tmem_ld_wait();
-                if (ci == 0) {
+                if (ci == kOverlapChunks - 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(bar_overlap);

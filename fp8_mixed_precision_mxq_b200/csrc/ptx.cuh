@@ -287,6 +287,27 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint6
             : "memory");
 }
 
+// Same, with the two shared-memory descriptors given as (low word, common high word).
+template <int kPair, bool kF8F6F4>
+__device__ __forceinline__ void mma_block_scaled(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t d_hi,
+                                                 uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                 uint32_t accumulate)
+{
+#define MXQ_MMA_ASM(GROUP, KIND)                                                                             \
+    asm volatile("{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\t"                                             \
+                 "mov.b64 ad, {%1, %3};\n\tmov.b64 bd, {%2, %3};\n\t"                                         \
+                 "setp.ne.b32 p, %5, 0;\n\t"                                                                   \
+                 "tcgen05.mma.cta_group::" GROUP ".kind::" KIND " [%0], ad, bd, %4, [%6], [%7], p;\n\t}" ::"r"(  \
+                     d_tmem),                                                                                  \
+                 "r"(a_lo), "r"(b_lo), "r"(d_hi), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)    \
+                 : "memory")
+    if constexpr (kPair == 2 && kF8F6F4) MXQ_MMA_ASM("2", "mxf8f6f4.block_scale");
+    else if constexpr (kPair == 2) MXQ_MMA_ASM("2", "mxf4.block_scale.block32");
+    else if constexpr (kF8F6F4) MXQ_MMA_ASM("1", "mxf8f6f4.block_scale");
+    else MXQ_MMA_ASM("1", "mxf4.block_scale.block32");
+#undef MXQ_MMA_ASM
+}
+
 // kind::mxf8f6f4: 8-bit A (E4M3), B in the byte-padded 4-bit layout (E2M1), K = 32.
 template <int kPair>
 __device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -328,6 +349,23 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32])
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Each thread of a warp writes 4 consecutive 32-bit TMEM columns of its own lane.
+__device__ __forceinline__ void tmem_st_x4(uint32_t taddr, uint4 v)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t saddr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr));
+    return v;
+}
+
 // Shared-memory matrix descriptor (sm_100 form, version 1) for a K-major tile whose
 // rows are 128 bytes wide, stored with the 128-byte swizzle: 8-row groups are
 // 1024 bytes apart.  The tile base must be 1024-byte aligned; stepping along K
@@ -342,6 +380,11 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr)
     d |= static_cast<uint64_t>(2u) << 61;                  // layout: 128-byte swizzle
     return d;
 }
+
+// Upper 32 bits of the K-major 128-byte-swizzle descriptor (stride, version, layout);
+// the lower word is the start address (>> 4) and the unused leading byte offset.
+constexpr uint32_t kSdescSw128Hi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t sdesc_sw128_lo(uint32_t saddr) { return ((saddr >> 4) & 0x3FFFu) | (1u << 16); }
 
 // Descriptor of a scale-factor atom: 32 rows x 16 bytes, no swizzle, 8-row core
 // matrices 128 bytes apart.
