@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "mxq_internal.h"
 
@@ -312,3 +313,69 @@ const char* mxq_last_error(void) { return g_err; }
 const char* mxq_last_path(void) { return g_path; }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------------------
+// Linear layer without any allocation.
+//
+// Some callers cannot allocate device memory at the point where they run a layer: code
+// that runs under a memory manager that owns the whole device pool, plugins that are
+// handed only the input and output buffers, or code paths that must not call into an
+// allocator at all.  mxq_linear_noalloc serves them: the one scratch buffer the native
+// linear needs (the quantized activation: element codes and tiled scales) lives in a
+// file-scope device array of fixed size instead of a caller-provided workspace.
+// ----------------------------------------------------------------------------------------
+namespace {
+
+constexpr int64_t kNoAllocScratchBytes = int64_t(32) << 20;  // 32 MiB per device
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device.  In host code the array's
+// name is only a stand-in, so the address is looked up once per device (with that
+// device current) and cached.
+int noalloc_scratch(void** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(MXQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kNoAllocMaxDevices)
+        return fail(MXQ_ERR_UNSUPPORTED, "device index %d is above the supported %d", dev, kNoAllocMaxDevices);
+    std::lock_guard<std::mutex> g(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return fail(MXQ_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return MXQ_OK;
+}
+
+}  // namespace
+
+extern "C" int64_t mxq_linear_noalloc_max_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+extern "C" int mxq_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const void* w_codes, const void* w_sf,
+                                  int64_t N, const void* bias_bf16, int act_fmt, void* y_bf16, void* stream)
+{
+    RETURN_IF(check_ptr(x_bf16, "x"));
+    // the scratch is 256-byte aligned by its declaration; stand in a non-null aligned value
+    const void* scratch_standin = reinterpret_cast<const void*>(uintptr_t(256));
+    RETURN_IF(check_gemm(scratch_standin, scratch_standin, act_fmt, M, K, w_codes, w_sf, N, bias_bf16, y_bf16));
+    const int64_t need = linear_ws(M, N, K, act_fmt, MXQ_MODE_NATIVE);
+    if (need > kNoAllocScratchBytes)
+        return fail(MXQ_ERR_WORKSPACE,
+                    "mxq_linear_noalloc: M=%lld K=%lld (%s) needs %lld bytes of scratch; the static scratch holds "
+                    "%lld bytes (use mxq_linear with a workspace for larger inputs)",
+                    (long long)M, (long long)K, act_fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1", (long long)need,
+                    (long long)kNoAllocScratchBytes);
+    RETURN_IF(check_device());
+    void* ws = nullptr;
+    RETURN_IF(noalloc_scratch(&ws));
+    return run_linear(x_bf16, M, K, w_codes, w_sf, N, bias_bf16, act_fmt, MXQ_MODE_NATIVE, ws, kNoAllocScratchBytes,
+                      y_bf16, static_cast<cudaStream_t>(stream));
+}

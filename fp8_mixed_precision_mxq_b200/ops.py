@@ -122,6 +122,21 @@ def linear(x: torch.Tensor, w: QWeight, fmt="e2m1", mode="native", workspace=Non
     return out
 
 
+def linear_noalloc(x: torch.Tensor, w: QWeight, fmt="e2m1", out=None, stream=None):
+    """As linear() in native mode, but the library takes its scratch from a fixed static
+    device buffer instead of a workspace (for callers that cannot allocate where they run
+    a layer; see mxq_linear_noalloc in include/mxq.h for the size limit and the rule that
+    calls must not overlap on the GPU).  Only the output is allocated here, and only when
+    `out` is not given."""
+    _cuda_bf16(x, "x")
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
+    check(_lib.lib().mxq_linear_noalloc(_p(x), M, K, _p(w.codes), _p(w.sf), w.N, _p(w.bias), _fmt(fmt), _p(out),
+                                        _stream(stream)), "mxq_linear_noalloc")
+    return out
+
+
 def block_workspace_bytes(weights, rows, w4a8_bits: int, mode="native") -> int:
     descs = (WDesc * 8)(*[w.desc() for w in weights])
     ms = (ctypes.c_int64 * 8)(*rows)

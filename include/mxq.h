@@ -143,6 +143,26 @@ int mxq_dit_block_linears(const mxq_wdesc* w, const void* const* x_in, const int
 /* Workspace bytes mxq_dit_block_linears needs for these weights and row counts. */
 int64_t mxq_block_workspace_bytes(const mxq_wdesc* w, const int64_t* M_in, uint32_t w4a8_bits, int mode);
 
+/* The native linear layer (as mxq_linear with mode NATIVE) for callers that cannot
+ * allocate device memory where they run a layer -- for example code under a memory
+ * manager that owns the whole device pool, or a plugin that is handed only its input and
+ * output buffers.  The scratch it needs (the quantized activation) lives in a file-scope
+ * device array of mxq_linear_noalloc_max_scratch_bytes() bytes (32 MiB) that every GPU
+ * loading the library holds until the process exits; the call allocates and frees
+ * nothing.  Inputs and outputs are as for mxq_linear.  Inputs whose scratch would not fit
+ * (M*K above about 63 million elements for E2M1, 32 million for E4M3) return
+ * MXQ_ERR_WORKSPACE and launch nothing.  The first call on a device looks up the array's device address and
+ * caches it; make that first call before any stream capture.  All calls on a device share
+ * the one array, and it keeps the last call's contents (nothing in it needs to start at
+ * zero: every byte the GEMM reads is written by the same call's quantizer), so calls that
+ * overlap on the GPU -- on different streams or from different threads without ordering --
+ * race and must be avoided.  The blog has no counterpart of this entry point. */
+int mxq_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const void* w_codes, const void* w_sf, int64_t N,
+                       const void* bias_bf16, int act_fmt, void* y_bf16, void* stream);
+
+/* Size in bytes of the static scratch used by mxq_linear_noalloc. */
+int64_t mxq_linear_noalloc_max_scratch_bytes(void);
+
 /* Tiled scale factors -> logical row-major [rows, K/32] bytes (for tests). */
 int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_rowmajor, void* stream);
 
