@@ -17,19 +17,22 @@
 //   warp 0      TMA producer (each CTA): A / W tiles (128-byte swizzle) and the
 //               scale-factor atoms (512-byte chunks, as 2-D TMA boxes) into the
 //               shared-memory ring; a pair's loads all complete on the leader's barrier;
-//   warp 1      MMA issuer (leader CTA): for a batch of up to four landed stages,
-//               copies their scale atoms into TMEM (tcgen05.cp 32x128b.warpx4, one
-//               buffer per stage) and then issues their block-scaled MMAs; commits
-//               release each stage in both CTAs; in every CTA this warp allocates and
-//               frees TMEM.  A copy issued behind MMAs waits for them to drain, so the
-//               copies are batched to pay that once per batch rather than per stage;
+//   warp 1      MMA issuer (leader CTA): issues the block-scaled MMAs of each landed
+//               stage into the TMEM accumulators; its commits release the stage (in
+//               both CTAs) and the stage's TMEM scale buffer; in every CTA this warp
+//               allocates and frees TMEM;
 //   warps 2..5  epilogue (each CTA): tcgen05.ld 32 columns at a time, + bias, -> bf16,
-//               staged in swizzled shared memory and written with TMA stores.
+//               staged in swizzled shared memory and written with TMA stores;
+//   warp 6      scale copies (leader CTA): copies each stage's scale atoms into one of
+//               kSfBufs TMEM scale buffers (tcgen05.cp 32x128b.warpx4) ahead of the
+//               MMAs.  tcgen05 operations of one thread run in order, so copies issued
+//               by the MMA thread would stall behind its MMAs; from their own thread
+//               they overlap them.
 // L2 policies: the weight is loaded evict-last (it is reused by every m-block and fits
 // in L2), the output is stored evict-first.
-// TMEM (512 columns): accumulator slot 0 = columns [0, 256), slot 1 = [208, 464),
-// two scale buffers = [464, 512).  The two slots overlap in [208, 256); the epilogue
-// drains those columns first and signals it, so the next tile's MMAs can start while
+// TMEM (512 columns): accumulator slot 0 = [0, 256), slot 1 = [kAccCol1, kAccCol1 + 256),
+// kSfBufs scale buffers above.  The two slots share 256 - kAccCol1 columns; the
+// epilogue drains those first and signals it, so the next tile's MMAs can start while
 // the rest of the previous accumulator is still being written out.
 // Every wait is bounded; a wait that runs out records MXQ_ERR_TIMEOUT in a device
 // status word and the kernel winds down (in-flight copies and MMAs drained, TMEM
@@ -50,19 +53,23 @@ __device__ uint32_t g_device_status;
 
 namespace {
 
-constexpr int BN = 256;                   // output columns per tile (both variants)
+constexpr int BN = 256;                   // output columns per tile (both variants): 256 or 192
 constexpr int kEpiWarps = 4;
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kThreads = 64 + 32 * kEpiWarps + 32;  // + one scale-copy warp
 constexpr uint32_t kEpiBuf = 32 * 64;     // 32 rows x 32 bf16
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: accumulator slot 0 [0, 256), slot 1 [kAccCol1, kSfCol) (the slots
-// share 256 - kAccCol1 columns), then kSfBufs scale-factor buffers of 24 columns:
-// SFA at +0 (4 columns per k-atom), SFB at +8 (8 columns per k-atom: both halves).
-constexpr uint32_t kSfBufs = 3;            // scale buffers in TMEM = stages per copy batch
+// TMEM columns: accumulator slot 0 [0, BN), slot 1 [kAccCol1, kAccCol1 + BN) (sharing
+// BN - kAccCol1 columns with slot 0 when they do not both fit), then kSfBufs
+// scale-factor buffers of 24 columns: SFA at +0 (4 columns per k-atom), SFB at +8
+// (8 columns per k-atom: the 256 weight rows of the 128-aligned window holding the tile).
+constexpr uint32_t kSfBufs = 3;            // scale buffers in TMEM (the copy thread runs ahead)
 constexpr uint32_t kSfBufCols = 24;
 constexpr uint32_t kSfCol = kTmemCols - kSfBufs * kSfBufCols;
-constexpr uint32_t kAccCol1 = kSfCol - 256;
-constexpr int kOverlapChunks = (256 - kAccCol1 + 31) / 32;  // 32-column chunks the slots share
+// slot 1 follows slot 0 when there is room, otherwise the two slots share columns
+constexpr uint32_t kAccCol1 = kSfCol - BN < uint32_t(BN) ? kSfCol - BN : uint32_t(BN);
+constexpr int kOverlapChunks = kAccCol1 < uint32_t(BN) ? (BN - kAccCol1 + 31) / 32 : 0;  // shared 32-col chunks
+static_assert(BN == 256 || BN == 192, "tile width");
+static_assert(kAccCol1 + BN <= kSfCol, "TMEM plan");
 constexpr uint64_t kWaitNs = 1000000000ull;
 
 // Shared-memory plan of one CTA.  kPair = 1: the CTA owns a 128 x 256 tile and loads
@@ -83,7 +90,7 @@ struct Cfg {
     static constexpr uint32_t kOffSFB = kOffSFA + kStages * kStageSFA;
     static constexpr uint32_t kOffEpi = kOffSFB + kStages * kStageSFB;
     static constexpr uint32_t kOffBar = kOffEpi + kEpiWarps * 2 * kEpiBuf;
-    static constexpr uint32_t kNumBars = 2 * kStages + 6;
+    static constexpr uint32_t kNumBars = 2 * kStages + 6 + 2 * 3;
     static constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16;
     static constexpr int kGroupM = kPair == 2 ? 8 : 16;  // tile rows per rasterization group
     static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -134,6 +141,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* tmem_empty = bars + 2 * S + 2;
     uint64_t* overlap_free = bars + 2 * S + 4;
     uint64_t* mma_done = bars + 2 * S + 5;
+    uint64_t* sf_ready = bars + 2 * S + 6;             // [kSfBufs] scale buffer copied into TMEM
+    uint64_t* sf_free = bars + 2 * S + 6 + kSfBufs;    // [kSfBufs] scale buffer's MMAs completed
     uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
 
     const int warp = threadIdx.x >> 5;
@@ -159,6 +168,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&tmem_empty[s], kEpiWarps * kPair);
         }
         mbar_init(overlap_free, kEpiWarps * kPair);
+        for (uint32_t b = 0; b < kSfBufs; ++b) {
+            mbar_init(&sf_ready[b], 1);
+            mbar_init(&sf_free[b], 1);
+        }
         mbar_init(mma_done, 1);
         fence_mbar_init();
     }
@@ -203,8 +216,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                        nb * BN + static_cast<int>(rank) * C::kRowsB, bar, pol_w);
                     tma_load_2d<kPair>(smem + C::kOffSFA + s * C::kStageSFA, &map_sfa, ks * AK * 128,
                                        mb * kPair + static_cast<int>(rank), bar, pol_a);
-                    tma_load_2d<kPair>(smem + C::kOffSFB + s * C::kStageSFB, &map_sfb, ks * AK * 128, nb * 2,
-                                       bar, pol_w);
+                    tma_load_2d<kPair>(smem + C::kOffSFB + s * C::kStageSFB, &map_sfb, ks * AK * 128,
+                                       (nb * BN) / 128, bar, pol_w);
                 }
             }
             // drain: the last stages' loads have landed once their consumer released them
@@ -226,79 +239,52 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t fb = kW4A8 ? 5u : 1u;  // B element type: E2M1 in both kinds
             constexpr int KPS = kW4A8 ? 128 : 256;    // K elements per stage
             constexpr int KPM = kW4A8 ? 32 : 64;      // K elements per MMA
-            constexpr int B = static_cast<int>(kSfBufs);
             const uint32_t a_lo0 = sdesc_sw128_lo(smem_u32(smem + C::kOffA));
             const uint32_t b_lo0 = sdesc_sw128_lo(smem_u32(smem + C::kOffB));
-            const uint32_t sfa_s0 = smem_u32(smem + C::kOffSFA);
-            const uint32_t sfb_s0 = smem_u32(smem + C::kOffSFB);
             uint32_t s = 0, ph = 0;  // ring slot and phase parity of the next stage to consume
+            uint32_t sfi = 0;        // stages consumed so far (selects the scale buffer)
             int tcount = 0;
             bool ok = true;
             for (int t = pair_id; t < p.num_tiles && ok; t += n_pairs, ++tcount) {
                 const int slot = tcount & 1;
                 const uint32_t acc = tmem_base + (slot ? kAccCol1 : 0u);
                 if (!mbar_wait(&tmem_empty[slot], ((tcount >> 1) & 1) ^ 1, kWaitNs) ||
-                    (tcount > 0 && !mbar_wait(overlap_free, (tcount - 1) & 1, kWaitNs))) {
+                    (kOverlapChunks > 0 && tcount > 0 && !mbar_wait(overlap_free, (tcount - 1) & 1, kWaitNs))) {
                     record_status(MXQ_ERR_TIMEOUT);
                     break;
                 }
                 tc_fence_after();
-                for (int ks = 0; ks < p.k_stages;) {
-                    // A batch of up to B landed stages: their scale copies go back to back into
-                    // the B scale buffers, then their MMAs.  A copy issued behind MMAs waits for
-                    // them to drain, so batching pays that once per batch rather than per stage.
-                    const int nbat = min(B, p.k_stages - ks);
-                    uint32_t ws = s, wp = ph;
-#pragma unroll
-                    for (int u = 0; u < B; ++u) {
-                        if (u < nbat && !mbar_wait(&full[ws], wp, kWaitNs)) ok = false;
-                        if (++ws == S) { ws = 0; wp ^= 1; }
-                    }
-                    if (!ok) {
+                int mb_t, nb_t;
+                tile_coords<C::kGroupM>(t, p.m_blocks, p.n_blocks, mb_t, nb_t);
+                // the tile's first weight row inside its 128-aligned scale window, in 32-row columns
+                const uint32_t sfb_shift = static_cast<uint32_t>(((nb_t * BN) % 128) / 32);
+                for (int ks = 0; ks < p.k_stages; ++ks) {
+                    const uint32_t bsf = sfi % kSfBufs;
+                    if (!mbar_wait(&full[s], ph, kWaitNs) ||
+                        !mbar_wait(&sf_ready[bsf], (sfi / kSfBufs) & 1, kWaitNs)) {
                         record_status(MXQ_ERR_TIMEOUT);
+                        ok = false;
                         break;
                     }
                     tc_fence_after();
-                    ws = s;
+                    const uint32_t sft = tmem_base + kSfCol + bsf * kSfBufCols;
+                    const uint32_t a_lo = a_lo0 + s * (C::kStageA >> 4);
+                    const uint32_t b_lo = b_lo0 + s * (C::kStageB >> 4);
+                    const int kvalid = p.K - ks * KPS;
 #pragma unroll
-                    for (int u = 0; u < B; ++u) {
-                        if (u < nbat) {
-                            const uint32_t sft = tmem_base + kSfCol + u * kSfBufCols;
-                            const uint32_t sfa_s = sfa_s0 + ws * C::kStageSFA;
-                            const uint32_t sfb_s = sfb_s0 + ws * C::kStageSFB;
-#pragma unroll
-                            for (int a = 0; a < AK; ++a) {
-                                tc_copy_sf_atom<kPair>(sft + 4 * a, sdesc_sf_atom(sfa_s + a * 512));
-#pragma unroll
-                                for (int h = 0; h < 2; ++h)
-                                    tc_copy_sf_atom<kPair>(sft + 8 + 8 * a + 4 * h,
-                                                           sdesc_sf_atom(sfb_s + (h * AK + a) * 512));
-                            }
-                        }
-                        if (++ws == S) ws = 0;
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t sf_id = kW4A8 ? static_cast<uint32_t>(j) : static_cast<uint32_t>((j & 1) * 2);
+                        const uint32_t atom = kW4A8 ? 0u : static_cast<uint32_t>(j >> 1);
+                        if (j * KPM < kvalid)
+                            mma_block_scaled<kPair, kW4A8>(acc, a_lo + 2 * j, b_lo + 2 * j, kSdescSw128Hi,
+                                                           idesc_block_scaled(fa, fb, C::BM, BN, sf_id, sf_id),
+                                                           sft + 4 * atom, sft + 8 + 8 * atom + sfb_shift,
+                                                           (ks > 0 || j > 0) ? 1u : 0u);
                     }
-#pragma unroll
-                    for (int u = 0; u < B; ++u) {
-                        if (u < nbat) {
-                            const uint32_t sft = tmem_base + kSfCol + u * kSfBufCols;
-                            const uint32_t a_lo = a_lo0 + s * (C::kStageA >> 4);
-                            const uint32_t b_lo = b_lo0 + s * (C::kStageB >> 4);
-                            const int kvalid = p.K - ks * KPS;
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const uint32_t sf_id = kW4A8 ? static_cast<uint32_t>(j) : static_cast<uint32_t>((j & 1) * 2);
-                                const uint32_t atom = kW4A8 ? 0u : static_cast<uint32_t>(j >> 1);
-                                if (j * KPM < kvalid)
-                                    mma_block_scaled<kPair, kW4A8>(acc, a_lo + 2 * j, b_lo + 2 * j, kSdescSw128Hi,
-                                                                   idesc_block_scaled(fa, fb, C::BM, BN, sf_id, sf_id),
-                                                                   sft + 4 * atom, sft + 8 + 8 * atom,
-                                                                   (ks > 0 || j > 0) ? 1u : 0u);
-                            }
-                            tc_commit<kPair>(&empty[s]);  // stage s free (in both CTAs) once these MMAs completed
-                            ++ks;
-                            if (++s == S) { s = 0; ph ^= 1; }
-                        }
-                    }
+                    tc_commit<kPair>(&empty[s]);             // stage s free (in both CTAs) after these MMAs
+                    tc_commit_local<kPair>(&sf_free[bsf]);  // and so is its scale buffer
+                    ++sfi;
+                    if (++s == S) { s = 0; ph ^= 1; }
                 }
                 if (!ok) break;
                 tc_commit<kPair>(&tmem_full[slot]);  // accumulators ready for both CTAs' epilogues
@@ -306,6 +292,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             // every MMA issued by this thread completes before TMEM is released
             tc_commit_local<kPair>(mma_done);
             if (!mbar_wait(mma_done, 0, kWaitNs)) record_status(MXQ_ERR_TIMEOUT);
+        }
+    } else if (warp == 2 + kEpiWarps) {
+        // ------------------------------------------------------------ scale copies (leader CTA)
+        // tcgen05 operations issued by one thread execute in order, so scale copies issued
+        // by the MMA thread would wait for its MMAs to drain.  This thread issues them
+        // instead, into kSfBufs buffers a stage or two ahead of the MMAs.
+        if (leader && lane == 0) {
+            const uint32_t sfa_s0 = smem_u32(smem + C::kOffSFA);
+            const uint32_t sfb_s0 = smem_u32(smem + C::kOffSFB);
+            uint32_t s = 0, ph = 0, sfi = 0;
+            bool ok = true;
+            for (int t = pair_id; t < p.num_tiles && ok; t += n_pairs) {
+                for (int ks = 0; ks < p.k_stages; ++ks, ++sfi) {
+                    const uint32_t bsf = sfi % kSfBufs;
+                    if (!mbar_wait(&full[s], ph, kWaitNs) ||
+                        !mbar_wait(&sf_free[bsf], ((sfi / kSfBufs) & 1) ^ 1, kWaitNs)) {
+                        record_status(MXQ_ERR_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sft = tmem_base + kSfCol + bsf * kSfBufCols;
+                    const uint32_t sfa_s = sfa_s0 + s * C::kStageSFA;
+                    const uint32_t sfb_s = sfb_s0 + s * C::kStageSFB;
+#pragma unroll
+                    for (int a = 0; a < AK; ++a) {
+                        tc_copy_sf_atom<kPair>(sft + 4 * a, sdesc_sf_atom(sfa_s + a * 512));
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tc_copy_sf_atom<kPair>(sft + 8 + 8 * a + 4 * h, sdesc_sf_atom(sfb_s + (h * AK + a) * 512));
+                    }
+                    tc_commit_local<kPair>(&sf_ready[bsf]);  // arrives when the copies (both CTAs) completed
+                    if (++s == S) { s = 0; ph ^= 1; }
+                }
+            }
         }
     } else {
         // ------------------------------------------------------------ epilogue (each CTA)
