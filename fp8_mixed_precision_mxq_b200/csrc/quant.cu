@@ -121,7 +121,9 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
             }
             if ((lane & 3u) == 0) {
                 const uint32_t blk = g[u] >> 2;
-                const uint32_t r = static_cast<uint32_t>((static_cast<uint64_t>(blk) * kb_magic) >> 40);
+                // (blk * kb_magic) >> 40 without a 64-bit overflow: blk < 2^29 and
+                // kb_magic <= 2^40, so the product needs up to 69 bits
+                const uint32_t r = static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(blk) << 24, kb_magic));
                 const uint32_t kb = blk - r * KB;
                 sf[sf_offset(r, kb, atoms_k)] = static_cast<uint8_t>(sc);
             }
@@ -236,7 +238,8 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, int fmt, voi
     // gains from a second round of blocks queued behind the resident ones)
     const int per_sm = fmt == kFmtE4M3 ? 16 : 8;
     const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * per_sm)));
-    // row = floor(block / KB) as a multiply-shift: exact for block < 2^29 and KB < 2^11
+    // row = floor(block / KB) as a multiply-shift, exact for block < 2^29 and KB <= 2^11:
+    // magic * KB - 2^40 < KB, so block * magic / 2^40 overshoots block / KB by less than 1 / KB
     const uint64_t kb_magic = ((uint64_t(1) << 40) + KB - 1) / KB;
     if (fmt == kFmtE4M3)
         quantize_kernel<kFmtE4M3><<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(x), n_groups, KB,

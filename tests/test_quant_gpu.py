@@ -140,3 +140,31 @@ def test_quantize_bitexact_full_workload(name):
     x = synth.activation(c["M"], c["K"], c["act"], seed=c["seed"], device="cuda",
                          outlier_frac=c.get("outlier_frac", 0.0), outlier_scale=c["outlier_scale"])
     assert_bitexact(x, c["fmt"])
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("fmt", ["e2m1", "e4m3"])
+@pytest.mark.parametrize("K", [32, 64])
+def test_quantize_max_rows_sampled_tiles(fmt, K):
+    """More than 2^24 rows at the smallest K: the kernel's row = block / (K/32) division
+    needs more than 64 bits of product there.  Every 128-row tile of the tiled scales is
+    a contiguous run of ceil(K/128) atoms, so sampled tiles (the first, the one starting
+    at row 2^24, the ragged last one and random ones) are checked byte for byte, codes and
+    scales, against the oracle on the same rows."""
+    from fp8_mixed_precision_mxq_b200 import ops
+    M = (1 << 24) + 200
+    x = synth.activation(M, K, "student_t", seed=K, device="cuda", outlier_frac=0.01, outlier_scale=40.0)
+    codes, sf = ops.quantize_act(x, fmt)
+    torch.cuda.synchronize()
+    rb = oracle.codes_row_bytes(K, _mx.FMT[fmt])
+    tile_bytes = oracle.sf_tiled_bytes(128, K)
+    n_tiles = (M + 127) // 128
+    g = torch.Generator().manual_seed(K)
+    tiles = {0, (1 << 24) // 128, n_tiles - 1} | {int(t) for t in torch.randint(n_tiles, (5,), generator=g)}
+    for t in sorted(tiles):
+        r0, r1 = 128 * t, min(M, 128 * t + 128)
+        c_ref, s_ref, _ = _mx.oracle_quantize(x[r0:r1], fmt)
+        c_gpu = codes[r0 * rb: r1 * rb].cpu().numpy().reshape(r1 - r0, rb)
+        assert np.array_equal(c_gpu, c_ref), "codes of rows %d..%d differ" % (r0, r1 - 1)
+        s_gpu = sf[t * tile_bytes: (t + 1) * tile_bytes].cpu().numpy()
+        assert np.array_equal(s_gpu, oracle.sf_to_tiled(s_ref, K)), "scales of rows %d..%d differ" % (r0, r1 - 1)
