@@ -40,6 +40,36 @@ FP4_OVER_BF16 = 4.0   # nominal dense ratio: 9 PFLOP/s FP4 vs 2.25 PFLOP/s bf16
 FP8_OVER_BF16 = 2.0   # 4.5 PFLOP/s FP8
 
 
+# DRAM traffic of one GEMM launch on a bench workload (dram__bytes_read.sum +
+# dram__bytes_write.sum from one ncu capture of that launch; the profile named holds the
+# command).  A record describes only the kernel built from the sources it was taken on:
+# when their hash differs the line reports traffic as null.
+GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precision_mxq_b200/csrc/ptx.cuh",
+                "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h"]
+GEMM_TRAFFIC = {
+    ("ffn_up_480p_w4a4", 32760): {
+        "bytes": 562497280 + 860919552,
+        "sources_sha256": "a645e26e1ace22f385b22da0f2f36738f7ed7e1dddc602abe412fa958c117b26",
+        "profile": "profiles/mx_gemm_mxf4_pair_ffn_up_480p_traffic.md"},
+}
+
+
+def gemm_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def gemm_traffic(workload: str, M: int):
+    rec = GEMM_TRAFFIC.get((workload, M))
+    if rec is None or rec["sources_sha256"] != gemm_sources_sha256():
+        return None
+    return rec["bytes"]
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -179,9 +209,12 @@ def dist_setup():
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """The largest of the ranks' values (every rank gets it); one all-reduce, on the
+    process group's device (cuda under nccl, cpu under gloo)."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -189,7 +222,19 @@ def max_over_ranks(v: float, world: int) -> float:
 def barrier(world):
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def replica_seed(seed: int, rank: int) -> int:
+    """Seed of a replica's activation batch: every rank quantizes its own tokens."""
+    return seed + 1000 * rank
+
+
+def job_tflops(flops_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job throughput of `world` replicas that each did flops_per_rank in at most
+    ms_max milliseconds."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
 
 
 def run_mxq(args):
@@ -205,7 +250,7 @@ def run_mxq(args):
     stream = torch.cuda.current_stream()
 
     # inputs (per-rank seed offset: every replica gets its own batch)
-    x = synth.activation(M, K, c["act"], seed=c["seed"] + 1000 * rank, device=dev,
+    x = synth.activation(M, K, c["act"], seed=replica_seed(c["seed"], rank), device=dev,
                          outlier_frac=c.get("outlier_frac", 0.0), outlier_scale=c["outlier_scale"])
     w = synth.weight(N, K, seed=c["seed"], device=dev)
     b = synth.bias(N, seed=c["seed"], device=dev)
@@ -233,7 +278,7 @@ def run_mxq(args):
     if status != 0:
         raise RuntimeError("device status %d after the timed steps" % status)
     flops = 2.0 * M * N * K
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = job_tflops(flops, ms, world)
 
     # the two kernels of the step, each timed alone on the launch stream
     xc = ws[: ops.codes_bytes(M, K, fmt)]
@@ -265,7 +310,7 @@ def run_mxq(args):
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(g_tflops / fp4_peak, 4),
                      "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal FP4/bf16 dense ratio)" % (
                          peak_src, peaks["bf16_tflops"], FP4_OVER_BF16),
-                     "ms": round(g_ms, 4), "traffic": None, "path": gemm_path},
+                     "ms": round(g_ms, 4), "traffic": gemm_traffic(wl_name, M), "path": gemm_path},
         "parts": {
             "quantize": {"ms": round(q_ms, 4), "GB/s": round(q_gbs, 1), "peak_GB/s": peaks["hbm_gbs"],
                          "frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4),
@@ -281,6 +326,10 @@ def run_mxq(args):
         result["ffn_up_720p_w4a4"] = bench_target(args, ops, synth, dev, stream, world, rank, peaks, qw, b)
     if args.w4a8:
         result["w4a8"] = bench_w4a8(args, ops, synth, dev, stream, world, rank, peaks)
+    if args.block:
+        result["dit_block_720p"] = bench_block(args, ops, synth, dev, stream, world, rank, peaks)
+    if args.stack:
+        result["expert_stack_480p"] = bench_stack(args, ops, synth, dev, stream, world, rank, peaks)
 
     # end to end: host buffers, H2D of x and D2H of y inside the timed region
     if args.e2e:
@@ -298,7 +347,7 @@ def run_mxq(args):
         barrier(world)
         e_steps = max(3, args.steps // 4)
         e_ms = max_over_ranks(time_loop(e2e_step, e_steps, stream), world)
-        result["e2e"] = {"value": round(world * flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        result["e2e"] = {"value": round(job_tflops(flops, e_ms, world), 2), "unit": "TFLOP/s",
                          "ms_per_step": round(e_ms, 3), "steps": e_steps,
                          "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2}
     if rank == 0 and world == 1 and args.cpu_baseline:
@@ -333,7 +382,7 @@ def bench_target(args, ops, synth, dev, stream, world, rank, peaks, qw, b):
     target is stated for; same weight as the headline workload."""
     c = synth.WORKLOADS["ffn_up_720p_w4a4"]
     M, K, N = c["M"], c["K"], c["N"]
-    x = synth.activation(M, K, c["act"], seed=c["seed"] + 1000 * rank, device=dev,
+    x = synth.activation(M, K, c["act"], seed=replica_seed(c["seed"], rank), device=dev,
                          outlier_frac=c["outlier_frac"], outlier_scale=c["outlier_scale"])
     ws = torch.empty(ops.workspace_bytes(M, N, K, "e2m1"), dtype=torch.uint8, device=dev)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
@@ -355,10 +404,97 @@ def bench_target(args, ops, synth, dev, stream, world, rank, peaks, qw, b):
                      "frac_fp4": round(flops / (g_ms * 1e-3) / 1e12 / fp4_peak, 4)}}
 
 
+def linears_roofline_ms(synth, rows_x, rows_ctx, bits, peaks):
+    """Tensor-core floor of one block's eight linears: each linear's FLOPs at the FP4
+    (W4A4) or FP8 (W4A8) dense peak, the peaks being the measured bf16 burst x the
+    nominal dtype ratio."""
+    fp4 = peaks["bf16_tflops"] * FP4_OVER_BF16 * 1e12
+    fp8 = peaks["bf16_tflops"] * FP8_OVER_BF16 * 1e12
+    t = 0.0
+    for i, (name, N, K, src) in enumerate(synth.BLOCK_LINEARS):
+        rows = rows_x if src == "x" else rows_ctx
+        t += 2.0 * rows * N * K / (fp8 if (bits >> i) & 1 else fp4)
+    return t * 1e3
+
+
+def bench_block(args, ops, synth, dev, stream, world, rank, peaks):
+    """One DiT block's eight linears at 720p / 81 frames (M = 75600, text context 512)
+    through the block entry point, under the three precision masks."""
+    c = synth.BLOCK_720P
+    M, ctx = c["M"], c["ctx"]
+    ws, bs = synth.block_weights(c["seed"], device=dev)
+    qws = [ops.quantize_weight(w, bias=b) for w, b in zip(ws, bs)]
+    del ws, bs
+    xs = synth.block_inputs(M, seed=replica_seed(c["seed"], rank), device=dev, ctx=ctx)
+    rows = [x.shape[0] for x in xs]
+    outs = [torch.empty((r, w.N), dtype=torch.bfloat16, device=dev) for r, w in zip(rows, qws)]
+    wsb = torch.empty(ops.block_workspace_bytes(qws, rows, 0xFF), dtype=torch.uint8, device=dev)
+    flops = synth.block_flops(M, ctx)
+    iters = max(3, args.steps // 10)
+    res = {"workload": "one Wan-A14B DiT block's 8 linears, M=%d video + %d text tokens (%.2f TFLOP)" % (
+        M, ctx, flops / 1e12)}
+    for name, bits in synth.BLOCK_MASKS.items():
+        fn = lambda bits=bits: ops.dit_block_linears(qws, xs, bits, workspace=wsb, outs=outs)  # noqa: E731
+        for _ in range(2):
+            fn()
+        ms = max_over_ranks(time_loop(fn, iters, stream), world)
+        roof = linears_roofline_ms(synth, M, ctx, bits, peaks)
+        res[name] = {"mask": "0x%02x" % bits, "ms": round(ms, 3),
+                     "TFLOP/s": round(job_tflops(flops, ms, world), 1),
+                     "roofline_ms": round(roof, 3), "frac": round(roof / ms, 4)}
+    if ops.poll_status() != 0:
+        raise RuntimeError("device status set during the block measurement")
+    return res
+
+
+def bench_stack(args, ops, synth, dev, stream, world, rank, peaks):
+    """The two-expert stack of 40 blocks at 480p / 81 frames: all 80 blocks' MXFP4
+    weights resident, 8 random blocks per expert in W4A8; one timed unit is the forward
+    of one expert through every linear of its 40 blocks."""
+    c = synth.STACK_480P
+    M, ctx, E, B = c["M"], c["ctx"], c["n_experts"], c["n_blocks"]
+    mask = synth.expert_masks(E, B, c["n_w4a8"], seed=c["seed"])
+    stack = []
+    for e in range(E):
+        blocks = []
+        for blk in range(B):
+            ws, bs = synth.block_weights(synth.stack_block_seed(e, blk), device=dev)
+            blocks.append([ops.quantize_weight(w, bias=b) for w, b in zip(ws, bs)])
+            del ws, bs
+        stack.append(blocks)
+    resident = sum(q.codes.numel() + q.sf.numel() for blocks in stack for blk in blocks for q in blk)
+    xs = synth.block_inputs(M, seed=replica_seed(c["seed"], rank), device=dev, ctx=ctx)
+    rows = [x.shape[0] for x in xs]
+    outs = [torch.empty((r, w.N), dtype=torch.bfloat16, device=dev) for r, w in zip(rows, stack[0][0])]
+    wsb = torch.empty(ops.block_workspace_bytes(stack[0][0], rows, 0xFF), dtype=torch.uint8, device=dev)
+    bits = [[0xFF if mask[e, blk] else 0x00 for blk in range(B)] for e in range(E)]
+
+    def forward(e):
+        for blk in range(B):
+            ops.dit_block_linears(stack[e][blk], xs, bits[e][blk], workspace=wsb, outs=outs)
+
+    for e in range(E):
+        forward(e)
+    iters = max(2, args.steps // 50)
+    flops = B * synth.block_flops(M, ctx)
+    res = {"workload": "two experts x %d blocks, MXFP4 weights resident (%.1f GB), %d W4A8 blocks per expert, "
+                       "M=%d video + %d text tokens; unit = one expert's forward (%.1f TFLOP)" % (
+                           B, resident / 1e9, c["n_w4a8"], M, ctx, flops / 1e12)}
+    for e in range(E):
+        ms = max_over_ranks(time_loop(lambda e=e: forward(e), iters, stream), world)
+        roof = sum(linears_roofline_ms(synth, M, ctx, bits[e][blk], peaks) for blk in range(B))
+        res["expert%d" % e] = {"w4a8_blocks": [blk for blk in range(B) if bits[e][blk]], "ms": round(ms, 2),
+                               "TFLOP/s": round(job_tflops(flops, ms, world), 1),
+                               "roofline_ms": round(roof, 2), "frac": round(roof / ms, 4)}
+    if ops.poll_status() != 0:
+        raise RuntimeError("device status set during the expert-stack measurement")
+    return res
+
+
 def bench_w4a8(args, ops, synth, dev, stream, world, rank, peaks):
     c = synth.WORKLOADS["ffn_down_720p_w4a8"]
     M, K, N = c["M"], c["K"], c["N"]
-    x = synth.activation(M, K, c["act"], seed=c["seed"] + 1000 * rank, device=dev,
+    x = synth.activation(M, K, c["act"], seed=replica_seed(c["seed"], rank), device=dev,
                          outlier_frac=c["outlier_frac"], outlier_scale=c["outlier_scale"])
     w = synth.weight(N, K, seed=c["seed"], device=dev)
     qw = ops.quantize_weight(w, bias=synth.bias(N, seed=c["seed"], device=dev))
@@ -401,7 +537,8 @@ def run_reference(args):
         return
     c = synth.WORKLOADS[args.workload]
     M, K, N, fmt = c["M"], c["K"], c["N"], c["fmt"]
-    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    # about 150 s of oracle work over the whole run, at least half a second per step
+    per_step = max(0.5, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         cpu_baseline(M, N, K, fmt, c["seed"], budget_s=per_step / 2)
     vals, samples = [], None
@@ -436,6 +573,10 @@ def main():
     ap.add_argument("--no-w4a8", dest="w4a8", action="store_false")
     ap.add_argument("--no-target", dest="target", action="store_false",
                     help="skip the 720p FFN-up (M=75600) measurement")
+    ap.add_argument("--no-block", dest="block", action="store_false",
+                    help="skip the DiT-block (M=75600) measurement under the three masks")
+    ap.add_argument("--no-stack", dest="stack", action="store_false",
+                    help="skip the two-expert 40-block stack measurement")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

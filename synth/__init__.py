@@ -51,6 +51,22 @@ WORKLOADS = {
 }
 
 
+# Block-level workloads.  BLOCK_720P: one DiT block's eight linears at 720p / 81 frames,
+# run under three precision masks (bit i set = linear i in W4A8): all W4A4, all W4A8, and
+# mixed with the FFN-down linear (whose post-GELU input is the heavy-tailed one) in W4A8.
+# STACK_480P: two experts of 40 blocks each, all weights resident in MXFP4, at 480p /
+# 81 frames, with n_w4a8 random blocks per expert promoted to W4A8; the per-linear inputs
+# are fixed buffers (attention and norms are not part of the path).
+BLOCK_720P = dict(M=TOKENS_720P, ctx=CTX, seed=40)
+BLOCK_MASKS = {"all_w4a4": 0x00, "all_w4a8": 0xFF, "mixed_ffn_down_w4a8": 0x80}
+STACK_480P = dict(M=TOKENS_480P, ctx=CTX, n_experts=2, n_blocks=40, n_w4a8=8, seed=50)
+
+
+def stack_block_seed(expert: int, block: int, base: int = STACK_480P["seed"]) -> int:
+    """Seed of block `block` of expert `expert` in the two-expert stack."""
+    return base * 1000 + expert * 100 + block
+
+
 def _gen(seed: int, device) -> torch.Generator:
     g = torch.Generator(device=device)
     g.manual_seed(int(seed))

@@ -89,3 +89,78 @@ def test_block_rejects_wrong_workspace():
     with pytest.raises(Exception) as ei:
         ops.dit_block_linears(qws, xs, 0xFF, workspace=small)
     assert "WORKSPACE" in str(ei.value)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("mask_name", list(synth.BLOCK_MASKS))
+def test_block_linears_full_720p_sampled_rows(mask_name):
+    """One block at full size (M = 75600 video tokens, 512 text tokens) under each of
+    the three masks; every linear's output is checked on one random row per 1024-row
+    span plus the first and last rows (the oracle quantizes just those rows: the MX
+    blocks of a row depend on nothing else)."""
+    ops = _ops()
+    c = synth.BLOCK_720P
+    bits = synth.BLOCK_MASKS[mask_name]
+    ws, bs = synth.block_weights(c["seed"], device="cuda")
+    qws = [ops.quantize_weight(w, bias=b) for w, b in zip(ws, bs)]
+    xs = synth.block_inputs(c["M"], seed=c["seed"], device="cuda", ctx=c["ctx"])
+    ys = ops.dit_block_linears(qws, xs, bits)
+    assert ops.poll_status() == 0
+    rows = {c["M"]: synth.sample_rows(c["M"], tile=1024), c["ctx"]: synth.sample_rows(c["ctx"], tile=64)}
+    for i, (name, N, K, src) in enumerate(synth.BLOCK_LINEARS):
+        fmt = "e4m3" if (bits >> i) & 1 else "e2m1"
+        r = rows[xs[i].shape[0]].cuda()
+        ref = oracle_linear(xs[i][r], ws[i], bs[i], fmt)
+        _mx.assert_gemm_close(_mx.bf16_to_f64(ys[i][r]), ref, "%s: linear %s (%s)" % (mask_name, name, fmt))
+
+
+@pytest.mark.slow
+def test_two_expert_stack_full_480p_sampled_linears():
+    """The two-expert, 40-block stack at full size: all 80 blocks quantized and resident
+    (~15 GB of MXFP4), 8 random blocks per expert promoted to W4A8 by the mask, and the
+    forward of each expert issued block by block through the block entry point.  Four
+    (block, linear) pairs per expert, two from W4A8 blocks and two from W4A4 blocks, are
+    checked against the oracle on sampled rows (the oracle re-derives their bf16 weights
+    from the same seeds)."""
+    ops = _ops()
+    c = synth.STACK_480P
+    M, ctx = c["M"], c["ctx"]
+    mask = synth.expert_masks(c["n_experts"], c["n_blocks"], c["n_w4a8"], seed=c["seed"])
+    xs = synth.block_inputs(M, seed=c["seed"], device="cuda", ctx=ctx)
+    stack = []
+    for e in range(c["n_experts"]):
+        blocks = []
+        for blk in range(c["n_blocks"]):
+            ws, bs = synth.block_weights(synth.stack_block_seed(e, blk), device="cuda")
+            blocks.append([ops.quantize_weight(w, bias=b) for w, b in zip(ws, bs)])
+            del ws, bs
+        stack.append(blocks)
+    g = torch.Generator().manual_seed(c["seed"])
+    samples = {}
+    for e in range(c["n_experts"]):
+        hi = [int(b) for b in torch.nonzero(mask[e]).flatten()]
+        lo = [int(b) for b in torch.nonzero(mask[e] == 0).flatten()]
+        for pool in (hi, lo):
+            for j in torch.randperm(len(pool), generator=g)[:2]:
+                samples[(e, pool[int(j)])] = int(torch.randint(8, (1,), generator=g))
+    rows = {M: synth.sample_rows(M, tile=1024).cuda(), ctx: synth.sample_rows(ctx, tile=64).cuda()}
+    rows_i = [rows[x.shape[0]] for x in xs]
+    ws_bytes = ops.block_workspace_bytes(stack[0][0], [x.shape[0] for x in xs], 0xFF)
+    workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    outs = [torch.empty((x.shape[0], w.N), dtype=torch.bfloat16, device="cuda") for x, w in zip(xs, stack[0][0])]
+    got = {}
+    for e in range(c["n_experts"]):
+        for blk in range(c["n_blocks"]):
+            bits = 0xFF if mask[e, blk] else 0x00
+            ops.dit_block_linears(stack[e][blk], xs, bits, workspace=workspace, outs=outs)
+            if (e, blk) in samples:
+                i = samples[(e, blk)]
+                got[(e, blk, i)] = outs[i][rows_i[i]].clone()
+    assert ops.poll_status() == 0
+    assert len(got) == 4 * c["n_experts"]
+    for (e, blk, i), y in sorted(got.items()):
+        ws, bs = synth.block_weights(synth.stack_block_seed(e, blk), device="cuda")
+        fmt = "e4m3" if mask[e, blk] else "e2m1"
+        ref = oracle_linear(xs[i][rows_i[i]], ws[i], bs[i], fmt)
+        _mx.assert_gemm_close(_mx.bf16_to_f64(y), ref, "expert %d block %d linear %s (%s)" % (
+            e, blk, synth.BLOCK_LINEARS[i][0], fmt))
