@@ -330,47 +330,74 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue (each CTA)
+        // Each warp owns the 32 TMEM lanes (= output rows) of its quarter.  Per tile it
+        // drains the accumulator in 32-column chunks: the load of chunk c+1 is in flight
+        // while chunk c gets its bias, is rounded to bf16, staged (64-byte swizzle) and
+        // written by a TMA store.  The shared columns go first; the slot is handed back to
+        // the MMA issuer as soon as its last chunk is in registers.
         const uint64_t pol_y = policy_evict_first();
         const int ew = warp - 2;
         const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const uint32_t lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
         uint8_t* ebuf0 = smem + C::kOffEpi + ew * 2 * kEpiBuf;
         const uint32_t bar_overlap = kPair == 2 ? mapa_shared(smem_u32(overlap_free), 0) : smem_u32(overlap_free);
+        const bool has_bias = p.bias != nullptr;
         int eb = 0;
         int tcount = 0;
         for (int t = pair_id; t < p.num_tiles; t += n_pairs, ++tcount) {
             const int slot = tcount & 1;
+            int mb, nb;
+            tile_coords<C::kGroupM>(t, p.m_blocks, p.n_blocks, mb, nb);
+            // this lane's 8 bias values (tile columns 8*lane ..), loaded before the wait so
+            // the load latency hides behind the tile's MMAs; chunks fetch them by shuffle
+            uint4 bias8 = make_uint4(0u, 0u, 0u, 0u);
+            const int nbias = nb * BN + 8 * lane;
+            if (has_bias && nbias + 8 <= p.N) bias8 = __ldg(reinterpret_cast<const uint4*>(p.bias + nbias));
             const bool waited = mbar_wait(&tmem_full[slot], (tcount >> 1) & 1, kWaitNs);
             if (!__all_sync(0xFFFFFFFFu, waited)) {  // the warp leaves together (tcgen05.ld is .aligned)
                 if (lane == 0) record_status(MXQ_ERR_TIMEOUT);
                 break;
             }
             tc_fence_after();
-            int mb, nb;
-            tile_coords<C::kGroupM>(t, p.m_blocks, p.n_blocks, mb, nb);
             const uint32_t col0 = slot ? kAccCol1 : 0u;
             const int row0 = mb * C::BM + static_cast<int>(rank) * 128 + q * 32;
-            for (int ci = 0; ci < BN / 32; ++ci) {
-                // the columns shared by both slots (kOverlapChunks chunks) go first
-                const int c = slot ? ci : (ci < kOverlapChunks ? BN / 32 - kOverlapChunks + ci : ci - kOverlapChunks);
-                uint32_t r[32];
-                tmem_ld_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + col0 + c * 32, r);
-                tmem_ld_wait();
-                if (ci == kOverlapChunks - 1) {
+            const uint32_t tmem_empty_bar = kPair == 2 ? mapa_shared(smem_u32(&tmem_empty[slot]), 0)
+                                                       : smem_u32(&tmem_empty[slot]);
+            // chunk order: slot 0 drains its shared (top) columns first, slot 1 its bottom ones
+            auto chunk_of = [&](int ci) {
+                return slot ? ci : (ci < kOverlapChunks ? BN / 32 - kOverlapChunks + ci : ci - kOverlapChunks);
+            };
+            // after the load of chunk ci has landed: release what the MMA issuer waits for
+            auto landed = [&](int ci) {
+                if (ci == kOverlapChunks - 1 || ci == BN / 32 - 1) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(bar_overlap);
+                    if (lane == 0) mbar_arrive_cluster(ci == BN / 32 - 1 ? tmem_empty_bar : bar_overlap);
                 }
+            };
+            uint32_t r[2][32];
+            tmem_ld_x32(lanes + col0 + chunk_of(0) * 32, r[0]);
+            tmem_ld_wait();
+            tmem_regs_ready(r[0]);
+            landed(0);
+#pragma unroll
+            for (int ci = 0; ci < BN / 32; ++ci) {
+                if (ci + 1 < BN / 32) tmem_ld_x32(lanes + col0 + chunk_of(ci + 1) * 32, r[(ci + 1) & 1]);
+                const int c = chunk_of(ci);
                 const int n = nb * BN + c * 32;
-                if (n >= p.N) continue;
-                float bv[32];
+                if (n < p.N) {  // warp-uniform
+                    const uint32_t* acc = r[ci & 1];
+                    float bv[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) bv[i] = 0.f;
-                if (p.bias != nullptr) {
+                    for (int i = 0; i < 32; ++i) bv[i] = 0.f;
+                    if (has_bias) {
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        if (n + 8 * g + 8 <= p.N) {
-                            const uint4 u = __ldg(reinterpret_cast<const uint4*>(p.bias + n + 8 * g));
-                            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+                        for (int g = 0; g < 4; ++g) {
+                            const int src = 4 * c + g;  // lane holding columns c*32 + 8g ..
+                            const uint32_t w[4] = {__shfl_sync(0xFFFFFFFFu, bias8.x, src),
+                                                   __shfl_sync(0xFFFFFFFFu, bias8.y, src),
+                                                   __shfl_sync(0xFFFFFFFFu, bias8.z, src),
+                                                   __shfl_sync(0xFFFFFFFFu, bias8.w, src)};
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
                                 bv[8 * g + 2 * i] = __uint_as_float(w[i] << 16);
@@ -378,36 +405,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                     }
-                }
-                uint32_t o[16];
+                    uint32_t o[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * i]) + bv[2 * i],
-                                                             __uint_as_float(r[2 * i + 1]) + bv[2 * i + 1]);
-                    o[i] = *reinterpret_cast<uint32_t*>(&h);
-                }
-                uint8_t* buf = ebuf0 + eb * kEpiBuf;
-                if (lane == 0) bulk_wait_read<1>();  // the store that last used buf has read it
-                __syncwarp();
-                const uint32_t rsw = (static_cast<uint32_t>(lane) >> 1) & 3u;
+                    for (int i = 0; i < 16; ++i) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(acc[2 * i]) + bv[2 * i],
+                                                                 __uint_as_float(acc[2 * i + 1]) + bv[2 * i + 1]);
+                        o[i] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                    uint8_t* buf = ebuf0 + eb * kEpiBuf;
+                    if (lane == 0) bulk_wait_read<1>();  // the store that last used buf has read it
+                    __syncwarp();
+                    const uint32_t rsw = (static_cast<uint32_t>(lane) >> 1) & 3u;
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint4* dst = reinterpret_cast<uint4*>(buf + lane * 64 + ((ch ^ rsw) * 16));
-                    *dst = make_uint4(o[4 * ch], o[4 * ch + 1], o[4 * ch + 2], o[4 * ch + 3]);
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint4* dst = reinterpret_cast<uint4*>(buf + lane * 64 + ((ch ^ rsw) * 16));
+                        *dst = make_uint4(o[4 * ch], o[4 * ch + 1], o[4 * ch + 2], o[4 * ch + 3]);
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&map_y, buf, n, row0, pol_y);
+                        bulk_commit();
+                    }
+                    eb ^= 1;
                 }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&map_y, buf, n, row0, pol_y);
-                    bulk_commit();
+                if (ci + 1 < BN / 32) {
+                    tmem_ld_wait();
+                    tmem_regs_ready(r[(ci + 1) & 1]);
+                    landed(ci + 1);
                 }
-                eb ^= 1;
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive_cluster(kPair == 2 ? mapa_shared(smem_u32(&tmem_empty[slot]), 0)
-                                               : smem_u32(&tmem_empty[slot]));
         }
         if (lane == 0) bulk_wait<0>();
         __syncwarp();

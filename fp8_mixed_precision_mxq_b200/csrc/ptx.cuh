@@ -349,6 +349,15 @@ __device__ __forceinline__ void tmem_ld_x32(uint32_t taddr, uint32_t (&r)[32])
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// After tmem_ld_wait(): ties the 32 destination registers of a finished tcgen05.ld to
+// the wait, so the compiler cannot schedule a use of them above it (the registers of
+// an asynchronous load hold garbage until the wait).
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[32])
+{
+#pragma unroll
+    for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 // Each thread of a warp writes 4 consecutive 32-bit TMEM columns of its own lane.
 __device__ __forceinline__ void tmem_st_x4(uint32_t taddr, uint4 v)
 {
