@@ -71,6 +71,8 @@ constexpr int kOverlapChunks = kAccCol1 < uint32_t(BN) ? (BN - kAccCol1 + 31) / 
 static_assert(BN == 256 || BN == 192, "tile width");
 static_assert(kAccCol1 + BN <= kSfCol, "TMEM plan");
 constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr int kLdBufs = 3;  // epilogue chunk registers in flight (32 columns each)
+static_assert(kOverlapChunks <= kLdBufs, "the shared columns must fit the first round of loads");
 
 // Shared-memory plan of one CTA.  kPair = 1: the CTA owns a 128 x 256 tile and loads
 // all 256 weight rows; kPair = 2: a CTA pair owns a 256 x 256 tile, each CTA loads its
@@ -375,18 +377,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0) mbar_arrive_cluster(ci == BN / 32 - 1 ? tmem_empty_bar : bar_overlap);
                 }
             };
-            uint32_t r[2][32];
-            tmem_ld_x32(lanes + col0 + chunk_of(0) * 32, r[0]);
-            tmem_ld_wait();
-            tmem_regs_ready(r[0]);
-            landed(0);
+            // a ring of kLdBufs chunk registers: the first kLdBufs loads go out back to back, so
+            // the shared columns (kOverlapChunks <= kLdBufs chunks) are released after one wait
+            uint32_t r[kLdBufs][32];
+#pragma unroll
+            for (int j = 0; j < kLdBufs; ++j) tmem_ld_x32(lanes + col0 + chunk_of(j) * 32, r[j]);
+            int issued = kLdBufs, landed_upto = 0;  // constants once the loop below is unrolled
 #pragma unroll
             for (int ci = 0; ci < BN / 32; ++ci) {
-                if (ci + 1 < BN / 32) tmem_ld_x32(lanes + col0 + chunk_of(ci + 1) * 32, r[(ci + 1) & 1]);
+                if (ci >= landed_upto) {  // everything issued so far lands together
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < BN / 32; ++j)
+                        if (j >= landed_upto && j < issued) {
+                            tmem_regs_ready(r[j % kLdBufs]);
+                            landed(j);
+                        }
+                    landed_upto = issued;
+                }
                 const int c = chunk_of(ci);
                 const int n = nb * BN + c * 32;
                 if (n < p.N) {  // warp-uniform
-                    const uint32_t* acc = r[ci & 1];
+                    const uint32_t* acc = r[ci % kLdBufs];
                     float bv[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) bv[i] = 0.f;
@@ -429,10 +441,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     eb ^= 1;
                 }
-                if (ci + 1 < BN / 32) {
-                    tmem_ld_wait();
-                    tmem_regs_ready(r[(ci + 1) & 1]);
-                    landed(ci + 1);
+                if (ci + kLdBufs < BN / 32) {  // refill the buffer just drained
+                    tmem_ld_x32(lanes + col0 + chunk_of(ci + kLdBufs) * 32, r[ci % kLdBufs]);
+                    issued = ci + kLdBufs + 1;
                 }
             }
         }
