@@ -48,8 +48,8 @@ GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precisio
                 "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h"]
 GEMM_TRAFFIC = {
     ("ffn_up_480p_w4a4", 32760): {
-        "bytes": 562497280 + 860919552,
-        "sources_sha256": "a645e26e1ace22f385b22da0f2f36738f7ed7e1dddc602abe412fa958c117b26",
+        "bytes": 542322944 + 860596480,
+        "sources_sha256": "47d069a7afec31613132083a51abcc337e124ad9ffd4ab5d689f421516cee05a",
         "profile": "profiles/mx_gemm_mxf4_pair_ffn_up_480p_traffic.md"},
 }
 
