@@ -18,7 +18,7 @@
  *     even and saturation at the largest finite element;
  *   * the linear layer is Y = deq(Xq) . deq(Wq)^T (+ bias), here in fp64.
  *
- * Readings taken where the pages are silent (each one also listed in the design doc):
+ * Readings taken where the pages are silent:
  *   R1 scale = floor rule above (OCP v1.0);  R2 zero / subnormal amax -> scale code 0;
  *   R3 a block holding Inf or NaN -> scale code 0xFF and all element codes 0;
  *   R4 "RTN" = IEEE round-to-nearest-even, saturating to +-max;
