@@ -68,6 +68,14 @@ def lib():
         L.mxo_sf_to_tiled.restype = i32
         L.mxo_linear_rows.argtypes = [vp, vp, i32, vp, i64, i64, vp, vp, i64, vp, vp, i32]
         L.mxo_linear_rows.restype = i32
+        L.mxo_double_to_bf16.argtypes = [dbl]
+        L.mxo_double_to_bf16.restype = ctypes.c_uint16
+        L.mxo_gelu.argtypes = [dbl]
+        L.mxo_gelu.restype = dbl
+        L.mxo_round_bf16.argtypes = [vp, i64, vp]
+        L.mxo_round_bf16.restype = None
+        L.mxo_gelu_bf16.argtypes = [vp, i64, vp]
+        L.mxo_gelu_bf16.restype = None
     return _lib
 
 
@@ -167,3 +175,41 @@ def linear(a_codes, a_sf, a_fmt, K, w_codes, w_sf, bias_bits=None, nthreads=None
     M = a_codes.shape[0]
     return linear_rows(a_codes, a_sf, a_fmt, np.arange(M, dtype=np.int64), K, w_codes, w_sf,
                        bias_bits, nthreads)
+
+
+def double_to_bf16(v: float) -> int:
+    """bf16 bits of v rounded to nearest, ties to even (overflow -> Inf)."""
+    return int(lib().mxo_double_to_bf16(float(v)))
+
+
+def gelu(x: float) -> float:
+    """GELU(x) = x * Phi(x) in fp64 (the plain erf form)."""
+    return lib().mxo_gelu(float(x))
+
+
+def round_bf16(y: np.ndarray) -> np.ndarray:
+    """fp64 array -> bf16 bit patterns (uint16), same shape."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    out = np.empty(y.shape, dtype=np.uint16)
+    lib().mxo_round_bf16(_ptr(y), y.size, _ptr(out))
+    return out
+
+
+def gelu_bf16(y_bits: np.ndarray) -> np.ndarray:
+    """bf16 bits y -> bf16 bits of GELU(y) (fp64 GELU, one rounding to bf16)."""
+    y_bits = np.ascontiguousarray(y_bits, dtype=np.uint16)
+    out = np.empty(y_bits.shape, dtype=np.uint16)
+    lib().mxo_gelu_bf16(_ptr(y_bits), y_bits.size, _ptr(out))
+    return out
+
+
+def ffn_hidden_rows(a_codes, a_sf, a_fmt, rows, K, w1_codes, w1_sf, b1_bits, h_fmt,
+                    nthreads: int | None = None):
+    """The hidden activation between a FFN's two linears, for the listed rows, as a
+    bf16 network computes it and as the next linear consumes it:
+    y = x . W1^T + b1 (fp64) -> bf16 -> GELU -> bf16 (h) -> MX quantized in h_fmt.
+    Returns (h bits [nrows, N], codes, logical scales)."""
+    y = linear_rows(a_codes, a_sf, a_fmt, rows, K, w1_codes, w1_sf, b1_bits, nthreads)
+    h = gelu_bf16(round_bf16(y))
+    codes, sf = quantize(h, h_fmt, nthreads)
+    return h, codes, sf

@@ -367,3 +367,49 @@ int mxo_linear_rows(const uint8_t *a_codes, const uint8_t *a_sf, int a_fmt,
     free(wdeq);
     return 0;
 }
+
+/* ---- the FFN hidden activation: bf16 rounding and GELU --------------------------- */
+
+/* Round v to the nearest bf16 value, ties to even, returned as bf16 bits.  bf16 is
+ * binary32 with its fraction cut to 7 bits: 8 significant bits, exponent bias 127,
+ * subnormals below 2^-126.  As for any IEEE binary format, a result whose rounded
+ * magnitude (with an unbounded exponent) exceeds the largest finite value is Inf.
+ * NaN stays NaN (the quiet pattern 0x7FC0 with v's sign). */
+uint16_t mxo_double_to_bf16(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    if (isnan(v)) return (uint16_t)(sign | 0x7FC0u);
+    double a = fabs(v);
+    if (isinf(a)) return (uint16_t)(sign | 0x7F80u);
+    if (a == 0.0) return sign;
+    int e2;
+    frexp(a, &e2);
+    int e = e2 - 1;                          /* a = 1.f * 2^e                    */
+    if (e < -126) e = -126;                  /* subnormal spacing below 2^-126   */
+    double q = ldexp(1.0, e - 7);            /* spacing of the bf16 grid near a  */
+    double r = nearbyint(a / q) * q;         /* default rounding: ties to even   */
+    if (r >= ldexp(1.0, 128)) return (uint16_t)(sign | 0x7F80u);
+    float f = (float)r;                      /* exact: every bf16 value is a binary32 value */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(sign | (u >> 16));
+}
+
+/* GELU in its plain form, x * Phi(x) = x/2 * (1 + erf(x / sqrt 2)), in fp64.  The
+ * same function is evaluated as x/2 * erfc(-x / sqrt 2): 1 + erf(t) cancels to
+ * nothing for t below about -6, where erfc keeps full relative accuracy. */
+double mxo_gelu(double x) { return 0.5 * x * erfc(-x / sqrt(2.0)); }
+
+/* n elements: y (fp64) -> bf16 bits, the rounding of a linear layer's output. */
+void mxo_round_bf16(const double *y, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = mxo_double_to_bf16(y[i]);
+}
+
+/* n elements: h = bf16(GELU(y)) for bf16 inputs y, the activation between the FFN's
+ * two linears as a bf16 network computes it (GELU of the bf16 linear output,
+ * rounded back to bf16). */
+void mxo_gelu_bf16(const uint16_t *y, int64_t n, uint16_t *h)
+{
+    for (int64_t i = 0; i < n; ++i) h[i] = mxo_double_to_bf16(mxo_gelu(mxo_bf16_to_double(y[i])));
+}

@@ -33,6 +33,15 @@ MUTANTS = [
      "return atom * 512 + (r % 32) * 4 + ((r / 32) % 4) * 16 + (kb % 4);"),
     ("dequant_wrong_block_index", "mxo_scale_value(sf[r * KB + k / 32]);",
      "mxo_scale_value(sf[r * KB + (k / 32 + 1) % KB]);"),
+    ("bf16_round_truncates", "double r = nearbyint(a / q) * q;", "double r = floor(a / q) * q;"),
+    ("bf16_ties_away_from_zero", "double r = nearbyint(a / q) * q;", "double r = round(a / q) * q;"),
+    ("bf16_overflow_saturates", "if (r >= ldexp(1.0, 128)) return (uint16_t)(sign | 0x7F80u);",
+     "if (r >= ldexp(1.0, 128)) return (uint16_t)(sign | 0x7F7Fu);"),
+    ("gelu_without_sqrt2", "erfc(-x / sqrt(2.0));", "erfc(-x);"),
+    ("gelu_tanh_form", "double mxo_gelu(double x) { return 0.5 * x * erfc(-x / sqrt(2.0)); }",
+     "double mxo_gelu(double x) { return 0.5 * x * (1.0 + tanh(sqrt(2.0 / M_PI) * (x + 0.044715 * x * x * x))); }"),
+    ("gelu_cancelling_form", "double mxo_gelu(double x) { return 0.5 * x * erfc(-x / sqrt(2.0)); }",
+     "double mxo_gelu(double x) { return 0.5 * x * (1.0 + erf(x / sqrt(2.0))); }"),
 ]
 
 

@@ -353,3 +353,100 @@ def test_linear_lossless_case_matches_numpy(fmt):
     rows = np.array([36, 0, 17])
     y2 = oracle.linear_rows(xc, xs, fmt, rows, K, wc, ws, nthreads=3)
     assert np.array_equal(y2, y[rows])
+
+
+# --- the FFN hidden activation: bf16 rounding and GELU --------------------------------------
+#
+# Pins for the two elementwise steps between a FFN's linears (y -> bf16 -> GELU -> bf16):
+# IEEE round-to-nearest-even onto the bf16 grid, and GELU(x) = x * Phi(x) in its erf form.
+
+def _bf16_value(bits):
+    return float(np.array([int(bits) << 16], dtype=np.uint32).view(np.float32)[0])
+
+
+def test_bf16_round_fixed_points():
+    """Every finite bf16 value (both zeros, subnormals, the largest) rounds to itself."""
+    bits, vals = all_finite_bf16()
+    got = oracle.round_bf16(vals)
+    assert np.array_equal(got, bits)
+
+
+def test_bf16_round_midpoints_go_to_even():
+    """The exact midpoint of two neighbouring bf16 values rounds to the one with an even
+    last fraction bit; a hair off the midpoint it rounds to the nearer one."""
+    lo = np.arange(0x0000, 0x7F7F, 97, dtype=np.uint32)  # positive finite, neighbour lo+1 finite
+    for s in (0, 0x8000):
+        for b in lo:
+            a, c = _bf16_value(b | s), _bf16_value((b + 1) | s)
+            mid = (a + c) / 2.0  # exact in double
+            even = b if b % 2 == 0 else b + 1
+            assert oracle.double_to_bf16(mid) == (even | s), hex(b | s)
+            assert oracle.double_to_bf16(math.nextafter(mid, a)) == (b | s)
+            assert oracle.double_to_bf16(math.nextafter(mid, c)) == ((b + 1) | s)
+
+
+def test_bf16_round_matches_integer_rounding_of_binary32():
+    """For values that are binary32 numbers, rounding to bf16 is the rounding of the
+    low 16 bits of the binary32 pattern to even: an integer formula independent of the
+    oracle's arithmetic."""
+    rng = np.random.default_rng(11)
+    u = rng.integers(0, 2 ** 32, size=200000, dtype=np.uint64).astype(np.uint32)
+    f = u.view(np.float32)
+    keep = np.isfinite(f) & (np.abs(f) <= np.float32(3.3895313892515355e38))  # no overflow
+    u, f = u[keep], f[keep]
+    want = ((u.astype(np.uint64) + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+    got = oracle.round_bf16(f.astype(np.float64))
+    assert np.array_equal(got, want)
+
+
+def test_bf16_round_nearest_on_random_doubles():
+    """Doubles with more precision than binary32: the result is the nearer of the two
+    bf16 neighbours that bracket the value."""
+    rng = np.random.default_rng(12)
+    vals = rng.standard_normal(5000) * np.exp2(rng.integers(-140, 120, size=5000))
+    for v in vals:
+        r = oracle.double_to_bf16(v)
+        rv = _bf16_value(r)
+        for nb in (r - 1, r + 1):
+            if (nb & 0x7FFF) < 0x7F80 and (nb & 0x8000) == (r & 0x8000):
+                assert abs(v - rv) <= abs(v - _bf16_value(nb)), (v, hex(r))
+
+
+def test_bf16_round_overflow_and_nan():
+    top = _bf16_value(0x7F7F)                        # largest finite bf16, odd fraction
+    mid = (top + 2.0 ** 128) / 2.0                   # its midpoint with 2^128
+    assert oracle.double_to_bf16(mid) == 0x7F80      # tie goes to even: past the top -> Inf
+    assert oracle.double_to_bf16(math.nextafter(mid, 0.0)) == 0x7F7F
+    assert oracle.double_to_bf16(-mid) == 0xFF80
+    assert oracle.double_to_bf16(float("inf")) == 0x7F80
+    assert oracle.double_to_bf16(float("nan")) & 0x7FC0 == 0x7FC0
+    assert oracle.double_to_bf16(2.0 ** -134) == 0x0000  # half the smallest subnormal: tie to even 0
+    assert oracle.double_to_bf16(3 * 2.0 ** -134) == 0x0002  # 1.5 x smallest: tie to even (2)
+
+
+def test_gelu_is_x_times_normal_cdf():
+    """GELU(x) = x * Phi(x), Phi the standard normal CDF (scipy's ndtr)."""
+    from scipy.special import ndtr
+    xs = np.concatenate([np.linspace(-9.0, 9.0, 3601), [1e-300, -1e-300, 37.5, -5.5]])
+    for x in xs:
+        want = x * ndtr(x)
+        got = oracle.gelu(x)
+        assert abs(got - want) <= 2e-14 * max(abs(want), 1e-300) + 1e-300, (x, got, want)
+
+
+def test_gelu_reflection_and_limits():
+    """GELU(x) - GELU(-x) = x; GELU(0) = 0; GELU(x) = x once Phi(x) rounds to 1."""
+    for x in np.linspace(-6.0, 6.0, 1201):
+        assert abs((oracle.gelu(x) - oracle.gelu(-x)) - x) <= 1e-15 * max(1.0, abs(x)), x
+    assert oracle.gelu(0.0) == 0.0
+    assert oracle.gelu(10.0) == 10.0
+
+
+def test_gelu_bf16_hand_values():
+    """Worked by hand: GELU(1) = 0.84134..., bf16 spacing 2^-8 there, nearest 0.83984375
+    (0x3F57); GELU(-1) = -0.15865..., spacing 2^-10, nearest -0.158203125 (0xBE22);
+    GELU(2) = 1.95449..., spacing 2^-7, nearest 1.953125 (0x3FFA)."""
+    y = np.array([0x3F80, 0xBF80, 0x4000, 0x0000, 0x8000], dtype=np.uint16)  # 1, -1, 2, +0, -0
+    h = oracle.gelu_bf16(y)
+    assert [hex(v) for v in h[:3]] == ["0x3f57", "0xbe22", "0x3ffa"]
+    assert h[3] == 0x0000 and h[4] in (0x0000, 0x8000)  # GELU(-0) = -0 * 1/2
