@@ -48,6 +48,10 @@ SIGNATURES = {
     "mxq_block_workspace_bytes": ([ctypes.POINTER(WDesc), ctypes.POINTER(_i64), _u32, _i32], _i64),
     "mxq_linear_noalloc": ([_vp, _i64, _i64, _vp, _vp, _i64, _vp, _i32, _vp, _vp], _i32),
     "mxq_linear_noalloc_max_scratch_bytes": ([], _i64),
+    "mxq_gemm_gelu_quant": ([_vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp], _i32),
+    "mxq_ffn": ([_vp, _i64, _i64, ctypes.POINTER(WDesc), ctypes.POINTER(WDesc), _i32, _i32, _vp, _i64, _vp, _vp],
+                _i32),
+    "mxq_ffn_workspace_bytes": ([_i64, _i64, _i64, _i32, _i32], _i64),
     "mxq_sf_to_logical": ([_vp, _i64, _i64, _vp, _vp], _i32),
     "mxq_poll_status": ([_vp], _i32),
     "mxq_set_debug": ([_u32], _i32),

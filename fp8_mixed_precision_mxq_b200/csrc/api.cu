@@ -161,6 +161,40 @@ int check_mode(int mode)
     return MXQ_OK;
 }
 
+// Checks of the quantizing-epilogue GEMM beyond those of the plain GEMM: the output is
+// the next layer's activation [M, N] (K = N), so N follows the activation rules.
+int check_gelu_quant(int64_t M, int64_t N, int out_fmt, const void* out_codes, const void* out_sf, const void* h)
+{
+    RETURN_IF(check_fmt(out_fmt));
+    RETURN_IF(check_rows_k(M, N, "hidden activation"));
+    RETURN_IF(check_ptr(out_codes, "out_codes"));
+    RETURN_IF(check_ptr(out_sf, "out_sf"));
+    if (h) RETURN_IF(check_ptr(h, "h"));
+    return MXQ_OK;
+}
+
+int run_gemm_gelu_quant(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K,
+                        const void* w_codes, const void* w_sf, int64_t N, const void* bias, int out_fmt,
+                        void* out_codes, void* out_sf, void* h, cudaStream_t stream)
+{
+    GemmArgs g{a_codes, a_sf, a_fmt, M, N, K, w_codes, w_sf, bias, h};
+    g.out_fmt = out_fmt;
+    g.q_codes = out_codes;
+    g.q_sf = out_sf;
+    const char* msg = nullptr;
+    int rc = launch_gemm(g, stream, &msg, g_path, sizeof g_path);
+    if (rc != MXQ_OK) return fail(rc, "gemm: %s", msg ? msg : "launch failed");
+    return ok();
+}
+
+// FFN workspace: the quantized input (up_fmt) and the quantized hidden activation
+// (down_fmt), each codes then tiled scales, 256-byte aligned.
+int64_t ffn_ws(int64_t M, int64_t K, int64_t H, int up_fmt, int down_fmt)
+{
+    return round_up(codes_bytes(M, K, up_fmt), kWsAlign) + round_up(sf_bytes(M, K), kWsAlign) +
+           round_up(codes_bytes(M, H, down_fmt), kWsAlign) + round_up(sf_bytes(M, H), kWsAlign);
+}
+
 }  // namespace
 
 extern "C" {
@@ -281,6 +315,60 @@ int mxq_dit_block_linears(const mxq_wdesc* w, const void* const* x_in, const int
     }
     snprintf(g_path, sizeof g_path, "block %s w4a8_bits 0x%02x", mode == MXQ_MODE_QDQ ? "qdq" : "native",
              w4a8_bits);
+    return ok();
+}
+
+int mxq_gemm_gelu_quant(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K,
+                        const void* w_codes, const void* w_sf, int64_t N, const void* bias_bf16, int out_fmt,
+                        void* out_codes, void* out_sf, void* h_bf16, void* stream)
+{
+    // out_codes stands in for y in the plain GEMM checks (h is optional)
+    RETURN_IF(check_gemm(a_codes, a_sf, a_fmt, M, K, w_codes, w_sf, N, bias_bf16, out_codes));
+    RETURN_IF(check_gelu_quant(M, N, out_fmt, out_codes, out_sf, h_bf16));
+    RETURN_IF(check_device());
+    return run_gemm_gelu_quant(a_codes, a_sf, a_fmt, M, K, w_codes, w_sf, N, bias_bf16, out_fmt, out_codes, out_sf,
+                               h_bf16, static_cast<cudaStream_t>(stream));
+}
+
+int64_t mxq_ffn_workspace_bytes(int64_t M, int64_t K, int64_t H, int up_fmt, int down_fmt)
+{
+    if (M <= 0 || K <= 0 || H <= 0 || K % 32 != 0 || H % 32 != 0) return -1;
+    if ((up_fmt != MXQ_FMT_E2M1 && up_fmt != MXQ_FMT_E4M3) || (down_fmt != MXQ_FMT_E2M1 && down_fmt != MXQ_FMT_E4M3))
+        return -1;
+    return ffn_ws(M, K, H, up_fmt, down_fmt);
+}
+
+int mxq_ffn(const void* x_bf16, int64_t M, int64_t K, const mxq_wdesc* up, const mxq_wdesc* down, int up_fmt,
+            int down_fmt, void* workspace, int64_t ws_bytes, void* y_bf16, void* stream)
+{
+    if (!up || !down) return fail(MXQ_ERR_INVALID_ARG, "ffn: NULL weight descriptor");
+    if (up->K != K) return fail(MXQ_ERR_SHAPE, "ffn: up-projection K=%lld but x has K=%lld", (long long)up->K,
+                                (long long)K);
+    if (down->K != up->N)
+        return fail(MXQ_ERR_SHAPE, "ffn: down-projection K=%lld differs from the hidden width %lld",
+                    (long long)down->K, (long long)up->N);
+    RETURN_IF(check_ptr(x_bf16, "x"));
+    RETURN_IF(check_ptr(workspace, "workspace", kWsAlign));
+    const int64_t H = up->N;
+    RETURN_IF(check_gemm(workspace, workspace, up_fmt, M, K, up->codes, up->sf, H, up->bias, workspace));
+    RETURN_IF(check_gelu_quant(M, H, down_fmt, workspace, workspace, nullptr));
+    RETURN_IF(check_gemm(workspace, workspace, down_fmt, M, H, down->codes, down->sf, down->N, down->bias, y_bf16));
+    const int64_t need = ffn_ws(M, K, H, up_fmt, down_fmt);
+    if (ws_bytes < need)
+        return fail(MXQ_ERR_WORKSPACE, "ffn workspace has %lld bytes, needs %lld", (long long)ws_bytes,
+                    (long long)need);
+    RETURN_IF(check_device());
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* xc = static_cast<uint8_t*>(workspace);
+    uint8_t* xs = xc + round_up(codes_bytes(M, K, up_fmt), kWsAlign);
+    uint8_t* hc = xs + round_up(sf_bytes(M, K), kWsAlign);
+    uint8_t* hs = hc + round_up(codes_bytes(M, H, down_fmt), kWsAlign);
+    RETURN_IF(cuda_rc(launch_quantize(x_bf16, M, K, up_fmt, xc, xs, st), "quantize launch"));
+    RETURN_IF(run_gemm_gelu_quant(xc, xs, up_fmt, M, K, up->codes, up->sf, H, up->bias, down_fmt, hc, hs, nullptr,
+                                  st));
+    RETURN_IF(run_gemm(hc, hs, down_fmt, M, H, down->codes, down->sf, down->N, down->bias, y_bf16, st));
+    snprintf(g_path, sizeof g_path, "ffn %s -> gelu -> %s fused", up_fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1",
+             down_fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1");
     return ok();
 }
 

@@ -44,6 +44,7 @@
 #include <cstdio>
 #include <cstring>
 
+#include "mx_elem.cuh"
 #include "mxq_internal.h"
 #include "ptx.cuh"
 
@@ -71,15 +72,27 @@ constexpr int kOverlapChunks = kAccCol1 < uint32_t(BN) ? (BN - kAccCol1 + 31) / 
 static_assert(BN == 256 || BN == 192, "tile width");
 static_assert(kAccCol1 + BN <= kSfCol, "TMEM plan");
 constexpr uint64_t kWaitNs = 1000000000ull;
-constexpr int kLdBufs = 3;  // epilogue chunk registers in flight (32 columns each)
-static_assert(kOverlapChunks <= kLdBufs, "the shared columns must fit the first round of loads");
+// Epilogue chunk registers in flight (32 columns each): three for the bf16 output, so the
+// shared columns (kOverlapChunks chunks) leave TMEM after one wait; two when the epilogue
+// also quantizes, which needs the registers.
+constexpr int kLdBufsPlain = 3;
+constexpr int kLdBufsQuant = 2;
+static_assert(kOverlapChunks <= kLdBufsPlain, "the shared columns must fit the first round of loads");
+
+// Output of the epilogue: bf16 y = acc + bias; or the next layer's MX-quantized input,
+// h = bf16(GELU(bf16(acc + bias))) as E2M1 / E4M3 codes with tiled E8M0 scales (and h
+// itself in bf16 when asked for).
+constexpr int kOutBf16 = 0;
+constexpr int kOutGeluE2M1 = 1;
+constexpr int kOutGeluE4M3 = 2;
 
 // Shared-memory plan of one CTA.  kPair = 1: the CTA owns a 128 x 256 tile and loads
 // all 256 weight rows; kPair = 2: a CTA pair owns a 256 x 256 tile, each CTA loads its
 // own 128 activation rows and 128 of the 256 weight rows (the pair MMA reads both).
-template <int kPair>
+template <int kPair, int kOut>
 struct Cfg {
-    static constexpr int kStages = kPair == 2 ? 6 : 4;
+    // the quantizing epilogue's code staging takes one pipeline stage's worth of memory
+    static constexpr int kStages = kPair == 2 ? (kOut ? 5 : 6) : (kOut ? 3 : 4);
     static constexpr int BM = 128 * kPair;
     static constexpr int kRowsB = BN / kPair;
     static constexpr uint32_t kStageA = 128 * 128;
@@ -91,7 +104,9 @@ struct Cfg {
     static constexpr uint32_t kOffSFA = kOffB + kStages * kStageB;
     static constexpr uint32_t kOffSFB = kOffSFA + kStages * kStageSFA;
     static constexpr uint32_t kOffEpi = kOffSFB + kStages * kStageSFB;
-    static constexpr uint32_t kOffBar = kOffEpi + kEpiWarps * 2 * kEpiBuf;
+    static constexpr uint32_t kQBuf = kOut == kOutGeluE4M3 ? 32 * 32 : 32 * 16;  // 32 rows of one block's codes
+    static constexpr uint32_t kOffQ = kOffEpi + kEpiWarps * 2 * kEpiBuf;
+    static constexpr uint32_t kOffBar = kOffQ + (kOut ? kEpiWarps * 2 * kQBuf : 0u);
     static constexpr uint32_t kNumBars = 2 * kStages + 6 + 2 * 3;
     static constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16;
     static constexpr int kGroupM = kPair == 2 ? 8 : 16;  // tile rows per rasterization group
@@ -104,6 +119,12 @@ struct Params {
     int M, N, K;
     int m_blocks, n_blocks, num_tiles, k_stages;
     uint32_t debug;
+    // quantizing epilogue: tiled scales of the output (K = N), their k-atoms, rows padded
+    // to 128, and whether h is also written in bf16 through map_y
+    uint8_t* q_sf;
+    uint32_t q_atoms_k;
+    int q_rows_pad;
+    int write_h;
 };
 
 __device__ __forceinline__ void record_status(uint32_t code) { atomicCAS(&g_device_status, 0u, code); }
@@ -120,13 +141,15 @@ __device__ __forceinline__ void tile_coords(int t, int m_blocks, int n_blocks, i
     mb = first_m + (local - nb * gsize);
 }
 
-template <bool kW4A8, int kPair>
+template <bool kW4A8, int kPair, int kOut>
 __global__ void __launch_bounds__(kThreads, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                    const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
-                   const __grid_constant__ CUtensorMap map_y, const Params p)
+                   const __grid_constant__ CUtensorMap map_y, const __grid_constant__ CUtensorMap map_q,
+                   const Params p)
 {
-    using C = Cfg<kPair>;
+    using C = Cfg<kPair, kOut>;
+    constexpr int kLdBufs = kOut ? kLdBufsQuant : kLdBufsPlain;
     constexpr int S = C::kStages;
     constexpr int AK = kW4A8 ? 1 : 2;  // scale atoms (128 K-elements each) per stage
 
@@ -160,7 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&map_b);
         prefetch_tmap(&map_sfa);
         prefetch_tmap(&map_sfb);
-        prefetch_tmap(&map_y);
+        if (kOut == kOutBf16 || p.write_h) prefetch_tmap(&map_y);
+        if (kOut != kOutBf16) prefetch_tmap(&map_q);
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
@@ -342,6 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const uint32_t lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
         uint8_t* ebuf0 = smem + C::kOffEpi + ew * 2 * kEpiBuf;
+        uint8_t* qbuf0 = smem + C::kOffQ + ew * 2 * C::kQBuf;
         const uint32_t bar_overlap = kPair == 2 ? mapa_shared(smem_u32(overlap_free), 0) : smem_u32(overlap_free);
         const bool has_bias = p.bias != nullptr;
         int eb = 0;
@@ -379,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             // a ring of kLdBufs chunk registers: the first kLdBufs loads go out back to back, so
             // the shared columns (kOverlapChunks <= kLdBufs chunks) are released after one wait
+            uint32_t sfw0 = 0u, sfw1 = 0u;  // quantizing epilogue: this row's 8 scale bytes of the tile
             uint32_t r[kLdBufs][32];
 #pragma unroll
             for (int j = 0; j < kLdBufs; ++j) tmem_ld_x32(lanes + col0 + chunk_of(j) * 32, r[j]);
@@ -417,26 +443,75 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                     }
+                    // o: the chunk in bf16 -- y = acc + bias, or h = GELU of that rounded to bf16
                     uint32_t o[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(acc[2 * i]) + bv[2 * i],
-                                                                 __uint_as_float(acc[2 * i + 1]) + bv[2 * i + 1]);
-                        o[i] = *reinterpret_cast<uint32_t*>(&h);
+                        __nv_bfloat162 y2 = __floats2bfloat162_rn(__uint_as_float(acc[2 * i]) + bv[2 * i],
+                                                                  __uint_as_float(acc[2 * i + 1]) + bv[2 * i + 1]);
+                        if constexpr (kOut != kOutBf16) {
+                            // GELU(y) = y * Phi(y); normcdf keeps the negative tail accurate
+                            const float y0 = __low2float(y2), y1 = __high2float(y2);
+                            y2 = __floats2bfloat162_rn(y0 * normcdff(y0), y1 * normcdff(y1));
+                        }
+                        o[i] = *reinterpret_cast<uint32_t*>(&y2);
                     }
+                    const bool store_y = kOut == kOutBf16 || p.write_h;
                     uint8_t* buf = ebuf0 + eb * kEpiBuf;
-                    if (lane == 0) bulk_wait_read<1>();  // the store that last used buf has read it
+                    if (lane == 0) bulk_wait_read<1>();  // the stores that last used buf have read it
                     __syncwarp();
-                    const uint32_t rsw = (static_cast<uint32_t>(lane) >> 1) & 3u;
+                    if (store_y) {
+                        const uint32_t rsw = (static_cast<uint32_t>(lane) >> 1) & 3u;
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        uint4* dst = reinterpret_cast<uint4*>(buf + lane * 64 + ((ch ^ rsw) * 16));
-                        *dst = make_uint4(o[4 * ch], o[4 * ch + 1], o[4 * ch + 2], o[4 * ch + 3]);
+                        for (int ch = 0; ch < 4; ++ch) {
+                            uint4* dst = reinterpret_cast<uint4*>(buf + lane * 64 + ((ch ^ rsw) * 16));
+                            *dst = make_uint4(o[4 * ch], o[4 * ch + 1], o[4 * ch + 2], o[4 * ch + 3]);
+                        }
+                    }
+                    if constexpr (kOut != kOutBf16) {
+                        // this lane's 32 values are one MX block of the next layer's K: its
+                        // E8M0 scale and element codes, rounded to nearest even by cvt
+                        constexpr uint32_t kEmax = kOut == kOutGeluE4M3 ? 8u : 2u;
+                        uint32_t m2 = o[0];
+#pragma unroll
+                        for (int i = 1; i < 16; ++i) m2 = absmax_bf16x2(m2, o[i]);
+                        m2 = absmax_bf16x2(m2, __byte_perm(m2, 0, 0x1032));
+                        const uint32_t sc = e8m0_code<kEmax>(m2);
+                        const float inv = e8m0_inverse(sc);
+                        const uint32_t keep = sc == 255u ? 0u : 0xFFFFFFFFu;  // a non-finite block: codes 0
+                        uint8_t* qb = qbuf0 + eb * C::kQBuf;
+                        if constexpr (kOut == kOutGeluE2M1) {
+                            uint32_t cw[4];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                uint32_t w = 0;
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    w |= cvt_e2m1x2(lo_f(o[4 * k + i]) * inv, hi_f(o[4 * k + i]) * inv) << (8 * i);
+                                cw[k] = w & keep;
+                            }
+                            *reinterpret_cast<uint4*>(qb + lane * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                        } else {
+                            uint32_t cw[8];
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                cw[k] = (cvt_e4m3x2(lo_f(o[2 * k]) * inv, hi_f(o[2 * k]) * inv) |
+                                         (cvt_e4m3x2(lo_f(o[2 * k + 1]) * inv, hi_f(o[2 * k + 1]) * inv) << 16)) &
+                                        keep;
+                            *reinterpret_cast<uint4*>(qb + lane * 32) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                            *reinterpret_cast<uint4*>(qb + lane * 32 + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+                        }
+                        // scale byte of k-block c of this tile: byte c%4 of word c/4
+                        if (c < 4) sfw0 |= sc << (8 * (c & 3));
+                        else sfw1 |= sc << (8 * (c & 3));
                     }
                     fence_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&map_y, buf, n, row0, pol_y);
+                        if (store_y) tma_store_2d(&map_y, buf, n, row0, pol_y);
+                        if constexpr (kOut != kOutBf16)
+                            tma_store_2d(&map_q, qbuf0 + eb * C::kQBuf, kOut == kOutGeluE2M1 ? n / 2 : n, row0,
+                                         pol_y);
                         bulk_commit();
                     }
                     eb ^= 1;
@@ -444,6 +519,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ci + kLdBufs < BN / 32) {  // refill the buffer just drained
                     tmem_ld_x32(lanes + col0 + chunk_of(ci + kLdBufs) * 32, r[ci % kLdBufs]);
                     issued = ci + kLdBufs + 1;
+                }
+            }
+            if constexpr (kOut != kOutBf16) {
+                // the row's scale bytes of this tile's 8 k-blocks: two 32-bit words of the
+                // tiled layout (k-blocks 4g..4g+3 of one row are 4 consecutive bytes).  Rows
+                // between M and the 128-row padding, and k-blocks past N inside the padding,
+                // get 0, as the layout requires.
+                const int row = row0 + lane;
+                if (row < p.q_rows_pad) {
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        const uint32_t kb0 = static_cast<uint32_t>(nb) * 8u + 4u * g;
+                        if (kb0 < 4u * p.q_atoms_k) {
+                            const size_t off = (static_cast<size_t>(row >> 7) * p.q_atoms_k + (kb0 >> 2)) * 512u +
+                                               (row & 31) * 16u + ((row >> 5) & 3) * 4u;
+                            *reinterpret_cast<uint32_t*>(p.q_sf + off) = row < p.M ? (g ? sfw1 : sfw0) : 0u;
+                        }
+                    }
                 }
             }
         }
@@ -505,13 +598,13 @@ int read_and_clear_device_status(cudaStream_t stream, uint32_t* out)
 
 namespace {
 
-template <bool kW4A8, int kPair>
+template <bool kW4A8, int kPair, int kOut>
 cudaError_t launch_variant(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa,
-                           const CUtensorMap& msb, const CUtensorMap& my, const Params& p, int grid,
-                           cudaStream_t stream)
+                           const CUtensorMap& msb, const CUtensorMap& my, const CUtensorMap& mq, const Params& p,
+                           int grid, cudaStream_t stream)
 {
-    using C = Cfg<kPair>;
-    auto kern = mx_gemm_kernel<kW4A8, kPair>;
+    using C = Cfg<kPair, kOut>;
+    auto kern = mx_gemm_kernel<kW4A8, kPair, kOut>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -526,7 +619,17 @@ cudaError_t launch_variant(const CUtensorMap& ma, const CUtensorMap& mb, const C
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = kPair == 2 ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, my, p);
+    return cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, my, mq, p);
+}
+
+template <bool kW4A8, int kPair>
+cudaError_t launch_out(int out, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa,
+                       const CUtensorMap& msb, const CUtensorMap& my, const CUtensorMap& mq, const Params& p,
+                       int grid, cudaStream_t stream)
+{
+    if (out == kOutGeluE2M1) return launch_variant<kW4A8, kPair, kOutGeluE2M1>(ma, mb, msa, msb, my, mq, p, grid, stream);
+    if (out == kOutGeluE4M3) return launch_variant<kW4A8, kPair, kOutGeluE4M3>(ma, mb, msa, msb, my, mq, p, grid, stream);
+    return launch_variant<kW4A8, kPair, kOutBf16>(ma, mb, msa, msb, my, mq, p, grid, stream);
 }
 
 }  // namespace
@@ -534,12 +637,13 @@ cudaError_t launch_variant(const CUtensorMap& ma, const CUtensorMap& mb, const C
 int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* path, size_t path_len)
 {
     const bool w4a8 = g.a_fmt == kFmtE4M3;
+    const bool quant_out = g.out_fmt >= 0;
     // CTA pairs for anything taller than one 128-row tile; a lone CTA otherwise.
     const int pair = g.M > 128 ? 2 : 1;
     const int rows_b = BN / pair;
     const int64_t atoms_k = sf_atoms_k(g.K);
     const int ak = w4a8 ? 1 : 2;
-    CUtensorMap ma, mb, msa, msb, my;
+    CUtensorMap ma, mb, msa, msb, my, mq;
     const uint64_t a_row = w4a8 ? g.K : g.K / 2;
     bool ok = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a_codes, a_row, g.M, a_row, 128, 128,
                           CU_TENSOR_MAP_SWIZZLE_128B);
@@ -554,8 +658,18 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
                            atoms_k * 512, ak * 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
     ok = ok && make_map_2d(&msb, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.w_sf, atoms_k * 128, ceil_div(g.N, 128),
                            atoms_k * 512, ak * 128, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
-    ok = ok && make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.y, g.N, g.M, g.N * 2, 32, 32,
+    // bf16 output (y, or h of the quantizing epilogue): 32 x 32 boxes, 64-byte swizzle
+    const void* ybase = g.y ? g.y : g.q_codes;  // without h the map is never used
+    ok = ok && make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ybase, g.N, g.M, g.N * 2, 32, 32,
                            CU_TENSOR_MAP_SWIZZLE_64B);
+    if (quant_out) {
+        // codes of the quantized output: one 32-element block (16 or 32 bytes) x 32 rows per box
+        const uint64_t q_row = g.out_fmt == kFmtE4M3 ? g.N : g.N / 2;
+        ok = ok && make_map_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.q_codes, q_row, g.M, q_row,
+                               g.out_fmt == kFmtE4M3 ? 32 : 16, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+    } else {
+        mq = my;  // never used by the bf16 epilogue
+    }
     if (!ok) {
         *msg = "cuTensorMapEncodeTiled failed (driver entry point unavailable or invalid operand layout)";
         return MXQ_ERR_CUDA;
@@ -570,6 +684,11 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     p.num_tiles = p.m_blocks * p.n_blocks;
     p.k_stages = static_cast<int>(ceil_div(g.K, w4a8 ? 128 : 256));
     p.debug = g_debug_flags;
+    p.q_sf = static_cast<uint8_t*>(g.q_sf);
+    p.q_atoms_k = quant_out ? static_cast<uint32_t>(sf_atoms_k(g.N)) : 0u;
+    p.q_rows_pad = static_cast<int>(ceil_div(g.M, 128) * 128);
+    p.write_h = quant_out && g.y != nullptr ? 1 : 0;
+    const int out = !quant_out ? kOutBf16 : (g.out_fmt == kFmtE4M3 ? kOutGeluE4M3 : kOutGeluE2M1);
 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -577,19 +696,20 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     const int grid = std::min(p.num_tiles, sms / pair) * pair;
     cudaError_t e;
     if (w4a8)
-        e = pair == 2 ? launch_variant<true, 2>(ma, mb, msa, msb, my, p, grid, stream)
-                      : launch_variant<true, 1>(ma, mb, msa, msb, my, p, grid, stream);
+        e = pair == 2 ? launch_out<true, 2>(out, ma, mb, msa, msb, my, mq, p, grid, stream)
+                      : launch_out<true, 1>(out, ma, mb, msa, msb, my, mq, p, grid, stream);
     else
-        e = pair == 2 ? launch_variant<false, 2>(ma, mb, msa, msb, my, p, grid, stream)
-                      : launch_variant<false, 1>(ma, mb, msa, msb, my, p, grid, stream);
+        e = pair == 2 ? launch_out<false, 2>(out, ma, mb, msa, msb, my, mq, p, grid, stream)
+                      : launch_out<false, 1>(out, ma, mb, msa, msb, my, mq, p, grid, stream);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) {
         *msg = cudaGetErrorString(e);
         return MXQ_ERR_CUDA;
     }
     if (path)
-        snprintf(path, path_len, "native %s %s %dx%d grid %d tiles %d", w4a8 ? "mxf8f6f4" : "mxf4",
-                 pair == 2 ? "2cta" : "1cta", 128 * pair, BN, grid, p.num_tiles);
+        snprintf(path, path_len, "native %s %s %dx%d grid %d tiles %d%s", w4a8 ? "mxf8f6f4" : "mxf4",
+                 pair == 2 ? "2cta" : "1cta", 128 * pair, BN, grid, p.num_tiles,
+                 !quant_out ? "" : (g.out_fmt == kFmtE4M3 ? " +gelu->e4m3" : " +gelu->e2m1"));
     return MXQ_OK;
 }
 

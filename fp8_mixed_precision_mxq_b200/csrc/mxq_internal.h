@@ -34,7 +34,12 @@ struct GemmArgs {
     const void* w_codes;
     const void* w_sf;
     const void* bias;  // bf16 [N] or null
-    void* y;           // bf16 [M, N]
+    void* y;           // bf16 [M, N]; with out_fmt >= 0: h in bf16, or null
+    // out_fmt >= 0: the epilogue applies GELU and writes the result MX-quantized in that
+    // format (codes [M, N/2] or [M, N], tiled scales with K = N), the next layer's input
+    int out_fmt = -1;
+    void* q_codes = nullptr;
+    void* q_sf = nullptr;
 };
 
 // Builds the tensor maps and launches the tcgen05 GEMM.  Returns an mxq_status;

@@ -13,6 +13,7 @@
 // keeps several 16-byte loads in flight per lane.
 #include <cuda_bf16.h>
 
+#include "mx_elem.cuh"
 #include "mxq_internal.h"
 
 namespace mxq {
@@ -30,37 +31,6 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p)
     return v;
 }
 
-// Packed max of |a| and |b| over two bf16 lanes (sign of the result is the xor of the
-// signs, which the caller masks off); a NaN in either input yields NaN.
-__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b)
-{
-    uint32_t d;
-    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-__device__ __forceinline__ float lo_f(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// Two fp32 -> one byte of two E2M1 codes (first argument in the low nibble).
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi)
-{
-    uint32_t r;
-    asm("{\n\t.reg .b8 t;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
-        "cvt.u32.u8 %0, t;\n\t}"
-        : "=r"(r)
-        : "f"(lo), "f"(hi));
-    return r;
-}
-
-// Two fp32 -> two E4M3 codes in a 16-bit word (first argument in the low byte).
-__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi)
-{
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(lo), "f"(hi));
-    return r;
-}
 
 // Byte offset of scale (r, kb) in the tiled 128x4 atom layout.
 __device__ __forceinline__ uint32_t sf_offset(uint32_t r, uint32_t kb, uint32_t atoms_k)

@@ -137,6 +137,45 @@ def linear_noalloc(x: torch.Tensor, w: QWeight, fmt="e2m1", out=None, stream=Non
     return out
 
 
+def gemm_gelu_quant(a_codes, a_sf, fmt, M: int, K: int, w: QWeight, out_fmt="e2m1", codes=None, sf=None,
+                    h=None, stream=None):
+    """GEMM whose epilogue applies bias + GELU and writes the result MX-quantized in
+    out_fmt (the next layer's input): returns (codes, tiled scales).  Pass a bf16 [M, N]
+    tensor as h to also receive the GELU output."""
+    f = _fmt(out_fmt)
+    if codes is None:
+        codes = torch.empty(max(1, codes_bytes(M, w.N, f)), dtype=torch.uint8, device=a_codes.device)
+    if sf is None:
+        sf = torch.empty(max(1, sf_bytes(M, w.N)), dtype=torch.uint8, device=a_codes.device)
+    if h is not None:
+        _cuda_bf16(h, "h")
+    check(_lib.lib().mxq_gemm_gelu_quant(_p(a_codes), _p(a_sf), _fmt(fmt), M, K, _p(w.codes), _p(w.sf), w.N,
+                                         _p(w.bias), f, _p(codes), _p(sf), _p(h), _stream(stream)),
+          "mxq_gemm_gelu_quant")
+    return codes, sf
+
+
+def ffn_workspace_bytes(M: int, K: int, H: int, up_fmt="e2m1", down_fmt="e2m1") -> int:
+    return int(_lib.lib().mxq_ffn_workspace_bytes(M, K, H, _fmt(up_fmt), _fmt(down_fmt)))
+
+
+def ffn(x: torch.Tensor, up: QWeight, down: QWeight, up_fmt="e2m1", down_fmt="e2m1", workspace=None, out=None,
+        stream=None):
+    """y = quant(GELU(x . up^T + b_up)) . down^T + b_down with the hidden activation kept
+    MX-quantized between the two linears."""
+    _cuda_bf16(x, "x")
+    M, K = x.shape
+    if workspace is None:
+        workspace = torch.empty(ffn_workspace_bytes(M, K, up.N, up_fmt, down_fmt), dtype=torch.uint8,
+                                device=x.device)
+    if out is None:
+        out = torch.empty((M, down.N), dtype=torch.bfloat16, device=x.device)
+    du, dd = up.desc(), down.desc()
+    check(_lib.lib().mxq_ffn(_p(x), M, K, ctypes.byref(du), ctypes.byref(dd), _fmt(up_fmt), _fmt(down_fmt),
+                             _p(workspace), workspace.numel(), _p(out), _stream(stream)), "mxq_ffn")
+    return out
+
+
 def block_workspace_bytes(weights, rows, w4a8_bits: int, mode="native") -> int:
     descs = (WDesc * 8)(*[w.desc() for w in weights])
     ms = (ctypes.c_int64 * 8)(*rows)

@@ -163,6 +163,37 @@ int mxq_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const void* w_c
 /* Size in bytes of the static scratch used by mxq_linear_noalloc. */
 int64_t mxq_linear_noalloc_max_scratch_bytes(void);
 
+/* GEMM whose epilogue produces the next layer's MX-quantized input: the FFN's first
+ * linear followed by its GELU, with the hidden activation never written in bf16.
+ *   y = acc + bias (fp32) rounded to bf16 (the linear's output type);
+ *   h = GELU(y) = y * Phi(y) (the plain erf form, in fp32) rounded to bf16;
+ *   h quantized as mxq_quantize_act would quantize it: per row, each 32 consecutive
+ *   columns form one block (the next layer's K = N), E8M0 scale, E2M1 or E4M3 codes.
+ * Blog section "Quantization formats" for the formats; the FFN whose hidden activation
+ * this is ("WanFeedForward ... GELU") is the one the FP8 page keeps quantized.  The
+ * fusion itself has no counterpart in the pages: it saves the bf16 round trip of h.
+ *   Inputs as for mxq_gemm.  out_fmt: MXQ_FMT_E2M1 or MXQ_FMT_E4M3.
+ *   out_codes: mxq_codes_bytes(M, N, out_fmt) bytes; out_sf: mxq_sf_bytes(M, N) bytes in
+ *   the tiled layout, padding written as 0.  h_bf16: NULL, or [M, N] bf16 to also receive
+ *   h (for checking).  Requires N % 32 == 0 and N <= 65536 (N is the next layer's K);
+ *   all pointers 16-byte aligned.  Errors as for mxq_gemm. */
+int mxq_gemm_gelu_quant(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K,
+                        const void* w_codes, const void* w_sf, int64_t N, const void* bias_bf16, int out_fmt,
+                        void* out_codes, void* out_sf, void* h_bf16, void* stream);
+
+/* The FFN of a DiT block with its hidden activation kept quantized:
+ *   y = (GELU(x . up^T + up.bias) quantized to down_fmt) . down^T + down.bias,
+ * i.e. quantize x to up_fmt, mxq_gemm_gelu_quant into the workspace, then mxq_gemm.
+ * Each linear runs W4A4 or W4A8 as its activation format says (the blog's per-block
+ * policy may pick them independently).  x_bf16 [M, K]; up: N = H, K = K; down: K = H;
+ * y_bf16 [M, down.N].  down_fmt E4M3 needs H % 128 == 0.  workspace holds
+ * mxq_ffn_workspace_bytes(M, K, H, up_fmt, down_fmt) bytes, 256-byte aligned. */
+int mxq_ffn(const void* x_bf16, int64_t M, int64_t K, const mxq_wdesc* up, const mxq_wdesc* down, int up_fmt,
+            int down_fmt, void* workspace, int64_t ws_bytes, void* y_bf16, void* stream);
+
+/* Workspace bytes of mxq_ffn (the quantized input and hidden activation), or -1. */
+int64_t mxq_ffn_workspace_bytes(int64_t M, int64_t K, int64_t H, int up_fmt, int down_fmt);
+
 /* Tiled scale factors -> logical row-major [rows, K/32] bytes (for tests). */
 int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_rowmajor, void* stream);
 

@@ -98,3 +98,36 @@ def test_block_rejects_bad_mask():
     ys = (ctypes.c_void_p * 8)()
     assert L.mxq_dit_block_linears(descs, xs, ms, ys, 0x100, 0, A16, 0, None) == _lib.ERR_INVALID_ARG
     assert L.mxq_dit_block_linears(None, xs, ms, ys, 0, 0, A16, 0, None) == _lib.ERR_INVALID_ARG
+
+
+def test_gemm_gelu_quant_rejects_bad_arguments():
+    L = _lib.lib()
+    #        a_codes a_sf fmt  M    K   w_codes w_sf  N   bias out_fmt codes sf  h  stream
+    bad = [
+        ((A16, A16, 0, 128, 256, A16, A16, 264, None, 0, A16, A16, None, None), _lib.ERR_SHAPE),  # N % 32
+        ((A16, A16, 0, 128, 256, A16, A16, 256, None, 5, A16, A16, None, None), _lib.ERR_INVALID_ARG),  # out_fmt
+        ((A16, A16, 0, 128, 256, A16, A16, 256, None, 1, A16, None, None, None), _lib.ERR_INVALID_ARG),  # out_sf
+        ((A16, A16, 0, 128, 256, A16, A16, 256, None, 1, A8, A16, None, None), _lib.ERR_ALIGN),  # out_codes
+        ((A16, A16, 0, 128, 256, A16, A16, 256, None, 0, A16, A16, A8, None), _lib.ERR_ALIGN),  # h
+    ]
+    for args, status in bad:
+        assert L.mxq_gemm_gelu_quant(*args) == status, (args, _lib.last_error())
+
+
+def test_ffn_workspace_and_shape_checks():
+    L = _lib.lib()
+    assert L.mxq_ffn_workspace_bytes(128, 256, 512, 0, 1) > 0
+    assert L.mxq_ffn_workspace_bytes(128, 250, 512, 0, 1) == -1
+    assert L.mxq_ffn_workspace_bytes(128, 256, 512, 0, 3) == -1
+    up = _lib.WDesc(4096, 4096, None, 512, 256)
+    down = _lib.WDesc(4096, 4096, None, 256, 512)
+    wrong = _lib.WDesc(4096, 4096, None, 256, 384)  # K differs from the hidden width
+    ws = V(1 << 20)
+    need = L.mxq_ffn_workspace_bytes(128, 256, 512, 0, 0)
+    assert L.mxq_ffn(A16, 128, 256, ctypes.byref(up), ctypes.byref(wrong), 0, 0, ws, need, A16,
+                     None) == _lib.ERR_SHAPE
+    assert L.mxq_ffn(A16, 128, 128, ctypes.byref(up), ctypes.byref(down), 0, 0, ws, need, A16,
+                     None) == _lib.ERR_SHAPE
+    assert L.mxq_ffn(A16, 128, 256, ctypes.byref(up), ctypes.byref(down), 0, 0, ws, need - 1, A16,
+                     None) == _lib.ERR_WORKSPACE
+    assert L.mxq_ffn(A16, 128, 256, None, ctypes.byref(down), 0, 0, ws, need, A16, None) == _lib.ERR_INVALID_ARG

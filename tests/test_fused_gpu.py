@@ -1,0 +1,176 @@
+"""The GEMM whose epilogue emits the next layer's MX-quantized input (bias -> bf16 ->
+GELU -> bf16 -> MX block quantization), and the FFN built on it.
+
+The oracle computes the same chain from the same bf16 inputs in fp64
+(oracle.ffn_hidden_rows).  The GPU accumulates in fp32 in another order, so its bf16
+rounding of the linear output differs from the oracle's on a small fraction of
+elements; the checks are therefore:
+  * h (the GELU output, returned for checking) equals the oracle's on >= 99 % of the
+    elements and stays within the GEMM tolerance everywhere;
+  * codes and scales are bit-exact against the oracle on every block whose 32 h values
+    agree with the oracle's;
+  * codes and scales (padding included) are bit-exact against the library's own
+    quantizer -- itself pinned bit-exact to the oracle -- run on the GPU's h;
+  * the FFN output is within the GEMM tolerance of the oracle's FFN chain.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import _mx
+
+pytestmark = pytest.mark.gpu
+
+
+def _ops():
+    from fp8_mixed_precision_mxq_b200 import ops
+    return ops
+
+
+def _bits_np(t):
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def oracle_hidden(x, w1, b1, a_fmt, h_fmt):
+    """Oracle h (bf16 bits), codes and logical scales for all rows of x."""
+    xc, xs, _ = _mx.oracle_quantize(x, a_fmt)
+    wc, ws, _ = _mx.oracle_quantize(w1, "e2m1")
+    rows = np.arange(x.shape[0], dtype=np.int64)
+    bb = _mx.bits(b1) if b1 is not None else None
+    return oracle.ffn_hidden_rows(xc, xs, _mx.FMT[a_fmt], rows, x.shape[1], wc, ws, bb, _mx.FMT[h_fmt])
+
+
+def check_hidden(M, N, h_gpu, codes, sf, h_ref, c_ref, s_ref, h_fmt, what):
+    ops = _ops()
+    hg = _bits_np(h_gpu).reshape(M, N)
+    eq = hg == h_ref
+    assert eq.mean() >= 0.99, "%s: only %.4f of h equals the oracle's" % (what, eq.mean())
+    _mx.assert_gemm_close(_mx.bf16_to_f64(h_gpu),
+                          torch.from_numpy(h_ref.view(np.int16)).view(torch.bfloat16).double().numpy(), what + " h")
+    # bit-exact on every block whose h agrees with the oracle
+    KB = N // 32
+    blk_eq = eq.reshape(M, KB, 32).all(axis=2)
+    s_gpu = ops.sf_to_logical(sf, M, N).cpu().numpy()
+    assert np.array_equal(s_gpu[blk_eq], s_ref[blk_eq]), what + ": scales differ on agreeing blocks"
+    per = 32 if h_fmt == "e4m3" else 16
+    c_gpu = codes.cpu().numpy()[: M * KB * per].reshape(M, KB, per)
+    assert np.array_equal(c_gpu[blk_eq], c_ref.reshape(M, KB, per)[blk_eq]), what + ": codes differ on agreeing blocks"
+    assert blk_eq.mean() >= 0.8, what
+    # every block (and the layout's padding) equals the library quantizer run on the GPU's h
+    c2, s2 = ops.quantize_act(h_gpu, h_fmt)
+    assert torch.equal(codes[: c2.numel()], c2), what + ": codes differ from quantize(h)"
+    assert torch.equal(sf[: s2.numel()], s2), what + ": tiled scales differ from quantize(h)"
+
+
+CASES = [  # M, N, K, a_fmt, h_fmt
+    (128, 256, 512, "e2m1", "e2m1"),
+    (128, 256, 512, "e2m1", "e4m3"),
+    (300, 544, 512, "e2m1", "e2m1"),   # ragged M (CTA pairs) and N (last tile 32 columns)
+    (300, 544, 512, "e4m3", "e4m3"),   # W4A8 GEMM feeding an E4M3 hidden activation
+    (1, 32, 128, "e2m1", "e2m1"),      # one row, one output block (k-blocks padded to 4)
+    (513, 1056, 1024, "e4m3", "e2m1"),
+]
+
+
+@pytest.mark.parametrize("M,N,K,a_fmt,h_fmt", CASES)
+def test_gemm_gelu_quant_against_oracle(M, N, K, a_fmt, h_fmt):
+    ops = _ops()
+    x = synth.activation(M, K, "normal", seed=M + N, device="cuda", outlier_frac=0.02, outlier_scale=30.0)
+    w = synth.weight(N, K, seed=N + K, device="cuda")
+    b = synth.bias(N, seed=N, device="cuda")
+    qw = ops.quantize_weight(w, bias=b)
+    xc, xs = ops.quantize_act(x, a_fmt)
+    h = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    codes, sf = ops.gemm_gelu_quant(xc, xs, a_fmt, M, K, qw, out_fmt=h_fmt, h=h)
+    assert ops.poll_status() == 0
+    assert "+gelu->" + h_fmt in ops.last_path()
+    h_ref, c_ref, s_ref = oracle_hidden(x, w, b, a_fmt, h_fmt)
+    check_hidden(M, N, h, codes, sf, h_ref, c_ref, s_ref, h_fmt, "M=%d N=%d %s->%s" % (M, N, a_fmt, h_fmt))
+    # without the h output the codes and scales are the same
+    codes2, sf2 = ops.gemm_gelu_quant(xc, xs, a_fmt, M, K, qw, out_fmt=h_fmt)
+    assert torch.equal(codes2, codes) and torch.equal(sf2, sf)
+
+
+def test_gemm_gelu_quant_padding_rows_are_zero():
+    """Rows between M and the next multiple of 128 get scale 0 in the tiled layout,
+    whatever the buffer held before."""
+    ops = _ops()
+    M, N, K = 200, 256, 256
+    x = synth.activation(M, K, "normal", seed=3, device="cuda")
+    qw = ops.quantize_weight(synth.weight(N, K, seed=4, device="cuda"))
+    xc, xs = ops.quantize_act(x, "e2m1")
+    sf = torch.full((ops.sf_bytes(M, N),), 0x77, dtype=torch.uint8, device="cuda")
+    codes = torch.empty((ops.codes_bytes(M, N, "e2m1"),), dtype=torch.uint8, device="cuda")
+    ops.gemm_gelu_quant(xc, xs, "e2m1", M, K, qw, out_fmt="e2m1", codes=codes, sf=sf)
+    assert ops.poll_status() == 0
+    h = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ops.gemm_gelu_quant(xc, xs, "e2m1", M, K, qw, out_fmt="e2m1", h=h)
+    _, s2 = ops.quantize_act(h, "e2m1")
+    assert torch.equal(sf, s2)
+    assert not (sf == 0x77).any()
+
+
+def oracle_ffn_rows(x, w1, b1, w2, b2, up_fmt, down_fmt, rows):
+    """The unfused FFN in fp64 on the listed rows: linear -> bf16 -> GELU -> bf16 ->
+    MX quantize -> linear."""
+    xr = x[torch.as_tensor(rows, device=x.device)]
+    h, hc, hs = oracle_hidden(xr, w1, b1, up_fmt, down_fmt)
+    wc, ws, _ = _mx.oracle_quantize(w2, "e2m1")
+    return oracle.linear_rows(hc, hs, _mx.FMT[down_fmt], np.arange(len(rows), dtype=np.int64), w1.shape[0], wc, ws,
+                              _mx.bits(b2))
+
+
+@pytest.mark.parametrize("up_fmt,down_fmt", [("e2m1", "e2m1"), ("e2m1", "e4m3"), ("e4m3", "e2m1"),
+                                             ("e4m3", "e4m3")])
+def test_ffn_against_oracle(up_fmt, down_fmt):
+    ops = _ops()
+    M, K, H, N2 = 300, 512, 1024, 256
+    x = synth.activation(M, K, "normal", seed=5, device="cuda", outlier_frac=0.02, outlier_scale=30.0)
+    w1, b1 = synth.weight(H, K, seed=6, device="cuda"), synth.bias(H, seed=6, device="cuda")
+    w2, b2 = synth.weight(N2, H, seed=7, device="cuda"), synth.bias(N2, seed=7, device="cuda")
+    up, down = ops.quantize_weight(w1, bias=b1), ops.quantize_weight(w2, bias=b2)
+    y = ops.ffn(x, up, down, up_fmt, down_fmt)
+    assert ops.poll_status() == 0
+    assert "ffn" in ops.last_path()
+    ref = oracle_ffn_rows(x, w1, b1, w2, b2, up_fmt, down_fmt, np.arange(M))
+    _mx.assert_gemm_close(_mx.bf16_to_f64(y), ref, "ffn %s->%s" % (up_fmt, down_fmt))
+    # the same chain through the separate entry points gives the same bits
+    xc, xs = ops.quantize_act(x, up_fmt)
+    hc, hs = ops.gemm_gelu_quant(xc, xs, up_fmt, M, K, up, out_fmt=down_fmt)
+    y2 = ops.gemm(hc, hs, down_fmt, M, H, down)
+    assert torch.equal(y, y2)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("down_fmt", ["e2m1", "e4m3"])
+def test_ffn_full_720p_sampled_rows(down_fmt):
+    """The block's FFN at full size (M = 75600 tokens, dim 5120, hidden 13824), FFN-down in
+    W4A4 or W4A8; h and the output checked on one row per 1024-row span plus the ends."""
+    ops = _ops()
+    c = synth.BLOCK_720P
+    M = c["M"]
+    ws, bs = synth.block_weights(c["seed"], device="cuda")
+    i_up = [n for n, *_ in synth.BLOCK_LINEARS].index("ffn_up")
+    i_dn = [n for n, *_ in synth.BLOCK_LINEARS].index("ffn_down")
+    w1, b1, w2, b2 = ws[i_up], bs[i_up], ws[i_dn], bs[i_dn]
+    x = synth.activation(M, w1.shape[1], "normal", seed=c["seed"] * 100 + i_up, device="cuda",
+                         outlier_frac=0.01, outlier_scale=30.0)
+    up, down = ops.quantize_weight(w1, bias=b1), ops.quantize_weight(w2, bias=b2)
+    y = ops.ffn(x, up, down, "e2m1", down_fmt)
+    assert ops.poll_status() == 0
+    rows = synth.sample_rows(M, tile=1024).numpy()
+    ref = oracle_ffn_rows(x, w1, b1, w2, b2, "e2m1", down_fmt, rows)
+    _mx.assert_gemm_close(_mx.bf16_to_f64(y[torch.from_numpy(rows).cuda()]), ref, "ffn 720p ->" + down_fmt)
+    # the hidden activation of the same launch configuration, on the sampled rows
+    xc, xs = ops.quantize_act(x, "e2m1")
+    h = torch.empty((M, w1.shape[0]), dtype=torch.bfloat16, device="cuda")
+    codes, sf = ops.gemm_gelu_quant(xc, xs, "e2m1", M, w1.shape[1], up, out_fmt=down_fmt, h=h)
+    assert ops.poll_status() == 0
+    r = torch.from_numpy(rows).cuda()
+    h_ref, _, _ = oracle_hidden(x[r], w1, b1, "e2m1", down_fmt)
+    eq = _bits_np(h[r]) == h_ref
+    assert eq.mean() >= 0.99
+    c2, s2 = ops.quantize_act(h, down_fmt)
+    assert torch.equal(codes, c2) and torch.equal(sf, s2)
