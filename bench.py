@@ -9,8 +9,15 @@ load-time step).  Beside the headline number the JSON line carries:
   roofline      the dominant kernel (the GEMM) against the tensor-core peak, timed
                 alone with CUDA events on its launch stream;
   parts         the quantizer (GB/s against HBM) and the GEMM separately;
+  ffn_up_720p_w4a4  the same linear at 720p / 81 frames (M = 75600);
   w4a8          the W4A8 FFN-down linear at 720p (quantize to E4M3 + mxf8f6f4 GEMM)
                 and its quantize-dequantize emulation (QDQ) path;
+  ffn_720p      the block's FFN with its hidden activation kept MX-quantized (the
+                FFN-up GEMM's epilogue applies GELU and quantizes), FFN-down W4A4 or W4A8;
+  dit_block_720p  one DiT block's eight linears under the all-W4A4, all-W4A8 and mixed
+                masks;
+  expert_stack_480p  the two-expert stack of 40 blocks, MXFP4 weights resident, one
+                expert's forward per timed unit;
   e2e           the same step through host buffers (pinned H2D of x, D2H of y);
   cpu_baseline  the CPU oracle on a bounded sample of the same workload.
 
@@ -326,6 +333,8 @@ def run_mxq(args):
         result["ffn_up_720p_w4a4"] = bench_target(args, ops, synth, dev, stream, world, rank, peaks, qw, b)
     if args.w4a8:
         result["w4a8"] = bench_w4a8(args, ops, synth, dev, stream, world, rank, peaks)
+    if args.ffn:
+        result["ffn_720p"] = bench_ffn(args, ops, synth, dev, stream, world, rank, peaks)
     if args.block:
         result["dit_block_720p"] = bench_block(args, ops, synth, dev, stream, world, rank, peaks)
     if args.stack:
@@ -415,6 +424,61 @@ def linears_roofline_ms(synth, rows_x, rows_ctx, bits, peaks):
         rows = rows_x if src == "x" else rows_ctx
         t += 2.0 * rows * N * K / (fp8 if (bits >> i) & 1 else fp4)
     return t * 1e3
+
+
+def bench_ffn(args, ops, synth, dev, stream, world, rank, peaks):
+    """The block's FFN at 720p / 81 frames (M = 75600, dim 5120, hidden 13824) with the
+    hidden activation kept MX-quantized (mxq_ffn: quantize, FFN-up GEMM whose epilogue
+    applies GELU and quantizes, FFN-down GEMM), FFN-down in W4A4 or W4A8.  Beside it,
+    for comparison only, the unfused pipeline: mxq_linear, torch's GELU on the bf16
+    hidden activation, mxq_linear."""
+    c = synth.BLOCK_720P
+    M = c["M"]
+    names = [n for n, *_ in synth.BLOCK_LINEARS]
+    i_up, i_dn = names.index("ffn_up"), names.index("ffn_down")
+    ws, bs = synth.block_weights(c["seed"], device=dev)
+    up, down = ops.quantize_weight(ws[i_up], bias=bs[i_up]), ops.quantize_weight(ws[i_dn], bias=bs[i_dn])
+    del ws, bs
+    K, H, N2 = up.K, up.N, down.N
+    x = synth.activation(M, K, "normal", seed=replica_seed(c["seed"] * 100 + i_up, rank), device=dev,
+                         outlier_frac=0.01, outlier_scale=30.0)
+    y = torch.empty((M, N2), dtype=torch.bfloat16, device=dev)
+    flops = 2.0 * M * (K * H + H * N2)
+    fp4 = peaks["bf16_tflops"] * FP4_OVER_BF16 * 1e12
+    fp8 = peaks["bf16_tflops"] * FP8_OVER_BF16 * 1e12
+    iters = max(3, args.steps // 10)
+    res = {"workload": "Wan-A14B FFN at 720p: M=%d, %d -> %d -> %d, FFN-up W4A4 (%.2f TFLOP)" % (
+        M, K, H, N2, flops / 1e12)}
+    for down_fmt in ("e2m1", "e4m3"):
+        wsb = torch.empty(ops.ffn_workspace_bytes(M, K, H, "e2m1", down_fmt), dtype=torch.uint8, device=dev)
+        fn = lambda f=down_fmt, w=wsb: ops.ffn(x, up, down, "e2m1", f, workspace=w, out=y)  # noqa: E731
+        for _ in range(2):
+            fn()
+        ms = max_over_ranks(time_loop(fn, iters, stream), world)
+        roof = (2.0 * M * K * H / fp4 + 2.0 * M * H * N2 / (fp8 if down_fmt == "e4m3" else fp4)) * 1e3
+        res["fused_down_" + down_fmt] = {"ms": round(ms, 3), "TFLOP/s": round(job_tflops(flops, ms, world), 1),
+                                         "roofline_ms": round(roof, 3), "frac": round(roof / ms, 4),
+                                         "launches": 3, "path": ops.last_path()}
+        del wsb
+    # unfused comparison (W4A4 down): bf16 hidden activation written, GELU by torch, read back
+    hbuf = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+    wsl = torch.empty(max(ops.workspace_bytes(M, H, K, "e2m1"), ops.workspace_bytes(M, N2, H, "e2m1")),
+                      dtype=torch.uint8, device=dev)
+
+    def unfused():
+        ops.linear(x, up, "e2m1", workspace=wsl, out=hbuf)
+        h = torch.nn.functional.gelu(hbuf)
+        ops.linear(h, down, "e2m1", workspace=wsl, out=y)
+
+    for _ in range(2):
+        unfused()
+    ms = max_over_ranks(time_loop(unfused, iters, stream), world)
+    res["unfused_down_e2m1"] = {"ms": round(ms, 3), "TFLOP/s": round(job_tflops(flops, ms, world), 1),
+                                "bf16_hidden_bytes_round_trip": 2 * M * H * 2 * 2,
+                                "note": "comparison only: includes torch's GELU kernel"}
+    if ops.poll_status() != 0:
+        raise RuntimeError("device status set during the FFN measurement")
+    return res
 
 
 def bench_block(args, ops, synth, dev, stream, world, rank, peaks):
@@ -573,6 +637,8 @@ def main():
     ap.add_argument("--no-w4a8", dest="w4a8", action="store_false")
     ap.add_argument("--no-target", dest="target", action="store_false",
                     help="skip the 720p FFN-up (M=75600) measurement")
+    ap.add_argument("--no-ffn", dest="ffn", action="store_false",
+                    help="skip the fused-FFN (M=75600) measurement")
     ap.add_argument("--no-block", dest="block", action="store_false",
                     help="skip the DiT-block (M=75600) measurement under the three masks")
     ap.add_argument("--no-stack", dest="stack", action="store_false",

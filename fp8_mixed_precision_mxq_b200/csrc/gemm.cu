@@ -72,12 +72,11 @@ constexpr int kOverlapChunks = kAccCol1 < uint32_t(BN) ? (BN - kAccCol1 + 31) / 
 static_assert(BN == 256 || BN == 192, "tile width");
 static_assert(kAccCol1 + BN <= kSfCol, "TMEM plan");
 constexpr uint64_t kWaitNs = 1000000000ull;
-// Epilogue chunk registers in flight (32 columns each): three for the bf16 output, so the
-// shared columns (kOverlapChunks chunks) leave TMEM after one wait; two when the epilogue
-// also quantizes, which needs the registers.
-constexpr int kLdBufsPlain = 3;
-constexpr int kLdBufsQuant = 2;
-static_assert(kOverlapChunks <= kLdBufsPlain, "the shared columns must fit the first round of loads");
+// Epilogue chunk registers in flight (32 columns each): three, so the shared columns
+// (kOverlapChunks chunks) leave TMEM after one wait.
+constexpr int kLdBufs = 3;
+static_assert(kOverlapChunks <= kLdBufs, "the shared columns must fit the first round of loads");
+static_assert(BN / 32 >= 3, "the quantizing epilogue's ring holds three chunks");
 
 // Output of the epilogue: bf16 y = acc + bias; or the next layer's MX-quantized input,
 // h = bf16(GELU(bf16(acc + bias))) as E2M1 / E4M3 codes with tiled E8M0 scales (and h
@@ -129,6 +128,31 @@ struct Params {
 
 __device__ __forceinline__ void record_status(uint32_t code) { atomicCAS(&g_device_status, 0u, code); }
 
+// GELU(x) = x * Phi(x) = x/2 * erfc(-x / sqrt 2) in fp32 (the plain erf form).  erfc(z)
+// for z >= 0 by the Chebyshev-fitted formula of Numerical Recipes (2nd ed., section 6.2,
+// "erfcc"): erfc(z) = t * exp(-z^2 + P(t)), t = 1 / (1 + z/2), P of degree 9, fractional
+// error below 1.2e-7; the other side from erfc(-z) = 2 - erfc(z).  Relative accuracy
+// holds in the negative tail, where GELU is tiny (1 + erf would cancel there).  Below
+// x of about -13 the exponential underflows and the result is -0.
+__device__ __forceinline__ float gelu_f32(float x)
+{
+    const float z = fabsf(x) * 0.70710678118654752f;
+    const float t = __fdividef(1.0f, fmaf(0.5f, z, 1.0f));
+    float q = 0.17087277f;
+    q = fmaf(q, t, -0.82215223f);
+    q = fmaf(q, t, 1.48851587f);
+    q = fmaf(q, t, -1.13520398f);
+    q = fmaf(q, t, 0.27886807f);
+    q = fmaf(q, t, -0.18628806f);
+    q = fmaf(q, t, 0.09678418f);
+    q = fmaf(q, t, 0.37409196f);
+    q = fmaf(q, t, 1.00002368f);
+    q = fmaf(q, t, -1.26551223f);
+    const float e = t * __expf(fmaf(-z, z, q));  // erfc(z)
+    const float phi = x <= 0.0f ? 0.5f * e : fmaf(-0.5f, e, 1.0f);
+    return x * phi;
+}
+
 template <int kGroupM>
 __device__ __forceinline__ void tile_coords(int t, int m_blocks, int n_blocks, int& mb, int& nb)
 {
@@ -149,7 +173,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const Params p)
 {
     using C = Cfg<kPair, kOut>;
-    constexpr int kLdBufs = kOut ? kLdBufsQuant : kLdBufsPlain;
     constexpr int S = C::kStages;
     constexpr int AK = kW4A8 ? 1 : 2;  // scale atoms (128 K-elements each) per stage
 
@@ -405,26 +428,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             // a ring of kLdBufs chunk registers: the first kLdBufs loads go out back to back, so
             // the shared columns (kOverlapChunks <= kLdBufs chunks) are released after one wait
             uint32_t sfw0 = 0u, sfw1 = 0u;  // quantizing epilogue: this row's 8 scale bytes of the tile
-            uint32_t r[kLdBufs][32];
-#pragma unroll
-            for (int j = 0; j < kLdBufs; ++j) tmem_ld_x32(lanes + col0 + chunk_of(j) * 32, r[j]);
-            int issued = kLdBufs, landed_upto = 0;  // constants once the loop below is unrolled
-#pragma unroll
-            for (int ci = 0; ci < BN / 32; ++ci) {
-                if (ci >= landed_upto) {  // everything issued so far lands together
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int j = 0; j < BN / 32; ++j)
-                        if (j >= landed_upto && j < issued) {
-                            tmem_regs_ready(r[j % kLdBufs]);
-                            landed(j);
-                        }
-                    landed_upto = issued;
-                }
+            // one 32-column chunk (the ci-th in drain order) whose accumulators are in acc
+            auto process = [&](const uint32_t(&acc)[32], int ci) __attribute__((always_inline)) {
                 const int c = chunk_of(ci);
                 const int n = nb * BN + c * 32;
                 if (n < p.N) {  // warp-uniform
-                    const uint32_t* acc = r[ci % kLdBufs];
                     float bv[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) bv[i] = 0.f;
@@ -450,9 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         __nv_bfloat162 y2 = __floats2bfloat162_rn(__uint_as_float(acc[2 * i]) + bv[2 * i],
                                                                   __uint_as_float(acc[2 * i + 1]) + bv[2 * i + 1]);
                         if constexpr (kOut != kOutBf16) {
-                            // GELU(y) = y * Phi(y); normcdf keeps the negative tail accurate
                             const float y0 = __low2float(y2), y1 = __high2float(y2);
-                            y2 = __floats2bfloat162_rn(y0 * normcdff(y0), y1 * normcdff(y1));
+                            y2 = __floats2bfloat162_rn(gelu_f32(y0), gelu_f32(y1));
                         }
                         o[i] = *reinterpret_cast<uint32_t*>(&y2);
                     }
@@ -516,9 +523,62 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     eb ^= 1;
                 }
-                if (ci + kLdBufs < BN / 32) {  // refill the buffer just drained
-                    tmem_ld_x32(lanes + col0 + chunk_of(ci + kLdBufs) * 32, r[ci % kLdBufs]);
-                    issued = ci + kLdBufs + 1;
+            };
+            if constexpr (kOut == kOutBf16) {
+                // a ring of kLdBufs chunk registers, fully unrolled: the first kLdBufs loads go
+                // out back to back, so the shared columns are released after one wait
+                uint32_t r[kLdBufs][32];
+#pragma unroll
+                for (int j = 0; j < kLdBufs; ++j) tmem_ld_x32(lanes + col0 + chunk_of(j) * 32, r[j]);
+                int issued = kLdBufs, landed_upto = 0;  // constants once the loop below is unrolled
+#pragma unroll
+                for (int ci = 0; ci < BN / 32; ++ci) {
+                    if (ci >= landed_upto) {  // everything issued so far lands together
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int j = 0; j < BN / 32; ++j)
+                            if (j >= landed_upto && j < issued) {
+                                tmem_regs_ready(r[j % kLdBufs]);
+                                landed(j);
+                            }
+                        landed_upto = issued;
+                    }
+                    process(r[ci % kLdBufs], ci);
+                    if (ci + kLdBufs < BN / 32) {  // refill the buffer just drained
+                        tmem_ld_x32(lanes + col0 + chunk_of(ci + kLdBufs) * 32, r[ci % kLdBufs]);
+                        issued = ci + kLdBufs + 1;
+                    }
+                }
+            } else {
+                // The quantizing chunk body is long (GELU of 32 values); unrolled eight times
+                // it would not fit the instruction cache, so this loop stays rolled and the
+                // three-chunk ring (ra = chunk ci, rb = ci+1, rc = ci+2) advances by register
+                // moves.  Chunks 0-2 land before any work, which releases the shared columns.
+                uint32_t ra[32], rb[32], rc[32];
+                tmem_ld_x32(lanes + col0 + chunk_of(0) * 32, ra);
+                tmem_ld_x32(lanes + col0 + chunk_of(1) * 32, rb);
+                tmem_ld_x32(lanes + col0 + chunk_of(2) * 32, rc);
+                tmem_ld_wait();
+                tmem_regs_ready(ra);
+                tmem_regs_ready(rb);
+                tmem_regs_ready(rc);
+                landed(0);
+                landed(1);
+                landed(2);
+#pragma unroll 1
+                for (int ci = 0; ci < BN / 32; ++ci) {
+                    process(ra, ci);
+                    if (ci + 1 < BN / 32) {
+                        tmem_ld_wait();  // chunk ci+2, loaded during this chunk's work
+                        tmem_regs_ready(rc);
+                        if (ci >= 1 && ci + 2 < BN / 32) landed(ci + 2);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            ra[i] = rb[i];
+                            rb[i] = rc[i];
+                        }
+                        if (ci + 3 < BN / 32) tmem_ld_x32(lanes + col0 + chunk_of(ci + 3) * 32, rc);
+                    }
                 }
             }
             if constexpr (kOut != kOutBf16) {
