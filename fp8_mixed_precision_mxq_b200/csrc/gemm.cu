@@ -55,8 +55,14 @@ __device__ uint32_t g_device_status;
 namespace {
 
 constexpr int BN = 256;                   // output columns per tile (both variants): 256 or 192
-constexpr int kEpiWarps = 4;
-constexpr int kThreads = 64 + 32 * kEpiWarps + 32;  // + one scale-copy warp
+// Warp roles: 0 TMA producer, 1 MMA issuer, then the epilogue warps, then one scale-copy
+// warp.  The bf16 epilogue has four warps, one per TMEM lane quarter; the quantizing
+// epilogue eight, two per lane quarter taking alternate chunks, so that its GELU
+// arithmetic has twice the warps to hide latency with.
+template <int kOut>
+constexpr int kEpiWarpsOf = kOut ? 8 : 4;
+template <int kOut>
+constexpr int kThreadsOf = 64 + 32 * kEpiWarpsOf<kOut> + 32;
 constexpr uint32_t kEpiBuf = 32 * 64;     // 32 rows x 32 bf16
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: accumulator slot 0 [0, BN), slot 1 [kAccCol1, kAccCol1 + BN) (sharing
@@ -104,6 +110,7 @@ struct Cfg {
     static constexpr uint32_t kOffSFB = kOffSFA + kStages * kStageSFA;
     static constexpr uint32_t kOffEpi = kOffSFB + kStages * kStageSFB;
     static constexpr uint32_t kQBuf = kOut == kOutGeluE4M3 ? 32 * 32 : 32 * 16;  // 32 rows of one block's codes
+    static constexpr int kEpiWarps = kEpiWarpsOf<kOut>;
     static constexpr uint32_t kOffQ = kOffEpi + kEpiWarps * 2 * kEpiBuf;
     static constexpr uint32_t kOffBar = kOffQ + (kOut ? kEpiWarps * 2 * kQBuf : 0u);
     static constexpr uint32_t kNumBars = 2 * kStages + 6 + 2 * 3;
@@ -166,7 +173,7 @@ __device__ __forceinline__ void tile_coords(int t, int m_blocks, int n_blocks, i
 }
 
 template <bool kW4A8, int kPair, int kOut>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                    const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                    const __grid_constant__ CUtensorMap map_y, const __grid_constant__ CUtensorMap map_q,
@@ -174,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     using C = Cfg<kPair, kOut>;
     constexpr int S = C::kStages;
+    constexpr int kEpiWarps = C::kEpiWarps;
     constexpr int AK = kW4A8 ? 1 : 2;  // scale atoms (128 K-elements each) per stage
 
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -417,20 +425,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto chunk_of = [&](int ci) {
                 return slot ? ci : (ci < kOverlapChunks ? BN / 32 - kOverlapChunks + ci : ci - kOverlapChunks);
             };
-            // after the load of chunk ci has landed: release what the MMA issuer waits for
-            auto landed = [&](int ci) {
-                if (ci == kOverlapChunks - 1 || ci == BN / 32 - 1) {
+            // after the loads of this warp's chunks up to drain index ci have landed:
+            // release what the MMA issuer waits for (every epilogue warp arrives on both)
+            auto landed = [&](int ci, int last_shared, int last) {
+                if (ci == last_shared || ci == last) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(ci == BN / 32 - 1 ? tmem_empty_bar : bar_overlap);
+                    if (lane == 0) mbar_arrive_cluster(ci == last ? tmem_empty_bar : bar_overlap);
                 }
             };
             // a ring of kLdBufs chunk registers: the first kLdBufs loads go out back to back, so
             // the shared columns (kOverlapChunks <= kLdBufs chunks) are released after one wait
-            uint32_t sfw0 = 0u, sfw1 = 0u;  // quantizing epilogue: this row's 8 scale bytes of the tile
             // one 32-column chunk (the ci-th in drain order) whose accumulators are in acc
             auto process = [&](const uint32_t(&acc)[32], int ci) __attribute__((always_inline)) {
                 const int c = chunk_of(ci);
+                uint32_t sc_byte = 0u;  // quantizing epilogue: the chunk's E8M0 scale
                 const int n = nb * BN + c * 32;
                 if (n < p.N) {  // warp-uniform
                     float bv[32];
@@ -508,9 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<uint4*>(qb + lane * 32) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
                             *reinterpret_cast<uint4*>(qb + lane * 32 + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
                         }
-                        // scale byte of k-block c of this tile: byte c%4 of word c/4
-                        if (c < 4) sfw0 |= sc << (8 * (c & 3));
-                        else sfw1 |= sc << (8 * (c & 3));
+                        sc_byte = sc;
                     }
                     fence_async_smem();
                     __syncwarp();
@@ -522,6 +529,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         bulk_commit();
                     }
                     eb ^= 1;
+                }
+                if constexpr (kOut != kOutBf16) {
+                    // this row's scale byte of k-block nb*8 + c, straight into the tiled
+                    // layout; rows between M and the 128-row padding, and k-blocks past N
+                    // inside the padding, get 0 as the layout requires
+                    const int row = row0 + lane;
+                    const uint32_t kb = static_cast<uint32_t>(nb) * 8u + static_cast<uint32_t>(c);
+                    if (row < p.q_rows_pad && kb < 4u * p.q_atoms_k) {
+                        const size_t off = (static_cast<size_t>(row >> 7) * p.q_atoms_k + (kb >> 2)) * 512u +
+                                           (row & 31) * 16u + ((row >> 5) & 3) * 4u + (kb & 3u);
+                        p.q_sf[off] = row < p.M ? static_cast<uint8_t>(sc_byte) : uint8_t(0);
+                    }
                 }
             };
             if constexpr (kOut == kOutBf16) {
@@ -539,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int j = 0; j < BN / 32; ++j)
                             if (j >= landed_upto && j < issued) {
                                 tmem_regs_ready(r[j % kLdBufs]);
-                                landed(j);
+                                landed(j, kOverlapChunks - 1, BN / 32 - 1);
                             }
                         landed_upto = issued;
                     }
@@ -550,52 +569,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else {
-                // The quantizing chunk body is long (GELU of 32 values); unrolled eight times
-                // it would not fit the instruction cache, so this loop stays rolled and the
-                // three-chunk ring (ra = chunk ci, rb = ci+1, rc = ci+2) advances by register
-                // moves.  Chunks 0-2 land before any work, which releases the shared columns.
-                uint32_t ra[32], rb[32], rc[32];
-                tmem_ld_x32(lanes + col0 + chunk_of(0) * 32, ra);
-                tmem_ld_x32(lanes + col0 + chunk_of(1) * 32, rb);
-                tmem_ld_x32(lanes + col0 + chunk_of(2) * 32, rc);
+                // Two warps per lane quarter take alternate chunks of the drain order (the
+                // first group, warps 2-5, even ones; warps 6-9 odd ones), so the three shared
+                // chunks split 2 + 1 and each warp frees them after its first two loads.  The
+                // chunk body is long (GELU of 32 values), so the loop stays rolled, with a
+                // two-chunk register ring advanced by moves.
+                static_assert(BN / 32 == 8 && kOverlapChunks == 3 && C::kEpiWarps == 8, "chunk split");
+                const int grp = ew >> 2;
+                constexpr int kMine = 4;
+                const int last_shared = grp == 0 ? 1 : 0;  // local index of its last shared chunk
+                uint32_t ra[32], rb[32];
+                tmem_ld_x32(lanes + col0 + chunk_of(grp) * 32, ra);
+                tmem_ld_x32(lanes + col0 + chunk_of(grp + 2) * 32, rb);
                 tmem_ld_wait();
                 tmem_regs_ready(ra);
                 tmem_regs_ready(rb);
-                tmem_regs_ready(rc);
-                landed(0);
-                landed(1);
-                landed(2);
+                landed(0, last_shared, kMine - 1);
+                landed(1, last_shared, kMine - 1);
 #pragma unroll 1
-                for (int ci = 0; ci < BN / 32; ++ci) {
-                    process(ra, ci);
-                    if (ci + 1 < BN / 32) {
-                        tmem_ld_wait();  // chunk ci+2, loaded during this chunk's work
-                        tmem_regs_ready(rc);
-                        if (ci >= 1 && ci + 2 < BN / 32) landed(ci + 2);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            ra[i] = rb[i];
-                            rb[i] = rc[i];
+                for (int i = 0; i < kMine; ++i) {
+                    process(ra, grp + 2 * i);
+                    if (i + 1 < kMine) {
+                        if (i >= 1) {  // chunk i+1, loaded during this chunk's work
+                            tmem_ld_wait();
+                            tmem_regs_ready(rb);
+                            landed(i + 1, last_shared, kMine - 1);
                         }
-                        if (ci + 3 < BN / 32) tmem_ld_x32(lanes + col0 + chunk_of(ci + 3) * 32, rc);
-                    }
-                }
-            }
-            if constexpr (kOut != kOutBf16) {
-                // the row's scale bytes of this tile's 8 k-blocks: two 32-bit words of the
-                // tiled layout (k-blocks 4g..4g+3 of one row are 4 consecutive bytes).  Rows
-                // between M and the 128-row padding, and k-blocks past N inside the padding,
-                // get 0, as the layout requires.
-                const int row = row0 + lane;
-                if (row < p.q_rows_pad) {
 #pragma unroll
-                    for (int g = 0; g < 2; ++g) {
-                        const uint32_t kb0 = static_cast<uint32_t>(nb) * 8u + 4u * g;
-                        if (kb0 < 4u * p.q_atoms_k) {
-                            const size_t off = (static_cast<size_t>(row >> 7) * p.q_atoms_k + (kb0 >> 2)) * 512u +
-                                               (row & 31) * 16u + ((row >> 5) & 3) * 4u;
-                            *reinterpret_cast<uint32_t*>(p.q_sf + off) = row < p.M ? (g ? sfw1 : sfw0) : 0u;
-                        }
+                        for (int k = 0; k < 32; ++k) ra[k] = rb[k];
+                        if (i + 2 < kMine) tmem_ld_x32(lanes + col0 + chunk_of(grp + 2 * (i + 2)) * 32, rb);
                     }
                 }
             }
@@ -669,7 +671,7 @@ cudaError_t launch_variant(const CUtensorMap& ma, const CUtensorMap& mb, const C
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(kThreadsOf<kOut>, 1, 1);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
