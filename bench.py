@@ -55,8 +55,8 @@ GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precisio
                 "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h"]
 GEMM_TRAFFIC = {
     ("ffn_up_480p_w4a4", 32760): {
-        "bytes": 542322944 + 860596480,
-        "sources_sha256": "47d069a7afec31613132083a51abcc337e124ad9ffd4ab5d689f421516cee05a",
+        "bytes": 573767936 + 859632896,
+        "sources_sha256": "2be218dbd825847859b1dbf0a0838b1dbaf4a6fe73c8679a351b9ba01e7981b3",
         "profile": "profiles/mx_gemm_mxf4_pair_ffn_up_480p_traffic.md"},
 }
 
