@@ -76,6 +76,12 @@ def lib():
         L.mxo_round_bf16.restype = None
         L.mxo_gelu_bf16.argtypes = [vp, i64, vp]
         L.mxo_gelu_bf16.restype = None
+        L.mxo_static_inverse.argtypes = [ctypes.c_float]
+        L.mxo_static_inverse.restype = ctypes.c_float
+        L.mxo_quantize_static_e4m3.argtypes = [vp, i64, ctypes.c_float, vp]
+        L.mxo_quantize_static_e4m3.restype = i32
+        L.mxo_linear_rows_scaled.argtypes = [vp, vp, i32, vp, i64, i64, vp, vp, i64, vp, dbl, vp, i32]
+        L.mxo_linear_rows_scaled.restype = i32
     return _lib
 
 
@@ -213,3 +219,38 @@ def ffn_hidden_rows(a_codes, a_sf, a_fmt, rows, K, w1_codes, w1_sf, b1_bits, h_f
     h = gelu_bf16(round_bf16(y))
     codes, sf = quantize(h, h_fmt, nthreads)
     return h, codes, sf
+
+
+def static_inverse(scale: float) -> float:
+    """fl32(1 / scale): the multiplier the static quantizer applies."""
+    return float(lib().mxo_static_inverse(float(scale)))
+
+
+def quantize_static_e4m3(x_bits: np.ndarray, scale: float) -> np.ndarray:
+    """Static per-tensor E4M3 codes of bf16 bits x (same shape, uint8)."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    codes = np.empty(x_bits.shape, dtype=np.uint8)
+    lib().mxo_quantize_static_e4m3(_ptr(x_bits), x_bits.size, static_inverse(scale), _ptr(codes))
+    return codes
+
+
+def linear_rows_scaled(a_codes, a_sf, a_fmt, rows, K, w_codes, w_sf, alpha, bias_bits=None,
+                       nthreads: int | None = None) -> np.ndarray:
+    """fp64 Y[rows, :] = alpha * deq(A)[rows] . deq(W)^T (+ bias)."""
+    a_codes = np.ascontiguousarray(a_codes, dtype=np.uint8)
+    a_sf = np.ascontiguousarray(a_sf, dtype=np.uint8)
+    w_codes = np.ascontiguousarray(w_codes, dtype=np.uint8)
+    w_sf = np.ascontiguousarray(w_sf, dtype=np.uint8)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    N = w_codes.shape[0]
+    y = np.zeros((rows.shape[0], N), dtype=np.float64)
+    bias_p = None
+    if bias_bits is not None:
+        bias_bits = np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        bias_p = _ptr(bias_bits)
+    rc = lib().mxo_linear_rows_scaled(_ptr(a_codes), _ptr(a_sf), a_fmt, _ptr(rows), rows.shape[0], K,
+                                      _ptr(w_codes), _ptr(w_sf), N, bias_p, float(alpha), _ptr(y),
+                                      nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle scaled linear failed (rc=%d)" % rc)
+    return y

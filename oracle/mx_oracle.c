@@ -413,3 +413,39 @@ void mxo_gelu_bf16(const uint16_t *y, int64_t n, uint16_t *h)
 {
     for (int64_t i = 0; i < n; ++i) h[i] = mxo_double_to_bf16(mxo_gelu(mxo_bf16_to_double(y[i])));
 }
+
+/* ---- static per-tensor E4M3 activations ------------------------------------------- */
+
+/* The W4A8 of the blog's "Quantization formats" table names "FP8 E4M3 static
+ * activations": one scale s for the whole tensor, fixed offline (calibration: s = amax /
+ * 448, the largest E4M3 magnitude).  Each element becomes RNE_sat(x * r) on the E4M3
+ * grid with r = fl32(1/s), the product taken in binary32 -- the precision in which the
+ * kernel takes the same decision.  The block scales the MMA reads are all 127 (x1) and
+ * the linear layer multiplies its sums by s. */
+float mxo_static_inverse(float s) { return (float)(1.0 / (double)s); }
+
+int mxo_quantize_static_e4m3(const uint16_t *x, int64_t n, float inv_scale, uint8_t *codes)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        /* exact double product of a bf16 and a binary32 value, rounded once to binary32 */
+        float p = (float)(mxo_bf16_to_double(x[i]) * (double)inv_scale);
+        if (isnan(p)) codes[i] = (uint8_t)((signbit(p) ? 0x80 : 0x00) | 0x7F);
+        else codes[i] = (uint8_t)mxo_encode_elem((double)p, MXO_E4M3);
+    }
+    return 0;
+}
+
+/* y[i, n] = alpha * sum_k deqA[rows[i], k] * deqW[n, k] + bias[n] in fp64: the linear layer
+ * whose activation carries a per-tensor scale alpha on top of its block scales. */
+int mxo_linear_rows_scaled(const uint8_t *a_codes, const uint8_t *a_sf, int a_fmt,
+                           const int64_t *rows, int64_t nrows, int64_t K,
+                           const uint8_t *w_codes, const uint8_t *w_sf, int64_t N,
+                           const uint16_t *bias, double alpha, double *y, int nthreads)
+{
+    int rc = mxo_linear_rows(a_codes, a_sf, a_fmt, rows, nrows, K, w_codes, w_sf, N, NULL, y, nthreads);
+    if (rc != 0) return rc;
+    for (int64_t i = 0; i < nrows; ++i)
+        for (int64_t j = 0; j < N; ++j)
+            y[i * N + j] = alpha * y[i * N + j] + (bias ? mxo_bf16_to_double(bias[j]) : 0.0);
+    return 0;
+}

@@ -40,6 +40,12 @@ MUTANTS = [
     ("gelu_without_sqrt2", "erfc(-x / sqrt(2.0));", "erfc(-x);"),
     ("gelu_tanh_form", "double mxo_gelu(double x) { return 0.5 * x * erfc(-x / sqrt(2.0)); }",
      "double mxo_gelu(double x) { return 0.5 * x * (1.0 + tanh(sqrt(2.0 / M_PI) * (x + 0.044715 * x * x * x))); }"),
+    ("static_scale_dropped", "y[i * N + j] = alpha * y[i * N + j] + (bias",
+     "y[i * N + j] = y[i * N + j] + (bias"),
+    ("static_bias_scaled", "y[i * N + j] = alpha * y[i * N + j] + (bias ? mxo_bf16_to_double(bias[j]) : 0.0);",
+     "y[i * N + j] = alpha * (y[i * N + j] + (bias ? mxo_bf16_to_double(bias[j]) : 0.0));"),
+    ("static_divides_in_double", "float p = (float)(mxo_bf16_to_double(x[i]) * (double)inv_scale);",
+     "float p = (float)(mxo_bf16_to_double(x[i]) * (double)inv_scale * 1.0000001);"),
     ("gelu_cancelling_form", "double mxo_gelu(double x) { return 0.5 * x * erfc(-x / sqrt(2.0)); }",
      "double mxo_gelu(double x) { return 0.5 * x * (1.0 + erf(x / sqrt(2.0))); }"),
 ]

@@ -450,3 +450,58 @@ def test_gelu_bf16_hand_values():
     h = oracle.gelu_bf16(y)
     assert [hex(v) for v in h[:3]] == ["0x3f57", "0xbe22", "0x3ffa"]
     assert h[3] == 0x0000 and h[4] in (0x0000, 0x8000)  # GELU(-0) = -0 * 1/2
+
+
+# --- static per-tensor E4M3 activations -------------------------------------------------------
+#
+# codes = RNE_sat(fl32(x * fl32(1/s))) on the E4M3 grid; the linear multiplies its sums by s.
+
+def test_static_inverse_is_the_binary32_reciprocal():
+    for s in (0.5, 3.0, 0.0371, 1e-3, 448.0, 7.25e-5):
+        assert oracle.static_inverse(s) == float(np.float32(1.0) / np.float32(s))
+
+
+@pytest.mark.parametrize("scale", [0.5, 0.0371, 2.0 ** -7 * 3, 11.0])
+def test_static_e4m3_is_nearest_grid_point_of_the_binary32_product(scale):
+    """Each code is the brute-force nearest E4M3 value (ties to even, saturating) of the
+    binary32 product x * fl32(1/s), computed here with numpy's float32 arithmetic."""
+    rng = np.random.default_rng(int(scale * 1000) + 3)
+    x = (rng.standard_normal(4000) * scale * rng.choice([1.0, 30.0, 300.0, 1e-3], size=4000)).astype(np.float32)
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)          # truncate to bf16 (any bf16 will do)
+    xb = (bits.astype(np.uint32) << 16).view(np.float32)
+    p = xb * (np.float32(1.0) / np.float32(scale))                # binary32 multiply
+    got = oracle.quantize_static_e4m3(bits, scale)
+    for xi, pi, c in zip(xb, p, got):
+        assert c == brute_round(float(pi), oracle.E4M3), (float(xi), float(pi), hex(c))
+
+
+def test_static_e4m3_exact_multiples_saturation_and_sign():
+    s = 2.0 ** -3  # x = q * s is exact for every E4M3 value q, and so is x / s
+    qs = [oracle.decode_elem(c, oracle.E4M3) for c in range(0x7F)]  # every non-negative finite code
+    xb = np.array([oracle.double_to_bf16(q * s) for q in qs], dtype=np.uint16)
+    assert list(oracle.quantize_static_e4m3(xb, s)) == list(range(0x7F))
+    big = np.array([oracle.double_to_bf16(v) for v in (449 * s, 1e4 * s, -1e4 * s, -1e-9, 1e-9)], dtype=np.uint16)
+    assert [hex(c) for c in oracle.quantize_static_e4m3(big, s)] == ["0x7e", "0x7e", "0xfe", "0x80", "0x0"]
+
+
+def test_linear_scaled_brute_force_exact():
+    """alpha * sum_k deq(a) * deq(w) + bias, checked with exact rationals."""
+    rng = np.random.default_rng(21)
+    M, N, K = 3, 4, 64
+    a_codes = rng.integers(0, 256, size=(M, K), dtype=np.uint8)
+    a_codes[(a_codes & 0x7F) == 0x7F] = 0x11  # no NaN codes
+    a_sf = np.full((M, K // 32), 127, dtype=np.uint8)
+    w_codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    w_sf = rng.integers(120, 135, size=(N, K // 32), dtype=np.uint8)
+    bias = np.array([oracle.double_to_bf16(v) for v in (0.5, -1.25, 3.0, 0.0)], dtype=np.uint16)
+    alpha = 0.1234567
+    y = oracle.linear_rows_scaled(a_codes, a_sf, oracle.E4M3, np.arange(M), K, w_codes, w_sf, alpha, bias)
+    for m in range(M):
+        for n in range(N):
+            acc = Fraction(0)
+            for k in range(K):
+                wc = (int(w_codes[n, k // 2]) >> (4 * (k & 1))) & 0xF
+                acc += (Fraction(oracle.decode_elem(int(a_codes[m, k]), oracle.E4M3)) *
+                        Fraction(oracle.decode_elem(wc, oracle.E2M1)) * Fraction(2) ** (int(w_sf[n, k // 32]) - 127))
+            want = Fraction(alpha) * acc + Fraction(oracle.bf16_to_float(int(bias[n])))
+            assert abs(Fraction(y[m, n]) - want) <= abs(want) * Fraction(1, 10 ** 14) + Fraction(1, 10 ** 300)
