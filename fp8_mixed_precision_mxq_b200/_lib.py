@@ -52,6 +52,9 @@ SIGNATURES = {
     "mxq_ffn": ([_vp, _i64, _i64, ctypes.POINTER(WDesc), ctypes.POINTER(WDesc), _i32, _i32, _vp, _i64, _vp, _vp],
                 _i32),
     "mxq_ffn_workspace_bytes": ([_i64, _i64, _i64, _i32, _i32], _i64),
+    "mxq_quantize_act_static": ([_vp, _i64, _i64, ctypes.c_float, _vp, _vp, _vp], _i32),
+    "mxq_linear_static": ([_vp, _i64, _i64, _vp, _vp, _i64, _vp, ctypes.c_float, _vp, _i64, _vp, _vp], _i32),
+    "mxq_absmax": ([_vp, _i64, _vp, _vp], _i32),
     "mxq_sf_to_logical": ([_vp, _i64, _i64, _vp, _vp], _i32),
     "mxq_poll_status": ([_vp], _i32),
     "mxq_set_debug": ([_u32], _i32),

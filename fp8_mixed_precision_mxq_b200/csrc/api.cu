@@ -1,6 +1,7 @@
 // api.cu -- the C ABI of libmxq.so (declared in include/mxq.h): argument checks,
 // workspace layout, and dispatch to the quantizer, dequantizer and GEMM kernels.
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -154,6 +155,10 @@ int run_linear(const void* x, int64_t M, int64_t K, const void* w_codes, const v
     snprintf(g_path, sizeof g_path, "qdq %s dequant + cublasLt bf16", fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1");
     return ok();
 }
+
+// fl32(1/s): the reciprocal the static quantizer multiplies by (an IEEE double division
+// rounded to binary32, which equals the correctly rounded binary32 division).
+float static_inverse(float s) { return static_cast<float>(1.0 / static_cast<double>(s)); }
 
 int check_mode(int mode)
 {
@@ -370,6 +375,58 @@ int mxq_ffn(const void* x_bf16, int64_t M, int64_t K, const mxq_wdesc* up, const
     snprintf(g_path, sizeof g_path, "ffn %s -> gelu -> %s fused", up_fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1",
              down_fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1");
     return ok();
+}
+
+int mxq_quantize_act_static(const void* x_bf16, int64_t M, int64_t K, float scale, void* codes, void* sf,
+                            void* stream)
+{
+    if (!(scale > 0.0f) || !std::isfinite(scale))
+        return fail(MXQ_ERR_INVALID_ARG, "static scale must be positive and finite (got %g)", (double)scale);
+    RETURN_IF(check_rows_k(M, K, "quantize_static"));
+    RETURN_IF(check_ptr(x_bf16, "x"));
+    RETURN_IF(check_ptr(codes, "codes"));
+    RETURN_IF(check_ptr(sf, "sf"));
+    RETURN_IF(check_device());
+    snprintf(g_path, sizeof g_path, "quantize static e4m3");
+    return cuda_rc(launch_quantize_static(x_bf16, M, K, static_inverse(scale), codes, sf,
+                                          static_cast<cudaStream_t>(stream)),
+                   "quantize launch");
+}
+
+int mxq_linear_static(const void* x_bf16, int64_t M, int64_t K, const void* w_codes, const void* w_sf, int64_t N,
+                      const void* bias_bf16, float act_scale, void* workspace, int64_t ws_bytes, void* y_bf16,
+                      void* stream)
+{
+    if (!(act_scale > 0.0f) || !std::isfinite(act_scale))
+        return fail(MXQ_ERR_INVALID_ARG, "static scale must be positive and finite (got %g)", (double)act_scale);
+    RETURN_IF(check_ptr(x_bf16, "x"));
+    RETURN_IF(check_ptr(workspace, "workspace", kWsAlign));
+    RETURN_IF(check_gemm(workspace, workspace, MXQ_FMT_E4M3, M, K, w_codes, w_sf, N, bias_bf16, y_bf16));
+    const int64_t need = linear_ws(M, N, K, MXQ_FMT_E4M3, MXQ_MODE_NATIVE);
+    if (ws_bytes < need)
+        return fail(MXQ_ERR_WORKSPACE, "workspace has %lld bytes, needs %lld", (long long)ws_bytes, (long long)need);
+    RETURN_IF(check_device());
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* xc = static_cast<uint8_t*>(workspace);
+    uint8_t* xs = xc + round_up(codes_bytes(M, K, MXQ_FMT_E4M3), kWsAlign);
+    RETURN_IF(cuda_rc(launch_quantize_static(x_bf16, M, K, static_inverse(act_scale), xc, xs, st), "quantize launch"));
+    GemmArgs g{xc, xs, MXQ_FMT_E4M3, M, N, K, w_codes, w_sf, bias_bf16, y_bf16};
+    g.alpha = act_scale;
+    const char* msg = nullptr;
+    int rc = launch_gemm(g, st, &msg, g_path, sizeof g_path);
+    if (rc != MXQ_OK) return fail(rc, "gemm: %s", msg ? msg : "launch failed");
+    snprintf(g_path + strlen(g_path), sizeof g_path - strlen(g_path), " static-scale");
+    return ok();
+}
+
+int mxq_absmax(const void* x_bf16, int64_t n, void* out_f32, void* stream)
+{
+    if (n <= 0 || n % 8 != 0) return fail(MXQ_ERR_SHAPE, "absmax: n=%lld must be a positive multiple of 8", (long long)n);
+    RETURN_IF(check_ptr(x_bf16, "x"));
+    RETURN_IF(check_ptr(out_f32, "out", 4));
+    RETURN_IF(check_device());
+    return cuda_rc(launch_absmax(x_bf16, n, static_cast<float*>(out_f32), static_cast<cudaStream_t>(stream)),
+                   "absmax launch");
 }
 
 int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_rowmajor, void* stream)

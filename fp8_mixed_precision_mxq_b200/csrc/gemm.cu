@@ -131,6 +131,7 @@ struct Params {
     uint32_t q_atoms_k;
     int q_rows_pad;
     int write_h;
+    float alpha;  // per-tensor activation scale applied to the sums (1 for MX activations)
 };
 
 __device__ __forceinline__ void record_status(uint32_t code) { atomicCAS(&g_device_status, 0u, code); }
@@ -464,8 +465,9 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                     uint32_t o[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 y2 = __floats2bfloat162_rn(__uint_as_float(acc[2 * i]) + bv[2 * i],
-                                                                  __uint_as_float(acc[2 * i + 1]) + bv[2 * i + 1]);
+                        __nv_bfloat162 y2 = __floats2bfloat162_rn(fmaf(__uint_as_float(acc[2 * i]), p.alpha, bv[2 * i]),
+                                                                  fmaf(__uint_as_float(acc[2 * i + 1]), p.alpha,
+                                                                       bv[2 * i + 1]));
                         if constexpr (kOut != kOutBf16) {
                             const float y0 = __low2float(y2), y1 = __high2float(y2);
                             y2 = __floats2bfloat162_rn(gelu_f32(y0), gelu_f32(y1));
@@ -750,6 +752,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     p.q_atoms_k = quant_out ? static_cast<uint32_t>(sf_atoms_k(g.N)) : 0u;
     p.q_rows_pad = static_cast<int>(ceil_div(g.M, 128) * 128);
     p.write_h = quant_out && g.y != nullptr ? 1 : 0;
+    p.alpha = g.alpha;
     const int out = !quant_out ? kOutBf16 : (g.out_fmt == kFmtE4M3 ? kOutGeluE4M3 : kOutGeluE2M1);
 
     int dev = 0, sms = 148;

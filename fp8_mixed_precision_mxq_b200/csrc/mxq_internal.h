@@ -22,6 +22,11 @@ inline int64_t codes_bytes(int64_t rows, int64_t K, int fmt) { return fmt == kFm
 // ---- launchers (return cudaError_t of the launch) ----
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, int fmt, void* codes, void* sf,
                             cudaStream_t stream);
+// Static per-tensor E4M3: codes = RNE_sat(x * inv_scale), block scales 127.
+cudaError_t launch_quantize_static(const void* x, int64_t rows, int64_t K, float inv_scale, void* codes, void* sf,
+                                   cudaStream_t stream);
+// *out = max |x| over n bf16 values (n % 8 == 0), as fp32.
+cudaError_t launch_absmax(const void* x, int64_t n, float* out, cudaStream_t stream);
 cudaError_t launch_dequantize(const void* codes, const void* sf, int64_t rows, int64_t K, int fmt, void* out,
                               cudaStream_t stream);
 cudaError_t launch_sf_to_logical(const void* sf, int64_t rows, int64_t K, void* out, cudaStream_t stream);
@@ -40,6 +45,8 @@ struct GemmArgs {
     int out_fmt = -1;
     void* q_codes = nullptr;
     void* q_sf = nullptr;
+    // per-tensor scale of the activation (static E4M3): y = alpha * acc + bias
+    float alpha = 1.0f;
 };
 
 // Builds the tensor maps and launches the tcgen05 GEMM.  Returns an mxq_status;

@@ -38,13 +38,20 @@ __device__ __forceinline__ uint32_t sf_offset(uint32_t r, uint32_t kb, uint32_t 
     return ((r >> 7) * atoms_k + (kb >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + (kb & 3u);
 }
 
+// Static per-tensor E4M3 (the format template argument kFmtStatic): every element is
+// multiplied by the tensor's fp32 inverse scale and rounded onto the E4M3 grid; the
+// block scales are all 127 (x1) and the GEMM applies the tensor scale to its sums.
+constexpr int kFmtStatic = 2;
+
 template <int FMT>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restrict__ x, uint32_t n_groups,
                                                             uint32_t KB, uint64_t kb_magic, uint32_t atoms_k,
                                                             uint32_t rows, uint8_t* __restrict__ codes,
-                                                            uint8_t* __restrict__ sf)
+                                                            uint8_t* __restrict__ sf, float static_inv)
 {
-    constexpr uint32_t kEmax = FMT == kFmtE4M3 ? 8u : 2u;
+    constexpr bool kStatic = FMT == kFmtStatic;
+    constexpr int kElem = kStatic ? kFmtE4M3 : FMT;
+    constexpr uint32_t kEmax = kElem == kFmtE4M3 ? 8u : 2u;
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t nwarps = gridDim.x * (kThreads / 32);
     const uint32_t warp = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
@@ -59,20 +66,28 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            // block absmax over the quad of lanes holding the 32 elements
-            uint32_t m2 = absmax_bf16x2(absmax_bf16x2(v[u].x, v[u].y), absmax_bf16x2(v[u].z, v[u].w));
-            m2 = absmax_bf16x2(m2, __byte_perm(m2, 0, 0x1032));
-            uint32_t amax = m2 & 0x7FFFu;
-            amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-            amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-            if (g[u] >= n_groups) continue;
-            const uint32_t eb = amax >> 7;  // biased exponent of amax (bf16 and E8M0 share bias 127)
-            const uint32_t sc = eb == 255u ? 255u : (eb > kEmax ? eb - kEmax : 0u);
-            const float inv = __uint_as_float((254u - min(sc, 253u)) << 23);  // 2^(127 - sc)
+            uint32_t sc;
+            float inv;
+            if constexpr (kStatic) {
+                if (g[u] >= n_groups) continue;
+                sc = 127u;
+                inv = static_inv;
+            } else {
+                // block absmax over the quad of lanes holding the 32 elements
+                uint32_t m2 = absmax_bf16x2(absmax_bf16x2(v[u].x, v[u].y), absmax_bf16x2(v[u].z, v[u].w));
+                m2 = absmax_bf16x2(m2, __byte_perm(m2, 0, 0x1032));
+                uint32_t amax = m2 & 0x7FFFu;
+                amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+                amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+                if (g[u] >= n_groups) continue;
+                const uint32_t eb = amax >> 7;  // biased exponent of amax (bf16 and E8M0 share bias 127)
+                sc = eb == 255u ? 255u : (eb > kEmax ? eb - kEmax : 0u);
+                inv = __uint_as_float((254u - min(sc, 253u)) << 23);  // 2^(127 - sc)
+            }
             const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
             // cvt rounds to nearest even, saturates, and keeps the sign of a value that
             // rounds to zero (-0 = 0x8 / 0x80), as the format reading requires
-            if (FMT == kFmtE2M1) {
+            if (kElem == kFmtE2M1) {
                 uint32_t out = 0;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) out |= cvt_e2m1x2(lo_f(w[i]) * inv, hi_f(w[i]) * inv) << (8 * i);
@@ -197,8 +212,10 @@ int num_sms()
 
 }  // namespace
 
-cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, int fmt, void* codes, void* sf,
-                            cudaStream_t stream)
+// fmt: kFmtE2M1 / kFmtE4M3 (MX, scales from each block's abs-max) or kFmtStatic (E4M3
+// with the fixed inverse scale static_inv and block scales 127).
+cudaError_t launch_quantize_any(const void* x, int64_t rows, int64_t K, int fmt, float static_inv, void* codes,
+                                void* sf, cudaStream_t stream)
 {
     const uint32_t n_groups = static_cast<uint32_t>(rows * K / 8);
     const uint32_t KB = static_cast<uint32_t>(K / 32);
@@ -206,22 +223,35 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, int fmt, voi
     const int64_t want = ceil_div(n_groups, kThreads * kUnroll);
     // blocks per SM (measured on B200: E4M3, with twice the bytes written per element,
     // gains from a second round of blocks queued behind the resident ones)
-    const int per_sm = fmt == kFmtE4M3 ? 16 : 8;
+    const int per_sm = fmt == kFmtE2M1 ? 8 : 16;
     const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * per_sm)));
     // row = floor(block / KB) as a multiply-shift, exact for block < 2^29 and KB <= 2^11:
     // magic * KB - 2^40 < KB, so block * magic / 2^40 overshoots block / KB by less than 1 / KB
     const uint64_t kb_magic = ((uint64_t(1) << 40) + KB - 1) / KB;
-    if (fmt == kFmtE4M3)
-        quantize_kernel<kFmtE4M3><<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(x), n_groups, KB,
-                                                                 kb_magic, atoms_k, static_cast<uint32_t>(rows),
-                                                                 static_cast<uint8_t*>(codes),
-                                                                 static_cast<uint8_t*>(sf));
+    const uint4* xv = static_cast<const uint4*>(x);
+    uint8_t* c = static_cast<uint8_t*>(codes);
+    uint8_t* f = static_cast<uint8_t*>(sf);
+    const uint32_t r = static_cast<uint32_t>(rows);
+    if (fmt == kFmtStatic)
+        quantize_kernel<kFmtStatic><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k, r, c, f,
+                                                                   static_inv);
+    else if (fmt == kFmtE4M3)
+        quantize_kernel<kFmtE4M3><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k, r, c, f, 0.f);
     else
-        quantize_kernel<kFmtE2M1><<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(x), n_groups, KB,
-                                                                 kb_magic, atoms_k, static_cast<uint32_t>(rows),
-                                                                 static_cast<uint8_t*>(codes),
-                                                                 static_cast<uint8_t*>(sf));
+        quantize_kernel<kFmtE2M1><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k, r, c, f, 0.f);
     return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, int fmt, void* codes, void* sf,
+                            cudaStream_t stream)
+{
+    return launch_quantize_any(x, rows, K, fmt, 0.f, codes, sf, stream);
+}
+
+cudaError_t launch_quantize_static(const void* x, int64_t rows, int64_t K, float inv_scale, void* codes, void* sf,
+                                   cudaStream_t stream)
+{
+    return launch_quantize_any(x, rows, K, kFmtStatic, inv_scale, codes, sf, stream);
 }
 
 cudaError_t launch_dequantize(const void* codes, const void* sf, int64_t rows, int64_t K, int fmt, void* out,
@@ -251,6 +281,43 @@ cudaError_t launch_sf_to_logical(const void* sf, int64_t rows, int64_t K, void* 
                                                    static_cast<uint32_t>(K / 32),
                                                    static_cast<uint32_t>(sf_atoms_k(K)),
                                                    static_cast<uint8_t*>(out));
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------- calibration
+namespace {
+
+// max |x| over n bf16 values (n a multiple of 8): packed abs-max per 16-byte group, a
+// warp reduction, and one atomicMax per warp on the float's bits (non-negative floats
+// order like their bit patterns).  *out must hold 0 before the launch.  An Inf or NaN
+// input makes the result Inf or NaN (their bit patterns lie above every finite one).
+__global__ void __launch_bounds__(kThreads) absmax_kernel(const uint4* __restrict__ x, uint64_t n_groups,
+                                                          uint32_t* __restrict__ out)
+{
+    uint32_t m = 0;
+    for (uint64_t g = blockIdx.x * uint64_t(kThreads) + threadIdx.x; g < n_groups;
+         g += uint64_t(gridDim.x) * kThreads) {
+        const uint4 v = ld_stream(x + g);
+        uint32_t m2 = absmax_bf16x2(absmax_bf16x2(v.x, v.y), absmax_bf16x2(v.z, v.w));
+        m2 &= 0x7FFF7FFFu;
+        m = max(m, max(m2 & 0xFFFFu, m2 >> 16));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31u) == 0) atomicMax(out, m << 16);  // bf16 bits -> fp32 bits
+}
+
+}  // namespace
+
+cudaError_t launch_absmax(const void* x, int64_t n, float* out, cudaStream_t stream)
+{
+    cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+    const uint64_t n_groups = static_cast<uint64_t>(n / 8);
+    const int64_t want = ceil_div(static_cast<int64_t>(n_groups), kThreads);
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * 8)));
+    absmax_kernel<<<grid, kThreads, 0, stream>>>(static_cast<const uint4*>(x), n_groups,
+                                                 reinterpret_cast<uint32_t*>(out));
     return cudaGetLastError();
 }
 

@@ -176,6 +176,43 @@ def ffn(x: torch.Tensor, up: QWeight, down: QWeight, up_fmt="e2m1", down_fmt="e2
     return out
 
 
+def absmax(x: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """max |x| over a bf16 tensor, as a one-element fp32 CUDA tensor (calibration)."""
+    _cuda_bf16(x, "x")
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    check(_lib.lib().mxq_absmax(_p(x), x.numel(), _p(out), _stream(stream)), "mxq_absmax")
+    return out
+
+
+def quantize_act_static(x: torch.Tensor, scale: float, codes=None, sf=None, stream=None):
+    """x [M, K] bf16 -> static per-tensor E4M3 codes [M, K] and tiled scales (all 127)."""
+    _cuda_bf16(x, "x")
+    M, K = x.shape
+    if codes is None:
+        codes = torch.empty(max(1, codes_bytes(M, K, FMT_E4M3)), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(max(1, sf_bytes(M, K)), dtype=torch.uint8, device=x.device)
+    check(_lib.lib().mxq_quantize_act_static(_p(x), M, K, float(scale), _p(codes), _p(sf), _stream(stream)),
+          "mxq_quantize_act_static")
+    return codes, sf
+
+
+def linear_static(x: torch.Tensor, w: QWeight, act_scale: float, workspace=None, out=None, stream=None):
+    """y = act_scale * (static E4M3 codes of x) . deq(w)^T + bias (W4A8, static activations)."""
+    _cuda_bf16(x, "x")
+    M, K = x.shape
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(M, w.N, K, FMT_E4M3, MODE_NATIVE), dtype=torch.uint8,
+                                device=x.device)
+    if out is None:
+        out = torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
+    check(_lib.lib().mxq_linear_static(_p(x), M, K, _p(w.codes), _p(w.sf), w.N, _p(w.bias), float(act_scale),
+                                       _p(workspace), workspace.numel(), _p(out), _stream(stream)),
+          "mxq_linear_static")
+    return out
+
+
 def block_workspace_bytes(weights, rows, w4a8_bits: int, mode="native") -> int:
     descs = (WDesc * 8)(*[w.desc() for w in weights])
     ms = (ctypes.c_int64 * 8)(*rows)

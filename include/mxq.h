@@ -194,6 +194,31 @@ int mxq_ffn(const void* x_bf16, int64_t M, int64_t K, const mxq_wdesc* up, const
 /* Workspace bytes of mxq_ffn (the quantized input and hidden activation), or -1. */
 int64_t mxq_ffn_workspace_bytes(int64_t M, int64_t K, int64_t H, int up_fmt, int down_fmt);
 
+/* Static per-tensor FP8 E4M3 activations: the blog's W4A8 as its "Quantization formats"
+ * table names it ("FP8 E4M3 static activations"), one scale for the whole tensor fixed
+ * offline.  codes[m, k] = E4M3 RNE, saturating, of fl32(x[m, k] * fl32(1/scale)); sf is
+ * written in the tiled layout with every block's scale 127 (x1) and the padding 0, so
+ * the codes feed the kind::mxf8f6f4 GEMM unchanged; the tensor scale goes to the GEMM
+ * (mxq_linear_static).  scale > 0 and finite (MXQ_ERR_INVALID_ARG otherwise); inputs
+ * are expected finite (Inf saturates to +-448, NaN gives an E4M3 NaN code).  Sizes and
+ * alignment as for mxq_quantize_act with fmt E4M3. */
+int mxq_quantize_act_static(const void* x_bf16, int64_t M, int64_t K, float scale, void* codes, void* sf,
+                            void* stream);
+
+/* The W4A8 linear with a static per-tensor activation scale:
+ *   y = bf16( act_scale * sum_k q[m, k] * deqW[n, k] + bias[n] ),
+ * q the static E4M3 codes of x (mxq_quantize_act_static).  Arguments as for mxq_linear
+ * with act_fmt E4M3 and mode NATIVE (K % 128 == 0; workspace of
+ * mxq_workspace_bytes(M, N, K, MXQ_FMT_E4M3, MXQ_MODE_NATIVE) bytes). */
+int mxq_linear_static(const void* x_bf16, int64_t M, int64_t K, const void* w_codes, const void* w_sf, int64_t N,
+                      const void* bias_bf16, float act_scale, void* workspace, int64_t ws_bytes, void* y_bf16,
+                      void* stream);
+
+/* Calibration of a static scale: out_f32 (one float, device) = max |x| over n bf16
+ * values (n % 8 == 0, x 16-byte aligned); the scale is then max / 448.  An Inf or NaN
+ * input makes the result Inf or NaN. */
+int mxq_absmax(const void* x_bf16, int64_t n, void* out_f32, void* stream);
+
 /* Tiled scale factors -> logical row-major [rows, K/32] bytes (for tests). */
 int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_rowmajor, void* stream);
 

@@ -131,3 +131,18 @@ def test_ffn_workspace_and_shape_checks():
     assert L.mxq_ffn(A16, 128, 256, ctypes.byref(up), ctypes.byref(down), 0, 0, ws, need - 1, A16,
                      None) == _lib.ERR_WORKSPACE
     assert L.mxq_ffn(A16, 128, 256, None, ctypes.byref(down), 0, 0, ws, need, A16, None) == _lib.ERR_INVALID_ARG
+
+
+def test_static_entry_points_reject_bad_arguments():
+    L = _lib.lib()
+    for bad_scale in (0.0, -1.0, float("inf"), float("nan")):
+        assert L.mxq_quantize_act_static(A16, 128, 256, bad_scale, A16, A16, None) == _lib.ERR_INVALID_ARG
+        assert L.mxq_linear_static(A16, 128, 256, A16, A16, 256, None, bad_scale, V(1 << 20), 1 << 30, A16,
+                                   None) == _lib.ERR_INVALID_ARG
+    assert L.mxq_quantize_act_static(A16, 128, 250, 0.5, A16, A16, None) == _lib.ERR_SHAPE
+    assert L.mxq_linear_static(A16, 128, 96, A16, A16, 256, None, 0.5, V(1 << 20), 1 << 30, A16,
+                               None) == _lib.ERR_SHAPE  # W4A8 GEMM needs K % 128
+    assert L.mxq_linear_static(A16, 128, 256, A16, A16, 256, None, 0.5, V(1 << 20), 16, A16,
+                               None) == _lib.ERR_WORKSPACE
+    assert L.mxq_absmax(A16, 12, A16, None) == _lib.ERR_SHAPE
+    assert L.mxq_absmax(A8, 16, A16, None) == _lib.ERR_ALIGN
