@@ -82,6 +82,12 @@ def lib():
         L.mxo_quantize_static_e4m3.restype = i32
         L.mxo_linear_rows_scaled.argtypes = [vp, vp, i32, vp, i64, i64, vp, vp, i64, vp, dbl, vp, i32]
         L.mxo_linear_rows_scaled.restype = i32
+        L.mxo_hadamard_norm.argtypes = [i32]
+        L.mxo_hadamard_norm.restype = ctypes.c_float
+        L.mxo_fwht_f32.argtypes = [vp, i32]
+        L.mxo_fwht_f32.restype = None
+        L.mxo_quantize_transformed.argtypes = [vp, i64, i64, vp, i32, i32, vp, vp, vp]
+        L.mxo_quantize_transformed.restype = i32
     return _lib
 
 
@@ -254,3 +260,34 @@ def linear_rows_scaled(a_codes, a_sf, a_fmt, rows, K, w_codes, w_sf, alpha, bias
     if rc != 0:
         raise ValueError("oracle scaled linear failed (rc=%d)" % rc)
     return y
+
+
+def hadamard_norm(B: int) -> float:
+    """fl32(1 / sqrt(B)), the normalization of the block Hadamard rotation."""
+    return float(lib().mxo_hadamard_norm(int(B)))
+
+
+def fwht_f32(v: np.ndarray) -> np.ndarray:
+    """Fast Walsh-Hadamard transform (Sylvester order, unnormalized) of a float32 vector
+    whose length is a power of two, in binary32 arithmetic."""
+    out = np.ascontiguousarray(v, dtype=np.float32).copy()
+    lib().mxo_fwht_f32(_ptr(out), out.size)
+    return out
+
+
+def quantize_transformed(x_bits: np.ndarray, fmt: int, B: int, mul: np.ndarray | None = None):
+    """Smooth (t = x * mul), rotate each B-block by the normalized Hadamard, MX-quantize.
+    Returns (codes, logical scales, transformed float32 values)."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    rows, K = x_bits.shape
+    codes = np.zeros((rows, codes_row_bytes(K, fmt)), dtype=np.uint8)
+    sf = np.zeros((rows, K // 32), dtype=np.uint8)
+    t = np.zeros((rows, K), dtype=np.float32)
+    mp = None
+    if mul is not None:
+        mul = np.ascontiguousarray(mul, dtype=np.float32)
+        mp = _ptr(mul)
+    rc = lib().mxo_quantize_transformed(_ptr(x_bits), rows, K, mp, B, fmt, _ptr(codes), _ptr(sf), _ptr(t))
+    if rc != 0:
+        raise ValueError("oracle transform failed (rc=%d)" % rc)
+    return codes, sf, t

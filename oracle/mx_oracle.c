@@ -153,14 +153,12 @@ double mxo_scale_value(int sc)
 
 /* ---- block and tensor quantization ------------------------------------------- */
 
-/* Quantize one block of 32 bf16 values into 32 element codes and a scale code. */
-static int quantize_block(const uint16_t *x, int fmt, int codes[32])
+/* Quantize one block of 32 values into 32 element codes and a scale code. */
+static int quantize_values(const double *v, int fmt, int codes[32])
 {
-    double v[32];
     double amax = 0.0;
     int nonfinite = 0;
     for (int i = 0; i < 32; ++i) {
-        v[i] = mxo_bf16_to_double(x[i]);
         if (isnan(v[i]) || isinf(v[i])) nonfinite = 1;
         else if (fabs(v[i]) > amax) amax = fabs(v[i]);
     }
@@ -170,6 +168,29 @@ static int quantize_block(const uint16_t *x, int fmt, int codes[32])
         else codes[i] = mxo_encode_elem(v[i] / mxo_scale_value(sc), fmt);
     }
     return sc;
+}
+
+/* One block of 32 bf16 values. */
+static int quantize_block(const uint16_t *x, int fmt, int codes[32])
+{
+    double v[32];
+    for (int i = 0; i < 32; ++i) v[i] = mxo_bf16_to_double(x[i]);
+    return quantize_values(v, fmt, codes);
+}
+
+/* Place the 32 codes of block kb into a row of element codes (R6). */
+static void store_block_codes(uint8_t *out, int64_t kb, const int codes[32], int fmt)
+{
+    for (int i = 0; i < 32; ++i) {
+        int64_t k = kb * 32 + i;
+        if (fmt == MXO_E4M3) {
+            out[k] = (uint8_t)codes[i];
+        } else if ((k & 1) == 0) {
+            out[k / 2] = (uint8_t)(codes[i] & 0xF);
+        } else {
+            out[k / 2] |= (uint8_t)((codes[i] & 0xF) << 4);
+        }
+    }
 }
 
 /* Bytes of element codes per row: K/2 (E2M1, two per byte, R6) or K (E4M3). */
@@ -193,17 +214,7 @@ static void *quant_rows(void *arg)
         for (int64_t kb = 0; kb < KB; ++kb) {
             int sc = quantize_block(j->x + r * j->K + kb * 32, j->fmt, codes);
             j->sf[r * KB + kb] = (uint8_t)sc;
-            uint8_t *out = j->codes + r * rb;
-            for (int i = 0; i < 32; ++i) {
-                int64_t k = kb * 32 + i;
-                if (j->fmt == MXO_E4M3) {
-                    out[k] = (uint8_t)codes[i];
-                } else if ((k & 1) == 0) {
-                    out[k / 2] = (uint8_t)(codes[i] & 0xF);
-                } else {
-                    out[k / 2] |= (uint8_t)((codes[i] & 0xF) << 4);
-                }
-            }
+            store_block_codes(j->codes + r * rb, kb, codes, j->fmt);
         }
     }
     return NULL;
@@ -447,5 +458,72 @@ int mxo_linear_rows_scaled(const uint8_t *a_codes, const uint8_t *a_sf, int a_fm
     for (int64_t i = 0; i < nrows; ++i)
         for (int64_t j = 0; j < N; ++j)
             y[i * N + j] = alpha * y[i * N + j] + (bias ? mxo_bf16_to_double(bias[j]) : 0.0);
+    return 0;
+}
+
+/* ---- transform_on: per-channel smoothing and block Hadamard rotation --------------- */
+
+/* The third policy value of the blog's "Mixed-Precision selection": the activation is
+ * transformed before it is quantized -- divided per channel by SmoothQuant scales (the
+ * weights carry the scales instead) and rotated by a fixed block Hadamard matrix (the
+ * weights rotated the same way offline), so x . W^T is unchanged while outliers spread
+ * over a block.  The codes are decided from the transformed binary32 values, so this
+ * oracle takes every step in binary32, in the kernel's order:
+ *   t_k = fl32(x_k * mul_k)            (mul = 1/s for activations, s for weights; NULL: t = x)
+ *   each block of B consecutive t's:  fast Walsh-Hadamard transform (below), then each
+ *   value times c_B = fl32(1/sqrt B), rounded;
+ *   the rows then MX-quantized from those values exactly as mxo_quantize does. */
+
+/* c_B = fl32(1/sqrt B) for B = 2^j: 2^(-j/2) for even j, fl32(sqrt 2) * 2^(-(j+1)/2) for odd
+ * j (the scaling by a power of two is exact, so this is the correctly rounded value). */
+float mxo_hadamard_norm(int B)
+{
+    int j = 0;
+    while ((1 << j) < B) ++j;
+    if (j % 2 == 0) return ldexpf(1.0f, -j / 2);
+    return ldexpf((float)M_SQRT2, -(j + 1) / 2);
+}
+
+/* In-place fast Walsh-Hadamard transform of n = 2^j binary32 values in Sylvester order
+ * (the result is v . H_n with H_n[a][b] = (-1)^popcount(a & b)): for h = 1, 2, 4, ..., n/2
+ * in that order, every pair (i, i + h) with bit h of i clear becomes (v_i + v_i+h,
+ * v_i - v_i+h), each sum and difference rounded to binary32. */
+void mxo_fwht_f32(float *v, int n)
+{
+    for (int h = 1; h < n; h <<= 1)
+        for (int i = 0; i < n; ++i)
+            if ((i & h) == 0) {
+                float a = v[i], b = v[i + h];
+                v[i] = a + b;
+                v[i + h] = a - b;
+            }
+}
+
+int mxo_quantize_transformed(const uint16_t *x, int64_t rows, int64_t K, const float *mul, int B, int fmt,
+                             uint8_t *codes, uint8_t *sf, float *t_out)
+{
+    if (K % 32 != 0 || B < 32 || (B & (B - 1)) != 0 || K % B != 0) return -1;
+    const float c = mxo_hadamard_norm(B);
+    const int64_t KB = K / 32, rb = mxo_codes_row_bytes(K, fmt);
+    float *t = (float *)malloc(sizeof(float) * (size_t)K);
+    double v[32];
+    int cd[32];
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t k = 0; k < K; ++k) {
+            float xk = (float)mxo_bf16_to_double(x[r * K + k]);
+            t[k] = mul ? xk * mul[k] : xk;
+        }
+        for (int64_t b0 = 0; b0 < K; b0 += B) {
+            mxo_fwht_f32(t + b0, B);
+            for (int i = 0; i < B; ++i) t[b0 + i] = t[b0 + i] * c;
+        }
+        if (t_out) memcpy(t_out + r * K, t, sizeof(float) * (size_t)K);
+        for (int64_t kb = 0; kb < KB; ++kb) {
+            for (int i = 0; i < 32; ++i) v[i] = (double)t[kb * 32 + i];
+            sf[r * KB + kb] = (uint8_t)quantize_values(v, fmt, cd);
+            store_block_codes(codes + r * rb, kb, cd, fmt);
+        }
+    }
+    free(t);
     return 0;
 }

@@ -46,6 +46,10 @@ MUTANTS = [
      "y[i * N + j] = alpha * (y[i * N + j] + (bias ? mxo_bf16_to_double(bias[j]) : 0.0));"),
     ("static_divides_in_double", "float p = (float)(mxo_bf16_to_double(x[i]) * (double)inv_scale);",
      "float p = (float)(mxo_bf16_to_double(x[i]) * (double)inv_scale * 1.0000001);"),
+    ("fwht_difference_flipped", "                v[i + h] = a - b;", "                v[i + h] = b - a;"),
+    ("hadamard_unnormalized", "for (int i = 0; i < B; ++i) t[b0 + i] = t[b0 + i] * c;",
+     "for (int i = 0; i < B; ++i) t[b0 + i] = t[b0 + i] * 1.0f;"),
+    ("smoothing_divides", "t[k] = mul ? xk * mul[k] : xk;", "t[k] = mul ? xk / mul[k] : xk;"),
     ("gelu_cancelling_form", "double mxo_gelu(double x) { return 0.5 * x * erfc(-x / sqrt(2.0)); }",
      "double mxo_gelu(double x) { return 0.5 * x * (1.0 + erf(x / sqrt(2.0))); }"),
 ]

@@ -505,3 +505,74 @@ def test_linear_scaled_brute_force_exact():
                         Fraction(oracle.decode_elem(wc, oracle.E2M1)) * Fraction(2) ** (int(w_sf[n, k // 32]) - 127))
             want = Fraction(alpha) * acc + Fraction(oracle.bf16_to_float(int(bias[n])))
             assert abs(Fraction(y[m, n]) - want) <= abs(want) * Fraction(1, 10 ** 14) + Fraction(1, 10 ** 300)
+
+
+# --- transform_on: smoothing and block Hadamard rotation ------------------------------------
+
+@pytest.mark.parametrize("n", [32, 128])
+def test_fwht_matches_sylvester_matrix(n):
+    """The binary32 FWHT equals v . H_n (scipy's Sylvester Hadamard, fp64) within the
+    rounding of its log2(n) stages."""
+    from scipy.linalg import hadamard
+    rng = np.random.default_rng(n)
+    H = hadamard(n).astype(np.float64)
+    for _ in range(50):
+        v = (rng.standard_normal(n) * rng.choice([1e-3, 1.0, 40.0], size=n)).astype(np.float32)
+        got = oracle.fwht_f32(v).astype(np.float64)
+        want = v.astype(np.float64) @ H
+        bound = np.log2(n) * 2.0 ** -23 * np.abs(v).astype(np.float64).sum() * 2
+        assert np.abs(got - want).max() <= bound
+
+
+def test_fwht_involution_and_norm():
+    rng = np.random.default_rng(5)
+    for n in (32, 128):
+        v = rng.standard_normal(n).astype(np.float32)
+        back = oracle.fwht_f32(oracle.fwht_f32(v)).astype(np.float64) / n
+        assert np.abs(back - v).max() <= 1e-5 * np.abs(v).max()
+        c = oracle.hadamard_norm(n)
+        assert c == float(np.float32(1.0 / np.sqrt(n)))
+        assert abs(c * c * n - 1.0) < 1e-6
+
+
+@pytest.mark.parametrize("B", [32, 128])
+def test_transform_is_scaled_hadamard_rotation(B):
+    """The transformed values equal (x * mul) . blockdiag(H_B) / sqrt(B) (fp64) within
+    binary32 rounding; codes and scales dequantize to within one element step of them."""
+    from scipy.linalg import hadamard
+    rng = np.random.default_rng(B + 1)
+    M, K = 6, 256
+    x = (rng.standard_normal((M, K)) * 3).astype(np.float32)
+    x[:, 5] *= 60.0                                          # an outlier channel
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
+    xb = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    mul = rng.uniform(0.5, 2.0, size=K).astype(np.float32)
+    codes, sf, t = oracle.quantize_transformed(bits, oracle.E2M1, B, mul)
+    H = hadamard(B).astype(np.float64) / np.sqrt(B)
+    want = np.concatenate([(xb * mul.astype(np.float64))[:, b0:b0 + B] @ H for b0 in range(0, K, B)], axis=1)
+    assert np.abs(t.astype(np.float64) - want).max() <= 1e-5 * np.abs(want).max()
+    deq = oracle.dequantize(codes, sf, K, oracle.E2M1)
+    scale = np.repeat(2.0 ** (sf.astype(np.float64) - 127), 32, axis=1)
+    assert (np.abs(deq - t) <= 2.0 * scale + 1e-30).all()   # within the largest E2M1 step (4 -> 6)
+
+
+def test_transform_power_of_two_smoothing_shifts_only_the_scales():
+    """A smoothing multiplier of 2^j on every channel scales the transformed values exactly,
+    so the element codes are unchanged and every scale code moves by j."""
+    rng = np.random.default_rng(9)
+    x = (rng.standard_normal((4, 128)) * 2).astype(np.float32)
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
+    c0, s0, _ = oracle.quantize_transformed(bits, oracle.E4M3, 32, None)
+    c1, s1, _ = oracle.quantize_transformed(bits, oracle.E4M3, 32, np.full(128, 8.0, dtype=np.float32))
+    assert np.array_equal(c0, c1)
+    assert np.array_equal(s1.astype(int), s0.astype(int) + 3)
+
+
+def test_transform_sign_symmetry():
+    rng = np.random.default_rng(10)
+    x = rng.standard_normal((3, 128)).astype(np.float32)
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
+    c0, s0, t0 = oracle.quantize_transformed(bits, oracle.E4M3, 128, None)
+    c1, s1, t1 = oracle.quantize_transformed(bits ^ 0x8000, oracle.E4M3, 128, None)
+    assert np.array_equal(t1, -t0) and np.array_equal(s0, s1)
+    assert np.array_equal(c1[t0 != 0], c0[t0 != 0] ^ 0x80)
