@@ -55,6 +55,10 @@ SIGNATURES = {
     "mxq_quantize_act_static": ([_vp, _i64, _i64, ctypes.c_float, _vp, _vp, _vp], _i32),
     "mxq_linear_static": ([_vp, _i64, _i64, _vp, _vp, _i64, _vp, ctypes.c_float, _vp, _i64, _vp, _vp], _i32),
     "mxq_absmax": ([_vp, _i64, _vp, _vp], _i32),
+    "mxq_quantize_act_transformed": ([_vp, _i64, _i64, _i32, _vp, _i32, _vp, _vp, _vp], _i32),
+    "mxq_quantize_weight_transformed": ([_vp, _i64, _i64, _vp, _i32, _vp, _vp, _vp], _i32),
+    "mxq_linear_transformed": ([_vp, _i64, _i64, _vp, _vp, _i64, _vp, _i32, _vp, _i32, _vp, _i64, _vp, _vp],
+                               _i32),
     "mxq_sf_to_logical": ([_vp, _i64, _i64, _vp, _vp], _i32),
     "mxq_poll_status": ([_vp], _i32),
     "mxq_set_debug": ([_u32], _i32),

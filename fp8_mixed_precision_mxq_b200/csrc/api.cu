@@ -160,6 +160,24 @@ int run_linear(const void* x, int64_t M, int64_t K, const void* w_codes, const v
 // rounded to binary32, which equals the correctly rounded binary32 division).
 float static_inverse(float s) { return static_cast<float>(1.0 / static_cast<double>(s)); }
 
+// fl32(1/sqrt B) for B = 2^j: 2^(-j/2) for even j, fl32(sqrt 2) * 2^(-(j+1)/2) for odd j
+// (scaling by a power of two is exact, so both are the correctly rounded value).
+float hadamard_norm(int B)
+{
+    int j = 0;
+    while ((1 << j) < B) ++j;
+    if (j % 2 == 0) return std::ldexp(1.0f, -j / 2);
+    return std::ldexp(static_cast<float>(M_SQRT2), -(j + 1) / 2);
+}
+
+int check_transform(int64_t K, int block, const void* mul)
+{
+    if (block != 32 && block != 128) return fail(MXQ_ERR_INVALID_ARG, "rotation block must be 32 or 128 (got %d)", block);
+    if (K % block != 0) return fail(MXQ_ERR_SHAPE, "K=%lld is not a multiple of the rotation block %d", (long long)K, block);
+    if (mul) RETURN_IF(check_ptr(mul, "channel multiplier"));
+    return MXQ_OK;
+}
+
 int check_mode(int mode)
 {
     if (mode != MXQ_MODE_NATIVE && mode != MXQ_MODE_QDQ) return fail(MXQ_ERR_INVALID_ARG, "unknown mode %d", mode);
@@ -416,6 +434,51 @@ int mxq_linear_static(const void* x_bf16, int64_t M, int64_t K, const void* w_co
     int rc = launch_gemm(g, st, &msg, g_path, sizeof g_path);
     if (rc != MXQ_OK) return fail(rc, "gemm: %s", msg ? msg : "launch failed");
     snprintf(g_path + strlen(g_path), sizeof g_path - strlen(g_path), " static-scale");
+    return ok();
+}
+
+int mxq_quantize_act_transformed(const void* x_bf16, int64_t M, int64_t K, int fmt, const float* mul, int block,
+                                 void* codes, void* sf, void* stream)
+{
+    RETURN_IF(check_fmt(fmt));
+    RETURN_IF(check_rows_k(M, K, "quantize_transformed"));
+    RETURN_IF(check_transform(K, block, mul));
+    RETURN_IF(check_ptr(x_bf16, "x"));
+    RETURN_IF(check_ptr(codes, "codes"));
+    RETURN_IF(check_ptr(sf, "sf"));
+    RETURN_IF(check_device());
+    snprintf(g_path, sizeof g_path, "quantize %s hadamard%d%s", fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1", block,
+             mul ? " smooth" : "");
+    return cuda_rc(launch_quantize_transform(x_bf16, M, K, fmt, mul, block, hadamard_norm(block), codes, sf,
+                                             static_cast<cudaStream_t>(stream)),
+                   "quantize launch");
+}
+
+int mxq_quantize_weight_transformed(const void* w_bf16, int64_t N, int64_t K, const float* mul, int block, void* codes,
+                                    void* sf, void* stream)
+{
+    return mxq_quantize_act_transformed(w_bf16, N, K, MXQ_FMT_E2M1, mul, block, codes, sf, stream);
+}
+
+int mxq_linear_transformed(const void* x_bf16, int64_t M, int64_t K, const void* w_codes, const void* w_sf, int64_t N,
+                           const void* bias_bf16, int act_fmt, const float* act_mul, int block, void* workspace,
+                           int64_t ws_bytes, void* y_bf16, void* stream)
+{
+    RETURN_IF(check_ptr(x_bf16, "x"));
+    RETURN_IF(check_ptr(workspace, "workspace", kWsAlign));
+    RETURN_IF(check_gemm(workspace, workspace, act_fmt, M, K, w_codes, w_sf, N, bias_bf16, y_bf16));
+    RETURN_IF(check_transform(K, block, act_mul));
+    const int64_t need = linear_ws(M, N, K, act_fmt, MXQ_MODE_NATIVE);
+    if (ws_bytes < need)
+        return fail(MXQ_ERR_WORKSPACE, "workspace has %lld bytes, needs %lld", (long long)ws_bytes, (long long)need);
+    RETURN_IF(check_device());
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* xc = static_cast<uint8_t*>(workspace);
+    uint8_t* xs = xc + round_up(codes_bytes(M, K, act_fmt), kWsAlign);
+    RETURN_IF(cuda_rc(launch_quantize_transform(x_bf16, M, K, act_fmt, act_mul, block, hadamard_norm(block), xc, xs, st),
+                      "quantize launch"));
+    RETURN_IF(run_gemm(xc, xs, act_fmt, M, K, w_codes, w_sf, N, bias_bf16, y_bf16, st));
+    snprintf(g_path + strlen(g_path), sizeof g_path - strlen(g_path), " hadamard%d%s", block, act_mul ? " smooth" : "");
     return ok();
 }
 

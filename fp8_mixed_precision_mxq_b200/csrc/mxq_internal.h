@@ -25,6 +25,10 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, int fmt, voi
 // Static per-tensor E4M3: codes = RNE_sat(x * inv_scale), block scales 127.
 cudaError_t launch_quantize_static(const void* x, int64_t rows, int64_t K, float inv_scale, void* codes, void* sf,
                                    cudaStream_t stream);
+// transform_on: t = x * mul (per channel; mul may be null), each `block` (32 or 128)
+// values along K rotated by the Hadamard matrix times norm, then MX-quantized in fmt.
+cudaError_t launch_quantize_transform(const void* x, int64_t rows, int64_t K, int fmt, const float* mul, int block,
+                                      float norm, void* codes, void* sf, cudaStream_t stream);
 // *out = max |x| over n bf16 values (n % 8 == 0), as fp32.
 cudaError_t launch_absmax(const void* x, int64_t n, float* out, cudaStream_t stream);
 cudaError_t launch_dequantize(const void* codes, const void* sf, int64_t rows, int64_t K, int fmt, void* out,

@@ -213,6 +213,60 @@ def linear_static(x: torch.Tensor, w: QWeight, act_scale: float, workspace=None,
     return out
 
 
+def _f32_or_none(t, name):
+    if t is None:
+        return None
+    if not (t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()):
+        raise ValueError("%s must be a contiguous float32 CUDA tensor" % name)
+    return t
+
+
+def quantize_act_transformed(x: torch.Tensor, fmt="e2m1", block=32, mul=None, codes=None, sf=None, stream=None):
+    """x [M, K] bf16 -> MX codes and tiled scales of (x * mul) rotated by the block Hadamard."""
+    _cuda_bf16(x, "x")
+    M, K = x.shape
+    f = _fmt(fmt)
+    mul = _f32_or_none(mul, "mul")
+    if codes is None:
+        codes = torch.empty(max(1, codes_bytes(M, K, f)), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(max(1, sf_bytes(M, K)), dtype=torch.uint8, device=x.device)
+    check(_lib.lib().mxq_quantize_act_transformed(_p(x), M, K, f, _p(mul), int(block), _p(codes), _p(sf),
+                                                  _stream(stream)), "mxq_quantize_act_transformed")
+    return codes, sf
+
+
+def quantize_weight_transformed(w: torch.Tensor, bias=None, block=32, mul=None, stream=None) -> QWeight:
+    """w [N, K] bf16 -> QWeight of (w * mul) rotated by the block Hadamard (mul = s)."""
+    _cuda_bf16(w, "w")
+    N, K = w.shape
+    mul = _f32_or_none(mul, "mul")
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    sf = torch.empty(max(1, sf_bytes(N, K)), dtype=torch.uint8, device=w.device)
+    check(_lib.lib().mxq_quantize_weight_transformed(_p(w), N, K, _p(mul), int(block), _p(codes), _p(sf),
+                                                     _stream(stream)), "mxq_quantize_weight_transformed")
+    if bias is not None:
+        _cuda_bf16(bias, "bias")
+    return QWeight(codes, sf, N, K, bias)
+
+
+def linear_transformed(x: torch.Tensor, w: QWeight, fmt="e2m1", block=32, act_mul=None, workspace=None, out=None,
+                       stream=None):
+    """The linear on the transformed path (w from quantize_weight_transformed, same block)."""
+    _cuda_bf16(x, "x")
+    M, K = x.shape
+    f = _fmt(fmt)
+    act_mul = _f32_or_none(act_mul, "act_mul")
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(M, w.N, K, f, MODE_NATIVE), dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty((M, w.N), dtype=torch.bfloat16, device=x.device)
+    check(_lib.lib().mxq_linear_transformed(_p(x), M, K, _p(w.codes), _p(w.sf), w.N, _p(w.bias), f, _p(act_mul),
+                                            int(block), _p(workspace), workspace.numel(), _p(out), _stream(stream)),
+          "mxq_linear_transformed")
+    return out
+
+
 def block_workspace_bytes(weights, rows, w4a8_bits: int, mode="native") -> int:
     descs = (WDesc * 8)(*[w.desc() for w in weights])
     ms = (ctypes.c_int64 * 8)(*rows)

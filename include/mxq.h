@@ -219,6 +219,35 @@ int mxq_linear_static(const void* x_bf16, int64_t M, int64_t K, const void* w_co
  * input makes the result Inf or NaN. */
 int mxq_absmax(const void* x_bf16, int64_t n, void* out_f32, void* stream);
 
+/* The "transform_on" policy of the blog's section "Mixed-Precision selection": a block is
+ * quantized after a fixed transform that spreads its outliers -- per-channel smoothing
+ * (SmoothQuant: activations divided by s, weights multiplied by s) and a block Hadamard
+ * rotation along K (activations and weights rotated alike, so x . W^T is unchanged).
+ *   t[m, k] = fl32(x[m, k] * mul[k])        (mul NULL: t = x; mul = 1/s for activations)
+ *   each `block` (32 or 128) consecutive t's along K <- t . H_block * fl32(1/sqrt(block)),
+ *     H the Sylvester Hadamard matrix (entries +-1), as a fast Walsh-Hadamard transform in
+ *     binary32 (butterflies (a, b) -> (a + b, a - b), h = 1, 2, 4, ..., then the scaling);
+ *   t MX-quantized in fmt as by mxq_quantize_act (scale from the block's binary32 abs-max).
+ * mul: NULL or K floats on the device, 16-byte aligned.  Requires K % block == 0.  Other
+ * arguments and errors as for mxq_quantize_act. */
+int mxq_quantize_act_transformed(const void* x_bf16, int64_t M, int64_t K, int fmt, const float* mul, int block,
+                                 void* codes, void* sf, void* stream);
+
+/* Weight side of the transform: as mxq_quantize_act_transformed with fmt E2M1 and
+ * mul = s (the SmoothQuant scales; NULL for rotation only).  A linear computes the same
+ * product when its weight was quantized with the same block and its activation with
+ * mul = 1/s. */
+int mxq_quantize_weight_transformed(const void* w_bf16, int64_t N, int64_t K, const float* mul, int block, void* codes,
+                                    void* sf, void* stream);
+
+/* Linear layer on the transformed path: mxq_quantize_act_transformed(x, act_mul, block)
+ * into the workspace, then the native GEMM against a weight from
+ * mxq_quantize_weight_transformed with the same block.  Arguments as for mxq_linear in
+ * NATIVE mode plus act_mul and block. */
+int mxq_linear_transformed(const void* x_bf16, int64_t M, int64_t K, const void* w_codes, const void* w_sf, int64_t N,
+                           const void* bias_bf16, int act_fmt, const float* act_mul, int block, void* workspace,
+                           int64_t ws_bytes, void* y_bf16, void* stream);
+
 /* Tiled scale factors -> logical row-major [rows, K/32] bytes (for tests). */
 int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_rowmajor, void* stream);
 

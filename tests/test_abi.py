@@ -146,3 +146,15 @@ def test_static_entry_points_reject_bad_arguments():
                                None) == _lib.ERR_WORKSPACE
     assert L.mxq_absmax(A16, 12, A16, None) == _lib.ERR_SHAPE
     assert L.mxq_absmax(A8, 16, A16, None) == _lib.ERR_ALIGN
+
+
+def test_transform_entry_points_reject_bad_arguments():
+    L = _lib.lib()
+    assert L.mxq_quantize_act_transformed(A16, 128, 256, 0, None, 64, A16, A16, None) == _lib.ERR_INVALID_ARG
+    assert L.mxq_quantize_act_transformed(A16, 128, 96, 0, None, 128, A16, A16, None) == _lib.ERR_SHAPE
+    assert L.mxq_quantize_act_transformed(A16, 128, 256, 0, A8, 32, A16, A16, None) == _lib.ERR_ALIGN
+    assert L.mxq_quantize_weight_transformed(A16, 128, 256, None, 33, A16, A16, None) == _lib.ERR_INVALID_ARG
+    assert L.mxq_linear_transformed(A16, 128, 256, A16, A16, 256, None, 0, None, 48, V(1 << 20), 1 << 30, A16,
+                                    None) == _lib.ERR_INVALID_ARG
+    assert L.mxq_linear_transformed(A16, 128, 256, A16, A16, 256, None, 0, None, 32, V(1 << 20), 16, A16,
+                                    None) == _lib.ERR_WORKSPACE

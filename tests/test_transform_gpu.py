@@ -1,0 +1,87 @@
+"""The transform_on path (blog section "Mixed-Precision selection": smoothing and a fixed
+Hadamard rotation before quantization): codes and scales bit-exact against the oracle,
+which takes the same binary32 steps in the same order, and the transformed linear within
+the GEMM tolerance of the oracle's product of the transformed operands."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import _mx
+
+pytestmark = pytest.mark.gpu
+
+
+def _ops():
+    from fp8_mixed_precision_mxq_b200 import ops
+    return ops
+
+
+def smooth_scales(x, alpha=0.5, seed=0):
+    """SmoothQuant-style per-channel scales s_k = max|x_k|^alpha (a calibration stand-in)."""
+    s = x.abs().amax(dim=0).float().clamp_min(1e-3) ** alpha
+    return s.contiguous()
+
+
+@pytest.mark.parametrize("fmt", ["e2m1", "e4m3"])
+@pytest.mark.parametrize("block", [32, 128])
+@pytest.mark.parametrize("smooth", [False, True])
+@pytest.mark.parametrize("M,K", [(1, 128), (129, 256), (300, 1024)])
+def test_quantize_transformed_bitexact(fmt, block, smooth, M, K):
+    ops = _ops()
+    x = synth.activation(M, K, "student_t", seed=M + K + block, device="cuda", outlier_frac=0.02, outlier_scale=40.0)
+    mul = (1.0 / smooth_scales(x)).contiguous() if smooth else None
+    codes, sf = ops.quantize_act_transformed(x, fmt, block, mul)
+    torch.cuda.synchronize()
+    c_ref, s_ref, _ = oracle.quantize_transformed(_mx.bits(x), _mx.FMT[fmt], block,
+                                                  None if mul is None else mul.cpu().numpy())
+    c_gpu = codes.cpu().numpy()
+    if not np.array_equal(c_gpu, c_ref.reshape(-1)):
+        i = int(np.nonzero(c_gpu != c_ref.reshape(-1))[0][0])
+        raise AssertionError("%d codes differ, first at byte %d: gpu %#x oracle %#x" % (
+            int((c_gpu != c_ref.reshape(-1)).sum()), i, c_gpu[i], c_ref.reshape(-1)[i]))
+    assert np.array_equal(sf.cpu().numpy(), oracle.sf_to_tiled(s_ref, K))
+
+
+@pytest.mark.parametrize("block", [32, 128])
+def test_transformed_linear_against_oracle(block):
+    ops = _ops()
+    M, N, K = 300, 520, 1024
+    x = synth.activation(M, K, "student_t", seed=11, device="cuda", outlier_frac=0.01, outlier_scale=50.0)
+    w = synth.weight(N, K, seed=12, device="cuda")
+    b = synth.bias(N, seed=12, device="cuda")
+    s = smooth_scales(x)
+    inv_s = (1.0 / s).contiguous()
+    qw = ops.quantize_weight_transformed(w, bias=b, block=block, mul=s)
+    y = ops.linear_transformed(x, qw, "e2m1", block, inv_s)
+    assert ops.poll_status() == 0
+    assert "hadamard%d smooth" % block in ops.last_path()
+    xc, xs, _ = oracle.quantize_transformed(_mx.bits(x), oracle.E2M1, block, inv_s.cpu().numpy())
+    wc, ws, _ = oracle.quantize_transformed(_mx.bits(w), oracle.E2M1, block, s.cpu().numpy())
+    ref = oracle.linear_rows(xc, xs, oracle.E2M1, np.arange(M), K, wc, ws, _mx.bits(b))
+    _mx.assert_gemm_close(_mx.bf16_to_f64(y), ref, "transformed linear, block %d" % block)
+    # the transforms cancel: the result approximates the unquantized product
+    exact = (x.double() @ w.double().T + b.double()).cpu().numpy()
+    assert _mx.sqnr_db(exact, _mx.bf16_to_f64(y)) > 15.0
+
+
+def test_transform_sqnr_report():
+    """W4A4 SQNR against the unquantized product on the outlier recipe, plain vs rotated
+    vs smoothed + rotated (a diagnostic; the values are printed, only a floor is asserted)."""
+    ops = _ops()
+    M, N, K = 512, 512, 2048
+    x = synth.activation(M, K, "student_t", seed=21, device="cuda", outlier_frac=0.01, outlier_scale=50.0)
+    w = synth.weight(N, K, seed=22, device="cuda")
+    exact = (x.double() @ w.double().T).cpu().numpy()
+    plain = _mx.sqnr_db(exact, _mx.bf16_to_f64(ops.linear(x, ops.quantize_weight(w), "e2m1")))
+    res = {"plain": plain}
+    for block in (32, 128):
+        rot = ops.linear_transformed(x, ops.quantize_weight_transformed(w, block=block), "e2m1", block)
+        res["hadamard%d" % block] = _mx.sqnr_db(exact, _mx.bf16_to_f64(rot))
+        s = smooth_scales(x)
+        sm = ops.linear_transformed(x, ops.quantize_weight_transformed(w, block=block, mul=s), "e2m1", block,
+                                    (1.0 / s).contiguous())
+        res["smooth+hadamard%d" % block] = _mx.sqnr_db(exact, _mx.bf16_to_f64(sm))
+    print("W4A4 SQNR (dB):", {k: round(v, 2) for k, v in res.items()})
+    assert min(res.values()) > 10.0
