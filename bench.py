@@ -10,8 +10,11 @@ load-time step).  Beside the headline number the JSON line carries:
                 alone with CUDA events on its launch stream;
   parts         the quantizer (GB/s against HBM) and the GEMM separately;
   ffn_up_720p_w4a4  the same linear at 720p / 81 frames (M = 75600);
-  w4a8          the W4A8 FFN-down linear at 720p (quantize to E4M3 + mxf8f6f4 GEMM)
-                and its quantize-dequantize emulation (QDQ) path;
+  w4a8          the W4A8 FFN-down linear at 720p (quantize to E4M3 + mxf8f6f4 GEMM),
+                its quantize-dequantize emulation (QDQ) path, and the same linear with
+                static per-tensor E4M3 activations;
+  transform_480p  the transform_on quantizer (smoothing + block Hadamard) and linear on
+                the headline workload;
   ffn_720p      the block's FFN with its hidden activation kept MX-quantized (the
                 FFN-up GEMM's epilogue applies GELU and quantizes), FFN-down W4A4 or W4A8;
   dit_block_720p  one DiT block's eight linears under the all-W4A4, all-W4A8 and mixed
@@ -333,6 +336,8 @@ def run_mxq(args):
         result["ffn_up_720p_w4a4"] = bench_target(args, ops, synth, dev, stream, world, rank, peaks, qw, b)
     if args.w4a8:
         result["w4a8"] = bench_w4a8(args, ops, synth, dev, stream, world, rank, peaks)
+    if args.transform:
+        result["transform_480p"] = bench_transform(args, ops, synth, dev, stream, world, rank, peaks, x, w, b)
     if args.ffn:
         result["ffn_720p"] = bench_ffn(args, ops, synth, dev, stream, world, rank, peaks)
     if args.block:
@@ -481,6 +486,39 @@ def bench_ffn(args, ops, synth, dev, stream, world, rank, peaks):
     return res
 
 
+def bench_transform(args, ops, synth, dev, stream, world, rank, peaks, x, w, b):
+    """The transform_on path on the headline workload: quantizer with per-channel smoothing
+    and a block Hadamard rotation (32 or 128), and the linear built on it."""
+    M, K = x.shape
+    N = w.shape[0]
+    s = x.abs().amax(dim=0).float().clamp_min(1e-3).sqrt().contiguous()  # SmoothQuant-style scales
+    inv_s = (1.0 / s).contiguous()
+    flops = 2.0 * M * N * K
+    qbytes = quant_bytes(M, K, "e2m1") + K * 4
+    iters = max(3, args.steps // 4)
+    codes = torch.empty(ops.codes_bytes(M, K, "e2m1"), dtype=torch.uint8, device=dev)
+    sf = torch.empty(ops.sf_bytes(M, K), dtype=torch.uint8, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(ops.workspace_bytes(M, N, K, "e2m1"), dtype=torch.uint8, device=dev)
+    res = {"workload": "FFN-up 480p (M=%d K=%d N=%d) W4A4, SmoothQuant-style scales + block Hadamard" % (M, K, N)}
+    for block in (32, 128):
+        qw = ops.quantize_weight_transformed(w, bias=b, block=block, mul=s)
+        fq = lambda blk=block: ops.quantize_act_transformed(x, "e2m1", blk, inv_s, codes=codes, sf=sf)  # noqa: E731
+        fl = lambda blk=block, q=qw: ops.linear_transformed(x, q, "e2m1", blk, inv_s, workspace=ws, out=y)  # noqa
+        for _ in range(2):
+            fq()
+            fl()
+        q_ms = max_over_ranks(time_loop(fq, iters, stream), world)
+        l_ms = max_over_ranks(time_loop(fl, iters, stream), world)
+        res["hadamard%d" % block] = {
+            "quantize_ms": round(q_ms, 4), "quantize_GB/s": round(qbytes / (q_ms * 1e-3) / 1e9, 1),
+            "quantize_frac_hbm": round(qbytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "linear_ms": round(l_ms, 4), "linear_TFLOP/s": round(job_tflops(flops, l_ms, world), 1)}
+    if ops.poll_status() != 0:
+        raise RuntimeError("device status set during the transform measurement")
+    return res
+
+
 def bench_block(args, ops, synth, dev, stream, world, rank, peaks):
     """One DiT block's eight linears at 720p / 81 frames (M = 75600, text context 512)
     through the block entry point, under the three precision masks."""
@@ -587,6 +625,20 @@ def bench_w4a8(args, ops, synth, dev, stream, world, rank, peaks):
     out["gemm_mxf8f6f4"] = {"ms": round(g_ms, 4), "TFLOP/s": round(flops / (g_ms * 1e-3) / 1e12, 1),
                             "frac_fp8": round(flops / (g_ms * 1e-3) / 1e12 / fp8_peak, 4),
                             "peak_fp8": round(fp8_peak, 1)}
+    # static per-tensor E4M3 activations (calibrated once, outside the timed region)
+    scale = ops.absmax(x).item() / 448.0
+    for _ in range(2):
+        ops.linear_static(x, qw, scale, workspace=ws, out=y)
+    s_ms = max_over_ranks(time_loop(lambda: ops.linear_static(x, qw, scale, workspace=ws, out=y), iters, stream),
+                          world)
+    sq_ms = max_over_ranks(time_loop(lambda: ops.quantize_act_static(x, scale, codes=xc, sf=xs), iters, stream),
+                           world)
+    out["static_e4m3"] = {"scale": scale, "linear_ms": round(s_ms, 4),
+                          "linear_TFLOP/s": round(flops / (s_ms * 1e-3) / 1e12, 1),
+                          "quantize_ms": round(sq_ms, 4),
+                          "quantize_GB/s": round(quant_bytes(M, K, "e4m3") / (sq_ms * 1e-3) / 1e9, 1),
+                          "quantize_frac_hbm": round(quant_bytes(M, K, "e4m3") / (sq_ms * 1e-3) / 1e9 /
+                                                     peaks["hbm_gbs"], 4)}
     if ops.poll_status() != 0:
         raise RuntimeError("device status set during the W4A8 measurement")
     return out
@@ -637,6 +689,8 @@ def main():
     ap.add_argument("--no-w4a8", dest="w4a8", action="store_false")
     ap.add_argument("--no-target", dest="target", action="store_false",
                     help="skip the 720p FFN-up (M=75600) measurement")
+    ap.add_argument("--no-transform", dest="transform", action="store_false",
+                    help="skip the smoothing + Hadamard quantizer measurement")
     ap.add_argument("--no-ffn", dest="ffn", action="store_false",
                     help="skip the fused-FFN (M=75600) measurement")
     ap.add_argument("--no-block", dest="block", action="store_false",

@@ -231,80 +231,96 @@ __global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t nwarps = gridDim.x * (kThreads / 32);
     const uint32_t warp = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-    for (uint32_t w0 = warp; w0 * 32u < n_groups; w0 += nwarps) {
+    constexpr int kU = 4;  // independent groups per lane per step (loads in flight)
+    for (uint32_t w0 = warp; w0 * 32u < n_groups; w0 += nwarps * kU) {
         // n_groups is a multiple of 4 * (kB / 32) lanes' worth, so a rotation block is
         // either wholly inside the tensor or wholly outside; lanes past the end carry zeros
-        const uint32_t g = w0 * 32u + lane;
-        const bool live = g < n_groups;
-        const uint4 v = live ? ld_stream(x + g) : make_uint4(0, 0, 0, 0);
-        const uint32_t blk = g >> 2;
-        const uint32_t r = static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(blk) << 24, kb_magic));
-        const uint32_t kb = blk - r * KB;
-        float t[8];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t g[kU];
+        uint4 v[kU];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            t[2 * i] = lo_f(w[i]);
-            t[2 * i + 1] = hi_f(w[i]);
+        for (int u = 0; u < kU; ++u) {
+            g[u] = (w0 + u * nwarps) * 32u + lane;
+            v[u] = g[u] < n_groups ? ld_stream(x + g[u]) : make_uint4(0, 0, 0, 0);
         }
-        if (mul != nullptr && live) {
-            const float4* m4 = reinterpret_cast<const float4*>(mul + kb * 32u + (g & 3u) * 8u);
-            const float4 a = __ldg(m4), b = __ldg(m4 + 1);
-            const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        float t[kU][8];
+        uint32_t r[kU], kb[kU];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) t[i] = __fmul_rn(t[i], mv[i]);
+        for (int u = 0; u < kU; ++u) {
+            const uint32_t blk = g[u] >> 2;
+            r[u] = static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(blk) << 24, kb_magic));
+            kb[u] = blk - r[u] * KB;
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                t[u][2 * i] = lo_f(w[i]);
+                t[u][2 * i + 1] = hi_f(w[i]);
+            }
+            if (mul != nullptr && g[u] < n_groups) {
+                const float4* m4 = reinterpret_cast<const float4*>(mul + kb[u] * 32u + (g[u] & 3u) * 8u);
+                const float4 a = __ldg(m4), b = __ldg(m4 + 1);
+                const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) t[u][i] = __fmul_rn(t[u][i], mv[i]);
+            }
         }
         // butterflies inside the lane: h = 1, 2, 4
 #pragma unroll
-        for (int h = 1; h < 8; h <<= 1)
+        for (int u = 0; u < kU; ++u)
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if ((i & h) == 0) {
-                    const float a = t[i], b = t[i + h];
-                    t[i] = __fadd_rn(a, b);
-                    t[i + h] = __fsub_rn(a, b);
-                }
+            for (int h = 1; h < 8; h <<= 1)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if ((i & h) == 0) {
+                        const float a = t[u][i], b = t[u][i + h];
+                        t[u][i] = __fadd_rn(a, b);
+                        t[u][i + h] = __fsub_rn(a, b);
+                    }
         // butterflies across lanes: h = 8, 16 (, 32, 64): partner lane = lane ^ (h / 8)
 #pragma unroll
         for (uint32_t d = 1; d < kB / 8; d <<= 1) {
             const bool upper = (lane & d) != 0;  // this lane holds the v[i + h] of its pairs
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float p = __shfl_xor_sync(0xFFFFFFFFu, t[i], d);
-                t[i] = upper ? __fsub_rn(p, t[i]) : __fadd_rn(t[i], p);
-            }
+            for (int u = 0; u < kU; ++u)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float p = __shfl_xor_sync(0xFFFFFFFFu, t[u][i], d);
+                    t[u][i] = upper ? __fsub_rn(p, t[u][i]) : __fadd_rn(t[u][i], p);
+                }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) t[i] = __fmul_rn(t[i], c);
-        // MX block (4 lanes) from the binary32 values: abs-max as integers (Inf and NaN
-        // patterns lie above every finite one, so a non-finite block gets scale code 255)
-        uint32_t amax = 0;
+        for (int u = 0; u < kU; ++u) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) amax = max(amax, __float_as_uint(t[i]) & 0x7FFFFFFFu);
-        amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-        amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-        if (!live) continue;
-        const uint32_t eb = amax >> 23;
-        const uint32_t sc = eb == 255u ? 255u : (eb > kEmax ? eb - kEmax : 0u);
-        const float inv = e8m0_inverse(sc);
-        if (FMT == kFmtE2M1) {
-            uint32_t out = 0;
+            for (int i = 0; i < 8; ++i) t[u][i] = __fmul_rn(t[u][i], c);
+            // MX block (4 lanes) from the binary32 values: abs-max as integers (Inf and NaN
+            // patterns lie above every finite one, so a non-finite block gets scale code 255)
+            uint32_t amax = 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                out |= cvt_e2m1x2(__fmul_rn(t[2 * i], inv), __fmul_rn(t[2 * i + 1], inv)) << (8 * i);
-            if (sc == 255u) out = 0;
-            reinterpret_cast<uint32_t*>(codes)[g] = out;
-        } else {
-            uint32_t out[2];
+            for (int i = 0; i < 8; ++i) amax = max(amax, __float_as_uint(t[u][i]) & 0x7FFFFFFFu);
+            amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+            amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+            if (g[u] >= n_groups) continue;
+            const uint32_t eb = amax >> 23;
+            const uint32_t sc = eb == 255u ? 255u : (eb > kEmax ? eb - kEmax : 0u);
+            const float inv = e8m0_inverse(sc);
+            if (FMT == kFmtE2M1) {
+                uint32_t out = 0;
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                out[i] = cvt_e4m3x2(__fmul_rn(t[4 * i], inv), __fmul_rn(t[4 * i + 1], inv)) |
-                         (cvt_e4m3x2(__fmul_rn(t[4 * i + 2], inv), __fmul_rn(t[4 * i + 3], inv)) << 16);
-                if (sc == 255u) out[i] = 0;
+                for (int i = 0; i < 4; ++i)
+                    out |= cvt_e2m1x2(__fmul_rn(t[u][2 * i], inv), __fmul_rn(t[u][2 * i + 1], inv)) << (8 * i);
+                if (sc == 255u) out = 0;
+                reinterpret_cast<uint32_t*>(codes)[g[u]] = out;
+            } else {
+                uint32_t out[2];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    out[i] = cvt_e4m3x2(__fmul_rn(t[u][4 * i], inv), __fmul_rn(t[u][4 * i + 1], inv)) |
+                             (cvt_e4m3x2(__fmul_rn(t[u][4 * i + 2], inv), __fmul_rn(t[u][4 * i + 3], inv)) << 16);
+                    if (sc == 255u) out[i] = 0;
+                }
+                reinterpret_cast<uint2*>(codes)[g[u]] = make_uint2(out[0], out[1]);
             }
-            reinterpret_cast<uint2*>(codes)[g] = make_uint2(out[0], out[1]);
+            if ((lane & 3u) == 0) sf[sf_offset(r[u], kb[u], atoms_k)] = static_cast<uint8_t>(sc);
         }
-        if ((lane & 3u) == 0) sf[sf_offset(r, kb, atoms_k)] = static_cast<uint8_t>(sc);
     }
     // the padding of the tiled scale buffer, as in quantize_kernel
     const uint32_t kbp = atoms_k * 4u;
@@ -376,8 +392,8 @@ cudaError_t launch_quantize_transform(const void* x, int64_t rows, int64_t K, in
     const uint32_t n_groups = static_cast<uint32_t>(rows * K / 8);
     const uint32_t KB = static_cast<uint32_t>(K / 32);
     const uint32_t atoms_k = static_cast<uint32_t>(sf_atoms_k(K));
-    const int64_t want = ceil_div(n_groups, kThreads);
-    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * 16)));
+    const int64_t want = ceil_div(n_groups, kThreads * 4);
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * 8)));
     const uint64_t kb_magic = ((uint64_t(1) << 40) + KB - 1) / KB;
     const uint4* xv = static_cast<const uint4*>(x);
     uint8_t* c = static_cast<uint8_t*>(codes);
