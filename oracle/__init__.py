@@ -88,6 +88,8 @@ def lib():
         L.mxo_fwht_f32.restype = None
         L.mxo_quantize_transformed.argtypes = [vp, i64, i64, vp, i32, i32, vp, vp, vp]
         L.mxo_quantize_transformed.restype = i32
+        L.mxo_linear_lowrank_rows.argtypes = [vp, vp, i32, vp, i64, i64, vp, vp, i64, vp, vp, vp, i64, vp, vp, i32]
+        L.mxo_linear_lowrank_rows.restype = i32
     return _lib
 
 
@@ -291,3 +293,28 @@ def quantize_transformed(x_bits: np.ndarray, fmt: int, B: int, mul: np.ndarray |
     if rc != 0:
         raise ValueError("oracle transform failed (rc=%d)" % rc)
     return codes, sf, t
+
+
+def linear_lowrank_rows(a_codes, a_sf, a_fmt, rows, K, r_codes, r_sf, x_bits, l1t_bits, l2t_bits, bias_bits=None,
+                        nthreads: int | None = None) -> np.ndarray:
+    """fp64 y[rows] = deq(A)[rows] . deq(R)^T + bf16(x[rows] . l1t^T) . l2t^T (+ bias)."""
+    a_codes = np.ascontiguousarray(a_codes, dtype=np.uint8)
+    a_sf = np.ascontiguousarray(a_sf, dtype=np.uint8)
+    r_codes = np.ascontiguousarray(r_codes, dtype=np.uint8)
+    r_sf = np.ascontiguousarray(r_sf, dtype=np.uint8)
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    l1t_bits = np.ascontiguousarray(l1t_bits, dtype=np.uint16)
+    l2t_bits = np.ascontiguousarray(l2t_bits, dtype=np.uint16)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    N, r = l2t_bits.shape
+    y = np.zeros((rows.shape[0], N), dtype=np.float64)
+    bias_p = None
+    if bias_bits is not None:
+        bias_bits = np.ascontiguousarray(bias_bits, dtype=np.uint16)
+        bias_p = _ptr(bias_bits)
+    rc = lib().mxo_linear_lowrank_rows(_ptr(a_codes), _ptr(a_sf), a_fmt, _ptr(rows), rows.shape[0], K,
+                                       _ptr(r_codes), _ptr(r_sf), N, _ptr(x_bits), _ptr(l1t_bits), _ptr(l2t_bits),
+                                       r, bias_p, _ptr(y), nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle low-rank linear failed (rc=%d)" % rc)
+    return y

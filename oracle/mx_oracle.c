@@ -527,3 +527,39 @@ int mxo_quantize_transformed(const uint16_t *x, int64_t rows, int64_t K, const f
     free(t);
     return 0;
 }
+
+/* ---- SVDQuant low-rank branch ---------------------------------------------------- */
+
+/* The blog's best mixed configuration adds SVDQuant ("Results", "Calibration-driven block
+ * selection"): a weight W [N, K] is split offline into a rank-r product B . A kept in 16-bit
+ * (A = l1t [r, K], B = l2t [N, r], bf16) and a residual R = W - B . A quantized to MXFP4.
+ * The linear layer is
+ *   y = deq(xq) . deq(Rq)^T + u . B^T + bias,   u = bf16(x . A^T)  [rows, r],
+ * the branch's activation u being a 16-bit tensor like any linear output (rounded once to
+ * bf16), everything else in fp64.  x_bits are the layer's bf16 inputs [M, K]; the rows
+ * listed are the output rows wanted. */
+int mxo_linear_lowrank_rows(const uint8_t *a_codes, const uint8_t *a_sf, int a_fmt, const int64_t *rows,
+                            int64_t nrows, int64_t K, const uint8_t *r_codes, const uint8_t *r_sf, int64_t N,
+                            const uint16_t *x_bits, const uint16_t *l1t, const uint16_t *l2t, int64_t r,
+                            const uint16_t *bias, double *y, int nthreads)
+{
+    int rc = mxo_linear_rows(a_codes, a_sf, a_fmt, rows, nrows, K, r_codes, r_sf, N, NULL, y, nthreads);
+    if (rc != 0) return rc;
+    double *u = (double *)malloc(sizeof(double) * (size_t)r);
+    for (int64_t i = 0; i < nrows; ++i) {
+        const int64_t m = rows[i];
+        for (int64_t j = 0; j < r; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += mxo_bf16_to_double(x_bits[m * K + k]) * mxo_bf16_to_double(l1t[j * K + k]);
+            u[j] = mxo_bf16_to_double(mxo_double_to_bf16(acc));
+        }
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < r; ++j) acc += u[j] * mxo_bf16_to_double(l2t[n * r + j]);
+            y[i * N + n] += acc + (bias ? mxo_bf16_to_double(bias[n]) : 0.0);
+        }
+    }
+    free(u);
+    return 0;
+}

@@ -50,6 +50,9 @@ MUTANTS = [
     ("hadamard_unnormalized", "for (int i = 0; i < B; ++i) t[b0 + i] = t[b0 + i] * c;",
      "for (int i = 0; i < B; ++i) t[b0 + i] = t[b0 + i] * 1.0f;"),
     ("smoothing_divides", "t[k] = mul ? xk * mul[k] : xk;", "t[k] = mul ? xk / mul[k] : xk;"),
+    ("lowrank_u_not_rounded", "            u[j] = mxo_bf16_to_double(mxo_double_to_bf16(acc));", "            u[j] = acc;"),
+    ("lowrank_l2_transposed", "for (int64_t j = 0; j < r; ++j) acc += u[j] * mxo_bf16_to_double(l2t[n * r + j]);",
+     "for (int64_t j = 0; j < r; ++j) acc += u[j] * mxo_bf16_to_double(l2t[(j * N + n) % (N * r)]);"),
     ("gelu_cancelling_form", "double mxo_gelu(double x) { return 0.5 * x * erfc(-x / sqrt(2.0)); }",
      "double mxo_gelu(double x) { return 0.5 * x * (1.0 + erf(x / sqrt(2.0))); }"),
 ]

@@ -576,3 +576,52 @@ def test_transform_sign_symmetry():
     c1, s1, t1 = oracle.quantize_transformed(bits ^ 0x8000, oracle.E4M3, 128, None)
     assert np.array_equal(t1, -t0) and np.array_equal(s0, s1)
     assert np.array_equal(c1[t0 != 0], c0[t0 != 0] ^ 0x80)
+
+
+# --- SVDQuant low-rank branch ------------------------------------------------------------------
+
+def _lowrank_case(rng, M, N, K, r):
+    a_codes = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    a_sf = rng.integers(120, 132, size=(M, K // 32), dtype=np.uint8)
+    r_codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    r_sf = rng.integers(120, 132, size=(N, K // 32), dtype=np.uint8)
+    bf = lambda a: (np.asarray(a, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)  # noqa: E731
+    x = bf(rng.standard_normal((M, K)))
+    l1t = bf(rng.standard_normal((r, K)) * 0.1)
+    l2t = bf(rng.standard_normal((N, r)) * 0.1)
+    bias = bf(rng.standard_normal(N))
+    return a_codes, a_sf, r_codes, r_sf, x, l1t, l2t, bias
+
+
+def test_lowrank_with_zero_branch_is_the_linear():
+    rng = np.random.default_rng(31)
+    M, N, K, r = 5, 7, 64, 16
+    a_codes, a_sf, r_codes, r_sf, x, l1t, l2t, bias = _lowrank_case(rng, M, N, K, r)
+    zero = np.zeros_like(l1t)
+    y = oracle.linear_lowrank_rows(a_codes, a_sf, oracle.E2M1, np.arange(M), K, r_codes, r_sf, x, zero, l2t, bias)
+    want = oracle.linear_rows(a_codes, a_sf, oracle.E2M1, np.arange(M), K, r_codes, r_sf, bias)
+    assert np.array_equal(y, want)
+
+
+def test_lowrank_brute_force_exact():
+    """Exact rationals: the quantized product, the bf16-rounded branch activation u (its
+    rounding checked against the pinned bf16 rounding) times l2t, and the bias."""
+    rng = np.random.default_rng(32)
+    M, N, K, r = 2, 3, 32, 4
+    a_codes, a_sf, r_codes, r_sf, x, l1t, l2t, bias = _lowrank_case(rng, M, N, K, r)
+    y = oracle.linear_lowrank_rows(a_codes, a_sf, oracle.E2M1, np.arange(M), K, r_codes, r_sf, x, l1t, l2t, bias)
+    f = lambda b: Fraction(oracle.bf16_to_float(int(b)))  # noqa: E731
+    for m in range(M):
+        u = []
+        for j in range(r):
+            exact = sum(f(x[m, k]) * f(l1t[j, k]) for k in range(K))
+            u.append(f(oracle.double_to_bf16(float(exact))))
+        for n in range(N):
+            acc = Fraction(0)
+            for k in range(K):
+                ac = (int(a_codes[m, k // 2]) >> (4 * (k & 1))) & 0xF
+                rc = (int(r_codes[n, k // 2]) >> (4 * (k & 1))) & 0xF
+                acc += (Fraction(oracle.decode_elem(ac, oracle.E2M1)) * Fraction(2) ** (int(a_sf[m, k // 32]) - 127) *
+                        Fraction(oracle.decode_elem(rc, oracle.E2M1)) * Fraction(2) ** (int(r_sf[n, k // 32]) - 127))
+            want = acc + sum(u[j] * f(l2t[n, j]) for j in range(r)) + f(bias[n])
+            assert abs(Fraction(y[m, n]) - want) <= abs(want) * Fraction(1, 10 ** 13) + Fraction(1, 10 ** 300)
