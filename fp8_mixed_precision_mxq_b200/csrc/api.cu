@@ -482,6 +482,48 @@ int mxq_linear_transformed(const void* x_bf16, int64_t M, int64_t K, const void*
     return ok();
 }
 
+int64_t mxq_lowrank_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int64_t rank)
+{
+    const int64_t base = mxq_workspace_bytes(M, N, K, fmt, MXQ_MODE_NATIVE);
+    if (base < 0 || rank <= 0 || rank % 64 != 0 || rank > 256) return -1;
+    return base + round_up(M * rank * 2, kWsAlign) + kLtWorkspace;
+}
+
+int mxq_linear_lowrank(const void* x_bf16, int64_t M, int64_t K, const void* r_codes, const void* r_sf, int64_t N,
+                       const void* bias_bf16, int act_fmt, const void* l1t_bf16, const void* l2t_bf16, int64_t rank,
+                       void* workspace, int64_t ws_bytes, void* y_bf16, void* stream)
+{
+    if (rank <= 0 || rank % 64 != 0 || rank > 256)
+        return fail(MXQ_ERR_INVALID_ARG, "low-rank branch: rank must be 64, 128, 192 or 256 (got %lld)",
+                    (long long)rank);
+    RETURN_IF(check_ptr(x_bf16, "x"));
+    RETURN_IF(check_ptr(l1t_bf16, "l1t"));
+    RETURN_IF(check_ptr(l2t_bf16, "l2t"));
+    RETURN_IF(check_ptr(workspace, "workspace", kWsAlign));
+    RETURN_IF(check_gemm(workspace, workspace, act_fmt, M, K, r_codes, r_sf, N, bias_bf16, y_bf16));
+    const int64_t need = mxq_lowrank_workspace_bytes(M, N, K, act_fmt, rank);
+    if (ws_bytes < need)
+        return fail(MXQ_ERR_WORKSPACE, "workspace has %lld bytes, needs %lld", (long long)ws_bytes, (long long)need);
+    RETURN_IF(check_device());
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* xc = static_cast<uint8_t*>(workspace);
+    uint8_t* xs = xc + round_up(codes_bytes(M, K, act_fmt), kWsAlign);
+    uint8_t* u = xs + round_up(sf_bytes(M, K), kWsAlign);
+    uint8_t* lt = u + round_up(M * rank * 2, kWsAlign);
+    RETURN_IF(cuda_rc(launch_quantize(x_bf16, M, K, act_fmt, xc, xs, st), "quantize launch"));
+    // u = x . l1t^T: [M, K] x [K, rank], a thin plain bf16 GEMM (library)
+    const char* msg = nullptr;
+    int rc = qdq_bf16_gemm(x_bf16, l1t_bf16, nullptr, u, M, rank, K, lt, static_cast<size_t>(kLtWorkspace), st, &msg);
+    if (rc != MXQ_OK) return fail(rc, "low-rank u gemm: %s", msg ? msg : "failed");
+    GemmArgs g{xc, xs, act_fmt, M, N, K, r_codes, r_sf, bias_bf16, y_bf16};
+    g.lr_rank = rank;
+    g.lr_u = u;
+    g.lr_l2t = l2t_bf16;
+    rc = launch_gemm(g, st, &msg, g_path, sizeof g_path);
+    if (rc != MXQ_OK) return fail(rc, "gemm: %s", msg ? msg : "launch failed");
+    return ok();
+}
+
 int mxq_absmax(const void* x_bf16, int64_t n, void* out_f32, void* stream)
 {
     if (n <= 0 || n % 8 != 0) return fail(MXQ_ERR_SHAPE, "absmax: n=%lld must be a positive multiple of 8", (long long)n);

@@ -132,6 +132,9 @@ struct Params {
     int q_rows_pad;
     int write_h;
     float alpha;  // per-tensor activation scale applied to the sums (1 for MX activations)
+    // low-rank branch: stages of 64 K-elements of u (activation, bf16 [M, r]) and B^T
+    // (bf16 [N, r]) MMA'd (kind::f16) into the accumulator before the block-scaled stages
+    int lr_stages;
 };
 
 __device__ __forceinline__ void record_status(uint32_t code) { atomicCAS(&g_device_status, 0u, code); }
@@ -178,6 +181,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                    const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                    const __grid_constant__ CUtensorMap map_y, const __grid_constant__ CUtensorMap map_q,
+                   const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_l2,
                    const Params p)
 {
     using C = Cfg<kPair, kOut>;
@@ -217,6 +221,10 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
         prefetch_tmap(&map_sfb);
         if (kOut == kOutBf16 || p.write_h) prefetch_tmap(&map_y);
         if (kOut != kOutBf16) prefetch_tmap(&map_q);
+        if (p.lr_stages > 0) {
+            prefetch_tmap(&map_u);
+            prefetch_tmap(&map_l2);
+        }
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
@@ -249,13 +257,14 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
             const uint64_t pol_a = policy_evict_normal();  // activations: reused within a group
             constexpr uint32_t kTx = kPair * (C::kStageA + (kW4A8 ? C::kStageB / 2 : C::kStageB) +
                                               AK * 512u * 3u);
+            constexpr uint32_t kTxLr = kPair * (C::kStageA + C::kRowsB * 128u);  // 128-byte rows of u and B^T
             uint32_t it = 0;
             int64_t skipped = -1;
             bool ok = true;
             for (int t = pair_id; t < p.num_tiles && ok; t += n_pairs) {
                 int mb, nb;
                 tile_coords<C::kGroupM>(t, p.m_blocks, p.n_blocks, mb, nb);
-                for (int ks = 0; ks < p.k_stages; ++ks, ++it) {
+                for (int ks = 0; ks < p.lr_stages + p.k_stages; ++ks, ++it) {
                     const uint32_t s = it % S;
                     if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1, kWaitNs)) {
                         record_status(MXQ_ERR_TIMEOUT);
@@ -266,15 +275,25 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                         skipped = 0;  // deliberately leave stage 0 unfilled: the MMA wait runs out
                         continue;
                     }
-                    if (leader) mbar_arrive_expect_tx(&full[s], kTx);
                     const uint32_t bar = kPair == 2 ? mapa_shared(smem_u32(&full[s]), 0) : smem_u32(&full[s]);
-                    tma_load_2d<kPair>(smem + C::kOffA + s * C::kStageA, &map_a, ks * 128,
+                    if (ks < p.lr_stages) {
+                        // low-rank stage: 64 columns of u as A, the same columns of B^T as B
+                        if (leader) mbar_arrive_expect_tx(&full[s], kTxLr);
+                        tma_load_2d<kPair>(smem + C::kOffA + s * C::kStageA, &map_u, ks * 64,
+                                           mb * C::BM + static_cast<int>(rank) * 128, bar, pol_a);
+                        tma_load_2d<kPair>(smem + C::kOffB + s * C::kStageB, &map_l2, ks * 64,
+                                           nb * BN + static_cast<int>(rank) * C::kRowsB, bar, pol_w);
+                        continue;
+                    }
+                    const int kq = ks - p.lr_stages;
+                    if (leader) mbar_arrive_expect_tx(&full[s], kTx);
+                    tma_load_2d<kPair>(smem + C::kOffA + s * C::kStageA, &map_a, kq * 128,
                                        mb * C::BM + static_cast<int>(rank) * 128, bar, pol_a);
-                    tma_load_2d<kPair>(smem + C::kOffB + s * C::kStageB, &map_b, ks * 128,
+                    tma_load_2d<kPair>(smem + C::kOffB + s * C::kStageB, &map_b, kq * 128,
                                        nb * BN + static_cast<int>(rank) * C::kRowsB, bar, pol_w);
-                    tma_load_2d<kPair>(smem + C::kOffSFA + s * C::kStageSFA, &map_sfa, ks * AK * 128,
+                    tma_load_2d<kPair>(smem + C::kOffSFA + s * C::kStageSFA, &map_sfa, kq * AK * 128,
                                        mb * kPair + static_cast<int>(rank), bar, pol_a);
-                    tma_load_2d<kPair>(smem + C::kOffSFB + s * C::kStageSFB, &map_sfb, ks * AK * 128,
+                    tma_load_2d<kPair>(smem + C::kOffSFB + s * C::kStageSFB, &map_sfb, kq * AK * 128,
                                        (nb * BN) / 128, bar, pol_w);
                 }
             }
@@ -316,7 +335,27 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                 tile_coords<C::kGroupM>(t, p.m_blocks, p.n_blocks, mb_t, nb_t);
                 // the tile's first weight row inside its 128-aligned scale window, in 32-row columns
                 const uint32_t sfb_shift = static_cast<uint32_t>(((nb_t * BN) % 128) / 32);
-                for (int ks = 0; ks < p.k_stages; ++ks) {
+                for (int ks = 0; ks < p.lr_stages + p.k_stages; ++ks) {
+                    if (ks < p.lr_stages) {
+                        // low-rank stage: four bf16 MMAs (K = 16 each, 32 bytes of every row);
+                        // the first one of the tile initializes the accumulator
+                        if (!mbar_wait(&full[s], ph, kWaitNs)) {
+                            record_status(MXQ_ERR_TIMEOUT);
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t a_lo = a_lo0 + s * (C::kStageA >> 4);
+                        const uint32_t b_lo = b_lo0 + s * (C::kStageB >> 4);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            mma_bf16<kPair>(acc, a_lo + 2 * j, b_lo + 2 * j, kSdescSw128Hi, idesc_bf16(C::BM, BN),
+                                            (ks > 0 || j > 0) ? 1u : 0u);
+                        tc_commit<kPair>(&empty[s]);
+                        if (++s == S) { s = 0; ph ^= 1; }
+                        continue;
+                    }
+                    const int kq = ks - p.lr_stages;
                     const uint32_t bsf = sfi % kSfBufs;
                     if (!mbar_wait(&full[s], ph, kWaitNs) ||
                         !mbar_wait(&sf_ready[bsf], (sfi / kSfBufs) & 1, kWaitNs)) {
@@ -328,7 +367,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                     const uint32_t sft = tmem_base + kSfCol + bsf * kSfBufCols;
                     const uint32_t a_lo = a_lo0 + s * (C::kStageA >> 4);
                     const uint32_t b_lo = b_lo0 + s * (C::kStageB >> 4);
-                    const int kvalid = p.K - ks * KPS;
+                    const int kvalid = p.K - kq * KPS;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint32_t sf_id = kW4A8 ? static_cast<uint32_t>(j) : static_cast<uint32_t>((j & 1) * 2);
@@ -337,7 +376,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                             mma_block_scaled<kPair, kW4A8>(acc, a_lo + 2 * j, b_lo + 2 * j, kSdescSw128Hi,
                                                            idesc_block_scaled(fa, fb, C::BM, BN, sf_id, sf_id),
                                                            sft + 4 * atom, sft + 8 + 8 * atom + sfb_shift,
-                                                           (ks > 0 || j > 0) ? 1u : 0u);
+                                                           (ks > 0 || j > 0) ? 1u : 0u);  // ks counts low-rank stages
                     }
                     tc_commit<kPair>(&empty[s]);             // stage s free (in both CTAs) after these MMAs
                     tc_commit_local<kPair>(&sf_free[bsf]);  // and so is its scale buffer
@@ -362,7 +401,11 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
             uint32_t s = 0, ph = 0, sfi = 0;
             bool ok = true;
             for (int t = pair_id; t < p.num_tiles && ok; t += n_pairs) {
-                for (int ks = 0; ks < p.k_stages; ++ks, ++sfi) {
+                for (int ks = 0; ks < p.lr_stages + p.k_stages; ++ks) {
+                    if (ks < p.lr_stages) {  // low-rank stages carry no scales: keep the ring position
+                        if (++s == S) { s = 0; ph ^= 1; }
+                        continue;
+                    }
                     const uint32_t bsf = sfi % kSfBufs;
                     if (!mbar_wait(&full[s], ph, kWaitNs) ||
                         !mbar_wait(&sf_free[bsf], ((sfi / kSfBufs) & 1) ^ 1, kWaitNs)) {
@@ -382,6 +425,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                             tc_copy_sf_atom<kPair>(sft + 8 + 8 * a + 4 * h, sdesc_sf_atom(sfb_s + (h * AK + a) * 512));
                     }
                     tc_commit_local<kPair>(&sf_ready[bsf]);  // arrives when the copies (both CTAs) completed
+                    ++sfi;
                     if (++s == S) { s = 0; ph ^= 1; }
                 }
             }
@@ -664,8 +708,9 @@ namespace {
 
 template <bool kW4A8, int kPair, int kOut>
 cudaError_t launch_variant(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa,
-                           const CUtensorMap& msb, const CUtensorMap& my, const CUtensorMap& mq, const Params& p,
-                           int grid, cudaStream_t stream)
+                           const CUtensorMap& msb, const CUtensorMap& my, const CUtensorMap& mq,
+                           const CUtensorMap& mu, const CUtensorMap& ml, const Params& p, int grid,
+                           cudaStream_t stream)
 {
     using C = Cfg<kPair, kOut>;
     auto kern = mx_gemm_kernel<kW4A8, kPair, kOut>;
@@ -683,17 +728,19 @@ cudaError_t launch_variant(const CUtensorMap& ma, const CUtensorMap& mb, const C
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = kPair == 2 ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, my, mq, p);
+    return cudaLaunchKernelEx(&cfg, kern, ma, mb, msa, msb, my, mq, mu, ml, p);
 }
 
 template <bool kW4A8, int kPair>
 cudaError_t launch_out(int out, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa,
-                       const CUtensorMap& msb, const CUtensorMap& my, const CUtensorMap& mq, const Params& p,
-                       int grid, cudaStream_t stream)
+                       const CUtensorMap& msb, const CUtensorMap& my, const CUtensorMap& mq, const CUtensorMap& mu,
+                       const CUtensorMap& ml, const Params& p, int grid, cudaStream_t stream)
 {
-    if (out == kOutGeluE2M1) return launch_variant<kW4A8, kPair, kOutGeluE2M1>(ma, mb, msa, msb, my, mq, p, grid, stream);
-    if (out == kOutGeluE4M3) return launch_variant<kW4A8, kPair, kOutGeluE4M3>(ma, mb, msa, msb, my, mq, p, grid, stream);
-    return launch_variant<kW4A8, kPair, kOutBf16>(ma, mb, msa, msb, my, mq, p, grid, stream);
+    if (out == kOutGeluE2M1)
+        return launch_variant<kW4A8, kPair, kOutGeluE2M1>(ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream);
+    if (out == kOutGeluE4M3)
+        return launch_variant<kW4A8, kPair, kOutGeluE4M3>(ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream);
+    return launch_variant<kW4A8, kPair, kOutBf16>(ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream);
 }
 
 }  // namespace
@@ -707,7 +754,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     const int rows_b = BN / pair;
     const int64_t atoms_k = sf_atoms_k(g.K);
     const int ak = w4a8 ? 1 : 2;
-    CUtensorMap ma, mb, msa, msb, my, mq;
+    CUtensorMap ma, mb, msa, msb, my, mq, mu, ml;
     const uint64_t a_row = w4a8 ? g.K : g.K / 2;
     bool ok = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a_codes, a_row, g.M, a_row, 128, 128,
                           CU_TENSOR_MAP_SWIZZLE_128B);
@@ -734,6 +781,18 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     } else {
         mq = my;  // never used by the bf16 epilogue
     }
+    const int lr_stages = g.lr_rank > 0 ? static_cast<int>(g.lr_rank / 64) : 0;
+    if (lr_stages > 0) {
+        // low-rank operands, bf16 and K-major with K = r: u [M, r] and B^T [N, r], one
+        // 64-element (128-byte) column block per stage, as the A and B tiles of a stage
+        ok = ok && make_map_2d(&mu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.lr_u, g.lr_rank, g.M, g.lr_rank * 2, 64, 128,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+        ok = ok && make_map_2d(&ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.lr_l2t, g.lr_rank, g.N, g.lr_rank * 2, 64,
+                               rows_b, CU_TENSOR_MAP_SWIZZLE_128B);
+    } else {
+        mu = ma;  // never used without a low-rank branch
+        ml = mb;
+    }
     if (!ok) {
         *msg = "cuTensorMapEncodeTiled failed (driver entry point unavailable or invalid operand layout)";
         return MXQ_ERR_CUDA;
@@ -753,6 +812,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     p.q_rows_pad = static_cast<int>(ceil_div(g.M, 128) * 128);
     p.write_h = quant_out && g.y != nullptr ? 1 : 0;
     p.alpha = g.alpha;
+    p.lr_stages = lr_stages;
     const int out = !quant_out ? kOutBf16 : (g.out_fmt == kFmtE4M3 ? kOutGeluE4M3 : kOutGeluE2M1);
 
     int dev = 0, sms = 148;
@@ -761,20 +821,21 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     const int grid = std::min(p.num_tiles, sms / pair) * pair;
     cudaError_t e;
     if (w4a8)
-        e = pair == 2 ? launch_out<true, 2>(out, ma, mb, msa, msb, my, mq, p, grid, stream)
-                      : launch_out<true, 1>(out, ma, mb, msa, msb, my, mq, p, grid, stream);
+        e = pair == 2 ? launch_out<true, 2>(out, ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream)
+                      : launch_out<true, 1>(out, ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream);
     else
-        e = pair == 2 ? launch_out<false, 2>(out, ma, mb, msa, msb, my, mq, p, grid, stream)
-                      : launch_out<false, 1>(out, ma, mb, msa, msb, my, mq, p, grid, stream);
+        e = pair == 2 ? launch_out<false, 2>(out, ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream)
+                      : launch_out<false, 1>(out, ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) {
         *msg = cudaGetErrorString(e);
         return MXQ_ERR_CUDA;
     }
     if (path)
-        snprintf(path, path_len, "native %s %s %dx%d grid %d tiles %d%s", w4a8 ? "mxf8f6f4" : "mxf4",
+        snprintf(path, path_len, "native %s %s %dx%d grid %d tiles %d%s%s", w4a8 ? "mxf8f6f4" : "mxf4",
                  pair == 2 ? "2cta" : "1cta", 128 * pair, BN, grid, p.num_tiles,
-                 !quant_out ? "" : (g.out_fmt == kFmtE4M3 ? " +gelu->e4m3" : " +gelu->e2m1"));
+                 !quant_out ? "" : (g.out_fmt == kFmtE4M3 ? " +gelu->e4m3" : " +gelu->e2m1"),
+                 lr_stages ? " +lowrank(bf16 f16-mma)" : "");
     return MXQ_OK;
 }
 

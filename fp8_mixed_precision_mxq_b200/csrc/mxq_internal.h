@@ -51,6 +51,11 @@ struct GemmArgs {
     void* q_sf = nullptr;
     // per-tensor scale of the activation (static E4M3): y = alpha * acc + bias
     float alpha = 1.0f;
+    // low-rank branch (rank a multiple of 64, or 0): y += u . l2t^T, u bf16 [M, r],
+    // l2t bf16 [N, r]
+    int64_t lr_rank = 0;
+    const void* lr_u = nullptr;
+    const void* lr_l2t = nullptr;
 };
 
 // Builds the tensor maps and launches the tcgen05 GEMM.  Returns an mxq_status;

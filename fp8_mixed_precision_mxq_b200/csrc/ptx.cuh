@@ -308,6 +308,25 @@ __device__ __forceinline__ void mma_block_scaled(uint32_t d_tmem, uint32_t a_lo,
 #undef MXQ_MMA_ASM
 }
 
+// kind::f16 with bf16 A and B (both K-major, the same type as this kind requires), fp32
+// accumulation, K = 16: a 16-bit operand pair added into the same TMEM accumulator the
+// block-scaled MMAs use.  Descriptors as for mma_block_scaled.
+template <int kPair>
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t d_hi, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+#define MXQ_MMA16_ASM(GROUP)                                                                     \
+    asm volatile("{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\t"                                 \
+                 "mov.b64 ad, {%1, %3};\n\tmov.b64 bd, {%2, %3};\n\t"                             \
+                 "setp.ne.b32 p, %5, 0;\n\t"                                                       \
+                 "tcgen05.mma.cta_group::" GROUP ".kind::f16 [%0], ad, bd, %4, p;\n\t}" ::"r"(d_tmem), \
+                 "r"(a_lo), "r"(b_lo), "r"(d_hi), "r"(idesc), "r"(accumulate)                          \
+                 : "memory")
+    if constexpr (kPair == 2) MXQ_MMA16_ASM("2");
+    else MXQ_MMA16_ASM("1");
+#undef MXQ_MMA16_ASM
+}
+
 // kind::mxf8f6f4: 8-bit A (E4M3), B in the byte-padded 4-bit layout (E2M1), K = 32.
 template <int kPair>
 __device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -420,6 +439,18 @@ __host__ __device__ __forceinline__ uint32_t idesc_block_scaled(uint32_t a_fmt, 
     d |= 1u << 23;  // scale type: UE8M0
     d |= ((M >> 4) & 31u) << 24;
     d |= (sfa_id & 3u) << 29;
+    return d;
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B (K-major) and an fp32 accumulator.
+__host__ __device__ __forceinline__ uint32_t idesc_bf16(uint32_t M, uint32_t N)
+{
+    uint32_t d = 0;
+    d |= 1u << 4;   // D format: F32
+    d |= 1u << 7;   // A format: BF16
+    d |= 1u << 10;  // B format: BF16
+    d |= ((N >> 3) & 63u) << 17;
+    d |= ((M >> 4) & 31u) << 24;
     return d;
 }
 

@@ -267,6 +267,46 @@ def linear_transformed(x: torch.Tensor, w: QWeight, fmt="e2m1", block=32, act_mu
     return out
 
 
+def svd_split(w: torch.Tensor, rank: int):
+    """Offline weight preparation of the SVDQuant branch (load time, not the layer's path):
+    w [N, K] bf16 ~= l2t . l1t + residual with the top `rank` singular triplets split as
+    l2t = U_r sqrt(S_r) [N, rank], l1t = sqrt(S_r) V_r^T [rank, K] (bf16), and the residual
+    w - l2t . l1t rounded to bf16 (to be quantized with quantize_weight).  Uses torch's SVD
+    in fp32."""
+    _cuda_bf16(w, "w")
+    U, S, Vh = torch.linalg.svd(w.float(), full_matrices=False)
+    rs = S[:rank].sqrt()
+    l2t = (U[:, :rank] * rs).to(torch.bfloat16).contiguous()
+    l1t = (rs[:, None] * Vh[:rank]).to(torch.bfloat16).contiguous()
+    residual = (w.float() - l2t.float() @ l1t.float()).to(torch.bfloat16).contiguous()
+    return l1t, l2t, residual
+
+
+def lowrank_workspace_bytes(M: int, N: int, K: int, fmt="e2m1", rank=64) -> int:
+    return int(_lib.lib().mxq_lowrank_workspace_bytes(M, N, K, _fmt(fmt), int(rank)))
+
+
+def linear_lowrank(x: torch.Tensor, residual: QWeight, l1t: torch.Tensor, l2t: torch.Tensor, fmt="e2m1",
+                   workspace=None, out=None, stream=None):
+    """y = deq(xq) . deq(Rq)^T + bf16(x . l1t^T) . l2t^T + bias (SVDQuant branch in the
+    same accumulator)."""
+    _cuda_bf16(x, "x")
+    _cuda_bf16(l1t, "l1t")
+    _cuda_bf16(l2t, "l2t")
+    M, K = x.shape
+    rank = l1t.shape[0]
+    f = _fmt(fmt)
+    if workspace is None:
+        workspace = torch.empty(lowrank_workspace_bytes(M, residual.N, K, f, rank), dtype=torch.uint8,
+                                device=x.device)
+    if out is None:
+        out = torch.empty((M, residual.N), dtype=torch.bfloat16, device=x.device)
+    check(_lib.lib().mxq_linear_lowrank(_p(x), M, K, _p(residual.codes), _p(residual.sf), residual.N,
+                                        _p(residual.bias), f, _p(l1t), _p(l2t), rank, _p(workspace),
+                                        workspace.numel(), _p(out), _stream(stream)), "mxq_linear_lowrank")
+    return out
+
+
 def block_workspace_bytes(weights, rows, w4a8_bits: int, mode="native") -> int:
     descs = (WDesc * 8)(*[w.desc() for w in weights])
     ms = (ctypes.c_int64 * 8)(*rows)

@@ -248,6 +248,24 @@ int mxq_linear_transformed(const void* x_bf16, int64_t M, int64_t K, const void*
                            const void* bias_bf16, int act_fmt, const float* act_mul, int block, void* workspace,
                            int64_t ws_bytes, void* y_bf16, void* stream);
 
+/* The SVDQuant low-rank branch of the blog's best mixed result (sections "Results",
+ * "Calibration-driven block selection"): the weight is split offline into a bf16 rank-r
+ * product l2t . l1t (l1t [r, K], l2t [N, r]) and a residual R quantized to MXFP4
+ * (r_codes, r_sf as from mxq_quantize_weight), and the layer computes
+ *   y = bf16( deq(xq) . deq(Rq)^T + u . l2t^T + bias ),  u = bf16(x . l1t^T) [M, r],
+ * x quantized in act_fmt.  u comes from a plain bf16 GEMM (cuBLASLt); u . l2t^T runs as
+ * bf16 tensor-core MMAs (kind::f16) into the same TMEM accumulator as the block-scaled
+ * product, in stages of 64 along r ahead of it.  rank: 64, 128, 192 or 256; l1t, l2t
+ * 16-byte aligned; workspace of mxq_lowrank_workspace_bytes(...) bytes, 256-byte aligned.
+ * Other arguments and errors as for mxq_linear in NATIVE mode. */
+int mxq_linear_lowrank(const void* x_bf16, int64_t M, int64_t K, const void* r_codes, const void* r_sf, int64_t N,
+                       const void* bias_bf16, int act_fmt, const void* l1t_bf16, const void* l2t_bf16, int64_t rank,
+                       void* workspace, int64_t ws_bytes, void* y_bf16, void* stream);
+
+/* Workspace bytes of mxq_linear_lowrank (quantized x, u, and the library GEMM's
+ * workspace), or -1 for invalid arguments. */
+int64_t mxq_lowrank_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int64_t rank);
+
 /* Tiled scale factors -> logical row-major [rows, K/32] bytes (for tests). */
 int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_rowmajor, void* stream);
 

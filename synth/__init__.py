@@ -185,3 +185,16 @@ def sample_rows(M: int, seed: int = 0, tile: int = 128) -> torch.Tensor:
         rows.add(t0 + int(torch.randint(span, (1,), generator=g)))
     return torch.tensor(sorted(rows), dtype=torch.int64)
 
+
+
+def lowrank_weight(N: int, K: int, rank: int, seed: int = 0, device="cpu", std: float = 0.02,
+                   lr_scale: float = 4.0):
+    """A weight with a dominant rank-`rank` part, returned already split as the SVDQuant
+    branch uses it: l1t [rank, K] and l2t [N, rank] (bf16) with l2t . l1t of entry std
+    about lr_scale * std, and a residual [N, K] ~ N(0, std^2) (bf16); W = l2t . l1t + residual."""
+    g = _gen(seed + 3_000_017, device)
+    s = (lr_scale * std / rank ** 0.5) ** 0.5
+    l1t = (torch.randn((rank, K), generator=g, device=device, dtype=torch.float32) * s).to(torch.bfloat16)
+    l2t = (torch.randn((N, rank), generator=g, device=device, dtype=torch.float32) * s).to(torch.bfloat16)
+    residual = (torch.randn((N, K), generator=g, device=device, dtype=torch.float32) * std).to(torch.bfloat16)
+    return l1t, l2t, residual

@@ -158,3 +158,17 @@ def test_transform_entry_points_reject_bad_arguments():
                                     None) == _lib.ERR_INVALID_ARG
     assert L.mxq_linear_transformed(A16, 128, 256, A16, A16, 256, None, 0, None, 32, V(1 << 20), 16, A16,
                                     None) == _lib.ERR_WORKSPACE
+
+
+def test_lowrank_entry_point_rejects_bad_arguments():
+    L = _lib.lib()
+    for bad_rank in (0, 32, 96, 320):
+        assert L.mxq_linear_lowrank(A16, 128, 256, A16, A16, 256, None, 0, A16, A16, bad_rank, V(1 << 20), 1 << 30,
+                                    A16, None) == _lib.ERR_INVALID_ARG
+        assert L.mxq_lowrank_workspace_bytes(128, 256, 256, 0, bad_rank) == -1
+    assert L.mxq_linear_lowrank(A16, 128, 256, A16, A16, 256, None, 0, A8, A16, 64, V(1 << 20), 1 << 30, A16,
+                                None) == _lib.ERR_ALIGN
+    need = L.mxq_lowrank_workspace_bytes(128, 256, 256, 0, 64)
+    assert need > L.mxq_workspace_bytes(128, 256, 256, 0, 0)
+    assert L.mxq_linear_lowrank(A16, 128, 256, A16, A16, 256, None, 0, A16, A16, 64, V(1 << 20), need - 1, A16,
+                                None) == _lib.ERR_WORKSPACE
