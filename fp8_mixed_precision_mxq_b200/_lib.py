@@ -55,6 +55,9 @@ SIGNATURES = {
     "mxq_quantize_act_static": ([_vp, _i64, _i64, ctypes.c_float, _vp, _vp, _vp], _i32),
     "mxq_linear_static": ([_vp, _i64, _i64, _vp, _vp, _i64, _vp, ctypes.c_float, _vp, _i64, _vp, _vp], _i32),
     "mxq_absmax": ([_vp, _i64, _vp, _vp], _i32),
+    "mxq_select_policy": ([ctypes.c_double, ctypes.c_double, _i32], _i32),
+    "mxq_tier_thresholds": ([_i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
+                             ctypes.POINTER(ctypes.c_double)], _i32),
     "mxq_linear_lowrank": ([_vp, _i64, _i64, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _i64, _vp, _i64, _vp, _vp], _i32),
     "mxq_lowrank_workspace_bytes": ([_i64, _i64, _i64, _i32, _i64], _i64),
     "mxq_quantize_act_transformed": ([_vp, _i64, _i64, _i32, _vp, _i32, _vp, _vp, _vp], _i32),

@@ -524,6 +524,31 @@ int mxq_linear_lowrank(const void* x_bf16, int64_t M, int64_t K, const void* r_c
     return ok();
 }
 
+int mxq_tier_thresholds(int tier, double* floor_db, double* w4a8_db, double* margin_db)
+{
+    static const double kTiers[3][3] = {{8.0, 21.0, 0.5}, {10.0, 23.0, 0.5}, {12.0, 25.0, 0.5}};
+    if (tier < MXQ_TIER_LOW || tier > MXQ_TIER_HIGH) return fail(MXQ_ERR_INVALID_ARG, "unknown tier %d", tier);
+    if (floor_db) *floor_db = kTiers[tier][0];
+    if (w4a8_db) *w4a8_db = kTiers[tier][1];
+    if (margin_db) *margin_db = kTiers[tier][2];
+    return ok();
+}
+
+int mxq_select_policy(double sqnr_off, double sqnr_on, int tier)
+{
+    double floor_db, w4a8_db, margin_db;
+    if (mxq_tier_thresholds(tier, &floor_db, &w4a8_db, &margin_db) != MXQ_OK) return -1;
+    if (std::isnan(sqnr_off) || std::isnan(sqnr_on)) {
+        fail(MXQ_ERR_INVALID_ARG, "NaN SQNR");
+        return -1;
+    }
+    const double best = std::max(sqnr_off, sqnr_on);
+    if (best < floor_db) return MXQ_POLICY_BF16;
+    if (best < w4a8_db) return MXQ_POLICY_W4A8;
+    if (sqnr_on - sqnr_off > margin_db) return MXQ_POLICY_TRANSFORM_ON;
+    return MXQ_POLICY_PLAIN_MXFP4;
+}
+
 int mxq_absmax(const void* x_bf16, int64_t n, void* out_f32, void* stream)
 {
     if (n <= 0 || n % 8 != 0) return fail(MXQ_ERR_SHAPE, "absmax: n=%lld must be a positive multiple of 8", (long long)n);

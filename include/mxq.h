@@ -266,6 +266,23 @@ int mxq_linear_lowrank(const void* x_bf16, int64_t M, int64_t K, const void* r_c
  * workspace), or -1 for invalid arguments. */
 int64_t mxq_lowrank_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int64_t rank);
 
+/* The per-block policy of the blog's section "Calibration-driven block selection": from a
+ * block's whole-output SQNR (dB, against the bf16 block) with plain MXFP4 W4A4 (sqnr_off)
+ * and with MXFP4 plus a transform (sqnr_on), in this order of precedence:
+ *   max(off, on) <  floor      -> MXQ_POLICY_BF16       (keep the block in bf16)
+ *   max(off, on) <  w4a8_sqnr  -> MXQ_POLICY_W4A8       (promote to W4A8)
+ *   on - off     >  margin     -> MXQ_POLICY_TRANSFORM_ON (W4A4 with the transform)
+ *   otherwise                  -> MXQ_POLICY_PLAIN_MXFP4
+ * with (floor, w4a8_sqnr, margin) = (8, 21, 0.5) dB for tier LOW, (10, 23, 0.5) for MID and
+ * (12, 25, 0.5) for HIGH, the blog's tier table.  Returns the policy, or -1 for an unknown
+ * tier or a NaN SQNR.  Runs on the host. */
+enum { MXQ_POLICY_PLAIN_MXFP4 = 0, MXQ_POLICY_TRANSFORM_ON = 1, MXQ_POLICY_W4A8 = 2, MXQ_POLICY_BF16 = 3 };
+enum { MXQ_TIER_LOW = 0, MXQ_TIER_MID = 1, MXQ_TIER_HIGH = 2 };
+int mxq_select_policy(double sqnr_off, double sqnr_on, int tier);
+
+/* The thresholds of a tier (dB); returns MXQ_OK or MXQ_ERR_INVALID_ARG. */
+int mxq_tier_thresholds(int tier, double* floor_db, double* w4a8_db, double* margin_db);
+
 /* Tiled scale factors -> logical row-major [rows, K/32] bytes (for tests). */
 int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_rowmajor, void* stream);
 
