@@ -15,6 +15,8 @@ load-time step).  Beside the headline number the JSON line carries:
                 static per-tensor E4M3 activations;
   transform_480p  the transform_on quantizer (smoothing + block Hadamard) and linear on
                 the headline workload;
+  lowrank_480p  the headline linear with an SVDQuant bf16 rank-64 / 128 branch in the same
+                accumulator;
   ffn_720p      the block's FFN with its hidden activation kept MX-quantized (the
                 FFN-up GEMM's epilogue applies GELU and quantizes), FFN-down W4A4 or W4A8;
   dit_block_720p  one DiT block's eight linears under the all-W4A4, all-W4A8 and mixed
@@ -338,6 +340,8 @@ def run_mxq(args):
         result["w4a8"] = bench_w4a8(args, ops, synth, dev, stream, world, rank, peaks)
     if args.transform:
         result["transform_480p"] = bench_transform(args, ops, synth, dev, stream, world, rank, peaks, x, w, b)
+    if args.lowrank:
+        result["lowrank_480p"] = bench_lowrank(args, ops, synth, dev, stream, world, rank, peaks, x, b)
     if args.ffn:
         result["ffn_720p"] = bench_ffn(args, ops, synth, dev, stream, world, rank, peaks)
     if args.block:
@@ -519,6 +523,31 @@ def bench_transform(args, ops, synth, dev, stream, world, rank, peaks, x, w, b):
     return res
 
 
+def bench_lowrank(args, ops, synth, dev, stream, world, rank, peaks, x, b):
+    """The SVDQuant low-rank branch on the headline workload: the linear with a rank-r bf16
+    branch in the same accumulator (u from a thin library GEMM), r = 64 and 128."""
+    c = synth.WORKLOADS["ffn_up_480p_w4a4"]
+    M, K, N = x.shape[0], c["K"], c["N"]
+    iters = max(3, args.steps // 4)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    res = {"workload": "FFN-up 480p (M=%d K=%d N=%d) W4A4 + bf16 rank-r branch" % (M, K, N)}
+    for r in (64, 128):
+        l1t, l2t, resid = synth.lowrank_weight(N, K, r, seed=c["seed"], device=dev)
+        qr = ops.quantize_weight(resid, bias=b)
+        ws = torch.empty(ops.lowrank_workspace_bytes(M, N, K, "e2m1", r), dtype=torch.uint8, device=dev)
+        fn = lambda q=qr, a=l1t, c2=l2t, w=ws: ops.linear_lowrank(x, q, a, c2, "e2m1", workspace=w, out=y)  # noqa
+        for _ in range(2):
+            fn()
+        ms = max_over_ranks(time_loop(fn, iters, stream), world)
+        flops = 2.0 * M * N * K + 2.0 * M * r * (K + N)
+        res["rank%d" % r] = {"ms": round(ms, 4), "TFLOP/s": round(job_tflops(flops, ms, world), 1),
+                             "branch_flop_share": round(2.0 * M * r * (K + N) / flops, 4), "path": ops.last_path()}
+        del ws
+    if ops.poll_status() != 0:
+        raise RuntimeError("device status set during the low-rank measurement")
+    return res
+
+
 def bench_block(args, ops, synth, dev, stream, world, rank, peaks):
     """One DiT block's eight linears at 720p / 81 frames (M = 75600, text context 512)
     through the block entry point, under the three precision masks."""
@@ -691,6 +720,8 @@ def main():
                     help="skip the 720p FFN-up (M=75600) measurement")
     ap.add_argument("--no-transform", dest="transform", action="store_false",
                     help="skip the smoothing + Hadamard quantizer measurement")
+    ap.add_argument("--no-lowrank", dest="lowrank", action="store_false",
+                    help="skip the SVDQuant low-rank branch measurement")
     ap.add_argument("--no-ffn", dest="ffn", action="store_false",
                     help="skip the fused-FFN (M=75600) measurement")
     ap.add_argument("--no-block", dest="block", action="store_false",
