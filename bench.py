@@ -432,6 +432,13 @@ def profile_one(args, ops, x, qw, ws, y, M, N, K, fmt, stream):
     ops.quantize_act(x, fmt, codes=xc, sf=xs)
     if args.only == "gemm":
         fn = lambda: ops.gemm(xc, xs, fmt, M, K, qw, out=y)  # noqa: E731
+    elif args.only == "gelu_quant":
+        hc = torch.empty(ops.codes_bytes(M, N, "e2m1"), dtype=torch.uint8, device=x.device)
+        hs = torch.empty(ops.sf_bytes(M, N), dtype=torch.uint8, device=x.device)
+        fn = lambda: ops.gemm_gelu_quant(xc, xs, fmt, M, K, qw, out_fmt="e2m1", codes=hc, sf=hs)  # noqa: E731
+    elif args.only == "transform":
+        mul = torch.ones(K, dtype=torch.float32, device=x.device)
+        fn = lambda: ops.quantize_act_transformed(x, fmt, 32, mul, codes=xc, sf=xs)  # noqa: E731
     else:
         fn = lambda: ops.quantize_act(x, fmt, codes=xc, sf=xs)  # noqa: E731
     for _ in range(args.warmup):
@@ -781,7 +788,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--M", type=int, default=0, help="override the workload's row count (profiling)")
-    ap.add_argument("--only", choices=["gemm", "quantize"], default=None,
+    ap.add_argument("--only", choices=["gemm", "quantize", "gelu_quant", "transform"], default=None,
                     help="profiling mode: launch only this kernel, --steps times")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
