@@ -218,12 +218,14 @@ int num_sms()
 // values.  Every step is one binary32 operation in a fixed order -- butterflies
 // (a, b) -> (a + b, a - b) for h = 1, 2, 4, ..., kB/2, then the multiply by c -- written
 // with the _rn intrinsics so the compiler cannot fuse them, which makes the codes the
-// exact function of x the definition states.  Lane layout as in quantize_kernel: each
-// lane holds 8 consecutive values, so h = 1, 2, 4 pair values inside a lane and larger h
-// pair lanes (xor-shuffles).
+// exact function of x the definition states.
+// Layout: one lane per 32-element MX block; the 32-point transform, the block's abs-max
+// and its scale byte stay in the lane.  For kB = 128 four consecutive lanes hold one
+// rotation block and the last two butterfly stages (h = 32, 64) pair lanes by
+// xor-shuffles.
 template <int FMT, int kB>
 __global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
-    const uint4* __restrict__ x, uint32_t n_groups, uint32_t KB, uint64_t kb_magic, uint32_t atoms_k, uint32_t rows,
+    const uint4* __restrict__ x, uint32_t n_blocks, uint32_t KB, uint64_t kb_magic, uint32_t atoms_k, uint32_t rows,
     const float* __restrict__ mul, float c, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf)
 {
     static_assert(kB == 32 || kB == 128, "rotation block");
@@ -231,96 +233,121 @@ __global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t nwarps = gridDim.x * (kThreads / 32);
     const uint32_t warp = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-    constexpr int kU = 4;  // independent groups per lane per step (loads in flight)
-    for (uint32_t w0 = warp; w0 * 32u < n_groups; w0 += nwarps * kU) {
-        // n_groups is a multiple of 4 * (kB / 32) lanes' worth, so a rotation block is
-        // either wholly inside the tensor or wholly outside; lanes past the end carry zeros
-        uint32_t g[kU];
-        uint4 v[kU];
+    // The warp's 32 blocks go through shared memory: read from HBM 16 bytes per lane in
+    // order (a contiguous stream), multiplied per channel in that layout (each lane's 8
+    // consecutive channels: coalesced multiplier loads), staged as binary32, then each lane
+    // reads its own block.  Float4 q of block b sits at 8 b + (q ^ (b & 7)), which keeps
+    // both sides free of bank conflicts.  The next span's loads are issued before this
+    // span's work.
+    __shared__ __align__(16) float4 stage[kThreads / 32][256];
+    float4* my = stage[threadIdx.x >> 5];
+    auto load_span = [&](uint32_t b0, uint4 (&v)[4]) {
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            g[u] = (w0 + u * nwarps) * 32u + lane;
-            v[u] = g[u] < n_groups ? ld_stream(x + g[u]) : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t gi = b0 * 4u + 32u * j + lane;  // 16-byte group of the warp's span
+            v[j] = gi < n_blocks * 4u ? ld_stream(x + gi) : make_uint4(0, 0, 0, 0);
         }
-        float t[kU][8];
-        uint32_t r[kU], kb[kU];
+    };
+    uint4 vn[4];
+    // warp-uniform loop: n_blocks is a multiple of kB / 32, so a rotation block is either
+    // wholly inside the tensor or wholly outside; lanes past the end carry zeros
+    load_span(warp * 32u, vn);
+    for (uint32_t base = warp * 32u; base < n_blocks; base += nwarps * 32u) {
+        const uint32_t blk = base + lane;
+        const bool live = blk < n_blocks;
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const uint32_t blk = g[u] >> 2;
-            r[u] = static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(blk) << 24, kb_magic));
-            kb[u] = blk - r[u] * KB;
-            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t gi = base * 4u + 32u * j + lane;
+            const uint32_t w[4] = {vn[j].x, vn[j].y, vn[j].z, vn[j].w};
+            float e[8];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                t[u][2 * i] = lo_f(w[i]);
-                t[u][2 * i + 1] = hi_f(w[i]);
+                e[2 * i] = lo_f(w[i]);
+                e[2 * i + 1] = hi_f(w[i]);
             }
-            if (mul != nullptr && g[u] < n_groups) {
-                const float4* m4 = reinterpret_cast<const float4*>(mul + kb[u] * 32u + (g[u] & 3u) * 8u);
-                const float4 a = __ldg(m4), b = __ldg(m4 + 1);
-                const float mv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            if (mul != nullptr && gi < n_blocks * 4u) {
+                const uint32_t gb = gi >> 2;  // this group's MX block and its row
+                const uint32_t gr = static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(gb) << 24, kb_magic));
+                const float4* m4 = reinterpret_cast<const float4*>(mul + (gb - gr * KB) * 32u + (gi & 3u) * 8u);
+                const float4 m0 = __ldg(m4), m1 = __ldg(m4 + 1);
+                const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
-                for (int i = 0; i < 8; ++i) t[u][i] = __fmul_rn(t[u][i], mv[i]);
+                for (int i = 0; i < 8; ++i) e[i] = __fmul_rn(e[i], mv[i]);
             }
+            const uint32_t bb = 8u * j + (lane >> 2), q = 2u * (lane & 3u);
+            my[8u * bb + (q ^ (bb & 7u))] = make_float4(e[0], e[1], e[2], e[3]);
+            my[8u * bb + ((q + 1u) ^ (bb & 7u))] = make_float4(e[4], e[5], e[6], e[7]);
         }
-        // butterflies inside the lane: h = 1, 2, 4
+        __syncwarp();
+        float t[32];
 #pragma unroll
-        for (int u = 0; u < kU; ++u)
+        for (int q = 0; q < 8; ++q) {
+            const float4 v = my[8u * lane + (static_cast<uint32_t>(q) ^ (lane & 7u))];
+            t[4 * q] = v.x;
+            t[4 * q + 1] = v.y;
+            t[4 * q + 2] = v.z;
+            t[4 * q + 3] = v.w;
+        }
+        __syncwarp();  // every lane has read its block before the next span overwrites them
+        load_span(base + nwarps * 32u, vn);
+        const uint32_t r = static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(blk) << 24, kb_magic));
+        const uint32_t kb = blk - r * KB;
+        // butterflies inside the lane: h = 1, 2, 4, 8, 16
 #pragma unroll
-            for (int h = 1; h < 8; h <<= 1)
+        for (int h = 1; h < 32; h <<= 1)
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    if ((i & h) == 0) {
-                        const float a = t[u][i], b = t[u][i + h];
-                        t[u][i] = __fadd_rn(a, b);
-                        t[u][i + h] = __fsub_rn(a, b);
-                    }
-        // butterflies across lanes: h = 8, 16 (, 32, 64): partner lane = lane ^ (h / 8)
+            for (int i = 0; i < 32; ++i)
+                if ((i & h) == 0) {
+                    const float a = t[i], b = t[i + h];
+                    t[i] = __fadd_rn(a, b);
+                    t[i + h] = __fsub_rn(a, b);
+                }
+        // butterflies across lanes (kB = 128): h = 32, 64 pair lane ^ 1, lane ^ 2
 #pragma unroll
-        for (uint32_t d = 1; d < kB / 8; d <<= 1) {
+        for (uint32_t d = 1; d < kB / 32; d <<= 1) {
             const bool upper = (lane & d) != 0;  // this lane holds the v[i + h] of its pairs
 #pragma unroll
-            for (int u = 0; u < kU; ++u)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float p = __shfl_xor_sync(0xFFFFFFFFu, t[u][i], d);
-                    t[u][i] = upper ? __fsub_rn(p, t[u][i]) : __fadd_rn(t[u][i], p);
-                }
+            for (int i = 0; i < 32; ++i) {
+                const float p = __shfl_xor_sync(0xFFFFFFFFu, t[i], d);
+                t[i] = upper ? __fsub_rn(p, t[i]) : __fadd_rn(t[i], p);
+            }
         }
+        if (!live) continue;
+        // normalization, then the MX block from the binary32 values: abs-max as integers
+        // (Inf and NaN patterns lie above every finite one, so such a block gets code 255)
+        uint32_t amax = 0;
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
+        for (int i = 0; i < 32; ++i) {
+            t[i] = __fmul_rn(t[i], c);
+            amax = max(amax, __float_as_uint(t[i]) & 0x7FFFFFFFu);
+        }
+        const uint32_t eb = amax >> 23;
+        const uint32_t sc = eb == 255u ? 255u : (eb > kEmax ? eb - kEmax : 0u);
+        const float inv = e8m0_inverse(sc);
+        const uint32_t keep = sc == 255u ? 0u : 0xFFFFFFFFu;
+        if (FMT == kFmtE2M1) {
+            uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) t[u][i] = __fmul_rn(t[u][i], c);
-            // MX block (4 lanes) from the binary32 values: abs-max as integers (Inf and NaN
-            // patterns lie above every finite one, so a non-finite block gets scale code 255)
-            uint32_t amax = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) amax = max(amax, __float_as_uint(t[u][i]) & 0x7FFFFFFFu);
-            amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-            amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-            if (g[u] >= n_groups) continue;
-            const uint32_t eb = amax >> 23;
-            const uint32_t sc = eb == 255u ? 255u : (eb > kEmax ? eb - kEmax : 0u);
-            const float inv = e8m0_inverse(sc);
-            if (FMT == kFmtE2M1) {
-                uint32_t out = 0;
+            for (int k = 0; k < 4; ++k) {
+                uint32_t o = 0;
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
-                    out |= cvt_e2m1x2(__fmul_rn(t[u][2 * i], inv), __fmul_rn(t[u][2 * i + 1], inv)) << (8 * i);
-                if (sc == 255u) out = 0;
-                reinterpret_cast<uint32_t*>(codes)[g[u]] = out;
-            } else {
-                uint32_t out[2];
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    out[i] = cvt_e4m3x2(__fmul_rn(t[u][4 * i], inv), __fmul_rn(t[u][4 * i + 1], inv)) |
-                             (cvt_e4m3x2(__fmul_rn(t[u][4 * i + 2], inv), __fmul_rn(t[u][4 * i + 3], inv)) << 16);
-                    if (sc == 255u) out[i] = 0;
-                }
-                reinterpret_cast<uint2*>(codes)[g[u]] = make_uint2(out[0], out[1]);
+                    o |= cvt_e2m1x2(__fmul_rn(t[8 * k + 2 * i], inv), __fmul_rn(t[8 * k + 2 * i + 1], inv)) << (8 * i);
+                w[k] = o & keep;
             }
-            if ((lane & 3u) == 0) sf[sf_offset(r[u], kb[u], atoms_k)] = static_cast<uint8_t>(sc);
+            reinterpret_cast<uint4*>(codes)[blk] = make_uint4(w[0], w[1], w[2], w[3]);
+        } else {
+            uint32_t w[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                w[k] = (cvt_e4m3x2(__fmul_rn(t[4 * k], inv), __fmul_rn(t[4 * k + 1], inv)) |
+                        (cvt_e4m3x2(__fmul_rn(t[4 * k + 2], inv), __fmul_rn(t[4 * k + 3], inv)) << 16)) &
+                       keep;
+            uint4* dst = reinterpret_cast<uint4*>(codes) + static_cast<size_t>(blk) * 2u;
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
         }
+        sf[sf_offset(r, kb, atoms_k)] = static_cast<uint8_t>(sc);
     }
     // the padding of the tiled scale buffer, as in quantize_kernel
     const uint32_t kbp = atoms_k * 4u;
@@ -389,10 +416,10 @@ cudaError_t launch_quantize_static(const void* x, int64_t rows, int64_t K, float
 cudaError_t launch_quantize_transform(const void* x, int64_t rows, int64_t K, int fmt, const float* mul, int block,
                                       float norm, void* codes, void* sf, cudaStream_t stream)
 {
-    const uint32_t n_groups = static_cast<uint32_t>(rows * K / 8);
+    const uint32_t n_blocks = static_cast<uint32_t>(rows * K / 32);
     const uint32_t KB = static_cast<uint32_t>(K / 32);
     const uint32_t atoms_k = static_cast<uint32_t>(sf_atoms_k(K));
-    const int64_t want = ceil_div(n_groups, kThreads * 4);
+    const int64_t want = ceil_div(n_blocks, kThreads);
     const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * 8)));
     const uint64_t kb_magic = ((uint64_t(1) << 40) + KB - 1) / KB;
     const uint4* xv = static_cast<const uint4*>(x);
@@ -401,17 +428,17 @@ cudaError_t launch_quantize_transform(const void* x, int64_t rows, int64_t K, in
     const uint32_t r = static_cast<uint32_t>(rows);
     if (fmt == kFmtE4M3) {
         if (block == 128)
-            quantize_transform_kernel<kFmtE4M3, 128><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k,
+            quantize_transform_kernel<kFmtE4M3, 128><<<grid, kThreads, 0, stream>>>(xv, n_blocks, KB, kb_magic, atoms_k,
                                                                                    r, mul, norm, c, f);
         else
-            quantize_transform_kernel<kFmtE4M3, 32><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k,
+            quantize_transform_kernel<kFmtE4M3, 32><<<grid, kThreads, 0, stream>>>(xv, n_blocks, KB, kb_magic, atoms_k,
                                                                                   r, mul, norm, c, f);
     } else {
         if (block == 128)
-            quantize_transform_kernel<kFmtE2M1, 128><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k,
+            quantize_transform_kernel<kFmtE2M1, 128><<<grid, kThreads, 0, stream>>>(xv, n_blocks, KB, kb_magic, atoms_k,
                                                                                    r, mul, norm, c, f);
         else
-            quantize_transform_kernel<kFmtE2M1, 32><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k,
+            quantize_transform_kernel<kFmtE2M1, 32><<<grid, kThreads, 0, stream>>>(xv, n_blocks, KB, kb_magic, atoms_k,
                                                                                   r, mul, norm, c, f);
     }
     return cudaGetLastError();
