@@ -32,6 +32,21 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi)
     return r;
 }
 
+// Eight fp32 -> one word of eight E2M1 codes (v[i] in nibble i).
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8])
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
+}
+
 // Two fp32 -> two E4M3 codes in a 16-bit word (first argument in the low byte).
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi)
 {

@@ -248,6 +248,14 @@ __global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
             v[j] = gi < n_blocks * 4u ? ld_stream(x + gi) : make_uint4(0, 0, 0, 0);
         }
     };
+    // The multiplier of a 16-byte group starts at channel 8 (g mod G), G = 4 KB groups a
+    // row; g mod G advances by 32 within a span and by 128 nwarps between spans, each step
+    // taken mod G by one conditional subtraction (both operands are below G).
+    const uint32_t G = KB * 4u;
+    const uint32_t step_j = 32u % G;
+    const uint32_t step_span = static_cast<uint32_t>((static_cast<uint64_t>(nwarps) * 128u) % G);
+    uint32_t g0 = static_cast<uint32_t>((static_cast<uint64_t>(warp) * 128u + lane) % G);
+    auto wrap = [G](uint32_t v) { return min(v, v - G); };  // v mod G for v < 2 G
     uint4 vn[4];
     // warp-uniform loop: n_blocks is a multiple of kB / 32, so a rotation block is either
     // wholly inside the tensor or wholly outside; lanes past the end carry zeros
@@ -255,9 +263,9 @@ __global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
     for (uint32_t base = warp * 32u; base < n_blocks; base += nwarps * 32u) {
         const uint32_t blk = base + lane;
         const bool live = blk < n_blocks;
+        uint32_t cg = g0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const uint32_t gi = base * 4u + 32u * j + lane;
             const uint32_t w[4] = {vn[j].x, vn[j].y, vn[j].z, vn[j].w};
             float e[8];
 #pragma unroll
@@ -265,14 +273,13 @@ __global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
                 e[2 * i] = lo_f(w[i]);
                 e[2 * i + 1] = hi_f(w[i]);
             }
-            if (mul != nullptr && gi < n_blocks * 4u) {
-                const uint32_t gb = gi >> 2;  // this group's MX block and its row
-                const uint32_t gr = static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(gb) << 24, kb_magic));
-                const float4* m4 = reinterpret_cast<const float4*>(mul + (gb - gr * KB) * 32u + (gi & 3u) * 8u);
+            if (mul != nullptr) {  // past the tensor's end the zeros times any multiplier stay dead
+                const float4* m4 = reinterpret_cast<const float4*>(mul) + cg * 2u;
                 const float4 m0 = __ldg(m4), m1 = __ldg(m4 + 1);
                 const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
 #pragma unroll
                 for (int i = 0; i < 8; ++i) e[i] = __fmul_rn(e[i], mv[i]);
+                cg = wrap(cg + step_j);
             }
             const uint32_t bb = 8u * j + (lane >> 2), q = 2u * (lane & 3u);
             my[8u * bb + (q ^ (bb & 7u))] = make_float4(e[0], e[1], e[2], e[3]);
@@ -290,6 +297,7 @@ __global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
         }
         __syncwarp();  // every lane has read its block before the next span overwrites them
         load_span(base + nwarps * 32u, vn);
+        g0 = wrap(g0 + step_span);
         const uint32_t r = static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(blk) << 24, kb_magic));
         const uint32_t kb = blk - r * KB;
         // butterflies inside the lane: h = 1, 2, 4, 8, 16
@@ -302,46 +310,54 @@ __global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
                     t[i] = __fadd_rn(a, b);
                     t[i + h] = __fsub_rn(a, b);
                 }
-        // butterflies across lanes (kB = 128): h = 32, 64 pair lane ^ 1, lane ^ 2
+        // butterflies across lanes (kB = 128): h = 32, 64 pair lane ^ 1, lane ^ 2.  The
+        // lane holding v[i] gets v[i] + p, the one holding v[i + h] gets p - v[i + h]: both
+        // are fma(v, sign, p), exact products and one rounding, the IEEE sum or difference.
 #pragma unroll
         for (uint32_t d = 1; d < kB / 32; d <<= 1) {
-            const bool upper = (lane & d) != 0;  // this lane holds the v[i + h] of its pairs
+            const float sgn = (lane & d) != 0 ? -1.f : 1.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float p = __shfl_xor_sync(0xFFFFFFFFu, t[i], d);
-                t[i] = upper ? __fsub_rn(p, t[i]) : __fadd_rn(t[i], p);
-            }
+            for (int i = 0; i < 32; ++i) t[i] = __fmaf_rn(t[i], sgn, __shfl_xor_sync(0xFFFFFFFFu, t[i], d));
         }
         if (!live) continue;
-        // normalization, then the MX block from the binary32 values: abs-max as integers
-        // (Inf and NaN patterns lie above every finite one, so such a block gets code 255)
-        uint32_t amax = 0;
+        // The block's scale comes from max |t c| = fl(max |t| c) (rounding is monotone and
+        // c > 0; a NaN propagates through the max, and Inf or NaN gives exponent field 255,
+        // so such a block gets code 255).  The element codes are cvt(fl(fl(t c) / 2^s)).
+        // For 11 <= code <= 249 that equals cvt(fl(t (c 2^-s))), one multiply: c 2^-s is
+        // a normal binary32, so wherever fl(t c) and the result are normal, scaling by the
+        // power of two commutes with the rounding; where fl(t c) is subnormal, both
+        // results lie at or below 2^-126 2^(127 - 11) = 2^-10, which E2M1 and E4M3 round
+        // to a zero of the value's sign.  Other codes take the two multiplies.
+        float m = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            t[i] = __fmul_rn(t[i], c);
-            amax = max(amax, __float_as_uint(t[i]) & 0x7FFFFFFFu);
-        }
-        const uint32_t eb = amax >> 23;
+        for (int i = 0; i < 32; i += 2)
+            asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(m), "f"(t[i]), "f"(t[i + 1]));
+        const uint32_t eb = (__float_as_uint(__fmul_rn(m, c)) & 0x7FFFFFFFu) >> 23;
         const uint32_t sc = eb == 255u ? 255u : (eb > kEmax ? eb - kEmax : 0u);
-        const float inv = e8m0_inverse(sc);
+        float mult = e8m0_inverse(sc);  // 2^-s, or c 2^-s on the one-multiply path
         const uint32_t keep = sc == 255u ? 0u : 0xFFFFFFFFu;
+        if (sc - 11u <= 249u - 11u) {
+            mult = __fmul_rn(c, mult);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) t[i] = __fmul_rn(t[i], c);
+        }
         if (FMT == kFmtE2M1) {
             uint32_t w[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                uint32_t o = 0;
+                float q[8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    o |= cvt_e2m1x2(__fmul_rn(t[8 * k + 2 * i], inv), __fmul_rn(t[8 * k + 2 * i + 1], inv)) << (8 * i);
-                w[k] = o & keep;
+                for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(t[8 * k + i], mult);
+                w[k] = cvt_e2m1x8(q) & keep;
             }
             reinterpret_cast<uint4*>(codes)[blk] = make_uint4(w[0], w[1], w[2], w[3]);
         } else {
             uint32_t w[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                w[k] = (cvt_e4m3x2(__fmul_rn(t[4 * k], inv), __fmul_rn(t[4 * k + 1], inv)) |
-                        (cvt_e4m3x2(__fmul_rn(t[4 * k + 2], inv), __fmul_rn(t[4 * k + 3], inv)) << 16)) &
+                w[k] = (cvt_e4m3x2(__fmul_rn(t[4 * k], mult), __fmul_rn(t[4 * k + 1], mult)) |
+                        (cvt_e4m3x2(__fmul_rn(t[4 * k + 2], mult), __fmul_rn(t[4 * k + 3], mult)) << 16)) &
                        keep;
             uint4* dst = reinterpret_cast<uint4*>(codes) + static_cast<size_t>(blk) * 2u;
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);

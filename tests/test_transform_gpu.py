@@ -85,3 +85,50 @@ def test_transform_sqnr_report():
         res["smooth+hadamard%d" % block] = _mx.sqnr_db(exact, _mx.bf16_to_f64(sm))
     print("W4A4 SQNR (dB):", {k: round(v, 2) for k, v in res.items()})
     assert min(res.values()) > 10.0
+
+
+def special_input(M, K, seed):
+    """bf16 rows whose 32-value blocks take magnitudes from 2^-140 (bf16 subnormals) to
+    2^126 (the butterflies overflow to Inf there), plus NaN, +-Inf, +-0 and blocks of
+    equal values (their rotation is exact zeros but one)."""
+    g = torch.Generator().manual_seed(seed)
+    exps = torch.tensor([-140, -134, -130, -127, -124, -120, -117, -115, -100, 0, 100, 115, 118, 120, 122, 124, 125,
+                         126], dtype=torch.float64)
+    pick = exps[torch.randint(len(exps), (M, K // 32), generator=g)]
+    x = torch.randn(M, K, generator=g, dtype=torch.float64) * torch.repeat_interleave(2.0 ** pick, 32, dim=1)
+    x = x.to(torch.bfloat16)
+    x[0, 5] = float("nan")
+    x[1, 77] = float("inf")
+    x[2, 300 % K] = float("-inf")
+    x[3] = 0.0
+    x[4, : K // 2] = -0.0
+    x[5, :32] = 1.0
+    x[5, 7] = 1.0 + 2.0 ** -7
+    x[6, 32:64] = 2.0 ** -125
+    return x
+
+
+@pytest.mark.parametrize("fmt", ["e2m1", "e4m3"])
+@pytest.mark.parametrize("block", [32, 128])
+@pytest.mark.parametrize("smooth", [False, True])
+def test_quantize_transformed_special_values(fmt, block, smooth):
+    """Codes and scales bit-exact against the oracle on subnormal, overflowing and
+    non-finite inputs: the binary32 steps round there exactly as the oracle's."""
+    ops = _ops()
+    M, K = 48, 512
+    x = special_input(M, K, seed=block + (7 if smooth else 0))
+    mul = None
+    if smooth:
+        g = torch.Generator().manual_seed(5)
+        mul = (2.0 ** (torch.rand(K, generator=g) * 8.0 - 4.0)).float().contiguous()
+    xd = x.cuda()
+    codes, sf = ops.quantize_act_transformed(xd, fmt, block, None if mul is None else mul.cuda())
+    torch.cuda.synchronize()
+    c_ref, s_ref, _ = oracle.quantize_transformed(_mx.bits(x), _mx.FMT[fmt], block,
+                                                  None if mul is None else mul.numpy())
+    assert (s_ref == 255).any() and (s_ref == 0).any()  # the input reaches both ends of the scale range
+    assert np.array_equal(sf.cpu().numpy(), oracle.sf_to_tiled(s_ref, K))
+    c_gpu = codes.cpu().numpy()
+    bad = np.nonzero(c_gpu != c_ref.reshape(-1))[0]
+    assert bad.size == 0, "%d codes differ, first at byte %d: gpu %#x oracle %#x" % (
+        bad.size, bad[0], c_gpu[bad[0]], c_ref.reshape(-1)[bad[0]])
