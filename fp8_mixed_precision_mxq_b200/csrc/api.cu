@@ -571,10 +571,12 @@ int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_ro
 
 int mxq_poll_status(void* stream)
 {
-    uint32_t v = 0;
+    uint32_t v = 0, q = 0;
     int rc = read_and_clear_device_status(static_cast<cudaStream_t>(stream), &v);
+    if (rc == MXQ_OK) rc = read_and_clear_quant_status(static_cast<cudaStream_t>(stream), &q);
     if (rc != MXQ_OK) return fail(rc, "reading the device status word failed");
     if (v != 0) return fail(static_cast<int>(v), "a GEMM kernel's bounded wait ran out");
+    if (q != 0) return fail(static_cast<int>(q), "a quantizer kernel's bounded wait ran out");
     return ok();
 }
 

@@ -660,6 +660,10 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
 
 // ---------------------------------------------------------------------------- host
 
+uint32_t g_debug_flags = 0;
+
+}  // namespace
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -686,10 +690,6 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
     return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-uint32_t g_debug_flags = 0;
-
-}  // namespace
 
 void set_debug_flags(uint32_t flags) { g_debug_flags = flags; }
 uint32_t debug_flags() { return g_debug_flags; }

@@ -62,8 +62,15 @@ struct GemmArgs {
 // on failure *msg points to a static description.
 int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* path, size_t path_len);
 
-// Device status word written by kernels whose bounded waits ran out.
+// Device status words written by kernels whose bounded waits ran out (the GEMM's and
+// the quantizers'); each call synchronizes the stream, returns the word and clears it.
 int read_and_clear_device_status(cudaStream_t stream, uint32_t* out);
+int read_and_clear_quant_status(cudaStream_t stream, uint32_t* out);
+
+// 2-D tiled tensor map (dims d0 inner, d1 outer; row stride in bytes; box b0 x b1);
+// false if the driver entry point is missing or the encoding is refused.
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+                 uint64_t stride_bytes, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw);
 void set_debug_flags(uint32_t flags);
 uint32_t debug_flags();
 

@@ -13,8 +13,12 @@
 // keeps several 16-byte loads in flight per lane.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+#include <numeric>
+
 #include "mx_elem.cuh"
 #include "mxq_internal.h"
+#include "ptx.cuh"
 
 namespace mxq {
 namespace {
@@ -222,104 +226,134 @@ int num_sms()
 // Layout: one lane per 32-element MX block; the 32-point transform, the block's abs-max
 // and its scale byte stay in the lane.  For kB = 128 four consecutive lanes hold one
 // rotation block and the last two butterfly stages (h = 32, 64) pair lanes by
-// xor-shuffles.
+// xor-shuffles.  Input: x seen as a [n_blocks, 32] bf16 tensor; each warp streams spans
+// of 32 blocks (2 KB) into its own ring of shared-memory stages with TMA (64-byte
+// swizzle: 16-byte chunk q of row r sits at chunk q ^ ((r >> 1) & 3), so the lanes'
+// 16-byte reads of their own rows are free of bank conflicts).
+
+// threads of the transform quantizer's CTAs: 4 warps, 5 CTAs an SM
+constexpr int kTThreads = 128;
+constexpr int kTStages = 3;  // spans in flight per warp
+constexpr uint32_t kSpanBytes = 32u * 64u;
+constexpr uint64_t kTWaitNs = 1000000000ull;
+
+__device__ uint32_t g_quant_status;
+
 template <int FMT, int kB>
-__global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
-    const uint4* __restrict__ x, uint32_t n_blocks, uint32_t KB, uint64_t kb_magic, uint32_t atoms_k, uint32_t rows,
-    const float* __restrict__ mul, float c, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf)
+__global__ void __launch_bounds__(kTThreads, 5) quantize_transform_kernel(
+    const __grid_constant__ CUtensorMap map_x, uint32_t n_blocks, uint32_t KB, uint64_t kb_magic, uint32_t atoms_k,
+    uint32_t rows, const float* __restrict__ mul, float c, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf)
 {
     static_assert(kB == 32 || kB == 128, "rotation block");
     constexpr uint32_t kEmax = FMT == kFmtE4M3 ? 8u : 2u;
+    constexpr int kWarps = kTThreads / 32;
     const uint32_t lane = threadIdx.x & 31u;
-    const uint32_t nwarps = gridDim.x * (kThreads / 32);
-    const uint32_t warp = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-    // The warp's 32 blocks go through shared memory: read from HBM 16 bytes per lane in
-    // order (a contiguous stream), multiplied per channel in that layout (each lane's 8
-    // consecutive channels: coalesced multiplier loads), staged as binary32, then each lane
-    // reads its own block.  Float4 q of block b sits at 8 b + (q ^ (b & 7)), which keeps
-    // both sides free of bank conflicts.  The next span's loads are issued before this
-    // span's work.
-    __shared__ __align__(16) float4 stage[kThreads / 32][256];
-    float4* my = stage[threadIdx.x >> 5];
-    auto load_span = [&](uint32_t b0, uint4 (&v)[4]) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t gi = b0 * 4u + 32u * j + lane;  // 16-byte group of the warp's span
-            v[j] = gi < n_blocks * 4u ? ld_stream(x + gi) : make_uint4(0, 0, 0, 0);
-        }
-    };
-    // The multiplier of a 16-byte group starts at channel 8 (g mod G), G = 4 KB groups a
-    // row; g mod G advances by 32 within a span and by 128 nwarps between spans, each step
-    // taken mod G by one conditional subtraction (both operands are below G).
-    const uint32_t G = KB * 4u;
-    const uint32_t step_j = 32u % G;
-    const uint32_t step_span = static_cast<uint32_t>((static_cast<uint64_t>(nwarps) * 128u) % G);
-    uint32_t g0 = static_cast<uint32_t>((static_cast<uint64_t>(warp) * 128u + lane) % G);
-    auto wrap = [G](uint32_t v) { return min(v, v - G); };  // v mod G for v < 2 G
-    uint4 vn[4];
-    // warp-uniform loop: n_blocks is a multiple of kB / 32, so a rotation block is either
-    // wholly inside the tensor or wholly outside; lanes past the end carry zeros
-    load_span(warp * 32u, vn);
-    for (uint32_t base = warp * 32u; base < n_blocks; base += nwarps * 32u) {
-        const uint32_t blk = base + lane;
-        const bool live = blk < n_blocks;
-        uint32_t cg = g0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t w[4] = {vn[j].x, vn[j].y, vn[j].z, vn[j].w};
-            float e[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                e[2 * i] = lo_f(w[i]);
-                e[2 * i + 1] = hi_f(w[i]);
-            }
-            if (mul != nullptr) {  // past the tensor's end the zeros times any multiplier stay dead
-                const float4* m4 = reinterpret_cast<const float4*>(mul) + cg * 2u;
-                const float4 m0 = __ldg(m4), m1 = __ldg(m4 + 1);
-                const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-#pragma unroll
-                for (int i = 0; i < 8; ++i) e[i] = __fmul_rn(e[i], mv[i]);
-                cg = wrap(cg + step_j);
-            }
-            const uint32_t bb = 8u * j + (lane >> 2), q = 2u * (lane & 3u);
-            my[8u * bb + (q ^ (bb & 7u))] = make_float4(e[0], e[1], e[2], e[3]);
-            my[8u * bb + ((q + 1u) ^ (bb & 7u))] = make_float4(e[4], e[5], e[6], e[7]);
-        }
-        __syncwarp();
-        float t[32];
+    const uint32_t wid = threadIdx.x >> 5;
+    const uint32_t nwarps = gridDim.x * kWarps;
+    const uint32_t warp = blockIdx.x * kWarps + wid;
+    __shared__ __align__(1024) uint8_t ring[kWarps][kTStages][kSpanBytes];
+    __shared__ __align__(8) uint64_t full[kWarps][kTStages];
+    // The launch makes every span of a warp hold the same k-blocks in the same lanes (a
+    // warp has one span, or the warp count times 32 is a multiple of KB), so each lane
+    // loads the multipliers of its 32 channels once and keeps them in registers.
+    float2 mreg[16];
+    if (mul != nullptr) {
+        const uint32_t kb0 = static_cast<uint32_t>((static_cast<uint64_t>(warp) * 32u + lane) % KB);
+        const float4* m4 = reinterpret_cast<const float4*>(mul + kb0 * 32u);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-            const float4 v = my[8u * lane + (static_cast<uint32_t>(q) ^ (lane & 7u))];
-            t[4 * q] = v.x;
-            t[4 * q + 1] = v.y;
-            t[4 * q + 2] = v.z;
-            t[4 * q + 3] = v.w;
+            const float4 v = __ldg(m4 + q);
+            mreg[2 * q] = make_float2(v.x, v.y);
+            mreg[2 * q + 1] = make_float2(v.z, v.w);
         }
-        __syncwarp();  // every lane has read its block before the next span overwrites them
-        load_span(base + nwarps * 32u, vn);
-        g0 = wrap(g0 + step_span);
-        const uint32_t r = static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(blk) << 24, kb_magic));
-        const uint32_t kb = blk - r * KB;
-        // butterflies inside the lane: h = 1, 2, 4, 8, 16
+    }
+    const float2 neg1 = make_float2(-1.f, -1.f);
+    const uint32_t stride = nwarps * 32u;
+    const uint32_t first = warp * 32u;
+    // spans of this warp: first, first + stride, ...; the one with index i sits in stage
+    // i % kTStages, whose barrier completes its (i / kTStages)-th phase when it lands
+    const uint32_t n_spans = first < n_blocks ? (n_blocks - first + stride - 1) / stride : 0u;
+    if (lane == 0) {
+        for (int st = 0; st < kTStages; ++st) mbar_init(&full[wid][st], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    const uint64_t policy = policy_evict_first();
+    auto issue = [&](uint32_t i) {  // lane 0 only
+        const int st = static_cast<int>(i % kTStages);
+        fence_async_smem();  // the lanes' reads of this stage come before the copy's writes
+        mbar_arrive_expect_tx(&full[wid][st], kSpanBytes);
+        tma_load_2d<1>(ring[wid][st], &map_x, 0, static_cast<int32_t>(first + i * stride),
+                       smem_u32(&full[wid][st]), policy);
+    };
+    if (lane == 0)
+        for (uint32_t i = 0; i < n_spans && i < static_cast<uint32_t>(kTStages); ++i) issue(i);
+    for (uint32_t i = 0; i < n_spans; ++i) {
+        const int st = static_cast<int>(i % kTStages);
+        const bool landed = mbar_wait(&full[wid][st], (i / kTStages) & 1u, kTWaitNs);
+        if (!__all_sync(0xFFFFFFFFu, landed)) {
+            // a copy never landed: report it, let the copies still in flight finish
+            // (each wait again bounded), and leave
+            if (lane == 0) {
+                atomicCAS(&g_quant_status, 0u, static_cast<uint32_t>(MXQ_ERR_TIMEOUT));
+                const uint32_t issued = min(n_spans, i + static_cast<uint32_t>(kTStages));
+                for (uint32_t j = i; j < issued; ++j)
+                    mbar_wait(&full[wid][j % kTStages], (j / kTStages) & 1u, kTWaitNs);
+            }
+            __syncwarp();
+            return;
+        }
+        const uint8_t* row = ring[wid][st] + lane * 64u;
+        const uint32_t sw = (lane >> 1) & 3u;
+        uint4 v[4];
 #pragma unroll
-        for (int h = 1; h < 32; h <<= 1)
+        for (int q = 0; q < 4; ++q) v[q] = *reinterpret_cast<const uint4*>(row + 16u * (static_cast<uint32_t>(q) ^ sw));
+        __syncwarp();  // every lane has read the stage before it is refilled
+        if (lane == 0 && i + kTStages < n_spans) issue(i + kTStages);
+        const uint32_t blk = first + i * stride + lane;
+        const bool live = blk < n_blocks;
+        float2 t[16];  // t[k] holds values 2k and 2k + 1 of the lane's block
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if ((i & h) == 0) {
-                    const float a = t[i], b = t[i + h];
-                    t[i] = __fadd_rn(a, b);
-                    t[i + h] = __fsub_rn(a, b);
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t w[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) t[4 * q + e] = make_float2(lo_f(w[e]), hi_f(w[e]));
+        }
+        if (mul != nullptr)
+#pragma unroll
+            for (int k = 0; k < 16; ++k) t[k] = __fmul2_rn(t[k], mreg[k]);
+        // Butterflies inside the lane.  h = 1 pairs the two halves of a register pair and
+        // runs on scalars; h = 2, 4, 8, 16 pair whole register pairs and run as packed
+        // binary32 operations (each half rounded as the scalar one), the difference a - b
+        // as fma(b, -1, a): an exact product and one rounding, the IEEE difference.
+#pragma unroll
+        for (int k = 0; k < 16; ++k) t[k] = make_float2(__fadd_rn(t[k].x, t[k].y), __fsub_rn(t[k].x, t[k].y));
+#pragma unroll
+        for (int m = 1; m < 16; m <<= 1)
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                if ((k & m) == 0) {
+                    const float2 a = t[k], b = t[k + m];
+                    t[k] = __fadd2_rn(a, b);
+                    t[k + m] = __ffma2_rn(b, neg1, a);
                 }
         // butterflies across lanes (kB = 128): h = 32, 64 pair lane ^ 1, lane ^ 2.  The
         // lane holding v[i] gets v[i] + p, the one holding v[i + h] gets p - v[i + h]: both
         // are fma(v, sign, p), exact products and one rounding, the IEEE sum or difference.
 #pragma unroll
         for (uint32_t d = 1; d < kB / 32; d <<= 1) {
-            const float sgn = (lane & d) != 0 ? -1.f : 1.f;
+            const float sg = (lane & d) != 0 ? -1.f : 1.f;
+            const float2 sgn = make_float2(sg, sg);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) t[i] = __fmaf_rn(t[i], sgn, __shfl_xor_sync(0xFFFFFFFFu, t[i], d));
+            for (int k = 0; k < 16; ++k) {
+                const float2 p = make_float2(__shfl_xor_sync(0xFFFFFFFFu, t[k].x, d),
+                                             __shfl_xor_sync(0xFFFFFFFFu, t[k].y, d));
+                t[k] = __ffma2_rn(t[k], sgn, p);
+            }
         }
         if (!live) continue;
+        const uint32_t r = static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(blk) << 24, kb_magic));
+        const uint32_t kb = blk - r * KB;
         // The block's scale comes from max |t c| = fl(max |t| c) (rounding is monotone and
         // c > 0; a NaN propagates through the max, and Inf or NaN gives exponent field 255,
         // so such a block gets code 255).  The element codes are cvt(fl(fl(t c) / 2^s)).
@@ -330,8 +364,8 @@ __global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
         // to a zero of the value's sign.  Other codes take the two multiplies.
         float m = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2)
-            asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(m), "f"(t[i]), "f"(t[i + 1]));
+        for (int k = 0; k < 16; ++k)
+            asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(m), "f"(t[k].x), "f"(t[k].y));
         const uint32_t eb = (__float_as_uint(__fmul_rn(m, c)) & 0x7FFFFFFFu) >> 23;
         const uint32_t sc = eb == 255u ? 255u : (eb > kEmax ? eb - kEmax : 0u);
         float mult = e8m0_inverse(sc);  // 2^-s, or c 2^-s on the one-multiply path
@@ -339,16 +373,19 @@ __global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
         if (sc - 11u <= 249u - 11u) {
             mult = __fmul_rn(c, mult);
         } else {
+            const float2 c2 = make_float2(c, c);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) t[i] = __fmul_rn(t[i], c);
+            for (int k = 0; k < 16; ++k) t[k] = __fmul2_rn(t[k], c2);
         }
+        const float2 mult2 = make_float2(mult, mult);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) t[k] = __fmul2_rn(t[k], mult2);
         if (FMT == kFmtE2M1) {
             uint32_t w[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                float q[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) q[i] = __fmul_rn(t[8 * k + i], mult);
+                const float q[8] = {t[4 * k].x,     t[4 * k].y,     t[4 * k + 1].x, t[4 * k + 1].y,
+                                    t[4 * k + 2].x, t[4 * k + 2].y, t[4 * k + 3].x, t[4 * k + 3].y};
                 w[k] = cvt_e2m1x8(q) & keep;
             }
             reinterpret_cast<uint4*>(codes)[blk] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -356,9 +393,7 @@ __global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
             uint32_t w[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k)
-                w[k] = (cvt_e4m3x2(__fmul_rn(t[4 * k], mult), __fmul_rn(t[4 * k + 1], mult)) |
-                        (cvt_e4m3x2(__fmul_rn(t[4 * k + 2], mult), __fmul_rn(t[4 * k + 3], mult)) << 16)) &
-                       keep;
+                w[k] = (cvt_e4m3x2(t[2 * k].x, t[2 * k].y) | (cvt_e4m3x2(t[2 * k + 1].x, t[2 * k + 1].y) << 16)) & keep;
             uint4* dst = reinterpret_cast<uint4*>(codes) + static_cast<size_t>(blk) * 2u;
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
             dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -371,7 +406,7 @@ __global__ void __launch_bounds__(kThreads) quantize_transform_kernel(
     const uint32_t rows_p = (rows + 127u) & ~127u;
     const uint32_t n_pad_a = rows * pad_k;
     const uint32_t n_pad = n_pad_a + (rows_p - rows) * kbp;
-    for (uint32_t p = blockIdx.x * kThreads + threadIdx.x; p < n_pad; p += gridDim.x * kThreads) {
+    for (uint32_t p = blockIdx.x * kTThreads + threadIdx.x; p < n_pad; p += gridDim.x * kTThreads) {
         uint32_t rr, k;
         if (p < n_pad_a) {
             rr = p / pad_k;
@@ -435,29 +470,53 @@ cudaError_t launch_quantize_transform(const void* x, int64_t rows, int64_t K, in
     const uint32_t n_blocks = static_cast<uint32_t>(rows * K / 32);
     const uint32_t KB = static_cast<uint32_t>(K / 32);
     const uint32_t atoms_k = static_cast<uint32_t>(sf_atoms_k(K));
-    const int64_t want = ceil_div(n_blocks, kThreads);
-    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * 8)));
+    const int64_t want = ceil_div(n_blocks, kTThreads);  // CTAs for one span per warp
+    int64_t grid64 = std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * 32));
+    if (mul != nullptr && grid64 < want) {
+        // several spans per warp: the warp count (4 per CTA) times 32 blocks must be a
+        // multiple of KB, so that the multipliers a lane holds stay the ones of its channels
+        const int64_t m = KB / std::gcd<int64_t>(KB, 32);  // warps
+        const int64_t step = m / std::gcd<int64_t>(m, kTThreads / 32);  // CTAs
+        grid64 = std::max<int64_t>(step, grid64 / step * step);
+    }
+    const int grid = static_cast<int>(grid64);
+    // x as n_blocks rows of 32 bf16 (64 bytes), boxes of 32 rows, 64-byte swizzle; rows
+    // past the end read as zeros
+    CUtensorMap map;
+    if (n_blocks == 0) return cudaSuccess;
+    if (!make_map_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, 32, n_blocks, 64, 32, 32,
+                     CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
     const uint64_t kb_magic = ((uint64_t(1) << 40) + KB - 1) / KB;
-    const uint4* xv = static_cast<const uint4*>(x);
     uint8_t* c = static_cast<uint8_t*>(codes);
     uint8_t* f = static_cast<uint8_t*>(sf);
     const uint32_t r = static_cast<uint32_t>(rows);
     if (fmt == kFmtE4M3) {
         if (block == 128)
-            quantize_transform_kernel<kFmtE4M3, 128><<<grid, kThreads, 0, stream>>>(xv, n_blocks, KB, kb_magic, atoms_k,
-                                                                                   r, mul, norm, c, f);
+            quantize_transform_kernel<kFmtE4M3, 128><<<grid, kTThreads, 0, stream>>>(map, n_blocks, KB, kb_magic, atoms_k,
+                                                                                    r, mul, norm, c, f);
         else
-            quantize_transform_kernel<kFmtE4M3, 32><<<grid, kThreads, 0, stream>>>(xv, n_blocks, KB, kb_magic, atoms_k,
-                                                                                  r, mul, norm, c, f);
+            quantize_transform_kernel<kFmtE4M3, 32><<<grid, kTThreads, 0, stream>>>(map, n_blocks, KB, kb_magic, atoms_k,
+                                                                                   r, mul, norm, c, f);
     } else {
         if (block == 128)
-            quantize_transform_kernel<kFmtE2M1, 128><<<grid, kThreads, 0, stream>>>(xv, n_blocks, KB, kb_magic, atoms_k,
-                                                                                   r, mul, norm, c, f);
+            quantize_transform_kernel<kFmtE2M1, 128><<<grid, kTThreads, 0, stream>>>(map, n_blocks, KB, kb_magic, atoms_k,
+                                                                                    r, mul, norm, c, f);
         else
-            quantize_transform_kernel<kFmtE2M1, 32><<<grid, kThreads, 0, stream>>>(xv, n_blocks, KB, kb_magic, atoms_k,
-                                                                                  r, mul, norm, c, f);
+            quantize_transform_kernel<kFmtE2M1, 32><<<grid, kTThreads, 0, stream>>>(map, n_blocks, KB, kb_magic, atoms_k,
+                                                                                   r, mul, norm, c, f);
     }
     return cudaGetLastError();
+}
+
+int read_and_clear_quant_status(cudaStream_t stream, uint32_t* out)
+{
+    uint32_t v = 0, zero = 0;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MXQ_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, g_quant_status, sizeof v) != cudaSuccess) return MXQ_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_quant_status, &zero, sizeof zero) != cudaSuccess) return MXQ_ERR_CUDA;
+    *out = v;
+    return MXQ_OK;
 }
 
 cudaError_t launch_dequantize(const void* codes, const void* sf, int64_t rows, int64_t K, int fmt, void* out,

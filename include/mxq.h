@@ -36,9 +36,10 @@
  *     multiple of 4; the quantizers write the padding as 0.
  *   - Every call returns an mxq_status.  Arguments are validated before anything
  *     is enqueued, so on an error nothing was launched; mxq_last_error() then
- *     describes it.  Kernel launch failures return MXQ_ERR_CUDA.  The GEMM's
- *     internal waits are bounded; if one ever runs out, the kernel records
- *     MXQ_ERR_TIMEOUT in a device status word that mxq_poll_status() returns.
+ *     describes it.  Kernel launch failures return MXQ_ERR_CUDA.  The internal
+ *     waits of the GEMM and of the transform quantizer are bounded; if one ever runs
+ *     out, the kernel records MXQ_ERR_TIMEOUT in a device status word that
+ *     mxq_poll_status() returns.
  */
 #ifndef MXQ_H
 #define MXQ_H
@@ -286,8 +287,9 @@ int mxq_tier_thresholds(int tier, double* floor_db, double* w4a8_db, double* mar
 /* Tiled scale factors -> logical row-major [rows, K/32] bytes (for tests). */
 int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_rowmajor, void* stream);
 
-/* Synchronizes `stream`, then returns (and clears) the device status word: MXQ_OK,
- * or MXQ_ERR_TIMEOUT if a bounded wait of a GEMM kernel ran out since the last poll. */
+/* Synchronizes `stream`, then returns (and clears) the device status words: MXQ_OK,
+ * or MXQ_ERR_TIMEOUT if a bounded wait of a GEMM or transform-quantizer kernel ran out
+ * since the last poll. */
 int mxq_poll_status(void* stream);
 
 /* Debug flags (0 = none).  Bit 0: the GEMM's producer skips the first stage's load,

@@ -132,3 +132,23 @@ def test_quantize_transformed_special_values(fmt, block, smooth):
     bad = np.nonzero(c_gpu != c_ref.reshape(-1))[0]
     assert bad.size == 0, "%d codes differ, first at byte %d: gpu %#x oracle %#x" % (
         bad.size, bad[0], c_gpu[bad[0]], c_ref.reshape(-1)[bad[0]])
+
+
+@pytest.mark.parametrize("fmt", ["e2m1", "e4m3"])
+@pytest.mark.parametrize("block", [32, 128])
+@pytest.mark.parametrize("M,K", [(9000, 2176), (4000, 5120)])
+def test_quantize_transformed_multi_span(fmt, block, M, K):
+    """Tensors of more MX blocks than the launch has lanes (148 SMs x 32 CTAs x 128), so
+    every warp takes several spans and the per-channel multipliers it holds must stay the
+    ones of its channels; K = 2176 and 5120 make the launch round its grid to multiples of
+    17 and 5 CTAs.  Whole tensor bit-exact against the oracle."""
+    ops = _ops()
+    x = synth.activation(M, K, "student_t", seed=M + block, device="cuda", outlier_frac=0.02, outlier_scale=40.0)
+    mul = (1.0 / smooth_scales(x)).contiguous()
+    codes, sf = ops.quantize_act_transformed(x, fmt, block, mul)
+    torch.cuda.synchronize()
+    c_ref, s_ref, _ = oracle.quantize_transformed(_mx.bits(x), _mx.FMT[fmt], block, mul.cpu().numpy())
+    assert np.array_equal(sf.cpu().numpy(), oracle.sf_to_tiled(s_ref, K))
+    c_gpu = codes.cpu().numpy()
+    bad = np.nonzero(c_gpu != c_ref.reshape(-1))[0]
+    assert bad.size == 0, "%d codes differ, first at byte %d (row %d)" % (bad.size, bad[0], bad[0] // (c_gpu.size // M))
