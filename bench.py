@@ -62,8 +62,8 @@ GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precisio
                 "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h"]
 GEMM_TRAFFIC = {
     ("ffn_up_480p_w4a4", 32760): {
-        "bytes": 585765120 + 860025856,
-        "sources_sha256": "0566dc121fd2321a8672a6f0e65913c6edd4da954ce60f78fa3523a82b46facf",
+        "bytes": 535662848 + 858918144,
+        "sources_sha256": "e1c9d29169a1130aa0cdab70d735b03c652f3e0d4e9e845b28d6eb1fc14da8c8",
         "profile": "profiles/mx_gemm_mxf4_pair_ffn_up_480p_traffic.md"},
 }
 

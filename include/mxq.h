@@ -293,7 +293,9 @@ int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_ro
 int mxq_poll_status(void* stream);
 
 /* Debug flags (0 = none).  Bit 0: the GEMM's producer skips the first stage's load,
- * so the consumer's bounded wait runs out and the kernel reports MXQ_ERR_TIMEOUT. */
+ * so the consumer's bounded wait runs out and the kernel reports MXQ_ERR_TIMEOUT.
+ * Bit 1: the transform quantizer's first warp skips its first span's copy, with the
+ * same outcome. */
 int mxq_set_debug(uint32_t flags);
 
 /* Thread-local description of the last error, and of the last path taken

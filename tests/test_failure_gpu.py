@@ -67,3 +67,32 @@ def test_quantize_and_gemm_still_match_oracle_after_timeout():
     wc, ws, _ = _mx.oracle_quantize(w, "e2m1")
     y_ref = oracle.linear(xc, xs, _mx.FMT["e2m1"], K, wc, ws)
     _mx.assert_gemm_close(_mx.bf16_to_f64(y), y_ref, "linear after a timed-out launch")
+
+
+@pytest.mark.parametrize("block", [32, 128])
+def test_transform_quantizer_bounded_wait_reports_timeout(block):
+    """Debug bit 1: the transform quantizer's first warp never issues its first span's
+    copy, so that warp's bounded wait (one second) runs out; the kernel records
+    MXQ_ERR_TIMEOUT, waits for its other copies and returns, and the next call with the
+    flag cleared gives the clean result."""
+    from fp8_mixed_precision_mxq_b200 import _lib, ops
+    M, K = 300, 1024
+    x = synth.activation(M, K, "student_t", seed=31, device="cuda")
+    mul = torch.rand(K, device="cuda", dtype=torch.float32) + 0.5
+    c_clean, s_clean = ops.quantize_act_transformed(x, "e2m1", block, mul)
+    assert ops.poll_status() == _lib.OK
+    ops.set_debug(2)
+    try:
+        t0 = time.monotonic()
+        ops.quantize_act_transformed(x, "e2m1", block, mul)
+        status = ops.poll_status()
+        elapsed = time.monotonic() - t0
+    finally:
+        ops.set_debug(0)
+    assert status == _lib.ERR_TIMEOUT, _lib.STATUS_NAMES.get(status, status)
+    assert "quantizer" in _lib.last_error()
+    assert elapsed < 30.0, "the kernel took %.1f s to wind down" % elapsed
+    assert ops.poll_status() == _lib.OK
+    c_again, s_again = ops.quantize_act_transformed(x, "e2m1", block, mul)
+    assert ops.poll_status() == _lib.OK
+    assert torch.equal(c_again, c_clean) and torch.equal(s_again, s_clean)
