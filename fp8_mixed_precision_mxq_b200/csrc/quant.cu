@@ -60,9 +60,11 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
     const uint32_t nwarps = gridDim.x * (kThreads / 32);
     const uint32_t warp = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
 
+    static_assert(kUnroll == 8, "the scale bytes of a step are stored two per lane");
     for (uint32_t w0 = warp; w0 * 32u < n_groups; w0 += nwarps * kUnroll) {
         uint4 v[kUnroll];
         uint32_t g[kUnroll];
+        uint32_t scw[2] = {0u, 0u};  // the scale codes of this quad's block for u = 0..7, a byte each
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             g[u] = (w0 + u * nwarps) * 32u + lane;
@@ -89,32 +91,40 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
                 inv = __uint_as_float((254u - min(sc, 253u)) << 23);  // 2^(127 - sc)
             }
             const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            // x * 2^-s, two lanes of binary32 a multiply (each rounded as the scalar one)
+            const float2 inv2 = make_float2(inv, inv);
+            float2 f[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) f[i] = __fmul2_rn(make_float2(lo_f(w[i]), hi_f(w[i])), inv2);
+            const uint32_t keep = sc == 255u ? 0u : 0xFFFFFFFFu;
             // cvt rounds to nearest even, saturates, and keeps the sign of a value that
             // rounds to zero (-0 = 0x8 / 0x80), as the format reading requires
             if (kElem == kFmtE2M1) {
-                uint32_t out = 0;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) out |= cvt_e2m1x2(lo_f(w[i]) * inv, hi_f(w[i]) * inv) << (8 * i);
-                if (sc == 255u) out = 0;
-                reinterpret_cast<uint32_t*>(codes)[g[u]] = out;
+                const float q[8] = {f[0].x, f[0].y, f[1].x, f[1].y, f[2].x, f[2].y, f[3].x, f[3].y};
+                reinterpret_cast<uint32_t*>(codes)[g[u]] = cvt_e2m1x8(q) & keep;
             } else {
                 uint32_t out[2];
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const uint32_t a = w[2 * i], b = w[2 * i + 1];
-                    out[i] = cvt_e4m3x2(lo_f(a) * inv, hi_f(a) * inv) |
-                             (cvt_e4m3x2(lo_f(b) * inv, hi_f(b) * inv) << 16);
-                    if (sc == 255u) out[i] = 0;
-                }
+                for (int i = 0; i < 2; ++i)
+                    out[i] = (cvt_e4m3x2(f[2 * i].x, f[2 * i].y) | (cvt_e4m3x2(f[2 * i + 1].x, f[2 * i + 1].y) << 16)) &
+                             keep;
                 reinterpret_cast<uint2*>(codes)[g[u]] = make_uint2(out[0], out[1]);
             }
-            if ((lane & 3u) == 0) {
-                const uint32_t blk = g[u] >> 2;
+            scw[u >> 2] |= sc << (8 * (u & 3));
+        }
+        // The step's 64 scale bytes (8 blocks for each u), two per lane: lane 4 q + j
+        // stores those of block q for u = j and u = j + 4.
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t u = (lane & 3u) + 4u * h;
+            const uint32_t gq = (w0 + u * nwarps) * 32u + (lane & ~3u);  // the block's first group
+            if (gq < n_groups) {
+                const uint32_t blk = gq >> 2;
                 // (blk * kb_magic) >> 40 without a 64-bit overflow: blk < 2^29 and
                 // kb_magic <= 2^40, so the product needs up to 69 bits
                 const uint32_t r = static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(blk) << 24, kb_magic));
                 const uint32_t kb = blk - r * KB;
-                sf[sf_offset(r, kb, atoms_k)] = static_cast<uint8_t>(sc);
+                sf[sf_offset(r, kb, atoms_k)] = static_cast<uint8_t>(scw[h] >> (8u * (lane & 3u)));
             }
         }
     }
