@@ -469,13 +469,17 @@ def bench_target(args, ops, synth, dev, stream, world, rank, peaks, qw, b):
     off = (ops.codes_bytes(M, K, "e2m1") + 255) // 256 * 256
     xs = ws[off: off + ops.sf_bytes(M, K)]
     g_ms = max_over_ranks(time_loop(lambda: ops.gemm(xc, xs, "e2m1", M, K, qw, out=y), iters, stream), world)
+    q_ms = max_over_ranks(time_loop(lambda: ops.quantize_act(x, "e2m1", codes=xc, sf=xs), iters, stream), world)
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     if ops.poll_status() != 0:
         raise RuntimeError("device status set during the 720p measurement")
+    q_gbs = quant_bytes(M, K, "e2m1") / (q_ms * 1e-3) / 1e9
     return {"workload": "ffn_up_720p_w4a4: M=%d K=%d N=%d W4A4" % (M, K, N),
             "linear": {"ms": round(ms, 4), "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 1)},
             "gemm": {"ms": round(g_ms, 4), "TFLOP/s": round(flops / (g_ms * 1e-3) / 1e12, 1),
-                     "frac_fp4": round(flops / (g_ms * 1e-3) / 1e12 / fp4_peak, 4)}}
+                     "frac_fp4": round(flops / (g_ms * 1e-3) / 1e12 / fp4_peak, 4)},
+            "quantize": {"ms": round(q_ms, 4), "GB/s": round(q_gbs, 1),
+                         "frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4)}}
 
 
 def linears_roofline_ms(synth, rows_x, rows_ctx, bits, peaks):

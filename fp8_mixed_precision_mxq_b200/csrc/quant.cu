@@ -26,12 +26,18 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kUnroll = 8;  // 16-byte loads in flight per lane per step
 
+// The quantizers stream their input once and write their output once: the loads carry
+// an L2 evict-first policy and bypass L1, the code stores are streaming (.cs) stores, so
+// neither side keeps lines in L2 that the next launch's stream would have to evict
+// (measured on the 720p activations: +7 % for E2M1, +13 % for E4M3).
 __device__ __forceinline__ uint4 ld_stream(const uint4* p)
 {
     uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+    uint64_t pol;
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
+                 : "l"(p), "l"(pol));
     return v;
 }
 
@@ -101,14 +107,14 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
             // rounds to zero (-0 = 0x8 / 0x80), as the format reading requires
             if (kElem == kFmtE2M1) {
                 const float q[8] = {f[0].x, f[0].y, f[1].x, f[1].y, f[2].x, f[2].y, f[3].x, f[3].y};
-                reinterpret_cast<uint32_t*>(codes)[g[u]] = cvt_e2m1x8(q) & keep;
+                __stcs(reinterpret_cast<unsigned int*>(codes) + g[u], cvt_e2m1x8(q) & keep);
             } else {
                 uint32_t out[2];
 #pragma unroll
                 for (int i = 0; i < 2; ++i)
                     out[i] = (cvt_e4m3x2(f[2 * i].x, f[2 * i].y) | (cvt_e4m3x2(f[2 * i + 1].x, f[2 * i + 1].y) << 16)) &
                              keep;
-                reinterpret_cast<uint2*>(codes)[g[u]] = make_uint2(out[0], out[1]);
+                __stcs(reinterpret_cast<uint2*>(codes) + g[u], make_uint2(out[0], out[1]));
             }
             scw[u >> 2] |= sc << (8 * (u & 3));
         }
@@ -403,15 +409,15 @@ __global__ void __launch_bounds__(kTThreads, 5) quantize_transform_kernel(
                                     t[4 * k + 2].x, t[4 * k + 2].y, t[4 * k + 3].x, t[4 * k + 3].y};
                 w[k] = cvt_e2m1x8(q) & keep;
             }
-            reinterpret_cast<uint4*>(codes)[blk] = make_uint4(w[0], w[1], w[2], w[3]);
+            __stcs(reinterpret_cast<uint4*>(codes) + blk, make_uint4(w[0], w[1], w[2], w[3]));
         } else {
             uint32_t w[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k)
                 w[k] = (cvt_e4m3x2(t[2 * k].x, t[2 * k].y) | (cvt_e4m3x2(t[2 * k + 1].x, t[2 * k + 1].y) << 16)) & keep;
             uint4* dst = reinterpret_cast<uint4*>(codes) + static_cast<size_t>(blk) * 2u;
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            __stcs(dst, make_uint4(w[0], w[1], w[2], w[3]));
+            __stcs(dst + 1, make_uint4(w[4], w[5], w[6], w[7]));
         }
         sf[sf_offset(r, kb, atoms_k)] = static_cast<uint8_t>(sc);
     }
