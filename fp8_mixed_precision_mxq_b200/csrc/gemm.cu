@@ -113,7 +113,7 @@ struct Cfg {
     static constexpr int kEpiWarps = kEpiWarpsOf<kOut>;
     static constexpr uint32_t kOffQ = kOffEpi + kEpiWarps * 2 * kEpiBuf;
     static constexpr uint32_t kOffBar = kOffQ + (kOut ? kEpiWarps * 2 * kQBuf : 0u);
-    static constexpr uint32_t kNumBars = 2 * kStages + 6 + 2 * 3;
+    static constexpr uint32_t kNumBars = 2 * kStages + 6 + 2 * kSfBufs;
     static constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16;
     static constexpr int kGroupM = kPair == 2 ? 8 : 16;  // tile rows per rasterization group
     static_assert(kSmemBytes <= 232448, "shared memory budget");
