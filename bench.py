@@ -62,8 +62,8 @@ GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precisio
                 "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h"]
 GEMM_TRAFFIC = {
     ("ffn_up_480p_w4a4", 32760): {
-        "bytes": 535662848 + 858918144,
-        "sources_sha256": "e1c9d29169a1130aa0cdab70d735b03c652f3e0d4e9e845b28d6eb1fc14da8c8",
+        "bytes": 566400256 + 859681536,
+        "sources_sha256": "5e0deadca84c75f0a1e94ff788b6eb4d1399e1e0aa023d5d0b6aa5e7878ea51d",
         "profile": "profiles/mx_gemm_mxf4_pair_ffn_up_480p_traffic.md"},
 }
 
