@@ -145,23 +145,25 @@ __device__ __forceinline__ void record_status(uint32_t code) { atomicCAS(&g_devi
 // error below 1.2e-7; the other side from erfc(-z) = 2 - erfc(z).  Relative accuracy
 // holds in the negative tail, where GELU is tiny (1 + erf would cancel there).  Below
 // x of about -13 the exponential underflows and the result is -0.
-__device__ __forceinline__ float gelu_f32(float x)
+// Two values at a time: the multiplies and fused multiply-adds run packed (each half
+// rounded as the scalar operation would be), the reciprocal and the exponential scalar.
+__device__ __forceinline__ float2 gelu2_f32(float2 x)
 {
-    const float z = fabsf(x) * 0.70710678118654752f;
-    const float t = __fdividef(1.0f, fmaf(0.5f, z, 1.0f));
-    float q = 0.17087277f;
-    q = fmaf(q, t, -0.82215223f);
-    q = fmaf(q, t, 1.48851587f);
-    q = fmaf(q, t, -1.13520398f);
-    q = fmaf(q, t, 0.27886807f);
-    q = fmaf(q, t, -0.18628806f);
-    q = fmaf(q, t, 0.09678418f);
-    q = fmaf(q, t, 0.37409196f);
-    q = fmaf(q, t, 1.00002368f);
-    q = fmaf(q, t, -1.26551223f);
-    const float e = t * __expf(fmaf(-z, z, q));  // erfc(z)
-    const float phi = x <= 0.0f ? 0.5f * e : fmaf(-0.5f, e, 1.0f);
-    return x * phi;
+    const float2 one = make_float2(1.0f, 1.0f), half = make_float2(0.5f, 0.5f);
+    const float2 z = __fmul2_rn(make_float2(fabsf(x.x), fabsf(x.y)),
+                                make_float2(0.70710678118654752f, 0.70710678118654752f));
+    const float2 d = __ffma2_rn(half, z, one);
+    const float2 t = make_float2(__fdividef(1.0f, d.x), __fdividef(1.0f, d.y));
+    const float c[10] = {0.17087277f, -0.82215223f, 1.48851587f, -1.13520398f, 0.27886807f,
+                         -0.18628806f, 0.09678418f, 0.37409196f, 1.00002368f, -1.26551223f};
+    float2 q = make_float2(c[0], c[0]);
+#pragma unroll
+    for (int i = 1; i < 10; ++i) q = __ffma2_rn(q, t, make_float2(c[i], c[i]));
+    const float2 a = __ffma2_rn(make_float2(-z.x, -z.y), z, q);
+    const float2 e = __fmul2_rn(t, make_float2(__expf(a.x), __expf(a.y)));  // erfc(z)
+    const float2 lo = __fmul2_rn(half, e), hi = __ffma2_rn(make_float2(-0.5f, -0.5f), e, one);
+    const float2 phi = make_float2(x.x <= 0.0f ? lo.x : hi.x, x.y <= 0.0f ? lo.y : hi.y);
+    return __fmul2_rn(x, phi);
 }
 
 template <int kGroupM>
@@ -507,14 +509,15 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                     }
                     // o: the chunk in bf16 -- y = acc + bias, or h = GELU of that rounded to bf16
                     uint32_t o[16];
+                    const float2 alpha2 = make_float2(p.alpha, p.alpha);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 y2 = __floats2bfloat162_rn(fmaf(__uint_as_float(acc[2 * i]), p.alpha, bv[2 * i]),
-                                                                  fmaf(__uint_as_float(acc[2 * i + 1]), p.alpha,
-                                                                       bv[2 * i + 1]));
+                        const float2 y = __ffma2_rn(make_float2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1])),
+                                                    alpha2, make_float2(bv[2 * i], bv[2 * i + 1]));
+                        __nv_bfloat162 y2 = __floats2bfloat162_rn(y.x, y.y);
                         if constexpr (kOut != kOutBf16) {
-                            const float y0 = __low2float(y2), y1 = __high2float(y2);
-                            y2 = __floats2bfloat162_rn(gelu_f32(y0), gelu_f32(y1));
+                            const float2 g = gelu2_f32(make_float2(__low2float(y2), __high2float(y2)));
+                            y2 = __floats2bfloat162_rn(g.x, g.y);
                         }
                         o[i] = *reinterpret_cast<uint32_t*>(&y2);
                     }
@@ -544,22 +547,28 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                         uint8_t* qb = qbuf0 + eb * C::kQBuf;
                         if constexpr (kOut == kOutGeluE2M1) {
                             uint32_t cw[4];
+                            const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
                             for (int k = 0; k < 4; ++k) {
-                                uint32_t w = 0;
+                                float v[8];
 #pragma unroll
-                                for (int i = 0; i < 4; ++i)
-                                    w |= cvt_e2m1x2(lo_f(o[4 * k + i]) * inv, hi_f(o[4 * k + i]) * inv) << (8 * i);
-                                cw[k] = w & keep;
+                                for (int i = 0; i < 4; ++i) {
+                                    const float2 f = __fmul2_rn(make_float2(lo_f(o[4 * k + i]), hi_f(o[4 * k + i])), inv2);
+                                    v[2 * i] = f.x;
+                                    v[2 * i + 1] = f.y;
+                                }
+                                cw[k] = cvt_e2m1x8(v) & keep;
                             }
                             *reinterpret_cast<uint4*>(qb + lane * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
                         } else {
                             uint32_t cw[8];
+                            const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                cw[k] = (cvt_e4m3x2(lo_f(o[2 * k]) * inv, hi_f(o[2 * k]) * inv) |
-                                         (cvt_e4m3x2(lo_f(o[2 * k + 1]) * inv, hi_f(o[2 * k + 1]) * inv) << 16)) &
-                                        keep;
+                            for (int k = 0; k < 8; ++k) {
+                                const float2 f0 = __fmul2_rn(make_float2(lo_f(o[2 * k]), hi_f(o[2 * k])), inv2);
+                                const float2 f1 = __fmul2_rn(make_float2(lo_f(o[2 * k + 1]), hi_f(o[2 * k + 1])), inv2);
+                                cw[k] = (cvt_e4m3x2(f0.x, f0.y) | (cvt_e4m3x2(f1.x, f1.y) << 16)) & keep;
+                            }
                             *reinterpret_cast<uint4*>(qb + lane * 32) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
                             *reinterpret_cast<uint4*>(qb + lane * 32 + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
                         }
