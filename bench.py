@@ -62,8 +62,8 @@ GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precisio
                 "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h"]
 GEMM_TRAFFIC = {
     ("ffn_up_480p_w4a4", 32760): {
-        "bytes": 566400256 + 859681536,
-        "sources_sha256": "5e0deadca84c75f0a1e94ff788b6eb4d1399e1e0aa023d5d0b6aa5e7878ea51d",
+        "bytes": 589257984 + 859933440,
+        "sources_sha256": "166a3b24c5e4ff2dfe37203b6c8d42fd8a1e619f6329701c1440256fb440e787",
         "profile": "profiles/mx_gemm_mxf4_pair_ffn_up_480p_traffic.md"},
 }
 
