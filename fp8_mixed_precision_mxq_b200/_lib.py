@@ -21,6 +21,8 @@ STATUS_NAMES = {0: "MXQ_OK", 1: "MXQ_ERR_INVALID_ARG", 2: "MXQ_ERR_SHAPE", 3: "M
 
 FMT_E2M1 = 0
 FMT_E4M3 = 1
+ACT_NONE = 0
+ACT_GELU = 1
 MODE_NATIVE = 0
 MODE_QDQ = 1
 
@@ -49,6 +51,7 @@ SIGNATURES = {
     "mxq_linear_noalloc": ([_vp, _i64, _i64, _vp, _vp, _i64, _vp, _i32, _vp, _vp], _i32),
     "mxq_linear_noalloc_max_scratch_bytes": ([], _i64),
     "mxq_gemm_gelu_quant": ([_vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp], _i32),
+    "mxq_gemm_quant": ([_vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp], _i32),
     "mxq_ffn": ([_vp, _i64, _i64, ctypes.POINTER(WDesc), ctypes.POINTER(WDesc), _i32, _i32, _vp, _i64, _vp, _vp],
                 _i32),
     "mxq_ffn_workspace_bytes": ([_i64, _i64, _i64, _i32, _i32], _i64),

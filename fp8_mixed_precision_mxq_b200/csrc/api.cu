@@ -198,10 +198,11 @@ int check_gelu_quant(int64_t M, int64_t N, int out_fmt, const void* out_codes, c
 
 int run_gemm_gelu_quant(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K,
                         const void* w_codes, const void* w_sf, int64_t N, const void* bias, int out_fmt,
-                        void* out_codes, void* out_sf, void* h, cudaStream_t stream)
+                        void* out_codes, void* out_sf, void* h, cudaStream_t stream, bool gelu = true)
 {
     GemmArgs g{a_codes, a_sf, a_fmt, M, N, K, w_codes, w_sf, bias, h};
     g.out_fmt = out_fmt;
+    g.out_gelu = gelu;
     g.q_codes = out_codes;
     g.q_sf = out_sf;
     const char* msg = nullptr;
@@ -351,6 +352,18 @@ int mxq_gemm_gelu_quant(const void* a_codes, const void* a_sf, int a_fmt, int64_
     RETURN_IF(check_device());
     return run_gemm_gelu_quant(a_codes, a_sf, a_fmt, M, K, w_codes, w_sf, N, bias_bf16, out_fmt, out_codes, out_sf,
                                h_bf16, static_cast<cudaStream_t>(stream));
+}
+
+int mxq_gemm_quant(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K, const void* w_codes,
+                   const void* w_sf, int64_t N, const void* bias_bf16, int act, int out_fmt, void* out_codes,
+                   void* out_sf, void* h_bf16, void* stream)
+{
+    if (act != MXQ_ACT_NONE && act != MXQ_ACT_GELU) return fail(MXQ_ERR_INVALID_ARG, "unknown activation %d", act);
+    RETURN_IF(check_gemm(a_codes, a_sf, a_fmt, M, K, w_codes, w_sf, N, bias_bf16, out_codes));
+    RETURN_IF(check_gelu_quant(M, N, out_fmt, out_codes, out_sf, h_bf16));
+    RETURN_IF(check_device());
+    return run_gemm_gelu_quant(a_codes, a_sf, a_fmt, M, K, w_codes, w_sf, N, bias_bf16, out_fmt, out_codes, out_sf,
+                               h_bf16, static_cast<cudaStream_t>(stream), act == MXQ_ACT_GELU);
 }
 
 int64_t mxq_ffn_workspace_bytes(int64_t M, int64_t K, int64_t H, int up_fmt, int down_fmt)

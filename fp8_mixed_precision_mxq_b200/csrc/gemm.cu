@@ -43,6 +43,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <type_traits>
 
 #include "mx_elem.cuh"
 #include "mxq_internal.h"
@@ -85,8 +86,9 @@ static_assert(kOverlapChunks <= kLdBufs, "the shared columns must fit the first 
 static_assert(BN / 32 >= 3, "the quantizing epilogue's ring holds three chunks");
 
 // Output of the epilogue: bf16 y = acc + bias; or the next layer's MX-quantized input,
-// h = bf16(GELU(bf16(acc + bias))) as E2M1 / E4M3 codes with tiled E8M0 scales (and h
-// itself in bf16 when asked for).
+// h = bf16(GELU(bf16(acc + bias))) -- or h = bf16(acc + bias) when the launch asks for no
+// activation (Params::gelu) -- as E2M1 / E4M3 codes with tiled E8M0 scales (and h itself
+// in bf16 when asked for).
 constexpr int kOutBf16 = 0;
 constexpr int kOutGeluE2M1 = 1;
 constexpr int kOutGeluE4M3 = 2;
@@ -131,6 +133,7 @@ struct Params {
     uint32_t q_atoms_k;
     int q_rows_pad;
     int write_h;
+    int gelu;     // quantizing epilogue: 1 = h is GELU of the linear's output, 0 = h is that output
     float alpha;  // per-tensor activation scale applied to the sums (1 for MX activations)
     // low-rank branch: stages of 64 K-elements of u (activation, bf16 [M, r]) and B^T
     // (bf16 [N, r]) MMA'd (kind::f16) into the accumulator before the block-scaled stages
@@ -510,17 +513,26 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                     // o: the chunk in bf16 -- y = acc + bias, or h = GELU of that rounded to bf16
                     uint32_t o[16];
                     const float2 alpha2 = make_float2(p.alpha, p.alpha);
+                    // the activation choice is taken once per chunk, outside the unrolled
+                    // loops, so that the 16 independent GELU chains interleave
+                    auto chunk_out = [&](auto gelu) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float2 y = __ffma2_rn(make_float2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1])),
-                                                    alpha2, make_float2(bv[2 * i], bv[2 * i + 1]));
-                        __nv_bfloat162 y2 = __floats2bfloat162_rn(y.x, y.y);
-                        if constexpr (kOut != kOutBf16) {
-                            const float2 g = gelu2_f32(make_float2(__low2float(y2), __high2float(y2)));
-                            y2 = __floats2bfloat162_rn(g.x, g.y);
+                        for (int i = 0; i < 16; ++i) {
+                            const float2 y = __ffma2_rn(
+                                make_float2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1])), alpha2,
+                                make_float2(bv[2 * i], bv[2 * i + 1]));
+                            __nv_bfloat162 y2 = __floats2bfloat162_rn(y.x, y.y);
+                            if constexpr (decltype(gelu)::value) {
+                                const float2 g = gelu2_f32(make_float2(__low2float(y2), __high2float(y2)));
+                                y2 = __floats2bfloat162_rn(g.x, g.y);
+                            }
+                            o[i] = *reinterpret_cast<uint32_t*>(&y2);
                         }
-                        o[i] = *reinterpret_cast<uint32_t*>(&y2);
-                    }
+                    };
+                    if (kOut != kOutBf16 && p.gelu)
+                        chunk_out(std::true_type{});
+                    else
+                        chunk_out(std::false_type{});
                     const bool store_y = kOut == kOutBf16 || p.write_h;
                     uint8_t* buf = ebuf0 + eb * kEpiBuf;
                     if (lane == 0) bulk_wait_read<1>();  // the stores that last used buf have read it
@@ -820,6 +832,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     p.q_atoms_k = quant_out ? static_cast<uint32_t>(sf_atoms_k(g.N)) : 0u;
     p.q_rows_pad = static_cast<int>(ceil_div(g.M, 128) * 128);
     p.write_h = quant_out && g.y != nullptr ? 1 : 0;
+    p.gelu = g.out_gelu ? 1 : 0;
     p.alpha = g.alpha;
     p.lr_stages = lr_stages;
     const int out = !quant_out ? kOutBf16 : (g.out_fmt == kFmtE4M3 ? kOutGeluE4M3 : kOutGeluE2M1);
@@ -843,7 +856,8 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     if (path)
         snprintf(path, path_len, "native %s %s %dx%d grid %d tiles %d%s%s", w4a8 ? "mxf8f6f4" : "mxf4",
                  pair == 2 ? "2cta" : "1cta", 128 * pair, BN, grid, p.num_tiles,
-                 !quant_out ? "" : (g.out_fmt == kFmtE4M3 ? " +gelu->e4m3" : " +gelu->e2m1"),
+                 !quant_out ? "" : g.out_gelu ? (g.out_fmt == kFmtE4M3 ? " +gelu->e4m3" : " +gelu->e2m1")
+                                              : (g.out_fmt == kFmtE4M3 ? " +quant->e4m3" : " +quant->e2m1"),
                  lr_stages ? " +lowrank(bf16 f16-mma)" : "");
     return MXQ_OK;
 }

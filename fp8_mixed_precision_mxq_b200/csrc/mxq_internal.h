@@ -44,9 +44,11 @@ struct GemmArgs {
     const void* w_sf;
     const void* bias;  // bf16 [N] or null
     void* y;           // bf16 [M, N]; with out_fmt >= 0: h in bf16, or null
-    // out_fmt >= 0: the epilogue applies GELU and writes the result MX-quantized in that
-    // format (codes [M, N/2] or [M, N], tiled scales with K = N), the next layer's input
+    // out_fmt >= 0: the epilogue writes its output MX-quantized in that format (codes
+    // [M, N/2] or [M, N], tiled scales with K = N), the next layer's input; with
+    // out_gelu, GELU of it (rounded to bf16 first and after)
     int out_fmt = -1;
+    bool out_gelu = true;
     void* q_codes = nullptr;
     void* q_sf = nullptr;
     // per-tensor scale of the activation (static E4M3): y = alpha * acc + bias

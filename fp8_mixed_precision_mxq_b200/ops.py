@@ -155,6 +155,26 @@ def gemm_gelu_quant(a_codes, a_sf, fmt, M: int, K: int, w: QWeight, out_fmt="e2m
     return codes, sf
 
 
+def gemm_quant(a_codes, a_sf, fmt, M: int, K: int, w: QWeight, act="none", out_fmt="e2m1", codes=None, sf=None,
+               h=None, stream=None):
+    """GEMM whose epilogue writes its output MX-quantized in out_fmt, after GELU when
+    act is "gelu" (mxq_gemm_gelu_quant) or as it is when act is "none": returns (codes,
+    tiled scales).  Pass a bf16 [M, N] tensor as h to also receive the quantizer's input."""
+    acts = {"none": _lib.ACT_NONE, "gelu": _lib.ACT_GELU}
+    if act not in acts:
+        raise ValueError("act must be 'none' or 'gelu', got %r" % (act,))
+    f = _fmt(out_fmt)
+    if codes is None:
+        codes = torch.empty(max(1, codes_bytes(M, w.N, f)), dtype=torch.uint8, device=a_codes.device)
+    if sf is None:
+        sf = torch.empty(max(1, sf_bytes(M, w.N)), dtype=torch.uint8, device=a_codes.device)
+    if h is not None:
+        _cuda_bf16(h, "h")
+    check(_lib.lib().mxq_gemm_quant(_p(a_codes), _p(a_sf), _fmt(fmt), M, K, _p(w.codes), _p(w.sf), w.N, _p(w.bias),
+                                    acts[act], f, _p(codes), _p(sf), _p(h), _stream(stream)), "mxq_gemm_quant")
+    return codes, sf
+
+
 def ffn_workspace_bytes(M: int, K: int, H: int, up_fmt="e2m1", down_fmt="e2m1") -> int:
     return int(_lib.lib().mxq_ffn_workspace_bytes(M, K, H, _fmt(up_fmt), _fmt(down_fmt)))
 

@@ -64,6 +64,7 @@ typedef enum {
 
 typedef enum { MXQ_FMT_E2M1 = 0, MXQ_FMT_E4M3 = 1 } mxq_fmt;      /* activation element format */
 typedef enum { MXQ_MODE_NATIVE = 0, MXQ_MODE_QDQ = 1 } mxq_mode;  /* GEMM execution mode       */
+typedef enum { MXQ_ACT_NONE = 0, MXQ_ACT_GELU = 1 } mxq_act;       /* quantizing epilogue's activation */
 
 /* Library version (major*10000 + minor*100 + patch). */
 int mxq_version(void);
@@ -181,6 +182,16 @@ int64_t mxq_linear_noalloc_max_scratch_bytes(void);
 int mxq_gemm_gelu_quant(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K,
                         const void* w_codes, const void* w_sf, int64_t N, const void* bias_bf16, int out_fmt,
                         void* out_codes, void* out_sf, void* h_bf16, void* stream);
+
+/* mxq_gemm_gelu_quant with the activation chosen: act MXQ_ACT_GELU is that entry point;
+ * MXQ_ACT_NONE quantizes the linear's own output, h = bf16(x . deq(w)^T + bias), so the
+ * epilogue of any producer linear can emit its consumer's MX-quantized operand (codes and
+ * tiled scales equal those of mxq_quantize_act run on mxq_gemm's bf16 output).  Other act
+ * values: MXQ_ERR_INVALID_ARG.  Arguments, layouts and errors otherwise as for
+ * mxq_gemm_gelu_quant. */
+int mxq_gemm_quant(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K, const void* w_codes,
+                   const void* w_sf, int64_t N, const void* bias_bf16, int act, int out_fmt, void* out_codes,
+                   void* out_sf, void* h_bf16, void* stream);
 
 /* The FFN of a DiT block with its hidden activation kept quantized:
  *   y = (GELU(x . up^T + up.bias) quantized to down_fmt) . down^T + down.bias,

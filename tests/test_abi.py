@@ -114,6 +114,20 @@ def test_gemm_gelu_quant_rejects_bad_arguments():
         assert L.mxq_gemm_gelu_quant(*args) == status, (args, _lib.last_error())
 
 
+def test_gemm_quant_rejects_bad_arguments():
+    L = _lib.lib()
+    #        a_codes a_sf fmt  M    K   w_codes w_sf  N   bias act out_fmt codes sf  h  stream
+    bad = [
+        ((A16, A16, 0, 128, 256, A16, A16, 256, None, 2, 0, A16, A16, None, None), _lib.ERR_INVALID_ARG),  # act
+        ((A16, A16, 0, 128, 256, A16, A16, 256, None, -1, 0, A16, A16, None, None), _lib.ERR_INVALID_ARG),  # act
+        ((A16, A16, 0, 128, 256, A16, A16, 264, None, 0, 0, A16, A16, None, None), _lib.ERR_SHAPE),  # N % 32
+        ((A16, A16, 0, 128, 256, A16, A16, 256, None, 0, 5, A16, A16, None, None), _lib.ERR_INVALID_ARG),  # out_fmt
+        ((A16, A16, 0, 128, 256, A16, A16, 256, None, 1, 1, A8, A16, None, None), _lib.ERR_ALIGN),  # out_codes
+    ]
+    for args, status in bad:
+        assert L.mxq_gemm_quant(*args) == status, (args, _lib.last_error())
+
+
 def test_ffn_workspace_and_shape_checks():
     L = _lib.lib()
     assert L.mxq_ffn_workspace_bytes(128, 256, 512, 0, 1) > 0

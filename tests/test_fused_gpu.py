@@ -93,6 +93,36 @@ def test_gemm_gelu_quant_against_oracle(M, N, K, a_fmt, h_fmt):
     assert torch.equal(codes2, codes) and torch.equal(sf2, sf)
 
 
+@pytest.mark.parametrize("M,N,K,a_fmt,h_fmt", CASES)
+def test_gemm_quant_identity_is_quantize_of_gemm(M, N, K, a_fmt, h_fmt):
+    """With no activation the quantizing epilogue emits exactly what the library
+    quantizer (pinned bit-exact to the oracle) makes of the plain GEMM's bf16 output:
+    h, codes and tiled scales (padding included) equal bit for bit; the GELU choice equals
+    mxq_gemm_gelu_quant."""
+    ops = _ops()
+    x = synth.activation(M, K, "normal", seed=M + 7 * N, device="cuda", outlier_frac=0.02, outlier_scale=30.0)
+    w = synth.weight(N, K, seed=N + 3 * K, device="cuda")
+    b = synth.bias(N, seed=N + 1, device="cuda")
+    qw = ops.quantize_weight(w, bias=b)
+    xc, xs = ops.quantize_act(x, a_fmt)
+    y = ops.gemm(xc, xs, a_fmt, M, K, qw)
+    h = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    codes, sf = ops.gemm_quant(xc, xs, a_fmt, M, K, qw, act="none", out_fmt=h_fmt, h=h)
+    assert ops.poll_status() == 0
+    assert "+quant->" + h_fmt in ops.last_path()
+    assert torch.equal(h, y)
+    c2, s2 = ops.quantize_act(y, h_fmt)
+    assert torch.equal(codes[: c2.numel()], c2) and torch.equal(sf[: s2.numel()], s2)
+    # and the product is the oracle's linear within the GEMM tolerance
+    xo, xso, _ = _mx.oracle_quantize(x, a_fmt)
+    wo, wso, _ = _mx.oracle_quantize(w, "e2m1")
+    ref = oracle.linear_rows(xo, xso, _mx.FMT[a_fmt], np.arange(M), K, wo, wso, _mx.bits(b))
+    _mx.assert_gemm_close(_mx.bf16_to_f64(h), ref, "identity-quant epilogue M=%d N=%d" % (M, N))
+    cg, sg = ops.gemm_quant(xc, xs, a_fmt, M, K, qw, act="gelu", out_fmt=h_fmt)
+    cg2, sg2 = ops.gemm_gelu_quant(xc, xs, a_fmt, M, K, qw, out_fmt=h_fmt)
+    assert torch.equal(cg, cg2) and torch.equal(sg, sg2)
+
+
 def test_gemm_gelu_quant_padding_rows_are_zero():
     """Rows between M and the next multiple of 128 get scale 0 in the tiled layout,
     whatever the buffer held before."""
