@@ -62,8 +62,8 @@ GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precisio
                 "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h"]
 GEMM_TRAFFIC = {
     ("ffn_up_480p_w4a4", 32760): {
-        "bytes": 589257984 + 859933440,
-        "sources_sha256": "166a3b24c5e4ff2dfe37203b6c8d42fd8a1e619f6329701c1440256fb440e787",
+        "bytes": 549302528 + 860230912,
+        "sources_sha256": "25c7623c771e8946c5f1af7474e871ec4b63718013fc81d9605c57aedd991de4",
         "profile": "profiles/mx_gemm_mxf4_pair_ffn_up_480p_traffic.md"},
 }
 
