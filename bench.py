@@ -59,11 +59,11 @@ FP8_OVER_BF16 = 2.0   # 4.5 PFLOP/s FP8
 # command).  A record describes only the kernel built from the sources it was taken on:
 # when their hash differs the line reports traffic as null.
 GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precision_mxq_b200/csrc/ptx.cuh",
-                "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h"]
+                "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h", "fp8_mixed_precision_mxq_b200/csrc/mx_elem.cuh"]
 GEMM_TRAFFIC = {
     ("ffn_up_480p_w4a4", 32760): {
-        "bytes": 549302528 + 860230912,
-        "sources_sha256": "25c7623c771e8946c5f1af7474e871ec4b63718013fc81d9605c57aedd991de4",
+        "bytes": 520476160 + 858972928,
+        "sources_sha256": "13b7f59ad754856866f6332333f54f8dc3b573ec9e3af510abdcaf603db0c90c",
         "profile": "profiles/mx_gemm_mxf4_pair_ffn_up_480p_traffic.md"},
 }
 

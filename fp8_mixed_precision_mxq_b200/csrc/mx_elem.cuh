@@ -20,18 +20,6 @@ __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b)
 __device__ __forceinline__ float lo_f(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float hi_f(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Two fp32 -> one byte of two E2M1 codes (first argument in the low nibble).
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi)
-{
-    uint32_t r;
-    asm("{\n\t.reg .b8 t;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
-        "cvt.u32.u8 %0, t;\n\t}"
-        : "=r"(r)
-        : "f"(lo), "f"(hi));
-    return r;
-}
-
 // Eight fp32 -> one word of eight E2M1 codes (v[i] in nibble i).
 __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8])
 {
