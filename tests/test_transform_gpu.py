@@ -152,3 +152,34 @@ def test_quantize_transformed_multi_span(fmt, block, M, K):
     c_gpu = codes.cpu().numpy()
     bad = np.nonzero(c_gpu != c_ref.reshape(-1))[0]
     assert bad.size == 0, "%d codes differ, first at byte %d (row %d)" % (bad.size, bad[0], bad[0] // (c_gpu.size // M))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("block", [32, 128])
+def test_transform_full_ffn_up_480p(block):
+    """The bench's transform_on workload at full size (M = 32760, K = 5120, SmoothQuant-style
+    multipliers): the quantizer's codes and scales bit-exact against the oracle on the whole
+    tensor, in the launch configuration the bench times; the transformed linear (N = 13824)
+    within the GEMM tolerance on one row per 128-row tile plus the ends."""
+    ops = _ops()
+    wl = synth.workload("ffn_up_480p_w4a4", device="cuda", with_bias=True)
+    x, w, b, M, K = wl["x"], wl["w"], wl["bias"], wl["M"], wl["K"]
+    s = smooth_scales(x)
+    inv_s = (1.0 / s).contiguous()
+    codes, sf = ops.quantize_act_transformed(x, "e2m1", block, inv_s)
+    torch.cuda.synchronize()
+    xb = _mx.bits(x)
+    c_ref, s_ref, _ = oracle.quantize_transformed(xb, oracle.E2M1, block, inv_s.cpu().numpy())
+    assert np.array_equal(sf.cpu().numpy(), oracle.sf_to_tiled(s_ref, K))
+    c_gpu = codes.cpu().numpy()
+    bad = np.nonzero(c_gpu != c_ref.reshape(-1))[0]
+    assert bad.size == 0, "%d codes differ, first at byte %d" % (bad.size, bad[0])
+    qw = ops.quantize_weight_transformed(w, bias=b, block=block, mul=s)
+    y = ops.linear_transformed(x, qw, "e2m1", block, inv_s)
+    assert ops.poll_status() == 0
+    rows = synth.sample_rows(M).numpy()
+    wc, ws, _ = oracle.quantize_transformed(_mx.bits(w), oracle.E2M1, block, s.cpu().numpy())
+    K2 = K // 2
+    ref = oracle.linear_rows(c_ref.reshape(M, K2)[rows], s_ref[rows], oracle.E2M1, np.arange(len(rows)), K, wc, ws,
+                             _mx.bits(b))
+    _mx.assert_gemm_close(_mx.bf16_to_f64(y[torch.from_numpy(rows).cuda()]), ref, "transformed linear 480p")
