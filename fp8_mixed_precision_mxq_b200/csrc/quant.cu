@@ -451,11 +451,11 @@ cudaError_t launch_quantize_any(const void* x, int64_t rows, int64_t K, int fmt,
     const uint32_t n_groups = static_cast<uint32_t>(rows * K / 8);
     const uint32_t KB = static_cast<uint32_t>(K / 32);
     const uint32_t atoms_k = static_cast<uint32_t>(sf_atoms_k(K));
+    // one step (8 groups per lane) per warp: the block scheduler streams CTAs in as others
+    // finish, which measured 9-13 % faster on B200 than grids capped at 8-16 CTAs per SM
+    // looping over the tensor (and faster than every cap between)
     const int64_t want = ceil_div(n_groups, kThreads * kUnroll);
-    // blocks per SM (measured on B200: E4M3, with twice the bytes written per element,
-    // gains from a second round of blocks queued behind the resident ones)
-    const int per_sm = fmt == kFmtE2M1 ? 8 : 16;
-    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * per_sm)));
+    const int grid = static_cast<int>(std::max<int64_t>(1, want));
     // row = floor(block / KB) as a multiply-shift, exact for block < 2^29 and KB <= 2^11:
     // magic * KB - 2^40 < KB, so block * magic / 2^40 overshoots block / KB by less than 1 / KB
     const uint64_t kb_magic = ((uint64_t(1) << 40) + KB - 1) / KB;
