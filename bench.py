@@ -62,8 +62,8 @@ GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precisio
                 "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h", "fp8_mixed_precision_mxq_b200/csrc/mx_elem.cuh"]
 GEMM_TRAFFIC = {
     ("ffn_up_480p_w4a4", 32760): {
-        "bytes": 520476160 + 858972928,
-        "sources_sha256": "13b7f59ad754856866f6332333f54f8dc3b573ec9e3af510abdcaf603db0c90c",
+        "bytes": 382355200 + 857401344,
+        "sources_sha256": "4ead914060badceb676f2b238216b77003cb214ce2fbea7c8c3ffcd69c695b4c",
         "profile": "profiles/mx_gemm_mxf4_pair_ffn_up_480p_traffic.md"},
 }
 
