@@ -47,6 +47,8 @@ MUTANTS = [
     ("static_divides_in_double", "float p = (float)(mxo_bf16_to_double(x[i]) * (double)inv_scale);",
      "float p = (float)(mxo_bf16_to_double(x[i]) * (double)inv_scale * 1.0000001);"),
     ("fwht_difference_flipped", "                v[i + h] = a - b;", "                v[i + h] = b - a;"),
+    ("fwht_descending_stages", "    for (int h = 1; h < n; h <<= 1)\n        for (int i = 0; i < n; ++i)",
+     "    for (int h = n >> 1; h >= 1; h >>= 1)\n        for (int i = 0; i < n; ++i)"),
     ("hadamard_unnormalized", "for (int i = 0; i < B; ++i) t[b0 + i] = t[b0 + i] * c;",
      "for (int i = 0; i < B; ++i) t[b0 + i] = t[b0 + i] * 1.0f;"),
     ("smoothing_divides", "t[k] = mul ? xk * mul[k] : xk;", "t[k] = mul ? xk / mul[k] : xk;"),

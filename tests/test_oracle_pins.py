@@ -524,6 +524,23 @@ def test_fwht_matches_sylvester_matrix(n):
         assert np.abs(got - want).max() <= bound
 
 
+def test_fwht_butterfly_order_is_ascending():
+    """The rounding reading: butterflies run h = 1, 2, 4, ... and every stage rounds to
+    binary32.  Hand-worked on v = [1, e, e, 0, 0, ...] (32 values), e = 2^-24:
+      h = 1: [1 + e, 1 - e, e + 0, e - 0] = [1 (a tie, to even), 1 - 2^-24, e, e]
+      h = 2: [1 + e, (1 - e) + e, 1 - e, (1 - e) - e] = [1, 1, 1 - 2^-24, 1 - 2^-23]
+    and the stages h = 4, 8, 16 pair every value with a zero, so they only copy it: the
+    pattern repeats every four values (sums) and its copies (differences with zero).
+    Descending h would give [1, 1 - 2^-24, 1, 1 - 2^-23]; the exact transform gives
+    [1 + 2^-23, 1, 1, 1 - 2^-23]."""
+    e = np.float32(2.0 ** -24)
+    v = np.zeros(32, dtype=np.float32)
+    v[0], v[1], v[2] = 1.0, e, e
+    got = oracle.fwht_f32(v)
+    quad = np.array([1.0, 1.0, 1.0 - 2.0 ** -24, 1.0 - 2.0 ** -23], dtype=np.float32)
+    assert np.array_equal(got, np.tile(quad, 8)), got[:8]
+
+
 def test_fwht_involution_and_norm():
     rng = np.random.default_rng(5)
     for n in (32, 128):
