@@ -184,10 +184,10 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t pair)
 
 // Lanes take 8-element groups in order (four lanes per MX block, like the quantizer), so the
 // warp's code loads and its 16-byte bf16 stores are contiguous; kDqGroups groups per lane, one
-// step per warp (the grid covers the tensor).  value = code value x 2^(scale - 127) in binary32,
-// rounded to bf16: exact but for an overflow to Inf (3- and 4-bit significands times a power of
-// two, results at least 2^-133).  Measured on B200 against one lane per 32-element block: +27 to
-// +37 %, 5.6-6.6 TB/s.
+// step per warp (the grid covers the tensor).  value = code value x 2^(scale - 127), a product
+// binary32 holds exactly, rounded once to bf16 (nearest even): exact except that large scales
+// overflow to Inf and E4M3 codes under scale codes 0-2 can fall below bf16's 2^-133 step.
+// Measured on B200 against one lane per 32-element block: +27 to +37 %, 5.6-6.6 TB/s.
 constexpr int kDqGroups = 4;
 template <int FMT>
 __global__ void __launch_bounds__(kThreads) dequantize_kernel(const uint8_t* __restrict__ codes,

@@ -168,3 +168,28 @@ def test_quantize_max_rows_sampled_tiles(fmt, K):
         assert np.array_equal(c_gpu, c_ref), "codes of rows %d..%d differ" % (r0, r1 - 1)
         s_gpu = sf[t * tile_bytes: (t + 1) * tile_bytes].cpu().numpy()
         assert np.array_equal(s_gpu, oracle.sf_to_tiled(s_ref, K)), "scales of rows %d..%d differ" % (r0, r1 - 1)
+
+
+@pytest.mark.parametrize("fmt", ["e2m1", "e4m3"])
+def test_dequantize_every_code_at_extreme_scales(fmt):
+    """Every element code under scale codes 0-12, 120-130 and 240-255: the dequantized bf16
+    equals the oracle's exact value rounded to nearest even (the binary32 product the
+    kernel forms is exact, so one rounding to bf16 remains: E4M3 products below bf16's
+    2^-133 step at scale codes 0-2 round, large scales overflow to Inf); NaN codes and the
+    NaN scale give NaN."""
+    from fp8_mixed_precision_mxq_b200 import ops
+    scales = list(range(0, 13)) + list(range(120, 131)) + list(range(240, 256))
+    M, K = len(scales), 512
+    if fmt == "e4m3":
+        row = np.tile(np.arange(256, dtype=np.uint8), K // 256)
+    else:
+        row = np.arange(256, dtype=np.uint8)  # every pair of E2M1 codes, K / 2 bytes
+    codes = np.tile(row, (M, 1))
+    logical = np.repeat(np.array(scales, dtype=np.uint8)[:, None], K // 32, axis=1)
+    sf = oracle.sf_to_tiled(logical, K)
+    deq = ops.dequantize(torch.from_numpy(codes.reshape(-1)).cuda(), torch.from_numpy(sf).cuda(), M, K, fmt)
+    want = torch.from_numpy(oracle.dequantize(codes, logical, K, _mx.FMT[fmt])).to(torch.bfloat16)
+    got = deq.cpu()
+    nan_w, nan_g = torch.isnan(want), torch.isnan(got)
+    assert torch.equal(nan_w, nan_g)
+    assert torch.equal(got[~nan_g].view(torch.int16), want[~nan_w].view(torch.int16))
