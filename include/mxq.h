@@ -96,9 +96,10 @@ int mxq_quantize_weight(const void* w_bf16, int64_t N, int64_t K, void* codes, v
 int mxq_quantize_act(const void* x_bf16, int64_t M, int64_t K, int fmt, void* codes, void* sf, void* stream);
 
 /* Dequantization to bf16 (the "QDQ" of the blog's intro and "Kernel note"):
- *   out[r, k] = bf16(decode(code[r, k]) * 2^(sf[r, k/32] - 127)).
- * The product is exact in bf16 except for E4M3 subnormals with scale codes below
- * about 6, which round.  Scale code 0xFF gives NaN. */
+ *   out[r, k] = bf16(decode(code[r, k]) * 2^(sf[r, k/32] - 127)),
+ * the product formed exactly in binary32 and rounded once to nearest even: exact in bf16
+ * except that large scales overflow to Inf and E4M3 values under scale codes 0-2 can fall
+ * below bf16's 2^-133 step and round.  Scale code 0xFF and E4M3 codes 0x7F / 0xFF give NaN. */
 int mxq_dequantize(const void* codes, const void* sf, int64_t rows, int64_t K, int fmt, void* out_bf16,
                    void* stream);
 
