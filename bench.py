@@ -439,6 +439,9 @@ def profile_one(args, ops, x, qw, ws, y, M, N, K, fmt, stream):
     elif args.only == "transform":
         mul = torch.ones(K, dtype=torch.float32, device=x.device)
         fn = lambda: ops.quantize_act_transformed(x, fmt, 32, mul, codes=xc, sf=xs)  # noqa: E731
+    elif args.only == "dequantize":
+        xd = torch.empty((M, K), dtype=torch.bfloat16, device=x.device)
+        fn = lambda: ops.dequantize(xc, xs, M, K, fmt, out=xd)  # noqa: E731
     else:
         fn = lambda: ops.quantize_act(x, fmt, codes=xc, sf=xs)  # noqa: E731
     for _ in range(args.warmup):
@@ -792,7 +795,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--M", type=int, default=0, help="override the workload's row count (profiling)")
-    ap.add_argument("--only", choices=["gemm", "quantize", "gelu_quant", "transform"], default=None,
+    ap.add_argument("--only", choices=["gemm", "quantize", "gelu_quant", "transform", "dequantize"], default=None,
                     help="profiling mode: launch only this kernel, --steps times")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
