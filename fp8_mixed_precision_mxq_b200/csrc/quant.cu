@@ -26,7 +26,7 @@ namespace mxq {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 8;  // 16-byte loads in flight per lane per step
+constexpr int kUnroll = 4;  // 16-byte loads in flight per lane per step (measured best of 4, 8, 16)
 
 // The quantizers stream their input once and write their output once: the loads carry
 // an L2 evict-first policy and bypass L1, the code stores are streaming (.cs) stores, so
@@ -68,11 +68,11 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
     const uint32_t nwarps = gridDim.x * (kThreads / 32);
     const uint32_t warp = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
 
-    static_assert(kUnroll == 8, "the scale bytes of a step are stored two per lane");
+    static_assert(kUnroll % 4 == 0, "the scale bytes of a step are stored kUnroll / 4 per lane");
     for (uint32_t w0 = warp; w0 * 32u < n_groups; w0 += nwarps * kUnroll) {
         uint4 v[kUnroll];
         uint32_t g[kUnroll];
-        uint32_t scw[2] = {0u, 0u};  // the scale codes of this quad's block for u = 0..7, a byte each
+        uint32_t scw[kUnroll / 4] = {};  // the scale codes of this quad's block, a byte per u
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             g[u] = (w0 + u * nwarps) * 32u + lane;
@@ -120,10 +120,10 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
             }
             scw[u >> 2] |= sc << (8 * (u & 3));
         }
-        // The step's 64 scale bytes (8 blocks for each u), two per lane: lane 4 q + j
-        // stores those of block q for u = j and u = j + 4.
+        // The step's 8 kUnroll scale bytes (8 blocks for each u), kUnroll / 4 per lane: lane
+        // 4 q + j stores those of block q for u = j, j + 4, ...
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < kUnroll / 4; ++h) {
             const uint32_t u = (lane & 3u) + 4u * h;
             const uint32_t gq = (w0 + u * nwarps) * 32u + (lane & ~3u);  // the block's first group
             if (gq < n_groups) {
