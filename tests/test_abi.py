@@ -186,3 +186,9 @@ def test_lowrank_entry_point_rejects_bad_arguments():
     assert need > L.mxq_workspace_bytes(128, 256, 256, 0, 0)
     assert L.mxq_linear_lowrank(A16, 128, 256, A16, A16, 256, None, 0, A16, A16, 64, V(1 << 20), need - 1, A16,
                                 None) == _lib.ERR_WORKSPACE
+
+
+def test_gemm_quant_binding_rejects_unknown_activation():
+    from fp8_mixed_precision_mxq_b200 import ops
+    with pytest.raises(ValueError):
+        ops.gemm_quant(None, None, "e2m1", 128, 256, None, act="relu")
