@@ -76,17 +76,11 @@ def lib():
         L.mxo_round_bf16.restype = None
         L.mxo_gelu_bf16.argtypes = [vp, i64, vp]
         L.mxo_gelu_bf16.restype = None
-        L.mxo_static_inverse.argtypes = [ctypes.c_float]
-        L.mxo_static_inverse.restype = ctypes.c_float
         L.mxo_quantize_static_e4m3.argtypes = [vp, i64, ctypes.c_float, vp]
         L.mxo_quantize_static_e4m3.restype = i32
         L.mxo_linear_rows_scaled.argtypes = [vp, vp, i32, vp, i64, i64, vp, vp, i64, vp, dbl, vp, i32]
         L.mxo_linear_rows_scaled.restype = i32
-        L.mxo_hadamard_norm.argtypes = [i32]
-        L.mxo_hadamard_norm.restype = ctypes.c_float
-        L.mxo_fwht_f32.argtypes = [vp, i32]
-        L.mxo_fwht_f32.restype = None
-        L.mxo_quantize_transformed.argtypes = [vp, i64, i64, vp, i32, i32, vp, vp, vp]
+        L.mxo_quantize_transformed.argtypes = [vp, i64, i64, vp, i32, i32, vp, vp, vp, vp, vp, vp, i32]
         L.mxo_quantize_transformed.restype = i32
         L.mxo_linear_lowrank_rows.argtypes = [vp, vp, i32, vp, i64, i64, vp, vp, i64, vp, vp, vp, i64, vp, vp, i32]
         L.mxo_linear_lowrank_rows.restype = i32
@@ -229,16 +223,12 @@ def ffn_hidden_rows(a_codes, a_sf, a_fmt, rows, K, w1_codes, w1_sf, b1_bits, h_f
     return h, codes, sf
 
 
-def static_inverse(scale: float) -> float:
-    """fl32(1 / scale): the multiplier the static quantizer applies."""
-    return float(lib().mxo_static_inverse(float(scale)))
-
-
 def quantize_static_e4m3(x_bits: np.ndarray, scale: float) -> np.ndarray:
-    """Static per-tensor E4M3 codes of bf16 bits x (same shape, uint8)."""
+    """Static per-tensor E4M3 codes of bf16 bits x (same shape, uint8): RNE_sat(x / s)
+    for the binary32 scale s (a Python float is first rounded to binary32)."""
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
     codes = np.empty(x_bits.shape, dtype=np.uint8)
-    lib().mxo_quantize_static_e4m3(_ptr(x_bits), x_bits.size, static_inverse(scale), _ptr(codes))
+    lib().mxo_quantize_static_e4m3(_ptr(x_bits), x_bits.size, float(scale), _ptr(codes))
     return codes
 
 
@@ -264,35 +254,34 @@ def linear_rows_scaled(a_codes, a_sf, a_fmt, rows, K, w_codes, w_sf, alpha, bias
     return y
 
 
-def hadamard_norm(B: int) -> float:
-    """fl32(1 / sqrt(B)), the normalization of the block Hadamard rotation."""
-    return float(lib().mxo_hadamard_norm(int(B)))
-
-
-def fwht_f32(v: np.ndarray) -> np.ndarray:
-    """Fast Walsh-Hadamard transform (Sylvester order, unnormalized) of a float32 vector
-    whose length is a power of two, in binary32 arithmetic."""
-    out = np.ascontiguousarray(v, dtype=np.float32).copy()
-    lib().mxo_fwht_f32(_ptr(out), out.size)
-    return out
-
-
-def quantize_transformed(x_bits: np.ndarray, fmt: int, B: int, mul: np.ndarray | None = None):
-    """Smooth (t = x * mul), rotate each B-block by the normalized Hadamard, MX-quantize.
-    Returns (codes, logical scales, transformed float32 values)."""
+def quantize_transformed(x_bits: np.ndarray, fmt: int, B: int, mul: np.ndarray | None = None,
+                         nthreads: int | None = None):
+    """The transform_on quantizer's definition: t = (x * mul) . blockdiag(H_B) / sqrt(B) in
+    fp64, then MX quantization of t.  Returns a dict with
+      codes, sf  -- the definition's element codes (packed) and logical scales [rows, K/32];
+      t          -- the transformed values [rows, K] (fp64);
+      code_lo, code_hi -- per element [rows, K], the codes of t -+ delta, delta the error
+                    bound of a binary32 evaluation: equal where the code is certain;
+      blk_amb    -- per MX block: 0 scale certain, 1 a binary32 evaluation may take a
+                    neighbouring scale, 2 it may overflow binary32."""
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
     rows, K = x_bits.shape
-    codes = np.zeros((rows, codes_row_bytes(K, fmt)), dtype=np.uint8)
-    sf = np.zeros((rows, K // 32), dtype=np.uint8)
-    t = np.zeros((rows, K), dtype=np.float32)
+    out = {"codes": np.zeros((rows, codes_row_bytes(K, fmt)), dtype=np.uint8),
+           "sf": np.zeros((rows, K // 32), dtype=np.uint8),
+           "t": np.zeros((rows, K), dtype=np.float64),
+           "code_lo": np.zeros((rows, K), dtype=np.uint8),
+           "code_hi": np.zeros((rows, K), dtype=np.uint8),
+           "blk_amb": np.zeros((rows, K // 32), dtype=np.uint8)}
     mp = None
     if mul is not None:
         mul = np.ascontiguousarray(mul, dtype=np.float32)
         mp = _ptr(mul)
-    rc = lib().mxo_quantize_transformed(_ptr(x_bits), rows, K, mp, B, fmt, _ptr(codes), _ptr(sf), _ptr(t))
+    rc = lib().mxo_quantize_transformed(_ptr(x_bits), rows, K, mp, B, fmt, _ptr(out["codes"]), _ptr(out["sf"]),
+                                        _ptr(out["t"]), _ptr(out["code_lo"]), _ptr(out["code_hi"]),
+                                        _ptr(out["blk_amb"]), nthreads or default_threads())
     if rc != 0:
         raise ValueError("oracle transform failed (rc=%d)" % rc)
-    return codes, sf, t
+    return out
 
 
 def linear_lowrank_rows(a_codes, a_sf, a_fmt, rows, K, r_codes, r_sf, x_bits, l1t_bits, l2t_bits, bias_bits=None,

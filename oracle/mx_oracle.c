@@ -429,19 +429,23 @@ void mxo_gelu_bf16(const uint16_t *y, int64_t n, uint16_t *h)
 
 /* The W4A8 of the blog's "Quantization formats" table names "FP8 E4M3 static
  * activations": one scale s for the whole tensor, fixed offline (calibration: s = amax /
- * 448, the largest E4M3 magnitude).  Each element becomes RNE_sat(x * r) on the E4M3
- * grid with r = fl32(1/s), the product taken in binary32 -- the precision in which the
- * kernel takes the same decision.  The block scales the MMA reads are all 127 (x1) and
- * the linear layer multiplies its sums by s. */
-float mxo_static_inverse(float s) { return (float)(1.0 / (double)s); }
-
-int mxo_quantize_static_e4m3(const uint16_t *x, int64_t n, float inv_scale, uint8_t *codes)
+ * 448, the largest E4M3 magnitude).  Each element becomes RNE_sat(x / s) on the E4M3
+ * grid, x / s the exact quotient.  The block scales the MMA reads are all 127 (x1) and
+ * the linear layer multiplies its sums by s.
+ *
+ * The quotient is taken as one IEEE double division of the exact operands (x is bf16, s
+ * binary32), so it carries a relative rounding error below 2^-53.  That never moves it
+ * across an E4M3 decision boundary: a boundary m (a midpoint between grid values, at most
+ * 5 significant bits) equals x / s only if x = s * m exactly, and otherwise x - s * m is a
+ * nonzero multiple of the coarser of x's and s*m's last-bit weights, which puts x / s more
+ * than 2^-30 |m| away from m.  So the double lands on the same side of every boundary as
+ * the exact quotient, and on a boundary only when x / s is one. */
+int mxo_quantize_static_e4m3(const uint16_t *x, int64_t n, float scale, uint8_t *codes)
 {
     for (int64_t i = 0; i < n; ++i) {
-        /* exact double product of a bf16 and a binary32 value, rounded once to binary32 */
-        float p = (float)(mxo_bf16_to_double(x[i]) * (double)inv_scale);
-        if (isnan(p)) codes[i] = (uint8_t)((signbit(p) ? 0x80 : 0x00) | 0x7F);
-        else codes[i] = (uint8_t)mxo_encode_elem((double)p, MXO_E4M3);
+        double q = mxo_bf16_to_double(x[i]) / (double)scale;
+        if (isnan(q)) codes[i] = (uint8_t)((signbit(q) ? 0x80 : 0x00) | 0x7F);
+        else codes[i] = (uint8_t)mxo_encode_elem(q, MXO_E4M3);
     }
     return 0;
 }
@@ -467,64 +471,137 @@ int mxo_linear_rows_scaled(const uint8_t *a_codes, const uint8_t *a_sf, int a_fm
  * transformed before it is quantized -- divided per channel by SmoothQuant scales (the
  * weights carry the scales instead) and rotated by a fixed block Hadamard matrix (the
  * weights rotated the same way offline), so x . W^T is unchanged while outliers spread
- * over a block.  The codes are decided from the transformed binary32 values, so this
- * oracle takes every step in binary32, in the kernel's order:
- *   t_k = fl32(x_k * mul_k)            (mul = 1/s for activations, s for weights; NULL: t = x)
- *   each block of B consecutive t's:  fast Walsh-Hadamard transform (below), then each
- *   value times c_B = fl32(1/sqrt B), rounded;
- *   the rows then MX-quantized from those values exactly as mxo_quantize does. */
+ * over a block.  The definition, taken here in fp64:
+ *   a_k = x_k * mul_k                 (mul = 1/s for activations, s for weights; NULL: a = x)
+ *   each block of B consecutive a's:  t = a . H_B / sqrt(B),  H_B the Sylvester Hadamard
+ *                                      matrix, H_B[j][k] = (-1)^popcount(j & k)
+ *   t MX-quantized exactly as mxo_quantize quantizes a row.
+ * a_k is exact in fp64 (8 + 24 significant bits), each t is a sum of B exact terms, so its
+ * fp64 error is below B * 2^-53 * L1 / sqrt(B), L1 = sum_k |a_k| over the rotation block.
+ *
+ * Evaluating t in binary32 (as a GPU does) moves it by more than that.  For any evaluation
+ * that rounds each product a_k once, each of the log2(B) butterfly sums and differences
+ * once (in any stage order) and the scaling by fl32(1/sqrt B) and by the power-of-two block
+ * scale at most twice, the standard error bounds of summation (N. J. Higham, "Accuracy and
+ * Stability of Numerical Algorithms", 2nd ed., section 4.2; products and quotients add their
+ * own relative u and, in the subnormal range, an absolute 2^-150) give
+ *   |t_binary32 - t| <= delta = 1.01 * ((log2(B) + 4) * u * L1 + (B + 2) * 2^-150) / sqrt(B),
+ * u = 2^-24.  So this oracle also reports, per MX block, whether the scale could differ
+ * (the codes of max |t| - delta and max |t| + delta differ, or L1 >= 2^127 so that a
+ * binary32 evaluation could overflow), and per element the two codes of t -+ delta under
+ * the definition's scale: an element whose two codes differ lies within delta of a
+ * decision boundary of the element grid (or of zero), and any binary32 evaluation may
+ * take either code there.  The codes reported as `codes` are always the definition's. */
+typedef struct {
+    const uint16_t *x;
+    int64_t r0, r1, K;
+    const float *mul;
+    int B, fmt;
+    uint8_t *codes, *sf, *code_lo, *code_hi, *blk_amb;
+    double *t_out;
+} transform_job;
 
-/* c_B = fl32(1/sqrt B) for B = 2^j: 2^(-j/2) for even j, fl32(sqrt 2) * 2^(-(j+1)/2) for odd
- * j (the scaling by a power of two is exact, so this is the correctly rounded value). */
-float mxo_hadamard_norm(int B)
+static void *transform_rows(void *arg)
 {
-    int j = 0;
-    while ((1 << j) < B) ++j;
-    if (j % 2 == 0) return ldexpf(1.0f, -j / 2);
-    return ldexpf((float)M_SQRT2, -(j + 1) / 2);
-}
-
-/* In-place fast Walsh-Hadamard transform of n = 2^j binary32 values in Sylvester order
- * (the result is v . H_n with H_n[a][b] = (-1)^popcount(a & b)): for h = 1, 2, 4, ..., n/2
- * in that order, every pair (i, i + h) with bit h of i clear becomes (v_i + v_i+h,
- * v_i - v_i+h), each sum and difference rounded to binary32. */
-void mxo_fwht_f32(float *v, int n)
-{
-    for (int h = 1; h < n; h <<= 1)
-        for (int i = 0; i < n; ++i)
-            if ((i & h) == 0) {
-                float a = v[i], b = v[i + h];
-                v[i] = a + b;
-                v[i + h] = a - b;
-            }
-}
-
-int mxo_quantize_transformed(const uint16_t *x, int64_t rows, int64_t K, const float *mul, int B, int fmt,
-                             uint8_t *codes, uint8_t *sf, float *t_out)
-{
-    if (K % 32 != 0 || B < 32 || (B & (B - 1)) != 0 || K % B != 0) return -1;
-    const float c = mxo_hadamard_norm(B);
+    const transform_job *jb = (const transform_job *)arg;
+    const uint16_t *x = jb->x;
+    const int64_t K = jb->K;
+    const float *mul = jb->mul;
+    const int B = jb->B, fmt = jb->fmt;
+    uint8_t *codes = jb->codes, *sf = jb->sf, *code_lo = jb->code_lo, *code_hi = jb->code_hi;
+    uint8_t *blk_amb = jb->blk_amb;
+    double *t_out = jb->t_out;
+    int d = 0;
+    while ((1 << d) < B) ++d;
+    const double inv_sqrt_b = 1.0 / sqrt((double)B);
+    const double u = ldexp(1.0, -24);
     const int64_t KB = K / 32, rb = mxo_codes_row_bytes(K, fmt);
-    float *t = (float *)malloc(sizeof(float) * (size_t)K);
-    double v[32];
+    double *a = (double *)malloc(sizeof(double) * (size_t)K);
+    double *t = (double *)malloc(sizeof(double) * (size_t)K);
+    double *delta = (double *)malloc(sizeof(double) * (size_t)K);
+    double *l1 = (double *)malloc(sizeof(double) * (size_t)K);
     int cd[32];
-    for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t r = jb->r0; r < jb->r1; ++r) {
         for (int64_t k = 0; k < K; ++k) {
-            float xk = (float)mxo_bf16_to_double(x[r * K + k]);
-            t[k] = mul ? xk * mul[k] : xk;
+            double xk = mxo_bf16_to_double(x[r * K + k]);
+            a[k] = mul ? xk * (double)mul[k] : xk;
         }
         for (int64_t b0 = 0; b0 < K; b0 += B) {
-            mxo_fwht_f32(t + b0, B);
-            for (int i = 0; i < B; ++i) t[b0 + i] = t[b0 + i] * c;
+            double s1 = 0.0;
+            for (int k = 0; k < B; ++k) s1 += fabs(a[b0 + k]);
+            for (int j = 0; j < B; ++j) {
+                double acc = 0.0;
+                for (int k = 0; k < B; ++k) {
+                    double h = (__builtin_popcount((unsigned)(j & k)) & 1) ? -1.0 : 1.0;
+                    acc += h * a[b0 + k];
+                }
+                t[b0 + j] = acc * inv_sqrt_b;
+                l1[b0 + j] = s1;
+                delta[b0 + j] = 1.01 * ((d + 4) * u * s1 + (B + 2) * ldexp(1.0, -150)) * inv_sqrt_b;
+            }
         }
-        if (t_out) memcpy(t_out + r * K, t, sizeof(float) * (size_t)K);
+        if (t_out) memcpy(t_out + r * K, t, sizeof(double) * (size_t)K);
         for (int64_t kb = 0; kb < KB; ++kb) {
-            for (int i = 0; i < 32; ++i) v[i] = (double)t[kb * 32 + i];
-            sf[r * KB + kb] = (uint8_t)quantize_values(v, fmt, cd);
+            const double *tb = t + kb * 32;
+            int sc = quantize_values(tb, fmt, cd);
+            sf[r * KB + kb] = (uint8_t)sc;
             store_block_codes(codes + r * rb, kb, cd, fmt);
+            int amb = 0;
+            if (sc != 255) {
+                double lo = 0.0, hi = 0.0;
+                for (int i = 0; i < 32; ++i) {
+                    double dl = fabs(tb[i]) - delta[kb * 32 + i], dh = fabs(tb[i]) + delta[kb * 32 + i];
+                    if (dl > lo) lo = dl;
+                    if (dh > hi) hi = dh;
+                    if (l1[kb * 32 + i] >= ldexp(1.0, 127)) amb = 2;
+                }
+                if (!amb && mxo_scale_code(lo, 0, fmt) != mxo_scale_code(hi, 0, fmt)) amb = 1;
+            }
+            if (blk_amb) blk_amb[r * KB + kb] = (uint8_t)amb;
+            for (int i = 0; i < 32; ++i) {
+                int c_lo = cd[i], c_hi = cd[i];
+                if (sc != 255) {
+                    double X = mxo_scale_value(sc), dv = delta[kb * 32 + i];
+                    c_lo = mxo_encode_elem((tb[i] - dv) / X, fmt);
+                    c_hi = mxo_encode_elem((tb[i] + dv) / X, fmt);
+                }
+                if (code_lo) code_lo[r * K + kb * 32 + i] = (uint8_t)c_lo;
+                if (code_hi) code_hi[r * K + kb * 32 + i] = (uint8_t)c_hi;
+            }
         }
     }
+    free(a);
     free(t);
+    free(delta);
+    free(l1);
+    return NULL;
+}
+
+static void set_transform_range(void *j, int64_t r0, int64_t r1)
+{
+    ((transform_job *)j)->r0 = r0;
+    ((transform_job *)j)->r1 = r1;
+}
+
+/* x: bf16 bits [rows, K]; mul: K floats or NULL; B: 32 or a larger power of two dividing K.
+ * Outputs: codes (packed as mxo_quantize packs them) and logical scales [rows, K/32] of the
+ * definition; optionally t [rows, K] (fp64), the two candidate codes per element
+ * code_lo / code_hi [rows, K] (one byte each), and blk_amb [rows, K/32] (0: the scale is
+ * certain; 1: a binary32 evaluation could take a neighbouring scale; 2: it could overflow). */
+int mxo_quantize_transformed(const uint16_t *x, int64_t rows, int64_t K, const float *mul, int B, int fmt,
+                             uint8_t *codes, uint8_t *sf, double *t_out, uint8_t *code_lo, uint8_t *code_hi,
+                             uint8_t *blk_amb, int nthreads)
+{
+    if (K % 32 != 0 || B < 32 || (B & (B - 1)) != 0 || K % B != 0 || rows < 0) return -1;
+    if (nthreads < 1) nthreads = 1;
+    transform_job *jobs = (transform_job *)calloc((size_t)nthreads, sizeof(transform_job));
+    for (int t = 0; t < nthreads; ++t) {
+        transform_job *j = &jobs[t];
+        j->x = x; j->K = K; j->mul = mul; j->B = B; j->fmt = fmt; j->codes = codes; j->sf = sf;
+        j->code_lo = code_lo; j->code_hi = code_hi; j->blk_amb = blk_amb; j->t_out = t_out;
+    }
+    run_rows(transform_rows, jobs, sizeof(transform_job), rows, nthreads, set_transform_range);
+    free(jobs);
     return 0;
 }
 

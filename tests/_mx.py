@@ -57,3 +57,63 @@ def assert_gemm_close(y_gpu: np.ndarray, y_ref: np.ndarray, what: str = ""):
 
 def sqnr_db(y_ref: np.ndarray, y: np.ndarray) -> float:
     return 10.0 * np.log10(np.sum(y_ref ** 2) / max(np.sum((y_ref - y) ** 2), 1e-300))
+
+
+def tiled_to_logical(tiled: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """Tiled scale bytes -> logical [rows, K/32], through the oracle's (pinned) layout: the
+    oracle scatters the 1-based logical index of every scale, one byte plane at a time."""
+    KB = K // 32
+    idx = np.arange(1, rows * KB + 1, dtype=np.int64)
+    where = np.zeros(oracle.sf_tiled_bytes(rows, K), dtype=np.int64)
+    for plane in range(4):
+        b = ((idx >> (8 * plane)) & 0xFF).astype(np.uint8).reshape(rows, KB)
+        where |= oracle.sf_to_tiled(b, K).astype(np.int64) << (8 * plane)
+    out = np.zeros(rows * KB, dtype=np.uint8)
+    live = where > 0
+    out[where[live] - 1] = np.asarray(tiled)[: where.size][live]
+    return out.reshape(rows, KB)
+
+
+def unpack_codes(codes: np.ndarray, rows: int, K: int, fmt: str) -> np.ndarray:
+    """Packed element codes -> one byte per element [rows, K]."""
+    c = np.asarray(codes).reshape(-1)
+    if fmt == "e4m3":
+        return c[: rows * K].reshape(rows, K)
+    c = c[: rows * K // 2]
+    return np.stack([c & 0xF, c >> 4], axis=-1).reshape(rows, K)
+
+
+def check_transformed(codes_gpu, sf_gpu, rows: int, K: int, fmt: str, ref: dict, what: str,
+                      max_uncertain: float | None = 1e-3):
+    """The transform_on quantizer against the oracle's definition (oracle.quantize_transformed):
+      * every block whose scale the oracle reports certain has the definition's scale, and on
+        it every element whose code is certain has the definition's code, bit for bit;
+      * the other elements of such blocks (within a binary32 error bound of a decision
+        boundary) have one of the two codes the oracle reports for them;
+      * a block reported uncertain has a scale at most one away (or 255 where binary32 may
+        overflow);
+      * at most max_uncertain of the elements are uncertain (None: no limit).
+    Returns the number of uncertain elements."""
+    sf_l = tiled_to_logical(sf_gpu.cpu().numpy() if hasattr(sf_gpu, "cpu") else sf_gpu, rows, K)
+    cg = unpack_codes(codes_gpu.cpu().numpy() if hasattr(codes_gpu, "cpu") else codes_gpu, rows, K, fmt)
+    cd = unpack_codes(ref["codes"], rows, K, fmt)
+    amb = ref["blk_amb"]
+    sure = amb == 0
+    bad = np.nonzero(sure & (sf_l != ref["sf"]))
+    assert bad[0].size == 0, "%s: %d certain scales differ, first (%d, %d): gpu %d oracle %d" % (
+        what, bad[0].size, bad[0][0], bad[1][0], sf_l[bad][0], ref["sf"][bad][0])
+    d = np.abs(sf_l.astype(int) - ref["sf"].astype(int))
+    unsure_ok = (d <= 1) | ((amb == 2) & (sf_l == 255))
+    assert unsure_ok[~sure].all(), what + ": an uncertain block's scale is off by more than one"
+    blk_sure = np.repeat(sure, 32, axis=1)
+    certain = blk_sure & (ref["code_lo"] == ref["code_hi"])
+    bad = np.nonzero(certain & (cg != cd))
+    assert bad[0].size == 0, "%s: %d certain codes differ, first (%d, %d): gpu %#x oracle %#x" % (
+        what, bad[0].size, bad[0][0], bad[1][0], cg[bad][0], cd[bad][0])
+    unc = blk_sure & ~certain
+    ok = (cg == ref["code_lo"]) | (cg == ref["code_hi"])
+    assert ok[unc].all(), what + ": an uncertain code is neither of the two candidates"
+    n_unc = int(unc.sum())
+    if max_uncertain is not None:
+        assert n_unc <= max_uncertain * cg.size, "%s: %d uncertain elements" % (what, n_unc)
+    return n_unc

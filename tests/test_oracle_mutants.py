@@ -44,14 +44,22 @@ MUTANTS = [
      "y[i * N + j] = y[i * N + j] + (bias"),
     ("static_bias_scaled", "y[i * N + j] = alpha * y[i * N + j] + (bias ? mxo_bf16_to_double(bias[j]) : 0.0);",
      "y[i * N + j] = alpha * (y[i * N + j] + (bias ? mxo_bf16_to_double(bias[j]) : 0.0));"),
-    ("static_divides_in_double", "float p = (float)(mxo_bf16_to_double(x[i]) * (double)inv_scale);",
-     "float p = (float)(mxo_bf16_to_double(x[i]) * (double)inv_scale * 1.0000001);"),
-    ("fwht_difference_flipped", "                v[i + h] = a - b;", "                v[i + h] = b - a;"),
-    ("fwht_descending_stages", "    for (int h = 1; h < n; h <<= 1)\n        for (int i = 0; i < n; ++i)",
-     "    for (int h = n >> 1; h >= 1; h >>= 1)\n        for (int i = 0; i < n; ++i)"),
-    ("hadamard_unnormalized", "for (int i = 0; i < B; ++i) t[b0 + i] = t[b0 + i] * c;",
-     "for (int i = 0; i < B; ++i) t[b0 + i] = t[b0 + i] * 1.0f;"),
-    ("smoothing_divides", "t[k] = mul ? xk * mul[k] : xk;", "t[k] = mul ? xk / mul[k] : xk;"),
+    ("static_binary32_quotient", "double q = mxo_bf16_to_double(x[i]) / (double)scale;",
+     "double q = (float)(mxo_bf16_to_double(x[i]) / (double)scale);"),
+    ("static_binary32_product", "double q = mxo_bf16_to_double(x[i]) / (double)scale;",
+     "double q = (float)(mxo_bf16_to_double(x[i]) * (double)(float)(1.0 / scale));"),
+    ("static_scale_multiplies", "double q = mxo_bf16_to_double(x[i]) / (double)scale;",
+     "double q = mxo_bf16_to_double(x[i]) * (double)scale;"),
+    ("hadamard_sign_rule", "double h = (__builtin_popcount((unsigned)(j & k)) & 1) ? -1.0 : 1.0;",
+     "double h = (__builtin_popcount((unsigned)(j | k)) & 1) ? -1.0 : 1.0;"),
+    ("hadamard_unnormalized", "const double inv_sqrt_b = 1.0 / sqrt((double)B);", "const double inv_sqrt_b = 1.0;"),
+    ("smoothing_divides", "a[k] = mul ? xk * (double)mul[k] : xk;", "a[k] = mul ? xk / (double)mul[k] : xk;"),
+    ("transform_bound_dropped",
+     "delta[b0 + j] = 1.01 * ((d + 4) * u * s1 + (B + 2) * ldexp(1.0, -150)) * inv_sqrt_b;",
+     "delta[b0 + j] = 0.0;"),
+    ("transform_scale_flag_dropped", "if (!amb && mxo_scale_code(lo, 0, fmt) != mxo_scale_code(hi, 0, fmt)) amb = 1;",
+     "(void)0;"),
+    ("transform_overflow_unflagged", "if (l1[kb * 32 + i] >= ldexp(1.0, 127)) amb = 2;", "(void)0;"),
     ("lowrank_u_not_rounded", "            u[j] = mxo_bf16_to_double(mxo_double_to_bf16(acc));", "            u[j] = acc;"),
     ("lowrank_l2_transposed", "for (int64_t j = 0; j < r; ++j) acc += u[j] * mxo_bf16_to_double(l2t[n * r + j]);",
      "for (int64_t j = 0; j < r; ++j) acc += u[j] * mxo_bf16_to_double(l2t[(j * N + n) % (N * r)]);"),

@@ -24,6 +24,7 @@ import numpy as np
 import pytest
 
 import oracle
+from tests import _exact
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 FMT = {"e2m1": oracle.E2M1, "e4m3": oracle.E4M3}
@@ -454,25 +455,50 @@ def test_gelu_bf16_hand_values():
 
 # --- static per-tensor E4M3 activations -------------------------------------------------------
 #
-# codes = RNE_sat(fl32(x * fl32(1/s))) on the E4M3 grid; the linear multiplies its sums by s.
+# codes = RNE_sat(x / s) on the E4M3 grid, x / s the exact quotient; the linear multiplies its
+# sums by s.  Pinned against exact rationals (tests/_exact.py), never against binary32
+# arithmetic.
 
-def test_static_inverse_is_the_binary32_reciprocal():
-    for s in (0.5, 3.0, 0.0371, 1e-3, 448.0, 7.25e-5):
-        assert oracle.static_inverse(s) == float(np.float32(1.0) / np.float32(s))
+def _f32(v: float) -> float:
+    return float(np.float32(v))
 
 
-@pytest.mark.parametrize("scale", [0.5, 0.0371, 2.0 ** -7 * 3, 11.0])
-def test_static_e4m3_is_nearest_grid_point_of_the_binary32_product(scale):
-    """Each code is the brute-force nearest E4M3 value (ties to even, saturating) of the
-    binary32 product x * fl32(1/s), computed here with numpy's float32 arithmetic."""
-    rng = np.random.default_rng(int(scale * 1000) + 3)
-    x = (rng.standard_normal(4000) * scale * rng.choice([1.0, 30.0, 300.0, 1e-3], size=4000)).astype(np.float32)
+@pytest.mark.parametrize("scale", [0.5, 0.0371, 2.0 ** -7 * 3, 11.0, 7.3e-31, 3.1e29])
+def test_static_e4m3_is_nearest_grid_point_of_the_exact_quotient(scale):
+    """Each code is the E4M3 value nearest to the exact rational x / s (ties to the even
+    code, saturating, sign kept), found by exact comparison with every grid neighbour."""
+    s = _f32(scale)
+    rng = np.random.default_rng(int(abs(np.log2(s))) + 3)
+    x = (rng.standard_normal(3000) * s * rng.choice([1.0, 30.0, 300.0, 1e-3, 1e-6], size=3000)).astype(np.float32)
     bits = (x.view(np.uint32) >> 16).astype(np.uint16)          # truncate to bf16 (any bf16 will do)
-    xb = (bits.astype(np.uint32) << 16).view(np.float32)
-    p = xb * (np.float32(1.0) / np.float32(scale))                # binary32 multiply
-    got = oracle.quantize_static_e4m3(bits, scale)
-    for xi, pi, c in zip(xb, p, got):
-        assert c == brute_round(float(pi), oracle.E4M3), (float(xi), float(pi), hex(c))
+    got = oracle.quantize_static_e4m3(bits, s)
+    S = _exact.f32_fraction(s)
+    for b, c in zip(bits, got):
+        xf = _exact.bf16_fraction(int(b))
+        want = _exact.nearest_code(xf / S, oracle.E4M3, negative=bool(b & 0x8000))
+        assert c == want, (hex(int(b)), s, hex(c), hex(want))
+
+
+def test_static_e4m3_near_ties_follow_the_exact_quotient():
+    """Inputs for which a binary32 evaluation of x / s -- the correctly rounded binary32
+    quotient (double rounding) or the binary32 product x * fl32(1/s) -- takes another code
+    than the exact quotient: the oracle takes the exact quotient's code, for x scaled by
+    powers of two across the E4M3 range and for both signs."""
+    cases = _exact.static_near_ties()
+    assert len(cases) > 400
+    checked = 0
+    for s, x in cases[::3]:
+        sf = float(s)
+        xs = [x * Fraction(2) ** j for j in range(-6, 9)]
+        xs = [v for v in xs if Fraction(2) ** -9 <= v / s <= 448]
+        bits = np.array([_exact.bf16_bits(v) for v in xs] + [_exact.bf16_bits(v) | 0x8000 for v in xs],
+                        dtype=np.uint16)
+        got = oracle.quantize_static_e4m3(bits, sf)
+        for b, c in zip(bits, got):
+            want = _exact.nearest_code(_exact.bf16_fraction(int(b)) / s, oracle.E4M3)
+            assert c == want, (hex(int(b)), s, hex(c), hex(want))
+            checked += 1
+    assert checked > 2000
 
 
 def test_static_e4m3_exact_multiples_saturation_and_sign():
@@ -508,91 +534,146 @@ def test_linear_scaled_brute_force_exact():
 
 
 # --- transform_on: smoothing and block Hadamard rotation ------------------------------------
+#
+# Definition: t = (x * mul) . blockdiag(H_B) / sqrt(B), then MX quantization of t.  Pinned
+# against exact rationals: the transformed values are S / sqrt(B) with S an exact sum, and
+# every scale and code decision compares squares exactly (tests/_exact.py).
 
-@pytest.mark.parametrize("n", [32, 128])
-def test_fwht_matches_sylvester_matrix(n):
-    """The binary32 FWHT equals v . H_n (scipy's Sylvester Hadamard, fp64) within the
-    rounding of its log2(n) stages."""
-    from scipy.linalg import hadamard
-    rng = np.random.default_rng(n)
-    H = hadamard(n).astype(np.float64)
-    for _ in range(50):
-        v = (rng.standard_normal(n) * rng.choice([1e-3, 1.0, 40.0], size=n)).astype(np.float32)
-        got = oracle.fwht_f32(v).astype(np.float64)
-        want = v.astype(np.float64) @ H
-        bound = np.log2(n) * 2.0 ** -23 * np.abs(v).astype(np.float64).sum() * 2
-        assert np.abs(got - want).max() <= bound
+def _bf16_bits(a):
+    return (np.asarray(a, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16)
 
 
-def test_fwht_butterfly_order_is_ascending():
-    """The rounding reading: butterflies run h = 1, 2, 4, ... and every stage rounds to
-    binary32.  Hand-worked on v = [1, e, e, 0, 0, ...] (32 values), e = 2^-24:
-      h = 1: [1 + e, 1 - e, e + 0, e - 0] = [1 (a tie, to even), 1 - 2^-24, e, e]
-      h = 2: [1 + e, (1 - e) + e, 1 - e, (1 - e) - e] = [1, 1, 1 - 2^-24, 1 - 2^-23]
-    and the stages h = 4, 8, 16 pair every value with a zero, so they only copy it: the
-    pattern repeats every four values (sums) and its copies (differences with zero).
-    Descending h would give [1, 1 - 2^-24, 1, 1 - 2^-23]; the exact transform gives
-    [1 + 2^-23, 1, 1, 1 - 2^-23]."""
-    e = np.float32(2.0 ** -24)
-    v = np.zeros(32, dtype=np.float32)
-    v[0], v[1], v[2] = 1.0, e, e
-    got = oracle.fwht_f32(v)
-    quad = np.array([1.0, 1.0, 1.0 - 2.0 ** -24, 1.0 - 2.0 ** -23], dtype=np.float32)
-    assert np.array_equal(got, np.tile(quad, 8)), got[:8]
+def _unpack_codes(codes, K, fmt):
+    if fmt == oracle.E4M3:
+        return codes.reshape(-1, K)
+    lo, hi = codes & 0xF, codes >> 4
+    return np.stack([lo, hi], axis=-1).reshape(-1, K)
 
 
-def test_fwht_involution_and_norm():
-    rng = np.random.default_rng(5)
-    for n in (32, 128):
-        v = rng.standard_normal(n).astype(np.float32)
-        back = oracle.fwht_f32(oracle.fwht_f32(v)).astype(np.float64) / n
-        assert np.abs(back - v).max() <= 1e-5 * np.abs(v).max()
-        c = oracle.hadamard_norm(n)
-        assert c == float(np.float32(1.0 / np.sqrt(n)))
-        assert abs(c * c * n - 1.0) < 1e-6
+@pytest.mark.parametrize("B", [32, 128])
+@pytest.mark.parametrize("fmt", ["e2m1", "e4m3"])
+@pytest.mark.parametrize("smooth", [False, True])
+def test_transform_matches_exact_rationals(B, fmt, smooth):
+    """Scales and codes of the definition on random rows with an outlier channel, every
+    one decided by exact rational comparisons."""
+    f = FMT[fmt]
+    emax = 2 if f == oracle.E2M1 else 8
+    rng = np.random.default_rng(B + 7 * f + int(smooth))
+    M, K = 3, 256
+    x = rng.standard_normal((M, K)) * 3.0
+    x[:, 5] *= 60.0
+    x[1, 40:72] *= 1e-3
+    bits = _bf16_bits(x)
+    mul = rng.uniform(0.25, 4.0, size=K).astype(np.float32) if smooth else None
+    o = oracle.quantize_transformed(bits, f, B, mul)
+    got_codes = _unpack_codes(o["codes"], K, f)
+    for r in range(M):
+        S = _exact.transform_exact(bits[r], B, mul)
+        for kb in range(K // 32):
+            blk = S[kb * 32:(kb + 1) * 32]
+            sc = _exact.scale_code_sqrt(blk, B, emax)
+            assert o["sf"][r, kb] == sc, (r, kb, o["sf"][r, kb], sc)
+            X = Fraction(2) ** (sc - 127)
+            for i, v in enumerate(blk):
+                want = _exact.nearest_code_sqrt(v, B, X, f)
+                assert got_codes[r, kb * 32 + i] == want, (r, kb, i, got_codes[r, kb * 32 + i], want)
+
+
+def _near_boundary_row(B, target):
+    """A row whose first rotation block is [x0, x1, x2, x3, 0, ...] with x0 + x1 + x2 + x3
+    equal to target to about 32 bits (four bf16 values taking 8 bits each), so that output
+    0 of the rotation, (x0 + .. + x3) / sqrt(B), lands within about 2^-30 of target / sqrt(B)."""
+    xs, rest = [], Fraction(target)
+    for _ in range(4):
+        b = int(_bf16_bits([float(rest)])[0])
+        xs.append(b)
+        rest -= _exact.bf16_fraction(b)
+    row = np.zeros(B, dtype=np.uint16)
+    row[:4] = xs
+    return row
+
+
+def test_transform_flags_values_near_a_grid_midpoint():
+    """Output 0 placed within 2^-30 (relative) of the E2M1 midpoint 5 (between 4 and 6) at
+    scale 1: a binary32 evaluation could round it either way, so the oracle reports two
+    candidate codes; its own code is the exact value's."""
+    import math
+    B = 32
+    for side in (-1, 1):
+        target = Fraction(5) * Fraction(math.sqrt(B)) * (1 + side * Fraction(1, 2 ** 31))
+        row = _near_boundary_row(B, target)
+        o = oracle.quantize_transformed(row[None, :], oracle.E2M1, B)
+        S = _exact.transform_exact(row, B)
+        sc = _exact.scale_code_sqrt(S[:32], B, 2)
+        assert o["sf"][0, 0] == sc == 127
+        want = _exact.nearest_code_sqrt(S[0], B, Fraction(1), oracle.E2M1)
+        assert _unpack_codes(o["codes"], B, oracle.E2M1)[0, 0] == want
+        assert {o["code_lo"][0, 0], o["code_hi"][0, 0]} == {6, 7}          # 4 or 6
+        assert (o["code_lo"][0, 1:] == o["code_hi"][0, 1:]).sum() >= 24  # the others mostly certain
+
+
+def test_transform_flags_a_scale_near_a_power_of_two():
+    """A block whose largest transformed value is within 2^-30 of 8: floor(log2) is 2 or 3
+    depending on rounding, so the block's scale is flagged; a block well inside a binade
+    is not."""
+    import math
+    B = 32
+    row = _near_boundary_row(B, Fraction(8) * Fraction(math.sqrt(B)) * (1 - Fraction(1, 2 ** 31)))
+    o = oracle.quantize_transformed(row[None, :], oracle.E2M1, B)
+    assert o["blk_amb"][0, 0] == 1
+    row2 = _near_boundary_row(B, Fraction(11) * Fraction(math.sqrt(B)))
+    o2 = oracle.quantize_transformed(row2[None, :], oracle.E2M1, B)
+    assert o2["blk_amb"][0, 0] == 0
+
+
+def test_transform_flags_possible_binary32_overflow():
+    x = np.zeros((1, 32), dtype=np.float32)
+    x[0, :4] = 2.0 ** 126
+    o = oracle.quantize_transformed(_bf16_bits(x), oracle.E4M3, 32)
+    assert o["blk_amb"][0, 0] == 2
+    assert o["sf"][0, 0] != 255        # the definition's block is finite (t = 2^126 * 4 / sqrt 32)
 
 
 @pytest.mark.parametrize("B", [32, 128])
 def test_transform_is_scaled_hadamard_rotation(B):
-    """The transformed values equal (x * mul) . blockdiag(H_B) / sqrt(B) (fp64) within
-    binary32 rounding; codes and scales dequantize to within one element step of them."""
+    """t equals (x * mul) . blockdiag(H_B) / sqrt(B) with scipy's Sylvester matrix in fp64 to
+    fp64 rounding; codes and scales dequantize to within one element step of t."""
     from scipy.linalg import hadamard
     rng = np.random.default_rng(B + 1)
     M, K = 6, 256
     x = (rng.standard_normal((M, K)) * 3).astype(np.float32)
-    x[:, 5] *= 60.0                                          # an outlier channel
-    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
+    x[:, 5] *= 60.0
+    bits = _bf16_bits(x)
     xb = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     mul = rng.uniform(0.5, 2.0, size=K).astype(np.float32)
-    codes, sf, t = oracle.quantize_transformed(bits, oracle.E2M1, B, mul)
+    o = oracle.quantize_transformed(bits, oracle.E2M1, B, mul)
     H = hadamard(B).astype(np.float64) / np.sqrt(B)
     want = np.concatenate([(xb * mul.astype(np.float64))[:, b0:b0 + B] @ H for b0 in range(0, K, B)], axis=1)
-    assert np.abs(t.astype(np.float64) - want).max() <= 1e-5 * np.abs(want).max()
-    deq = oracle.dequantize(codes, sf, K, oracle.E2M1)
-    scale = np.repeat(2.0 ** (sf.astype(np.float64) - 127), 32, axis=1)
-    assert (np.abs(deq - t) <= 2.0 * scale + 1e-30).all()   # within the largest E2M1 step (4 -> 6)
+    assert np.abs(o["t"] - want).max() <= 1e-13 * np.abs(want).max()
+    deq = oracle.dequantize(o["codes"], o["sf"], K, oracle.E2M1)
+    scale = np.repeat(2.0 ** (o["sf"].astype(np.float64) - 127), 32, axis=1)
+    assert (np.abs(deq - o["t"]) <= 2.0 * scale + 1e-30).all()   # within the largest E2M1 step (4 -> 6)
 
 
 def test_transform_power_of_two_smoothing_shifts_only_the_scales():
     """A smoothing multiplier of 2^j on every channel scales the transformed values exactly,
     so the element codes are unchanged and every scale code moves by j."""
     rng = np.random.default_rng(9)
-    x = (rng.standard_normal((4, 128)) * 2).astype(np.float32)
-    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
-    c0, s0, _ = oracle.quantize_transformed(bits, oracle.E4M3, 32, None)
-    c1, s1, _ = oracle.quantize_transformed(bits, oracle.E4M3, 32, np.full(128, 8.0, dtype=np.float32))
-    assert np.array_equal(c0, c1)
-    assert np.array_equal(s1.astype(int), s0.astype(int) + 3)
+    bits = _bf16_bits(rng.standard_normal((4, 128)) * 2)
+    o0 = oracle.quantize_transformed(bits, oracle.E4M3, 32, None)
+    o1 = oracle.quantize_transformed(bits, oracle.E4M3, 32, np.full(128, 8.0, dtype=np.float32))
+    assert np.array_equal(o0["codes"], o1["codes"])
+    assert np.array_equal(o1["sf"].astype(int), o0["sf"].astype(int) + 3)
 
 
 def test_transform_sign_symmetry():
     rng = np.random.default_rng(10)
-    x = rng.standard_normal((3, 128)).astype(np.float32)
-    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
-    c0, s0, t0 = oracle.quantize_transformed(bits, oracle.E4M3, 128, None)
-    c1, s1, t1 = oracle.quantize_transformed(bits ^ 0x8000, oracle.E4M3, 128, None)
-    assert np.array_equal(t1, -t0) and np.array_equal(s0, s1)
-    assert np.array_equal(c1[t0 != 0], c0[t0 != 0] ^ 0x80)
+    bits = _bf16_bits(rng.standard_normal((3, 128)))
+    o0 = oracle.quantize_transformed(bits, oracle.E4M3, 128, None)
+    o1 = oracle.quantize_transformed(bits ^ 0x8000, oracle.E4M3, 128, None)
+    assert np.array_equal(o1["t"], -o0["t"]) and np.array_equal(o0["sf"], o1["sf"])
+    nz = o0["t"] != 0
+    assert np.array_equal(o1["codes"][nz], o0["codes"][nz] ^ 0x80)
 
 
 # --- SVDQuant low-rank branch ------------------------------------------------------------------
