@@ -55,16 +55,15 @@ FP8_OVER_BF16 = 2.0   # 4.5 PFLOP/s FP8
 
 
 # DRAM traffic of one GEMM launch on a bench workload (dram__bytes_read.sum +
-# dram__bytes_write.sum from one ncu capture of that launch; the profile named holds the
-# command).  A record describes only the kernel built from the sources it was taken on:
-# when their hash differs the line reports traffic as null.
+# dram__bytes_write.sum from one ncu capture of that launch).  A record describes only the
+# kernel built from the sources it was taken on: when their hash differs the line reports
+# traffic as null.
 GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precision_mxq_b200/csrc/ptx.cuh",
                 "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h", "fp8_mixed_precision_mxq_b200/csrc/mx_elem.cuh"]
 GEMM_TRAFFIC = {
     ("ffn_up_480p_w4a4", 32760): {
         "bytes": 382355200 + 857401344,
-        "sources_sha256": "4ead914060badceb676f2b238216b77003cb214ce2fbea7c8c3ffcd69c695b4c",
-        "profile": "profiles/mx_gemm_mxf4_pair_ffn_up_480p_traffic.md"},
+        "sources_sha256": "4ead914060badceb676f2b238216b77003cb214ce2fbea7c8c3ffcd69c695b4c"},
 }
 
 

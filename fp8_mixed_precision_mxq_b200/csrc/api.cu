@@ -156,10 +156,6 @@ int run_linear(const void* x, int64_t M, int64_t K, const void* w_codes, const v
     return ok();
 }
 
-// fl32(1/s): the reciprocal the static quantizer multiplies by (an IEEE double division
-// rounded to binary32, which equals the correctly rounded binary32 division).
-float static_inverse(float s) { return static_cast<float>(1.0 / static_cast<double>(s)); }
-
 // fl32(1/sqrt B) for B = 2^j: 2^(-j/2) for even j, fl32(sqrt 2) * 2^(-(j+1)/2) for odd j
 // (scaling by a power of two is exact, so both are the correctly rounded value).
 float hadamard_norm(int B)
@@ -419,7 +415,7 @@ int mxq_quantize_act_static(const void* x_bf16, int64_t M, int64_t K, float scal
     RETURN_IF(check_ptr(sf, "sf"));
     RETURN_IF(check_device());
     snprintf(g_path, sizeof g_path, "quantize static e4m3");
-    return cuda_rc(launch_quantize_static(x_bf16, M, K, static_inverse(scale), codes, sf,
+    return cuda_rc(launch_quantize_static(x_bf16, M, K, scale, codes, sf,
                                           static_cast<cudaStream_t>(stream)),
                    "quantize launch");
 }
@@ -440,7 +436,7 @@ int mxq_linear_static(const void* x_bf16, int64_t M, int64_t K, const void* w_co
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* xc = static_cast<uint8_t*>(workspace);
     uint8_t* xs = xc + round_up(codes_bytes(M, K, MXQ_FMT_E4M3), kWsAlign);
-    RETURN_IF(cuda_rc(launch_quantize_static(x_bf16, M, K, static_inverse(act_scale), xc, xs, st), "quantize launch"));
+    RETURN_IF(cuda_rc(launch_quantize_static(x_bf16, M, K, act_scale, xc, xs, st), "quantize launch"));
     GemmArgs g{xc, xs, MXQ_FMT_E4M3, M, N, K, w_codes, w_sf, bias_bf16, y_bf16};
     g.alpha = act_scale;
     const char* msg = nullptr;
@@ -620,12 +616,49 @@ constexpr int64_t kNoAllocScratchBytes = int64_t(32) << 20;  // 32 MiB per devic
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kNoAllocMaxDevices = 64;
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+// Per device: the address found and the CUDA context it belongs to.  A device reset (or
+// the primary context being released and created again) loads the module anew, and the
+// array can then sit at another address; keying the cache on the context's unique ID
+// makes the first call in a new context look the address up again.
+struct NoAllocSlot {
+    void* ptr = nullptr;
+    unsigned long long ctx_id = 0;
+    bool have_id = false;
+};
+NoAllocSlot g_noalloc[kNoAllocMaxDevices];
 std::mutex g_noalloc_mu;
 
-// Device address of the scratch array on the current device.  In host code the array's
-// name is only a stand-in, so the address is looked up once per device (with that
-// device current) and cached.
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique ID of the calling thread's current CUDA context (the runtime's primary context
+// of the current device once it has been initialized), through the driver entry points
+// the runtime exposes; false if the driver lacks them.
+bool current_context_id(unsigned long long* id)
+{
+    static PfnCtxGetCurrent get_current = nullptr;
+    static PfnCtxGetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PfnCtxGetCurrent>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PfnCtxGetId>(p);
+    });
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array in the current device's context.  In host code the
+// array's name is only a stand-in, so the address is looked up (with that device current)
+// on the first call in each context and cached.
 int noalloc_scratch(void** out)
 {
     int dev = 0;
@@ -633,15 +666,27 @@ int noalloc_scratch(void** out)
     if (e != cudaSuccess) return fail(MXQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
     if (dev < 0 || dev >= kNoAllocMaxDevices)
         return fail(MXQ_ERR_UNSUPPORTED, "device index %d is above the supported %d", dev, kNoAllocMaxDevices);
+    unsigned long long id = 0;
+    bool have_id = current_context_id(&id);
+    if (!have_id) {
+        // no context current on this thread yet: make the device's primary context current
+        // (cudaSetDevice initializes it), then ask again
+        e = cudaSetDevice(dev);
+        if (e != cudaSuccess) return fail(MXQ_ERR_CUDA, "cudaSetDevice: %s", cudaGetErrorString(e));
+        have_id = current_context_id(&id);
+    }
     std::lock_guard<std::mutex> g(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    NoAllocSlot& slot = g_noalloc[dev];
+    if (!slot.ptr || slot.have_id != have_id || (have_id && slot.ctx_id != id)) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess || !p)
             return fail(MXQ_ERR_CUDA, "cudaGetSymbolAddress of the static scratch: %s", cudaGetErrorString(e));
-        g_noalloc_ptr[dev] = p;
+        slot.ptr = p;
+        slot.ctx_id = id;
+        slot.have_id = have_id;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = slot.ptr;
     return MXQ_OK;
 }
 

@@ -22,8 +22,8 @@ inline int64_t codes_bytes(int64_t rows, int64_t K, int fmt) { return fmt == kFm
 // ---- launchers (return cudaError_t of the launch) ----
 cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, int fmt, void* codes, void* sf,
                             cudaStream_t stream);
-// Static per-tensor E4M3: codes = RNE_sat(x * inv_scale), block scales 127.
-cudaError_t launch_quantize_static(const void* x, int64_t rows, int64_t K, float inv_scale, void* codes, void* sf,
+// Static per-tensor E4M3: codes = RNE_sat(x / scale) (the exact quotient), block scales 127.
+cudaError_t launch_quantize_static(const void* x, int64_t rows, int64_t K, float scale, void* codes, void* sf,
                                    cudaStream_t stream);
 // transform_on: t = x * mul (per channel; mul may be null), each `block` (32 or 128)
 // values along K rotated by the Hadamard matrix times norm, then MX-quantized in fmt.

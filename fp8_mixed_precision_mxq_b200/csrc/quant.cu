@@ -15,6 +15,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <cmath>
 #include <numeric>
 
 #include "mx_elem.cuh"
@@ -50,16 +51,72 @@ __device__ __forceinline__ uint32_t sf_offset(uint32_t r, uint32_t kb, uint32_t 
     return ((r >> 7) * atoms_k + (kb >> 2)) * 512u + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + (kb & 3u);
 }
 
-// Static per-tensor E4M3 (the format template argument kFmtStatic): every element is
-// multiplied by the tensor's fp32 inverse scale and rounded onto the E4M3 grid; the
-// block scales are all 127 (x1) and the GEMM applies the tensor scale to its sums.
+// Static per-tensor E4M3 (the format template argument kFmtStatic): every element x
+// becomes RNE_sat(x / s) on the E4M3 grid, x / s the exact quotient by the tensor's
+// scale s; the block scales are all 127 (x1) and the GEMM applies s to its sums.
 constexpr int kFmtStatic = 2;
+
+// The scale as the static quantizer takes it: s = sn * 2^-k with sn in [1, 2), the
+// reciprocal r = fl32(1/sn) in (1/2, 1], and 2^k split into two factors p1 * p2 that are
+// binary32 normals (k runs from -127 to 149).
+struct StaticScale {
+    float sn, r, p1, p2;
+};
+
+// One value's E4M3 code is RNE_sat(x / s), decided exactly in binary32:
+//  * xs = x * 2^k, so that x / s = xs / sn with sn in [1, 2) (exact, except overflow,
+//    where x / s is above 2^127 and saturates either way, and underflow, where x / s is
+//    below 2^-125 and rounds to a zero of x's sign either way); xs is clamped to the
+//    finite range (NaN kept), so that r <= 1 keeps every product below finite;
+//  * q0 = fl(xs * r), then one correction q = fl(q0 + fl(xs - q0 sn) * r) (fused
+//    multiply-adds: Markstein's iteration, M. Cornea, J. Harrison, P. Tang, "Scientific
+//    Computing on Itanium-based Systems", and J.-M. Muller et al., "Handbook of
+//    Floating-Point Arithmetic", section on division by Newton-Raphson iterations): the
+//    relative error of q0 is at most about 2^-23, the correction leaves about 2^-46 before
+//    its own rounding, so q is one of the two binary32 neighbours of xs / sn (faithful);
+//  * the remainder e = xs - q sn of a faithful quotient is a binary32 number whenever
+//    |xs| >= 2^-102 (both terms are multiples of 2^(floor(log2 |xs|) - 47)), so the fused
+//    multiply-add returns it exactly and its sign tells on which side of q the quotient
+//    lies; below 2^-102 the quotient is far under E4M3's smallest midpoint 2^-10;
+//  * q is then replaced by the quotient rounded to odd (truncated toward zero, the last
+//    bit set when inexact: S. Boldo, G. Melquiond, "Emulation of FMA and correctly rounded
+//    sums: proved algorithms using rounding to odd", IEEE TC 2008), and rounding a
+//    round-to-odd value of at least two more bits than the target gives the same result
+//    as rounding the exact value once: cvt's round-to-nearest-even then is the exact
+//    quotient's.
+__device__ __forceinline__ float round_to_odd(float q, float e)
+{
+    const uint32_t b = __float_as_uint(q);
+    // inexact and finite: step toward zero when the remainder's sign differs from q's
+    // (|x / s| < |q|), then set the last bit
+    const bool adj = e != 0.0f && (b & 0x7FFFFFFFu) < 0x7F800000u;
+    return __uint_as_float(adj ? ((b - ((__float_as_uint(e) ^ b) >> 31)) | 1u) : b);
+}
+
+__device__ __forceinline__ float clamp_finite_nan(float v)
+{
+    float d;
+    asm("min.NaN.f32 %0, %1, 0f7F7FFFFF;" : "=f"(d) : "f"(v));
+    asm("max.NaN.f32 %0, %1, 0fFF7FFFFF;" : "=f"(d) : "f"(d));
+    return d;
+}
+
+__device__ __forceinline__ float2 static_quotient2(float2 x, const StaticScale& st)
+{
+    float2 xs = __fmul2_rn(__fmul2_rn(x, make_float2(st.p1, st.p1)), make_float2(st.p2, st.p2));
+    xs = make_float2(clamp_finite_nan(xs.x), clamp_finite_nan(xs.y));
+    const float2 r = make_float2(st.r, st.r), ns = make_float2(-st.sn, -st.sn);
+    const float2 q0 = __fmul2_rn(xs, r);
+    const float2 q = __ffma2_rn(__ffma2_rn(q0, ns, xs), r, q0);
+    const float2 e = __ffma2_rn(q, ns, xs);
+    return make_float2(round_to_odd(q.x, e.x), round_to_odd(q.y, e.y));
+}
 
 template <int FMT>
 __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restrict__ x, uint32_t n_groups,
                                                             uint32_t KB, uint64_t kb_magic, uint32_t atoms_k,
                                                             uint32_t rows, uint8_t* __restrict__ codes,
-                                                            uint8_t* __restrict__ sf, float static_inv)
+                                                            uint8_t* __restrict__ sf, StaticScale st)
 {
     constexpr bool kStatic = FMT == kFmtStatic;
     constexpr int kElem = kStatic ? kFmtE4M3 : FMT;
@@ -81,11 +138,10 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             uint32_t sc;
-            float inv;
+            float inv = 1.0f;
             if constexpr (kStatic) {
                 if (g[u] >= n_groups) continue;
                 sc = 127u;
-                inv = static_inv;
             } else {
                 // block absmax over the quad of lanes holding the 32 elements
                 uint32_t m2 = absmax_bf16x2(absmax_bf16x2(v[u].x, v[u].y), absmax_bf16x2(v[u].z, v[u].w));
@@ -99,11 +155,16 @@ __global__ void __launch_bounds__(kThreads) quantize_kernel(const uint4* __restr
                 inv = __uint_as_float((254u - min(sc, 253u)) << 23);  // 2^(127 - sc)
             }
             const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-            // x * 2^-s, two lanes of binary32 a multiply (each rounded as the scalar one)
-            const float2 inv2 = make_float2(inv, inv);
             float2 f[4];
+            if constexpr (kStatic) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) f[i] = __fmul2_rn(make_float2(lo_f(w[i]), hi_f(w[i])), inv2);
+                for (int i = 0; i < 4; ++i) f[i] = static_quotient2(make_float2(lo_f(w[i]), hi_f(w[i])), st);
+            } else {
+                // x * 2^-s, two lanes of binary32 a multiply (each rounded as the scalar one)
+                const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) f[i] = __fmul2_rn(make_float2(lo_f(w[i]), hi_f(w[i])), inv2);
+            }
             const uint32_t keep = sc == 255u ? 0u : 0xFFFFFFFFu;
             // cvt rounds to nearest even, saturates, and keeps the sign of a value that
             // rounds to zero (-0 = 0x8 / 0x80), as the format reading requires
@@ -463,10 +524,22 @@ __global__ void __launch_bounds__(kTThreads, 5) quantize_transform_kernel(
 }  // namespace
 
 // fmt: kFmtE2M1 / kFmtE4M3 (MX, scales from each block's abs-max) or kFmtStatic (E4M3
-// with the fixed inverse scale static_inv and block scales 127).
-cudaError_t launch_quantize_any(const void* x, int64_t rows, int64_t K, int fmt, float static_inv, void* codes,
+// of x / scale with block scales 127; scale positive and finite).
+cudaError_t launch_quantize_any(const void* x, int64_t rows, int64_t K, int fmt, float scale, void* codes,
                                 void* sf, cudaStream_t stream)
 {
+    StaticScale st{1.0f, 1.0f, 1.0f, 1.0f};
+    if (fmt == kFmtStatic) {
+        int e = 0;
+        const float m = std::frexp(scale, &e);  // scale = m 2^e, m in [1/2, 1)
+        const int k = 1 - e;                    // sn = scale 2^k in [1, 2)
+        st.sn = 2.0f * m;
+        // fl32(1/sn): the double quotient is never within 2^-53 of a binary32 midpoint
+        // unless it is one, so rounding it to binary32 gives the correctly rounded value
+        st.r = static_cast<float>(1.0 / static_cast<double>(st.sn));
+        st.p1 = std::ldexp(1.0f, k / 2);
+        st.p2 = std::ldexp(1.0f, k - k / 2);
+    }
     const uint32_t n_groups = static_cast<uint32_t>(rows * K / 8);
     const uint32_t KB = static_cast<uint32_t>(K / 32);
     const uint32_t atoms_k = static_cast<uint32_t>(sf_atoms_k(K));
@@ -483,12 +556,11 @@ cudaError_t launch_quantize_any(const void* x, int64_t rows, int64_t K, int fmt,
     uint8_t* f = static_cast<uint8_t*>(sf);
     const uint32_t r = static_cast<uint32_t>(rows);
     if (fmt == kFmtStatic)
-        quantize_kernel<kFmtStatic><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k, r, c, f,
-                                                                   static_inv);
+        quantize_kernel<kFmtStatic><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k, r, c, f, st);
     else if (fmt == kFmtE4M3)
-        quantize_kernel<kFmtE4M3><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k, r, c, f, 0.f);
+        quantize_kernel<kFmtE4M3><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k, r, c, f, st);
     else
-        quantize_kernel<kFmtE2M1><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k, r, c, f, 0.f);
+        quantize_kernel<kFmtE2M1><<<grid, kThreads, 0, stream>>>(xv, n_groups, KB, kb_magic, atoms_k, r, c, f, st);
     return cudaGetLastError();
 }
 
@@ -498,10 +570,10 @@ cudaError_t launch_quantize(const void* x, int64_t rows, int64_t K, int fmt, voi
     return launch_quantize_any(x, rows, K, fmt, 0.f, codes, sf, stream);
 }
 
-cudaError_t launch_quantize_static(const void* x, int64_t rows, int64_t K, float inv_scale, void* codes, void* sf,
+cudaError_t launch_quantize_static(const void* x, int64_t rows, int64_t K, float scale, void* codes, void* sf,
                                    cudaStream_t stream)
 {
-    return launch_quantize_any(x, rows, K, kFmtStatic, inv_scale, codes, sf, stream);
+    return launch_quantize_any(x, rows, K, kFmtStatic, scale, codes, sf, stream);
 }
 
 cudaError_t launch_quantize_transform(const void* x, int64_t rows, int64_t K, int fmt, const float* mul, int block,

@@ -153,13 +153,17 @@ int64_t mxq_block_workspace_bytes(const mxq_wdesc* w, const int64_t* M_in, uint3
  * device array of mxq_linear_noalloc_max_scratch_bytes() bytes (32 MiB) that every GPU
  * loading the library holds until the process exits; the call allocates and frees
  * nothing.  Inputs and outputs are as for mxq_linear.  Inputs whose scratch would not fit
- * (M*K above about 63 million elements for E2M1, 32 million for E4M3) return
- * MXQ_ERR_WORKSPACE and launch nothing.  The first call on a device looks up the array's device address and
- * caches it; make that first call before any stream capture.  All calls on a device share
- * the one array, and it keeps the last call's contents (nothing in it needs to start at
- * zero: every byte the GEMM reads is written by the same call's quantizer), so calls that
- * overlap on the GPU -- on different streams or from different threads without ordering --
- * race and must be avoided.  The blog has no counterpart of this entry point. */
+ * (mxq_workspace_bytes(M, N, K, act_fmt, MXQ_MODE_NATIVE) above the array's size: M*K
+ * above about 63 million elements for E2M1, 32 million for E4M3) return
+ * MXQ_ERR_WORKSPACE and launch nothing.  The first call on a device looks up the array's
+ * device address and caches it; make that first call before any stream capture.  The
+ * cache is keyed on the device's CUDA context, so after a device reset (or a new primary
+ * context) the next call looks the address up again, and that call too should come
+ * before any capture.  All calls on a device share the one array, and it keeps the last
+ * call's contents (nothing in it needs to start at zero: every byte the GEMM reads is
+ * written by the same call's quantizer), so calls that overlap on the GPU -- on
+ * different streams or from different threads without ordering -- race and must be
+ * avoided.  The blog has no counterpart of this entry point. */
 int mxq_linear_noalloc(const void* x_bf16, int64_t M, int64_t K, const void* w_codes, const void* w_sf, int64_t N,
                        const void* bias_bf16, int act_fmt, void* y_bf16, void* stream);
 
@@ -209,12 +213,13 @@ int64_t mxq_ffn_workspace_bytes(int64_t M, int64_t K, int64_t H, int up_fmt, int
 
 /* Static per-tensor FP8 E4M3 activations: the blog's W4A8 as its "Quantization formats"
  * table names it ("FP8 E4M3 static activations"), one scale for the whole tensor fixed
- * offline.  codes[m, k] = E4M3 RNE, saturating, of fl32(x[m, k] * fl32(1/scale)); sf is
- * written in the tiled layout with every block's scale 127 (x1) and the padding 0, so
- * the codes feed the kind::mxf8f6f4 GEMM unchanged; the tensor scale goes to the GEMM
- * (mxq_linear_static).  scale > 0 and finite (MXQ_ERR_INVALID_ARG otherwise); inputs
- * are expected finite (Inf saturates to +-448, NaN gives an E4M3 NaN code).  Sizes and
- * alignment as for mxq_quantize_act with fmt E4M3. */
+ * offline.  codes[m, k] = E4M3 RNE, saturating, of the exact quotient x[m, k] / scale
+ * (decided exactly for every bf16 input and every positive finite binary32 scale: no
+ * rounding of the quotient to binary32 comes between); sf is written in the tiled layout
+ * with every block's scale 127 (x1) and the padding 0, so the codes feed the
+ * kind::mxf8f6f4 GEMM unchanged; the tensor scale goes to the GEMM (mxq_linear_static).
+ * scale > 0 and finite (MXQ_ERR_INVALID_ARG otherwise); Inf inputs saturate to +-448, NaN
+ * gives an E4M3 NaN code.  Sizes and alignment as for mxq_quantize_act with fmt E4M3. */
 int mxq_quantize_act_static(const void* x_bf16, int64_t M, int64_t K, float scale, void* codes, void* sf,
                             void* stream);
 

@@ -192,3 +192,29 @@ def test_gemm_quant_binding_rejects_unknown_activation():
     from fp8_mixed_precision_mxq_b200 import ops
     with pytest.raises(ValueError):
         ops.gemm_quant(None, None, "e2m1", 128, 256, None, act="relu")
+
+
+def test_linear_entry_points_reject_unsupported_shapes_with_their_reason():
+    """The shape limits the header states, through every entry point that runs a GEMM:
+    N % 8 != 0 and, for native W4A8, K % 128 != 0 return MXQ_ERR_SHAPE with the reason
+    in mxq_last_error(), before anything needs a device."""
+    L = _lib.lib()
+    ws = V(1 << 20)
+    for mode in (0, 1):
+        assert L.mxq_linear(A16, 128, 256, A16, A16, 250, None, 0, mode, ws, 1 << 30, A16, None) == _lib.ERR_SHAPE
+        assert "multiple of 8" in _lib.last_error()
+    assert L.mxq_linear(A16, 128, 96, A16, A16, 256, None, 1, 0, ws, 1 << 30, A16, None) == _lib.ERR_SHAPE
+    assert "K % 128" in _lib.last_error()
+    assert L.mxq_linear_noalloc(A16, 128, 96, A16, A16, 256, None, 1, A16, None) == _lib.ERR_SHAPE
+    assert "K % 128" in _lib.last_error()
+    assert L.mxq_linear_noalloc(A16, 128, 256, A16, A16, 252, None, 0, A16, None) == _lib.ERR_SHAPE
+    assert "multiple of 8" in _lib.last_error()
+    # W4A4 takes K = 96 (only native W4A8 expands the weight in 128-element steps)
+    rc = L.mxq_linear(A16, 128, 96, A16, A16, 256, None, 0, 0, ws, 1 << 30, A16, None)
+    assert rc != _lib.ERR_SHAPE, _lib.last_error()
+    descs = (_lib.WDesc * 8)(*[_lib.WDesc(4096, 4096, None, 256, 96)] * 8)
+    xs = (ctypes.c_void_p * 8)(*[4096] * 8)
+    ms = (ctypes.c_int64 * 8)(*[128] * 8)
+    ys = (ctypes.c_void_p * 8)(*[4096] * 8)
+    assert L.mxq_dit_block_linears(descs, xs, ms, ys, 0x80, 0, ws, 1 << 30, None) == _lib.ERR_SHAPE
+    assert "block linear 7" in _lib.last_error() and "K % 128" in _lib.last_error()

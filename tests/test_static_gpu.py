@@ -1,13 +1,17 @@
 """Static per-tensor FP8 E4M3 activations (the blog's W4A8 as its "Quantization formats"
-table names it): calibration by abs-max, codes bit-exact against the oracle, block scales
-all 127 in the tiled layout, and the scaled W4A8 linear within the GEMM tolerance."""
+table names it): calibration by abs-max, codes bit-exact against the oracle's exact
+quotient RNE_sat(x / s) -- including inputs whose code a binary32 evaluation of x / s would
+get wrong, and scales across the whole binary32 range -- block scales all 127 in the tiled
+layout, and the scaled W4A8 linear within the GEMM tolerance."""
+from fractions import Fraction
+
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import synth
-from tests import _mx
+from tests import _exact, _mx
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +46,58 @@ def test_quantize_static_bitexact(M, K, scale_kind):
             i, int((got != want).sum()), got[i], want[i], _mx.bits(x).reshape(-1)[i]))
     logical = np.full((M, K // 32), 127, dtype=np.uint8)
     assert np.array_equal(sf.cpu().numpy(), oracle.sf_to_tiled(logical, K))
+
+
+def _check_static(x_cpu, scale, what):
+    ops = _ops()
+    codes, sf = ops.quantize_act_static(x_cpu.cuda(), scale)
+    torch.cuda.synchronize()
+    want = oracle.quantize_static_e4m3(_mx.bits(x_cpu), scale).reshape(-1)
+    got = codes.cpu().numpy()[: x_cpu.numel()]
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, "%s: %d codes differ, first %d: gpu %#x oracle %#x (x bits %#x, s %r)" % (
+        what, bad.size, bad[0], got[bad[0]], want[bad[0]], _mx.bits(x_cpu).reshape(-1)[bad[0]], scale)
+
+
+def test_quantize_static_near_ties():
+    """Inputs whose E4M3 code is decided by less than a binary32 rounding: for each scale s
+    of the exhaustive search in tests/_exact.py, the bf16 values x whose binary32 quotient
+    or binary32 product x * fl32(1/s) lies on or across an E4M3 midpoint from x / s,
+    scaled by powers of two across the E4M3 range, both signs, amid random fill."""
+    cases = _exact.static_near_ties()
+    by_scale = {}
+    for s, x in cases:
+        by_scale.setdefault(s, []).append(x)
+    scales = sorted(by_scale)[:: max(1, len(by_scale) // 24)]
+    g = torch.Generator().manual_seed(7)
+    for s in scales:
+        vals = [x * Fraction(2) ** j for x in by_scale[s] for j in range(-6, 9)]
+        vals = [v for v in vals if Fraction(2) ** -9 <= v / s <= 448]
+        bits = [_exact.bf16_bits(v) for v in vals] + [_exact.bf16_bits(v) | 0x8000 for v in vals]
+        K = 64
+        n = (len(bits) + K - 1) // K * K
+        fill = (torch.randn(n, generator=g) * float(s) * 30).to(torch.bfloat16)
+        fb = fill.view(torch.int16).numpy().view(np.uint16).copy()
+        fb[: len(bits)] = np.array(bits, dtype=np.uint16)
+        x = torch.from_numpy(fb.view(np.int16)).view(torch.bfloat16).reshape(n // K, K)
+        _check_static(x, float(s), "near ties, s=%r" % float(s))
+
+
+@pytest.mark.parametrize("scale", [2.0 ** -149, 3.0 * 2.0 ** -140, 1.1e-30, 0.7, 5.5e20, 3.0e38])
+def test_quantize_static_extreme_scales_and_special_values(scale):
+    """Scales from the smallest binary32 subnormal to near the largest finite value, with
+    inputs from bf16 subnormals to the largest bf16, infinities (saturate to +-448) and
+    NaN (the E4M3 NaN code)."""
+    g = torch.Generator().manual_seed(int(np.log2(scale) + 200))
+    M, K = 64, 256
+    e = torch.randint(-140, 128, (M, K), generator=g).double()
+    x = (torch.randn(M, K, generator=g, dtype=torch.float64) * 2.0 ** e).clamp(-3.0e38, 3.0e38).to(torch.bfloat16)
+    x[0, 0], x[0, 1], x[0, 2], x[0, 3] = float("inf"), float("-inf"), float("nan"), -0.0
+    x[1, :8] = torch.tensor([3.3895e38, -3.3895e38, 2.0 ** -133, -(2.0 ** -133), 2.0 ** -126, 1.0, -1.0, 0.0])
+    # values near the scale itself, where the codes are neither zero nor saturated
+    x[2:10] = (torch.randn(8, K, generator=g, dtype=torch.float64) * scale * 100).clamp(-3.0e38, 3.0e38).to(
+        torch.bfloat16)
+    _check_static(x, scale, "extreme scale")
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 128), (300, 520, 1024), (1, 8, 128), (513, 768, 2048)])

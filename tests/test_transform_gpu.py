@@ -1,7 +1,10 @@
 """The transform_on path (blog section "Mixed-Precision selection": smoothing and a fixed
-Hadamard rotation before quantization): codes and scales bit-exact against the oracle,
-which takes the same binary32 steps in the same order, and the transformed linear within
-the GEMM tolerance of the oracle's product of the transformed operands."""
+Hadamard rotation before quantization), checked against the oracle's definition
+t = (x * mul) . blockdiag(H_B) / sqrt(B) taken in fp64: scales and codes bit-exact wherever
+the definition's value is farther from a decision boundary than the error bound of a
+binary32 evaluation, one of the two neighbouring codes within it (tests/_mx.py,
+check_transformed); the transformed linear within the GEMM tolerance of the oracle's
+product of the transformed operands."""
 import numpy as np
 import pytest
 import torch
@@ -28,20 +31,15 @@ def smooth_scales(x, alpha=0.5, seed=0):
 @pytest.mark.parametrize("block", [32, 128])
 @pytest.mark.parametrize("smooth", [False, True])
 @pytest.mark.parametrize("M,K", [(1, 128), (129, 256), (300, 1024)])
-def test_quantize_transformed_bitexact(fmt, block, smooth, M, K):
+def test_quantize_transformed_against_definition(fmt, block, smooth, M, K):
     ops = _ops()
     x = synth.activation(M, K, "student_t", seed=M + K + block, device="cuda", outlier_frac=0.02, outlier_scale=40.0)
     mul = (1.0 / smooth_scales(x)).contiguous() if smooth else None
     codes, sf = ops.quantize_act_transformed(x, fmt, block, mul)
     torch.cuda.synchronize()
-    c_ref, s_ref, _ = oracle.quantize_transformed(_mx.bits(x), _mx.FMT[fmt], block,
-                                                  None if mul is None else mul.cpu().numpy())
-    c_gpu = codes.cpu().numpy()
-    if not np.array_equal(c_gpu, c_ref.reshape(-1)):
-        i = int(np.nonzero(c_gpu != c_ref.reshape(-1))[0][0])
-        raise AssertionError("%d codes differ, first at byte %d: gpu %#x oracle %#x" % (
-            int((c_gpu != c_ref.reshape(-1)).sum()), i, c_gpu[i], c_ref.reshape(-1)[i]))
-    assert np.array_equal(sf.cpu().numpy(), oracle.sf_to_tiled(s_ref, K))
+    ref = oracle.quantize_transformed(_mx.bits(x), _mx.FMT[fmt], block, None if mul is None else mul.cpu().numpy())
+    _mx.check_transformed(codes, sf, M, K, fmt, ref, "%s B=%d smooth=%s %dx%d" % (fmt, block, smooth, M, K),
+                          max_uncertain=1e-3 if M * K >= 10000 else 0.01)
 
 
 @pytest.mark.parametrize("block", [32, 128])
@@ -57,9 +55,9 @@ def test_transformed_linear_against_oracle(block):
     y = ops.linear_transformed(x, qw, "e2m1", block, inv_s)
     assert ops.poll_status() == 0
     assert "hadamard%d smooth" % block in ops.last_path()
-    xc, xs, _ = oracle.quantize_transformed(_mx.bits(x), oracle.E2M1, block, inv_s.cpu().numpy())
-    wc, ws, _ = oracle.quantize_transformed(_mx.bits(w), oracle.E2M1, block, s.cpu().numpy())
-    ref = oracle.linear_rows(xc, xs, oracle.E2M1, np.arange(M), K, wc, ws, _mx.bits(b))
+    xo = oracle.quantize_transformed(_mx.bits(x), oracle.E2M1, block, inv_s.cpu().numpy())
+    wo = oracle.quantize_transformed(_mx.bits(w), oracle.E2M1, block, s.cpu().numpy())
+    ref = oracle.linear_rows(xo["codes"], xo["sf"], oracle.E2M1, np.arange(M), K, wo["codes"], wo["sf"], _mx.bits(b))
     _mx.assert_gemm_close(_mx.bf16_to_f64(y), ref, "transformed linear, block %d" % block)
     # the transforms cancel: the result approximates the unquantized product
     exact = (x.double() @ w.double().T + b.double()).cpu().numpy()
@@ -112,8 +110,10 @@ def special_input(M, K, seed):
 @pytest.mark.parametrize("block", [32, 128])
 @pytest.mark.parametrize("smooth", [False, True])
 def test_quantize_transformed_special_values(fmt, block, smooth):
-    """Codes and scales bit-exact against the oracle on subnormal, overflowing and
-    non-finite inputs: the binary32 steps round there exactly as the oracle's."""
+    """Subnormal, overflowing and non-finite inputs against the definition: non-finite
+    blocks get scale 255 and zero codes on both sides; blocks whose rotation could overflow
+    binary32, or whose values sit in the subnormal range where binary32 rounds absolutely,
+    fall in the oracle's uncertain set, and every certain scale and code is exact."""
     ops = _ops()
     M, K = 48, 512
     x = special_input(M, K, seed=block + (7 if smooth else 0))
@@ -124,14 +124,9 @@ def test_quantize_transformed_special_values(fmt, block, smooth):
     xd = x.cuda()
     codes, sf = ops.quantize_act_transformed(xd, fmt, block, None if mul is None else mul.cuda())
     torch.cuda.synchronize()
-    c_ref, s_ref, _ = oracle.quantize_transformed(_mx.bits(x), _mx.FMT[fmt], block,
-                                                  None if mul is None else mul.numpy())
-    assert (s_ref == 255).any() and (s_ref == 0).any()  # the input reaches both ends of the scale range
-    assert np.array_equal(sf.cpu().numpy(), oracle.sf_to_tiled(s_ref, K))
-    c_gpu = codes.cpu().numpy()
-    bad = np.nonzero(c_gpu != c_ref.reshape(-1))[0]
-    assert bad.size == 0, "%d codes differ, first at byte %d: gpu %#x oracle %#x" % (
-        bad.size, bad[0], c_gpu[bad[0]], c_ref.reshape(-1)[bad[0]])
+    ref = oracle.quantize_transformed(_mx.bits(x), _mx.FMT[fmt], block, None if mul is None else mul.numpy())
+    assert (ref["sf"] == 255).any() and (ref["sf"] == 0).any()  # the input reaches both ends of the scale range
+    _mx.check_transformed(codes, sf, M, K, fmt, ref, "special values", max_uncertain=None)
 
 
 @pytest.mark.parametrize("fmt", ["e2m1", "e4m3"])
@@ -141,24 +136,21 @@ def test_quantize_transformed_multi_span(fmt, block, M, K):
     """Tensors of more MX blocks than the launch has lanes (148 SMs x 32 CTAs x 128), so
     every warp takes several spans and the per-channel multipliers it holds must stay the
     ones of its channels; K = 2176 and 5120 make the launch round its grid to multiples of
-    17 and 5 CTAs.  Whole tensor bit-exact against the oracle."""
+    17 and 5 CTAs.  Whole tensor against the definition."""
     ops = _ops()
     x = synth.activation(M, K, "student_t", seed=M + block, device="cuda", outlier_frac=0.02, outlier_scale=40.0)
     mul = (1.0 / smooth_scales(x)).contiguous()
     codes, sf = ops.quantize_act_transformed(x, fmt, block, mul)
     torch.cuda.synchronize()
-    c_ref, s_ref, _ = oracle.quantize_transformed(_mx.bits(x), _mx.FMT[fmt], block, mul.cpu().numpy())
-    assert np.array_equal(sf.cpu().numpy(), oracle.sf_to_tiled(s_ref, K))
-    c_gpu = codes.cpu().numpy()
-    bad = np.nonzero(c_gpu != c_ref.reshape(-1))[0]
-    assert bad.size == 0, "%d codes differ, first at byte %d (row %d)" % (bad.size, bad[0], bad[0] // (c_gpu.size // M))
+    ref = oracle.quantize_transformed(_mx.bits(x), _mx.FMT[fmt], block, mul.cpu().numpy())
+    _mx.check_transformed(codes, sf, M, K, fmt, ref, "multi-span %dx%d" % (M, K))
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("block", [32, 128])
 def test_transform_full_ffn_up_480p(block):
     """The bench's transform_on workload at full size (M = 32760, K = 5120, SmoothQuant-style
-    multipliers): the quantizer's codes and scales bit-exact against the oracle on the whole
+    multipliers): the quantizer's codes and scales against the definition on the whole
     tensor, in the launch configuration the bench times; the transformed linear (N = 13824)
     within the GEMM tolerance on one row per 128-row tile plus the ends."""
     ops = _ops()
@@ -169,17 +161,15 @@ def test_transform_full_ffn_up_480p(block):
     codes, sf = ops.quantize_act_transformed(x, "e2m1", block, inv_s)
     torch.cuda.synchronize()
     xb = _mx.bits(x)
-    c_ref, s_ref, _ = oracle.quantize_transformed(xb, oracle.E2M1, block, inv_s.cpu().numpy())
-    assert np.array_equal(sf.cpu().numpy(), oracle.sf_to_tiled(s_ref, K))
-    c_gpu = codes.cpu().numpy()
-    bad = np.nonzero(c_gpu != c_ref.reshape(-1))[0]
-    assert bad.size == 0, "%d codes differ, first at byte %d" % (bad.size, bad[0])
+    ref = oracle.quantize_transformed(xb, oracle.E2M1, block, inv_s.cpu().numpy())
+    n_unc = _mx.check_transformed(codes, sf, M, K, "e2m1", ref, "480p B=%d" % block)
+    print("480p transform B=%d: %d uncertain elements of %d" % (block, n_unc, M * K))
     qw = ops.quantize_weight_transformed(w, bias=b, block=block, mul=s)
     y = ops.linear_transformed(x, qw, "e2m1", block, inv_s)
     assert ops.poll_status() == 0
     rows = synth.sample_rows(M).numpy()
-    wc, ws, _ = oracle.quantize_transformed(_mx.bits(w), oracle.E2M1, block, s.cpu().numpy())
+    wo = oracle.quantize_transformed(_mx.bits(w), oracle.E2M1, block, s.cpu().numpy())
     K2 = K // 2
-    ref = oracle.linear_rows(c_ref.reshape(M, K2)[rows], s_ref[rows], oracle.E2M1, np.arange(len(rows)), K, wc, ws,
-                             _mx.bits(b))
-    _mx.assert_gemm_close(_mx.bf16_to_f64(y[torch.from_numpy(rows).cuda()]), ref, "transformed linear 480p")
+    ref_y = oracle.linear_rows(ref["codes"].reshape(M, K2)[rows], ref["sf"][rows], oracle.E2M1, np.arange(len(rows)),
+                               K, wo["codes"], wo["sf"], _mx.bits(b))
+    _mx.assert_gemm_close(_mx.bf16_to_f64(y[torch.from_numpy(rows).cuda()]), ref_y, "transformed linear 480p")

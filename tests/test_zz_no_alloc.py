@@ -1,15 +1,18 @@
 """mxq_linear_noalloc: the native linear for callers that cannot allocate device memory
 where they run a layer (for example under a memory manager that owns the device pool, or
 in a plugin handed only its input and output buffers).  Its scratch is a fixed static
-device array, so these tests check, through the C ABI, that it gives the same result as
-mxq_linear with a caller workspace on two calls in a row (the second call reuses the
-array the first one left behind), and that inputs too large for the array are refused."""
+device array, so these tests check, through the C ABI, that it gives bit for bit the
+result of mxq_linear with a caller workspace on two calls in a row (the second call
+reuses the array the first one left behind), that the result is the oracle's linear
+within the GEMM tolerance, that the largest inputs the array holds work and the next
+larger ones are refused."""
 import ctypes
 
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 from tests import _mx
 
@@ -35,7 +38,9 @@ def test_noalloc_matches_workspace_linear_on_two_calls(fmt):
     L = lib.lib()
     M, N, K = 1000, 1288, 2048
     w = synth.weight(N, K, seed=41, device="cuda")
-    qw = ops.quantize_weight(w, bias=synth.bias(N, seed=41, device="cuda"))
+    b = synth.bias(N, seed=41, device="cuda")
+    qw = ops.quantize_weight(w, bias=b)
+    wc, ws, _ = _mx.oracle_quantize(w, "e2m1")
     for call, seed in enumerate((42, 43)):
         x = synth.activation(M, K, "student_t" if fmt == "e2m1" else "gelu", seed=seed, device="cuda",
                              outlier_frac=0.02, outlier_scale=40.0)
@@ -44,22 +49,50 @@ def test_noalloc_matches_workspace_linear_on_two_calls(fmt):
         rc = _call_noalloc(L, x, qw, fmt, y)
         assert rc == lib.OK, lib.last_error()
         assert ops.poll_status() == 0
-        _mx.assert_gemm_close(_mx.bf16_to_f64(y), _mx.bf16_to_f64(y_ref), "noalloc %s call %d" % (fmt, call))
+        # the same kernels on the same bytes: identical output
+        assert torch.equal(y, y_ref), "noalloc %s call %d differs from mxq_linear" % (fmt, call)
+        if call == 0:
+            xc, xs, _ = _mx.oracle_quantize(x, fmt)
+            rows = np.arange(0, M, 7)
+            ref = oracle.linear_rows(xc, xs, _mx.FMT[fmt], rows, K, wc, ws, _mx.bits(b))
+            _mx.assert_gemm_close(_mx.bf16_to_f64(y[torch.from_numpy(rows).cuda()]), ref, "noalloc %s" % fmt)
 
 
-def test_noalloc_rejects_inputs_beyond_the_static_scratch():
+def _largest_rows(ops, K, N, fmt, cap):
+    """The largest M whose native workspace fits the static scratch."""
+    lo, hi = 1, cap
+    while lo < hi:
+        mid = (lo + hi + 1) // 2
+        if ops.workspace_bytes(mid, N, K, fmt) <= cap:
+            lo = mid
+        else:
+            hi = mid - 1
+    return lo
+
+
+@pytest.mark.parametrize("fmt", ["e2m1", "e4m3"])
+def test_noalloc_largest_accepted_input_and_the_next_one(fmt):
+    """At the largest M whose scratch fits the array exactly (K = 5120) the entry point runs
+    and equals mxq_linear bit for bit; M + 1 needs more and is refused with nothing
+    launched.  The header's limits (about 63 M elements of M*K for E2M1, 32 M for E4M3)
+    follow from it."""
     from fp8_mixed_precision_mxq_b200 import ops
     lib = _abi()
     L = lib.lib()
     cap = L.mxq_linear_noalloc_max_scratch_bytes()
-    assert cap > 0
     K, N = 5120, 256
-    M = int(cap // K) + 256  # E4M3 needs a little over M*K bytes: beyond the array
-    x = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
-    qw = ops.quantize_weight(synth.weight(N, K, seed=1, device="cuda"))
-    y = torch.zeros((M, N), dtype=torch.bfloat16, device="cuda")
-    rc = _call_noalloc(L, x, qw, "e4m3", y)
-    assert rc == lib.ERR_WORKSPACE
+    M = _largest_rows(ops, K, N, fmt, cap)
+    assert ops.workspace_bytes(M, N, K, fmt) <= cap < ops.workspace_bytes(M + 1, N, K, fmt)
+    limit = 63e6 if fmt == "e2m1" else 32e6
+    assert abs(M * K - limit) < 0.05 * limit, M * K
+    qw = ops.quantize_weight(synth.weight(N, K, seed=2, device="cuda"), bias=synth.bias(N, seed=2, device="cuda"))
+    x = synth.activation(M + 1, K, "normal", seed=3, device="cuda", outlier_frac=0.01, outlier_scale=30.0)
+    xm = x[:M]
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    assert _call_noalloc(L, xm, qw, fmt, y) == lib.OK, lib.last_error()
+    assert torch.equal(y, ops.linear(xm, qw, fmt=fmt))
+    y1 = torch.zeros((M + 1, N), dtype=torch.bfloat16, device="cuda")
+    assert _call_noalloc(L, x, qw, fmt, y1) == lib.ERR_WORKSPACE
     assert "static scratch" in lib.last_error()
     torch.cuda.synchronize()
-    assert not y.any()  # nothing was launched
+    assert not y1.any()  # nothing was launched
