@@ -2,20 +2,22 @@
 
 A step is one pass of the hot path over one batch: the dynamic activation quantizer
 followed by the block-scaled tcgen05 GEMM (mxq_linear), on the W4A4 FFN-up linear of a
-Wan2.2-A14B-shaped DiT block at 480p / 81 frames (M = 32760 tokens, K = 5120,
-N = 13824; Student-t activations with 1% outlier channels, N(0, 0.02^2) weights,
-random-init, synthetic).  The MXFP4 weight is quantized once, before timing (it is a
-load-time step).  Beside the headline number the JSON line carries:
+Wan2.2-A14B-shaped DiT block at 720p / 81 frames (M = 75600 tokens, K = 5120, N = 13824;
+Student-t activations with 1% outlier channels, N(0, 0.02^2) weights, random-init,
+synthetic), the shape the 60 %-of-FP4 target is stated for.  The MXFP4 weight is quantized
+once, before timing (a load-time step).  Beside the headline number the JSON line carries:
+  step_ms       median / min / p90 of the timed steps (events around every step);
   roofline      the dominant kernel (the GEMM) against the tensor-core peak, timed
-                alone with CUDA events on its launch stream;
+                alone with CUDA events on its launch stream (50 launches, an event each),
+                as a fraction of the measured-derived peak and of the nominal 9 PFLOP/s;
   parts         the quantizer (GB/s against HBM) and the GEMM separately;
-  ffn_up_720p_w4a4  the same linear at 720p / 81 frames (M = 75600);
+  ffn_up_480p_w4a4  the same linear at 480p / 81 frames (M = 32760);
   w4a8          the W4A8 FFN-down linear at 720p (quantize to E4M3 + mxf8f6f4 GEMM),
                 its quantize-dequantize emulation (QDQ) path, and the same linear with
                 static per-tensor E4M3 activations;
-  transform_480p  the transform_on quantizer (smoothing + block Hadamard) and linear on
-                the headline workload;
-  lowrank_480p  the headline linear with an SVDQuant bf16 rank-64 / 128 branch in the same
+  transform_720p  the transform_on quantizer (SmoothQuant scales + block Hadamard) and
+                linear on the headline workload;
+  lowrank_720p  the headline linear with an SVDQuant bf16 rank-64 / 128 branch in the same
                 accumulator;
   ffn_720p      the block's FFN with its hidden activation kept MX-quantized (the
                 FFN-up GEMM's epilogue applies GELU and quantizes), FFN-down W4A4 or W4A8;
@@ -26,11 +28,13 @@ load-time step).  Beside the headline number the JSON line carries:
   e2e           the same step through host buffers (pinned H2D of x, D2H of y every step),
                 copies of neighbouring steps overlapped on separate streams; the serial
                 form beside it;
-  cpu_baseline  the CPU oracle on a bounded sample of the same workload.
+  cpu_baseline  the CPU oracle on the machine's host cores: the linear on a bounded sample of
+                rows and the quantizer on the whole activation, single-threaded and on all
+                cores.
 
 Multi-GPU: the layer has no exchange step (token rows are independent), so N GPUs
-run N replicas, each on its own 32760-row batch (weak scaling, no collective on the
-data path); the time is the max over ranks.
+run N replicas, each on its own batch (weak scaling, no collective on the data path);
+the time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -50,6 +54,8 @@ if ROOT not in sys.path:
 import torch  # noqa: E402
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_FP4_TFLOPS = 9000.0   # dense FP4, nominal (the figure the roofline reporting names)
+NOMINAL_HBM_GBS = 8000.0
 FP4_OVER_BF16 = 4.0   # nominal dense ratio: 9 PFLOP/s FP4 vs 2.25 PFLOP/s bf16
 FP8_OVER_BF16 = 2.0   # 4.5 PFLOP/s FP8
 
@@ -170,40 +176,116 @@ def time_loop(fn, iters: int, stream) -> float:
     return start.elapsed_time(end) / iters
 
 
+def time_steps(fn, iters: int, stream):
+    """(total ms, per-step ms list) of iters runs of fn(): one CUDA event before the first
+    run, one after each, all on `stream`; the per-step times come from the same timed
+    region as the total."""
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(iters + 1)]
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for i in range(iters):
+        fn()
+        ev[i + 1].record(stream)
+    ev[-1].synchronize()
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(iters)]
+    return ev[0].elapsed_time(ev[-1]), per
+
+
+def step_stats(per):
+    """median / min / p90 / mean of per-step milliseconds."""
+    v = sorted(per)
+    p90 = v[min(len(v) - 1, int(round(0.9 * (len(v) - 1))))]
+    return {"median": round(statistics.median(v), 4), "min": round(v[0], 4), "p90": round(p90, 4),
+            "mean": round(sum(v) / len(v), 4), "n": len(v)}
+
+
+def time_kernel(fn, stream, min_iters: int = 50, min_ms: float = 0.0):
+    """A kernel timed alone on its stream: min_iters launches, more if needed to fill min_ms
+    of device time (a short probe sizes the loop), one event per launch.  Returns the mean
+    launch time (ms) and the per-launch statistics."""
+    probe = time_loop(fn, 3, stream)
+    iters = max(min_iters, int(min_ms / max(probe, 1e-3)) + 1)
+    total, per = time_steps(fn, iters, stream)
+    return total / iters, step_stats(per)
+
+
 def quant_bytes(M, K, fmt):
     return 2 * M * K + (M * K if fmt == "e4m3" else M * K // 2) + M * K // 32
 
 
 # ---------------------------------------------------------------------------- CPU oracle
-def cpu_baseline(M, N, K, fmt, seed, budget_s=12.0):
-    """The CPU oracle as it stands: quantize a slice of activation rows and run the
-    fp64 linear for them against the pre-quantized weight, for about budget_s seconds."""
+def cpu_model() -> str:
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.lower().startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except (OSError, subprocess.SubprocessError):
+        pass
+    return "unknown"
+
+
+def cpu_gemm_rate(M, N, K, fmt, seed, budget_s, nthreads):
+    """The CPU oracle's quantize + fp64 linear on activation rows against a pre-quantized
+    weight, for about budget_s seconds: (TFLOP/s, rows done, seconds)."""
     import numpy as np
 
     import oracle
     import synth
     f = oracle.E2M1 if fmt == "e2m1" else oracle.E4M3
     w = synth.weight(N, K, seed=seed)
-    wb = w.view(torch.int16).numpy().view(np.uint16)
-    wc, ws = oracle.quantize(wb, oracle.E2M1)
-    chunk = 32
+    wc, ws = oracle.quantize(w.view(torch.int16).numpy().view(np.uint16), oracle.E2M1, nthreads)
+    chunk = max(4, 4 * nthreads)
     rows_done, flops = 0, 0.0
     t0 = time.perf_counter()
     while True:
         x = synth.activation(chunk, K, "student_t" if fmt == "e2m1" else "gelu", seed=seed + rows_done,
                              outlier_frac=0.01, outlier_scale=50.0)
-        xb = x.view(torch.int16).numpy().view(np.uint16)
-        xc, xs = oracle.quantize(xb, f)
-        oracle.linear(xc, xs, f, K, wc, ws)
+        xc, xs = oracle.quantize(x.view(torch.int16).numpy().view(np.uint16), f, nthreads)
+        oracle.linear(xc, xs, f, K, wc, ws, nthreads=nthreads)
         flops += 2.0 * chunk * N * K
         rows_done += chunk
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.default_threads(), "kind": "oracle",
-            "sample": "%d of %d activation rows of the %dx%dx%d %s linear (quantize + fp64 GEMM on the "
-                      "dequantized operands; weight quantized beforehand), %.1f s" % (rows_done, M, M, N, K, fmt,
-                                                                                    dt)}
+    return flops / dt / 1e12, rows_done, dt
+
+
+def cpu_quantize_rate(x_bits, fmt, nthreads):
+    """The CPU oracle's quantizer on the whole activation tensor: (GB/s, seconds), bytes
+    counted as the GPU quantizer's (bf16 in, codes and scales out)."""
+    import oracle
+    f = oracle.E2M1 if fmt == "e2m1" else oracle.E4M3
+    M, K = x_bits.shape
+    t0 = time.perf_counter()
+    oracle.quantize(x_bits, f, nthreads)
+    dt = time.perf_counter() - t0
+    return quant_bytes(M, K, fmt) / dt / 1e9, dt
+
+
+def cpu_baseline(M, N, K, fmt, seed, budget_s=6.0, x_bits=None):
+    """The CPU oracle as it stands, on the machine's host cores: the linear (quantize + fp64 GEMM)
+    on a bounded sample of activation rows, single-threaded and on all cores (about budget_s
+    seconds each), and, when the activation's bits are given, the quantizer on the whole
+    tensor, single-threaded and on all cores.  `value` is the all-core linear rate."""
+    import oracle
+    cores = oracle.default_threads()
+    g1, r1, t1 = cpu_gemm_rate(M, N, K, fmt, seed, budget_s, 1)
+    ga, ra, ta = cpu_gemm_rate(M, N, K, fmt, seed, budget_s, cores)
+    out = {"value": ga, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
+           "sample": "%d of %d activation rows of the %dx%dx%d %s linear (quantize + fp64 GEMM on the "
+                     "dequantized operands; weight quantized beforehand), %.1f s on %d threads; single thread: "
+                     "%d rows in %.1f s" % (ra, M, M, N, K, fmt, ta, cores, r1, t1),
+           "linear": {"TFLOP/s_all_cores": ga, "TFLOP/s_1_thread": g1,
+                      "full_M_extrapolated_s_all_cores": round(2.0 * M * N * K / (ga * 1e12), 1)}}
+    if x_bits is not None:
+        q1, s1 = cpu_quantize_rate(x_bits, fmt, 1)
+        qa, sa = cpu_quantize_rate(x_bits, fmt, cores)
+        out["quantize"] = {"GB/s_all_cores": round(qa, 4), "GB/s_1_thread": round(q1, 4),
+                           "s_all_cores": round(sa, 2), "s_1_thread": round(s1, 2),
+                           "tensor": "the whole %dx%d activation (%.0f MB of bf16)" % (
+                               x_bits.shape[0], x_bits.shape[1], x_bits.size * 2 / 1e6)}
+    return out
 
 
 # ---------------------------------------------------------------------------- main arms
@@ -279,31 +361,32 @@ def run_mxq(args):
         # profiling mode: only the named kernel, `steps` launches after the warm-up
         return profile_one(args, ops, x, qw, ws, y, M, N, K, fmt, stream)
 
+    xc = ws[: ops.codes_bytes(M, K, fmt)]
+    xs_off = (ops.codes_bytes(M, K, fmt) + 255) // 256 * 256
+    xs = ws[xs_off: xs_off + ops.sf_bytes(M, K)]
     for _ in range(args.warmup):
         step()
     barrier(world)
     with ClockSampler(local) as clk:
         barrier(world)
-        ms = time_loop(step, args.steps, stream)
+        ms_total, per_step = time_steps(step, args.steps, stream)
         barrier(world)
-    ms = max_over_ranks(ms, world)
+        # the two kernels of the step, each timed alone on the launch stream (50 launches
+        # each; the clocks are sampled through these loops as well)
+        for _ in range(3):
+            ops.quantize_act(x, fmt, codes=xc, sf=xs)
+        q_ms, q_stats = time_kernel(lambda: ops.quantize_act(x, fmt, codes=xc, sf=xs), stream)
+        for _ in range(3):
+            ops.gemm(xc, xs, fmt, M, K, qw, out=y)
+        g_ms, g_stats = time_kernel(lambda: ops.gemm(xc, xs, fmt, M, K, qw, out=y), stream)
+        gemm_path = ops.last_path()
+        barrier(world)
+    ms = max_over_ranks(ms_total / args.steps, world)
     status = ops.poll_status()
     if status != 0:
         raise RuntimeError("device status %d after the timed steps" % status)
     flops = 2.0 * M * N * K
     value = job_tflops(flops, ms, world)
-
-    # the two kernels of the step, each timed alone on the launch stream
-    xc = ws[: ops.codes_bytes(M, K, fmt)]
-    xs_off = (ops.codes_bytes(M, K, fmt) + 255) // 256 * 256
-    xs = ws[xs_off: xs_off + ops.sf_bytes(M, K)]
-    for _ in range(3):
-        ops.quantize_act(x, fmt, codes=xc, sf=xs)
-    q_ms = time_loop(lambda: ops.quantize_act(x, fmt, codes=xc, sf=xs), args.steps, stream)
-    for _ in range(3):
-        ops.gemm(xc, xs, fmt, M, K, qw, out=y)
-    g_ms = time_loop(lambda: ops.gemm(xc, xs, fmt, M, K, qw, out=y), args.steps, stream)
-    gemm_path = ops.last_path()
     q_ms, g_ms = max_over_ranks(q_ms, world), max_over_ranks(g_ms, world)
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     g_tflops = flops / (g_ms * 1e-3) / 1e12
@@ -319,15 +402,20 @@ def run_mxq(args):
                    "M": M, "K": K, "N": N, "act_fmt": fmt, "parallelism": "replicas%d" % world,
                    "l2": "inputs larger than L2 (x %.0f MB, y %.0f MB; L2 126 MB)" % (M * K * 2 / 1e6,
                                                                                        M * N * 2 / 1e6)},
+        "step_ms": step_stats(per_step),
         "roofline": {"bound": "tensor", "kernel": "mx_gemm_kernel<mxf4>", "achieved": round(g_tflops, 1),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(g_tflops / fp4_peak, 4),
                      "peak_source": "%s bf16 burst %.1f TFLOP/s x %.0f (nominal FP4/bf16 dense ratio)" % (
                          peak_src, peaks["bf16_tflops"], FP4_OVER_BF16),
-                     "ms": round(g_ms, 4), "traffic": gemm_traffic(wl_name, M), "path": gemm_path},
+                     "frac_nominal": round(g_tflops / NOMINAL_FP4_TFLOPS, 4),
+                     "nominal_peak": NOMINAL_FP4_TFLOPS,
+                     "ms": round(g_ms, 4), "launch_ms": g_stats, "traffic": gemm_traffic(wl_name, M),
+                     "path": gemm_path},
         "parts": {
             "quantize": {"ms": round(q_ms, 4), "GB/s": round(q_gbs, 1), "peak_GB/s": peaks["hbm_gbs"],
                          "frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4),
-                         "bytes": quant_bytes(M, K, fmt)},
+                         "frac_nominal_hbm": round(q_gbs / NOMINAL_HBM_GBS, 4),
+                         "bytes": quant_bytes(M, K, fmt), "launch_ms": q_stats},
             "gemm": {"ms": round(g_ms, 4), "TFLOP/s": round(g_tflops, 1),
                      "frac_fp4": round(g_tflops / fp4_peak, 4)},
         },
@@ -335,14 +423,15 @@ def run_mxq(args):
         "clocks": clk.summary(),
     }
 
-    if args.target:
-        result["ffn_up_720p_w4a4"] = bench_target(args, ops, synth, dev, stream, world, rank, peaks, qw, b)
+    if args.extra_linear:
+        result["ffn_up_480p_w4a4"] = bench_linear(args, ops, synth, "ffn_up_480p_w4a4", dev, stream, world, rank,
+                                                  peaks)
     if args.w4a8:
         result["w4a8"] = bench_w4a8(args, ops, synth, dev, stream, world, rank, peaks)
     if args.transform:
-        result["transform_480p"] = bench_transform(args, ops, synth, dev, stream, world, rank, peaks, x, w, b)
+        result["transform_720p"] = bench_transform(args, ops, synth, dev, stream, world, rank, peaks, x, w, b)
     if args.lowrank:
-        result["lowrank_480p"] = bench_lowrank(args, ops, synth, dev, stream, world, rank, peaks, x, b)
+        result["lowrank_720p"] = bench_lowrank(args, ops, synth, dev, stream, world, rank, peaks, x, b)
     if args.ffn:
         result["ffn_720p"] = bench_ffn(args, ops, synth, dev, stream, world, rank, peaks)
     if args.block:
@@ -354,7 +443,10 @@ def run_mxq(args):
     if args.e2e:
         result["e2e"] = bench_e2e(args, ops, x, qw, fmt, ws, M, N, K, flops, world, dev)
     if rank == 0 and world == 1 and args.cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(M, N, K, fmt, c["seed"], budget_s=args.cpu_seconds)
+        import numpy as np
+        xb = x.view(torch.int16).cpu().numpy().view(np.uint16)
+        result["cpu_baseline"] = cpu_baseline(M, N, K, fmt, c["seed"], budget_s=args.cpu_seconds, x_bits=xb)
+        del xb
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
@@ -453,13 +545,15 @@ def profile_one(args, ops, x, qw, ws, y, M, N, K, fmt, stream):
         raise RuntimeError("device status %d" % status)
 
 
-def bench_target(args, ops, synth, dev, stream, world, rank, peaks, qw, b):
-    """The W4A4 FFN-up linear at 720p / 81 frames (M = 75600), the shape the 60 %-of-FP4
-    target is stated for; same weight as the headline workload."""
-    c = synth.WORKLOADS["ffn_up_720p_w4a4"]
+def bench_linear(args, ops, synth, wl_name, dev, stream, world, rank, peaks):
+    """Another W4A4 linear workload beside the headline one (the FFN-up linear at 480p /
+    81 frames, M = 32760): the whole step, then its GEMM and quantizer timed alone."""
+    c = synth.WORKLOADS[wl_name]
     M, K, N = c["M"], c["K"], c["N"]
     x = synth.activation(M, K, c["act"], seed=replica_seed(c["seed"], rank), device=dev,
                          outlier_frac=c["outlier_frac"], outlier_scale=c["outlier_scale"])
+    qw = ops.quantize_weight(synth.weight(N, K, seed=c["seed"], device=dev),
+                             bias=synth.bias(N, seed=c["seed"], device=dev))
     ws = torch.empty(ops.workspace_bytes(M, N, K, "e2m1"), dtype=torch.uint8, device=dev)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     flops = 2.0 * M * N * K
@@ -474,12 +568,13 @@ def bench_target(args, ops, synth, dev, stream, world, rank, peaks, qw, b):
     q_ms = max_over_ranks(time_loop(lambda: ops.quantize_act(x, "e2m1", codes=xc, sf=xs), iters, stream), world)
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     if ops.poll_status() != 0:
-        raise RuntimeError("device status set during the 720p measurement")
+        raise RuntimeError("device status set during the %s measurement" % wl_name)
     q_gbs = quant_bytes(M, K, "e2m1") / (q_ms * 1e-3) / 1e9
-    return {"workload": "ffn_up_720p_w4a4: M=%d K=%d N=%d W4A4" % (M, K, N),
+    return {"workload": "%s: M=%d K=%d N=%d W4A4" % (wl_name, M, K, N),
             "linear": {"ms": round(ms, 4), "TFLOP/s": round(flops / (ms * 1e-3) / 1e12, 1)},
             "gemm": {"ms": round(g_ms, 4), "TFLOP/s": round(flops / (g_ms * 1e-3) / 1e12, 1),
-                     "frac_fp4": round(flops / (g_ms * 1e-3) / 1e12 / fp4_peak, 4)},
+                     "frac_fp4": round(flops / (g_ms * 1e-3) / 1e12 / fp4_peak, 4),
+                     "traffic": gemm_traffic(wl_name, M)},
             "quantize": {"ms": round(q_ms, 4), "GB/s": round(q_gbs, 1),
                          "frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4)}}
 
@@ -557,8 +652,8 @@ def bench_transform(args, ops, synth, dev, stream, world, rank, peaks, x, w, b):
     and a block Hadamard rotation (32 or 128), and the linear built on it."""
     M, K = x.shape
     N = w.shape[0]
-    s = x.abs().amax(dim=0).float().clamp_min(1e-3).sqrt().contiguous()  # SmoothQuant-style scales
-    inv_s = (1.0 / s).contiguous()
+    from fp8_mixed_precision_mxq_b200 import policy
+    s, inv_s = policy.smoothquant_scales(x, w, 0.5)  # SmoothQuant's scales, from the library
     flops = 2.0 * M * N * K
     qbytes = quant_bytes(M, K, "e2m1") + K * 4
     iters = max(3, args.steps // 4)
@@ -566,7 +661,8 @@ def bench_transform(args, ops, synth, dev, stream, world, rank, peaks, x, w, b):
     sf = torch.empty(ops.sf_bytes(M, K), dtype=torch.uint8, device=dev)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     ws = torch.empty(ops.workspace_bytes(M, N, K, "e2m1"), dtype=torch.uint8, device=dev)
-    res = {"workload": "FFN-up 480p (M=%d K=%d N=%d) W4A4, SmoothQuant-style scales + block Hadamard" % (M, K, N)}
+    res = {"workload": "%s (M=%d K=%d N=%d) W4A4, SmoothQuant scales (alpha 0.5) + block Hadamard" % (
+        args.workload, M, K, N)}
     for block in (32, 128):
         qw = ops.quantize_weight_transformed(w, bias=b, block=block, mul=s)
         fq = lambda blk=block: ops.quantize_act_transformed(x, "e2m1", blk, inv_s, codes=codes, sf=sf)  # noqa: E731
@@ -587,12 +683,12 @@ def bench_transform(args, ops, synth, dev, stream, world, rank, peaks, x, w, b):
 
 def bench_lowrank(args, ops, synth, dev, stream, world, rank, peaks, x, b):
     """The SVDQuant low-rank branch on the headline workload: the linear with a rank-r bf16
-    branch in the same accumulator (u from a thin library GEMM), r = 64 and 128."""
-    c = synth.WORKLOADS["ffn_up_480p_w4a4"]
+    branch in the same accumulator (u from the library's bf16 GEMM), r = 64 and 128."""
+    c = synth.WORKLOADS[args.workload]
     M, K, N = x.shape[0], c["K"], c["N"]
     iters = max(3, args.steps // 4)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    res = {"workload": "FFN-up 480p (M=%d K=%d N=%d) W4A4 + bf16 rank-r branch" % (M, K, N)}
+    res = {"workload": "%s (M=%d K=%d N=%d) W4A4 + bf16 rank-r branch" % (args.workload, M, K, N)}
     for r in (64, 128):
         l1t, l2t, resid = synth.lowrank_weight(N, K, r, seed=c["seed"], device=dev)
         qr = ops.quantize_weight(resid, bias=b)
@@ -742,20 +838,27 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import oracle
     c = synth.WORKLOADS[args.workload]
     M, K, N, fmt = c["M"], c["K"], c["N"], c["fmt"]
+    cores = oracle.default_threads()
     # about 150 s of oracle work over the whole run, at least half a second per step
     per_step = max(0.5, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    if args.ref_step_seconds:
+        per_step = args.ref_step_seconds
     for _ in range(args.warmup):
-        cpu_baseline(M, N, K, fmt, c["seed"], budget_s=per_step / 2)
-    vals, samples = [], None
+        cpu_gemm_rate(M, N, K, fmt, c["seed"], per_step / 2, cores)
+    vals, rows = [], 0
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        r = cpu_baseline(M, N, K, fmt, c["seed"], budget_s=per_step)
-        vals.append(r["value"])
-        samples = r
+        v_step, r_step, _ = cpu_gemm_rate(M, N, K, fmt, c["seed"], per_step, cores)
+        vals.append(v_step)
+        rows += r_step
     dt = time.perf_counter() - t0
     v = statistics.mean(vals)
+    samples = {"cores": cores, "sample": "%d activation rows in all (about %.1f s per step) of the %dx%dx%d %s "
+                                         "linear: quantize + fp64 GEMM on the dequantized operands, weight "
+                                         "quantized beforehand, %d threads" % (rows, per_step, M, N, K, fmt, cores)}
     out = {"impl": "reference", "metric": "W4A4 MX linear TFLOP/s (fused dynamic MXFP4 activation quantize + "
                                           "tcgen05 mxf4 GEMM)",
            "value": v, "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
@@ -776,10 +879,10 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mxq", "reference"], default="mxq")
-    ap.add_argument("--workload", default="ffn_up_480p_w4a4")
+    ap.add_argument("--workload", default="ffn_up_720p_w4a4")
     ap.add_argument("--no-w4a8", dest="w4a8", action="store_false")
-    ap.add_argument("--no-target", dest="target", action="store_false",
-                    help="skip the 720p FFN-up (M=75600) measurement")
+    ap.add_argument("--no-extra-linear", dest="extra_linear", action="store_false",
+                    help="skip the 480p FFN-up (M=32760) measurement beside the headline")
     ap.add_argument("--no-transform", dest="transform", action="store_false",
                     help="skip the smoothing + Hadamard quantizer measurement")
     ap.add_argument("--no-lowrank", dest="lowrank", action="store_false",
@@ -792,7 +895,10 @@ def main():
                     help="skip the two-expert 40-block stack measurement")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=6.0,
+                    help="seconds of CPU-oracle linear work per thread count")
+    ap.add_argument("--ref-step-seconds", type=float, default=0.0,
+                    help="reference arm: seconds of oracle work per step (default: about 150 s over the run)")
     ap.add_argument("--M", type=int, default=0, help="override the workload's row count (profiling)")
     ap.add_argument("--only", choices=["gemm", "quantize", "gelu_quant", "transform", "dequantize"], default=None,
                     help="profiling mode: launch only this kernel, --steps times")

@@ -47,7 +47,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     cuda_lib = os.path.join(os.path.dirname(os.path.dirname(_nvcc())), "lib64")
     tmp = LIB + ".tmp%d" % os.getpid()
     cmd = [_nvcc()] + nvcc_flags() + ["-shared"] + sources() + [
-        "-o", tmp, "-L" + cuda_lib, "-lcublasLt", "-Xlinker", "-rpath=" + cuda_lib]
+        "-o", tmp, "-L" + cuda_lib, "-Xlinker", "-rpath=" + cuda_lib]
     if verbose:
         print(" ".join(cmd))
     subprocess.check_call(cmd)

@@ -34,7 +34,6 @@ int ok()
 constexpr int64_t kMaxElems = int64_t(1) << 34;  // rows*K; keeps 32-bit group / scale indices exact
 constexpr int64_t kMaxK = int64_t(1) << 16;       // K/32 < 2^11 keeps the row division of the quantizer exact
 constexpr int64_t kWsAlign = 256;
-constexpr int64_t kLtWorkspace = int64_t(32) << 20;
 
 int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 
@@ -115,9 +114,38 @@ int check_gemm(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int6
 int64_t linear_ws(int64_t M, int64_t N, int64_t K, int fmt, int mode)
 {
     int64_t ws = round_up(codes_bytes(M, K, fmt), kWsAlign) + round_up(sf_bytes(M, K), kWsAlign);
-    if (mode == MXQ_MODE_QDQ)
-        ws += round_up(M * K * 2, kWsAlign) + round_up(N * K * 2, kWsAlign) + kLtWorkspace;
+    if (mode == MXQ_MODE_QDQ) ws += round_up(M * K * 2, kWsAlign) + round_up(N * K * 2, kWsAlign);
     return ws;
+}
+
+// y[M, N] = bf16(a[M, K] . b[N, K]^T + bias), both bf16 and K-major: the GEMM kernel with
+// only bf16 (kind::f16) stages.
+int run_gemm_bf16(const void* a, const void* b, const void* bias, void* y, int64_t M, int64_t N, int64_t K,
+                  cudaStream_t stream)
+{
+    GemmArgs g{a, nullptr, MXQ_FMT_E2M1, M, N, K, b, nullptr, bias, y};
+    g.bf16 = true;
+    const char* msg = nullptr;
+    int rc = launch_gemm(g, stream, &msg, g_path, sizeof g_path);
+    if (rc != MXQ_OK) return fail(rc, "bf16 gemm: %s", msg ? msg : "launch failed");
+    return ok();
+}
+
+int check_gemm_bf16(const void* a, int64_t M, int64_t K, const void* b, int64_t N, const void* bias, const void* y)
+{
+    if (M <= 0 || N <= 0 || K <= 0)
+        return fail(MXQ_ERR_INVALID_ARG, "bf16 gemm: sizes must be positive (M=%lld N=%lld K=%lld)", (long long)M,
+                    (long long)N, (long long)K);
+    if (K % 8 != 0) return fail(MXQ_ERR_SHAPE, "bf16 gemm: K=%lld is not a multiple of 8", (long long)K);
+    if (N % 8 != 0) return fail(MXQ_ERR_SHAPE, "N=%lld is not a multiple of 8", (long long)N);
+    if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1 || K > kMaxK * 4)
+        return fail(MXQ_ERR_SHAPE, "bf16 gemm: sizes above the supported maximum (M=%lld N=%lld K=%lld)",
+                    (long long)M, (long long)N, (long long)K);
+    RETURN_IF(check_ptr(a, "a"));
+    RETURN_IF(check_ptr(b, "b"));
+    RETURN_IF(check_ptr(y, "y"));
+    if (bias) RETURN_IF(check_ptr(bias, "bias"));
+    return MXQ_OK;
 }
 
 int run_gemm(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K, const void* w_codes,
@@ -146,13 +174,12 @@ int run_linear(const void* x, int64_t M, int64_t K, const void* w_codes, const v
 
     uint8_t* xd = xs + round_up(sf_bytes(M, K), kWsAlign);
     uint8_t* wd = xd + round_up(M * K * 2, kWsAlign);
-    uint8_t* lt = wd + round_up(N * K * 2, kWsAlign);
     RETURN_IF(cuda_rc(launch_dequantize(xc, xs, M, K, fmt, xd, stream), "dequantize launch"));
     RETURN_IF(cuda_rc(launch_dequantize(w_codes, w_sf, N, K, MXQ_FMT_E2M1, wd, stream), "dequantize launch"));
-    const char* msg = nullptr;
-    int rc = qdq_bf16_gemm(xd, wd, bias, y, M, N, K, lt, static_cast<size_t>(kLtWorkspace), stream, &msg);
-    if (rc != MXQ_OK) return fail(rc, "qdq gemm: %s", msg ? msg : "failed");
-    snprintf(g_path, sizeof g_path, "qdq %s dequant + cublasLt bf16", fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1");
+    RETURN_IF(run_gemm_bf16(xd, wd, bias, y, M, N, K, stream));
+    char gp[sizeof g_path];
+    snprintf(gp, sizeof gp, "%s", g_path);
+    snprintf(g_path, sizeof g_path, "qdq %s dequant + %s", fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1", gp);
     return ok();
 }
 
@@ -279,6 +306,14 @@ int mxq_gemm(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_
     RETURN_IF(check_device());
     return run_gemm(a_codes, a_sf, a_fmt, M, K, w_codes, w_sf, N, bias_bf16, y_bf16,
                     static_cast<cudaStream_t>(stream));
+}
+
+int mxq_gemm_bf16(const void* a_bf16, int64_t M, int64_t K, const void* b_bf16, int64_t N, const void* bias_bf16,
+                  void* y_bf16, void* stream)
+{
+    RETURN_IF(check_gemm_bf16(a_bf16, M, K, b_bf16, N, bias_bf16, y_bf16));
+    RETURN_IF(check_device());
+    return run_gemm_bf16(a_bf16, b_bf16, bias_bf16, y_bf16, M, N, K, static_cast<cudaStream_t>(stream));
 }
 
 int mxq_linear(const void* x_bf16, int64_t M, int64_t K, const void* w_codes, const void* w_sf, int64_t N,
@@ -495,7 +530,7 @@ int64_t mxq_lowrank_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, in
 {
     const int64_t base = mxq_workspace_bytes(M, N, K, fmt, MXQ_MODE_NATIVE);
     if (base < 0 || rank <= 0 || rank % 64 != 0 || rank > 256) return -1;
-    return base + round_up(M * rank * 2, kWsAlign) + kLtWorkspace;
+    return base + round_up(M * rank * 2, kWsAlign);
 }
 
 int mxq_linear_lowrank(const void* x_bf16, int64_t M, int64_t K, const void* r_codes, const void* r_sf, int64_t N,
@@ -518,16 +553,15 @@ int mxq_linear_lowrank(const void* x_bf16, int64_t M, int64_t K, const void* r_c
     uint8_t* xc = static_cast<uint8_t*>(workspace);
     uint8_t* xs = xc + round_up(codes_bytes(M, K, act_fmt), kWsAlign);
     uint8_t* u = xs + round_up(sf_bytes(M, K), kWsAlign);
-    uint8_t* lt = u + round_up(M * rank * 2, kWsAlign);
     RETURN_IF(cuda_rc(launch_quantize(x_bf16, M, K, act_fmt, xc, xs, st), "quantize launch"));
-    // u = x . l1t^T: [M, K] x [K, rank], a thin plain bf16 GEMM (library)
-    const char* msg = nullptr;
-    int rc = qdq_bf16_gemm(x_bf16, l1t_bf16, nullptr, u, M, rank, K, lt, static_cast<size_t>(kLtWorkspace), st, &msg);
-    if (rc != MXQ_OK) return fail(rc, "low-rank u gemm: %s", msg ? msg : "failed");
+    // u = x . l1t^T: [M, K] x [K, rank], the bf16 GEMM with N = rank
+    int rc = run_gemm_bf16(x_bf16, l1t_bf16, nullptr, u, M, rank, K, st);
+    if (rc != MXQ_OK) return fail(rc, "low-rank u: %s", g_err);
     GemmArgs g{xc, xs, act_fmt, M, N, K, r_codes, r_sf, bias_bf16, y_bf16};
     g.lr_rank = rank;
     g.lr_u = u;
     g.lr_l2t = l2t_bf16;
+    const char* msg = nullptr;
     rc = launch_gemm(g, st, &msg, g_path, sizeof g_path);
     if (rc != MXQ_OK) return fail(rc, "gemm: %s", msg ? msg : "launch failed");
     return ok();
@@ -566,6 +600,76 @@ int mxq_absmax(const void* x_bf16, int64_t n, void* out_f32, void* stream)
     RETURN_IF(check_device());
     return cuda_rc(launch_absmax(x_bf16, n, static_cast<float*>(out_f32), static_cast<cudaStream_t>(stream)),
                    "absmax launch");
+}
+
+int mxq_channel_absmax(const void* x_bf16, int64_t rows, int64_t K, float* out_f32, void* stream)
+{
+    if (rows <= 0 || K <= 0) return fail(MXQ_ERR_INVALID_ARG, "channel_absmax: sizes must be positive");
+    if (K % 8 != 0) return fail(MXQ_ERR_SHAPE, "channel_absmax: K=%lld is not a multiple of 8", (long long)K);
+    if (rows > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 1 || rows * K > kMaxElems)
+        return fail(MXQ_ERR_SHAPE, "channel_absmax: tensor too large");
+    RETURN_IF(check_ptr(x_bf16, "x"));
+    RETURN_IF(check_ptr(out_f32, "out", 4));
+    RETURN_IF(check_device());
+    snprintf(g_path, sizeof g_path, "channel absmax");
+    return cuda_rc(launch_channel_absmax(x_bf16, rows, K, out_f32, static_cast<cudaStream_t>(stream)),
+                   "channel_absmax launch");
+}
+
+int mxq_smooth_scales(const float* amax_x, const float* amax_w, int64_t K, float alpha, float* s, float* inv_s,
+                      void* stream)
+{
+    if (K <= 0 || K > (int64_t(1) << 31) - 1) return fail(MXQ_ERR_INVALID_ARG, "smooth_scales: bad K=%lld", (long long)K);
+    if (!(alpha >= 0.0f && alpha <= 1.0f))
+        return fail(MXQ_ERR_INVALID_ARG, "smooth_scales: alpha must lie in [0, 1] (got %g)", (double)alpha);
+    RETURN_IF(check_ptr(amax_x, "amax_x", 4));
+    RETURN_IF(check_ptr(amax_w, "amax_w", 4));
+    RETURN_IF(check_ptr(s, "s", 4));
+    if (inv_s) RETURN_IF(check_ptr(inv_s, "inv_s", 4));
+    RETURN_IF(check_device());
+    snprintf(g_path, sizeof g_path, "smooth scales");
+    return cuda_rc(launch_smooth_scales(amax_x, amax_w, K, alpha, s, inv_s, static_cast<cudaStream_t>(stream)),
+                   "smooth_scales launch");
+}
+
+int mxq_sqnr(const void* const* ref_bf16, const void* const* test_bf16, const int64_t* n, int count, double* out_f64,
+             void* stream)
+{
+    if (!ref_bf16 || !test_bf16 || !n || count <= 0) return fail(MXQ_ERR_INVALID_ARG, "sqnr: empty or NULL arrays");
+    for (int i = 0; i < count; ++i) {
+        if (n[i] <= 0 || n[i] % 8 != 0)
+            return fail(MXQ_ERR_SHAPE, "sqnr: tensor %d has n=%lld (a positive multiple of 8 is required)", i,
+                        (long long)n[i]);
+        RETURN_IF(check_ptr(ref_bf16[i], "ref"));
+        RETURN_IF(check_ptr(test_bf16[i], "test"));
+    }
+    RETURN_IF(check_ptr(out_f64, "out", 8));
+    RETURN_IF(check_device());
+    snprintf(g_path, sizeof g_path, "sqnr over %d tensors", count);
+    return cuda_rc(launch_sqnr(ref_bf16, test_bf16, n, count, out_f64, static_cast<cudaStream_t>(stream)),
+                   "sqnr launch");
+}
+
+int mxq_lowrank_split(const float* U, int64_t ldu, const float* S, const float* Vh, int64_t ldvh, const void* w_bf16,
+                      int64_t N, int64_t K, int64_t rank, void* l2t_bf16, void* l1t_bf16, void* resid_bf16,
+                      void* stream)
+{
+    if (N <= 0 || K <= 0 || rank <= 0) return fail(MXQ_ERR_INVALID_ARG, "lowrank_split: sizes must be positive");
+    if (ldu < rank || ldvh < K) return fail(MXQ_ERR_INVALID_ARG, "lowrank_split: row strides too small");
+    if (N > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 1 || rank > 4096 || N * K > kMaxElems)
+        return fail(MXQ_ERR_SHAPE, "lowrank_split: sizes above the supported maximum");
+    RETURN_IF(check_ptr(U, "U", 4));
+    RETURN_IF(check_ptr(S, "S", 4));
+    RETURN_IF(check_ptr(Vh, "Vh", 4));
+    RETURN_IF(check_ptr(w_bf16, "w"));
+    RETURN_IF(check_ptr(l2t_bf16, "l2t"));
+    RETURN_IF(check_ptr(l1t_bf16, "l1t"));
+    RETURN_IF(check_ptr(resid_bf16, "residual"));
+    RETURN_IF(check_device());
+    snprintf(g_path, sizeof g_path, "lowrank split rank %lld", (long long)rank);
+    return cuda_rc(launch_lowrank_split(U, ldu, S, Vh, ldvh, w_bf16, N, K, rank, l2t_bf16, l1t_bf16, resid_bf16,
+                                        static_cast<cudaStream_t>(stream)),
+                   "lowrank_split launch");
 }
 
 int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_rowmajor, void* stream)

@@ -768,7 +768,8 @@ cudaError_t launch_out(int out, const CUtensorMap& ma, const CUtensorMap& mb, co
 
 int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* path, size_t path_len)
 {
-    const bool w4a8 = g.a_fmt == kFmtE4M3;
+    const bool bf16 = g.bf16;
+    const bool w4a8 = !bf16 && g.a_fmt == kFmtE4M3;
     const bool quant_out = g.out_fmt >= 0;
     // CTA pairs for anything taller than one 128-row tile; a lone CTA otherwise.
     const int pair = g.M > 128 ? 2 : 1;
@@ -776,20 +777,23 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     const int64_t atoms_k = sf_atoms_k(g.K);
     const int ak = w4a8 ? 1 : 2;
     CUtensorMap ma, mb, msa, msb, my, mq, mu, ml;
-    const uint64_t a_row = w4a8 ? g.K : g.K / 2;
-    bool ok = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a_codes, a_row, g.M, a_row, 128, 128,
-                          CU_TENSOR_MAP_SWIZZLE_128B);
-    if (w4a8)
-        ok = ok && make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, g.w_codes, g.K, g.N, g.K / 2, 128,
-                               rows_b, CU_TENSOR_MAP_SWIZZLE_128B);
-    else
-        ok = ok && make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.w_codes, g.K / 2, g.N, g.K / 2, 128, rows_b,
-                               CU_TENSOR_MAP_SWIZZLE_128B);
-    // scale atoms as 32-bit words: one 2-D row of atoms_k*128 words per 128-row tile
-    ok = ok && make_map_2d(&msa, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.a_sf, atoms_k * 128, ceil_div(g.M, 128),
-                           atoms_k * 512, ak * 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
-    ok = ok && make_map_2d(&msb, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.w_sf, atoms_k * 128, ceil_div(g.N, 128),
-                           atoms_k * 512, ak * 128, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+    bool ok = true;
+    if (!bf16) {
+        const uint64_t a_row = w4a8 ? g.K : g.K / 2;
+        ok = make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a_codes, a_row, g.M, a_row, 128, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+        if (w4a8)
+            ok = ok && make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, g.w_codes, g.K, g.N, g.K / 2, 128,
+                                   rows_b, CU_TENSOR_MAP_SWIZZLE_128B);
+        else
+            ok = ok && make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.w_codes, g.K / 2, g.N, g.K / 2, 128, rows_b,
+                                   CU_TENSOR_MAP_SWIZZLE_128B);
+        // scale atoms as 32-bit words: one 2-D row of atoms_k*128 words per 128-row tile
+        ok = ok && make_map_2d(&msa, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.a_sf, atoms_k * 128, ceil_div(g.M, 128),
+                               atoms_k * 512, ak * 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
+        ok = ok && make_map_2d(&msb, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.w_sf, atoms_k * 128, ceil_div(g.N, 128),
+                               atoms_k * 512, ak * 128, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
     // bf16 output (y, or h of the quantizing epilogue): 32 x 32 boxes, 64-byte swizzle
     const void* ybase = g.y ? g.y : g.q_codes;  // without h the map is never used
     ok = ok && make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ybase, g.N, g.M, g.N * 2, 32, 32,
@@ -802,16 +806,24 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     } else {
         mq = my;  // never used by the bf16 epilogue
     }
-    const int lr_stages = g.lr_rank > 0 ? static_cast<int>(g.lr_rank / 64) : 0;
+    // bf16 stages (the low-rank branch, or every stage of a plain bf16 GEMM): operands bf16
+    // and K-major, one 64-element (128-byte) column block per stage as the A and B tiles of
+    // a stage; a K that is not a multiple of 64 reads zeros past its end
+    const int64_t lr_k = bf16 ? g.K : g.lr_rank;
+    const void* lr_a = bf16 ? g.a_codes : g.lr_u;
+    const void* lr_b = bf16 ? g.w_codes : g.lr_l2t;
+    const int lr_stages = lr_k > 0 ? static_cast<int>(ceil_div(lr_k, 64)) : 0;
     if (lr_stages > 0) {
-        // low-rank operands, bf16 and K-major with K = r: u [M, r] and B^T [N, r], one
-        // 64-element (128-byte) column block per stage, as the A and B tiles of a stage
-        ok = ok && make_map_2d(&mu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.lr_u, g.lr_rank, g.M, g.lr_rank * 2, 64, 128,
+        ok = ok && make_map_2d(&mu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lr_a, lr_k, g.M, lr_k * 2, 64, 128,
                                CU_TENSOR_MAP_SWIZZLE_128B);
-        ok = ok && make_map_2d(&ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, g.lr_l2t, g.lr_rank, g.N, g.lr_rank * 2, 64,
-                               rows_b, CU_TENSOR_MAP_SWIZZLE_128B);
-    } else {
-        mu = ma;  // never used without a low-rank branch
+        ok = ok && make_map_2d(&ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lr_b, lr_k, g.N, lr_k * 2, 64, rows_b,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    if (bf16) {
+        ma = msa = mu;  // never used without block-scaled stages
+        mb = msb = ml;
+    } else if (lr_stages == 0) {
+        mu = ma;  // never used without bf16 stages
         ml = mb;
     }
     if (!ok) {
@@ -826,7 +838,7 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     p.m_blocks = static_cast<int>(ceil_div(g.M, 128 * pair));
     p.n_blocks = static_cast<int>(ceil_div(g.N, BN));
     p.num_tiles = p.m_blocks * p.n_blocks;
-    p.k_stages = static_cast<int>(ceil_div(g.K, w4a8 ? 128 : 256));
+    p.k_stages = bf16 ? 0 : static_cast<int>(ceil_div(g.K, w4a8 ? 128 : 256));
     p.debug = g_debug_flags;
     p.q_sf = static_cast<uint8_t*>(g.q_sf);
     p.q_atoms_k = quant_out ? static_cast<uint32_t>(sf_atoms_k(g.N)) : 0u;
@@ -853,7 +865,10 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
         *msg = cudaGetErrorString(e);
         return MXQ_ERR_CUDA;
     }
-    if (path)
+    if (path && bf16)
+        snprintf(path, path_len, "bf16 kind::f16 %s %dx%d grid %d tiles %d", pair == 2 ? "2cta" : "1cta",
+                 128 * pair, BN, grid, p.num_tiles);
+    else if (path)
         snprintf(path, path_len, "native %s %s %dx%d grid %d tiles %d%s%s", w4a8 ? "mxf8f6f4" : "mxf4",
                  pair == 2 ? "2cta" : "1cta", 128 * pair, BN, grid, p.num_tiles,
                  !quant_out ? "" : g.out_gelu ? (g.out_fmt == kFmtE4M3 ? " +gelu->e4m3" : " +gelu->e2m1")

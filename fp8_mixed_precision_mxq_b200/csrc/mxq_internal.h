@@ -33,6 +33,15 @@ cudaError_t launch_quantize_transform(const void* x, int64_t rows, int64_t K, in
 cudaError_t launch_absmax(const void* x, int64_t n, float* out, cudaStream_t stream);
 cudaError_t launch_dequantize(const void* codes, const void* sf, int64_t rows, int64_t K, int fmt, void* out,
                               cudaStream_t stream);
+// Calibration and load-time arithmetic of the policy (calib.cu).
+cudaError_t launch_channel_absmax(const void* x, int64_t rows, int64_t K, float* out, cudaStream_t stream);
+cudaError_t launch_smooth_scales(const float* ax, const float* aw, int64_t K, float alpha, float* s, float* inv,
+                                 cudaStream_t stream);
+cudaError_t launch_sqnr(const void* const* ref, const void* const* test, const int64_t* n, int count, double* out,
+                        cudaStream_t stream);
+cudaError_t launch_lowrank_split(const float* U, int64_t ldu, const float* S, const float* Vh, int64_t ldvh,
+                                 const void* w, int64_t N, int64_t K, int64_t r, void* l2t, void* l1t, void* resid,
+                                 cudaStream_t stream);
 cudaError_t launch_sf_to_logical(const void* sf, int64_t rows, int64_t K, void* out, cudaStream_t stream);
 
 struct GemmArgs {
@@ -58,6 +67,9 @@ struct GemmArgs {
     int64_t lr_rank = 0;
     const void* lr_u = nullptr;
     const void* lr_l2t = nullptr;
+    // plain bf16 GEMM: a_codes is A bf16 [M, K], w_codes is B bf16 [N, K] (K-major, K % 8
+    // == 0), no scales; the same kernel runs only bf16 (kind::f16) stages of 64 along K
+    bool bf16 = false;
 };
 
 // Builds the tensor maps and launches the tcgen05 GEMM.  Returns an mxq_status;
@@ -75,9 +87,5 @@ bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint6
                  uint64_t stride_bytes, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw);
 void set_debug_flags(uint32_t flags);
 uint32_t debug_flags();
-
-// bf16 GEMM of the quantize-dequantize emulation path (cuBLASLt).
-int qdq_bf16_gemm(const void* xd, const void* wd, const void* bias, void* y, int64_t M, int64_t N, int64_t K,
-                  void* workspace, size_t ws_bytes, cudaStream_t stream, const char** msg);
 
 }  // namespace mxq

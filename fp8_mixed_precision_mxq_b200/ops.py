@@ -106,6 +106,23 @@ def gemm(a_codes, a_sf, fmt, M: int, K: int, w: QWeight, out=None, stream=None):
     return out
 
 
+def gemm_bf16(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = None, out=None, stream=None):
+    """y [M, N] = a [M, K] . b [N, K]^T (+ bias) in bf16 with fp32 accumulation, on the
+    library's tcgen05 kernel (kind::f16)."""
+    _cuda_bf16(a, "a")
+    _cuda_bf16(b, "b")
+    if bias is not None:
+        _cuda_bf16(bias, "bias")
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a is [%d, %d] but b is [%d, %d]" % (M, K, N, b.shape[1]))
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    check(_lib.lib().mxq_gemm_bf16(_p(a), M, K, _p(b), N, _p(bias), _p(out), _stream(stream)), "mxq_gemm_bf16")
+    return out
+
+
 def linear(x: torch.Tensor, w: QWeight, fmt="e2m1", mode="native", workspace=None, out=None, stream=None):
     """y = x . deq(w)^T + bias with x quantized on the fly to fmt (E2M1 = W4A4, E4M3 = W4A8)."""
     _cuda_bf16(x, "x")
@@ -287,19 +304,82 @@ def linear_transformed(x: torch.Tensor, w: QWeight, fmt="e2m1", block=32, act_mu
     return out
 
 
-def svd_split(w: torch.Tensor, rank: int):
+def lowrank_split(w: torch.Tensor, U: torch.Tensor, S: torch.Tensor, Vh: torch.Tensor, rank: int, stream=None):
+    """The SVDQuant split of w [N, K] bf16 from its singular triplets (U [N, >= rank],
+    S [>= rank], Vh [>= rank, K], fp32 CUDA tensors, the first `rank` used), in the library:
+    l2t = bf16(U sqrt(S)) [N, rank], l1t = bf16(sqrt(S) Vh) [rank, K] and the residual
+    bf16(w - l2t . l1t) [N, K].  Returns (l1t, l2t, residual)."""
+    _cuda_bf16(w, "w")
+    N, K = w.shape
+    for t, name in ((U, "U"), (S, "S"), (Vh, "Vh")):
+        if not (t.is_cuda and t.dtype == torch.float32 and t.stride(-1) == 1):
+            raise ValueError("%s must be a float32 CUDA tensor with unit inner stride" % name)
+    if U.shape[0] != N or Vh.shape[1] != K or min(U.shape[1], S.shape[0], Vh.shape[0]) < rank:
+        raise ValueError("factors of shapes %s, %s, %s do not fit w [%d, %d] at rank %d" % (
+            tuple(U.shape), tuple(S.shape), tuple(Vh.shape), N, K, rank))
+    l2t = torch.empty((N, rank), dtype=torch.bfloat16, device=w.device)
+    l1t = torch.empty((rank, K), dtype=torch.bfloat16, device=w.device)
+    resid = torch.empty((N, K), dtype=torch.bfloat16, device=w.device)
+    check(_lib.lib().mxq_lowrank_split(_p(U), U.stride(0), _p(S), _p(Vh), Vh.stride(0), _p(w), N, K, rank, _p(l2t),
+                                       _p(l1t), _p(resid), _stream(stream)), "mxq_lowrank_split")
+    return l1t, l2t, resid
+
+
+def svd_split(w: torch.Tensor, rank: int, stream=None):
     """Offline weight preparation of the SVDQuant branch (load time, not the layer's path):
-    w [N, K] bf16 ~= l2t . l1t + residual with the top `rank` singular triplets split as
-    l2t = U_r sqrt(S_r) [N, rank], l1t = sqrt(S_r) V_r^T [rank, K] (bf16), and the residual
-    w - l2t . l1t rounded to bf16 (to be quantized with quantize_weight).  Uses torch's SVD
-    in fp32."""
+    the singular value decomposition of w in fp32 is a library factorization (torch's),
+    the split into l2t = U_r sqrt(S_r), l1t = sqrt(S_r) V_r^T and the bf16 residual
+    w - l2t . l1t runs in this library (lowrank_split).  Returns (l1t, l2t, residual)."""
     _cuda_bf16(w, "w")
     U, S, Vh = torch.linalg.svd(w.float(), full_matrices=False)
-    rs = S[:rank].sqrt()
-    l2t = (U[:, :rank] * rs).to(torch.bfloat16).contiguous()
-    l1t = (rs[:, None] * Vh[:rank]).to(torch.bfloat16).contiguous()
-    residual = (w.float() - l2t.float() @ l1t.float()).to(torch.bfloat16).contiguous()
-    return l1t, l2t, residual
+    return lowrank_split(w, U.contiguous(), S.contiguous(), Vh.contiguous(), rank, stream=stream)
+
+
+def channel_absmax(x: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """max over rows of |x[:, k]| for a bf16 [rows, K] tensor, as K float32 values."""
+    _cuda_bf16(x, "x")
+    rows, K = x.shape
+    if out is None:
+        out = torch.empty(K, dtype=torch.float32, device=x.device)
+    check(_lib.lib().mxq_channel_absmax(_p(x), rows, K, _p(out), _stream(stream)), "mxq_channel_absmax")
+    return out
+
+
+def smooth_scales(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: float = 0.5, with_inverse: bool = False,
+                  stream=None):
+    """SmoothQuant's s_k = max(amax_x_k, 1e-5)^alpha / max(amax_w_k, 1e-5)^(1 - alpha);
+    with_inverse: also 1 / s_k (the activation's multiplier), returned as (s, 1/s)."""
+    amax_x = _f32_or_none(amax_x, "amax_x")
+    amax_w = _f32_or_none(amax_w, "amax_w")
+    K = amax_x.numel()
+    if amax_w.numel() != K:
+        raise ValueError("channel counts differ: %d vs %d" % (K, amax_w.numel()))
+    s = torch.empty(K, dtype=torch.float32, device=amax_x.device)
+    inv = torch.empty(K, dtype=torch.float32, device=amax_x.device) if with_inverse else None
+    check(_lib.lib().mxq_smooth_scales(_p(amax_x), _p(amax_w), K, float(alpha), _p(s), _p(inv), _stream(stream)),
+          "mxq_smooth_scales")
+    return (s, inv) if with_inverse else s
+
+
+def sqnr(refs, tests, out=None, stream=None) -> torch.Tensor:
+    """SQNR over pairs of bf16 tensors: a float64 CUDA tensor [sum ref^2, sum (ref - test)^2,
+    dB]."""
+    refs, tests = list(refs), list(tests)
+    if len(refs) != len(tests) or not refs:
+        raise ValueError("need as many test tensors as reference tensors, at least one")
+    for r, t in zip(refs, tests):
+        _cuda_bf16(r, "ref")
+        _cuda_bf16(t, "test")
+        if r.numel() != t.numel():
+            raise ValueError("a reference and its test tensor differ in size")
+    if out is None:
+        out = torch.empty(3, dtype=torch.float64, device=refs[0].device)
+    n = len(refs)
+    rp = (ctypes.c_void_p * n)(*[r.data_ptr() for r in refs])
+    tp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in tests])
+    ns = (ctypes.c_int64 * n)(*[r.numel() for r in refs])
+    check(_lib.lib().mxq_sqnr(rp, tp, ns, n, _p(out), _stream(stream)), "mxq_sqnr")
+    return out
 
 
 def lowrank_workspace_bytes(M: int, N: int, K: int, fmt="e2m1", rank=64) -> int:

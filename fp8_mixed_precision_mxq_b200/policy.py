@@ -5,8 +5,9 @@ rotation), measure the whole-block output SQNR of each against the bf16 block, a
 a policy per (expert, block) with the tier rule (mxq_select_policy in the library).
 
 The block's output here is the concatenation of its eight linears' outputs (attention and
-norms are not part of this path).  The quantized outputs come from the library's kernels;
-the bf16 reference is a plain bf16 matmul (torch), as a bf16 network computes it."""
+norms are not part of this path).  The quantized outputs, the bf16 reference (the
+library's bf16 GEMM, as a bf16 network computes the linear), the SmoothQuant scales and the
+SQNR all come from the library's kernels."""
 from __future__ import annotations
 
 import ctypes
@@ -35,17 +36,16 @@ def thresholds(tier="high"):
     return f.value, w.value, m.value
 
 
-def smoothquant_scales(x: torch.Tensor, w: torch.Tensor, alpha: float = 0.5) -> torch.Tensor:
-    """SmoothQuant's per-channel scales s_k = max|X_k|^alpha / max|W_k|^(1 - alpha)."""
-    ax = x.abs().amax(dim=0).float().clamp_min(1e-5)
-    aw = w.abs().amax(dim=0).float().clamp_min(1e-5)
-    return (ax.pow(alpha) / aw.pow(1.0 - alpha)).contiguous()
+def smoothquant_scales(x: torch.Tensor, w: torch.Tensor, alpha: float = 0.5):
+    """SmoothQuant's per-channel scales s_k = max|X_k|^alpha / max|W_k|^(1 - alpha) and their
+    reciprocals, the channel maxima and the scales computed by the library
+    (mxq_channel_absmax, mxq_smooth_scales).  Returns (s, 1/s)."""
+    return ops.smooth_scales(ops.channel_absmax(x), ops.channel_absmax(w), alpha, with_inverse=True)
 
 
 def _sqnr_db(ref: list, out: list) -> float:
-    num = sum(float((r.double() ** 2).sum()) for r in ref)
-    den = sum(float(((r.double() - o.double()) ** 2).sum()) for r, o in zip(ref, out))
-    return 10.0 * torch.log10(torch.tensor(num / max(den, 1e-300))).item()
+    """Whole-block SQNR (dB) of the outputs against the reference, by the library."""
+    return float(ops.sqnr(ref, out)[2].item())
 
 
 @dataclass
@@ -60,15 +60,12 @@ def score_block(weights, biases, xs, hadamard_block: int = 128, alpha: float = 0
     linears (w [N, K], b [N] or None), xs their captured bf16 inputs."""
     ref, off, on = [], [], []
     for w, b, x in zip(weights, biases, xs):
-        r = x @ w.T
-        if b is not None:
-            r = r + b
-        ref.append(r)
+        ref.append(ops.gemm_bf16(x, w, b))  # the bf16 block's linear
         qw = ops.quantize_weight(w, bias=b)
         off.append(ops.linear(x, qw, "e2m1"))
-        s = smoothquant_scales(x, w, alpha)
+        s, inv_s = smoothquant_scales(x, w, alpha)
         qt = ops.quantize_weight_transformed(w, bias=b, block=hadamard_block, mul=s)
-        on.append(ops.linear_transformed(x, qt, "e2m1", hadamard_block, (1.0 / s).contiguous()))
+        on.append(ops.linear_transformed(x, qt, "e2m1", hadamard_block, inv_s))
     return BlockScore(_sqnr_db(ref, off), _sqnr_db(ref, on))
 
 

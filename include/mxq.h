@@ -57,7 +57,7 @@ typedef enum {
     MXQ_ERR_SHAPE = 2,       /* K % 32 != 0, N % 8 != 0, W4A8 native with K % 128 != 0 */
     MXQ_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned (32 for W4A8 weights) */
     MXQ_ERR_UNSUPPORTED = 4, /* the current device is not sm_100                        */
-    MXQ_ERR_CUDA = 5,        /* a CUDA runtime / driver / cuBLASLt call failed          */
+    MXQ_ERR_CUDA = 5,        /* a CUDA runtime or driver call failed                    */
     MXQ_ERR_TIMEOUT = 6,     /* a bounded device-side wait ran out                      */
     MXQ_ERR_WORKSPACE = 7    /* the workspace passed is smaller than required           */
 } mxq_status;
@@ -77,8 +77,8 @@ int64_t mxq_codes_bytes(int64_t rows, int64_t K, int fmt);
 int64_t mxq_sf_bytes(int64_t rows, int64_t K);
 
 /* Workspace bytes mxq_linear needs for these sizes, format and mode (native: the
- * quantized activation; QDQ: also both dequantized operands in bf16 and a cuBLASLt
- * workspace).  Returns -1 on invalid sizes. */
+ * quantized activation; QDQ: also both dequantized operands in bf16).  Returns -1 on
+ * invalid sizes. */
 int64_t mxq_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int mode);
 
 /* Weight quantization (load time), always to MXFP4 (E2M1).
@@ -111,10 +111,21 @@ int mxq_dequantize(const void* codes, const void* sf, int64_t rows, int64_t K, i
 int mxq_gemm(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K, const void* w_codes,
              const void* w_sf, int64_t N, const void* bias_bf16, void* y_bf16, void* stream);
 
+/* Plain bf16 GEMM: y[M, N] = bf16( sum_k a[m, k] * b[n, k] + bias[n] ) with fp32
+ * accumulation, a [M, K] and b [N, K] bf16, K contiguous; bias_bf16 may be NULL.  The
+ * "standard BF16 GEMM" of the blog's "Kernel note" that the quantize-dequantize emulation
+ * runs on the dequantized operands; also the bf16 branch activation of
+ * mxq_linear_lowrank and the GEMM of blocks the policy keeps in bf16.  It is the tcgen05
+ * kernel of mxq_gemm with kind::f16 MMAs (bf16 x bf16) in 64-element K stages.  Requires
+ * K % 8 == 0 and N % 8 == 0; all pointers 16-byte aligned.  Errors as for mxq_gemm. */
+int mxq_gemm_bf16(const void* a_bf16, int64_t M, int64_t K, const void* b_bf16, int64_t N, const void* bias_bf16,
+                  void* y_bf16, void* stream);
+
 /* The quantized linear layer: quantize x (fmt act_fmt) into the workspace, then
  *   mode NATIVE: mxq_gemm on the quantized operands;
- *   mode QDQ:    dequantize both operands to bf16 and run a bf16 GEMM (cuBLASLt),
- *                the quantize-dequantize emulation the blog's W4A8 numbers use.
+ *   mode QDQ:    dequantize both operands to bf16 and run the bf16 GEMM of
+ *                mxq_gemm_bf16, the quantize-dequantize emulation the blog's W4A8
+ *                numbers use.
  * workspace: device buffer of at least mxq_workspace_bytes(M, N, K, act_fmt, mode)
  * bytes, 256-byte aligned; its contents are scratch.  Blog sections "Quantization
  * formats" and "Kernel note". */
@@ -271,7 +282,7 @@ int mxq_linear_transformed(const void* x_bf16, int64_t M, int64_t K, const void*
  * product l2t . l1t (l1t [r, K], l2t [N, r]) and a residual R quantized to MXFP4
  * (r_codes, r_sf as from mxq_quantize_weight), and the layer computes
  *   y = bf16( deq(xq) . deq(Rq)^T + u . l2t^T + bias ),  u = bf16(x . l1t^T) [M, r],
- * x quantized in act_fmt.  u comes from a plain bf16 GEMM (cuBLASLt); u . l2t^T runs as
+ * x quantized in act_fmt.  u comes from the bf16 GEMM (mxq_gemm_bf16); u . l2t^T runs as
  * bf16 tensor-core MMAs (kind::f16) into the same TMEM accumulator as the block-scaled
  * product, in stages of 64 along r ahead of it.  rank: 64, 128, 192 or 256; l1t, l2t
  * 16-byte aligned; workspace of mxq_lowrank_workspace_bytes(...) bytes, 256-byte aligned.
@@ -300,6 +311,46 @@ int mxq_select_policy(double sqnr_off, double sqnr_on, int tier);
 
 /* The thresholds of a tier (dB); returns MXQ_OK or MXQ_ERR_INVALID_ARG. */
 int mxq_tier_thresholds(int tier, double* floor_db, double* w4a8_db, double* margin_db);
+
+/* ---- calibration and load-time preparation of the policy's transforms --------------
+ * None of these runs on the layer's path; they prepare its inputs (blog sections
+ * "Mixed-Precision selection", "Calibration-driven block selection", "Results"). */
+
+/* Per-channel abs-max: out_f32[k] = max over rows of |x[r, k]| (x bf16 [rows, K], K % 8 ==
+ * 0, 16-byte aligned; out K floats, written from zero, so any earlier content is lost).  A
+ * NaN in a channel makes its result NaN.  The calibration statistic of SmoothQuant. */
+int mxq_channel_absmax(const void* x_bf16, int64_t rows, int64_t K, float* out_f32, void* stream);
+
+/* SmoothQuant's per-channel scales (the smoothing of the "transform_on" policy):
+ *   s[k] = max(amax_x[k], 1e-5)^alpha / max(amax_w[k], 1e-5)^(1 - alpha)
+ * in fp32 (powf), amax_x / amax_w the channel abs-maxima of the activation and of the
+ * weight (mxq_channel_absmax over x [M, K] and over w [N, K]); alpha in [0, 1].  inv_s
+ * (may be NULL) receives 1 / s[k].  The activation is then quantized with mul = inv_s and
+ * the weight with mul = s.  All arrays K floats on the device. */
+int mxq_smooth_scales(const float* amax_x, const float* amax_w, int64_t K, float alpha, float* s, float* inv_s,
+                      void* stream);
+
+/* The SQNR of a block's outputs against its reference (the whole-block SQNR the blog's
+ * "Calibration-driven block selection" compares against its tier thresholds), over
+ * `count` pairs of bf16 tensors (ref[i], test[i]) of n[i] elements each (n[i] % 8 == 0):
+ *   out_f64[0] = sum ref^2,  out_f64[1] = sum (ref - test)^2  (fp64, over all pairs),
+ *   out_f64[2] = 10 log10(out_f64[0] / out_f64[1])  dB.
+ * ref, test, n: host arrays of device pointers and sizes; out_f64: 3 doubles on the device
+ * (8-byte aligned), overwritten.  The sums are accumulated with atomics, so their last bits
+ * can vary from run to run. */
+int mxq_sqnr(const void* const* ref_bf16, const void* const* test_bf16, const int64_t* n, int count, double* out_f64,
+             void* stream);
+
+/* The SVDQuant split of a weight W [N, K] (bf16) from its leading singular triplets,
+ * U [N, rank] (fp32, row stride ldu >= rank), S [rank], Vh [rank, K] (fp32, row stride
+ * ldvh >= K), computed by any factorization:
+ *   l2t[n, j] = bf16(U[n, j] * sqrt(S[j])),   l1t[j, k] = bf16(sqrt(S[j]) * Vh[j, k]),
+ *   resid[n, k] = bf16(W[n, k] - sum_j l2t[n, j] * l1t[j, k])   (fp32 accumulation);
+ * l2t [N, rank], l1t [rank, K] and resid [N, K] bf16, 16-byte aligned.  The residual is
+ * then quantized with mxq_quantize_weight and the factors feed mxq_linear_lowrank. */
+int mxq_lowrank_split(const float* U, int64_t ldu, const float* S, const float* Vh, int64_t ldvh, const void* w_bf16,
+                      int64_t N, int64_t K, int64_t rank, void* l2t_bf16, void* l1t_bf16, void* resid_bf16,
+                      void* stream);
 
 /* Tiled scale factors -> logical row-major [rows, K/32] bytes (for tests). */
 int mxq_sf_to_logical(const void* sf_tiled, int64_t rows, int64_t K, void* sf_rowmajor, void* stream);

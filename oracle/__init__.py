@@ -307,3 +307,58 @@ def linear_lowrank_rows(a_codes, a_sf, a_fmt, rows, K, r_codes, r_sf, x_bits, l1
     if rc != 0:
         raise ValueError("oracle low-rank linear failed (rc=%d)" % rc)
     return y
+
+
+# ---- the bf16 GEMM and the policy's calibration / load-time arithmetic -----------------
+#
+# Plain numpy in fp64 on the exact values of the bf16 / fp32 inputs: the standard bf16
+# GEMM of the blog's "Kernel note" (the quantize-dequantize emulation's GEMM), SmoothQuant's
+# per-channel scales and the whole-block SQNR ("Mixed-Precision selection",
+# "Calibration-driven block selection"), and the SVDQuant split of a weight ("Results").
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact values of bf16 bit patterns."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def gemm_bf16(a_bits: np.ndarray, b_bits: np.ndarray, bias_bits: np.ndarray | None = None) -> np.ndarray:
+    """fp64 y = a . b^T (+ bias) for bf16 a [M, K], b [N, K]."""
+    y = bf16_bits_to_f64(a_bits) @ bf16_bits_to_f64(b_bits).T
+    if bias_bits is not None:
+        y = y + bf16_bits_to_f64(bias_bits)[None, :]
+    return y
+
+
+def channel_absmax(x_bits: np.ndarray) -> np.ndarray:
+    """max over rows of |x[:, k]| (fp64; exact, the values are bf16)."""
+    return np.abs(bf16_bits_to_f64(x_bits)).max(axis=0)
+
+
+def smooth_scales(amax_x: np.ndarray, amax_w: np.ndarray, alpha: float) -> np.ndarray:
+    """SmoothQuant's s_k = max(amax_x_k, 1e-5)^alpha / max(amax_w_k, 1e-5)^(1 - alpha) in fp64
+    (the 1e-5 floor as the binary32 value the library compares with)."""
+    floor = float(np.float32(1e-5))
+    ax = np.maximum(np.asarray(amax_x, dtype=np.float64), floor)
+    aw = np.maximum(np.asarray(amax_w, dtype=np.float64), floor)
+    return ax ** float(alpha) / aw ** (1.0 - float(alpha))
+
+
+def sqnr(ref_bits: list, test_bits: list):
+    """(sum ref^2, sum (ref - test)^2, 10 log10 of their ratio) over pairs of bf16 tensors."""
+    num = sum(float(np.sum(bf16_bits_to_f64(r) ** 2)) for r in ref_bits)
+    den = sum(float(np.sum((bf16_bits_to_f64(r) - bf16_bits_to_f64(t)) ** 2)) for r, t in zip(ref_bits, test_bits))
+    with np.errstate(divide="ignore"):
+        db = 10.0 * np.log10(num / den) if den > 0 else float("inf")
+    return num, den, db
+
+
+def lowrank_split(U: np.ndarray, S: np.ndarray, Vh: np.ndarray, w_bits: np.ndarray, rank: int):
+    """The SVDQuant split from singular triplets (fp32 U, S, Vh): l2t = bf16(U_r sqrt(S_r)),
+    l1t = bf16(sqrt(S_r) Vh_r) and the residual bf16(W - l2t . l1t), each product and sum in
+    fp64 and rounded once to bf16.  Returns bf16 bits (l1t, l2t, residual)."""
+    rs = np.sqrt(np.asarray(S[:rank], dtype=np.float64))
+    l2t = round_bf16(np.asarray(U[:, :rank], dtype=np.float64) * rs[None, :])
+    l1t = round_bf16(rs[:, None] * np.asarray(Vh[:rank], dtype=np.float64))
+    resid = round_bf16(bf16_bits_to_f64(w_bits) - bf16_bits_to_f64(l2t) @ bf16_bits_to_f64(l1t))
+    return l1t, l2t, resid

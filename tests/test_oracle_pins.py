@@ -723,3 +723,75 @@ def test_lowrank_brute_force_exact():
                         Fraction(oracle.decode_elem(rc, oracle.E2M1)) * Fraction(2) ** (int(r_sf[n, k // 32]) - 127))
             want = acc + sum(u[j] * f(l2t[n, j]) for j in range(r)) + f(bias[n])
             assert abs(Fraction(y[m, n]) - want) <= abs(want) * Fraction(1, 10 ** 13) + Fraction(1, 10 ** 300)
+
+
+# --- the bf16 GEMM and the policy's calibration arithmetic ----------------------------------
+
+def test_gemm_bf16_brute_force_exact():
+    rng = np.random.default_rng(41)
+    M, N, K = 3, 4, 24
+    a = _bf16_bits(rng.standard_normal((M, K)))
+    b = _bf16_bits(rng.standard_normal((N, K)) * 0.1)
+    bias = _bf16_bits(rng.standard_normal(N))
+    y = oracle.gemm_bf16(a, b, bias)
+    f = lambda v: _exact.bf16_fraction(int(v))  # noqa: E731
+    for m in range(M):
+        for n in range(N):
+            want = sum(f(a[m, k]) * f(b[n, k]) for k in range(K)) + f(bias[n])
+            assert abs(Fraction(y[m, n]) - want) <= abs(want) * Fraction(1, 10 ** 14)
+
+
+def test_channel_absmax_hand_values():
+    x = np.array([[1.0, -2.0, 0.0, 3.5], [-4.0, 1.5, -0.0, -3.5]], dtype=np.float32)
+    assert list(oracle.channel_absmax(_bf16_bits(x))) == [4.0, 2.0, 0.0, 3.5]
+
+
+def test_smooth_scales_closed_forms():
+    ax = np.array([4.0, 9.0, 0.0, 1e-9])
+    aw = np.array([1.0, 0.25, 2.0, 16.0])
+    # alpha = 1: s = max|X|; alpha = 0: s = 1 / max|W|; alpha = 1/2: sqrt(max|X| / max|W|)
+    f = float(np.float32(1e-5))
+    assert np.allclose(oracle.smooth_scales(ax, aw, 1.0), [4.0, 9.0, f, f], rtol=0, atol=0)
+    assert np.allclose(oracle.smooth_scales(ax, aw, 0.0), [1.0, 4.0, 0.5, 1 / 16.0], rtol=1e-15)
+    assert np.allclose(oracle.smooth_scales(ax, aw, 0.5), [2.0, 6.0, np.sqrt(f / 2.0), np.sqrt(f / 16.0)], rtol=1e-15)
+    # scaling the activation's channel maxima by c scales s by c^alpha
+    s1 = oracle.smooth_scales(ax[:2] * 16.0, aw[:2], 0.25)
+    assert np.allclose(s1, 2.0 * oracle.smooth_scales(ax[:2], aw[:2], 0.25), rtol=1e-15)
+
+
+def test_sqnr_known_ratio():
+    """test = ref * (1 + 2^-7) exactly: every error is ref * 2^-7, so the ratio of the sums is
+    2^14 and the SQNR 140 log10(2) dB; split over two tensors it is the same."""
+    ref = _bf16_bits(np.full(64, 2.0))
+    test = _bf16_bits(np.full(64, 2.0 * (1 + 2.0 ** -7)))
+    num, den, db = oracle.sqnr([ref], [test])
+    assert num == 64 * 4.0 and den == 64 * 4.0 * 2.0 ** -14
+    assert abs(db - 140 * math.log10(2.0)) < 1e-12
+    assert oracle.sqnr([ref[:32], ref[32:]], [test[:32], test[32:]])[2] == db
+
+
+def test_lowrank_split_exact_recomposition():
+    """Singular vectors and values chosen so that U sqrt(S) and sqrt(S) Vh are bf16 values
+    (S powers of 4): the factors are those products exactly, and W built as l2t . l1t + R with
+    a bf16 R whose sum is exact returns R as the residual."""
+    rng = np.random.default_rng(5)
+    N, K, r = 6, 40, 3
+    U = _bf16_f32(rng.standard_normal((N, r)))
+    Vh = _bf16_f32(rng.standard_normal((r, K)))
+    S = np.array([16.0, 4.0, 0.25], dtype=np.float32)
+    l2t_v = U.astype(np.float64) * np.sqrt(S)[None, :]
+    l1t_v = np.sqrt(S)[:, None] * Vh.astype(np.float64)
+    R = _bf16_f32(rng.standard_normal((N, K)) * 2.0 ** -20)
+    W = l2t_v @ l1t_v + R
+    w_bits = oracle.round_bf16(W)
+    l1t, l2t, resid = oracle.lowrank_split(U, S, Vh, w_bits, r)
+    assert np.array_equal(oracle.bf16_bits_to_f64(l2t), l2t_v)
+    assert np.array_equal(oracle.bf16_bits_to_f64(l1t), l1t_v)
+    want = oracle.round_bf16(oracle.bf16_bits_to_f64(w_bits) - l2t_v @ l1t_v)
+    assert np.array_equal(resid, want)
+    # rank 0 leaves the weight itself
+    assert np.array_equal(oracle.lowrank_split(U, S, Vh, w_bits, 0)[2], w_bits)
+
+
+def _bf16_f32(a):
+    return oracle.bf16_bits_to_f64(_bf16_bits(a)).astype(np.float32)

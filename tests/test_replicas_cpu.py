@@ -54,3 +54,26 @@ def test_reference_arm_other_ranks_exit_without_work():
                         "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
     assert p.returncode == 0, p.stderr
     assert p.stdout.strip() == ""
+
+
+def test_step_statistics():
+    sys.path.insert(0, ROOT)
+    import bench
+    st = bench.step_stats([3.0, 1.0, 2.0, 10.0, 4.0, 5.0, 6.0, 7.0, 8.0, 9.0, 2.5])
+    assert st["min"] == 1.0 and st["median"] == 5.0 and st["n"] == 11
+    assert st["p90"] == 9.0          # the 10th of 11 sorted values
+    assert st["mean"] == round(sum([3, 1, 2, 10, 4, 5, 6, 7, 8, 9, 2.5]) / 11, 4)
+
+
+def test_reference_arm_prints_one_line_with_its_own_baseline():
+    """Rank 0 of the reference arm: the CPU oracle on a bounded sample, one JSON line with the
+    same metric, impl "reference", an e2e that is the line's own value and no device copies."""
+    import json
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3", "--workload", "small_w4a4", "--ref-step-seconds", "0.5"],
+                       capture_output=True, text=True, timeout=600)
+    assert p.returncode == 0, p.stderr
+    line = json.loads(p.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
+    assert line["e2e"]["value"] == line["value"] and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
