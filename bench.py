@@ -7,10 +7,12 @@ Student-t activations with 1% outlier channels, N(0, 0.02^2) weights, random-ini
 synthetic), the shape the 60 %-of-FP4 target is stated for.  The MXFP4 weight is quantized
 once, before timing (a load-time step).  Beside the headline number the JSON line carries:
   step_ms       median / min / p90 of the timed steps (events around every step);
-  roofline      the dominant kernel (the GEMM) against the tensor-core peak, timed
-                alone with CUDA events on its launch stream (50 launches, an event each),
-                as a fraction of the measured-derived peak and of the nominal 9 PFLOP/s;
-  parts         the quantizer (GB/s against HBM) and the GEMM separately;
+  roofline      the dominant kernel (the GEMM) against the tensor-core peak: its average
+                launch inside the timed region (events between the step's two launches,
+                on their stream), as a fraction of the measured-derived peak and of the
+                nominal 9 PFLOP/s;
+  parts         the quantizer (GB/s against HBM) and the GEMM separately, inside the
+                timed region and, beside that, each alone over 50 back-to-back launches;
   ffn_up_480p_w4a4  the same linear at 480p / 81 frames (M = 32760);
   w4a8          the W4A8 FFN-down linear at 720p (quantize to E4M3 + mxf8f6f4 GEMM),
                 its quantize-dequantize emulation (QDQ) path, and the same linear with
@@ -191,6 +193,24 @@ def time_steps(fn, iters: int, stream):
     return ev[0].elapsed_time(ev[-1]), per
 
 
+def time_steps_parts(parts, iters: int, stream):
+    """iters steps, each the calls in `parts` in order, with a CUDA event on `stream` after
+    every call.  Returns (total ms, per-step ms, per-part ms lists) from the one timed
+    region."""
+    n = len(parts)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(iters * n + 1)]
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for i in range(iters):
+        for j, fn in enumerate(parts):
+            fn()
+            ev[i * n + j + 1].record(stream)
+    ev[-1].synchronize()
+    per_step = [ev[i * n].elapsed_time(ev[(i + 1) * n]) for i in range(iters)]
+    per_part = [[ev[i * n + j].elapsed_time(ev[i * n + j + 1]) for i in range(iters)] for j in range(n)]
+    return ev[0].elapsed_time(ev[-1]), per_step, per_part
+
+
 def step_stats(per):
     """median / min / p90 / mean of per-step milliseconds."""
     v = sorted(per)
@@ -354,40 +374,50 @@ def run_mxq(args):
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     assert ops.poll_status() == 0
 
+    # the timed step is mxq_linear's native path issued as its two launches, the quantizer
+    # into the workspace and the GEMM on it, so that each kernel's time inside the timed
+    # region can be read from events between them (the same kernels on the same buffers
+    # as one mxq_linear call)
+    xc = ws[: ops.codes_bytes(M, K, fmt)]
+    xs_off = (ops.codes_bytes(M, K, fmt) + 255) // 256 * 256
+    xs = ws[xs_off: xs_off + ops.sf_bytes(M, K)]
+
+    def quant():
+        ops.quantize_act(x, fmt, codes=xc, sf=xs)
+
+    def gemm():
+        ops.gemm(xc, xs, fmt, M, K, qw, out=y)
+
     def step():
-        ops.linear(x, qw, fmt=fmt, workspace=ws, out=y)
+        quant()
+        gemm()
 
     if args.only:
         # profiling mode: only the named kernel, `steps` launches after the warm-up
         return profile_one(args, ops, x, qw, ws, y, M, N, K, fmt, stream)
 
-    xc = ws[: ops.codes_bytes(M, K, fmt)]
-    xs_off = (ops.codes_bytes(M, K, fmt) + 255) // 256 * 256
-    xs = ws[xs_off: xs_off + ops.sf_bytes(M, K)]
     for _ in range(args.warmup):
         step()
     barrier(world)
     with ClockSampler(local) as clk:
         barrier(world)
-        ms_total, per_step = time_steps(step, args.steps, stream)
+        ms_total, per_step, (per_q, per_g) = time_steps_parts([quant, gemm], args.steps, stream)
         barrier(world)
-        # the two kernels of the step, each timed alone on the launch stream (50 launches
-        # each; the clocks are sampled through these loops as well)
-        for _ in range(3):
-            ops.quantize_act(x, fmt, codes=xc, sf=xs)
-        q_ms, q_stats = time_kernel(lambda: ops.quantize_act(x, fmt, codes=xc, sf=xs), stream)
-        for _ in range(3):
-            ops.gemm(xc, xs, fmt, M, K, qw, out=y)
-        g_ms, g_stats = time_kernel(lambda: ops.gemm(xc, xs, fmt, M, K, qw, out=y), stream)
-        gemm_path = ops.last_path()
-        barrier(world)
+    gemm_path = ops.last_path()
+    # beside them: each kernel timed alone, 50 launches back to back (a long loop: the
+    # GEMM runs into the 1 kW power cap there)
+    q_alone, q_alone_stats = time_kernel(quant, stream)
+    g_alone, g_alone_stats = time_kernel(gemm, stream)
     ms = max_over_ranks(ms_total / args.steps, world)
     status = ops.poll_status()
     if status != 0:
         raise RuntimeError("device status %d after the timed steps" % status)
     flops = 2.0 * M * N * K
     value = job_tflops(flops, ms, world)
-    q_ms, g_ms = max_over_ranks(q_ms, world), max_over_ranks(g_ms, world)
+    q_stats, g_stats = step_stats(per_q), step_stats(per_g)
+    q_ms = max_over_ranks(sum(per_q) / len(per_q), world)   # average launch inside the timed region
+    g_ms = max_over_ranks(sum(per_g) / len(per_g), world)
+    q_alone, g_alone = max_over_ranks(q_alone, world), max_over_ranks(g_alone, world)
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     g_tflops = flops / (g_ms * 1e-3) / 1e12
     q_gbs = quant_bytes(M, K, fmt) / (q_ms * 1e-3) / 1e9
@@ -415,9 +445,15 @@ def run_mxq(args):
             "quantize": {"ms": round(q_ms, 4), "GB/s": round(q_gbs, 1), "peak_GB/s": peaks["hbm_gbs"],
                          "frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4),
                          "frac_nominal_hbm": round(q_gbs / NOMINAL_HBM_GBS, 4),
-                         "bytes": quant_bytes(M, K, fmt), "launch_ms": q_stats},
+                         "bytes": quant_bytes(M, K, fmt), "launch_ms": q_stats,
+                         "alone_50": {"ms": round(q_alone, 4),
+                                      "GB/s": round(quant_bytes(M, K, fmt) / (q_alone * 1e-3) / 1e9, 1),
+                                      "launch_ms": q_alone_stats}},
             "gemm": {"ms": round(g_ms, 4), "TFLOP/s": round(g_tflops, 1),
-                     "frac_fp4": round(g_tflops / fp4_peak, 4)},
+                     "frac_fp4": round(g_tflops / fp4_peak, 4),
+                     "alone_50": {"ms": round(g_alone, 4), "TFLOP/s": round(flops / (g_alone * 1e-3) / 1e12, 1),
+                                  "frac_fp4": round(flops / (g_alone * 1e-3) / 1e12 / fp4_peak, 4),
+                                  "launch_ms": g_alone_stats}},
         },
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
@@ -529,7 +565,15 @@ def profile_one(args, ops, x, qw, ws, y, M, N, K, fmt, stream):
         fn = lambda: ops.gemm_gelu_quant(xc, xs, fmt, M, K, qw, out_fmt="e2m1", codes=hc, sf=hs)  # noqa: E731
     elif args.only == "transform":
         mul = torch.ones(K, dtype=torch.float32, device=x.device)
-        fn = lambda: ops.quantize_act_transformed(x, fmt, 32, mul, codes=xc, sf=xs)  # noqa: E731
+        fn = lambda: ops.quantize_act_transformed(x, fmt, args.block, mul, codes=xc, sf=xs)  # noqa: E731
+    elif args.only == "quantize_static":
+        codes8 = torch.empty(ops.codes_bytes(M, K, "e4m3"), dtype=torch.uint8, device=x.device)
+        scale = ops.absmax(x).item() / 448.0
+        fn = lambda: ops.quantize_act_static(x, scale, codes=codes8, sf=xs)  # noqa: E731
+    elif args.only == "gemm_bf16":
+        xd = ops.dequantize(xc, xs, M, K, fmt)
+        wd = ops.dequantize(qw.codes, qw.sf, N, K, "e2m1")
+        fn = lambda: ops.gemm_bf16(xd, wd, qw.bias, out=y)  # noqa: E731
     elif args.only == "dequantize":
         xd = torch.empty((M, K), dtype=torch.bfloat16, device=x.device)
         fn = lambda: ops.dequantize(xc, xs, M, K, fmt, out=xd)  # noqa: E731
@@ -540,7 +584,7 @@ def profile_one(args, ops, x, qw, ws, y, M, N, K, fmt, stream):
     ms = time_loop(fn, args.steps, stream)
     status = ops.poll_status()
     print(json.dumps({"only": args.only, "workload": args.workload, "M": M, "N": N, "K": K, "fmt": fmt,
-                      "ms": round(ms, 4), "status": status, "path": ops.last_path()}))
+                      "block": args.block, "ms": round(ms, 4), "status": status, "path": ops.last_path()}))
     if status != 0:
         raise RuntimeError("device status %d" % status)
 
@@ -900,8 +944,11 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=0.0,
                     help="reference arm: seconds of oracle work per step (default: about 150 s over the run)")
     ap.add_argument("--M", type=int, default=0, help="override the workload's row count (profiling)")
-    ap.add_argument("--only", choices=["gemm", "quantize", "gelu_quant", "transform", "dequantize"], default=None,
+    ap.add_argument("--only", choices=["gemm", "quantize", "gelu_quant", "transform", "dequantize", "quantize_static",
+                                       "gemm_bf16"], default=None,
                     help="profiling mode: launch only this kernel, --steps times")
+    ap.add_argument("--block", type=int, default=32, choices=[32, 128],
+                    help="profiling mode: rotation block of the transform quantizer")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.impl == "reference":

@@ -53,6 +53,7 @@ SIGNATURES = {
     "mxq_dit_block_linears": ([ctypes.POINTER(WDesc), ctypes.POINTER(_vp), ctypes.POINTER(_i64),
                                ctypes.POINTER(_vp), _u32, _i32, _vp, _i64, _vp], _i32),
     "mxq_block_workspace_bytes": ([ctypes.POINTER(WDesc), ctypes.POINTER(_i64), _u32, _i32], _i64),
+    "mxq_block_workspace_min_bytes": ([ctypes.POINTER(WDesc), ctypes.POINTER(_i64), _u32, _i32], _i64),
     "mxq_linear_noalloc": ([_vp, _i64, _i64, _vp, _vp, _i64, _vp, _i32, _vp, _vp], _i32),
     "mxq_linear_noalloc_max_scratch_bytes": ([], _i64),
     "mxq_gemm_gelu_quant": ([_vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp], _i32),

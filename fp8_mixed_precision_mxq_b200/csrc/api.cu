@@ -330,7 +330,7 @@ int mxq_linear(const void* x_bf16, int64_t M, int64_t K, const void* w_codes, co
                       static_cast<cudaStream_t>(stream));
 }
 
-int64_t mxq_block_workspace_bytes(const mxq_wdesc* w, const int64_t* M_in, uint32_t w4a8_bits, int mode)
+int64_t mxq_block_workspace_min_bytes(const mxq_wdesc* w, const int64_t* M_in, uint32_t w4a8_bits, int mode)
 {
     if (!w || !M_in) return -1;
     int64_t need = 0;
@@ -342,6 +342,96 @@ int64_t mxq_block_workspace_bytes(const mxq_wdesc* w, const int64_t* M_in, uint3
     }
     return need;
 }
+
+int64_t mxq_block_workspace_bytes(const mxq_wdesc* w, const int64_t* M_in, uint32_t w4a8_bits, int mode)
+{
+    const int64_t seq = mxq_block_workspace_min_bytes(w, M_in, w4a8_bits, mode);
+    if (seq < 0 || mode != MXQ_MODE_NATIVE) return seq;
+    int64_t sum = 0;  // one quantized activation per linear
+    for (int i = 0; i < 8; ++i)
+        sum += round_up(mxq_workspace_bytes(M_in[i], w[i].N, w[i].K, (w4a8_bits >> i) & 1u ? MXQ_FMT_E4M3 : MXQ_FMT_E2M1,
+                                            MXQ_MODE_NATIVE),
+                        kWsAlign);
+    return std::max(seq, sum);
+}
+
+}  // extern "C"
+
+namespace {
+
+// The stream and events the block entry point uses to quantize the next linears' inputs
+// while the GEMMs run: one stream (non-blocking) and nine events per device, created on
+// first use and kept until the process exits.  The enqueue sequence that uses them holds
+// g_side_mu, so calls from several host threads cannot interleave their records and waits.
+constexpr int kSideMaxDevices = 64;
+struct SideStream {
+    cudaStream_t s = nullptr;
+    cudaEvent_t ev[9] = {};
+};
+SideStream g_side[kSideMaxDevices];
+std::mutex g_side_mu;
+
+int side_stream(SideStream** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(MXQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kSideMaxDevices) return fail(MXQ_ERR_UNSUPPORTED, "device index %d is too large", dev);
+    SideStream& sd = g_side[dev];
+    if (!sd.s) {
+        e = cudaStreamCreateWithFlags(&sd.s, cudaStreamNonBlocking);
+        for (int i = 0; i < 9 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&sd.ev[i], cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            sd.s = nullptr;
+            return fail(MXQ_ERR_CUDA, "creating the block's side stream: %s", cudaGetErrorString(e));
+        }
+    }
+    *out = &sd;
+    return MXQ_OK;
+}
+
+// Native block with one quantized-activation buffer per linear: every input is quantized on
+// the side stream, back to back, starting after the caller's earlier work; each GEMM on the
+// caller's stream waits only for its own input's quantizer, so the later quantizers run
+// while the earlier GEMMs do (the quantizer's CTAs need no shared memory and fit beside the
+// GEMM's one CTA per SM).  The last GEMM waits for the last quantizer, so when the caller's
+// stream has passed this call, all of it has finished.
+int run_block_overlapped(const mxq_wdesc* w, const void* const* x_in, const int64_t* M_in, void* const* y_out,
+                         uint32_t w4a8_bits, void* workspace, cudaStream_t stream)
+{
+    std::lock_guard<std::mutex> g(g_side_mu);
+    SideStream* sd = nullptr;
+    RETURN_IF(side_stream(&sd));
+    uint8_t* buf[8];
+    uint8_t* p = static_cast<uint8_t*>(workspace);
+    for (int i = 0; i < 8; ++i) {
+        const int fmt = (w4a8_bits >> i) & 1u ? MXQ_FMT_E4M3 : MXQ_FMT_E2M1;
+        buf[i] = p;
+        p += round_up(linear_ws(M_in[i], w[i].N, w[i].K, fmt, MXQ_MODE_NATIVE), kWsAlign);
+    }
+    RETURN_IF(cuda_rc(cudaEventRecord(sd->ev[8], stream), "event record"));
+    RETURN_IF(cuda_rc(cudaStreamWaitEvent(sd->s, sd->ev[8], 0), "stream wait"));
+    for (int i = 0; i < 8; ++i) {
+        const int fmt = (w4a8_bits >> i) & 1u ? MXQ_FMT_E4M3 : MXQ_FMT_E2M1;
+        uint8_t* xc = buf[i];
+        uint8_t* xs = xc + round_up(codes_bytes(M_in[i], w[i].K, fmt), kWsAlign);
+        RETURN_IF(cuda_rc(launch_quantize(x_in[i], M_in[i], w[i].K, fmt, xc, xs, sd->s), "quantize launch"));
+        RETURN_IF(cuda_rc(cudaEventRecord(sd->ev[i], sd->s), "event record"));
+    }
+    for (int i = 0; i < 8; ++i) {
+        const int fmt = (w4a8_bits >> i) & 1u ? MXQ_FMT_E4M3 : MXQ_FMT_E2M1;
+        uint8_t* xc = buf[i];
+        uint8_t* xs = xc + round_up(codes_bytes(M_in[i], w[i].K, fmt), kWsAlign);
+        RETURN_IF(cuda_rc(cudaStreamWaitEvent(stream, sd->ev[i], 0), "stream wait"));
+        int rc = run_gemm(xc, xs, fmt, M_in[i], w[i].K, w[i].codes, w[i].sf, w[i].N, w[i].bias, y_out[i], stream);
+        if (rc != MXQ_OK) return fail(rc, "block linear %d: %s", i, g_err);
+    }
+    return MXQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
 
 int mxq_dit_block_linears(const mxq_wdesc* w, const void* const* x_in, const int64_t* M_in, void* const* y_out,
                           uint32_t w4a8_bits, int mode, void* workspace, int64_t ws_bytes, void* stream)
@@ -357,19 +447,24 @@ int mxq_dit_block_linears(const mxq_wdesc* w, const void* const* x_in, const int
                             y_out[i]);
         if (rc != MXQ_OK) return fail(rc, "block linear %d: %s", i, g_err);
     }
-    const int64_t need = mxq_block_workspace_bytes(w, M_in, w4a8_bits, mode);
+    const int64_t need = mxq_block_workspace_min_bytes(w, M_in, w4a8_bits, mode);
     if (ws_bytes < need)
         return fail(MXQ_ERR_WORKSPACE, "block workspace has %lld bytes, needs %lld", (long long)ws_bytes,
                     (long long)need);
     RETURN_IF(check_device());
-    for (int i = 0; i < 8; ++i) {
-        const int fmt = (w4a8_bits >> i) & 1u ? MXQ_FMT_E4M3 : MXQ_FMT_E2M1;
-        int rc = run_linear(x_in[i], M_in[i], w[i].K, w[i].codes, w[i].sf, w[i].N, w[i].bias, fmt, mode, workspace,
-                            ws_bytes, y_out[i], static_cast<cudaStream_t>(stream));
-        if (rc != MXQ_OK) return fail(rc, "block linear %d: %s", i, g_err);
+    const bool overlap = mode == MXQ_MODE_NATIVE && ws_bytes >= mxq_block_workspace_bytes(w, M_in, w4a8_bits, mode);
+    if (overlap) {
+        RETURN_IF(run_block_overlapped(w, x_in, M_in, y_out, w4a8_bits, workspace, static_cast<cudaStream_t>(stream)));
+    } else {
+        for (int i = 0; i < 8; ++i) {
+            const int fmt = (w4a8_bits >> i) & 1u ? MXQ_FMT_E4M3 : MXQ_FMT_E2M1;
+            int rc = run_linear(x_in[i], M_in[i], w[i].K, w[i].codes, w[i].sf, w[i].N, w[i].bias, fmt, mode,
+                                workspace, ws_bytes, y_out[i], static_cast<cudaStream_t>(stream));
+            if (rc != MXQ_OK) return fail(rc, "block linear %d: %s", i, g_err);
+        }
     }
-    snprintf(g_path, sizeof g_path, "block %s w4a8_bits 0x%02x", mode == MXQ_MODE_QDQ ? "qdq" : "native",
-             w4a8_bits);
+    snprintf(g_path, sizeof g_path, "block %s%s w4a8_bits 0x%02x", mode == MXQ_MODE_QDQ ? "qdq" : "native",
+             overlap ? " overlapped" : "", w4a8_bits);
     return ok();
 }
 

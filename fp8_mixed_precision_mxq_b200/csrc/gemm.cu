@@ -492,22 +492,19 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                 uint32_t sc_byte = 0u;  // quantizing epilogue: the chunk's E8M0 scale
                 const int n = nb * BN + c * 32;
                 if (n < p.N) {  // warp-uniform
-                    float bv[32];
+                    // the chunk's 32 bias values as 16 bf16 pairs (columns 2i, 2i + 1 in word
+                    // i), kept packed and widened where they are used
+                    uint32_t bw[16];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) bv[i] = 0.f;
+                    for (int i = 0; i < 16; ++i) bw[i] = 0u;
                     if (has_bias) {
 #pragma unroll
                         for (int g = 0; g < 4; ++g) {
                             const int src = 4 * c + g;  // lane holding columns c*32 + 8g ..
-                            const uint32_t w[4] = {__shfl_sync(0xFFFFFFFFu, bias8.x, src),
-                                                   __shfl_sync(0xFFFFFFFFu, bias8.y, src),
-                                                   __shfl_sync(0xFFFFFFFFu, bias8.z, src),
-                                                   __shfl_sync(0xFFFFFFFFu, bias8.w, src)};
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                bv[8 * g + 2 * i] = __uint_as_float(w[i] << 16);
-                                bv[8 * g + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-                            }
+                            bw[4 * g] = __shfl_sync(0xFFFFFFFFu, bias8.x, src);
+                            bw[4 * g + 1] = __shfl_sync(0xFFFFFFFFu, bias8.y, src);
+                            bw[4 * g + 2] = __shfl_sync(0xFFFFFFFFu, bias8.z, src);
+                            bw[4 * g + 3] = __shfl_sync(0xFFFFFFFFu, bias8.w, src);
                         }
                     }
                     // o: the chunk in bf16 -- y = acc + bias, or h = GELU of that rounded to bf16
@@ -520,7 +517,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                         for (int i = 0; i < 16; ++i) {
                             const float2 y = __ffma2_rn(
                                 make_float2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1])), alpha2,
-                                make_float2(bv[2 * i], bv[2 * i + 1]));
+                                make_float2(lo_f(bw[i]), hi_f(bw[i])));
                             __nv_bfloat162 y2 = __floats2bfloat162_rn(y.x, y.y);
                             if constexpr (decltype(gelu)::value) {
                                 const float2 g = gelu2_f32(make_float2(__low2float(y2), __high2float(y2)));

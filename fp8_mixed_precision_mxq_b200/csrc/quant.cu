@@ -57,59 +57,63 @@ __device__ __forceinline__ uint32_t sf_offset(uint32_t r, uint32_t kb, uint32_t 
 constexpr int kFmtStatic = 2;
 
 // The scale as the static quantizer takes it: s = sn * 2^-k with sn in [1, 2), the
-// reciprocal r = fl32(1/sn) in (1/2, 1], and 2^k split into two factors p1 * p2 that are
-// binary32 normals (k runs from -127 to 149).
+// reciprocal r = fl32(1/sn) in (1/2, 1], and 2^k as p1 (and p2 when two_step: k runs from
+// -127 to 149, and 2^k is a binary32 normal only up to 127).
 struct StaticScale {
     float sn, r, p1, p2;
+    int two_step;
 };
 
 // One value's E4M3 code is RNE_sat(x / s), decided exactly in binary32:
-//  * xs = x * 2^k, so that x / s = xs / sn with sn in [1, 2) (exact, except overflow,
-//    where x / s is above 2^127 and saturates either way, and underflow, where x / s is
-//    below 2^-125 and rounds to a zero of x's sign either way); xs is clamped to the
-//    finite range (NaN kept), so that r <= 1 keeps every product below finite;
-//  * q0 = fl(xs * r), then one correction q = fl(q0 + fl(xs - q0 sn) * r) (fused
-//    multiply-adds: Markstein's iteration, M. Cornea, J. Harrison, P. Tang, "Scientific
-//    Computing on Itanium-based Systems", and J.-M. Muller et al., "Handbook of
-//    Floating-Point Arithmetic", section on division by Newton-Raphson iterations): the
-//    relative error of q0 is at most about 2^-23, the correction leaves about 2^-46 before
-//    its own rounding, so q is one of the two binary32 neighbours of xs / sn (faithful);
-//  * the remainder e = xs - q sn of a faithful quotient is a binary32 number whenever
+//  * xs = x * 2^k, so that x / s = xs / sn with sn in [1, 2) (exact, except overflow, where
+//    x / s is above 2^127 and saturates either way, and underflow, where x / s is below
+//    2^-125 and rounds to a zero of x's sign either way); |xs| is then clamped to the
+//    largest finite binary32 (sign and NaN kept: Inf saturates like any huge value), so
+//    with r <= 1 every later value stays finite;
+//  * q0 = fl(xs * r), then one Markstein correction q1 = fl(q0 + fl(xs - q0 sn) * r)
+//    (fused multiply-adds; M. Cornea, J. Harrison, P. Tang, "Scientific Computing on
+//    Itanium-based Systems", and J.-M. Muller et al., "Handbook of Floating-Point
+//    Arithmetic", on division by Newton-Raphson iterations): q0 is within about 2^-23
+//    relative, the correction leaves about 2^-46 before its own rounding, so q1 is within
+//    half an ulp plus 2^-22 ulp of xs / sn: faithful, and the correctly rounded quotient
+//    unless xs / sn lies that close to a midpoint between binary32 values;
+//  * the remainder e1 = xs - q1 sn of a faithful quotient is a binary32 number whenever
 //    |xs| >= 2^-102 (both terms are multiples of 2^(floor(log2 |xs|) - 47)), so the fused
-//    multiply-add returns it exactly and its sign tells on which side of q the quotient
-//    lies; below 2^-102 the quotient is far under E4M3's smallest midpoint 2^-10;
-//  * q is then replaced by the quotient rounded to odd (truncated toward zero, the last
-//    bit set when inexact: S. Boldo, G. Melquiond, "Emulation of FMA and correctly rounded
-//    sums: proved algorithms using rounding to odd", IEEE TC 2008), and rounding a
-//    round-to-odd value of at least two more bits than the target gives the same result
-//    as rounding the exact value once: cvt's round-to-nearest-even then is the exact
-//    quotient's.
-__device__ __forceinline__ float round_to_odd(float q, float e)
-{
-    const uint32_t b = __float_as_uint(q);
-    // inexact and finite: step toward zero when the remainder's sign differs from q's
-    // (|x / s| < |q|), then set the last bit
-    const bool adj = e != 0.0f && (b & 0x7FFFFFFFu) < 0x7F800000u;
-    return __uint_as_float(adj ? ((b - ((__float_as_uint(e) ^ b) >> 31)) | 1u) : b);
-}
-
-__device__ __forceinline__ float clamp_finite_nan(float v)
+//    multiply-add returns it exactly; below 2^-102 the quotient is far under E4M3's
+//    smallest midpoint 2^-10 and only its sign matters;
+//  * z = fl_rz(q1 + e1 r) (a fused multiply-add rounded toward zero) is the quotient
+//    truncated to binary32: q1 + e1 / sn is the exact quotient, e1 r moves it by less than
+//    an ulp of q1 in the same direction, and it could reach the next binary32 value only if
+//    the quotient lay within 2^-24 ulp of it -- where q1 is the correctly rounded quotient
+//    and |e1 / sn| is at most half an ulp;
+//  * setting z's last bit when e1 != 0 gives the quotient rounded to odd (S. Boldo,
+//    G. Melquiond, "Emulation of FMA and correctly rounded sums: proved algorithms using
+//    rounding to odd", IEEE TC 2008), and rounding a round-to-odd value of at least two more
+//    bits than the target gives the same result as rounding the exact value once: cvt's
+//    round-to-nearest-even is then the exact quotient's.  The sign is copied from xs (a
+//    zero quotient keeps x's sign).
+__device__ __forceinline__ float clamp_finite(float v)
 {
     float d;
-    asm("min.NaN.f32 %0, %1, 0f7F7FFFFF;" : "=f"(d) : "f"(v));
-    asm("max.NaN.f32 %0, %1, 0fFF7FFFFF;" : "=f"(d) : "f"(d));
+    // sign(v) * min(|v|, largest finite), NaN kept
+    asm("min.NaN.xorsign.abs.f32 %0, %1, 0f7F7FFFFF;" : "=f"(d) : "f"(v));
     return d;
 }
 
 __device__ __forceinline__ float2 static_quotient2(float2 x, const StaticScale& st)
 {
-    float2 xs = __fmul2_rn(__fmul2_rn(x, make_float2(st.p1, st.p1)), make_float2(st.p2, st.p2));
-    xs = make_float2(clamp_finite_nan(xs.x), clamp_finite_nan(xs.y));
+    float2 xs = __fmul2_rn(x, make_float2(st.p1, st.p1));
+    if (st.two_step) xs = __fmul2_rn(xs, make_float2(st.p2, st.p2));
+    xs = make_float2(clamp_finite(xs.x), clamp_finite(xs.y));
     const float2 r = make_float2(st.r, st.r), ns = make_float2(-st.sn, -st.sn);
     const float2 q0 = __fmul2_rn(xs, r);
-    const float2 q = __ffma2_rn(__ffma2_rn(q0, ns, xs), r, q0);
-    const float2 e = __ffma2_rn(q, ns, xs);
-    return make_float2(round_to_odd(q.x, e.x), round_to_odd(q.y, e.y));
+    const float2 q1 = __ffma2_rn(__ffma2_rn(q0, ns, xs), r, q0);
+    const float2 e1 = __ffma2_rn(q1, ns, xs);
+    const float2 z = __ffma2_rz(e1, r, q1);
+    const uint32_t zx = (__float_as_uint(z.x) & 0x7FFFFFFFu) | (__float_as_uint(xs.x) & 0x80000000u);
+    const uint32_t zy = (__float_as_uint(z.y) & 0x7FFFFFFFu) | (__float_as_uint(xs.y) & 0x80000000u);
+    return make_float2(__uint_as_float(zx | (e1.x != 0.0f ? 1u : 0u)),
+                       __uint_as_float(zy | (e1.y != 0.0f ? 1u : 0u)));
 }
 
 template <int FMT>
@@ -528,7 +532,7 @@ __global__ void __launch_bounds__(kTThreads, 5) quantize_transform_kernel(
 cudaError_t launch_quantize_any(const void* x, int64_t rows, int64_t K, int fmt, float scale, void* codes,
                                 void* sf, cudaStream_t stream)
 {
-    StaticScale st{1.0f, 1.0f, 1.0f, 1.0f};
+    StaticScale st{1.0f, 1.0f, 1.0f, 1.0f, 0};
     if (fmt == kFmtStatic) {
         int e = 0;
         const float m = std::frexp(scale, &e);  // scale = m 2^e, m in [1/2, 1)
@@ -537,8 +541,9 @@ cudaError_t launch_quantize_any(const void* x, int64_t rows, int64_t K, int fmt,
         // fl32(1/sn): the double quotient is never within 2^-53 of a binary32 midpoint
         // unless it is one, so rounding it to binary32 gives the correctly rounded value
         st.r = static_cast<float>(1.0 / static_cast<double>(st.sn));
-        st.p1 = std::ldexp(1.0f, k / 2);
-        st.p2 = std::ldexp(1.0f, k - k / 2);
+        st.two_step = k > 127 ? 1 : 0;
+        st.p1 = std::ldexp(1.0f, st.two_step ? k / 2 : k);
+        st.p2 = std::ldexp(1.0f, st.two_step ? k - k / 2 : 0);
     }
     const uint32_t n_groups = static_cast<uint32_t>(rows * K / 8);
     const uint32_t KB = static_cast<uint32_t>(K / 32);

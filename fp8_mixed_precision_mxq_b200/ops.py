@@ -407,10 +407,13 @@ def linear_lowrank(x: torch.Tensor, residual: QWeight, l1t: torch.Tensor, l2t: t
     return out
 
 
-def block_workspace_bytes(weights, rows, w4a8_bits: int, mode="native") -> int:
+def block_workspace_bytes(weights, rows, w4a8_bits: int, mode="native", minimum: bool = False) -> int:
+    """Workspace of dit_block_linears: by default the size that lets the quantizers overlap
+    the GEMMs (native mode); minimum=True gives the least it accepts."""
     descs = (WDesc * 8)(*[w.desc() for w in weights])
     ms = (ctypes.c_int64 * 8)(*rows)
-    return int(_lib.lib().mxq_block_workspace_bytes(descs, ms, w4a8_bits, _mode(mode)))
+    fn = _lib.lib().mxq_block_workspace_min_bytes if minimum else _lib.lib().mxq_block_workspace_bytes
+    return int(fn(descs, ms, w4a8_bits, _mode(mode)))
 
 
 def dit_block_linears(weights, xs, w4a8_bits: int, mode="native", workspace=None, outs=None, stream=None):

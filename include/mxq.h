@@ -148,14 +148,23 @@ typedef struct {
  * bit i of w4a8_bits set -> that linear runs W4A8 (E4M3 activations), else W4A4.
  * The per-expert, per-block policy of the blog (sections "Mixed-Precision
  * selection", "Practical workflow" step 6) is applied by passing 0xFF or 0x00 (or a
- * per-linear refinement) for each (expert, block).  workspace must hold
- * mxq_block_workspace_bytes(...) bytes. */
+ * per-linear refinement) for each (expert, block).  workspace must hold at least
+ * mxq_block_workspace_min_bytes(...) bytes; mxq_block_workspace_bytes(...) lets the
+ * quantizers overlap the GEMMs (below). */
 int mxq_dit_block_linears(const mxq_wdesc* w, const void* const* x_in, const int64_t* M_in,
                           void* const* y_out, uint32_t w4a8_bits, int mode, void* workspace, int64_t ws_bytes,
                           void* stream);
 
-/* Workspace bytes mxq_dit_block_linears needs for these weights and row counts. */
+/* Workspace bytes of mxq_dit_block_linears.  mxq_block_workspace_min_bytes: the least it
+ * accepts (one linear's workspace, reused; the linears then run one after another).
+ * mxq_block_workspace_bytes: in NATIVE mode, a quantized-activation buffer for every
+ * linear; with a workspace of at least this size the call quantizes all eight inputs on
+ * a stream of the library's own (created once per device, with its events, on first use)
+ * while the GEMMs run on `stream`, each GEMM waiting only for its own input.  When
+ * `stream` has passed the call, all of its work is done.  In QDQ mode both sizes are the
+ * same. */
 int64_t mxq_block_workspace_bytes(const mxq_wdesc* w, const int64_t* M_in, uint32_t w4a8_bits, int mode);
+int64_t mxq_block_workspace_min_bytes(const mxq_wdesc* w, const int64_t* M_in, uint32_t w4a8_bits, int mode);
 
 /* The native linear layer (as mxq_linear with mode NATIVE) for callers that cannot
  * allocate device memory where they run a layer -- for example code under a memory

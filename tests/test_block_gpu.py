@@ -84,11 +84,33 @@ def test_block_rejects_wrong_workspace():
     ops = _ops()
     qws, _, _ = block(seed=5)
     xs = synth.block_inputs(64, seed=5, device="cuda", ctx=16)
-    need = ops.block_workspace_bytes(qws, [x.shape[0] for x in xs], 0xFF)
+    need = ops.block_workspace_bytes(qws, [x.shape[0] for x in xs], 0xFF, minimum=True)
     small = torch.empty(need // 2, dtype=torch.uint8, device="cuda")
     with pytest.raises(Exception) as ei:
         ops.dit_block_linears(qws, xs, 0xFF, workspace=small)
     assert "WORKSPACE" in str(ei.value)
+
+
+@pytest.mark.parametrize("bits", [0x00, 0xFF, 0x5A])
+def test_block_overlapped_equals_sequential(bits):
+    """With a workspace that holds every linear's quantized input the block quantizes them
+    on the library's side stream while the GEMMs run; with the minimum workspace it runs
+    the linears one after another.  Both give the same bits, on two calls in a row."""
+    ops = _ops()
+    qws, _, _ = block(seed=9)
+    xs = synth.block_inputs(300, seed=9, device="cuda", ctx=40)
+    rows = [x.shape[0] for x in xs]
+    big = torch.empty(ops.block_workspace_bytes(qws, rows, bits), dtype=torch.uint8, device="cuda")
+    small = torch.empty(ops.block_workspace_bytes(qws, rows, bits, minimum=True), dtype=torch.uint8, device="cuda")
+    assert big.numel() > small.numel()
+    for _ in range(2):
+        y_seq = ops.dit_block_linears(qws, xs, bits, workspace=small)
+        assert "overlapped" not in ops.last_path()
+        y_ovl = ops.dit_block_linears(qws, xs, bits, workspace=big)
+        assert "overlapped" in ops.last_path()
+        assert ops.poll_status() == 0
+        for i, (a, b) in enumerate(zip(y_seq, y_ovl)):
+            assert torch.equal(a, b), "linear %d differs" % i
 
 
 @pytest.mark.slow

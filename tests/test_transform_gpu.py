@@ -39,7 +39,7 @@ def test_quantize_transformed_against_definition(fmt, block, smooth, M, K):
     torch.cuda.synchronize()
     ref = oracle.quantize_transformed(_mx.bits(x), _mx.FMT[fmt], block, None if mul is None else mul.cpu().numpy())
     _mx.check_transformed(codes, sf, M, K, fmt, ref, "%s B=%d smooth=%s %dx%d" % (fmt, block, smooth, M, K),
-                          max_uncertain=1e-3 if M * K >= 10000 else 0.01)
+                          max_uncertain=_mx.UNCERTAIN_LIMIT[fmt] * (1 if M * K >= 10000 else 10))
 
 
 @pytest.mark.parametrize("block", [32, 128])
