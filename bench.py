@@ -69,9 +69,9 @@ FP8_OVER_BF16 = 2.0   # 4.5 PFLOP/s FP8
 GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precision_mxq_b200/csrc/ptx.cuh",
                 "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h", "fp8_mixed_precision_mxq_b200/csrc/mx_elem.cuh"]
 GEMM_TRAFFIC = {
-    ("ffn_up_480p_w4a4", 32760): {
-        "bytes": 382355200 + 857401344,
-        "sources_sha256": "4ead914060badceb676f2b238216b77003cb214ce2fbea7c8c3ffcd69c695b4c"},
+    ("ffn_up_720p_w4a4", 75600): {
+        "bytes": 854573568 + 2047664128,
+        "sources_sha256": "efdee61c67b6699c132e7ecc24ff8382e0e3745a06aa0d2fe4f087f9c46b6410"},
 }
 
 
@@ -565,7 +565,7 @@ def profile_one(args, ops, x, qw, ws, y, M, N, K, fmt, stream):
         fn = lambda: ops.gemm_gelu_quant(xc, xs, fmt, M, K, qw, out_fmt="e2m1", codes=hc, sf=hs)  # noqa: E731
     elif args.only == "transform":
         mul = torch.ones(K, dtype=torch.float32, device=x.device)
-        fn = lambda: ops.quantize_act_transformed(x, fmt, args.block, mul, codes=xc, sf=xs)  # noqa: E731
+        fn = lambda: ops.quantize_act_transformed(x, fmt, args.rot_block, mul, codes=xc, sf=xs)  # noqa: E731
     elif args.only == "quantize_static":
         codes8 = torch.empty(ops.codes_bytes(M, K, "e4m3"), dtype=torch.uint8, device=x.device)
         scale = ops.absmax(x).item() / 448.0
@@ -584,7 +584,7 @@ def profile_one(args, ops, x, qw, ws, y, M, N, K, fmt, stream):
     ms = time_loop(fn, args.steps, stream)
     status = ops.poll_status()
     print(json.dumps({"only": args.only, "workload": args.workload, "M": M, "N": N, "K": K, "fmt": fmt,
-                      "block": args.block, "ms": round(ms, 4), "status": status, "path": ops.last_path()}))
+                      "rot_block": args.rot_block, "ms": round(ms, 4), "status": status, "path": ops.last_path()}))
     if status != 0:
         raise RuntimeError("device status %d" % status)
 
@@ -947,7 +947,7 @@ def main():
     ap.add_argument("--only", choices=["gemm", "quantize", "gelu_quant", "transform", "dequantize", "quantize_static",
                                        "gemm_bf16"], default=None,
                     help="profiling mode: launch only this kernel, --steps times")
-    ap.add_argument("--block", type=int, default=32, choices=[32, 128],
+    ap.add_argument("--rot-block", type=int, default=32, choices=[32, 128],
                     help="profiling mode: rotation block of the transform quantizer")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
