@@ -144,7 +144,7 @@ class ClockSampler:
                 self.thread.join(timeout=2)
 
     def summary(self):
-        sm, smax, reasons = [], [], set()
+        sm, smax, watts, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.lines:
             parts = [x.strip() for x in line.split(",")]
@@ -155,13 +155,17 @@ class ClockSampler:
                 smax.append(float(parts[1]))
             except ValueError:
                 continue
+            try:
+                watts.append(float(parts[2]))
+            except ValueError:
+                pass
             for name, v in zip(names, parts[4:8]):
                 if v.lower().startswith("active"):
                     reasons.add(name)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "power_w": statistics.median(watts) if watts else None}
 
 
 # ---------------------------------------------------------------------------- timing
@@ -219,14 +223,23 @@ def step_stats(per):
             "mean": round(sum(v) / len(v), 4), "n": len(v)}
 
 
-def time_kernel(fn, stream, min_iters: int = 50, min_ms: float = 0.0):
+def time_kernel(fn, stream, min_iters: int = 50, min_ms: float = 0.0, idle_s: float = 0.0):
     """A kernel timed alone on its stream: min_iters launches, more if needed to fill min_ms
-    of device time (a short probe sizes the loop), one event per launch.  Returns the mean
+    of device time (a short probe sizes the loop), one event per launch, after idle_s
+    seconds with the GPU idle (a preceding loop of GEMMs leaves the SM clock below its
+    maximum for a while, which the partly issue-bound quantizers feel).  Returns the mean
     launch time (ms) and the per-launch statistics."""
+    if idle_s > 0:
+        torch.cuda.synchronize()
+        time.sleep(idle_s)
     probe = time_loop(fn, 3, stream)
     iters = max(min_iters, int(min_ms / max(probe, 1e-3)) + 1)
     total, per = time_steps(fn, iters, stream)
     return total / iters, step_stats(per)
+
+
+# seconds of idle GPU before each stand-alone quantizer loop that follows GEMM loops
+QUANT_IDLE_S = 1.0
 
 
 def quant_bytes(M, K, fmt):
@@ -363,6 +376,8 @@ def run_mxq(args):
     M, K, N, fmt = (args.M or c["M"]), c["K"], c["N"], c["fmt"]
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
+    if args.only == "block":
+        return profile_block(args, ops, synth, dev, stream)
 
     # inputs (per-rank seed offset: every replica gets its own batch)
     x = synth.activation(M, K, c["act"], seed=replica_seed(c["seed"], rank), device=dev,
@@ -609,7 +624,8 @@ def bench_linear(args, ops, synth, wl_name, dev, stream, world, rank, peaks):
     off = (ops.codes_bytes(M, K, "e2m1") + 255) // 256 * 256
     xs = ws[off: off + ops.sf_bytes(M, K)]
     g_ms = max_over_ranks(time_loop(lambda: ops.gemm(xc, xs, "e2m1", M, K, qw, out=y), iters, stream), world)
-    q_ms = max_over_ranks(time_loop(lambda: ops.quantize_act(x, "e2m1", codes=xc, sf=xs), iters, stream), world)
+    q_ms = max_over_ranks(time_kernel(lambda: ops.quantize_act(x, "e2m1", codes=xc, sf=xs), stream,
+                                      idle_s=QUANT_IDLE_S)[0], world)
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     if ops.poll_status() != 0:
         raise RuntimeError("device status set during the %s measurement" % wl_name)
@@ -711,14 +727,17 @@ def bench_transform(args, ops, synth, dev, stream, world, rank, peaks, x, w, b):
         qw = ops.quantize_weight_transformed(w, bias=b, block=block, mul=s)
         fq = lambda blk=block: ops.quantize_act_transformed(x, "e2m1", blk, inv_s, codes=codes, sf=sf)  # noqa: E731
         fl = lambda blk=block, q=qw: ops.linear_transformed(x, q, "e2m1", blk, inv_s, workspace=ws, out=y)  # noqa
+        # the quantizer alone first (50 launches after a short probe), then the linear
+        fq()
+        q_ms, q_stats = time_kernel(fq, stream, idle_s=QUANT_IDLE_S)
+        q_ms = max_over_ranks(q_ms, world)
         for _ in range(2):
-            fq()
             fl()
-        q_ms = max_over_ranks(time_loop(fq, iters, stream), world)
         l_ms = max_over_ranks(time_loop(fl, iters, stream), world)
         res["hadamard%d" % block] = {
             "quantize_ms": round(q_ms, 4), "quantize_GB/s": round(qbytes / (q_ms * 1e-3) / 1e9, 1),
             "quantize_frac_hbm": round(qbytes / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "quantize_launch_ms": q_stats,
             "linear_ms": round(l_ms, 4), "linear_TFLOP/s": round(job_tflops(flops, l_ms, world), 1)}
     if ops.poll_status() != 0:
         raise RuntimeError("device status set during the transform measurement")
@@ -770,14 +789,57 @@ def bench_block(args, ops, synth, dev, stream, world, rank, peaks):
         fn = lambda bits=bits: ops.dit_block_linears(qws, xs, bits, workspace=wsb, outs=outs)  # noqa: E731
         for _ in range(2):
             fn()
-        ms = max_over_ranks(time_loop(fn, iters, stream), world)
+        with ClockSampler(dev.index) as clk:
+            ms = time_loop(fn, iters, stream)
+        ms = max_over_ranks(ms, world)
         roof = linears_roofline_ms(synth, M, ctx, bits, peaks)
         res[name] = {"mask": "0x%02x" % bits, "ms": round(ms, 3),
                      "TFLOP/s": round(job_tflops(flops, ms, world), 1),
-                     "roofline_ms": round(roof, 3), "frac": round(roof / ms, 4)}
+                     "roofline_ms": round(roof, 3), "frac": round(roof / ms, 4), "clocks": clk.summary()}
+    # where the all-W4A4 block's time goes: each linear's quantizer and GEMM timed alone
+    # (50 launches each) against that linear's FP4 floor
+    fp4 = peaks["bf16_tflops"] * FP4_OVER_BF16 * 1e12
+    per = []
+    for i, (name, N, K, src) in enumerate(synth.BLOCK_LINEARS):
+        rows_i = rows[i]
+        xc = wsb[: ops.codes_bytes(rows_i, K, "e2m1")]
+        off = (ops.codes_bytes(rows_i, K, "e2m1") + 255) // 256 * 256
+        xsf = wsb[off: off + ops.sf_bytes(rows_i, K)]
+        fq = lambda i=i, K=K, xc=xc, xsf=xsf: ops.quantize_act(xs[i], "e2m1", codes=xc, sf=xsf)  # noqa: E731
+        fg = lambda i=i, K=K, r=rows_i, xc=xc, xsf=xsf: ops.gemm(xc, xsf, "e2m1", r, K, qws[i], out=outs[i])  # noqa
+        fq()
+        q_ms, _ = time_kernel(fq, stream)
+        g_ms, _ = time_kernel(fg, stream)
+        fl = 2.0 * rows_i * N * K
+        per.append({"linear": name, "M": rows_i, "N": N, "K": K, "quantize_ms": round(max_over_ranks(q_ms, world), 4),
+                    "gemm_ms": round(max_over_ranks(g_ms, world), 4),
+                    "gemm_frac_fp4": round(fl / fp4 / (g_ms * 1e-3), 4)})
+    res["all_w4a4_per_linear_alone"] = per
     if ops.poll_status() != 0:
         raise RuntimeError("device status set during the block measurement")
     return res
+
+
+def profile_block(args, ops, synth, dev, stream):
+    """Profiling mode for the block: one DiT block's eight linears at 720p under the
+    all-W4A4 mask (overlapped quantizers), `steps` calls after the warm-up."""
+    c = synth.BLOCK_720P
+    ws, bs = synth.block_weights(c["seed"], device=dev)
+    qws = [ops.quantize_weight(w, bias=b) for w, b in zip(ws, bs)]
+    del ws, bs
+    xs = synth.block_inputs(c["M"], seed=c["seed"], device=dev, ctx=c["ctx"])
+    rows = [x.shape[0] for x in xs]
+    outs = [torch.empty((r, w.N), dtype=torch.bfloat16, device=dev) for r, w in zip(rows, qws)]
+    wsb = torch.empty(ops.block_workspace_bytes(qws, rows, 0x00), dtype=torch.uint8, device=dev)
+    fn = lambda: ops.dit_block_linears(qws, xs, 0x00, workspace=wsb, outs=outs)  # noqa: E731
+    for _ in range(args.warmup):
+        fn()
+    ms = time_loop(fn, args.steps, stream)
+    status = ops.poll_status()
+    print(json.dumps({"only": "block", "workload": "dit_block_720p all_w4a4", "M": c["M"], "ctx": c["ctx"],
+                      "ms": round(ms, 4), "status": status, "path": ops.last_path()}))
+    if status != 0:
+        raise RuntimeError("device status %d" % status)
 
 
 def bench_stack(args, ops, synth, dev, stream, world, rank, peaks):
@@ -847,12 +909,13 @@ def bench_w4a8(args, ops, synth, dev, stream, world, rank, peaks):
     xc = ws[: ops.codes_bytes(M, K, "e4m3")]
     off = (ops.codes_bytes(M, K, "e4m3") + 255) // 256 * 256
     xs = ws[off: off + ops.sf_bytes(M, K)]
-    ops.quantize_act(x, "e4m3", codes=xc, sf=xs)
-    q_ms = max_over_ranks(time_loop(lambda: ops.quantize_act(x, "e4m3", codes=xc, sf=xs), iters, stream), world)
+    q_ms, q_stats = time_kernel(lambda: ops.quantize_act(x, "e4m3", codes=xc, sf=xs), stream, idle_s=QUANT_IDLE_S)
+    q_ms = max_over_ranks(q_ms, world)
     g_ms = max_over_ranks(time_loop(lambda: ops.gemm(xc, xs, "e4m3", M, K, qw, out=y), iters, stream), world)
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
     out["quantize_e4m3"] = {"ms": round(q_ms, 4), "GB/s": round(quant_bytes(M, K, "e4m3") / (q_ms * 1e-3) / 1e9, 1),
-                            "frac_hbm": round(quant_bytes(M, K, "e4m3") / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+                            "frac_hbm": round(quant_bytes(M, K, "e4m3") / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                            "launch_ms": q_stats}
     out["gemm_mxf8f6f4"] = {"ms": round(g_ms, 4), "TFLOP/s": round(flops / (g_ms * 1e-3) / 1e12, 1),
                             "frac_fp8": round(flops / (g_ms * 1e-3) / 1e12 / fp8_peak, 4),
                             "peak_fp8": round(fp8_peak, 1)}
@@ -862,14 +925,16 @@ def bench_w4a8(args, ops, synth, dev, stream, world, rank, peaks):
         ops.linear_static(x, qw, scale, workspace=ws, out=y)
     s_ms = max_over_ranks(time_loop(lambda: ops.linear_static(x, qw, scale, workspace=ws, out=y), iters, stream),
                           world)
-    sq_ms = max_over_ranks(time_loop(lambda: ops.quantize_act_static(x, scale, codes=xc, sf=xs), iters, stream),
-                           world)
+    sq_ms, sq_stats = time_kernel(lambda: ops.quantize_act_static(x, scale, codes=xc, sf=xs), stream,
+                                  idle_s=QUANT_IDLE_S)
+    sq_ms = max_over_ranks(sq_ms, world)
     out["static_e4m3"] = {"scale": scale, "linear_ms": round(s_ms, 4),
                           "linear_TFLOP/s": round(flops / (s_ms * 1e-3) / 1e12, 1),
                           "quantize_ms": round(sq_ms, 4),
                           "quantize_GB/s": round(quant_bytes(M, K, "e4m3") / (sq_ms * 1e-3) / 1e9, 1),
                           "quantize_frac_hbm": round(quant_bytes(M, K, "e4m3") / (sq_ms * 1e-3) / 1e9 /
-                                                     peaks["hbm_gbs"], 4)}
+                                                     peaks["hbm_gbs"], 4),
+                          "quantize_launch_ms": sq_stats}
     if ops.poll_status() != 0:
         raise RuntimeError("device status set during the W4A8 measurement")
     return out
@@ -945,7 +1010,7 @@ def main():
                     help="reference arm: seconds of oracle work per step (default: about 150 s over the run)")
     ap.add_argument("--M", type=int, default=0, help="override the workload's row count (profiling)")
     ap.add_argument("--only", choices=["gemm", "quantize", "gelu_quant", "transform", "dequantize", "quantize_static",
-                                       "gemm_bf16"], default=None,
+                                       "gemm_bf16", "block"], default=None,
                     help="profiling mode: launch only this kernel, --steps times")
     ap.add_argument("--rot-block", type=int, default=32, choices=[32, 128],
                     help="profiling mode: rotation block of the transform quantizer")

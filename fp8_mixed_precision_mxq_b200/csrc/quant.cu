@@ -319,17 +319,18 @@ int num_sms()
 // channel (SmoothQuant's 1/s for activations, s for weights; mul may be null), then each
 // block of kB consecutive values along K is rotated by the Sylvester Hadamard matrix
 // normalized by c = fl32(1/sqrt kB), and the result is MX-quantized from the binary32
-// values.  Every step is one binary32 operation in a fixed order -- butterflies
+// values.  Every step is one binary32 operation -- the multiply by mul, butterflies
 // (a, b) -> (a + b, a - b) for h = 1, 2, 4, ..., kB/2, then the multiply by c -- written
-// with the _rn intrinsics so the compiler cannot fuse them, which makes the codes the
-// exact function of x the definition states.
-// Layout: one lane per 32-element MX block; the 32-point transform, the block's abs-max
-// and its scale byte stay in the lane.  For kB = 128 four consecutive lanes hold one
-// rotation block and the last two butterfly stages (h = 32, 64) pair lanes by
-// xor-shuffles.  Input: x seen as a [n_blocks, 32] bf16 tensor; each warp streams spans
-// of 32 blocks (2 KB) into its own ring of shared-memory stages with TMA (64-byte
-// swizzle: 16-byte chunk q of row r sits at chunk q ^ ((r >> 1) & 3), so the lanes'
-// 16-byte reads of their own rows are free of bank conflicts).
+// with the _rn intrinsics so the compiler cannot fuse them.  A value t thus differs from
+// the exact transform by at most about (log2 kB + 4) u sum_i |x_i mul_i| / sqrt kB
+// (u = 2^-24), and its code is the exact transform's wherever that lies farther than
+// this from an MX rounding boundary.
+// Layout for kB = 32: one lane per 32-element MX block; the 32-point transform, the
+// block's abs-max and its scale byte stay in the lane.  Input: x seen as a [n_blocks, 32]
+// bf16 tensor; each warp streams spans of 32 blocks (2 KB) into its own ring of
+// shared-memory stages with TMA (64-byte swizzle: 16-byte chunk q of row r sits at chunk
+// q ^ ((r >> 1) & 3), so the lanes' 16-byte reads of their own rows are free of bank
+// conflicts).  kB = 128 has a kernel of its own below.
 
 // threads of the transform quantizer's CTAs: 4 warps, 5 CTAs an SM
 constexpr int kTThreads = 128;
@@ -339,13 +340,12 @@ constexpr uint64_t kTWaitNs = 1000000000ull;
 
 __device__ uint32_t g_quant_status;
 
-template <int FMT, int kB>
+template <int FMT>
 __global__ void __launch_bounds__(kTThreads, 5) quantize_transform_kernel(
     const __grid_constant__ CUtensorMap map_x, uint32_t n_blocks, uint32_t KB, uint64_t kb_magic, uint32_t atoms_k,
     uint32_t rows, const float* __restrict__ mul, float c, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
     uint32_t debug)
 {
-    static_assert(kB == 32 || kB == 128, "rotation block");
     constexpr uint32_t kEmax = FMT == kFmtE4M3 ? 8u : 2u;
     constexpr int kWarps = kTThreads / 32;
     const uint32_t lane = threadIdx.x & 31u;
@@ -439,20 +439,6 @@ __global__ void __launch_bounds__(kTThreads, 5) quantize_transform_kernel(
                     t[k] = __fadd2_rn(a, b);
                     t[k + m] = __ffma2_rn(b, neg1, a);
                 }
-        // butterflies across lanes (kB = 128): h = 32, 64 pair lane ^ 1, lane ^ 2.  The
-        // lane holding v[i] gets v[i] + p, the one holding v[i + h] gets p - v[i + h]: both
-        // are fma(v, sign, p), exact products and one rounding, the IEEE sum or difference.
-#pragma unroll
-        for (uint32_t d = 1; d < kB / 32; d <<= 1) {
-            const float sg = (lane & d) != 0 ? -1.f : 1.f;
-            const float2 sgn = make_float2(sg, sg);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float2 p = make_float2(__shfl_xor_sync(0xFFFFFFFFu, t[k].x, d),
-                                             __shfl_xor_sync(0xFFFFFFFFu, t[k].y, d));
-                t[k] = __ffma2_rn(t[k], sgn, p);
-            }
-        }
         if (!live) continue;
         const uint32_t r = static_cast<uint32_t>(__umul64hi(static_cast<uint64_t>(blk) << 24, kb_magic));
         const uint32_t kb = blk - r * KB;
@@ -512,6 +498,191 @@ __global__ void __launch_bounds__(kTThreads, 5) quantize_transform_kernel(
     const uint32_t n_pad_a = rows * pad_k;
     const uint32_t n_pad = n_pad_a + (rows_p - rows) * kbp;
     for (uint32_t p = blockIdx.x * kTThreads + threadIdx.x; p < n_pad; p += gridDim.x * kTThreads) {
+        uint32_t rr, k;
+        if (p < n_pad_a) {
+            rr = p / pad_k;
+            k = KB + (p - rr * pad_k);
+        } else {
+            const uint32_t q = p - n_pad_a;
+            rr = rows + q / kbp;
+            k = q - (q / kbp) * kbp;
+        }
+        sf[sf_offset(rr, k, atoms_k)] = 0;
+    }
+}
+
+// kB = 128: one lane per rotation block.  The lane holds the block's 128 values (four MX
+// blocks) as 64 register pairs, so all seven butterfly stages stay in the lane and no
+// value crosses lanes.  A warp streams spans of 32 rows x 128 channels -- two TMA boxes
+// of 32 rows x 64 channels with the 128-byte swizzle (16-byte chunk q of row r sits at
+// chunk q ^ (r & 7), so the lanes' reads of their own rows are free of bank conflicts)
+// -- and lane l takes row l; the 128 values take most of a thread's 164 registers, so an
+// SM holds 12 warps (three CTAs of four) with two spans in flight each.  The lanes of a
+// warp share the span's channels, so each multiplier is one warp-uniform load.  The
+// codes of a lane's four MX blocks are 64
+// (E2M1) or 128 (E4M3) contiguous bytes of its row, and its four scale bytes one 32-bit
+// word of the tiled scale layout (k-blocks 4g .. 4g + 3 of a row are adjacent there).
+constexpr int kT128Warps = 4;
+constexpr int kT128Stages = 2;
+constexpr uint32_t kBox128Bytes = 32u * 128u;          // 32 rows x 64 bf16
+constexpr uint32_t kSpan128Bytes = 2u * kBox128Bytes;  // 32 rows x 128 bf16
+constexpr uint32_t kT128Smem = kT128Warps * kT128Stages * kSpan128Bytes + 1024u;  // + alignment slack
+
+template <int FMT>
+__global__ void __launch_bounds__(kT128Warps * 32, 3) quantize_transform128_kernel(
+    const __grid_constant__ CUtensorMap map_x, uint32_t rows, uint32_t K, uint32_t KG, uint32_t n_spans_all,
+    uint32_t atoms_k, const float* __restrict__ mul, float c, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
+    uint32_t debug)
+{
+    constexpr uint32_t kEmax = FMT == kFmtE4M3 ? 8u : 2u;
+    extern __shared__ uint8_t dsm[];
+    __shared__ __align__(8) uint64_t full[kT128Warps][kT128Stages];
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t wid = threadIdx.x >> 5;
+    const uint32_t warp = blockIdx.x * kT128Warps + wid;
+    const uint32_t nwarps = gridDim.x * kT128Warps;
+    // the 128-byte swizzle wants 1024-byte aligned boxes
+    uint8_t* ring = dsm + ((1024u - (smem_u32(dsm) & 1023u)) & 1023u) + wid * (kT128Stages * kSpan128Bytes);
+    // spans of this warp: warp, warp + nwarps, ...; span s covers rows 32 (s / KG) ..
+    // 32 (s / KG) + 31 and channels 128 (s % KG) .. + 127; the one with index i sits in
+    // stage i % kT128Stages, whose barrier completes its (i / kT128Stages)-th phase when
+    // both boxes land
+    const uint32_t n_spans = warp < n_spans_all ? (n_spans_all - warp + nwarps - 1) / nwarps : 0u;
+    if (lane == 0) {
+        for (int st = 0; st < kT128Stages; ++st) mbar_init(&full[wid][st], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    const uint64_t policy = policy_evict_first();
+    auto issue = [&](uint32_t i) {  // lane 0 only
+        const int st = static_cast<int>(i % kT128Stages);
+        const uint32_t s = warp + i * nwarps;
+        const uint32_t rg = s / KG;
+        const int32_t c0 = static_cast<int32_t>((s - rg * KG) * 128u);
+        const int32_t c1 = static_cast<int32_t>(rg * 32u);
+        uint8_t* dst = ring + st * kSpan128Bytes;
+        fence_async_smem();  // the lanes' reads of this stage come before the copy's writes
+        mbar_arrive_expect_tx(&full[wid][st], kSpan128Bytes);
+        tma_load_2d<1>(dst, &map_x, c0, c1, smem_u32(&full[wid][st]), policy);
+        tma_load_2d<1>(dst + kBox128Bytes, &map_x, c0 + 64, c1, smem_u32(&full[wid][st]), policy);
+    };
+    if (lane == 0)
+        for (uint32_t i = 0; i < n_spans && i < static_cast<uint32_t>(kT128Stages); ++i)
+            if (!((debug & 2u) && warp == 0 && i == 0)) issue(i);  // debug bit 1: warp 0's first span never lands
+    const float2 neg1 = make_float2(-1.f, -1.f);
+    const uint32_t sw = lane & 7u;
+    for (uint32_t i = 0; i < n_spans; ++i) {
+        const int st = static_cast<int>(i % kT128Stages);
+        const bool landed = mbar_wait(&full[wid][st], (i / kT128Stages) & 1u, kTWaitNs);
+        if (!__all_sync(0xFFFFFFFFu, landed)) {
+            // a copy never landed: report it, let the copies still in flight finish
+            // (each wait again bounded), and leave
+            if (lane == 0) {
+                atomicCAS(&g_quant_status, 0u, static_cast<uint32_t>(MXQ_ERR_TIMEOUT));
+                const uint32_t issued = min(n_spans, i + static_cast<uint32_t>(kT128Stages));
+                for (uint32_t j = i; j < issued; ++j)
+                    mbar_wait(&full[wid][j % kT128Stages], (j / kT128Stages) & 1u, kTWaitNs);
+            }
+            __syncwarp();
+            return;
+        }
+        const uint32_t s = warp + i * nwarps;
+        const uint32_t rg = s / KG;
+        const uint32_t g = s - rg * KG;
+        const uint8_t* rowp = ring + st * kSpan128Bytes + lane * 128u;
+        const float4* m4 = mul != nullptr ? reinterpret_cast<const float4*>(mul + g * 128u) : nullptr;
+        float2 t[64];  // t[k] holds values 2k and 2k + 1 of the lane's rotation block
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const uint4 v = *reinterpret_cast<const uint4*>(rowp + (q >> 3) * kBox128Bytes +
+                                                            16u * ((static_cast<uint32_t>(q) & 7u) ^ sw));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) t[4 * q + e] = make_float2(lo_f(w[e]), hi_f(w[e]));
+            if (mul != nullptr) {
+                const float4 ma = __ldg(m4 + 2 * q), mb = __ldg(m4 + 2 * q + 1);
+                t[4 * q] = __fmul2_rn(t[4 * q], make_float2(ma.x, ma.y));
+                t[4 * q + 1] = __fmul2_rn(t[4 * q + 1], make_float2(ma.z, ma.w));
+                t[4 * q + 2] = __fmul2_rn(t[4 * q + 2], make_float2(mb.x, mb.y));
+                t[4 * q + 3] = __fmul2_rn(t[4 * q + 3], make_float2(mb.z, mb.w));
+            }
+        }
+        __syncwarp();  // every lane has read the stage before it is refilled
+        if (lane == 0 && i + kT128Stages < n_spans) issue(i + kT128Stages);
+        // butterflies: h = 1 on scalars, h = 2 ... 64 as packed binary32 operations (the
+        // difference as fma(b, -1, a), one rounding, the IEEE difference)
+#pragma unroll
+        for (int k = 0; k < 64; ++k) t[k] = make_float2(__fadd_rn(t[k].x, t[k].y), __fsub_rn(t[k].x, t[k].y));
+#pragma unroll
+        for (int m = 1; m < 64; m <<= 1)
+#pragma unroll
+            for (int k = 0; k < 64; ++k)
+                if ((k & m) == 0) {
+                    const float2 a = t[k], b = t[k + m];
+                    t[k] = __fadd2_rn(a, b);
+                    t[k + m] = __ffma2_rn(b, neg1, a);
+                }
+        const uint32_t row = rg * 32u + lane;
+        if (row >= rows) continue;
+        // each MX block b (values 32b .. 32b + 31, pairs t[16b .. 16b + 15]): scale and
+        // codes as in the 32-point kernel above
+        uint32_t scw = 0;
+        uint32_t cw[FMT == kFmtE2M1 ? 16 : 32];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            float2* tb = t + 16 * b;
+            float mc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(mc[k & 3]) : "f"(mc[k & 3]), "f"(tb[k].x), "f"(tb[k].y));
+            float m;
+            asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(mc[0]), "f"(mc[1]), "f"(mc[2]));
+            asm("max.NaN.f32 %0, %1, %2;" : "=f"(m) : "f"(m), "f"(mc[3]));
+            const uint32_t eb = (__float_as_uint(__fmul_rn(m, c)) & 0x7FFFFFFFu) >> 23;
+            const uint32_t sc = eb == 255u ? 255u : (eb > kEmax ? eb - kEmax : 0u);
+            float mult = e8m0_inverse(sc);
+            const uint32_t keep = sc == 255u ? 0u : 0xFFFFFFFFu;
+            if (sc - 11u <= 249u - 11u) {
+                mult = __fmul_rn(c, mult);
+            } else {
+                const float2 c2 = make_float2(c, c);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) tb[k] = __fmul2_rn(tb[k], c2);
+            }
+            const float2 mult2 = make_float2(mult, mult);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) tb[k] = __fmul2_rn(tb[k], mult2);
+            if (FMT == kFmtE2M1) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float q[8] = {tb[4 * k].x,     tb[4 * k].y,     tb[4 * k + 1].x, tb[4 * k + 1].y,
+                                        tb[4 * k + 2].x, tb[4 * k + 2].y, tb[4 * k + 3].x, tb[4 * k + 3].y};
+                    cw[4 * b + k] = cvt_e2m1x8(q) & keep;
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    cw[8 * b + k] = (cvt_e4m3x2(tb[2 * k].x, tb[2 * k].y) |
+                                     (cvt_e4m3x2(tb[2 * k + 1].x, tb[2 * k + 1].y) << 16)) & keep;
+            }
+            scw |= sc << (8 * b);
+        }
+        constexpr uint32_t kCodeBytes = FMT == kFmtE2M1 ? 64u : 128u;  // per rotation block
+        uint4* dst = reinterpret_cast<uint4*>(codes + static_cast<size_t>(row) * (K / (FMT == kFmtE2M1 ? 2u : 1u)) +
+                                              static_cast<size_t>(g) * kCodeBytes);
+#pragma unroll
+        for (int k = 0; k < static_cast<int>(kCodeBytes / 16u); ++k)
+            __stcs(dst + k, make_uint4(cw[4 * k], cw[4 * k + 1], cw[4 * k + 2], cw[4 * k + 3]));
+        *reinterpret_cast<uint32_t*>(sf + sf_offset(row, 4u * g, atoms_k)) = scw;
+    }
+    // the padding of the tiled scale buffer, as in quantize_kernel
+    const uint32_t KB = K / 32u;
+    const uint32_t kbp = atoms_k * 4u;
+    const uint32_t pad_k = kbp - KB;
+    const uint32_t rows_p = (rows + 127u) & ~127u;
+    const uint32_t n_pad_a = rows * pad_k;
+    const uint32_t n_pad = n_pad_a + (rows_p - rows) * kbp;
+    for (uint32_t p = blockIdx.x * blockDim.x + threadIdx.x; p < n_pad; p += gridDim.x * blockDim.x) {
         uint32_t rr, k;
         if (p < n_pad_a) {
             rr = p / pad_k;
@@ -587,6 +758,37 @@ cudaError_t launch_quantize_transform(const void* x, int64_t rows, int64_t K, in
     const uint32_t n_blocks = static_cast<uint32_t>(rows * K / 32);
     const uint32_t KB = static_cast<uint32_t>(K / 32);
     const uint32_t atoms_k = static_cast<uint32_t>(sf_atoms_k(K));
+    uint8_t* c = static_cast<uint8_t*>(codes);
+    uint8_t* f = static_cast<uint8_t*>(sf);
+    const uint32_t r = static_cast<uint32_t>(rows);
+    const uint32_t dbg = debug_flags();
+    CUtensorMap map;
+    if (n_blocks == 0) return cudaSuccess;
+    if (block == 128) {
+        // x as [rows, K] bf16, boxes of 32 rows x 64 channels, 128-byte swizzle; rows past
+        // the end read as zeros
+        const uint32_t KG = static_cast<uint32_t>(K / 128);
+        const uint32_t n_spans = static_cast<uint32_t>(ceil_div(rows, 32)) * KG;
+        if (!make_map_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(K),
+                         static_cast<uint64_t>(rows), static_cast<uint64_t>(K) * 2u, 64, 32,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        const int64_t want = ceil_div(n_spans, kT128Warps);
+        const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * 3)));
+        const uint32_t k32 = static_cast<uint32_t>(K);
+        if (fmt == kFmtE4M3) {
+            auto kern = quantize_transform128_kernel<kFmtE4M3>;
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kT128Smem);
+            if (e != cudaSuccess) return e;
+            kern<<<grid, kT128Warps * 32, kT128Smem, stream>>>(map, r, k32, KG, n_spans, atoms_k, mul, norm, c, f, dbg);
+        } else {
+            auto kern = quantize_transform128_kernel<kFmtE2M1>;
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kT128Smem);
+            if (e != cudaSuccess) return e;
+            kern<<<grid, kT128Warps * 32, kT128Smem, stream>>>(map, r, k32, KG, n_spans, atoms_k, mul, norm, c, f, dbg);
+        }
+        return cudaGetLastError();
+    }
     const int64_t want = ceil_div(n_blocks, kTThreads);  // CTAs for one span per warp
     int64_t grid64 = std::max<int64_t>(1, std::min<int64_t>(want, num_sms() * 32));
     if (mul != nullptr && grid64 < want) {
@@ -599,31 +801,16 @@ cudaError_t launch_quantize_transform(const void* x, int64_t rows, int64_t K, in
     const int grid = static_cast<int>(grid64);
     // x as n_blocks rows of 32 bf16 (64 bytes), boxes of 32 rows, 64-byte swizzle; rows
     // past the end read as zeros
-    CUtensorMap map;
-    if (n_blocks == 0) return cudaSuccess;
     if (!make_map_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, 32, n_blocks, 64, 32, 32,
                      CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     const uint64_t kb_magic = ((uint64_t(1) << 40) + KB - 1) / KB;
-    uint8_t* c = static_cast<uint8_t*>(codes);
-    uint8_t* f = static_cast<uint8_t*>(sf);
-    const uint32_t r = static_cast<uint32_t>(rows);
-    const uint32_t dbg = debug_flags();
-    if (fmt == kFmtE4M3) {
-        if (block == 128)
-            quantize_transform_kernel<kFmtE4M3, 128><<<grid, kTThreads, 0, stream>>>(map, n_blocks, KB, kb_magic, atoms_k,
-                                                                                    r, mul, norm, c, f, dbg);
-        else
-            quantize_transform_kernel<kFmtE4M3, 32><<<grid, kTThreads, 0, stream>>>(map, n_blocks, KB, kb_magic, atoms_k,
-                                                                                   r, mul, norm, c, f, dbg);
-    } else {
-        if (block == 128)
-            quantize_transform_kernel<kFmtE2M1, 128><<<grid, kTThreads, 0, stream>>>(map, n_blocks, KB, kb_magic, atoms_k,
-                                                                                    r, mul, norm, c, f, dbg);
-        else
-            quantize_transform_kernel<kFmtE2M1, 32><<<grid, kTThreads, 0, stream>>>(map, n_blocks, KB, kb_magic, atoms_k,
-                                                                                   r, mul, norm, c, f, dbg);
-    }
+    if (fmt == kFmtE4M3)
+        quantize_transform_kernel<kFmtE4M3><<<grid, kTThreads, 0, stream>>>(map, n_blocks, KB, kb_magic, atoms_k, r,
+                                                                               mul, norm, c, f, dbg);
+    else
+        quantize_transform_kernel<kFmtE2M1><<<grid, kTThreads, 0, stream>>>(map, n_blocks, KB, kb_magic, atoms_k, r,
+                                                                               mul, norm, c, f, dbg);
     return cudaGetLastError();
 }
 
