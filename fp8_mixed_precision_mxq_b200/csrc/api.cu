@@ -359,14 +359,46 @@ int64_t mxq_block_workspace_bytes(const mxq_wdesc* w, const int64_t* M_in, uint3
 
 namespace {
 
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique ID of the calling thread's current CUDA context (the runtime's primary context
+// of the current device once it has been initialized), through the driver entry points
+// the runtime exposes; false if the driver lacks them.
+bool current_context_id(unsigned long long* id)
+{
+    static PfnCtxGetCurrent get_current = nullptr;
+    static PfnCtxGetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PfnCtxGetCurrent>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PfnCtxGetId>(p);
+    });
+    if (!get_current || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 // The stream and events the block entry point uses to quantize the next linears' inputs
 // while the GEMMs run: one stream (non-blocking) and nine events per device, created on
-// first use and kept until the process exits.  The enqueue sequence that uses them holds
-// g_side_mu, so calls from several host threads cannot interleave their records and waits.
+// first use in each CUDA context (a device reset ends the old context and its handles, and
+// the next call creates new ones) and kept until the process exits.  The enqueue sequence
+// that uses them holds g_side_mu, so calls from several host threads cannot interleave
+// their records and waits.
 constexpr int kSideMaxDevices = 64;
 struct SideStream {
     cudaStream_t s = nullptr;
     cudaEvent_t ev[9] = {};
+    unsigned long long ctx_id = 0;
+    bool have_id = false;
 };
 SideStream g_side[kSideMaxDevices];
 std::mutex g_side_mu;
@@ -378,13 +410,19 @@ int side_stream(SideStream** out)
     if (e != cudaSuccess) return fail(MXQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
     if (dev < 0 || dev >= kSideMaxDevices) return fail(MXQ_ERR_UNSUPPORTED, "device index %d is too large", dev);
     SideStream& sd = g_side[dev];
-    if (!sd.s) {
+    unsigned long long id = 0;
+    const bool have_id = current_context_id(&id);
+    if (!sd.s || sd.have_id != have_id || (have_id && sd.ctx_id != id)) {
+        // first use in this context: the handles of an earlier context died with it
+        sd.s = nullptr;
         e = cudaStreamCreateWithFlags(&sd.s, cudaStreamNonBlocking);
         for (int i = 0; i < 9 && e == cudaSuccess; ++i) e = cudaEventCreateWithFlags(&sd.ev[i], cudaEventDisableTiming);
         if (e != cudaSuccess) {
             sd.s = nullptr;
             return fail(MXQ_ERR_CUDA, "creating the block's side stream: %s", cudaGetErrorString(e));
         }
+        sd.ctx_id = id;
+        sd.have_id = have_id;
     }
     *out = &sd;
     return MXQ_OK;
@@ -826,34 +864,6 @@ struct NoAllocSlot {
 };
 NoAllocSlot g_noalloc[kNoAllocMaxDevices];
 std::mutex g_noalloc_mu;
-
-using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
-using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
-
-// Unique ID of the calling thread's current CUDA context (the runtime's primary context
-// of the current device once it has been initialized), through the driver entry points
-// the runtime exposes; false if the driver lacks them.
-bool current_context_id(unsigned long long* id)
-{
-    static PfnCtxGetCurrent get_current = nullptr;
-    static PfnCtxGetId get_id = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_current = reinterpret_cast<PfnCtxGetCurrent>(p);
-        p = nullptr;
-        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            get_id = reinterpret_cast<PfnCtxGetId>(p);
-    });
-    if (!get_current || !get_id) return false;
-    CUcontext ctx = nullptr;
-    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
-    return get_id(ctx, id) == CUDA_SUCCESS;
-}
 
 // Device address of the scratch array in the current device's context.  In host code the
 // array's name is only a stand-in, so the address is looked up (with that device current)

@@ -554,12 +554,26 @@ __global__ void __launch_bounds__(kT128Warps * 32, 3) quantize_transform128_kern
     }
     __syncwarp();
     const uint64_t policy = policy_evict_first();
-    auto issue = [&](uint32_t i) {  // lane 0 only
+    // spans are visited in order, so their (row group, channel group) pairs are stepped by
+    // nwarps = d_rg KG + d_g instead of divided out: p_ for the next span to load (lane 0),
+    // c_ for the next one to quantize
+    const uint32_t d_rg = nwarps / KG, d_g = nwarps - d_rg * KG;
+    auto advance = [&](uint32_t& rg, uint32_t& g) {
+        g += d_g;
+        rg += d_rg;
+        if (g >= KG) {
+            g -= KG;
+            ++rg;
+        }
+    };
+    uint32_t p_rg = warp / KG, p_g = warp - (warp / KG) * KG;
+    uint32_t c_rg = p_rg, c_g = p_g;
+    auto issue = [&](uint32_t i, bool skip) {  // lane 0 only, spans in order
         const int st = static_cast<int>(i % kT128Stages);
-        const uint32_t s = warp + i * nwarps;
-        const uint32_t rg = s / KG;
-        const int32_t c0 = static_cast<int32_t>((s - rg * KG) * 128u);
-        const int32_t c1 = static_cast<int32_t>(rg * 32u);
+        const int32_t c0 = static_cast<int32_t>(p_g * 128u);
+        const int32_t c1 = static_cast<int32_t>(p_rg * 32u);
+        advance(p_rg, p_g);
+        if (skip) return;
         uint8_t* dst = ring + st * kSpan128Bytes;
         fence_async_smem();  // the lanes' reads of this stage come before the copy's writes
         mbar_arrive_expect_tx(&full[wid][st], kSpan128Bytes);
@@ -568,7 +582,7 @@ __global__ void __launch_bounds__(kT128Warps * 32, 3) quantize_transform128_kern
     };
     if (lane == 0)
         for (uint32_t i = 0; i < n_spans && i < static_cast<uint32_t>(kT128Stages); ++i)
-            if (!((debug & 2u) && warp == 0 && i == 0)) issue(i);  // debug bit 1: warp 0's first span never lands
+            issue(i, (debug & 2u) && warp == 0 && i == 0);  // debug bit 1: warp 0's first span never lands
     const float2 neg1 = make_float2(-1.f, -1.f);
     const uint32_t sw = lane & 7u;
     for (uint32_t i = 0; i < n_spans; ++i) {
@@ -586,9 +600,8 @@ __global__ void __launch_bounds__(kT128Warps * 32, 3) quantize_transform128_kern
             __syncwarp();
             return;
         }
-        const uint32_t s = warp + i * nwarps;
-        const uint32_t rg = s / KG;
-        const uint32_t g = s - rg * KG;
+        const uint32_t rg = c_rg, g = c_g;
+        advance(c_rg, c_g);
         const uint8_t* rowp = ring + st * kSpan128Bytes + lane * 128u;
         const float4* m4 = mul != nullptr ? reinterpret_cast<const float4*>(mul + g * 128u) : nullptr;
         float2 t[64];  // t[k] holds values 2k and 2k + 1 of the lane's rotation block
@@ -608,7 +621,7 @@ __global__ void __launch_bounds__(kT128Warps * 32, 3) quantize_transform128_kern
             }
         }
         __syncwarp();  // every lane has read the stage before it is refilled
-        if (lane == 0 && i + kT128Stages < n_spans) issue(i + kT128Stages);
+        if (lane == 0 && i + kT128Stages < n_spans) issue(i + kT128Stages, false);
         // butterflies: h = 1 on scalars, h = 2 ... 64 as packed binary32 operations (the
         // difference as fma(b, -1, a), one rounding, the IEEE difference)
 #pragma unroll

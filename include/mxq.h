@@ -159,7 +159,8 @@ int mxq_dit_block_linears(const mxq_wdesc* w, const void* const* x_in, const int
  * accepts (one linear's workspace, reused; the linears then run one after another).
  * mxq_block_workspace_bytes: in NATIVE mode, a quantized-activation buffer for every
  * linear; with a workspace of at least this size the call quantizes all eight inputs on
- * a stream of the library's own (created once per device, with its events, on first use)
+ * a stream of the library's own (created with its events on first use in each CUDA
+ * context of a device, so a device reset is followed by new ones)
  * while the GEMMs run on `stream`, each GEMM waiting only for its own input.  When
  * `stream` has passed the call, all of its work is done.  In QDQ mode both sizes are the
  * same. */
