@@ -70,8 +70,8 @@ GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precisio
                 "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h", "fp8_mixed_precision_mxq_b200/csrc/mx_elem.cuh"]
 GEMM_TRAFFIC = {
     ("ffn_up_720p_w4a4", 75600): {
-        "bytes": 854573568 + 2047664128,
-        "sources_sha256": "efdee61c67b6699c132e7ecc24ff8382e0e3745a06aa0d2fe4f087f9c46b6410"},
+        "bytes": 696092672 + 2052435456,
+        "sources_sha256": "65a7396b88df2a5f060fae480e333757c88e7f8db5c6b3d12586c6a0e4fb9018"},
 }
 
 

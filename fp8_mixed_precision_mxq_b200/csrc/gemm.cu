@@ -117,7 +117,7 @@ struct Cfg {
     static constexpr uint32_t kOffBar = kOffQ + (kOut ? kEpiWarps * 2 * kQBuf : 0u);
     static constexpr uint32_t kNumBars = 2 * kStages + 6 + 2 * kSfBufs;
     static constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16;
-    static constexpr int kGroupM = 16;  // tile rows (tiles along M) per rasterization group
+    static constexpr int kGroupM = 32;  // tile rows (tiles along M) per rasterization group
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kOffB % 1024 == 0 && kOffSFA % 1024 == 0 && kOffEpi % 1024 == 0, "alignment");
 };
