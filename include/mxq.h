@@ -267,8 +267,11 @@ int mxq_absmax(const void* x_bf16, int64_t n, void* out_f32, void* stream);
  *     H the Sylvester Hadamard matrix (entries +-1), as a fast Walsh-Hadamard transform in
  *     binary32 (butterflies (a, b) -> (a + b, a - b), h = 1, 2, 4, ..., then the scaling);
  *   t MX-quantized in fmt as by mxq_quantize_act (scale from the block's binary32 abs-max).
- * mul: NULL or K floats on the device, 16-byte aligned.  Requires K % block == 0.  Other
- * arguments and errors as for mxq_quantize_act. */
+ * Each t thus differs from the exact transform (x . diag(mul) . H_block / sqrt(block)) by at
+ * most about (log2(block) + 4) 2^-24 sum_i |x_i mul_i| / sqrt(block), and the codes and
+ * scales are the exact transform's wherever it lies farther than that from an MX rounding
+ * boundary.  mul: NULL or K floats on the device, 16-byte aligned.  Requires
+ * K % block == 0.  Other arguments and errors as for mxq_quantize_act. */
 int mxq_quantize_act_transformed(const void* x_bf16, int64_t M, int64_t K, int fmt, const float* mul, int block,
                                  void* codes, void* sf, void* stream);
 
