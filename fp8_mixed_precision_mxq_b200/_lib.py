@@ -58,6 +58,7 @@ SIGNATURES = {
     "mxq_linear_noalloc_max_scratch_bytes": ([], _i64),
     "mxq_gemm_gelu_quant": ([_vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp], _i32),
     "mxq_gemm_quant": ([_vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _i32, _i32, _vp, _vp, _vp, _vp], _i32),
+    "mxq_gelu_bf16": ([_vp, _i64, _vp, _vp], _i32),
     "mxq_ffn": ([_vp, _i64, _i64, ctypes.POINTER(WDesc), ctypes.POINTER(WDesc), _i32, _i32, _vp, _i64, _vp, _vp],
                 _i32),
     "mxq_ffn_workspace_bytes": ([_i64, _i64, _i64, _i32, _i32], _i64),

@@ -735,6 +735,15 @@ int mxq_absmax(const void* x_bf16, int64_t n, void* out_f32, void* stream)
                    "absmax launch");
 }
 
+int mxq_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream)
+{
+    if (n <= 0) return fail(MXQ_ERR_INVALID_ARG, "gelu_bf16: n=%lld must be positive", (long long)n);
+    RETURN_IF(check_ptr(x_bf16, "x", 2));
+    RETURN_IF(check_ptr(y_bf16, "y", 2));
+    RETURN_IF(check_device());
+    return cuda_rc(launch_gelu_bf16(x_bf16, n, y_bf16, static_cast<cudaStream_t>(stream)), "gelu launch");
+}
+
 int mxq_channel_absmax(const void* x_bf16, int64_t rows, int64_t K, float* out_f32, void* stream)
 {
     if (rows <= 0 || K <= 0) return fail(MXQ_ERR_INVALID_ARG, "channel_absmax: sizes must be positive");

@@ -112,9 +112,13 @@ struct Cfg {
     static constexpr uint32_t kOffSFB = kOffSFA + kStages * kStageSFA;
     static constexpr uint32_t kOffEpi = kOffSFB + kStages * kStageSFB;
     static constexpr uint32_t kQBuf = kOut == kOutGeluE4M3 ? 32 * 32 : 32 * 16;  // 32 rows of one block's codes
+    // code staging buffers per warp: two, or one for E4M3, whose larger codes would
+    // otherwise leave no room for the GELU table
+    static constexpr int kQBufs = kOut == kOutGeluE4M3 ? 1 : 2;
     static constexpr int kEpiWarps = kEpiWarpsOf<kOut>;
     static constexpr uint32_t kOffQ = kOffEpi + kEpiWarps * 2 * kEpiBuf;
-    static constexpr uint32_t kOffBar = kOffQ + (kOut ? kEpiWarps * 2 * kQBuf : 0u);
+    static constexpr uint32_t kOffLut = kOffQ + (kOut ? kEpiWarps * kQBufs * kQBuf : 0u);  // GELU table
+    static constexpr uint32_t kOffBar = kOffLut + (kOut ? kGeluTableBytes : 0u);
     static constexpr uint32_t kNumBars = 2 * kStages + 6 + 2 * kSfBufs;
     static constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16;
     static constexpr int kGroupM = 32;  // tile rows (tiles along M) per rasterization group
@@ -141,33 +145,6 @@ struct Params {
 };
 
 __device__ __forceinline__ void record_status(uint32_t code) { atomicCAS(&g_device_status, 0u, code); }
-
-// GELU(x) = x * Phi(x) = x/2 * erfc(-x / sqrt 2) in fp32 (the plain erf form).  erfc(z)
-// for z >= 0 by the Chebyshev-fitted formula of Numerical Recipes (2nd ed., section 6.2,
-// "erfcc"): erfc(z) = t * exp(-z^2 + P(t)), t = 1 / (1 + z/2), P of degree 9, fractional
-// error below 1.2e-7; the other side from erfc(-z) = 2 - erfc(z).  Relative accuracy
-// holds in the negative tail, where GELU is tiny (1 + erf would cancel there).  Below
-// x of about -13 the exponential underflows and the result is -0.
-// Two values at a time: the multiplies and fused multiply-adds run packed (each half
-// rounded as the scalar operation would be), the reciprocal and the exponential scalar.
-__device__ __forceinline__ float2 gelu2_f32(float2 x)
-{
-    const float2 one = make_float2(1.0f, 1.0f), half = make_float2(0.5f, 0.5f);
-    const float2 z = __fmul2_rn(make_float2(fabsf(x.x), fabsf(x.y)),
-                                make_float2(0.70710678118654752f, 0.70710678118654752f));
-    const float2 d = __ffma2_rn(half, z, one);
-    const float2 t = make_float2(__fdividef(1.0f, d.x), __fdividef(1.0f, d.y));
-    const float c[10] = {0.17087277f, -0.82215223f, 1.48851587f, -1.13520398f, 0.27886807f,
-                         -0.18628806f, 0.09678418f, 0.37409196f, 1.00002368f, -1.26551223f};
-    float2 q = make_float2(c[0], c[0]);
-#pragma unroll
-    for (int i = 1; i < 10; ++i) q = __ffma2_rn(q, t, make_float2(c[i], c[i]));
-    const float2 a = __ffma2_rn(make_float2(-z.x, -z.y), z, q);
-    const float2 e = __fmul2_rn(t, make_float2(__expf(a.x), __expf(a.y)));  // erfc(z)
-    const float2 lo = __fmul2_rn(half, e), hi = __ffma2_rn(make_float2(-0.5f, -0.5f), e, one);
-    const float2 phi = make_float2(x.x <= 0.0f ? lo.x : hi.x, x.y <= 0.0f ? lo.y : hi.y);
-    return __fmul2_rn(x, phi);
-}
 
 template <int kGroupM>
 __device__ __forceinline__ void tile_coords(int t, int m_blocks, int n_blocks, int& mb, int& nb)
@@ -447,7 +424,14 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         const uint32_t lanes = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
         uint8_t* ebuf0 = smem + C::kOffEpi + ew * 2 * kEpiBuf;
-        uint8_t* qbuf0 = smem + C::kOffQ + ew * 2 * C::kQBuf;
+        uint8_t* qbuf0 = smem + C::kOffQ + ew * C::kQBufs * C::kQBuf;
+        const uint16_t* lut = reinterpret_cast<const uint16_t*>(smem + C::kOffLut);
+        if constexpr (kOut != kOutBf16) {
+            // the GELU table, built by the epilogue warps while the first tile's MMAs run
+            if (p.gelu)
+                gelu_table_fill(reinterpret_cast<uint16_t*>(smem + C::kOffLut), threadIdx.x - 64u, kEpiWarps * 32u);
+            named_bar_sync(1, kEpiWarps * 32);
+        }
         const uint32_t bar_overlap = kPair == 2 ? mapa_shared(smem_u32(overlap_free), 0) : smem_u32(overlap_free);
         const bool has_bias = p.bias != nullptr;
         int eb = 0;
@@ -519,11 +503,11 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                                 make_float2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1])), alpha2,
                                 make_float2(lo_f(bw[i]), hi_f(bw[i])));
                             __nv_bfloat162 y2 = __floats2bfloat162_rn(y.x, y.y);
-                            if constexpr (decltype(gelu)::value) {
-                                const float2 g = gelu2_f32(make_float2(__low2float(y2), __high2float(y2)));
-                                y2 = __floats2bfloat162_rn(g.x, g.y);
-                            }
-                            o[i] = *reinterpret_cast<uint32_t*>(&y2);
+                            const uint32_t w = *reinterpret_cast<uint32_t*>(&y2);
+                            if constexpr (decltype(gelu)::value)
+                                o[i] = gelu_bf16_bits(w & 0xFFFFu, lut) | (gelu_bf16_bits(w >> 16, lut) << 16);
+                            else
+                                o[i] = w;
                         }
                     };
                     if (kOut != kOutBf16 && p.gelu)
@@ -532,7 +516,13 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                         chunk_out(std::false_type{});
                     const bool store_y = kOut == kOutBf16 || p.write_h;
                     uint8_t* buf = ebuf0 + eb * kEpiBuf;
-                    if (lane == 0) bulk_wait_read<1>();  // the stores that last used buf have read it
+                    // the stores that last used this chunk's buffers have read them
+                    if (lane == 0) {
+                        if constexpr (C::kQBufs == 1)
+                            bulk_wait_read<0>();
+                        else
+                            bulk_wait_read<1>();
+                    }
                     __syncwarp();
                     if (store_y) {
                         const uint32_t rsw = (static_cast<uint32_t>(lane) >> 1) & 3u;
@@ -553,7 +543,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                         const uint32_t sc = e8m0_code<kEmax>(m2);
                         const float inv = e8m0_inverse(sc);
                         const uint32_t keep = sc == 255u ? 0u : 0xFFFFFFFFu;  // a non-finite block: codes 0
-                        uint8_t* qb = qbuf0 + eb * C::kQBuf;
+                        uint8_t* qb = qbuf0 + (C::kQBufs == 2 ? eb : 0) * C::kQBuf;
                         if constexpr (kOut == kOutGeluE2M1) {
                             uint32_t cw[4];
                             const float2 inv2 = make_float2(inv, inv);
@@ -588,7 +578,8 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                     if (lane == 0) {
                         if (store_y) tma_store_2d(&map_y, buf, n, row0, pol_y);
                         if constexpr (kOut != kOutBf16)
-                            tma_store_2d(&map_q, qbuf0 + eb * C::kQBuf, kOut == kOutGeluE2M1 ? n / 2 : n, row0,
+                            tma_store_2d(&map_q, qbuf0 + (C::kQBufs == 2 ? eb : 0) * C::kQBuf,
+                                         kOut == kOutGeluE2M1 ? n / 2 : n, row0,
                                          pol_y);
                         bulk_commit();
                     }

@@ -1,9 +1,11 @@
 // mx_elem.cuh -- device helpers of the MX element formats shared by the quantizer and
 // the GEMM epilogue that quantizes its output: packed bf16 abs-max, the E8M0 scale of a
 // block, and the hardware conversions to E2M1 / E4M3 (round to nearest even,
-// saturating, sign of a zero result kept).
+// saturating, sign of a zero result kept); and the exact bf16 GELU of the fused FFN
+// epilogue (a shared-memory table and closed forms).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace mxq {
@@ -60,6 +62,56 @@ __device__ __forceinline__ uint32_t e8m0_code(uint32_t amax_bits)
 __device__ __forceinline__ float e8m0_inverse(uint32_t code)
 {
     return __uint_as_float((254u - min(code, 253u)) << 23);
+}
+
+// ---- GELU of bf16 values ---------------------------------------------------------------
+// h = bf16(GELU(x)) for a bf16 x, GELU(x) = x/2 erfc(-x / sqrt 2) (the plain erf form) rounded
+// once to bf16, nearest with ties to even: what a bf16 network's GELU gives when computed
+// exactly.  For 2^-10 <= |x| < 16 (14 binades of 128 significands, both signs: 3584 values)
+// the result comes from a table that the kernel using it builds in shared memory from the
+// fp64 erfc.  Elsewhere it has a closed form: below 2^-10 it is x/2 rounded to bf16 (the
+// next term, x^2 / sqrt(2 pi), moves x/2 by less than 0.8 |x| of itself, which is under half
+// a bf16 unit); from 16 up it is x (1 - Phi(16) < 2^-190); from -16 down it is -0 (below the
+// smallest bf16 magnitude); +Inf gives +Inf, -Inf and NaN give NaN (0x7FC0).
+constexpr uint32_t kGeluLo = 0x3A80u;                 // bf16 magnitude bits of 2^-10
+constexpr uint32_t kGeluSpan = 14u * 128u;            // magnitudes 2^-10 ... 16 (exclusive)
+constexpr uint32_t kGeluEntries = 2u * kGeluSpan;     // positive, then negative
+constexpr uint32_t kGeluTableBytes = 2u * kGeluEntries;
+
+// Entry i of the table: bf16 bits of GELU of the bf16 value with sign i / kGeluSpan and
+// magnitude bits kGeluLo + i % kGeluSpan.  The fp64 GELU is rounded to 8 significant bits
+// (to a multiple of 2^-133 below 2^-126, bf16's subnormal step) with rint, then read as
+// bf16: one rounding.
+__device__ __forceinline__ uint16_t gelu_table_value(uint32_t i)
+{
+    const uint32_t b = ((i / kGeluSpan) << 15) | (kGeluLo + i % kGeluSpan);
+    const double x = static_cast<double>(__uint_as_float(b << 16));
+    const double g = 0.5 * x * erfc(-x / sqrt(2.0));
+    int e = 0;
+    frexp(g, &e);  // |g| in [2^(e-1), 2^e)
+    const double ulp = ldexp(1.0, max(e - 8, -133));
+    const double r = rint(g / ulp) * ulp;
+    return static_cast<uint16_t>(__float_as_uint(static_cast<float>(r)) >> 16);
+}
+
+// Threads tid, tid + nthreads, ... fill their entries of the shared-memory table.
+__device__ __forceinline__ void gelu_table_fill(uint16_t* lut, uint32_t tid, uint32_t nthreads)
+{
+    for (uint32_t i = tid; i < kGeluEntries; i += nthreads) lut[i] = gelu_table_value(i);
+}
+
+// GELU of one bf16 value (bits b, low 16 bits) through the table.
+__device__ __forceinline__ uint32_t gelu_bf16_bits(uint32_t b, const uint16_t* lut)
+{
+    const uint32_t m = b & 0x7FFFu;
+    const uint32_t neg = b >> 15;
+    const uint32_t idx = m - kGeluLo;
+    const bool in = idx < kGeluSpan;
+    const uint32_t t = lut[in ? neg * kGeluSpan + idx : 0u];
+    const uint32_t half = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(b << 16) * 0.5f));
+    uint32_t big = neg ? 0x8000u : b;
+    if (m >= 0x7F80u) big = (m == 0x7F80u && !neg) ? b : 0x7FC0u;
+    return in ? t : (m < kGeluLo ? half : big);
 }
 
 }  // namespace mxq

@@ -31,6 +31,7 @@ cudaError_t launch_quantize_transform(const void* x, int64_t rows, int64_t K, in
                                       float norm, void* codes, void* sf, cudaStream_t stream);
 // *out = max |x| over n bf16 values (n % 8 == 0), as fp32.
 cudaError_t launch_absmax(const void* x, int64_t n, float* out, cudaStream_t stream);
+cudaError_t launch_gelu_bf16(const void* x, int64_t n, void* y, cudaStream_t stream);
 cudaError_t launch_dequantize(const void* codes, const void* sf, int64_t rows, int64_t K, int fmt, void* out,
                               cudaStream_t stream);
 // Calibration and load-time arithmetic of the policy (calib.cu).

@@ -182,6 +182,12 @@ __device__ __forceinline__ void bulk_wait()
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA store).
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// Named barrier `id` (1 ... 15) over `threads` threads of the CTA (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor cores
 // ---------------------------------------------------------------------------

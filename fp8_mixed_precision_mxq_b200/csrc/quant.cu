@@ -892,6 +892,30 @@ __global__ void __launch_bounds__(kThreads) absmax_kernel(const uint4* __restric
 
 }  // namespace
 
+namespace {
+
+// GELU of bf16 values, elementwise, through the same table as the fused FFN epilogue: each
+// CTA builds the table in shared memory, then maps its share of the elements.
+__global__ void __launch_bounds__(256) gelu_bf16_kernel(const uint16_t* __restrict__ x, int64_t n,
+                                                       uint16_t* __restrict__ y)
+{
+    __shared__ uint16_t lut[kGeluEntries];
+    gelu_table_fill(lut, threadIdx.x, blockDim.x);
+    __syncthreads();
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        y[i] = static_cast<uint16_t>(gelu_bf16_bits(x[i], lut));
+}
+
+}  // namespace
+
+cudaError_t launch_gelu_bf16(const void* x, int64_t n, void* y, cudaStream_t stream)
+{
+    const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(n, 256), num_sms() * 4)));
+    gelu_bf16_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(x), n, static_cast<uint16_t*>(y));
+    return cudaGetLastError();
+}
+
 cudaError_t launch_absmax(const void* x, int64_t n, float* out, cudaStream_t stream)
 {
     cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float), stream);

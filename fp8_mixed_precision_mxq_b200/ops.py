@@ -192,6 +192,18 @@ def gemm_quant(a_codes, a_sf, fmt, M: int, K: int, w: QWeight, act="none", out_f
     return codes, sf
 
 
+def gelu_bf16(x: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """GELU of bf16 values as the quantizing epilogue applies it (exact, rounded once to bf16)."""
+    _cuda_bf16(x, "x")
+    if out is None:
+        out = torch.empty_like(x)
+    _cuda_bf16(out, "out")
+    if out.numel() != x.numel():
+        raise ValueError("out must have as many elements as x")
+    check(_lib.lib().mxq_gelu_bf16(_p(x), x.numel(), _p(out), _stream(stream)), "mxq_gelu_bf16")
+    return out
+
+
 def ffn_workspace_bytes(M: int, K: int, H: int, up_fmt="e2m1", down_fmt="e2m1") -> int:
     return int(_lib.lib().mxq_ffn_workspace_bytes(M, K, H, _fmt(up_fmt), _fmt(down_fmt)))
 

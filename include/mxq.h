@@ -194,7 +194,8 @@ int64_t mxq_linear_noalloc_max_scratch_bytes(void);
 /* GEMM whose epilogue produces the next layer's MX-quantized input: the FFN's first
  * linear followed by its GELU, with the hidden activation never written in bf16.
  *   y = acc + bias (fp32) rounded to bf16 (the linear's output type);
- *   h = GELU(y) = y * Phi(y) (the plain erf form, in fp32) rounded to bf16;
+ *   h = GELU(y) = y * Phi(y) (the plain erf form) rounded to bf16 -- exactly, once: the
+ *       value of mxq_gelu_bf16 on y;
  *   h quantized as mxq_quantize_act would quantize it: per row, each 32 consecutive
  *   columns form one block (the next layer's K = N), E8M0 scale, E2M1 or E4M3 codes.
  * Blog section "Quantization formats" for the formats; the FFN whose hidden activation
@@ -208,6 +209,15 @@ int64_t mxq_linear_noalloc_max_scratch_bytes(void);
 int mxq_gemm_gelu_quant(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_t K,
                         const void* w_codes, const void* w_sf, int64_t N, const void* bias_bf16, int out_fmt,
                         void* out_codes, void* out_sf, void* h_bf16, void* stream);
+
+/* GELU of n bf16 values, elementwise, as the quantizing epilogue applies it: y[i] =
+ * GELU(x[i]) = x[i]/2 erfc(-x[i]/sqrt 2) rounded once to bf16 (nearest, ties to even), the
+ * exact value rounded; +Inf gives +Inf, -Inf and NaN give NaN (0x7FC0).  For 2^-10 <= |x|
+ * < 16 the kernel looks the result up in a 3584-entry table it builds in shared memory
+ * from the fp64 erfc; elsewhere GELU has a closed form at bf16 precision (x/2 rounded,
+ * x, or -0).  x, y: n bf16 values on the device, 2-byte aligned (they may be the same
+ * buffer).  n > 0, else MXQ_ERR_INVALID_ARG. */
+int mxq_gelu_bf16(const void* x_bf16, int64_t n, void* y_bf16, void* stream);
 
 /* mxq_gemm_gelu_quant with the activation chosen: act MXQ_ACT_GELU is that entry point;
  * MXQ_ACT_NONE quantizes the linear's own output, h = bf16(x . deq(w)^T + bias), so the

@@ -218,3 +218,11 @@ def test_linear_entry_points_reject_unsupported_shapes_with_their_reason():
     ys = (ctypes.c_void_p * 8)(*[4096] * 8)
     assert L.mxq_dit_block_linears(descs, xs, ms, ys, 0x80, 0, ws, 1 << 30, None) == _lib.ERR_SHAPE
     assert "block linear 7" in _lib.last_error() and "K % 128" in _lib.last_error()
+
+
+def test_gelu_entry_point_rejects_bad_arguments():
+    L = _lib.lib()
+    assert L.mxq_gelu_bf16(A16, 0, A16, None) == _lib.ERR_INVALID_ARG
+    assert L.mxq_gelu_bf16(None, 8, A16, None) == _lib.ERR_INVALID_ARG
+    assert L.mxq_gelu_bf16(V(4096 + 1), 8, A16, None) == _lib.ERR_ALIGN
+    assert L.mxq_gelu_bf16(A16, 8, V(4096 + 1), None) == _lib.ERR_ALIGN

@@ -5,6 +5,9 @@ The oracle computes the same chain from the same bf16 inputs in fp64
 (oracle.ffn_hidden_rows).  The GPU accumulates in fp32 in another order, so its bf16
 rounding of the linear output differs from the oracle's on a small fraction of
 elements; the checks are therefore:
+  * the GELU itself is exact: on every bf16 value (mxq_gelu_bf16, the epilogue's table),
+    and inside the epilogue, where h is bit for bit the oracle's bf16 GELU of the GPU's own
+    pre-activation (the no-activation epilogue's h);
   * h (the GELU output, returned for checking) equals the oracle's on >= 99 % of the
     elements and stays within the GEMM tolerance everywhere;
   * codes and scales are bit-exact against the oracle's chain on every block whose 32 h
@@ -120,9 +123,33 @@ def test_gemm_quant_identity_is_quantize_of_gemm(M, N, K, a_fmt, h_fmt):
     wo, wso, _ = _mx.oracle_quantize(w, "e2m1")
     ref = oracle.linear_rows(xo, xso, _mx.FMT[a_fmt], np.arange(M), K, wo, wso, _mx.bits(b))
     _mx.assert_gemm_close(_mx.bf16_to_f64(h), ref, "identity-quant epilogue M=%d N=%d" % (M, N))
-    cg, sg = ops.gemm_quant(xc, xs, a_fmt, M, K, qw, act="gelu", out_fmt=h_fmt)
+    hg = torch.empty_like(h)
+    cg, sg = ops.gemm_quant(xc, xs, a_fmt, M, K, qw, act="gelu", out_fmt=h_fmt, h=hg)
     cg2, sg2 = ops.gemm_gelu_quant(xc, xs, a_fmt, M, K, qw, out_fmt=h_fmt)
     assert torch.equal(cg, cg2) and torch.equal(sg, sg2)
+    # the GELU step inside the epilogue: exactly the oracle's bf16 GELU of the same y
+    assert np.array_equal(_bits_np(hg).reshape(M, N), oracle.gelu_bf16(_bits_np(y).reshape(M, N)))
+
+
+def _is_nan_bf16(b):
+    return ((b & 0x7F80) == 0x7F80) & ((b & 0x007F) != 0)
+
+
+def test_gelu_bf16_every_pattern():
+    """All 65536 bf16 bit patterns: the library's GELU (the epilogue's table and closed
+    forms) equals the oracle's fp64 GELU rounded once to bf16, bit for bit; where the
+    oracle gives NaN (NaN inputs, -Inf) the library gives NaN."""
+    ops = _ops()
+    allb = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    x = torch.from_numpy(allb.view(np.int16)).view(torch.bfloat16).cuda()
+    y = _bits_np(ops.gelu_bf16(x))
+    assert ops.poll_status() == 0
+    ref = oracle.gelu_bf16(allb)
+    nan_ref = _is_nan_bf16(ref)
+    assert np.array_equal(_is_nan_bf16(y), nan_ref)
+    bad = np.nonzero((y != ref) & ~nan_ref)[0]
+    assert bad.size == 0, "GELU differs on %d bf16 values, e.g. %s" % (
+        bad.size, [(hex(int(allb[i])), hex(int(y[i])), hex(int(ref[i]))) for i in bad[:5]])
 
 
 def test_gemm_gelu_quant_padding_rows_are_zero():
