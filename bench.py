@@ -70,8 +70,8 @@ GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precisio
                 "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h", "fp8_mixed_precision_mxq_b200/csrc/mx_elem.cuh"]
 GEMM_TRAFFIC = {
     ("ffn_up_720p_w4a4", 75600): {
-        "bytes": 695879424 + 2050994176,
-        "sources_sha256": "7cfa29bc9b1fd1cced51ef8ee728c3be90960ff0dfa28a80043001efe7a56a75"},
+        "bytes": 627211776 + 2045057792,
+        "sources_sha256": "2ad0fe01a26cefa370598c36b36ec6babb1c943f86055265f654b3bbf8230b61"},
 }
 
 
