@@ -70,8 +70,8 @@ GEMM_SOURCES = ["fp8_mixed_precision_mxq_b200/csrc/gemm.cu", "fp8_mixed_precisio
                 "fp8_mixed_precision_mxq_b200/csrc/mxq_internal.h", "fp8_mixed_precision_mxq_b200/csrc/mx_elem.cuh"]
 GEMM_TRAFFIC = {
     ("ffn_up_720p_w4a4", 75600): {
-        "bytes": 627211776 + 2045057792,
-        "sources_sha256": "2ad0fe01a26cefa370598c36b36ec6babb1c943f86055265f654b3bbf8230b61"},
+        "bytes": 662759936 + 2048216576,
+        "sources_sha256": "675093c7b3b204cfe9b1b37c800248eaea482b08cddd63523ef23a2e233f80ae"},
 }
 
 

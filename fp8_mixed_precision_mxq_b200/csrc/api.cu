@@ -179,7 +179,7 @@ int run_linear(const void* x, int64_t M, int64_t K, const void* w_codes, const v
     RETURN_IF(run_gemm_bf16(xd, wd, bias, y, M, N, K, stream));
     char gp[sizeof g_path];
     snprintf(gp, sizeof gp, "%s", g_path);
-    snprintf(g_path, sizeof g_path, "qdq %s dequant + %s", fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1", gp);
+    snprintf(g_path, sizeof g_path, "qdq %s dequant + %.200s", fmt == MXQ_FMT_E4M3 ? "e4m3" : "e2m1", gp);
     return ok();
 }
 

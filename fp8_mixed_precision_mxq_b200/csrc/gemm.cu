@@ -92,14 +92,24 @@ static_assert(BN / 32 >= 3, "the quantizing epilogue's ring holds three chunks")
 constexpr int kOutBf16 = 0;
 constexpr int kOutGeluE2M1 = 1;
 constexpr int kOutGeluE4M3 = 2;
+// The same two quantizing epilogues for launches that ask for no h: without the bf16
+// staging buffers they have room for the bf16 variant's six pipeline stages, and h's store
+// path is compiled out (1-2 % faster than the variants with h, paired A/B at 720p).
+constexpr int kOutQE2M1 = 3;
+constexpr int kOutQE4M3 = 4;
+template <int kOut>
+constexpr bool kOutE4M3 = kOut == kOutGeluE4M3 || kOut == kOutQE4M3;
+template <int kOut>
+constexpr bool kOutEbuf = kOut <= kOutGeluE4M3;  // bf16 staging buffers (y, or h on request)
 
 // Shared-memory plan of one CTA.  kPair = 1: the CTA owns a 128 x 256 tile and loads
 // all 256 weight rows; kPair = 2: a CTA pair owns a 256 x 256 tile, each CTA loads its
 // own 128 activation rows and 128 of the 256 weight rows (the pair MMA reads both).
 template <int kPair, int kOut>
 struct Cfg {
-    // the quantizing epilogue's code staging takes one pipeline stage's worth of memory
-    static constexpr int kStages = kPair == 2 ? (kOut ? 5 : 6) : (kOut ? 3 : 4);
+    // the quantizing epilogue's code staging takes one pipeline stage's worth of memory,
+    // unless the launch writes no h (no bf16 staging then)
+    static constexpr int kStages = kPair == 2 ? ((kOut && kOutEbuf<kOut>) ? 5 : 6) : (kOut ? 3 : 4);
     static constexpr int BM = 128 * kPair;
     static constexpr int kRowsB = BN / kPair;
     static constexpr uint32_t kStageA = 128 * 128;
@@ -111,12 +121,12 @@ struct Cfg {
     static constexpr uint32_t kOffSFA = kOffB + kStages * kStageB;
     static constexpr uint32_t kOffSFB = kOffSFA + kStages * kStageSFA;
     static constexpr uint32_t kOffEpi = kOffSFB + kStages * kStageSFB;
-    static constexpr uint32_t kQBuf = kOut == kOutGeluE4M3 ? 32 * 32 : 32 * 16;  // 32 rows of one block's codes
+    static constexpr uint32_t kQBuf = kOutE4M3<kOut> ? 32 * 32 : 32 * 16;  // 32 rows of one block's codes
     // code staging buffers per warp: two, or one for E4M3, whose larger codes would
     // otherwise leave no room for the GELU table
-    static constexpr int kQBufs = kOut == kOutGeluE4M3 ? 1 : 2;
+    static constexpr int kQBufs = kOutE4M3<kOut> ? 1 : 2;
     static constexpr int kEpiWarps = kEpiWarpsOf<kOut>;
-    static constexpr uint32_t kOffQ = kOffEpi + kEpiWarps * 2 * kEpiBuf;
+    static constexpr uint32_t kOffQ = kOffEpi + (kOutEbuf<kOut> ? kEpiWarps * 2 * kEpiBuf : 0u);
     static constexpr uint32_t kOffLut = kOffQ + (kOut ? kEpiWarps * kQBufs * kQBuf : 0u);  // GELU table
     static constexpr uint32_t kOffBar = kOffLut + (kOut ? kGeluTableBytes : 0u);
     static constexpr uint32_t kNumBars = 2 * kStages + 6 + 2 * kSfBufs;
@@ -201,7 +211,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
         prefetch_tmap(&map_b);
         prefetch_tmap(&map_sfa);
         prefetch_tmap(&map_sfb);
-        if (kOut == kOutBf16 || p.write_h) prefetch_tmap(&map_y);
+        if (kOut == kOutBf16 || (kOutEbuf<kOut> && p.write_h)) prefetch_tmap(&map_y);
         if (kOut != kOutBf16) prefetch_tmap(&map_q);
         if (p.lr_stages > 0) {
             prefetch_tmap(&map_u);
@@ -514,7 +524,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                         chunk_out(std::true_type{});
                     else
                         chunk_out(std::false_type{});
-                    const bool store_y = kOut == kOutBf16 || p.write_h;
+                    const bool store_y = kOut == kOutBf16 || (kOutEbuf<kOut> && p.write_h);
                     uint8_t* buf = ebuf0 + eb * kEpiBuf;
                     // the stores that last used this chunk's buffers have read them
                     if (lane == 0) {
@@ -535,7 +545,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                     if constexpr (kOut != kOutBf16) {
                         // this lane's 32 values are one MX block of the next layer's K: its
                         // E8M0 scale and element codes, rounded to nearest even by cvt
-                        constexpr uint32_t kEmax = kOut == kOutGeluE4M3 ? 8u : 2u;
+                        constexpr uint32_t kEmax = kOutE4M3<kOut> ? 8u : 2u;
                         uint32_t m2 = o[0];
 #pragma unroll
                         for (int i = 1; i < 16; ++i) m2 = absmax_bf16x2(m2, o[i]);
@@ -544,7 +554,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                         const float inv = e8m0_inverse(sc);
                         const uint32_t keep = sc == 255u ? 0u : 0xFFFFFFFFu;  // a non-finite block: codes 0
                         uint8_t* qb = qbuf0 + (C::kQBufs == 2 ? eb : 0) * C::kQBuf;
-                        if constexpr (kOut == kOutGeluE2M1) {
+                        if constexpr (!kOutE4M3<kOut>) {
                             uint32_t cw[4];
                             const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
@@ -579,7 +589,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                         if (store_y) tma_store_2d(&map_y, buf, n, row0, pol_y);
                         if constexpr (kOut != kOutBf16)
                             tma_store_2d(&map_q, qbuf0 + (C::kQBufs == 2 ? eb : 0) * C::kQBuf,
-                                         kOut == kOutGeluE2M1 ? n / 2 : n, row0,
+                                         kOutE4M3<kOut> ? n : n / 2, row0,
                                          pol_y);
                         bulk_commit();
                     }
@@ -749,6 +759,10 @@ cudaError_t launch_out(int out, const CUtensorMap& ma, const CUtensorMap& mb, co
         return launch_variant<kW4A8, kPair, kOutGeluE2M1>(ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream);
     if (out == kOutGeluE4M3)
         return launch_variant<kW4A8, kPair, kOutGeluE4M3>(ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream);
+    if (out == kOutQE2M1)
+        return launch_variant<kW4A8, kPair, kOutQE2M1>(ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream);
+    if (out == kOutQE4M3)
+        return launch_variant<kW4A8, kPair, kOutQE4M3>(ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream);
     return launch_variant<kW4A8, kPair, kOutBf16>(ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream);
 }
 
@@ -835,7 +849,9 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     p.gelu = g.out_gelu ? 1 : 0;
     p.alpha = g.alpha;
     p.lr_stages = lr_stages;
-    const int out = !quant_out ? kOutBf16 : (g.out_fmt == kFmtE4M3 ? kOutGeluE4M3 : kOutGeluE2M1);
+    const int out = !quant_out  ? kOutBf16
+                    : p.write_h ? (g.out_fmt == kFmtE4M3 ? kOutGeluE4M3 : kOutGeluE2M1)
+                                : (g.out_fmt == kFmtE4M3 ? kOutQE4M3 : kOutQE2M1);
 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
