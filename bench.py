@@ -30,7 +30,7 @@ once, before timing (a load-time step).  Beside the headline number the JSON lin
   e2e           the same step through host buffers (pinned H2D of x, D2H of y every step),
                 copies of neighbouring steps overlapped on separate streams; the serial
                 form beside it;
-  cpu_baseline  the CPU oracle on the machine's host cores: the linear on a bounded sample of
+  cpu_baseline  the CPU oracle on this machine's host cores: the linear on a bounded sample of
                 rows and the quantizer on the whole activation, single-threaded and on all
                 cores.
 
@@ -297,7 +297,7 @@ def cpu_quantize_rate(x_bits, fmt, nthreads):
 
 
 def cpu_baseline(M, N, K, fmt, seed, budget_s=6.0, x_bits=None):
-    """The CPU oracle as it stands, on the machine's host cores: the linear (quantize + fp64 GEMM)
+    """The CPU oracle as it stands, on the host's CPU cores: the linear (quantize + fp64 GEMM)
     on a bounded sample of activation rows, single-threaded and on all cores (about budget_s
     seconds each), and, when the activation's bits are given, the quantizer on the whole
     tensor, single-threaded and on all cores.  `value` is the all-core linear rate."""
@@ -941,7 +941,7 @@ def bench_w4a8(args, ops, synth, dev, stream, world, rank, peaks):
 
 
 def run_reference(args):
-    """The reference arm: the CPU oracle, on the machine's host cores, on a bounded sample
+    """The reference arm: the CPU oracle, on the host's CPU cores, on a bounded sample
     of the same workload per step.  Under torchrun only rank 0 runs it."""
     import synth
     rank = int(os.environ.get("RANK", "0"))
