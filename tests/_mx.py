@@ -116,7 +116,9 @@ def check_transformed(codes_gpu, sf_gpu, rows: int, K: int, fmt: str, ref: dict,
     Returns the number of uncertain elements."""
     if max_uncertain == "default":
         max_uncertain = UNCERTAIN_LIMIT[fmt]
-    sf_l = tiled_to_logical(sf_gpu.cpu().numpy() if hasattr(sf_gpu, "cpu") else sf_gpu, rows, K)
+    sf_np = sf_gpu.cpu().numpy() if hasattr(sf_gpu, "cpu") else sf_gpu
+    # scales in the tiled layout, or already logical [rows, K / 32] (a row subset)
+    sf_l = sf_np if sf_np.ndim == 2 else tiled_to_logical(sf_np, rows, K)
     cg = unpack_codes(codes_gpu.cpu().numpy() if hasattr(codes_gpu, "cpu") else codes_gpu, rows, K, fmt)
     cd = unpack_codes(ref["codes"], rows, K, fmt)
     amb = ref["blk_amb"]

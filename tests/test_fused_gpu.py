@@ -150,6 +150,9 @@ def test_gelu_bf16_every_pattern():
     bad = np.nonzero((y != ref) & ~nan_ref)[0]
     assert bad.size == 0, "GELU differs on %d bf16 values, e.g. %s" % (
         bad.size, [(hex(int(allb[i])), hex(int(y[i])), hex(int(ref[i]))) for i in bad[:5]])
+    # in place gives the same
+    ops.gelu_bf16(x, out=x)
+    assert np.array_equal(_bits_np(x), y)
 
 
 def test_gemm_gelu_quant_padding_rows_are_zero():

@@ -173,3 +173,25 @@ def test_transform_full_ffn_up_480p(block):
     ref_y = oracle.linear_rows(ref["codes"].reshape(M, K2)[rows], ref["sf"][rows], oracle.E2M1, np.arange(len(rows)),
                                K, wo["codes"], wo["sf"], _mx.bits(b))
     _mx.assert_gemm_close(_mx.bf16_to_f64(y[torch.from_numpy(rows).cuda()]), ref_y, "transformed linear 480p")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("block", [32, 128])
+def test_transform_720p_sampled_rows(block):
+    """The bench's headline transform_on shape (M = 75600, K = 5120) in the launch
+    configuration the bench times: the whole tensor quantized on the GPU, one row per
+    128-row tile plus the ends checked against the definition."""
+    ops = _ops()
+    wl = synth.workload("ffn_up_720p_w4a4", device="cuda", with_bias=False)
+    x, M, K = wl["x"], wl["M"], wl["K"]
+    s = smooth_scales(x)
+    inv_s = (1.0 / s).contiguous()
+    codes, sf = ops.quantize_act_transformed(x, "e2m1", block, inv_s)
+    assert ops.poll_status() == 0
+    rows = synth.sample_rows(M).numpy()
+    xs = _mx.bits(x[torch.from_numpy(rows).cuda()])
+    ref = oracle.quantize_transformed(xs, oracle.E2M1, block, inv_s.cpu().numpy())
+    cg = codes.view(M, K // 2)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    sg = _mx.tiled_to_logical(sf.cpu().numpy(), M, K)[rows]
+    n_unc = _mx.check_transformed(cg, sg, len(rows), K, "e2m1", ref, "720p B=%d sampled rows" % block)
+    print("720p transform B=%d: %d uncertain elements of %d sampled" % (block, n_unc, len(rows) * K))
