@@ -655,12 +655,19 @@ def bench_linear(args, ops, synth, wl_name, dev, stream, world, rank, peaks):
                          "frac_hbm": round(q_gbs / peaks["hbm_gbs"], 4)}}
 
 
-def linears_roofline_ms(synth, rows_x, rows_ctx, bits, peaks):
+def sustained_tflops(peaks):
+    """The bf16 figure measured as a seconds-long loop under the power cap (the burst
+    figure when the peaks file has none)."""
+    return peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+
+
+def linears_roofline_ms(synth, rows_x, rows_ctx, bits, peaks, sustained=False):
     """Tensor-core floor of one block's eight linears: each linear's FLOPs at the FP4
-    (W4A4) or FP8 (W4A8) dense peak, the peaks being the measured bf16 burst x the
-    nominal dtype ratio."""
-    fp4 = peaks["bf16_tflops"] * FP4_OVER_BF16 * 1e12
-    fp8 = peaks["bf16_tflops"] * FP8_OVER_BF16 * 1e12
+    (W4A4) or FP8 (W4A8) dense peak, the peaks being the measured bf16 burst (or, with
+    `sustained`, the bf16 loop under the power cap) x the nominal dtype ratio."""
+    bf16 = sustained_tflops(peaks) if sustained else peaks["bf16_tflops"]
+    fp4 = bf16 * FP4_OVER_BF16 * 1e12
+    fp8 = bf16 * FP8_OVER_BF16 * 1e12
     t = 0.0
     for i, (name, N, K, src) in enumerate(synth.BLOCK_LINEARS):
         rows = rows_x if src == "x" else rows_ctx
@@ -686,6 +693,7 @@ def bench_ffn(args, ops, synth, dev, stream, world, rank, peaks):
                          outlier_frac=0.01, outlier_scale=30.0)
     y = torch.empty((M, N2), dtype=torch.bfloat16, device=dev)
     flops = 2.0 * M * (K * H + H * N2)
+    sus = sustained_tflops(peaks) / peaks["bf16_tflops"]  # sustained / burst
     fp4 = peaks["bf16_tflops"] * FP4_OVER_BF16 * 1e12
     fp8 = peaks["bf16_tflops"] * FP8_OVER_BF16 * 1e12
     iters = max(3, args.steps // 10)
@@ -696,11 +704,14 @@ def bench_ffn(args, ops, synth, dev, stream, world, rank, peaks):
         fn = lambda f=down_fmt, w=wsb: ops.ffn(x, up, down, "e2m1", f, workspace=w, out=y)  # noqa: E731
         for _ in range(2):
             fn()
-        ms = max_over_ranks(time_loop(fn, iters, stream), world)
+        with ClockSampler(dev.index) as clk:
+            ms = time_loop(fn, iters, stream)
+        ms = max_over_ranks(ms, world)
         roof = (2.0 * M * K * H / fp4 + 2.0 * M * H * N2 / (fp8 if down_fmt == "e4m3" else fp4)) * 1e3
         res["fused_down_" + down_fmt] = {"ms": round(ms, 3), "TFLOP/s": round(job_tflops(flops, ms, world), 1),
                                          "roofline_ms": round(roof, 3), "frac": round(roof / ms, 4),
-                                         "launches": 3, "path": ops.last_path()}
+                                         "frac_sustained": round(roof / sus / ms, 4),
+                                         "launches": 3, "path": ops.last_path(), "clocks": clk.summary()}
         del wsb
     # unfused comparison (W4A4 down): bf16 hidden activation written, GELU by torch, read back
     hbuf = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
@@ -809,9 +820,11 @@ def bench_block(args, ops, synth, dev, stream, world, rank, peaks):
             ms = time_loop(fn, iters, stream)
         ms = max_over_ranks(ms, world)
         roof = linears_roofline_ms(synth, M, ctx, bits, peaks)
+        roof_s = linears_roofline_ms(synth, M, ctx, bits, peaks, sustained=True)
         res[name] = {"mask": "0x%02x" % bits, "ms": round(ms, 3),
                      "TFLOP/s": round(job_tflops(flops, ms, world), 1),
-                     "roofline_ms": round(roof, 3), "frac": round(roof / ms, 4), "clocks": clk.summary()}
+                     "roofline_ms": round(roof, 3), "frac": round(roof / ms, 4),
+                     "frac_sustained": round(roof_s / ms, 4), "clocks": clk.summary()}
     # where the all-W4A4 block's time goes: each linear's quantizer and GEMM timed alone
     # (50 launches each) against that linear's FP4 floor
     fp4 = peaks["bf16_tflops"] * FP4_OVER_BF16 * 1e12
@@ -892,11 +905,15 @@ def bench_stack(args, ops, synth, dev, stream, world, rank, peaks):
                        "M=%d video + %d text tokens; unit = one expert's forward (%.1f TFLOP)" % (
                            B, resident / 1e9, c["n_w4a8"], M, ctx, flops / 1e12)}
     for e in range(E):
-        ms = max_over_ranks(time_loop(lambda e=e: forward(e), iters, stream), world)
+        with ClockSampler(dev.index) as clk:
+            ms = time_loop(lambda e=e: forward(e), iters, stream)
+        ms = max_over_ranks(ms, world)
         roof = sum(linears_roofline_ms(synth, M, ctx, bits[e][blk], peaks) for blk in range(B))
+        roof_s = sum(linears_roofline_ms(synth, M, ctx, bits[e][blk], peaks, sustained=True) for blk in range(B))
         res["expert%d" % e] = {"w4a8_blocks": [blk for blk in range(B) if bits[e][blk]], "ms": round(ms, 2),
                                "TFLOP/s": round(job_tflops(flops, ms, world), 1),
-                               "roofline_ms": round(roof, 2), "frac": round(roof / ms, 4)}
+                               "roofline_ms": round(roof, 2), "frac": round(roof / ms, 4),
+                               "frac_sustained": round(roof_s / ms, 4), "clocks": clk.summary()}
     if ops.poll_status() != 0:
         raise RuntimeError("device status set during the expert-stack measurement")
     return res

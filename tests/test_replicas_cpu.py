@@ -65,6 +65,23 @@ def test_step_statistics():
     assert st["mean"] == round(sum([3, 1, 2, 10, 4, 5, 6, 7, 8, 9, 2.5]) / 11, 4)
 
 
+def test_block_roofline_burst_and_sustained():
+    """A block's tensor floor: each linear's FLOPs at 4x (W4A4) or 2x (W4A8) the bf16
+    figure, burst or sustained; an all-W4A4 block at 4 PFLOP/s bf16 takes its FLOPs / 16e15."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    M, ctx = 75600, 512
+    peaks = {"bf16_tflops": 4000.0, "bf16_tflops_sustained": 3000.0}
+    burst = bench.linears_roofline_ms(synth, M, ctx, 0x00, peaks)
+    assert abs(burst - synth.block_flops(M, ctx) / 16e15 * 1e3) < 1e-9
+    assert abs(bench.linears_roofline_ms(synth, M, ctx, 0x00, peaks, sustained=True) - burst * 4 / 3) < 1e-9
+    # every linear in W4A8 halves the rate
+    assert abs(bench.linears_roofline_ms(synth, M, ctx, 0xFF, peaks) - 2 * burst) < 1e-9
+    # no sustained figure: the burst one stands in
+    assert bench.linears_roofline_ms(synth, M, ctx, 0x00, {"bf16_tflops": 4000.0}, sustained=True) == burst
+
+
 def test_reference_arm_prints_one_line_with_its_own_baseline():
     """Rank 0 of the reference arm: the CPU oracle on a bounded sample, one JSON line with the
     same metric, impl "reference", an e2e that is the line's own value and no device copies."""
