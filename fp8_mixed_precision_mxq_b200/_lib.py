@@ -45,6 +45,7 @@ SIGNATURES = {
     "mxq_dequantize": ([_vp, _vp, _i64, _i64, _i32, _vp, _vp], _i32),
     "mxq_gemm": ([_vp, _vp, _i32, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp], _i32),
     "mxq_gemm_bf16": ([_vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp], _i32),
+    "mxq_gemm_bf16_quant_a": ([_vp, _i64, _i64, _vp, _i64, _vp, _vp, _i32, _vp, _vp, _vp], _i32),
     "mxq_channel_absmax": ([_vp, _i64, _i64, _vp, _vp], _i32),
     "mxq_smooth_scales": ([_vp, _vp, _i64, ctypes.c_float, _vp, _vp, _vp], _i32),
     "mxq_sqnr": ([ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.POINTER(_i64), _i32, _vp, _vp], _i32),

@@ -316,6 +316,36 @@ int mxq_gemm_bf16(const void* a_bf16, int64_t M, int64_t K, const void* b_bf16, 
     return run_gemm_bf16(a_bf16, b_bf16, bias_bf16, y_bf16, M, N, K, static_cast<cudaStream_t>(stream));
 }
 
+// y = a . b^T + bias in bf16 by the bf16 GEMM kernel, whose extra warps also write a's MX
+// quantization (format fmt) as its tiles pass through shared memory: one read of a.
+int run_gemm_bf16_quant_a(const void* a, const void* b, const void* bias, void* y, int64_t M, int64_t N, int64_t K,
+                          int fmt, void* codes, void* sf, cudaStream_t stream)
+{
+    GemmArgs g{a, nullptr, MXQ_FMT_E2M1, M, N, K, b, nullptr, bias, y};
+    g.bf16 = true;
+    g.qa_fmt = fmt;
+    g.qa_codes = codes;
+    g.qa_sf = sf;
+    const char* msg = nullptr;
+    int rc = launch_gemm(g, stream, &msg, g_path, sizeof g_path);
+    if (rc != MXQ_OK) return fail(rc, "bf16 gemm quantizing a: %s", msg ? msg : "launch failed");
+    return ok();
+}
+
+int mxq_gemm_bf16_quant_a(const void* a_bf16, int64_t M, int64_t K, const void* b_bf16, int64_t N,
+                          const void* bias_bf16, void* y_bf16, int fmt, void* codes, void* sf, void* stream)
+{
+    RETURN_IF(check_fmt(fmt));
+    RETURN_IF(check_rows_k(M, K, "a"));
+    RETURN_IF(check_gemm_bf16(a_bf16, M, K, b_bf16, N, bias_bf16, y_bf16));
+    if (N > 128) return fail(MXQ_ERR_SHAPE, "bf16 gemm quantizing a: N=%lld is above 128", (long long)N);
+    RETURN_IF(check_ptr(codes, "codes"));
+    RETURN_IF(check_ptr(sf, "sf"));
+    RETURN_IF(check_device());
+    return run_gemm_bf16_quant_a(a_bf16, b_bf16, bias_bf16, y_bf16, M, N, K, fmt, codes, sf,
+                                 static_cast<cudaStream_t>(stream));
+}
+
 int mxq_linear(const void* x_bf16, int64_t M, int64_t K, const void* w_codes, const void* w_sf, int64_t N,
                const void* bias_bf16, int act_fmt, int mode, void* workspace, int64_t ws_bytes, void* y_bf16,
                void* stream)
@@ -686,9 +716,15 @@ int mxq_linear_lowrank(const void* x_bf16, int64_t M, int64_t K, const void* r_c
     uint8_t* xc = static_cast<uint8_t*>(workspace);
     uint8_t* xs = xc + round_up(codes_bytes(M, K, act_fmt), kWsAlign);
     uint8_t* u = xs + round_up(sf_bytes(M, K), kWsAlign);
-    RETURN_IF(cuda_rc(launch_quantize(x_bf16, M, K, act_fmt, xc, xs, st), "quantize launch"));
-    // u = x . l1t^T: [M, K] x [K, rank], the bf16 GEMM with N = rank
-    int rc = run_gemm_bf16(x_bf16, l1t_bf16, nullptr, u, M, rank, K, st);
+    // u = x . l1t^T: [M, K] x [K, rank], the bf16 GEMM with N = rank; up to rank 128 the
+    // same launch writes x quantized in act_fmt (xc, xs), so x is read once for both
+    int rc;
+    if (rank <= 128) {
+        rc = run_gemm_bf16_quant_a(x_bf16, l1t_bf16, nullptr, u, M, rank, K, act_fmt, xc, xs, st);
+    } else {
+        RETURN_IF(cuda_rc(launch_quantize(x_bf16, M, K, act_fmt, xc, xs, st), "quantize launch"));
+        rc = run_gemm_bf16(x_bf16, l1t_bf16, nullptr, u, M, rank, K, st);
+    }
     if (rc != MXQ_OK) return fail(rc, "low-rank u: %s", g_err);
     GemmArgs g{xc, xs, act_fmt, M, N, K, r_codes, r_sf, bias_bf16, y_bf16};
     g.lr_rank = rank;

@@ -64,6 +64,11 @@ template <int kOut>
 constexpr int kEpiWarpsOf = kOut ? 8 : 4;
 template <int kOut>
 constexpr int kThreadsOf = 64 + 32 * kEpiWarpsOf<kOut> + 32;
+// A bf16 GEMM that also MX-quantizes its A operand (the bf16 activation) as its stages
+// stream through shared memory: eight more warps, one MX block of an A row per thread.
+constexpr int kQaWarps = 8;
+template <int kOut, bool kQA>
+constexpr int kThreadsFor = kThreadsOf<kOut> + (kQA ? 32 * kQaWarps : 0);
 constexpr uint32_t kEpiBuf = 32 * 64;     // 32 rows x 32 bf16
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: accumulator slot 0 [0, BN), slot 1 [kAccCol1, kAccCol1 + BN) (sharing
@@ -84,6 +89,18 @@ constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int kLdBufs = 3;
 static_assert(kOverlapChunks <= kLdBufs, "the shared columns must fit the first round of loads");
 static_assert(BN / 32 >= 3, "the quantizing epilogue's ring holds three chunks");
+// The kernel that quantizes its A (kQA) writes at most 128 output columns and copies no
+// scales into TMEM, so its two accumulator slots take [0, 256) and [256, 512) and share
+// nothing; its epilogue drains the four chunks that can hold output, two loads in flight
+// (which keeps it inside the registers the kernel's 480 threads leave each thread).
+template <bool kQA>
+constexpr uint32_t kAcc1Of = kQA ? 256u : kAccCol1;
+template <bool kQA>
+constexpr int kOverlapOf = kQA ? 0 : kOverlapChunks;
+template <bool kQA>
+constexpr int kLdBufsOf = kQA ? 2 : kLdBufs;
+template <bool kQA>
+constexpr int kChunksOf = kQA ? 4 : BN / 32;
 
 // Output of the epilogue: bf16 y = acc + bias; or the next layer's MX-quantized input,
 // h = bf16(GELU(bf16(acc + bias))) -- or h = bf16(acc + bias) when the launch asks for no
@@ -105,17 +122,19 @@ constexpr bool kOutEbuf = kOut <= kOutGeluE4M3;  // bf16 staging buffers (y, or 
 // Shared-memory plan of one CTA.  kPair = 1: the CTA owns a 128 x 256 tile and loads
 // all 256 weight rows; kPair = 2: a CTA pair owns a 256 x 256 tile, each CTA loads its
 // own 128 activation rows and 128 of the 256 weight rows (the pair MMA reads both).
-template <int kPair, int kOut>
+// kQA (the bf16 GEMM that quantizes its A, output at most 128 wide): B stages of 128 rows
+// and no scale stages, which leaves room for six stages of the activation in flight.
+template <int kPair, int kOut, bool kQA = false>
 struct Cfg {
     // the quantizing epilogue's code staging takes one pipeline stage's worth of memory,
     // unless the launch writes no h (no bf16 staging then)
-    static constexpr int kStages = kPair == 2 ? ((kOut && kOutEbuf<kOut>) ? 5 : 6) : (kOut ? 3 : 4);
+    static constexpr int kStages = kQA ? 6 : kPair == 2 ? ((kOut && kOutEbuf<kOut>) ? 5 : 6) : (kOut ? 3 : 4);
     static constexpr int BM = 128 * kPair;
-    static constexpr int kRowsB = BN / kPair;
+    static constexpr int kRowsB = kQA ? 128 : BN / kPair;
     static constexpr uint32_t kStageA = 128 * 128;
     static constexpr uint32_t kStageB = kRowsB * 128;
-    static constexpr uint32_t kStageSFA = 2 * 512;       // up to two k-atoms
-    static constexpr uint32_t kStageSFB = 2 * 2 * 512;   // both 128-row halves of the tile
+    static constexpr uint32_t kStageSFA = kQA ? 0 : 2 * 512;       // up to two k-atoms
+    static constexpr uint32_t kStageSFB = kQA ? 0 : 2 * 2 * 512;   // both 128-row halves of the tile
     static constexpr uint32_t kOffA = 0;
     static constexpr uint32_t kOffB = kOffA + kStages * kStageA;
     static constexpr uint32_t kOffSFA = kOffB + kStages * kStageB;
@@ -152,6 +171,12 @@ struct Params {
     // low-rank branch: stages of 64 K-elements of u (activation, bf16 [M, r]) and B^T
     // (bf16 [N, r]) MMA'd (kind::f16) into the accumulator before the block-scaled stages
     int lr_stages;
+    int mma_n;  // N of the bf16 MMAs: BN, or the output width rounded up to 16 for a lone CTA's only tile column
+    // A quantized on the side (kQA): codes [M, K/2] (E2M1) or [M, K] (E4M3) and tiled scales
+    uint8_t* qa_codes;
+    uint8_t* qa_sf;
+    uint32_t qa_atoms_k;
+    int qa_fmt;
 };
 
 __device__ __forceinline__ void record_status(uint32_t code) { atomicCAS(&g_device_status, 0u, code); }
@@ -168,16 +193,20 @@ __device__ __forceinline__ void tile_coords(int t, int m_blocks, int n_blocks, i
     mb = first_m + (local - nb * gsize);
 }
 
-template <bool kW4A8, int kPair, int kOut>
-__global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
+template <bool kW4A8, int kPair, int kOut, bool kQA>
+__global__ void __launch_bounds__(kThreadsFor<kOut, kQA>, 1)
     mx_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                    const __grid_constant__ CUtensorMap map_sfa, const __grid_constant__ CUtensorMap map_sfb,
                    const __grid_constant__ CUtensorMap map_y, const __grid_constant__ CUtensorMap map_q,
                    const __grid_constant__ CUtensorMap map_u, const __grid_constant__ CUtensorMap map_l2,
                    const Params p)
 {
-    using C = Cfg<kPair, kOut>;
+    using C = Cfg<kPair, kOut, kQA>;
     constexpr int S = C::kStages;
+    constexpr uint32_t kAcc1 = kAcc1Of<kQA>;     // accumulator slot 1's first column
+    constexpr int kOvl = kOverlapOf<kQA>;        // 32-column chunks the two slots share
+    constexpr int kLdb = kLdBufsOf<kQA>;         // epilogue chunk loads in flight
+    constexpr int kChunks = kChunksOf<kQA>;      // 32-column chunks the epilogue drains
     constexpr int kEpiWarps = C::kEpiWarps;
     constexpr int AK = kW4A8 ? 1 : 2;  // scale atoms (128 K-elements each) per stage
 
@@ -219,7 +248,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
         }
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], 1 + (kQA ? kQaWarps : 0));  // the MMAs' commit, and the A quantizer's warps
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&tmem_full[s], 1);
@@ -268,6 +297,7 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                         continue;
                     }
                     const uint32_t bar = kPair == 2 ? mapa_shared(smem_u32(&full[s]), 0) : smem_u32(&full[s]);
+                    if (kQA) fence_async_smem();  // the quantizer's reads of this stage before the copy's writes
                     if (ks < p.lr_stages) {
                         // low-rank stage: 64 columns of u as A, the same columns of B^T as B
                         if (leader) mbar_arrive_expect_tx(&full[s], kTxLr);
@@ -316,9 +346,9 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
             bool ok = true;
             for (int t = pair_id; t < p.num_tiles && ok; t += n_pairs, ++tcount) {
                 const int slot = tcount & 1;
-                const uint32_t acc = tmem_base + (slot ? kAccCol1 : 0u);
+                const uint32_t acc = tmem_base + (slot ? kAcc1 : 0u);
                 if (!mbar_wait(&tmem_empty[slot], ((tcount >> 1) & 1) ^ 1, kWaitNs) ||
-                    (kOverlapChunks > 0 && tcount > 0 && !mbar_wait(overlap_free, (tcount - 1) & 1, kWaitNs))) {
+                    (kOvl > 0 && tcount > 0 && !mbar_wait(overlap_free, (tcount - 1) & 1, kWaitNs))) {
                     record_status(MXQ_ERR_TIMEOUT);
                     break;
                 }
@@ -341,8 +371,8 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                         const uint32_t b_lo = b_lo0 + s * (C::kStageB >> 4);
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
-                            mma_bf16<kPair>(acc, a_lo + 2 * j, b_lo + 2 * j, kSdescSw128Hi, idesc_bf16(C::BM, BN),
-                                            (ks > 0 || j > 0) ? 1u : 0u);
+                            mma_bf16<kPair>(acc, a_lo + 2 * j, b_lo + 2 * j, kSdescSw128Hi,
+                                            idesc_bf16(C::BM, static_cast<uint32_t>(p.mma_n)), (ks > 0 || j > 0) ? 1u : 0u);
                         tc_commit<kPair>(&empty[s]);
                         if (++s == S) { s = 0; ph ^= 1; }
                         continue;
@@ -422,6 +452,110 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                 }
             }
         }
+    } else if (kQA && warp > 2 + kEpiWarps) {
+        // ------------------------------------------------------------ A quantizer (kQA, lone CTA)
+        // The bf16 stages' A tiles are rows of the activation, 64 channels (two MX blocks)
+        // a stage.  Eight warps, two to a scheduler: thread (row, block) takes block b of
+        // one of the tile's 128 rows, b by warp group.  Once a stage lands it reads its
+        // block (64 bytes; 16-byte chunk q of row r sits at chunk q ^ (r & 7) under the
+        // 128-byte swizzle), releases the stage (the stage's second consumer, beside the
+        // MMAs), and forms the block's E8M0 scale and codes with the activation quantizer's
+        // arithmetic: scale code max(0, E(amax) - emax) from the bf16 exponent field of the
+        // block's abs-max (255 for a NaN or Inf), codes cvt(x 2^-s) rounded to nearest even
+        // with saturation, all-zero codes under scale 255.  Rows past M (zeros from the
+        // copy) write only their scale byte, 0, as the tiled layout's padding; k-blocks past
+        // K / 32 get scale 0 and no codes.  One tile column (N <= 128), so every A stage is
+        // seen once.
+        static_assert(!kQA || (kPair == 1 && kOut == kOutBf16 && !kW4A8), "A quantizer: bf16 lone-CTA kernel only");
+        const int qw = warp - 3 - kEpiWarps;
+        const int r_in = (qw & 3) * 32 + lane;  // row within the tile
+        const uint32_t b = static_cast<uint32_t>(qw >> 2);  // which of a stage's two blocks
+        const uint32_t sw = static_cast<uint32_t>(r_in & 7);
+        const bool e4m3 = p.qa_fmt == kFmtE4M3;
+        const uint32_t emax = e4m3 ? 8u : 2u;
+        const uint32_t KB = static_cast<uint32_t>(p.K / 32);
+        const uint32_t kb_pad = 4u * p.qa_atoms_k;
+        const size_t row_bytes = e4m3 ? static_cast<size_t>(p.K) : static_cast<size_t>(p.K / 2);
+        uint32_t s = 0, ph = 0;
+        bool ok = true;
+        for (int t = pair_id; t < p.num_tiles && ok; t += n_pairs) {
+            int mb, nb;
+            tile_coords<C::kGroupM>(t, p.m_blocks, p.n_blocks, mb, nb);
+            const uint32_t row = static_cast<uint32_t>(mb * C::BM + r_in);
+            const bool live = static_cast<int>(row) < p.M;
+            // this row's scale bytes: atom row block, 32-row column inside the atom
+            uint8_t* sf_row = p.qa_sf + static_cast<size_t>(row >> 7) * p.qa_atoms_k * 512u + (row & 31u) * 16u +
+                              ((row >> 5) & 3u) * 4u;
+            uint8_t* code_row = p.qa_codes + static_cast<size_t>(row) * row_bytes;
+            for (int ks = 0; ks < p.lr_stages; ++ks) {
+                const bool landed = mbar_wait(&full[s], ph, kWaitNs);
+                if (!__all_sync(0xFFFFFFFFu, landed)) {
+                    if (lane == 0) record_status(MXQ_ERR_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+                const uint8_t* rowp = smem + C::kOffA + s * C::kStageA + r_in * 128;
+                uint32_t w[16];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 v =
+                        *reinterpret_cast<const uint4*>(rowp + 16u * ((4u * b + static_cast<uint32_t>(q)) ^ sw));
+                    w[4 * q] = v.x;
+                    w[4 * q + 1] = v.y;
+                    w[4 * q + 2] = v.z;
+                    w[4 * q + 3] = v.w;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                if (++s == S) { s = 0; ph ^= 1; }
+                const uint32_t kb = 2u * static_cast<uint32_t>(ks) + b;
+                if (ks == p.lr_stages - 1 && b == 0)  // the layout's padding k-blocks past the last stage
+                    for (uint32_t kp = kb + 2u; kp < kb_pad; kp += 2u)
+                        *reinterpret_cast<uint16_t*>(sf_row + (kp >> 2) * 512u + (kp & 3u)) = 0;
+                if (kb >= KB) {  // past K: scale 0, no codes
+                    sf_row[(kb >> 2) * 512u + (kb & 3u)] = 0;
+                    continue;
+                }
+                uint32_t m2 = absmax_bf16x2(absmax_bf16x2(w[0], w[1]), absmax_bf16x2(w[2], w[3]));
+#pragma unroll
+                for (int i = 4; i < 16; i += 4)
+                    m2 = absmax_bf16x2(m2, absmax_bf16x2(absmax_bf16x2(w[i], w[i + 1]), absmax_bf16x2(w[i + 2], w[i + 3])));
+                m2 = absmax_bf16x2(m2, __byte_perm(m2, 0, 0x1032));
+                const uint32_t eb = (m2 & 0x7FFFu) >> 7;  // bf16 and E8M0 share the bias 127
+                const uint32_t sc = eb == 255u ? 255u : (eb > emax ? eb - emax : 0u);
+                sf_row[(kb >> 2) * 512u + (kb & 3u)] = static_cast<uint8_t>(sc);
+                if (!live) continue;
+                const float inv = __uint_as_float((254u - min(sc, 253u)) << 23);  // 2^(127 - sc)
+                const float2 inv2 = make_float2(inv, inv);
+                const uint32_t keep = sc == 255u ? 0u : 0xFFFFFFFFu;
+                if (e4m3) {
+                    uint32_t c4[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float2 f0 = __fmul2_rn(make_float2(lo_f(w[2 * i]), hi_f(w[2 * i])), inv2);
+                        const float2 f1 = __fmul2_rn(make_float2(lo_f(w[2 * i + 1]), hi_f(w[2 * i + 1])), inv2);
+                        c4[i] = (cvt_e4m3x2(f0.x, f0.y) | (cvt_e4m3x2(f1.x, f1.y) << 16)) & keep;
+                    }
+                    uint4* d4 = reinterpret_cast<uint4*>(code_row + kb * 32u);
+                    __stcs(d4, make_uint4(c4[0], c4[1], c4[2], c4[3]));
+                    __stcs(d4 + 1, make_uint4(c4[4], c4[5], c4[6], c4[7]));
+                } else {
+                    uint32_t c2[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float q[8];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __fmul2_rn(make_float2(lo_f(w[4 * i + e]), hi_f(w[4 * i + e])), inv2);
+                            q[2 * e] = f.x;
+                            q[2 * e + 1] = f.y;
+                        }
+                        c2[i] = cvt_e2m1x8(q) & keep;
+                    }
+                    __stcs(reinterpret_cast<uint4*>(code_row + kb * 16u), make_uint4(c2[0], c2[1], c2[2], c2[3]));
+                }
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue (each CTA)
         // Each warp owns the 32 TMEM lanes (= output rows) of its quarter.  Per tile it
@@ -461,13 +595,13 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
                 break;
             }
             tc_fence_after();
-            const uint32_t col0 = slot ? kAccCol1 : 0u;
+            const uint32_t col0 = slot ? kAcc1 : 0u;
             const int row0 = mb * C::BM + static_cast<int>(rank) * 128 + q * 32;
             const uint32_t tmem_empty_bar = kPair == 2 ? mapa_shared(smem_u32(&tmem_empty[slot]), 0)
                                                        : smem_u32(&tmem_empty[slot]);
             // chunk order: slot 0 drains its shared (top) columns first, slot 1 its bottom ones
             auto chunk_of = [&](int ci) {
-                return slot ? ci : (ci < kOverlapChunks ? BN / 32 - kOverlapChunks + ci : ci - kOverlapChunks);
+                return slot ? ci : (ci < kOvl ? BN / 32 - kOvl + ci : ci - kOvl);
             };
             // after the loads of this warp's chunks up to drain index ci have landed:
             // release what the MMA issuer waits for (every epilogue warp arrives on both)
@@ -611,26 +745,26 @@ __global__ void __launch_bounds__(kThreadsOf<kOut>, 1)
             if constexpr (kOut == kOutBf16) {
                 // a ring of kLdBufs chunk registers, fully unrolled: the first kLdBufs loads go
                 // out back to back, so the shared columns are released after one wait
-                uint32_t r[kLdBufs][32];
+                uint32_t r[kLdb][32];
 #pragma unroll
-                for (int j = 0; j < kLdBufs; ++j) tmem_ld_x32(lanes + col0 + chunk_of(j) * 32, r[j]);
-                int issued = kLdBufs, landed_upto = 0;  // constants once the loop below is unrolled
+                for (int j = 0; j < kLdb; ++j) tmem_ld_x32(lanes + col0 + chunk_of(j) * 32, r[j]);
+                int issued = kLdb, landed_upto = 0;  // constants once the loop below is unrolled
 #pragma unroll
-                for (int ci = 0; ci < BN / 32; ++ci) {
+                for (int ci = 0; ci < kChunks; ++ci) {
                     if (ci >= landed_upto) {  // everything issued so far lands together
                         tmem_ld_wait();
 #pragma unroll
-                        for (int j = 0; j < BN / 32; ++j)
+                        for (int j = 0; j < kChunks; ++j)
                             if (j >= landed_upto && j < issued) {
-                                tmem_regs_ready(r[j % kLdBufs]);
-                                landed(j, kOverlapChunks - 1, BN / 32 - 1);
+                                tmem_regs_ready(r[j % kLdb]);
+                                landed(j, kOvl - 1, kChunks - 1);
                             }
                         landed_upto = issued;
                     }
-                    process(r[ci % kLdBufs], ci);
-                    if (ci + kLdBufs < BN / 32) {  // refill the buffer just drained
-                        tmem_ld_x32(lanes + col0 + chunk_of(ci + kLdBufs) * 32, r[ci % kLdBufs]);
-                        issued = ci + kLdBufs + 1;
+                    process(r[ci % kLdb], ci);
+                    if (ci + kLdb < kChunks) {  // refill the buffer just drained
+                        tmem_ld_x32(lanes + col0 + chunk_of(ci + kLdb) * 32, r[ci % kLdb]);
+                        issued = ci + kLdb + 1;
                     }
                 }
             } else {
@@ -725,19 +859,19 @@ int read_and_clear_device_status(cudaStream_t stream, uint32_t* out)
 
 namespace {
 
-template <bool kW4A8, int kPair, int kOut>
+template <bool kW4A8, int kPair, int kOut, bool kQA = false>
 cudaError_t launch_variant(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& msa,
                            const CUtensorMap& msb, const CUtensorMap& my, const CUtensorMap& mq,
                            const CUtensorMap& mu, const CUtensorMap& ml, const Params& p, int grid,
                            cudaStream_t stream)
 {
-    using C = Cfg<kPair, kOut>;
-    auto kern = mx_gemm_kernel<kW4A8, kPair, kOut>;
+    using C = Cfg<kPair, kOut, kQA>;
+    auto kern = mx_gemm_kernel<kW4A8, kPair, kOut, kQA>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(kThreadsOf<kOut>, 1, 1);
+    cfg.blockDim = dim3(kThreadsFor<kOut, kQA>, 1, 1);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -773,8 +907,15 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     const bool bf16 = g.bf16;
     const bool w4a8 = !bf16 && g.a_fmt == kFmtE4M3;
     const bool quant_out = g.out_fmt >= 0;
-    // CTA pairs for anything taller than one 128-row tile; a lone CTA otherwise.
-    const int pair = g.M > 128 ? 2 : 1;
+    const bool quant_a = bf16 && g.qa_fmt >= 0;
+    if (quant_a && (g.N > 128 || quant_out || g.qa_codes == nullptr || g.qa_sf == nullptr)) {
+        *msg = "quantizing A beside a bf16 GEMM needs N <= 128, a bf16 output and both MX buffers";
+        return MXQ_ERR_INVALID_ARG;
+    }
+    // CTA pairs for anything taller than one 128-row tile; a lone CTA otherwise, and for the
+    // bf16 GEMM that quantizes its A (each CTA's quantizer waits on its own stage barriers,
+    // where a pair's loads all complete on the leader's).
+    const int pair = g.M > 128 && !quant_a ? 2 : 1;
     const int rows_b = BN / pair;
     const int64_t atoms_k = sf_atoms_k(g.K);
     const int ak = w4a8 ? 1 : 2;
@@ -818,8 +959,8 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     if (lr_stages > 0) {
         ok = ok && make_map_2d(&mu, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lr_a, lr_k, g.M, lr_k * 2, 64, 128,
                                CU_TENSOR_MAP_SWIZZLE_128B);
-        ok = ok && make_map_2d(&ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lr_b, lr_k, g.N, lr_k * 2, 64, rows_b,
-                               CU_TENSOR_MAP_SWIZZLE_128B);
+        ok = ok && make_map_2d(&ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lr_b, lr_k, g.N, lr_k * 2, 64,
+                               quant_a ? 128 : rows_b, CU_TENSOR_MAP_SWIZZLE_128B);
     }
     if (bf16) {
         ma = msa = mu;  // never used without block-scaled stages
@@ -849,6 +990,14 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     p.gelu = g.out_gelu ? 1 : 0;
     p.alpha = g.alpha;
     p.lr_stages = lr_stages;
+    // a lone CTA's only tile column: bf16 MMAs as wide as the output (rounded up to 16, the
+    // M = 128 granule), not the tile's 256 columns; a pair's MMA of another width would
+    // take a different set of B rows from each CTA, so pairs keep 256
+    p.mma_n = bf16 && pair == 1 && p.n_blocks == 1 ? static_cast<int>((g.N + 15) / 16 * 16) : BN;
+    p.qa_codes = static_cast<uint8_t*>(g.qa_codes);
+    p.qa_sf = static_cast<uint8_t*>(g.qa_sf);
+    p.qa_atoms_k = quant_a ? static_cast<uint32_t>(sf_atoms_k(g.K)) : 0u;
+    p.qa_fmt = quant_a ? g.qa_fmt : -1;
     const int out = !quant_out  ? kOutBf16
                     : p.write_h ? (g.out_fmt == kFmtE4M3 ? kOutGeluE4M3 : kOutGeluE2M1)
                                 : (g.out_fmt == kFmtE4M3 ? kOutQE4M3 : kOutQE2M1);
@@ -858,7 +1007,9 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = std::min(p.num_tiles, sms / pair) * pair;
     cudaError_t e;
-    if (w4a8)
+    if (quant_a)
+        e = launch_variant<false, 1, kOutBf16, true>(ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream);
+    else if (w4a8)
         e = pair == 2 ? launch_out<true, 2>(out, ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream)
                       : launch_out<true, 1>(out, ma, mb, msa, msb, my, mq, mu, ml, p, grid, stream);
     else
@@ -870,8 +1021,9 @@ int launch_gemm(const GemmArgs& g, cudaStream_t stream, const char** msg, char* 
         return MXQ_ERR_CUDA;
     }
     if (path && bf16)
-        snprintf(path, path_len, "bf16 kind::f16 %s %dx%d grid %d tiles %d", pair == 2 ? "2cta" : "1cta",
-                 128 * pair, BN, grid, p.num_tiles);
+        snprintf(path, path_len, "bf16 kind::f16 %s %dx%d (mma n %d) grid %d tiles %d%s", pair == 2 ? "2cta" : "1cta",
+                 128 * pair, BN, p.mma_n, grid, p.num_tiles,
+                 quant_a ? (g.qa_fmt == kFmtE4M3 ? " +quantize a->e4m3" : " +quantize a->e2m1") : "");
     else if (path)
         snprintf(path, path_len, "native %s %s %dx%d grid %d tiles %d%s%s", w4a8 ? "mxf8f6f4" : "mxf4",
                  pair == 2 ? "2cta" : "1cta", 128 * pair, BN, grid, p.num_tiles,

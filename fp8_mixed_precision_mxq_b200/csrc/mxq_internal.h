@@ -71,6 +71,12 @@ struct GemmArgs {
     // plain bf16 GEMM: a_codes is A bf16 [M, K], w_codes is B bf16 [N, K] (K-major, K % 8
     // == 0), no scales; the same kernel runs only bf16 (kind::f16) stages of 64 along K
     bool bf16 = false;
+    // bf16 GEMM only, N <= 256, K % 32 == 0: also MX-quantize A (format qa_fmt, or -1 for
+    // no) into codes qa_codes and tiled scales qa_sf as its stages pass through the kernel,
+    // the same bits as the activation quantizer writes
+    int qa_fmt = -1;
+    void* qa_codes = nullptr;
+    void* qa_sf = nullptr;
 };
 
 // Builds the tensor maps and launches the tcgen05 GEMM.  Returns an mxq_status;

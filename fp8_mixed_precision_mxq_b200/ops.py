@@ -123,6 +123,31 @@ def gemm_bf16(a: torch.Tensor, b: torch.Tensor, bias: torch.Tensor | None = None
     return out
 
 
+def gemm_bf16_quant_a(a: torch.Tensor, b: torch.Tensor, fmt="e2m1", bias: torch.Tensor | None = None, out=None,
+                      codes=None, sf=None, stream=None):
+    """(y, codes, sf): y [M, N] = a [M, K] . b [N, K]^T (+ bias) in bf16 (N <= 128) by the
+    bf16 kernel, which also writes a's MX quantization in format fmt (codes, tiled scales:
+    the bits quantize_act writes) from the same read of a."""
+    _cuda_bf16(a, "a")
+    _cuda_bf16(b, "b")
+    if bias is not None:
+        _cuda_bf16(bias, "bias")
+    M, K = a.shape
+    N = b.shape[0]
+    if b.shape[1] != K:
+        raise ValueError("a is [%d, %d] but b is [%d, %d]" % (M, K, N, b.shape[1]))
+    f = _fmt(fmt)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    if codes is None:
+        codes = torch.empty(max(1, codes_bytes(M, K, f)), dtype=torch.uint8, device=a.device)
+    if sf is None:
+        sf = torch.empty(max(1, sf_bytes(M, K)), dtype=torch.uint8, device=a.device)
+    check(_lib.lib().mxq_gemm_bf16_quant_a(_p(a), M, K, _p(b), N, _p(bias), _p(out), f, _p(codes), _p(sf),
+                                           _stream(stream)), "mxq_gemm_bf16_quant_a")
+    return out, codes, sf
+
+
 def linear(x: torch.Tensor, w: QWeight, fmt="e2m1", mode="native", workspace=None, out=None, stream=None):
     """y = x . deq(w)^T + bias with x quantized on the fly to fmt (E2M1 = W4A4, E4M3 = W4A8)."""
     _cuda_bf16(x, "x")

@@ -121,6 +121,19 @@ int mxq_gemm(const void* a_codes, const void* a_sf, int a_fmt, int64_t M, int64_
 int mxq_gemm_bf16(const void* a_bf16, int64_t M, int64_t K, const void* b_bf16, int64_t N, const void* bias_bf16,
                   void* y_bf16, void* stream);
 
+/* mxq_gemm_bf16 for an output of at most 128 columns, which also writes a's MX
+ * quantization in format fmt -- codes [M, K/2] (E2M1) or [M, K] (E4M3) and tiled scales,
+ * the bits mxq_quantize_act writes -- from the same read of a: its extra warps quantize
+ * each 64-column stage of a as it passes through shared memory.  It serves the SVDQuant
+ * branch of mxq_linear_lowrank (blog section "Mixed-Precision selection"), whose u =
+ * x . l1t^T and whose quantized x both come from x.  Requires 0 < N <= 128, N % 8 == 0,
+ * K % 32 == 0 (a's MX blocks); codes and sf as mxq_quantize_act takes them (16-byte
+ * aligned, mxq_codes_bytes / mxq_sf_bytes); other arguments and errors as for
+ * mxq_gemm_bf16.  Runs on lone CTAs (128-row tiles, six 64-column stages of a in flight)
+ * with MMAs as wide as N (rounded up to 16). */
+int mxq_gemm_bf16_quant_a(const void* a_bf16, int64_t M, int64_t K, const void* b_bf16, int64_t N,
+                          const void* bias_bf16, void* y_bf16, int fmt, void* codes, void* sf, void* stream);
+
 /* The quantized linear layer: quantize x (fmt act_fmt) into the workspace, then
  *   mode NATIVE: mxq_gemm on the quantized operands;
  *   mode QDQ:    dequantize both operands to bf16 and run the bf16 GEMM of
@@ -305,7 +318,9 @@ int mxq_linear_transformed(const void* x_bf16, int64_t M, int64_t K, const void*
  * product l2t . l1t (l1t [r, K], l2t [N, r]) and a residual R quantized to MXFP4
  * (r_codes, r_sf as from mxq_quantize_weight), and the layer computes
  *   y = bf16( deq(xq) . deq(Rq)^T + u . l2t^T + bias ),  u = bf16(x . l1t^T) [M, r],
- * x quantized in act_fmt.  u comes from the bf16 GEMM (mxq_gemm_bf16); u . l2t^T runs as
+ * x quantized in act_fmt.  Up to rank 128, u and the quantized x come from one launch that
+ * reads x once (mxq_gemm_bf16_quant_a); ranks 192 and 256 quantize x and run the bf16 GEMM
+ * apart.  u . l2t^T runs as
  * bf16 tensor-core MMAs (kind::f16) into the same TMEM accumulator as the block-scaled
  * product, in stages of 64 along r ahead of it.  rank: 64, 128, 192 or 256; l1t, l2t
  * 16-byte aligned; workspace of mxq_lowrank_workspace_bytes(...) bytes, 256-byte aligned.

@@ -226,3 +226,19 @@ def test_gelu_entry_point_rejects_bad_arguments():
     assert L.mxq_gelu_bf16(None, 8, A16, None) == _lib.ERR_INVALID_ARG
     assert L.mxq_gelu_bf16(V(4096 + 1), 8, A16, None) == _lib.ERR_ALIGN
     assert L.mxq_gelu_bf16(A16, 8, V(4096 + 1), None) == _lib.ERR_ALIGN
+
+
+def test_bf16_gemm_quantizing_a_rejects_bad_arguments():
+    """mxq_gemm_bf16_quant_a checks before any launch: the output is at most 128 wide, a's K
+    holds whole MX blocks, the format is known, and the MX buffers are 16-byte aligned."""
+    L = _lib.lib()
+    args = lambda M=64, K=128, N=64, fmt=_lib.FMT_E2M1, codes=A16, sf=A16: (  # noqa: E731
+        A16, M, K, A16, N, None, A16, fmt, codes, sf, None)
+    assert L.mxq_gemm_bf16_quant_a(*args(N=136)) == _lib.ERR_SHAPE
+    assert "above 128" in _lib.last_error()
+    assert L.mxq_gemm_bf16_quant_a(*args(K=40)) == _lib.ERR_SHAPE
+    assert L.mxq_gemm_bf16_quant_a(*args(N=12)) == _lib.ERR_SHAPE
+    assert L.mxq_gemm_bf16_quant_a(*args(fmt=7)) == _lib.ERR_INVALID_ARG
+    assert L.mxq_gemm_bf16_quant_a(*args(M=0)) == _lib.ERR_INVALID_ARG
+    assert L.mxq_gemm_bf16_quant_a(*args(codes=V(4096 + 8))) == _lib.ERR_ALIGN
+    assert L.mxq_gemm_bf16_quant_a(*args(sf=None)) == _lib.ERR_INVALID_ARG
