@@ -773,7 +773,8 @@ def bench_transform(args, ops, synth, dev, stream, world, rank, peaks, x, w, b):
 
 def bench_lowrank(args, ops, synth, dev, stream, world, rank, peaks, x, b):
     """The SVDQuant low-rank branch on the headline workload: the linear with a rank-r bf16
-    branch in the same accumulator (u from the library's bf16 GEMM), r = 64 and 128."""
+    branch in the same accumulator, r = 64 and 128.  u = x . l1t^T and x's MX codes come
+    from one kernel that reads x once (mxq_gemm_bf16_quant_a), timed alone against HBM."""
     c = synth.WORKLOADS[args.workload]
     M, K, N = x.shape[0], c["K"], c["N"]
     iters = max(3, args.steps // 4)
@@ -790,7 +791,21 @@ def bench_lowrank(args, ops, synth, dev, stream, world, rank, peaks, x, b):
         flops = 2.0 * M * N * K + 2.0 * M * r * (K + N)
         res["rank%d" % r] = {"ms": round(ms, 4), "TFLOP/s": round(job_tflops(flops, ms, world), 1),
                              "branch_flop_share": round(2.0 * M * r * (K + N) / flops, 4), "path": ops.last_path()}
-        del ws
+        # the fused u + quantizer kernel alone: x in, codes + scales + u out (HBM-bound)
+        u = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+        xc = ws[: ops.codes_bytes(M, K, "e2m1")]
+        off = (ops.codes_bytes(M, K, "e2m1") + 255) // 256 * 256
+        xs = ws[off: off + ops.sf_bytes(M, K)]
+        fq = lambda a=l1t, u=u, xc=xc, xs=xs: ops.gemm_bf16_quant_a(x, a, "e2m1", out=u, codes=xc, sf=xs)  # noqa
+        fq()
+        q_ms, q_stats = time_kernel(fq, stream, idle_s=QUANT_IDLE_S)
+        q_ms = max_over_ranks(q_ms, world)
+        qb = quant_bytes(M, K, "e2m1") + 2 * M * r + 2 * r * K
+        res["rank%d" % r]["u_and_quantize"] = {
+            "ms": round(q_ms, 4), "GB/s": round(qb / (q_ms * 1e-3) / 1e9, 1),
+            "frac_hbm": round(qb / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4), "bytes": qb,
+            "launch_ms": q_stats, "path": ops.last_path()}
+        del ws, u
     if ops.poll_status() != 0:
         raise RuntimeError("device status set during the low-rank measurement")
     return res
