@@ -608,6 +608,10 @@ def profile_one(args, ops, x, qw, ws, y, M, N, K, fmt, stream):
     elif args.only == "dequantize":
         xd = torch.empty((M, K), dtype=torch.bfloat16, device=x.device)
         fn = lambda: ops.dequantize(xc, xs, M, K, fmt, out=xd)  # noqa: E731
+    elif args.only == "u_quantize":  # the low-rank branch's u (rank 64) with x's MX codes
+        l1t = (torch.randn(64, K, device=x.device) * 0.02).to(torch.bfloat16)
+        u = torch.empty((M, 64), dtype=torch.bfloat16, device=x.device)
+        fn = lambda: ops.gemm_bf16_quant_a(x, l1t, fmt, out=u, codes=xc, sf=xs)  # noqa: E731
     else:
         fn = lambda: ops.quantize_act(x, fmt, codes=xc, sf=xs)  # noqa: E731
     for _ in range(args.warmup):
@@ -1058,7 +1062,7 @@ def main():
                     help="reference arm: seconds of oracle work per step (default: about 150 s over the run)")
     ap.add_argument("--M", type=int, default=0, help="override the workload's row count (profiling)")
     ap.add_argument("--only", choices=["gemm", "quantize", "gelu_quant", "transform", "dequantize", "quantize_static",
-                                       "gemm_bf16", "block"], default=None,
+                                       "gemm_bf16", "u_quantize", "block"], default=None,
                     help="profiling mode: launch only this kernel, --steps times")
     ap.add_argument("--rot-block", type=int, default=32, choices=[32, 128],
                     help="profiling mode: rotation block of the transform quantizer")
