@@ -28,12 +28,19 @@
 //               MMAs.  tcgen05 operations of one thread run in order, so copies issued
 //               by the MMA thread would stall behind its MMAs; from their own thread
 //               they overlap them.
+// The same kernel runs bf16 x bf16 stages (kind::f16): the SVDQuant low-rank branch's
+// stages ahead of the block-scaled ones, or every stage of a plain bf16 GEMM.  One lone-CTA
+// bf16 variant (kQA) adds warps 7..14, which MX-quantize each landed stage of A from
+// shared memory and release it beside the MMAs (the branch's u and x's codes from one
+// read of x).
 // L2 policies: the weight is loaded evict-last (it is reused by every m-block and fits
 // in L2), the output is stored evict-first.
 // TMEM (512 columns): accumulator slot 0 = [0, 256), slot 1 = [kAccCol1, kAccCol1 + 256),
 // kSfBufs scale buffers above.  The two slots share 256 - kAccCol1 columns; the
 // epilogue drains those first and signals it, so the next tile's MMAs can start while
-// the rest of the previous accumulator is still being written out.
+// the rest of the previous accumulator is still being written out.  (The kQA variant,
+// whose output is at most 128 columns and which uses no scale buffers, puts slot 1 at
+// [256, 512) and shares nothing.)
 // Every wait is bounded; a wait that runs out records MXQ_ERR_TIMEOUT in a device
 // status word and the kernel winds down (in-flight copies and MMAs drained, TMEM
 // freed) instead of hanging.
