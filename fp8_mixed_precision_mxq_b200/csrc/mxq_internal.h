@@ -71,7 +71,7 @@ struct GemmArgs {
     // plain bf16 GEMM: a_codes is A bf16 [M, K], w_codes is B bf16 [N, K] (K-major, K % 8
     // == 0), no scales; the same kernel runs only bf16 (kind::f16) stages of 64 along K
     bool bf16 = false;
-    // bf16 GEMM only, N <= 256, K % 32 == 0: also MX-quantize A (format qa_fmt, or -1 for
+    // bf16 GEMM only, N <= 128, K % 32 == 0: also MX-quantize A (format qa_fmt, or -1 for
     // no) into codes qa_codes and tiled scales qa_sf as its stages pass through the kernel,
     // the same bits as the activation quantizer writes
     int qa_fmt = -1;
