@@ -470,6 +470,9 @@ def run_mxq(args):
                          peak_src, peaks["bf16_tflops"], FP4_OVER_BF16),
                      "frac_nominal": round(g_tflops / NOMINAL_FP4_TFLOPS, 4),
                      "nominal_peak": NOMINAL_FP4_TFLOPS,
+                     # against the bf16 loop of seconds under the power cap (x the same ratio),
+                     # the regime a long run of steps reaches; the clocks key says which it was
+                     "frac_sustained": round(g_tflops / (sustained_tflops(peaks) * FP4_OVER_BF16), 4),
                      "ms": round(g_ms, 4), "launch_ms": g_stats, "traffic": gemm_traffic(wl_name, M),
                      "path": gemm_path},
         "parts": {
